@@ -1,0 +1,250 @@
+/*
+ * fp64 CPU oracle for NABLA block-mask building and masked softmax attention.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the tests, the package's smoke check and the
+ * bench's CPU-baseline leg may load this library.  It shares no code with the
+ * CUDA path: plain loops, fp64 throughout, no blocking or fusion beyond what the
+ * definitions state.  Inputs are bf16 bit patterns (uint16), widened exactly.
+ *
+ * Sources (page titles and sections):
+ *  - "NABLA: Neighborhood Adaptive Block-Level Attention" (machine review on
+ *    pith.science), "What carries the argument" and "Core claim": Algorithm 1
+ *    average-pools Q and K over N-token blocks, takes a softmax over the S/N x
+ *    S/N reduced map, sorts each row, forms the cumulative sum and keeps the
+ *    smallest prefix of sorted entries whose mass reaches 1 - thr; the mask is
+ *    optionally OR-ed with a sliding-tile (STA) mask.  Referee report, minor
+ *    comment 2: sort and cumsum run along the key-block axis and "reorder"
+ *    returns the flags to block order.
+ *  - "Fast Video Generation with Sliding Tile Attention" (blog notes): queries
+ *    of one tile attend to the key tiles in a common local window, with the
+ *    tile equal to the attention block.
+ *  - FlashAttention abstract: attention is exact softmax(QK^T) V; the block
+ *    sparse extension computes it over the kept blocks only.
+ *
+ * Readings where the pages are silent (each is listed in the design notes):
+ *  - block size N = 64 (one 4x4x4 tile); the reduced map is scaled by 1/sqrt(d);
+ *  - ties in the sorted row go to the lower block index;
+ *  - keep sorted position k iff k == 0 or the exclusive prefix sum E_k < 1-thr
+ *    (so the argmax is always kept), and thr <= 0 keeps every block;
+ *  - the STA window is clipped at the grid edge (no shifted centre);
+ *  - LSE is the natural log of sum exp(scale * q.k) over kept keys; a row with
+ *    no kept key has O = 0 and LSE = -inf.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORACLE_BLOCK 64
+
+static double bf16_to_f64(uint16_t b) {
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    memcpy(&f, &u, 4);
+    return (double)f;
+}
+
+/* Block mean-pool (Algorithm 1, reshape to [.., S/N, N, d] and average over N).
+ * x: [BH, S, d] bf16 bits; out: [BH, S/64, d]. */
+void oracle_pool(const uint16_t* x, int64_t BH, int64_t S, int d, double* out) {
+    int64_t nb = S / ORACLE_BLOCK;
+#pragma omp parallel for schedule(static)
+    for (int64_t br = 0; br < BH * nb; ++br) {
+        int64_t bh = br / nb, r = br % nb;
+        for (int c = 0; c < d; ++c) {
+            double s = 0.0;
+            for (int t = 0; t < ORACLE_BLOCK; ++t)
+                s += bf16_to_f64(x[((bh * S) + r * ORACLE_BLOCK + t) * d + c]);
+            out[br * d + c] = s / ORACLE_BLOCK;
+        }
+    }
+}
+
+/* Reduced map of one head: L[r][c] = qbar_r . kbar_c / sqrt(d). */
+void oracle_logits(const double* qbar, const double* kbar, int nb, int d, double* L) {
+    double inv = 1.0 / sqrt((double)d);
+    for (int r = 0; r < nb; ++r)
+        for (int c = 0; c < nb; ++c) {
+            double s = 0.0;
+            for (int k = 0; k < d; ++k) s += qbar[(int64_t)r * d + k] * kbar[(int64_t)c * d + k];
+            L[(int64_t)r * nb + c] = s * inv;
+        }
+}
+
+/* Row softmax with the maximum subtracted first. */
+void oracle_softmax_row(const double* L, int n, double* P) {
+    double m = -INFINITY;
+    for (int c = 0; c < n; ++c) m = L[c] > m ? L[c] : m;
+    double z = 0.0;
+    for (int c = 0; c < n; ++c) z += exp(L[c] - m);
+    for (int c = 0; c < n; ++c) P[c] = exp(L[c] - m) / z;
+}
+
+typedef struct { double p; int idx; } pv_t;
+
+/* Descending probability; equal probabilities go to the lower block index. */
+static int cmp_desc(const void* a, const void* b) {
+    const pv_t* x = (const pv_t*)a;
+    const pv_t* y = (const pv_t*)b;
+    if (x->p > y->p) return -1;
+    if (x->p < y->p) return 1;
+    return (x->idx > y->idx) - (x->idx < y->idx);
+}
+
+/* CDF binarisation of one softmax row (Algorithm 1: sort, cumsum, threshold at
+ * 1 - thr, reorder).  keep[c] is set to 0/1 for c in [0, n).  Returns the kept
+ * count.  diag (may be NULL) receives, for the last kept sorted position k*:
+ *   diag[0] = E_{k*}   (exclusive prefix sum before k*),
+ *   diag[1] = E_{k*+1} (inclusive sum through k*),
+ *   diag[2] = p at k*,  diag[3] = p at k*+1 (or -1 when k* is the last). */
+int oracle_row_select(const double* p, int n, double thr, uint8_t* keep, double* diag) {
+    pv_t* v = (pv_t*)malloc(sizeof(pv_t) * (size_t)n);
+    for (int c = 0; c < n; ++c) { v[c].p = p[c]; v[c].idx = c; keep[c] = 0; }
+    qsort(v, (size_t)n, sizeof(pv_t), cmp_desc);
+    double target = 1.0 - thr;
+    double E = 0.0, E_star = 0.0;
+    int kstar = 0, count = 0;
+    for (int k = 0; k < n; ++k) {
+        int take = (thr <= 0.0) || k == 0 || E < target;
+        if (!take) break;
+        keep[v[k].idx] = 1;   /* "reorder": the flag goes back to the block's own index */
+        ++count;
+        kstar = k;
+        E_star = E;
+        E += v[k].p;
+    }
+    if (diag) {
+        diag[0] = E_star;
+        diag[1] = E_star + v[kstar].p;
+        diag[2] = v[kstar].p;
+        diag[3] = (kstar + 1 < n) ? v[kstar + 1].p : -1.0;
+    }
+    free(v);
+    return count;
+}
+
+/* OR the sliding-tile window of query tile r into one mask row (tile
+ * coordinates; the window is clipped to the grid). */
+void oracle_sta_or(uint8_t* row, int r, int Tt, int Th, int Tw, int wt, int wh, int ww) {
+    int rt = r / (Th * Tw), rh = (r / Tw) % Th, rw = r % Tw;
+    for (int c = 0; c < Tt * Th * Tw; ++c) {
+        int ct = c / (Th * Tw), ch = (c / Tw) % Th, cw = c % Tw;
+        if (abs(ct - rt) <= wt && abs(ch - rh) <= wh && abs(cw - rw) <= ww) row[c] = 1;
+    }
+}
+
+/* Full mask builder: q, k [BH, S, d] bf16 bits -> mask [BH, nb, nb] uint8.
+ * diag (may be NULL): [BH, nb, 4] as in oracle_row_select (before the STA OR).
+ * adaptive_counts (may be NULL): [BH, nb] kept count before the STA OR. */
+void oracle_build_mask(const uint16_t* q, const uint16_t* k, int64_t BH, int64_t S, int d,
+                       int Tt, int Th, int Tw, double thr, int use_sta, int wt, int wh, int ww,
+                       uint8_t* mask, double* diag, int32_t* adaptive_counts) {
+    int nb = (int)(S / ORACLE_BLOCK);
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t bh = 0; bh < BH; ++bh) {
+        double* qbar = (double*)malloc(sizeof(double) * (size_t)nb * d);
+        double* kbar = (double*)malloc(sizeof(double) * (size_t)nb * d);
+        double* L = (double*)malloc(sizeof(double) * (size_t)nb * nb);
+        double* P = (double*)malloc(sizeof(double) * (size_t)nb);
+        oracle_pool(q + bh * S * d, 1, S, d, qbar);
+        oracle_pool(k + bh * S * d, 1, S, d, kbar);
+        oracle_logits(qbar, kbar, nb, d, L);
+        for (int r = 0; r < nb; ++r) {
+            uint8_t* row = mask + (bh * nb + r) * (int64_t)nb;
+            oracle_softmax_row(L + (int64_t)r * nb, nb, P);
+            int cnt = oracle_row_select(P, nb, thr, row, diag ? diag + (bh * nb + r) * 4 : NULL);
+            if (adaptive_counts) adaptive_counts[bh * nb + r] = cnt;
+            if (use_sta) oracle_sta_or(row, r, Tt, Th, Tw, wt, wh, ww);
+        }
+        free(qbar); free(kbar); free(L); free(P);
+    }
+}
+
+/* Masked softmax attention for a list of query rows.
+ * q, k, v: [BH, S, d] bf16 bits; mask: [BH, nb, nb] uint8 (block keep flags).
+ * rows: global row ids bh*S + i.  O: [nrows, d]; LSE: [nrows] (natural log).
+ * s_ij = scale * q_i . k_j over keys j in kept blocks of row i's block. */
+void oracle_masked_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                             int64_t BH, int64_t S, int d, const uint8_t* mask, double scale,
+                             int64_t nrows, const int64_t* rows, double* O, double* LSE) {
+    int64_t nb = S / ORACLE_BLOCK;
+    (void)BH;
+#pragma omp parallel for schedule(dynamic, 4)
+    for (int64_t n = 0; n < nrows; ++n) {
+        int64_t g = rows[n], bh = g / S, i = g % S, r = i / ORACLE_BLOCK;
+        const uint8_t* mrow = mask + (bh * nb + r) * nb;
+        double* qi = (double*)malloc(sizeof(double) * d);
+        double* acc = (double*)calloc((size_t)d, sizeof(double));
+        double* s = (double*)malloc(sizeof(double) * (size_t)S);
+        for (int c = 0; c < d; ++c) qi[c] = bf16_to_f64(q[(bh * S + i) * d + c]);
+        double m = -INFINITY;
+        int64_t nk = 0;
+        for (int64_t cb = 0; cb < nb; ++cb) {
+            if (!mrow[cb]) continue;
+            for (int64_t j = cb * ORACLE_BLOCK; j < (cb + 1) * ORACLE_BLOCK; ++j) {
+                double dot = 0.0;
+                for (int c = 0; c < d; ++c) dot += qi[c] * bf16_to_f64(k[(bh * S + j) * d + c]);
+                s[j] = scale * dot;
+                if (s[j] > m) m = s[j];
+                ++nk;
+            }
+        }
+        if (nk == 0) {
+            for (int c = 0; c < d; ++c) O[n * d + c] = 0.0;
+            LSE[n] = -INFINITY;
+        } else {
+            double l = 0.0;
+            for (int64_t cb = 0; cb < nb; ++cb) {
+                if (!mrow[cb]) continue;
+                for (int64_t j = cb * ORACLE_BLOCK; j < (cb + 1) * ORACLE_BLOCK; ++j) {
+                    double w = exp(s[j] - m);
+                    l += w;
+                    for (int c = 0; c < d; ++c) acc[c] += w * bf16_to_f64(v[(bh * S + j) * d + c]);
+                }
+            }
+            for (int c = 0; c < d; ++c) O[n * d + c] = acc[c] / l;
+            LSE[n] = m + log(l);
+        }
+        free(qi); free(acc); free(s);
+    }
+}
+
+/* Dense softmax attention (every key of the head) for the self-checks. */
+void oracle_dense_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, int64_t BH,
+                            int64_t S, int d, double scale, int64_t nrows, const int64_t* rows,
+                            double* O, double* LSE) {
+    (void)BH;
+#pragma omp parallel for schedule(dynamic, 4)
+    for (int64_t n = 0; n < nrows; ++n) {
+        int64_t g = rows[n], bh = g / S, i = g % S;
+        double* s = (double*)malloc(sizeof(double) * (size_t)S);
+        double m = -INFINITY;
+        for (int64_t j = 0; j < S; ++j) {
+            double dot = 0.0;
+            for (int c = 0; c < d; ++c)
+                dot += bf16_to_f64(q[(bh * S + i) * d + c]) * bf16_to_f64(k[(bh * S + j) * d + c]);
+            s[j] = scale * dot;
+            if (s[j] > m) m = s[j];
+        }
+        double l = 0.0;
+        for (int c = 0; c < d; ++c) O[n * d + c] = 0.0;
+        for (int64_t j = 0; j < S; ++j) {
+            double w = exp(s[j] - m);
+            l += w;
+            for (int c = 0; c < d; ++c) O[n * d + c] += w * bf16_to_f64(v[(bh * S + j) * d + c]);
+        }
+        for (int c = 0; c < d; ++c) O[n * d + c] /= l;
+        LSE[n] = m + log(l);
+        free(s);
+    }
+}
+
+/* Threads OpenMP will use (for reporting the CPU baseline's core count). */
+int oracle_max_threads(void) {
+#ifdef _OPENMP
+    extern int omp_get_max_threads(void);
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}

@@ -1,0 +1,348 @@
+"""Pins for the fp64 oracle against facts fixed outside the oracle itself.
+
+Each test checks the oracle against something other than its own formulas:
+closed forms (the geometric-decay row model of the NABLA paper's Appendix C),
+hand-computed two-block reduced maps (tests/golden/two_block_cases.txt),
+library routines (numpy means, scipy softmax, torch fp64 attention), and
+invariants the selection rule must satisfy.  A dropped term, wrong sign,
+wrong index or transposed operand in the oracle fails at least one of them.
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _bf16_bits(x):
+    """float array -> bf16 bit patterns, exact for bf16-representable values."""
+    x = np.asarray(x, dtype=np.float32)
+    u = x.view(np.uint32)
+    assert np.all((u & 0xFFFF) == 0), "value not exactly representable in bf16"
+    return (u >> 16).astype(np.uint16)
+
+
+def _rand_bits(rng, shape, scale=1.0):
+    x = (rng.standard_normal(shape) * scale).astype(np.float32)
+    u = x.view(np.uint32)
+    u = (u + 0x7FFF + ((u >> 16) & 1)) >> 16
+    return u.astype(np.uint16)
+
+
+def _f(bits):
+    return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+# ---------------------------------------------------------------- pooling, logits, softmax
+
+def test_pool_matches_numpy_mean(oracle_mod):
+    rng = np.random.default_rng(1)
+    x = _rand_bits(rng, (2, 3, 256, 16))
+    got = oracle_mod.pool(x)
+    want = _f(x).reshape(2, 3, 4, 64, 16).mean(axis=3)
+    np.testing.assert_allclose(got, want, rtol=0, atol=1e-14)
+
+
+def test_pool_constant_blocks_exact(oracle_mod):
+    vals = np.array([0.5, -3.0, 1.25, 7.0], dtype=np.float32)
+    x = np.repeat(vals, 64)[:, None] * np.ones((1, 8), dtype=np.float32)
+    got = oracle_mod.pool(_bf16_bits(x))
+    assert got.shape == (4, 8)
+    assert np.array_equal(got, np.repeat(vals.astype(np.float64)[:, None], 8, axis=1))
+
+
+def test_pool_block_boundaries(oracle_mod):
+    # a single nonzero token at position 64*b + t only moves block b's mean
+    x = np.zeros((256, 4), dtype=np.float32)
+    x[64 * 2 + 63, 1] = 64.0
+    got = oracle_mod.pool(_bf16_bits(x))
+    want = np.zeros((4, 4))
+    want[2, 1] = 1.0
+    assert np.array_equal(got, want)
+
+
+def test_logits_hand_computed(oracle_mod):
+    qbar = np.array([[1.0, 2.0], [0.0, 1.0]])
+    kbar = np.array([[3.0, 0.0], [1.0, 1.0]])
+    got = oracle_mod.logits(qbar, kbar)
+    # rows: q0.k0 = 3, q0.k1 = 3, q1.k0 = 0, q1.k1 = 1; scaled by 1/sqrt(2)
+    want = np.array([[3.0, 3.0], [0.0, 1.0]]) / math.sqrt(2.0)
+    np.testing.assert_allclose(got, want, rtol=0, atol=1e-15)
+    # asymmetric operands: transposing them changes the answer
+    assert not np.allclose(oracle_mod.logits(kbar, qbar), got)
+
+
+def test_softmax_matches_scipy(oracle_mod):
+    from scipy.special import softmax
+    rng = np.random.default_rng(2)
+    for n in (1, 2, 17, 1200):
+        L = rng.standard_normal(n) * 5 + 300.0   # large offset: max subtraction needed
+        np.testing.assert_allclose(oracle_mod.softmax_row(L), softmax(L), rtol=1e-12, atol=0)
+
+
+# ---------------------------------------------------------------- selection rule
+
+def _geometric_count(rho, n, thr):
+    """Closed form for the geometric-decay row p_j = (1-rho) rho^(j-1) / (1-rho^n):
+    mass of the top r is (1-rho^r)/(1-rho^n); the smallest r with mass >= 1-thr
+    is ceil(log(1 - (1-thr)(1-rho^n)) / log(rho))."""
+    if thr <= 0:
+        return n
+    x = math.log(1.0 - (1.0 - thr) * (1.0 - rho ** n)) / math.log(rho)
+    return max(1, min(n, math.ceil(x - 1e-12)))
+
+
+@pytest.mark.parametrize("rho", [0.5, 0.8, 0.9, 0.97, 0.995])
+@pytest.mark.parametrize("n", [16, 128, 1200])
+@pytest.mark.parametrize("thr", [0.2, 0.4, 0.7])
+def test_row_select_geometric_closed_form(oracle_mod, rho, n, thr):
+    j = np.arange(n, dtype=np.float64)
+    p = (1 - rho) * rho ** j / (1 - rho ** n)
+    x = math.log(1.0 - (1.0 - thr) * (1.0 - rho ** n)) / math.log(rho)
+    if abs(x - round(x)) < 1e-6:
+        pytest.skip("cut falls on an exact boundary")
+    want = _geometric_count(rho, n, thr)
+    rng = np.random.default_rng(n)
+    perm = rng.permutation(n)
+    pp = np.empty(n)
+    pp[perm] = p          # block perm[j] holds the j-th largest probability
+    keep, cnt, _ = oracle_mod.row_select(pp, thr)
+    assert cnt == want
+    assert keep.sum() == want
+    assert set(np.nonzero(keep)[0]) == set(perm[:want])
+
+
+def test_row_select_two_block_golden(oracle_mod):
+    path = os.path.join(GOLDEN, "two_block_cases.txt")
+    n_cases = 0
+    for line in open(path):
+        if not line.strip() or line.startswith("#"):
+            continue
+        a, e0, e1, probs = [s.split() for s in line.split("|")]
+        q0, q1, k0, k1, thr = map(float, a)
+        x = np.zeros((128, 64), dtype=np.float32)
+        x[:64, 0], x[64:, 0] = q0, q1
+        y = np.zeros((128, 64), dtype=np.float32)
+        y[:64, 0], y[64:, 0] = k0, k1
+        q = _bf16_bits(x)[None, None]
+        k = _bf16_bits(y)[None, None]
+        mask = oracle_mod.build_mask(q, k, (1, 1, 2), thr, None)
+        assert mask[0, 0, 0].tolist() == [int(t) for t in e0], line
+        assert mask[0, 0, 1].tolist() == [int(t) for t in e1], line
+        # the pooled map itself: p[0][0] and p[1][1]
+        qb, kb = oracle_mod.pool(q[0, 0]), oracle_mod.pool(k[0, 0])
+        L = oracle_mod.logits(qb, kb)
+        p0, p1 = oracle_mod.softmax_row(L[0]), oracle_mod.softmax_row(L[1])
+        assert abs(p0[0] - float(probs[0])) < 1e-12 and abs(p1[1] - float(probs[1])) < 1e-12
+        n_cases += 1
+    assert n_cases >= 10
+
+
+def test_row_select_ties_go_to_lower_index(oracle_mod):
+    p = np.full(8, 1.0 / 8)           # exact in binary: E_k = k/8
+    keep, cnt, _ = oracle_mod.row_select(p, 0.5)
+    assert cnt == 4 and keep.tolist() == [1, 1, 1, 1, 0, 0, 0, 0]
+    keep, cnt, _ = oracle_mod.row_select(p, 0.3)   # k/8 < 0.7 -> k <= 5
+    assert cnt == 6 and keep.tolist() == [1, 1, 1, 1, 1, 1, 0, 0]
+
+
+def test_row_select_invariants_random(oracle_mod):
+    rng = np.random.default_rng(3)
+    for trial in range(300):
+        n = int(rng.integers(1, 300))
+        alpha = float(rng.choice([0.05, 0.3, 1.0, 5.0]))
+        p = rng.dirichlet(np.full(n, alpha))
+        thr = float(rng.choice([0.0, 0.05, 0.2, 0.4, 0.7, 0.95, 1.0]))
+        keep, cnt, diag = oracle_mod.row_select(p, thr)
+        kept = np.nonzero(keep)[0]
+        assert cnt == kept.size >= 1
+        assert keep[np.argmax(p)] == 1                          # argmax always kept
+        mass = p[kept].sum()
+        if thr <= 0:
+            assert cnt == n
+            continue
+        assert mass >= (1 - thr) - 1e-12 or cnt == n            # enough mass kept
+        smallest = kept[np.argmin(p[kept])]
+        if cnt > 1:                                              # minimal prefix
+            assert mass - p[smallest] < (1 - thr) + 1e-12
+        # kept blocks dominate dropped ones
+        dropped = np.nonzero(keep == 0)[0]
+        if dropped.size:
+            assert p[kept].min() >= p[dropped].max()
+        # diagnostics are consistent with the kept set
+        assert abs(diag[1] - mass) < 1e-9 and abs(diag[0] - (mass - diag[2])) < 1e-9
+
+
+def test_row_select_monotone_in_thr(oracle_mod):
+    rng = np.random.default_rng(4)
+    for _ in range(50):
+        p = rng.dirichlet(np.full(64, 0.5))
+        counts = [oracle_mod.row_select(p, t)[1] for t in (0.0, 0.1, 0.2, 0.4, 0.7, 0.9, 1.0)]
+        assert all(a >= b for a, b in zip(counts, counts[1:]))
+        assert counts[0] == 64 and counts[-1] == 1
+
+
+# ---------------------------------------------------------------- STA window
+
+def _clipped(c, w, T):
+    return min(c + w, T - 1) - max(c - w, 0) + 1
+
+
+@pytest.mark.parametrize("grid,window", [((2, 8, 8), (1, 1, 1)), ((5, 12, 20), (1, 2, 2)),
+                                         ((3, 4, 5), (0, 0, 0)), ((4, 4, 4), (5, 5, 5))])
+def test_sta_window_counts(oracle_mod, grid, window):
+    Tt, Th, Tw = grid
+    for r in range(Tt * Th * Tw):
+        row = oracle_mod.sta_row(r, grid, window)
+        rt, rh, rw = r // (Th * Tw), (r // Tw) % Th, r % Tw
+        want = (_clipped(rt, window[0], Tt) * _clipped(rh, window[1], Th) *
+                _clipped(rw, window[2], Tw))
+        assert row.sum() == want
+        assert row[r] == 1
+    if grid == (5, 12, 20):
+        interior = (2 * 12 + 6) * 20 + 10
+        assert oracle_mod.sta_row(interior, grid, window).sum() == 3 * 5 * 5
+
+
+def test_sta_window_membership_brute_force(oracle_mod):
+    grid, window = (3, 5, 4), (1, 2, 1)
+    Tt, Th, Tw = grid
+    coords = [(t, h, w) for t in range(Tt) for h in range(Th) for w in range(Tw)]
+    for r, (a, b, c) in enumerate(coords):
+        row = oracle_mod.sta_row(r, grid, window)
+        for j, (x, y, z) in enumerate(coords):
+            inside = abs(x - a) <= 1 and abs(y - b) <= 2 and abs(z - c) <= 1
+            assert row[j] == inside
+
+
+# ---------------------------------------------------------------- full mask builder
+
+def test_build_mask_geometric_pipeline(oracle_mod):
+    """Pooled logits L[r][c] = -(c) * delta for every query block: each row is
+    exactly the geometric model with rho = exp(-delta)."""
+    nb, d, delta = 32, 64, 0.125
+    x = np.zeros((nb * 64, d), dtype=np.float32)
+    x[:, 0] = 8.0                                  # qbar = 8 e0, sqrt(d) = 8
+    y = np.zeros((nb * 64, d), dtype=np.float32)
+    y[:, 0] = np.repeat(-delta * np.arange(nb), 64)
+    q, k = _bf16_bits(x)[None, None], _bf16_bits(y)[None, None]
+    rho = math.exp(-delta)
+    for thr in (0.2, 0.4, 0.7):
+        mask = oracle_mod.build_mask(q, k, (2, 4, 4), thr, None)
+        want = _geometric_count(rho, nb, thr)
+        assert (mask[0, 0].sum(axis=1) == want).all()
+        assert (mask[0, 0][:, :want] == 1).all() and (mask[0, 0][:, want:] == 0).all()
+
+
+def test_build_mask_invariants_tiny(oracle_mod, synth_mod):
+    w = synth_mod.WORKLOADS["tiny"]
+    q, k, _ = synth_mod.make_qkv(w)
+    # thr = 0 keeps every block
+    assert oracle_mod.build_mask(q, k, w.tile_grid, 0.0, None).min() == 1
+    # STA OR gives a superset, and contains the window
+    m0 = oracle_mod.build_mask(q, k, w.tile_grid, 0.7, None)
+    m1 = oracle_mod.build_mask(q, k, w.tile_grid, 0.7, (1, 1, 1))
+    assert (m1 >= m0).all() and (m1.sum() > m0.sum())
+    for r in range(w.nb):
+        assert (m1[0, 0, r] >= oracle_mod.sta_row(r, w.tile_grid, (1, 1, 1))).all()
+    # monotone in thr
+    m2 = oracle_mod.build_mask(q, k, w.tile_grid, 0.4, None)
+    m3 = oracle_mod.build_mask(q, k, w.tile_grid, 0.2, None)
+    assert (m3 >= m2).all() and (m2 >= m0).all()
+    # argmax and kept mass, from an independent numpy reduced map
+    qb = _f(q).reshape(1, 2, w.nb, 64, 64).mean(axis=3)
+    kb = _f(k).reshape(1, 2, w.nb, 64, 64).mean(axis=3)
+    L = qb @ np.swapaxes(kb, -1, -2) / 8.0
+    P = np.exp(L - L.max(-1, keepdims=True))
+    P /= P.sum(-1, keepdims=True)
+    mask, diag, counts = oracle_mod.build_mask(q, k, w.tile_grid, 0.2, None, with_diag=True)
+    assert (np.take_along_axis(mask, P.argmax(-1)[..., None], -1) == 1).all()
+    assert ((P * mask).sum(-1) >= 0.8 - 1e-12).all()
+
+
+def test_build_mask_key_permutation_invariance(oracle_mod):
+    """Permuting key blocks permutes mask columns (no STA, no ties)."""
+    rng = np.random.default_rng(5)
+    nb, d = 16, 32
+    q = _rand_bits(rng, (1, 1, nb * 64, d), 2.0)
+    k = _rand_bits(rng, (1, 1, nb * 64, d), 2.0)
+    perm = rng.permutation(nb)
+    kp = k.reshape(1, 1, nb, 64, d)[:, :, perm].reshape(1, 1, nb * 64, d)
+    m = oracle_mod.build_mask(q, k, (1, 4, 4), 0.3, None)
+    mp = oracle_mod.build_mask(q, kp, (1, 4, 4), 0.3, None)
+    assert np.array_equal(mp[0, 0], m[0, 0][:, perm])
+
+
+# ---------------------------------------------------------------- attention
+
+def _torch_ref(q, k, v, mask_tok, scale):
+    import torch
+    Q = torch.from_numpy(_f(q))
+    K = torch.from_numpy(_f(k))
+    V = torch.from_numpy(_f(v))
+    s = (Q @ K.transpose(-1, -2)) * scale
+    s = s.masked_fill(~torch.from_numpy(mask_tok), float("-inf"))
+    lse = torch.logsumexp(s, dim=-1)
+    o = torch.softmax(s, dim=-1) @ V
+    return o.numpy(), lse.numpy()
+
+
+def test_dense_attention_matches_torch_sdpa(oracle_mod):
+    import torch
+    rng = np.random.default_rng(6)
+    q = _rand_bits(rng, (1, 2, 192, 32))
+    k = _rand_bits(rng, (1, 2, 192, 32))
+    v = _rand_bits(rng, (1, 2, 192, 32))
+    O, lse = oracle_mod.dense_attention(q, k, v)
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(_f(q)), torch.from_numpy(_f(k)), torch.from_numpy(_f(v)))
+    np.testing.assert_allclose(O, ref.numpy().reshape(-1, 32), rtol=0, atol=1e-12)
+    # all-ones block mask reproduces dense attention
+    ones = np.ones((1, 2, 3, 3), dtype=np.uint8)
+    O2, lse2 = oracle_mod.masked_attention(q, k, v, ones)
+    np.testing.assert_allclose(O2, O, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(lse2, lse, rtol=0, atol=1e-13)
+
+
+def test_masked_attention_matches_torch_masked(oracle_mod):
+    rng = np.random.default_rng(7)
+    B, H, S, d, nb = 1, 3, 256, 64, 4
+    q, k, v = (_rand_bits(rng, (B, H, S, d)) for _ in range(3))
+    mask = (rng.random((B, H, nb, nb)) < 0.5).astype(np.uint8)
+    mask[..., np.arange(nb), np.arange(nb)] = 1
+    scale = 0.17
+    O, lse = oracle_mod.masked_attention(q, k, v, mask, scale=scale)
+    tok = np.repeat(np.repeat(mask.astype(bool), 64, axis=2), 64, axis=3)
+    ro, rl = _torch_ref(q, k, v, tok, scale)
+    np.testing.assert_allclose(O, ro.reshape(-1, d), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse, rl.reshape(-1), rtol=0, atol=1e-12)
+
+
+def test_single_block_rows_and_empty_rows(oracle_mod):
+    import torch
+    rng = np.random.default_rng(8)
+    S, d, nb = 192, 16, 3
+    q, k, v = (_rand_bits(rng, (1, 1, S, d)) for _ in range(3))
+    mask = np.zeros((1, 1, nb, nb), dtype=np.uint8)
+    mask[0, 0, 0, 2] = 1        # query block 0 sees only key block 2
+    mask[0, 0, 1, 1] = 1        # query block 1 sees only itself
+    # query block 2 sees nothing
+    O, lse = oracle_mod.masked_attention(q, k, v, mask)
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(_f(q[0, 0, :64])), torch.from_numpy(_f(k[0, 0, 128:])),
+        torch.from_numpy(_f(v[0, 0, 128:])))
+    np.testing.assert_allclose(O[:64], ref.numpy(), atol=1e-12, rtol=0)
+    assert np.all(O[128:] == 0.0) and np.all(np.isneginf(lse[128:]))
+
+
+def test_thr0_mask_reproduces_full_attention(oracle_mod, synth_mod):
+    w = synth_mod.WORKLOADS["tiny"]
+    q, k, v = synth_mod.make_qkv(w)
+    mask = oracle_mod.build_mask(q, k, w.tile_grid, 0.0, None)
+    rows = np.arange(0, w.H * w.S, 37, dtype=np.int64)
+    O1, l1 = oracle_mod.masked_attention(q, k, v, mask, rows)
+    O2, l2 = oracle_mod.dense_attention(q, k, v, rows)
+    np.testing.assert_allclose(O1, O2, atol=1e-13, rtol=0)
+    np.testing.assert_allclose(l1, l2, atol=1e-13, rtol=0)
