@@ -1,0 +1,260 @@
+"""Python binding for libnabla (NABLA block-sparse attention on B200, sm_100a).
+
+Argument marshalling only: every step of the mask builder and the attention
+forward runs in the CUDA kernels of ``libnabla.so`` (built from ``csrc/`` by
+``build.py``).  PyTorch is used for device memory and the current stream.
+There is no CPU fallback: if the library is missing or no CUDA device is
+present, the calls raise.
+
+The names mirror the C ABI in ``include/nabla.h``:
+
+* ``nabla_build_mask(q, k, tile_grid, thr, sta=None, ...)`` -> block CSR
+* ``bsa_fwd(q, k, v, row_ptr, col_idx, scale=None)`` -> (O, LSE)
+* ``bsa_fwd_with_mask(q, k, v, mask_u8, scale=None)`` -> (O, LSE)
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from dataclasses import dataclass
+from typing import Optional, Tuple
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libnabla.so")
+
+NABLA_OK = 0
+STATUS_NAMES = {0: "NABLA_OK", 1: "NABLA_ERR_INVALID_ARG", 2: "NABLA_ERR_UNSUPPORTED",
+                3: "NABLA_ERR_CAPACITY", 4: "NABLA_ERR_CUDA", 5: "NABLA_ERR_TIMEOUT",
+                6: "NABLA_ERR_BAD_INDEX"}
+OP_BUILD_MASK, OP_FWD, OP_FWD_WITH_MASK = 0, 1, 2
+EXPORTED = ["nabla_workspace_size", "nabla_workspace_init", "nabla_query_status",
+            "nabla_build_mask", "bsa_fwd", "bsa_fwd_with_mask", "nabla_last_error",
+            "nabla_version", "nabla_set_wait_limit_ns", "nabla_set_pv_variant",
+            "nabla_selftest_mma"]
+
+
+class NablaError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        self.status = status
+        super().__init__(f"{STATUS_NAMES.get(status, status)}: {message}")
+
+
+class _Shape(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int32), ("H", ctypes.c_int32), ("S", ctypes.c_int32),
+                ("d", ctypes.c_int32), ("Tt", ctypes.c_int32), ("Th", ctypes.c_int32),
+                ("Tw", ctypes.c_int32)]
+
+
+class _MaskParams(ctypes.Structure):
+    _fields_ = [("thr", ctypes.c_float), ("use_sta", ctypes.c_int32), ("wt", ctypes.c_int32),
+                ("wh", ctypes.c_int32), ("ww", ctypes.c_int32)]
+
+
+_lock = threading.Lock()
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    from .build import build as _build
+    return _build(force=force)
+
+
+def lib() -> ctypes.CDLL:
+    """Load libnabla.so (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                                   "`python -m block_sparse_attention_23_b200.build`")
+            L = ctypes.CDLL(LIB_PATH)
+            vp, i32, i64, f32, sz = (ctypes.c_void_p, ctypes.c_int, ctypes.c_int64,
+                                     ctypes.c_float, ctypes.c_size_t)
+            sp = ctypes.POINTER(_Shape)
+            L.nabla_workspace_size.restype = sz
+            L.nabla_workspace_size.argtypes = [sp, i32]
+            L.nabla_workspace_init.restype = i32
+            L.nabla_workspace_init.argtypes = [vp, vp]
+            L.nabla_query_status.restype = i32
+            L.nabla_query_status.argtypes = [vp, vp]
+            L.nabla_build_mask.restype = i32
+            L.nabla_build_mask.argtypes = [sp, ctypes.POINTER(_MaskParams), vp, vp, vp, vp, vp,
+                                           i64, vp, vp, vp]
+            L.bsa_fwd.restype = i32
+            L.bsa_fwd.argtypes = [sp, vp, vp, vp, vp, vp, f32, vp, vp, vp, vp]
+            L.bsa_fwd_with_mask.restype = i32
+            L.bsa_fwd_with_mask.argtypes = [sp, vp, vp, vp, vp, f32, vp, vp, vp, vp]
+            L.nabla_last_error.restype = ctypes.c_char_p
+            L.nabla_last_error.argtypes = []
+            L.nabla_version.restype = i32
+            L.nabla_version.argtypes = []
+            L.nabla_set_wait_limit_ns.restype = None
+            L.nabla_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
+            L.nabla_set_pv_variant.restype = None
+            L.nabla_set_pv_variant.argtypes = [i32]
+            L.nabla_selftest_mma.restype = i32
+            L.nabla_selftest_mma.argtypes = [i32, vp, vp, vp, vp, vp]
+            _lib = L
+    return _lib
+
+
+def _check(status: int) -> None:
+    if status != NABLA_OK:
+        raise NablaError(status, lib().nabla_last_error().decode())
+
+
+def _torch():
+    import torch
+    if not torch.cuda.is_available():
+        raise RuntimeError("libnabla needs a CUDA device; there is no CPU path")
+    return torch
+
+
+def _stream(stream=None):
+    torch = _torch()
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ptr(t) -> ctypes.c_void_p:
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+
+
+def make_shape(B: int, H: int, S: int, d: int, tile_grid=(0, 0, 0)) -> _Shape:
+    Tt, Th, Tw = tile_grid
+    return _Shape(B, H, S, d, Tt, Th, Tw)
+
+
+def workspace_size(shape: _Shape, op: int) -> int:
+    n = lib().nabla_workspace_size(ctypes.byref(shape), op)
+    if n == 0:
+        raise NablaError(1, lib().nabla_last_error().decode())
+    return int(n)
+
+
+@dataclass
+class Workspace:
+    """Caller-owned device workspace with a zeroed status header."""
+    buf: "object"
+    op: int
+
+    @classmethod
+    def create(cls, shape: _Shape, op: int, device=None, stream=None) -> "Workspace":
+        torch = _torch()
+        n = workspace_size(shape, op)
+        buf = torch.empty(n, dtype=torch.uint8, device=device or "cuda")
+        _check(lib().nabla_workspace_init(_ptr(buf), _stream(stream)))
+        return cls(buf, op)
+
+    def query_status(self, stream=None) -> int:
+        """Synchronise, read and clear the device status word (0 = OK)."""
+        return int(lib().nabla_query_status(_ptr(self.buf), _stream(stream)))
+
+    def check(self, stream=None) -> None:
+        _check(self.query_status(stream))
+
+
+def _shape_of(q, tile_grid=(0, 0, 0)) -> _Shape:
+    if q.dim() != 4:
+        raise ValueError("q must be [B, H, S, d]")
+    B, H, S, d = q.shape
+    return make_shape(B, H, S, d, tile_grid)
+
+
+def _bf16_contig(*ts):
+    torch = _torch()
+    for t in ts:
+        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
+            raise ValueError("q, k, v must be contiguous bf16 CUDA tensors [B, H, S, d]")
+
+
+def nabla_build_mask(q, k, tile_grid, thr: float, sta: Optional[Tuple[int, int, int]] = None,
+                     want_mask: bool = False, col_capacity: Optional[int] = None,
+                     workspace: Optional[Workspace] = None, out=None, stream=None):
+    """NABLA block mask of (q, k) as block CSR.
+
+    Returns (row_ptr int32 [B*H*nb+1], col_idx int32 [capacity], nnz int32 [1],
+    mask uint8 [B,H,nb,nb] or None).  Only the first nnz entries of col_idx
+    are meaningful.  ``out`` may pass preallocated (row_ptr, col_idx, nnz, mask)."""
+    torch = _torch()
+    _bf16_contig(q, k)
+    shape = _shape_of(q, tile_grid)
+    B, H, S, d = q.shape
+    nb = S // 64
+    if workspace is None:
+        workspace = Workspace.create(shape, OP_BUILD_MASK, q.device, stream)
+    if out is None:
+        cap = col_capacity if col_capacity is not None else B * H * nb * nb
+        row_ptr = torch.empty(B * H * nb + 1, dtype=torch.int32, device=q.device)
+        col_idx = torch.empty(max(cap, 1), dtype=torch.int32, device=q.device)
+        nnz = torch.empty(1, dtype=torch.int32, device=q.device)
+        mask = torch.empty((B, H, nb, nb), dtype=torch.uint8, device=q.device) if want_mask else None
+    else:
+        row_ptr, col_idx, nnz, mask = out
+        cap = col_idx.numel() if col_capacity is None else col_capacity
+    prm = _MaskParams(float(thr), 1 if sta is not None else 0, *(sta if sta is not None else (0, 0, 0)))
+    _check(lib().nabla_build_mask(ctypes.byref(shape), ctypes.byref(prm), _ptr(q), _ptr(k),
+                                  _ptr(mask), _ptr(row_ptr), _ptr(col_idx), int(cap), _ptr(nnz),
+                                  _ptr(workspace.buf), _stream(stream)))
+    return row_ptr, col_idx, nnz, mask
+
+
+def bsa_fwd(q, k, v, row_ptr, col_idx, scale: Optional[float] = None,
+            workspace: Optional[Workspace] = None, out=None, stream=None):
+    """Block-sparse attention forward over a block CSR.  Returns (O bf16, LSE fp32)."""
+    torch = _torch()
+    _bf16_contig(q, k, v)
+    shape = _shape_of(q)
+    if workspace is None:
+        workspace = Workspace.create(shape, OP_FWD, q.device, stream)
+    if out is None:
+        o = torch.empty_like(q)
+        lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device)
+    else:
+        o, lse = out
+    _check(lib().bsa_fwd(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(row_ptr),
+                         _ptr(col_idx), float(scale or 0.0), _ptr(o), _ptr(lse),
+                         _ptr(workspace.buf), _stream(stream)))
+    return o, lse
+
+
+def bsa_fwd_with_mask(q, k, v, mask_u8, scale: Optional[float] = None,
+                      workspace: Optional[Workspace] = None, out=None, stream=None):
+    """Block-sparse attention forward with a static uint8 block mask [B,H,nb,nb]."""
+    torch = _torch()
+    _bf16_contig(q, k, v)
+    shape = _shape_of(q)
+    if mask_u8.dtype != torch.uint8 or not mask_u8.is_cuda or not mask_u8.is_contiguous():
+        raise ValueError("mask must be a contiguous uint8 CUDA tensor [B, H, nb, nb]")
+    if workspace is None:
+        workspace = Workspace.create(shape, OP_FWD_WITH_MASK, q.device, stream)
+    if out is None:
+        o = torch.empty_like(q)
+        lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device)
+    else:
+        o, lse = out
+    _check(lib().bsa_fwd_with_mask(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v),
+                                   _ptr(mask_u8), float(scale or 0.0), _ptr(o), _ptr(lse),
+                                   _ptr(workspace.buf), _stream(stream)))
+    return o, lse
+
+
+def set_wait_limit_ns(ns: int) -> None:
+    lib().nabla_set_wait_limit_ns(int(ns))
+
+
+def set_pv_variant(variant: int) -> None:
+    lib().nabla_set_pv_variant(int(variant))
+
+
+def selftest_mma(variant: int, a, b, workspace: Optional[Workspace] = None, stream=None):
+    """One 128x128x128 tcgen05 product (layout check); returns C fp32 [128,128]."""
+    torch = _torch()
+    if workspace is None:
+        workspace = Workspace.create(make_shape(1, 1, 64, 64), OP_FWD, a.device, stream)
+    c = torch.empty((128, 128), dtype=torch.float32, device=a.device)
+    _check(lib().nabla_selftest_mma(int(variant), _ptr(a), _ptr(b), _ptr(c), _ptr(workspace.buf),
+                                    _stream(stream)))
+    workspace.check(stream)
+    return c

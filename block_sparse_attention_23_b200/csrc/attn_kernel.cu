@@ -1,0 +1,630 @@
+// Block-sparse attention forward on sm_100a: tcgen05 MMAs with tensor-memory
+// accumulators, TMA-fed K/V tiles gathered by block index, warp-specialised
+// load / MMA / softmax roles.
+//
+// The arithmetic is FlashAttention's (FlashAttention abstract: exact attention
+// by tiles with an online softmax; its block-sparse extension skips zero
+// blocks), driven by the NABLA block mask ("NABLA: Neighborhood Adaptive
+// Block-Level Attention": the binary block mask decides which N x N blocks
+// are computed).
+//
+// Work decomposition
+//   One CTA per (b, h, pair of query blocks): 128 query rows = query blocks
+//   2p and 2p+1.  The key blocks visited are the union of the two CSR rows;
+//   each union entry carries a 2-bit membership flag, and a query row whose
+//   block did not list the key block treats it as masked (probability 0).
+//   Key tiles are 128 keys = two union entries (the second may be a repeat
+//   that both rows mask).  Every 64-key block is one contiguous slab of the
+//   [B,H,S,d] tensor, so each is a plain 2D TMA box at row (bh*S + 64*j).
+//
+// Roles (256 threads)
+//   warps 0-3  softmax: thread i owns query row i (= tensor-memory lane i):
+//              tcgen05.ld S, online max/exp2/sum, P as bf16, O rescale in
+//              tensor memory, epilogue (O / l, LSE).
+//   warp 4     TMA producer: Q once, then K and V tiles into 2-stage rings.
+//   warp 5     tensor-memory allocation and the single MMA-issuing thread:
+//              S_t = Q K_t^T into one of two S buffers, then O += P_t V_t.
+//   warps 6-7  help build the union list, then wait.
+//
+// Tensor memory (512 columns): S0 [0,128), S1 [128,256), O [256,256+d),
+// P (tensor-memory variant) [384,448).
+//
+// Every mbarrier wait is time-bounded; a wait that runs out records
+// kStatusTimeout, raises a CTA-wide abort flag, and the CTA drains its own TMA
+// loads and MMAs (bounded again) before freeing tensor memory and returning.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <cstdint>
+
+#include "sm100_primitives.cuh"
+
+namespace nabla {
+
+constexpr int kBM = 128;        // query rows per CTA (two 64-token blocks)
+constexpr int kBN = 128;        // keys per tile (two 64-token blocks)
+constexpr int kStages = 2;      // K and V ring depth
+constexpr int kThreads = 256;
+constexpr int kMaxNb = 4096;    // blocks per head supported
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256, kColP = 384;
+constexpr uint64_t kDrainLimitNs = 1000000000ull;   // 1 s for draining in-flight work
+
+enum PvVariant : int { kPvSmemN64 = 1, kPvSmemNd = 2, kPvTmemNd = 3 };
+
+template <int D>
+struct AttnSmem {
+  static constexpr int kDH = D / 64;                       // 64-column halves of d
+  static constexpr uint32_t kQBytes = kBM * D * 2;
+  static constexpr uint32_t kKVBytes = kBN * D * 2;        // one K or V stage
+  static constexpr uint32_t kPBytes = kBM * kBN * 2;
+  static constexpr uint32_t kOffQ = 0;
+  static constexpr uint32_t kOffK = kOffQ + kQBytes;
+  static constexpr uint32_t kOffV = kOffK + kStages * kKVBytes;
+  static constexpr uint32_t kOffP = kOffV + kStages * kKVBytes;
+  static constexpr uint32_t kOffBar = kOffP + kPBytes;     // 32 mbarriers
+  static constexpr uint32_t kOffMisc = kOffBar + 256;      // tmem base, abort, n_u
+  static constexpr uint32_t kOffBitmap = kOffMisc + 64;    // 2 x kMaxNb/32 words
+  static constexpr uint32_t kOffList = kOffBitmap + 2 * (kMaxNb / 32) * 4;
+  static constexpr uint32_t kBytes = kOffList + kMaxNb * 4;
+  static constexpr uint32_t kAlloc = kBytes + 1024;        // slack for 1024-byte alignment
+};
+
+// Barrier slots inside the barrier area.
+enum : int {
+  kBarQFull = 0,
+  kBarKFull = 1,                   // + stage
+  kBarKEmpty = kBarKFull + kStages,
+  kBarVFull = kBarKEmpty + kStages,
+  kBarVEmpty = kBarVFull + kStages,
+  kBarSFull = kBarVEmpty + kStages,   // + buffer (2)
+  kBarSEmpty = kBarSFull + 2,
+  kBarPFull = kBarSEmpty + 2,
+  kBarOFull = kBarPFull + 1,
+  kBarDrain = kBarOFull + 1,
+  kNumBars = kBarDrain + 1
+};
+
+struct AttnParams {
+  const int32_t* row_ptr;
+  const int32_t* col_idx;
+  __nv_bfloat16* o;
+  float* lse;
+  int* status;
+  int H, S, nb, npairs;
+  float scale_log2;        // softmax scale * log2(e)
+  uint64_t wait_limit_ns;
+};
+
+__device__ __forceinline__ void record_abort(volatile int* abort, int* status, int bit) {
+  *abort = 1;
+  atomicOr(status, bit);
+}
+
+// Every lane waits; the warp proceeds only if all lanes saw the phase complete,
+// so the warp-collective tcgen05.ld/st that follow are never divergent.
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, uint64_t limit_ns,
+                                          const volatile int* abort) {
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity, limit_ns, abort));
+}
+
+template <int D, int PV>
+__global__ void __launch_bounds__(kThreads, 1)
+    bsa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                   const __grid_constant__ CUtensorMap tmV, const AttnParams prm) {
+  using L = AttnSmem<D>;
+  extern __shared__ uint8_t attn_smem_raw[];
+  const uint32_t raw = smem_addr(attn_smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* gbase = attn_smem_raw + (base - raw);
+
+  const uint32_t sQ = base + L::kOffQ;
+  const uint32_t sK = base + L::kOffK;
+  const uint32_t sV = base + L::kOffV;
+  const uint32_t sP = base + L::kOffP;
+  const uint32_t bar0 = base + L::kOffBar;
+  uint32_t* misc = reinterpret_cast<uint32_t*>(gbase + L::kOffMisc);
+  volatile uint32_t* tmem_holder = misc;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
+  volatile int* n_union_s = reinterpret_cast<volatile int*>(misc + 2);
+  uint32_t* bm1 = reinterpret_cast<uint32_t*>(gbase + L::kOffBitmap);
+  uint32_t* bm2 = bm1 + kMaxNb / 32;
+  int32_t* ulist = reinterpret_cast<int32_t*>(gbase + L::kOffList);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int item = blockIdx.x;
+  const int bh = item / prm.npairs;
+  const int pair = item % prm.npairs;
+  const int nb = prm.nb;
+  const int r1 = 2 * pair, r2 = 2 * pair + 1;
+  const bool has2 = r2 < nb;
+  auto bar = [&](int i) { return bar0 + 8u * static_cast<uint32_t>(i); };
+
+  // ---------------------------------------------------------------- setup
+  if (tid == 0) {
+    mbar_init(bar(kBarQFull), 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(bar(kBarKFull + s), 1);
+      mbar_init(bar(kBarKEmpty + s), 1);
+      mbar_init(bar(kBarVFull + s), 1);
+      mbar_init(bar(kBarVEmpty + s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar(kBarSFull + b), 1);
+      mbar_init(bar(kBarSEmpty + b), 128);
+    }
+    mbar_init(bar(kBarPFull), 128);
+    mbar_init(bar(kBarOFull), 1);
+    mbar_init(bar(kBarDrain), 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(smem_addr(misc), kTmemCols);
+    tmem_relinquish();
+  }
+  if (warp == 4 && lane == 0) {
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+  }
+  const int nw = (nb + 31) >> 5;
+  for (int i = tid; i < 2 * nw; i += kThreads) (i < nw ? bm1[i] : bm2[i - nw]) = 0u;
+  __syncthreads();
+  {
+    const int64_t g1 = static_cast<int64_t>(bh) * nb + r1;
+    const int b1 = prm.row_ptr[g1], e1 = prm.row_ptr[g1 + 1];
+    for (int i = b1 + tid; i < e1; i += kThreads) {
+      const int c = prm.col_idx[i];
+      if (static_cast<unsigned>(c) < static_cast<unsigned>(nb)) atomicOr(&bm1[c >> 5], 1u << (c & 31));
+      else atomicOr(prm.status, kStatusBadIndex);
+    }
+    if (has2) {
+      const int b2 = prm.row_ptr[g1 + 1], e2 = prm.row_ptr[g1 + 2];
+      for (int i = b2 + tid; i < e2; i += kThreads) {
+        const int c = prm.col_idx[i];
+        if (static_cast<unsigned>(c) < static_cast<unsigned>(nb)) atomicOr(&bm2[c >> 5], 1u << (c & 31));
+        else atomicOr(prm.status, kStatusBadIndex);
+      }
+    }
+  }
+  __syncthreads();
+  if (warp == 6) {   // compact the union in ascending block order
+    int run = 0;
+    for (int w0 = 0; w0 < nw; w0 += 32) {
+      const int w = w0 + lane;
+      const uint32_t u1 = w < nw ? bm1[w] : 0u, u2 = w < nw ? bm2[w] : 0u;
+      uint32_t u = u1 | u2;
+      const int cnt = __popc(u);
+      int incl = cnt;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += y;
+      }
+      int pos = run + incl - cnt;
+      while (u) {
+        const int b = __ffs(u) - 1;
+        u &= u - 1;
+        ulist[pos++] = (w * 32 + b) | (static_cast<int>((u1 >> b) & 1u) << 16) |
+                       (static_cast<int>((u2 >> b) & 1u) << 17);
+      }
+      run += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) *n_union_s = run;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  const int n_u = *n_union_s;
+  const int n_t = (n_u + 1) >> 1;
+  const uint64_t lim = prm.wait_limit_ns;
+
+  if (warp == 4) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0 && n_t > 0) {
+      const int64_t row0 = static_cast<int64_t>(bh) * prm.S;
+      int armed_k[kStages] = {}, armed_v[kStages] = {};
+      mbar_arrive_expect_tx(bar(kBarQFull), L::kQBytes);
+      for (int qb = 0; qb < 2; ++qb)
+        for (int h = 0; h < L::kDH; ++h)
+          tma_load_2d(sQ + h * kBM * 128 + qb * 64 * 128, &tmQ, bar(kBarQFull), h * 64,
+                      static_cast<int32_t>(row0 + (r1 + qb) * 64));
+      for (int t = 0; t < n_t; ++t) {
+        const int s = t % kStages, n = t / kStages;
+        const int j0 = ulist[2 * t] & 0xFFFF;
+        const int j1 = (2 * t + 1 < n_u) ? (ulist[2 * t + 1] & 0xFFFF) : j0;
+        if (t >= kStages && !mbar_wait(bar(kBarKEmpty + s), (n - 1) & 1, lim, abort_flag)) {
+          record_abort(abort_flag, prm.status, kStatusTimeout);
+          break;
+        }
+        mbar_arrive_expect_tx(bar(kBarKFull + s), L::kKVBytes);
+        ++armed_k[s];
+        for (int kb = 0; kb < 2; ++kb)
+          for (int h = 0; h < L::kDH; ++h)
+            tma_load_2d(sK + s * L::kKVBytes + h * kBN * 128 + kb * 64 * 128, &tmK,
+                        bar(kBarKFull + s), h * 64,
+                        static_cast<int32_t>(row0 + (kb ? j1 : j0) * 64));
+        if (t >= kStages && !mbar_wait(bar(kBarVEmpty + s), (n - 1) & 1, lim, abort_flag)) {
+          record_abort(abort_flag, prm.status, kStatusTimeout);
+          break;
+        }
+        mbar_arrive_expect_tx(bar(kBarVFull + s), L::kKVBytes);
+        ++armed_v[s];
+        for (int kb = 0; kb < 2; ++kb)
+          for (int h = 0; h < L::kDH; ++h)
+            tma_load_2d(sV + s * L::kKVBytes + h * kBN * 128 + kb * 64 * 128, &tmV,
+                        bar(kBarVFull + s), h * 64,
+                        static_cast<int32_t>(row0 + (kb ? j1 : j0) * 64));
+      }
+      // drain: every armed phase must complete before shared memory is released
+      mbar_wait(bar(kBarQFull), 0, kDrainLimitNs, nullptr);
+      for (int s = 0; s < kStages; ++s) {
+        if (armed_k[s]) mbar_wait(bar(kBarKFull + s), (armed_k[s] - 1) & 1, kDrainLimitNs, nullptr);
+        if (armed_v[s]) mbar_wait(bar(kBarVFull + s), (armed_v[s] - 1) & 1, kDrainLimitNs, nullptr);
+      }
+    }
+  } else if (warp == 5) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0 && n_t > 0) {
+      constexpr uint32_t idesc_qk = idesc_bf16_f32(kBM, kBN, false);
+      constexpr uint32_t idesc_pv = idesc_bf16_f32(kBM, PV == kPvSmemN64 ? 64 : D, true);
+      bool ok = mbar_wait(bar(kBarQFull), 0, lim, abort_flag);
+      tc_fence_after();
+      auto issue_s = [&](int u) -> bool {
+        const int b = u & 1, s = u % kStages;
+        if (u >= 2 && !mbar_wait(bar(kBarSEmpty + b), ((u >> 1) - 1) & 1, lim, abort_flag)) return false;
+        if (!mbar_wait(bar(kBarKFull + s), (u / kStages) & 1, lim, abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t kt = sK + s * L::kKVBytes;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * (kBM * 128) + (kk & 3) * 32;
+          const uint32_t offk = (kk >> 2) * (kBN * 128) + (kk & 3) * 32;
+          tc_mma_ss(tmem + (b ? kColS1 : kColS0), sdesc_sw128(sQ + off, 16, 1024),
+                    sdesc_sw128(kt + offk, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(bar(kBarKEmpty + s));
+        tc_commit(bar(kBarSFull + b));
+        return true;
+      };
+      if (ok) ok = issue_s(0);
+      for (int t = 0; ok && t < n_t; ++t) {
+        if (t + 1 < n_t && !issue_s(t + 1)) { ok = false; break; }
+        const int s = t % kStages;
+        if (!mbar_wait(bar(kBarPFull), t & 1, lim, abort_flag)) { ok = false; break; }
+        if (!mbar_wait(bar(kBarVFull + s), (t / kStages) & 1, lim, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t vt = sV + s * L::kKVBytes;
+#pragma unroll
+        for (int kk = 0; kk < kBN / 16; ++kk) {
+          const uint32_t acc = (t > 0 || kk > 0) ? 1u : 0u;
+          const uint32_t vrow = vt + kk * 16 * 128;     // 16 keys further down the tile
+          if constexpr (PV == kPvTmemNd) {
+            tc_mma_ts(tmem + kColO, tmem + kColP + kk * 8, sdesc_sw128(vrow, kBN * 128, 1024),
+                      idesc_pv, acc);
+          } else {
+            const uint64_t adesc =
+                sdesc_sw128(sP + (kk >> 2) * (kBM * 128) + (kk & 3) * 32, 16, 1024);
+            if constexpr (PV == kPvSmemNd) {
+              tc_mma_ss(tmem + kColO, adesc, sdesc_sw128(vrow, kBN * 128, 1024), idesc_pv, acc);
+            } else {
+#pragma unroll
+              for (int h = 0; h < L::kDH; ++h)
+                tc_mma_ss(tmem + kColO + h * 64, adesc,
+                          sdesc_sw128(vrow + h * kBN * 128, 1024, 1024), idesc_pv, acc);
+            }
+          }
+        }
+        tc_commit(bar(kBarVEmpty + s));
+        tc_commit(bar(kBarOFull));
+      }
+      if (!ok) record_abort(abort_flag, prm.status, kStatusTimeout);
+      // drain: all MMAs this thread issued must finish before tensor memory is freed
+      tc_commit(bar(kBarDrain));
+      mbar_wait(bar(kBarDrain), 0, kDrainLimitNs, nullptr);
+    }
+  } else if (warp < 4) {
+    // ------------------------------------------------------------ softmax
+    const int row = tid;                     // tensor-memory lane == query row
+    const int qh = row >> 6;                 // 0: block r1, 1: block r2
+    const bool row_valid = qh == 0 || has2;
+    const int bitsel = 1 << (16 + qh);
+    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const float sl2 = prm.scale_log2;
+    float m = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int t = 0; t < n_t; ++t) {
+      const int b = t & 1;
+      if (!warp_wait(bar(kBarSFull + b), (t >> 1) & 1, lim, abort_flag)) { ok = false; break; }
+      tc_fence_after();
+      const int e0 = ulist[2 * t];
+      const int e1 = (2 * t + 1 < n_u) ? ulist[2 * t + 1] : 0;
+      const bool v0 = (e0 & bitsel) != 0, v1 = (e1 & bitsel) != 0;   // uniform per warp
+      uint32_t sreg[4][32];
+      const uint32_t sbase = tmem + lane_off + (b ? kColS1 : kColS0);
+      if (v0) { tmem_ld32(sbase + 0, sreg[0]); tmem_ld32(sbase + 32, sreg[1]); }
+      if (v1) { tmem_ld32(sbase + 64, sreg[2]); tmem_ld32(sbase + 96, sreg[3]); }
+      tmem_ld_wait();
+      tc_fence_before();
+      mbar_arrive(bar(kBarSEmpty + b));
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        if ((c < 2 && v0) || (c >= 2 && v1)) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) mx = fmaxf(mx, __uint_as_float(sreg[c][i]));
+        }
+      }
+      const float m_new = fmaxf(m, mx * sl2);
+      if (t > 0) {
+        if (!warp_wait(bar(kBarOFull), (t - 1) & 1, lim, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+      }
+      const bool need = (m > -INFINITY) && (m_new > m);
+      if (__any_sync(0xffffffffu, need)) {
+        const float alpha = need ? fast_exp2(m - m_new) : 1.f;
+        l *= alpha;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          const uint32_t oa = tmem + lane_off + kColO + c * 32;
+          tmem_ld32(oa, o);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          tmem_st32(oa, o);
+        }
+        tmem_st_wait();
+      }
+      m = m_new;
+      const float mneg = (m == -INFINITY) ? 0.f : -m;   // all-masked so far: p stays 0
+      float rowsum = 0.f;
+      uint32_t pk[4][16];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const bool valid = (c < 2) ? v0 : v1;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          float p0 = 0.f, p1 = 0.f;
+          if (valid) {
+            p0 = fast_exp2(fmaf(__uint_as_float(sreg[c][2 * i]), sl2, mneg));
+            p1 = fast_exp2(fmaf(__uint_as_float(sreg[c][2 * i + 1]), sl2, mneg));
+          }
+          rowsum += p0 + p1;
+          pk[c][i] = pack_bf16x2(p0, p1);
+        }
+      }
+      if constexpr (PV == kPvTmemNd) {
+        uint32_t lo[32], hi[32];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) { lo[i] = pk[0][i]; lo[16 + i] = pk[1][i]; hi[i] = pk[2][i]; hi[16 + i] = pk[3][i]; }
+        tmem_st32(tmem + lane_off + kColP, lo);
+        tmem_st32(tmem + lane_off + kColP + 32, hi);
+        tmem_st_wait();
+      } else {
+        // P row into the 128-byte-swizzled K-major layout: half kh holds keys
+        // [64kh, 64kh+64); 16-byte chunk j of the row sits at chunk j ^ (row & 7).
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const uint32_t rowbase = sP + (c >> 1) * (kBM * 128) + row * 128;
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+            const int chunk = (c & 1) * 4 + q4;
+            const uint32_t addr = rowbase + ((chunk ^ (row & 7)) << 4);
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr),
+                         "r"(pk[c][4 * q4]), "r"(pk[c][4 * q4 + 1]), "r"(pk[c][4 * q4 + 2]),
+                         "r"(pk[c][4 * q4 + 3])
+                         : "memory");
+          }
+        }
+        fence_proxy_async_smem();
+      }
+      tc_fence_before();
+      mbar_arrive(bar(kBarPFull));
+      l += rowsum;
+    }
+    if (!ok) record_abort(abort_flag, prm.status, kStatusTimeout);
+    // ------------------------------------------------------------ epilogue
+    bool have_o = false;
+    if (ok && n_t > 0) {
+      have_o = warp_wait(bar(kBarOFull), (n_t - 1) & 1, lim, abort_flag);
+      if (!have_o) record_abort(abort_flag, prm.status, kStatusTimeout);
+      tc_fence_after();
+    }
+    const bool write = row_valid && (ok && (n_t == 0 || have_o));
+    const int qrow = (qh ? r2 : r1) * 64 + (row & 63);
+    const int64_t grow = static_cast<int64_t>(bh) * prm.S + qrow;
+    const float inv_l = l > 0.f ? 1.f / l : 0.f;
+    __nv_bfloat16* orow = prm.o + grow * D;
+#pragma unroll
+    for (int c = 0; c < D / 32; ++c) {
+      uint32_t o[32];
+      if (have_o) {
+        tmem_ld32(tmem + lane_off + kColO + c * 32, o);
+        tmem_ld_wait();
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) o[i] = 0u;
+      }
+      if (write) {
+        uint32_t w[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          w[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l);
+        uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+      }
+    }
+    if (write && prm.lse != nullptr)
+      prm.lse[grow] = l > 0.f ? (m + __log2f(l)) * 0.69314718055994530942f : -INFINITY;
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------- self-test
+// One 128 x 128 x 128 product through the same building blocks (see
+// nabla_selftest_mma in the public header for the variants).
+__global__ void __launch_bounds__(160, 1)
+    mma_selftest_kernel(const __grid_constant__ CUtensorMap tmA,
+                        const __grid_constant__ CUtensorMap tmB,
+                        const __nv_bfloat16* __restrict__ a_glob, float* __restrict__ c,
+                        int variant, int* status, uint64_t lim) {
+  extern __shared__ uint8_t st_smem_raw[];
+  const uint32_t raw = smem_addr(st_smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* gbase = st_smem_raw + (base - raw);
+  const uint32_t sA = base, sB = base + 32768, bars = base + 65536;
+  uint32_t* holder = reinterpret_cast<uint32_t*>(gbase + 65536 + 64);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t bar_tma = bars, bar_mma = bars + 8, bar_a = bars + 16;
+  if (tid == 0) {
+    mbar_init(bar_tma, 1);
+    mbar_init(bar_mma, 1);
+    mbar_init(bar_a, 128);
+    fence_barrier_init();
+  }
+  if (warp == 4) {
+    tmem_alloc(smem_addr(holder), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(holder);
+  bool ok = true;
+  if (warp == 4 && lane == 0) {
+    mbar_arrive_expect_tx(bar_tma, 65536);
+    for (int rh = 0; rh < 2; ++rh)
+      for (int h = 0; h < 2; ++h) {
+        tma_load_2d(sA + h * 16384 + rh * 8192, &tmA, bar_tma, h * 64, rh * 64);
+        tma_load_2d(sB + h * 16384 + rh * 8192, &tmB, bar_tma, h * 64, rh * 64);
+      }
+    ok = mbar_wait(bar_tma, 0, lim, nullptr);
+    if (ok && variant == 3) ok = mbar_wait(bar_a, 0, lim, nullptr);
+    tc_fence_after();
+    if (ok) {
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint32_t acc = kk > 0;
+        const uint64_t ad = sdesc_sw128(sA + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
+        if (variant == 0) {
+          tc_mma_ss(tmem, ad, sdesc_sw128(sB + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
+                    idesc_bf16_f32(128, 128, false), acc);
+        } else if (variant == 1) {
+          tc_mma_ss(tmem, ad, sdesc_sw128(sB + kk * 2048, 16384, 1024),
+                    idesc_bf16_f32(128, 128, true), acc);
+        } else if (variant == 2) {
+          for (int h = 0; h < 2; ++h)
+            tc_mma_ss(tmem + h * 64, ad, sdesc_sw128(sB + h * 16384 + kk * 2048, 1024, 1024),
+                      idesc_bf16_f32(128, 64, true), acc);
+        } else {
+          tc_mma_ts(tmem, tmem + 256 + kk * 8, sdesc_sw128(sB + kk * 2048, 16384, 1024),
+                    idesc_bf16_f32(128, 128, true), acc);
+        }
+      }
+      tc_commit(bar_mma);
+    } else {
+      atomicOr(status, kStatusTimeout);
+    }
+  }
+  if (warp < 4) {
+    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    if (variant == 3) {   // A row `tid` into tensor memory as packed bf16 pairs
+      const uint32_t* arow = reinterpret_cast<const uint32_t*>(a_glob + tid * 128);
+      for (int h = 0; h < 2; ++h) {
+        uint32_t r[32];
+        for (int i = 0; i < 32; ++i) r[i] = arow[h * 32 + i];
+        tmem_st32(tmem + lane_off + 256 + h * 32, r);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(bar_a);
+    }
+    const bool done = warp_wait(bar_mma, 0, lim, nullptr);
+    tc_fence_after();
+    if (done) {
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t r[32];
+        tmem_ld32(tmem + lane_off + cc * 32, r);
+        tmem_ld_wait();
+        for (int i = 0; i < 32; ++i) c[tid * 128 + cc * 32 + i] = __uint_as_float(r[i]);
+      }
+    } else {
+      atomicOr(status, kStatusTimeout);
+    }
+  }
+  if (warp == 4 && lane == 0 && ok) mbar_wait(bar_mma, 0, kDrainLimitNs, nullptr);
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 4) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------- launchers
+
+template <int D, int PV>
+static cudaError_t launch_fwd_t(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
+                                const AttnParams& prm, int64_t nitems, cudaStream_t st) {
+  constexpr uint32_t smem = AttnSmem<D>::kAlloc;
+  cudaError_t e = cudaFuncSetAttribute(bsa_fwd_kernel<D, PV>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  bsa_fwd_kernel<D, PV><<<static_cast<unsigned>(nitems), kThreads, smem, st>>>(q, k, v, prm);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_bsa_fwd(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
+                           const int32_t* row_ptr, const int32_t* col_idx, void* o, float* lse,
+                           int* status, int BH, int H, int S, int d, float scale,
+                           uint64_t wait_limit_ns, int pv_variant, cudaStream_t st) {
+  AttnParams prm;
+  prm.row_ptr = row_ptr;
+  prm.col_idx = col_idx;
+  prm.o = static_cast<__nv_bfloat16*>(o);
+  prm.lse = lse;
+  prm.status = status;
+  prm.H = H;
+  prm.S = S;
+  prm.nb = S / 64;
+  prm.npairs = (prm.nb + 1) / 2;
+  prm.scale_log2 = scale * 1.4426950408889634f;
+  prm.wait_limit_ns = wait_limit_ns;
+  const int64_t nitems = static_cast<int64_t>(BH) * prm.npairs;
+  if (nitems == 0) return cudaSuccess;
+  if (d == 128) {
+    switch (pv_variant) {
+      case kPvSmemN64: return launch_fwd_t<128, kPvSmemN64>(q, k, v, prm, nitems, st);
+      case kPvSmemNd: return launch_fwd_t<128, kPvSmemNd>(q, k, v, prm, nitems, st);
+      default: return launch_fwd_t<128, kPvTmemNd>(q, k, v, prm, nitems, st);
+    }
+  }
+  switch (pv_variant) {
+    case kPvSmemN64: return launch_fwd_t<64, kPvSmemN64>(q, k, v, prm, nitems, st);
+    case kPvSmemNd: return launch_fwd_t<64, kPvSmemNd>(q, k, v, prm, nitems, st);
+    default: return launch_fwd_t<64, kPvTmemNd>(q, k, v, prm, nitems, st);
+  }
+}
+
+cudaError_t launch_mma_selftest(const CUtensorMap& a, const CUtensorMap& b, const void* a_glob,
+                                float* c, int variant, int* status, uint64_t lim,
+                                cudaStream_t st) {
+  const uint32_t smem = 65536 + 1024 + 1024;
+  cudaError_t e = cudaFuncSetAttribute(mma_selftest_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  mma_selftest_kernel<<<1, 160, smem, st>>>(a, b, static_cast<const __nv_bfloat16*>(a_glob), c,
+                                            variant, status, lim);
+  return cudaGetLastError();
+}
+
+}  // namespace nabla

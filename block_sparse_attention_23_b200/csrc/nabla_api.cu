@@ -1,0 +1,327 @@
+// libnabla C ABI: argument checks, workspace layout, TMA descriptors and
+// kernel launches.  No entry point allocates device memory or synchronises,
+// except nabla_query_status (which must read the device status word).
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "../../include/nabla.h"
+#include "sm100_primitives.cuh"
+
+namespace nabla {
+cudaError_t launch_pool(const void* q, const void* k, float* qbar, float* kbar, int64_t nblocks,
+                        int d, cudaStream_t st);
+cudaError_t launch_logits(const float* qbar, const float* kbar, float* L, int BH, int nb, int d,
+                          cudaStream_t st);
+cudaError_t launch_select(const float* L, int64_t nrows, int nb, float thr, int use_sta, int wt,
+                          int wh, int ww, int Tt, int Th, int Tw, uint32_t* bits, int32_t* counts,
+                          uint8_t* mask_u8, cudaStream_t st);
+cudaError_t launch_mask_bits(const uint8_t* mask, int64_t nrows, int nb, uint32_t* bits,
+                             int32_t* counts, cudaStream_t st);
+cudaError_t launch_scan_fill(const uint32_t* bits, const int32_t* counts, int64_t nrows, int nb,
+                             int32_t* row_ptr, int32_t* col_idx, int64_t capacity,
+                             int32_t* nnz_out, int* status, cudaStream_t st);
+cudaError_t launch_bsa_fwd(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
+                           const int32_t* row_ptr, const int32_t* col_idx, void* o, float* lse,
+                           int* status, int BH, int H, int S, int d, float scale,
+                           uint64_t wait_limit_ns, int pv_variant, cudaStream_t st);
+cudaError_t launch_mma_selftest(const CUtensorMap& a, const CUtensorMap& b, const void* a_glob,
+                                float* c, int variant, int* status, uint64_t lim,
+                                cudaStream_t st);
+}  // namespace nabla
+
+namespace {
+
+constexpr size_t kHeaderBytes = 256;
+constexpr uint64_t kDefaultWaitLimitNs = 2000000000ull;   // 2 s
+constexpr int kMaxNbSupported = 4096;
+
+thread_local std::string g_last_error;
+std::atomic<uint64_t> g_wait_limit_ns{kDefaultWaitLimitNs};
+std::atomic<int> g_pv_variant{0};
+constexpr int kDefaultPvVariant = 1;
+
+nabla_status fail(nabla_status s, const std::string& msg) {
+  g_last_error = msg;
+  return s;
+}
+
+nabla_status cuda_fail(cudaError_t e, const char* where) {
+  g_last_error = std::string(where) + ": " + cudaGetErrorString(e);
+  return NABLA_ERR_CUDA;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Validates the tensor shape shared by every call.
+nabla_status check_shape(const nabla_shape* s) {
+  if (s == nullptr) return fail(NABLA_ERR_INVALID_ARG, "shape is NULL");
+  if (s->B <= 0 || s->H <= 0 || s->S <= 0 || s->d <= 0)
+    return fail(NABLA_ERR_INVALID_ARG, "B, H, S and d must be positive");
+  if (s->d != 64 && s->d != 128) return fail(NABLA_ERR_UNSUPPORTED, "d must be 64 or 128");
+  if (s->S % 64 != 0) return fail(NABLA_ERR_UNSUPPORTED, "S must be a multiple of 64");
+  const int64_t nb = s->S / 64;
+  if (nb > kMaxNbSupported) return fail(NABLA_ERR_UNSUPPORTED, "S/64 must be at most 4096");
+  const int64_t rows = static_cast<int64_t>(s->B) * s->H * nb;
+  if (rows * nb >= (static_cast<int64_t>(1) << 31))
+    return fail(NABLA_ERR_UNSUPPORTED, "B*H*nb*nb must stay below 2^31");
+  if (static_cast<int64_t>(s->B) * s->H * s->S >= (static_cast<int64_t>(1) << 31))
+    return fail(NABLA_ERR_UNSUPPORTED, "B*H*S must stay below 2^31");
+  return NABLA_OK;
+}
+
+struct BuildLayout {
+  size_t qbar, kbar, logits, bits, counts, total;
+};
+
+BuildLayout build_layout(const nabla_shape* s) {
+  const size_t nb = s->S / 64, BH = static_cast<size_t>(s->B) * s->H, nw = (nb + 31) / 32;
+  BuildLayout l;
+  size_t off = kHeaderBytes;
+  l.qbar = off; off = align256(off + BH * nb * s->d * 4);
+  l.kbar = off; off = align256(off + BH * nb * s->d * 4);
+  l.logits = off; off = align256(off + BH * nb * nb * 4);
+  l.bits = off; off = align256(off + BH * nb * nw * 4);
+  l.counts = off; off = align256(off + BH * nb * 4);
+  l.total = off;
+  return l;
+}
+
+struct MaskLayout {
+  size_t bits, counts, row_ptr, col_idx, total;
+};
+
+MaskLayout mask_layout(const nabla_shape* s) {
+  const size_t nb = s->S / 64, BH = static_cast<size_t>(s->B) * s->H, nw = (nb + 31) / 32;
+  MaskLayout l;
+  size_t off = kHeaderBytes;
+  l.bits = off; off = align256(off + BH * nb * nw * 4);
+  l.counts = off; off = align256(off + BH * nb * 4);
+  l.row_ptr = off; off = align256(off + (BH * nb + 1) * 4);
+  l.col_idx = off; off = align256(off + BH * nb * nb * 4);
+  l.total = off;
+  return l;
+}
+
+// cuTensorMapEncodeTiled, fetched from the driver at run time so the library
+// has no link-time dependency on libcuda.
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static std::once_flag once;
+  static EncodeTiledFn fn = nullptr;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// [rows, cols] bf16 row-major; 64 x 64 boxes with 128-byte swizzle.
+nabla_status make_map(CUtensorMap* map, const void* ptr, uint64_t rows, uint64_t cols) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return fail(NABLA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {64, 64};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(NABLA_ERR_CUDA, "cuTensorMapEncodeTiled failed");
+  return NABLA_OK;
+}
+
+int* status_ptr(void* ws) { return static_cast<int*>(ws); }
+
+int pv_variant() {
+  const int v = g_pv_variant.load();
+  return v == 0 ? kDefaultPvVariant : v;
+}
+
+nabla_status run_fwd(const nabla_shape* shape, const void* q, const void* k, const void* v,
+                     const int32_t* row_ptr, const int32_t* col_idx, float scale, void* o,
+                     float* lse, void* workspace, cudaStream_t st) {
+  const uint64_t rows = static_cast<uint64_t>(shape->B) * shape->H * shape->S;
+  CUtensorMap mq, mk, mv;
+  nabla_status s;
+  if ((s = make_map(&mq, q, rows, shape->d)) != NABLA_OK) return s;
+  if ((s = make_map(&mk, k, rows, shape->d)) != NABLA_OK) return s;
+  if ((s = make_map(&mv, v, rows, shape->d)) != NABLA_OK) return s;
+  if (!(scale > 0.f)) scale = 1.0f / std::sqrt(static_cast<float>(shape->d));
+  cudaError_t e = nabla::launch_bsa_fwd(mq, mk, mv, row_ptr, col_idx, o, lse,
+                                        status_ptr(workspace), shape->B * shape->H, shape->H,
+                                        shape->S, shape->d, scale, g_wait_limit_ns.load(),
+                                        pv_variant(), st);
+  if (e != cudaSuccess) return cuda_fail(e, "bsa_fwd launch");
+  return NABLA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int nabla_version(void) { return 100; }
+
+const char* nabla_last_error(void) { return g_last_error.c_str(); }
+
+void nabla_set_wait_limit_ns(uint64_t ns) {
+  g_wait_limit_ns.store(ns == 0 ? kDefaultWaitLimitNs : ns);
+}
+
+void nabla_set_pv_variant(int variant) {
+  g_pv_variant.store((variant >= 1 && variant <= 3) ? variant : 0);
+}
+
+size_t nabla_workspace_size(const nabla_shape* shape, int op) {
+  if (check_shape(shape) != NABLA_OK) return 0;
+  switch (op) {
+    case NABLA_OP_BUILD_MASK: return build_layout(shape).total;
+    case NABLA_OP_FWD: return kHeaderBytes;
+    case NABLA_OP_FWD_WITH_MASK: return mask_layout(shape).total;
+    default: g_last_error = "unknown op"; return 0;
+  }
+}
+
+nabla_status nabla_workspace_init(void* workspace, nabla_stream_t stream) {
+  if (workspace == nullptr) return fail(NABLA_ERR_INVALID_ARG, "workspace is NULL");
+  cudaError_t e = cudaMemsetAsync(workspace, 0, kHeaderBytes, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "nabla_workspace_init");
+  return NABLA_OK;
+}
+
+nabla_status nabla_query_status(void* workspace, nabla_stream_t stream) {
+  if (workspace == nullptr) return fail(NABLA_ERR_INVALID_ARG, "workspace is NULL");
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  int word = 0;
+  cudaError_t e = cudaMemcpyAsync(&word, workspace, sizeof(int), cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e, "nabla_query_status");
+  e = cudaMemsetAsync(workspace, 0, sizeof(int), st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e, "nabla_query_status");
+  if (word & nabla::kStatusTimeout) return fail(NABLA_ERR_TIMEOUT, "a device pipeline wait ran out");
+  if (word & nabla::kStatusCapacity) return fail(NABLA_ERR_CAPACITY, "kept blocks exceed col_capacity");
+  if (word & nabla::kStatusBadIndex) return fail(NABLA_ERR_BAD_INDEX, "a CSR column index was out of range");
+  return NABLA_OK;
+}
+
+nabla_status nabla_build_mask(const nabla_shape* shape, const nabla_mask_params* params,
+                              const void* q, const void* k, uint8_t* mask_u8, int32_t* row_ptr,
+                              int32_t* col_idx, int64_t col_capacity, int32_t* nnz_out,
+                              void* workspace, nabla_stream_t stream) {
+  nabla_status s = check_shape(shape);
+  if (s != NABLA_OK) return s;
+  if (params == nullptr) return fail(NABLA_ERR_INVALID_ARG, "params is NULL");
+  if (!(params->thr >= 0.f && params->thr <= 1.f))
+    return fail(NABLA_ERR_UNSUPPORTED, "thr must lie in [0, 1]");
+  if (params->use_sta && (params->wt < 0 || params->wh < 0 || params->ww < 0))
+    return fail(NABLA_ERR_INVALID_ARG, "STA half-windows must be non-negative");
+  if (shape->Tt <= 0 || shape->Th <= 0 || shape->Tw <= 0 ||
+      static_cast<int64_t>(shape->Tt) * shape->Th * shape->Tw != shape->S / 64)
+    return fail(NABLA_ERR_INVALID_ARG, "tile grid Tt*Th*Tw must equal S/64");
+  if (!q || !k || !row_ptr || !workspace) return fail(NABLA_ERR_INVALID_ARG, "null pointer");
+  if (col_capacity > 0 && col_idx == nullptr) return fail(NABLA_ERR_INVALID_ARG, "col_idx is NULL");
+  if (col_capacity < 0) return fail(NABLA_ERR_INVALID_ARG, "col_capacity is negative");
+  if (!aligned16(q) || !aligned16(k) || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return fail(NABLA_ERR_INVALID_ARG, "q, k need 16-byte and workspace 256-byte alignment");
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const BuildLayout lay = build_layout(shape);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  float* qbar = reinterpret_cast<float*>(ws + lay.qbar);
+  float* kbar = reinterpret_cast<float*>(ws + lay.kbar);
+  float* L = reinterpret_cast<float*>(ws + lay.logits);
+  uint32_t* bits = reinterpret_cast<uint32_t*>(ws + lay.bits);
+  int32_t* counts = reinterpret_cast<int32_t*>(ws + lay.counts);
+  const int nb = shape->S / 64, BH = shape->B * shape->H;
+  const int64_t nrows = static_cast<int64_t>(BH) * nb;
+  cudaError_t e = nabla::launch_pool(q, k, qbar, kbar, nrows, shape->d, st);
+  if (e != cudaSuccess) return cuda_fail(e, "pool launch");
+  e = nabla::launch_logits(qbar, kbar, L, BH, nb, shape->d, st);
+  if (e != cudaSuccess) return cuda_fail(e, "logits launch");
+  e = nabla::launch_select(L, nrows, nb, params->thr, params->use_sta ? 1 : 0, params->wt,
+                           params->wh, params->ww, shape->Tt, shape->Th, shape->Tw, bits, counts,
+                           mask_u8, st);
+  if (e != cudaSuccess) return cuda_fail(e, "select launch");
+  e = nabla::launch_scan_fill(bits, counts, nrows, nb, row_ptr, col_idx, col_capacity, nnz_out,
+                              status_ptr(workspace), st);
+  if (e != cudaSuccess) return cuda_fail(e, "scan/fill launch");
+  return NABLA_OK;
+}
+
+nabla_status bsa_fwd(const nabla_shape* shape, const void* q, const void* k, const void* v,
+                     const int32_t* row_ptr, const int32_t* col_idx, float scale, void* o,
+                     float* lse, void* workspace, nabla_stream_t stream) {
+  nabla_status s = check_shape(shape);
+  if (s != NABLA_OK) return s;
+  if (!q || !k || !v || !row_ptr || !col_idx || !o || !workspace)
+    return fail(NABLA_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
+    return fail(NABLA_ERR_INVALID_ARG, "q, k, v, o must be 16-byte aligned");
+  if (!std::isfinite(scale)) return fail(NABLA_ERR_INVALID_ARG, "scale must be finite");
+  return run_fwd(shape, q, k, v, row_ptr, col_idx, scale, o, lse, workspace,
+                 reinterpret_cast<cudaStream_t>(stream));
+}
+
+nabla_status bsa_fwd_with_mask(const nabla_shape* shape, const void* q, const void* k,
+                               const void* v, const uint8_t* mask_u8, float scale, void* o,
+                               float* lse, void* workspace, nabla_stream_t stream) {
+  nabla_status s = check_shape(shape);
+  if (s != NABLA_OK) return s;
+  if (!q || !k || !v || !mask_u8 || !o || !workspace)
+    return fail(NABLA_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return fail(NABLA_ERR_INVALID_ARG, "q, k, v, o need 16-byte and workspace 256-byte alignment");
+  if (!std::isfinite(scale)) return fail(NABLA_ERR_INVALID_ARG, "scale must be finite");
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const MaskLayout lay = mask_layout(shape);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  uint32_t* bits = reinterpret_cast<uint32_t*>(ws + lay.bits);
+  int32_t* counts = reinterpret_cast<int32_t*>(ws + lay.counts);
+  int32_t* row_ptr = reinterpret_cast<int32_t*>(ws + lay.row_ptr);
+  int32_t* col_idx = reinterpret_cast<int32_t*>(ws + lay.col_idx);
+  const int nb = shape->S / 64;
+  const int64_t nrows = static_cast<int64_t>(shape->B) * shape->H * nb;
+  const int64_t cap = nrows * nb;
+  cudaError_t e = nabla::launch_mask_bits(mask_u8, nrows, nb, bits, counts, st);
+  if (e != cudaSuccess) return cuda_fail(e, "mask_bits launch");
+  e = nabla::launch_scan_fill(bits, counts, nrows, nb, row_ptr, col_idx, cap, nullptr,
+                              status_ptr(workspace), st);
+  if (e != cudaSuccess) return cuda_fail(e, "scan/fill launch");
+  return run_fwd(shape, q, k, v, row_ptr, col_idx, scale, o, lse, workspace, st);
+}
+
+nabla_status nabla_selftest_mma(int variant, const void* a, const void* b, float* c,
+                                void* workspace, nabla_stream_t stream) {
+  if (variant < 0 || variant > 3) return fail(NABLA_ERR_INVALID_ARG, "variant must be 0..3");
+  if (!a || !b || !c || !workspace) return fail(NABLA_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(a) || !aligned16(b)) return fail(NABLA_ERR_INVALID_ARG, "a, b need 16-byte alignment");
+  CUtensorMap ma, mb;
+  nabla_status s;
+  if ((s = make_map(&ma, a, 128, 128)) != NABLA_OK) return s;
+  if ((s = make_map(&mb, b, 128, 128)) != NABLA_OK) return s;
+  cudaError_t e = nabla::launch_mma_selftest(ma, mb, a, c, variant, status_ptr(workspace),
+                                             g_wait_limit_ns.load(),
+                                             reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "selftest launch");
+  return NABLA_OK;
+}
+
+}  // extern "C"

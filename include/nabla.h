@@ -1,0 +1,185 @@
+/*
+ * libnabla — NABLA adaptive block-sparse attention for 3D video token grids,
+ * native to NVIDIA B200 (sm_100a).
+ *
+ * The library exports a plain C ABI: device pointers, sizes and a CUDA stream
+ * (passed as an opaque pointer; cudaStream_t converts to it).  No call
+ * allocates device memory; the caller owns every buffer, including the
+ * workspace.  Every call is asynchronous on the given stream and returns
+ * argument errors immediately.  Errors found on the device (a CSR capacity
+ * overflow, a bad block index, a pipeline wait that ran out) are OR-ed into a
+ * status word at the head of the workspace and reported by
+ * nabla_query_status().
+ *
+ * Conventions shared by all calls
+ *   Q, K, V, O : bf16, [B, H, S, d] row-major; 16-byte aligned base pointers.
+ *   LSE        : fp32, [B, H, S]; natural log of sum_j exp(scale * q_i . k_j)
+ *                over the keys row i attends to.
+ *   Blocks     : 64 consecutive tokens.  nb = S / 64.  Tokens are ordered
+ *                tile-major, so block r is the 4x4x4 token tile number r of a
+ *                tile grid Tt x Th x Tw in (t, h, w) raster order.
+ *   Block CSR  : row_ptr int32 [B*H*nb + 1], col_idx int32 [nnz]; global row
+ *                g = (b*H + h)*nb + r lists the key blocks query block r of
+ *                head (b, h) attends to.  Column indices are head-local
+ *                (0 <= c < nb).
+ *   Supported  : d in {64, 128}; S % 64 == 0; 1 <= nb <= 4096;
+ *                B*H*nb*nb < 2^31.
+ */
+#ifndef NABLA_H_
+#define NABLA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define NABLA_API __attribute__((visibility("default")))
+#else
+#define NABLA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* cudaStream_t is `struct CUstream_st*`; this alias keeps the header free of
+ * CUDA includes.  NULL is the legacy default stream. */
+typedef struct CUstream_st* nabla_stream_t;
+
+typedef enum {
+    NABLA_OK = 0,
+    NABLA_ERR_INVALID_ARG = 1,  /* null pointer, bad size, misaligned pointer */
+    NABLA_ERR_UNSUPPORTED = 2,  /* shape outside the supported set above */
+    NABLA_ERR_CAPACITY = 3,     /* the kept blocks did not fit col_capacity */
+    NABLA_ERR_CUDA = 4,         /* a CUDA runtime call failed; see nabla_last_error() */
+    NABLA_ERR_TIMEOUT = 5,      /* a device pipeline wait ran out; the kernel returned early */
+    NABLA_ERR_BAD_INDEX = 6     /* a CSR column index outside [0, nb) was skipped */
+} nabla_status;
+
+typedef struct {
+    int32_t B, H, S, d;   /* batch, heads, tokens, head dim */
+    int32_t Tt, Th, Tw;   /* tile grid (4x4x4-token tiles); Tt*Th*Tw must equal S/64 */
+} nabla_shape;
+
+typedef struct {
+    float thr;            /* keep the smallest sorted prefix with mass >= 1 - thr; thr in [0, 1] */
+    int32_t use_sta;      /* nonzero: OR in the sliding-tile window below */
+    int32_t wt, wh, ww;   /* STA half-window in tiles along t, h, w (>= 0) */
+} nabla_mask_params;
+
+enum {
+    NABLA_OP_BUILD_MASK = 0,     /* workspace for nabla_build_mask */
+    NABLA_OP_FWD = 1,            /* workspace for bsa_fwd */
+    NABLA_OP_FWD_WITH_MASK = 2   /* workspace for bsa_fwd_with_mask */
+};
+
+/* Bytes of workspace the operation needs for this shape (0 on a bad shape).
+ * The first 256 bytes are a header holding the device status word; zero them
+ * once with nabla_workspace_init() before the first call. */
+NABLA_API size_t nabla_workspace_size(const nabla_shape* shape, int op);
+
+/* Zero the workspace header (status word) on `stream`. */
+NABLA_API nabla_status nabla_workspace_init(void* workspace, nabla_stream_t stream);
+
+/* Read and clear the device status word: synchronises `stream`, returns
+ * NABLA_OK or the first device-side error recorded since the last query. */
+NABLA_API nabla_status nabla_query_status(void* workspace, nabla_stream_t stream);
+
+/*
+ * NABLA mask builder (Algorithm 1 of "NABLA: Neighborhood Adaptive
+ * Block-Level Attention"; its reading in the pith.science review, sections
+ * "What carries the argument" and "Core claim", and referee minor comment 2).
+ * Per head: mean-pool Q and K over each 64-token block, form the reduced map
+ * Qbar Kbar^T / sqrt(d), softmax each row, order each row's blocks by
+ * descending probability (ties: lower block index first) and keep the
+ * smallest prefix whose mass reaches 1 - thr (thr == 0 keeps every block; the
+ * top block is always kept).  With use_sta, OR in the sliding-tile window of
+ * "Sliding Tile Attention" (clipped at the grid edge).  The result is written
+ * as block CSR with ascending column indices per row.
+ *
+ *   q, k          device bf16 [B,H,S,d]
+ *   mask_u8       optional device uint8 [B,H,nb,nb] (1 = kept), or NULL
+ *   row_ptr       device int32 [B*H*nb + 1]
+ *   col_idx       device int32 [col_capacity]; B*H*nb*nb always suffices
+ *   nnz_out       optional device int32 [1]: total kept blocks, or NULL
+ *   workspace     device, nabla_workspace_size(shape, NABLA_OP_BUILD_MASK) bytes
+ * If the kept blocks exceed col_capacity, col_idx is left partly written and
+ * NABLA_ERR_CAPACITY is recorded in the status word; row_ptr is still exact.
+ */
+NABLA_API nabla_status nabla_build_mask(const nabla_shape* shape, const nabla_mask_params* params,
+                              const void* q, const void* k, uint8_t* mask_u8, int32_t* row_ptr,
+                              int32_t* col_idx, int64_t col_capacity, int32_t* nnz_out,
+                              void* workspace, nabla_stream_t stream);
+
+/*
+ * Block-sparse attention forward (FlashAttention's tiled online softmax, as
+ * in the FlashAttention abstract's block-sparse extension; NABLA feeds it the
+ * mask above in place of FlexAttention).  For each query block r of head
+ * (b, h) and each key block j listed in its CSR row, accumulate
+ * softmax(scale * Q_r K_j^T) V_j exactly over the listed blocks.
+ *
+ *   q, k, v       device bf16 [B,H,S,d]
+ *   row_ptr       device int32 [B*H*nb + 1], col_idx device int32 (head-local)
+ *   scale         softmax scale; <= 0 selects 1/sqrt(d)
+ *   o             device bf16 [B,H,S,d]
+ *   lse           device fp32 [B,H,S] (may be NULL)
+ *   workspace     device, nabla_workspace_size(shape, NABLA_OP_FWD) bytes
+ * A query block with an empty list gets O = 0 and LSE = -inf.  Duplicate
+ * column indices count once; indices outside [0, nb) are skipped and recorded
+ * as NABLA_ERR_BAD_INDEX.
+ */
+NABLA_API nabla_status bsa_fwd(const nabla_shape* shape, const void* q, const void* k, const void* v,
+                     const int32_t* row_ptr, const int32_t* col_idx, float scale, void* o,
+                     float* lse, void* workspace, nabla_stream_t stream);
+
+/*
+ * Block-sparse attention forward with a caller-supplied static block mask
+ * (the calibrated per-(timestep, layer, head) masks of "Accelerating
+ * Text-to-Video Generation with Calibrated Sparse Attention", section B
+ * "Inference": precomputed binary masks, only the selected blocks computed).
+ *
+ *   mask_u8       device uint8 [B,H,nb,nb]; nonzero = attend to the block
+ *   workspace     device, nabla_workspace_size(shape, NABLA_OP_FWD_WITH_MASK)
+ * Other arguments as for bsa_fwd.  The mask is compacted to block CSR inside
+ * the workspace, then bsa_fwd runs on it.
+ */
+NABLA_API nabla_status bsa_fwd_with_mask(const nabla_shape* shape, const void* q, const void* k,
+                               const void* v, const uint8_t* mask_u8, float scale, void* o,
+                               float* lse, void* workspace, nabla_stream_t stream);
+
+/* Message for the last error returned on the calling host thread. */
+NABLA_API const char* nabla_last_error(void);
+
+/* ABI version (major * 10000 + minor * 100 + patch). */
+NABLA_API int nabla_version(void);
+
+/*
+ * Diagnostics and tuning (not part of the method).
+ *
+ * nabla_set_wait_limit_ns: time limit of every pipeline wait inside the
+ * attention kernel, in nanoseconds (0 restores the default of 2 s).  A wait
+ * that runs out makes the kernel drain its copies in flight, free its tensor
+ * memory, record NABLA_ERR_TIMEOUT and return.  Tests set a tiny limit to
+ * check that path without hanging anything.
+ *
+ * nabla_set_pv_variant: which tcgen05 form the P.V product uses
+ * (0 = default; 1 = P in shared memory, two N=64 MMAs; 2 = P in shared
+ * memory, one N=d MMA; 3 = P in tensor memory, one N=d MMA).
+ *
+ * nabla_selftest_mma: one 128 x N x 128 bf16 product through the same
+ * tcgen05/TMA building blocks the attention kernel uses, for layout checks.
+ *   variant 0: C[m][n] = sum_k A[m][k] B[n][k]   (both K-major, N = 128)
+ *   variant 1: C[m][n] = sum_k A[m][k] B[k][n]   (B N-major, one N=128 MMA)
+ *   variant 2: as 1 with two N=64 MMAs
+ *   variant 3: as 1 with A staged in tensor memory
+ *   a, b: device bf16 [128][128] row-major; c: device fp32 [128][128].
+ */
+NABLA_API void nabla_set_wait_limit_ns(uint64_t ns);
+NABLA_API void nabla_set_pv_variant(int variant);
+NABLA_API nabla_status nabla_selftest_mma(int variant, const void* a, const void* b, float* c,
+                                void* workspace, nabla_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NABLA_H_ */

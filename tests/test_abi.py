@@ -1,0 +1,120 @@
+"""The C-ABI library: it builds, loads, exports every symbol include/nabla.h
+declares, and rejects bad arguments before touching the GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    text = open(os.path.join(ROOT, "include", "nabla.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"^NABLA_API [\w\s\*]*?\b((?:nabla|bsa)_\w+)\s*\(", text, flags=re.M)
+    return sorted(set(names))
+
+
+@pytest.fixture(scope="module")
+def nl():
+    import block_sparse_attention_23_b200 as nl
+    nl.build()
+    return nl
+
+
+def test_header_declares_the_boundary():
+    names = _declared_functions()
+    for required in ("nabla_build_mask", "bsa_fwd", "bsa_fwd_with_mask", "nabla_workspace_size",
+                     "nabla_last_error", "nabla_query_status"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(nl):
+    lib = nl.lib()
+    for name in _declared_functions():
+        assert hasattr(lib, name), name
+    assert set(_declared_functions()) <= set(nl.EXPORTED)
+
+
+def test_no_torch_types_in_signatures():
+    text = open(os.path.join(ROOT, "include", "nabla.h")).read()
+    assert "torch" not in text.lower().replace("pytorch", "")
+    assert "extern \"C\"" in text
+
+
+def test_version_and_workspace_sizes(nl):
+    lib = nl.lib()
+    assert lib.nabla_version() >= 100
+    s = nl.make_shape(1, 40, 76800, 128, (5, 12, 20))
+    n_fwd = nl.workspace_size(s, nl.OP_FWD)
+    n_build = nl.workspace_size(s, nl.OP_BUILD_MASK)
+    n_mask = nl.workspace_size(s, nl.OP_FWD_WITH_MASK)
+    assert n_fwd == 256
+    nb = 1200
+    # pooled Q and K + reduced map + bitmap + counts
+    assert n_build >= 2 * 40 * nb * 128 * 4 + 40 * nb * nb * 4
+    assert n_mask >= 40 * nb * nb * 4
+
+
+@pytest.mark.parametrize("shape,status", [
+    ((1, 1, 100, 64), 2),          # S % 64 != 0
+    ((1, 1, 128, 96), 2),          # d unsupported
+    ((0, 1, 128, 64), 1),          # bad size
+    ((1, 1, 64 * 4097, 64), 2),    # nb > 4096
+])
+def test_bad_shapes_rejected(nl, shape, status):
+    s = nl.make_shape(*shape)
+    assert nl.lib().nabla_workspace_size(ctypes.byref(s), 0) == 0
+    prm = nl._MaskParams(0.2, 0, 0, 0, 0)
+    null = ctypes.c_void_p(0)
+    dummy = ctypes.c_void_p(1 << 20)
+    rc = nl.lib().nabla_build_mask(ctypes.byref(s), ctypes.byref(prm), dummy, dummy, null, dummy,
+                                   dummy, 10, null, dummy, null)
+    assert rc == status
+
+
+def test_argument_errors_before_any_cuda_call(nl):
+    lib = nl.lib()
+    null = ctypes.c_void_p(0)
+    a = ctypes.c_void_p(1 << 20)
+    s = nl.make_shape(1, 1, 128, 64, (1, 1, 2))
+    prm = nl._MaskParams(0.2, 0, 0, 0, 0)
+    assert lib.nabla_build_mask(None, ctypes.byref(prm), a, a, null, a, a, 4, null, a, null) == 1
+    assert lib.nabla_build_mask(ctypes.byref(s), None, a, a, null, a, a, 4, null, a, null) == 1
+    bad = nl._MaskParams(1.5, 0, 0, 0, 0)
+    assert lib.nabla_build_mask(ctypes.byref(s), ctypes.byref(bad), a, a, null, a, a, 4, null, a,
+                                null) == 2
+    wrong_grid = nl.make_shape(1, 1, 128, 64, (1, 1, 3))
+    assert lib.nabla_build_mask(ctypes.byref(wrong_grid), ctypes.byref(prm), a, a, null, a, a, 4,
+                                null, a, null) == 1
+    neg = nl._MaskParams(0.2, 1, -1, 0, 0)
+    assert lib.nabla_build_mask(ctypes.byref(s), ctypes.byref(neg), a, a, null, a, a, 4, null, a,
+                                null) == 1
+    # null q / misaligned pointers
+    assert lib.bsa_fwd(ctypes.byref(s), null, a, a, a, a, 0.0, a, null, a, null) == 1
+    odd = ctypes.c_void_p((1 << 20) + 2)
+    assert lib.bsa_fwd(ctypes.byref(s), odd, a, a, a, a, 0.0, a, null, a, null) == 1
+    assert lib.bsa_fwd_with_mask(ctypes.byref(s), a, a, a, null, 0.0, a, null, a, null) == 1
+    assert lib.bsa_fwd(ctypes.byref(s), a, a, a, a, a, float("nan"), a, null, a, null) == 1
+    assert "scale" in lib.nabla_last_error().decode()
+    assert lib.nabla_selftest_mma(7, a, a, a, a, null) == 1
+
+
+def test_product_path_has_no_cpu_fallback(nl):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("CUDA present")
+    q = torch.zeros((1, 1, 64, 64), dtype=torch.bfloat16)
+    with pytest.raises(RuntimeError):
+        nl.bsa_fwd_with_mask(q, q, q, torch.ones((1, 1, 1, 1), dtype=torch.uint8))
+
+
+def test_package_does_not_import_oracle():
+    pkg = os.path.join(ROOT, "block_sparse_attention_23_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h", ".c")):
+                text = open(os.path.join(dirpath, f)).read()
+                assert "import oracle" not in text and "from oracle" not in text, f
+                assert "nabla_oracle" not in text, f

@@ -1,0 +1,26 @@
+"""tcgen05 / TMA building blocks: one 128x128x128 bf16 product per operand form,
+checked against a float64 matmul of the same bf16 values."""
+import numpy as np
+import pytest
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def nl():
+    import block_sparse_attention_23_b200 as nl
+    nl.lib()
+    return nl
+
+
+@pytest.mark.parametrize("variant", [0, 1, 2, 3])
+def test_mma_selftest(nl, variant):
+    import torch
+    g = torch.Generator().manual_seed(variant)
+    a = torch.randn(128, 128, generator=g).to(torch.bfloat16)
+    b = torch.randn(128, 128, generator=g).to(torch.bfloat16)
+    c = nl.selftest_mma(variant, a.cuda(), b.cuda()).cpu().numpy().astype(np.float64)
+    A = a.double().numpy()
+    Bm = b.double().numpy()
+    want = A @ Bm.T if variant == 0 else A @ Bm
+    np.testing.assert_allclose(c, want, rtol=0, atol=2e-3)
