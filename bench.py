@@ -1,0 +1,395 @@
+#!/usr/bin/env python
+"""Benchmark: one NABLA attention layer (mask build + block-sparse forward).
+
+A step is one pass of the whole hot path over one synthetic layer: pool Q/K,
+reduced map, row softmax + prefix selection + STA union, CSR compaction
+(nabla_build_mask), then the block-sparse attention forward (bsa_fwd).  The
+workload is the Wan-2.1-14B-720p-shaped layer: B=1, 40 heads, d=128, token grid
+20x48x80 (76,800 tokens, 1,200 blocks), thr=0.2, STA window (1,2,2) tiles.
+
+Metric: kept-block TFLOP/s (4*d*64^2 per kept block pair, summed over heads)
+over the step time, plus ms per layer and the fraction of dense-BF16 peak.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Multi-GPU (torchrun): every rank runs the full layer on its own replica inputs
+(weak scaling; the path shards by head with no data exchange); the time is the
+max over ranks.  ``--impl reference`` times the fp64 CPU oracle on a bounded
+sample of the same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOAD = "wan720p"
+METRIC = "kept-block attn TFLOP/s & ms/layer at 76.8k tokens; % of dense BF16 peak"
+ATTN_SRC = os.path.join(ROOT, "block_sparse_attention_23_b200", "csrc", "attn_kernel.cu")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "bsa_fwd_wan720p_traffic.json")
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+def _attn_src_sha():
+    return hashlib.sha256(open(ATTN_SRC, "rb").read()).hexdigest()[:16]
+
+
+def _traffic_per_launch():
+    """DRAM bytes per bsa_fwd launch from a committed ncu capture, or None if the
+    kernel source changed since the capture."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None
+    d = json.load(open(TRAFFIC_FILE))
+    if d.get("attn_src_sha") != _attn_src_sha():
+        return None
+    return d.get("bytes_per_launch")
+
+
+def _workload_desc(w):
+    T, Hh, W = w.grid
+    sta = f"STA half-window {w.sta} tiles" if w.sta else "no STA"
+    return (f"{w.name}: B={w.B} H={w.H} d={w.d} grid {T}x{Hh}x{W} ({w.S} tokens, {w.nb} blocks), "
+            f"thr={w.thr}, {sta}, Q,K = {w.pos_weight}*e(t,h,w) + {w.noise_weight}*z, V ~ N(0,1)")
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}",
+                                          f"--query-gpu={self.FIELDS}", "--format=csv,noheader",
+                                          "-lms", "200"], stdout=self.fh,
+                                         stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.fh.close()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [s.strip() for s in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1].split()[0]))
+                mx = float(parts[2].split()[0])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def _dist():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def _init_pg(ws, backend):
+    import torch.distributed as dist
+    from datetime import timedelta
+    if ws > 1 and not dist.is_initialized():
+        dist.init_process_group(backend=backend, timeout=timedelta(seconds=120))
+    return dist
+
+
+def _max_over_ranks(x: float, ws: int, device) -> float:
+    if ws == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ CPU oracle
+def oracle_sample(w, q, k, v, nrows: int, head: int = 0, seed: int = 0):
+    """Time the fp64 oracle on one head's full mask plus `nrows` sampled query
+    rows of that head; return (TFLOP/s of kept-block work, seconds, description)."""
+    import oracle
+    S, nb = w.S, w.nb
+    qh, kh, vh = q[:, head:head + 1], k[:, head:head + 1], v[:, head:head + 1]
+    t0 = time.perf_counter()
+    mask = oracle.build_mask(qh, kh, w.tile_grid, w.thr, w.sta)
+    t_mask = time.perf_counter() - t0
+    rng = np.random.default_rng(seed)
+    rows = np.sort(rng.choice(S, size=nrows, replace=False)).astype(np.int64)
+    t1 = time.perf_counter()
+    oracle.masked_attention(qh, kh, vh, mask, rows)
+    t_attn = time.perf_counter() - t1
+    kept_blocks = mask[0, 0].sum(axis=1)[rows // 64]
+    flops = float((4.0 * w.d * 64 * kept_blocks).sum())
+    t = t_attn + t_mask * nrows / S      # the mask cost of the sampled rows' share
+    desc = (f"head {head}: full oracle mask ({t_mask:.2f} s, charged pro rata) + oracle "
+            f"attention on {nrows} seeded query rows ({t_attn:.2f} s)")
+    return flops / t / 1e12, t, desc
+
+
+def run_reference(args):
+    ws, rank, _ = _dist()
+    if rank != 0:
+        return 0
+    import oracle
+    import synth
+    oracle.build()
+    w = synth.WORKLOADS[WORKLOAD]
+    q, k, v = synth.make_qkv(w)
+    cores = oracle.max_threads()
+    nrows = args.ref_rows
+    for i in range(args.warmup):
+        oracle_sample(w, q, k, v, nrows, head=i % w.H, seed=i)
+    vals, times, desc = [], [], ""
+    for i in range(args.steps):
+        val, t, desc = oracle_sample(w, q, k, v, nrows, head=(args.warmup + i) % w.H,
+                                     seed=1000 + i)
+        vals.append(val)
+        times.append(t)
+    value = float(np.mean(vals))
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": float(np.mean(times)) * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": _workload_desc(w), "global_batch": w.B, "seq_len": w.S,
+                   "parallelism": "cpu oracle (fp64, OpenMP)"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": f"per step: {desc}"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ GPU arm
+def run_ours(args):
+    import torch
+    ws, rank, local = _dist()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = _init_pg(ws, "nccl")
+    import synth
+    import block_sparse_attention_23_b200 as nl
+    nl.lib()
+    w = synth.WORKLOADS[WORKLOAD]
+    if args.profile_heads:
+        import dataclasses
+        w = dataclasses.replace(w, H=args.profile_heads)   # profiling subset, not a bench line
+    peaks = _peaks()
+
+    # inputs: generated on the host (pinned, for the end-to-end leg), resident copies in HBM
+    q16, k16, v16 = synth.make_qkv(w, seed=args.seed + rank)
+    pinned = []
+    for a in (q16, k16, v16):
+        t = torch.empty(a.shape, dtype=torch.bfloat16, pin_memory=True)
+        t.view(torch.int16).numpy()[...] = a.view(np.int16)
+        pinned.append(t)
+    q, k, v = (t.to(dev) for t in pinned)
+    B, H, S, d = q.shape
+    nb = S // 64
+    shape = nl.make_shape(B, H, S, d, w.tile_grid)
+    ws_mask = nl.Workspace.create(shape, nl.OP_BUILD_MASK, dev)
+    ws_fwd = nl.Workspace.create(shape, nl.OP_FWD, dev)
+    cap = B * H * nb * nb
+    mask_out = (torch.empty(B * H * nb + 1, dtype=torch.int32, device=dev),
+                torch.empty(cap, dtype=torch.int32, device=dev),
+                torch.empty(1, dtype=torch.int32, device=dev), None)
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, S), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        row_ptr, col_idx, nnz, _ = nl.nabla_build_mask(q, k, w.tile_grid, w.thr, w.sta,
+                                                       workspace=ws_mask, out=mask_out)
+        nl.bsa_fwd(q, k, v, row_ptr, col_idx, workspace=ws_fwd, out=(o, lse))
+
+    step()
+    torch.cuda.synchronize()
+    ws_mask.check()
+    ws_fwd.check()
+    kept = int(mask_out[2].item())
+    kept_flops = 4.0 * d * 64 * 64 * kept
+    mask_bytes = 2.0 * B * H * S * d * 2 + 4.0 * kept + 4.0 * (B * H * nb + 1)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if ws > 1:
+        dist.barrier()
+    clocks = ClockSampler(local)
+    clocks.start()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    t_start.record(stream)
+    for i in range(args.steps):
+        e0, e1, e2 = ev[i]
+        e0.record(stream)
+        row_ptr, col_idx, nnz, _ = nl.nabla_build_mask(q, k, w.tile_grid, w.thr, w.sta,
+                                                       workspace=ws_mask, out=mask_out)
+        e1.record(stream)
+        nl.bsa_fwd(q, k, v, row_ptr, col_idx, workspace=ws_fwd, out=(o, lse))
+        e2.record(stream)
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    if ws > 1:
+        dist.barrier()
+    total_ms = t_start.elapsed_time(t_end)
+    mask_ms = float(np.mean([a.elapsed_time(b) for a, b, _ in ev]))
+    attn_ms = float(np.mean([b.elapsed_time(c) for _, b, c in ev]))
+    total_ms_max = _max_over_ranks(total_ms, ws, dev)
+    ms_per_step = total_ms_max / args.steps
+    value = kept_flops * ws / (ms_per_step * 1e-3) / 1e12
+    ws_mask.check()
+    ws_fwd.check()
+
+    # end to end through the public API with host buffers: H2D of Q, K, V from
+    # pinned memory, mask + attention, D2H of O and LSE, every step
+    o_host = torch.empty(o.shape, dtype=torch.bfloat16, pin_memory=True)
+    lse_host = torch.empty(lse.shape, dtype=torch.float32, pin_memory=True)
+    qd, kd, vd = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+
+    def e2e_step():
+        qd.copy_(pinned[0], non_blocking=True)
+        kd.copy_(pinned[1], non_blocking=True)
+        vd.copy_(pinned[2], non_blocking=True)
+        row_ptr, col_idx, nnz, _ = nl.nabla_build_mask(qd, kd, w.tile_grid, w.thr, w.sta,
+                                                       workspace=ws_mask, out=mask_out)
+        nl.bsa_fwd(qd, kd, vd, row_ptr, col_idx, workspace=ws_fwd, out=(o, lse))
+        o_host.copy_(o, non_blocking=True)
+        lse_host.copy_(lse, non_blocking=True)
+
+    e2e_steps = max(1, min(args.steps, 5))
+    e2e_step()
+    torch.cuda.synchronize()
+    if ws > 1:
+        dist.barrier()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = _max_over_ranks(a.elapsed_time(b), ws, dev) / e2e_steps
+    e2e_val = kept_flops * ws / (e2e_ms * 1e-3) / 1e12
+    h2d = sum(t.numel() * t.element_size() for t in pinned)
+    d2h = o_host.numel() * 2 + lse_host.numel() * 4
+
+    attn_tflops = kept_flops / (attn_ms * 1e-3) / 1e12
+    peak = peaks["bf16_tflops_sustained"]
+    traffic = _traffic_per_launch()
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": ws,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": _workload_desc(w), "global_batch": B * ws, "seq_len": S,
+                   "heads": H, "head_dim": d,
+                   "parallelism": "replicas" if ws > 1 else "single GPU",
+                   "l2": "inputs (Q,K,V 2.36 GB per rank) larger than L2; no flush",
+                   "kept_blocks": kept, "density": kept / (B * H * nb * nb),
+                   "mask_arith": "fp64", "attn_arith": "bf16 MMA, fp32 accumulate"},
+        "ms_per_layer": ms_per_step, "mask_ms": mask_ms, "attn_ms": attn_ms,
+        "attn_kept_tflops": attn_tflops,
+        "pct_of_dense_bf16_peak": {"attn_vs_sustained": attn_tflops / peak,
+                                   "attn_vs_burst": attn_tflops / peaks["bf16_tflops"],
+                                   "layer_vs_sustained": value / ws / peak},
+        "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": peak,
+                     "unit": "TFLOP/s", "frac": attn_tflops / peak,
+                     "traffic": traffic, "kernel": "bsa_fwd_kernel",
+                     "peak_source": f"{peaks['source']} bf16 sustained (cuBLAS, power-capped)"},
+        "mask_roofline": {"bound": "hbm", "achieved": mask_bytes / (mask_ms * 1e-3) / 1e9,
+                          "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                          "frac": mask_bytes / (mask_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                          "bytes": mask_bytes},
+        "e2e": {"value": e2e_val, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": 6 * args.steps,
+        "clocks": clk,
+    }
+    if args.profile_heads:
+        line["config"]["profiling_subset_heads"] = args.profile_heads
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        import oracle
+        oracle.build()
+        val, t, desc = oracle_sample(w, q16, k16, v16, args.ref_rows, head=0, seed=0)
+        line["cpu_baseline"] = {"value": val, "unit": "TFLOP/s", "cores": oracle.max_threads(),
+                                "kind": "oracle", "sample": desc}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--ref-rows", type=int, default=2048,
+                    help="oracle attention rows per CPU sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile-heads", type=int, default=0,
+                    help="profiling only: run the layer with this many heads")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        print("warning: fewer than 3 warm-up steps", file=sys.stderr)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -33,13 +33,14 @@ namespace nabla {
 
 // ------------------------------------------------------------------ pooling
 // One warp per (tensor, bh, block): 64 rows of d bf16.  A row is d/8 16-byte
-// chunks; the warp covers 32/(d/8) rows per step with 128-bit loads.
+// chunks; the warp covers 32/(d/8) rows per step with 128-bit loads.  Sums are
+// fp64, so the mean of 64 bf16 values is exact.
 template <int D>
 __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restrict__ q,
                                                    const __nv_bfloat16* __restrict__ k,
-                                                   float* __restrict__ qbar,
-                                                   float* __restrict__ kbar, int64_t nblocks) {
-  constexpr int kLanesPerRow = D / 8;            // 16 (d=128) or 8 (d=64)
+                                                   double* __restrict__ qbar,
+                                                   double* __restrict__ kbar, int64_t nblocks) {
+  constexpr int kLanesPerRow = D / 8;              // 16 (d=128) or 8 (d=64)
   constexpr int kRowsPerStep = 32 / kLanesPerRow;  // 2 or 4
   constexpr int kSteps = 64 / kRowsPerStep;        // 32 or 16
   const int lane = threadIdx.x & 31;
@@ -48,12 +49,12 @@ __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restri
   const bool is_k = wid >= nblocks;
   const int64_t blk = is_k ? wid - nblocks : wid;
   const __nv_bfloat16* src = (is_k ? k : q) + blk * 64 * D;
-  float* dst = (is_k ? kbar : qbar) + blk * D;
+  double* dst = (is_k ? kbar : qbar) + blk * D;
   const int chunk = lane % kLanesPerRow;
   const int sub = lane / kLanesPerRow;
-  float acc[8];
+  double acc[8];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+  for (int i = 0; i < 8; ++i) acc[i] = 0.0;
 #pragma unroll 8
   for (int s = 0; s < kSteps; ++s) {
     const int row = s * kRowsPerStep + sub;
@@ -61,8 +62,8 @@ __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restri
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      acc[2 * i] += __uint_as_float(w[i] << 16);
-      acc[2 * i + 1] += __uint_as_float(w[i] & 0xFFFF0000u);
+      acc[2 * i] += static_cast<double>(__uint_as_float(w[i] << 16));
+      acc[2 * i + 1] += static_cast<double>(__uint_as_float(w[i] & 0xFFFF0000u));
     }
   }
   // combine the row groups (fixed order: deterministic)
@@ -72,67 +73,70 @@ __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restri
     for (int i = 0; i < 8; ++i) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], off);
   }
   if (sub == 0) {
-    float4* out = reinterpret_cast<float4*>(dst + chunk * 8);
-    out[0] = make_float4(acc[0] * (1.f / 64), acc[1] * (1.f / 64), acc[2] * (1.f / 64),
-                         acc[3] * (1.f / 64));
-    out[1] = make_float4(acc[4] * (1.f / 64), acc[5] * (1.f / 64), acc[6] * (1.f / 64),
-                         acc[7] * (1.f / 64));
+    double2* out = reinterpret_cast<double2*>(dst + chunk * 8);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      out[i] = make_double2(acc[2 * i] * (1.0 / 64), acc[2 * i + 1] * (1.0 / 64));
   }
 }
 
 // ------------------------------------------------------------------ reduced map
-// Per head: L = Qbar Kbar^T * inv_sqrt_d, 64x64 output tile per CTA, 4x4 per
-// thread, the whole d extent staged transposed in shared memory.  Every
-// element is one fixed-order fp32 FMA chain over k (deterministic).
+// Per head: L = Qbar Kbar^T * inv_sqrt_d in fp64.  128x128 output tile per CTA
+// of 256 threads; each thread owns rows {2ty, 2ty+1} + 32i and columns
+// {2tx, 2tx+1} + 32j (i, j < 4), so its shared-memory reads are 16-byte
+// vectors that are broadcast (A) or contiguous across the half-warp (B).
+// k is staged in chunks of 16.  Every element is one fixed-order FMA chain.
+constexpr int kLgT = 128, kLgK = 16, kLgLD = kLgT + 2;
+
 template <int D>
-__global__ void __launch_bounds__(256) logits_kernel(const float* __restrict__ qbar,
-                                                     const float* __restrict__ kbar,
-                                                     float* __restrict__ L, int nb,
-                                                     float inv_sqrt_d) {
-  constexpr int T = 64, LD = T + 4;
-  extern __shared__ float4 logits_smem4[];
-  float* As = reinterpret_cast<float*>(logits_smem4);  // [D][LD]: As[k][m]
-  float* Bs = As + D * LD;                             // [D][LD]: Bs[k][n]
+__global__ void __launch_bounds__(256) logits_kernel(const double* __restrict__ qbar,
+                                                     const double* __restrict__ kbar,
+                                                     double* __restrict__ L, int nb,
+                                                     double inv_sqrt_d) {
+  __shared__ __align__(16) double As[kLgK][kLgLD];   // As[k][m]
+  __shared__ __align__(16) double Bs[kLgK][kLgLD];   // Bs[k][n]
   const int bh = blockIdx.z;
-  const int m0 = blockIdx.y * T, n0 = blockIdx.x * T;
-  const float* qa = qbar + static_cast<int64_t>(bh) * nb * D;
-  const float* ka = kbar + static_cast<int64_t>(bh) * nb * D;
-  const int tid = threadIdx.x;
-  for (int i = tid; i < T * (D / 4); i += 256) {
-    const int r = i % T, c4 = i / T;   // consecutive threads: consecutive smem columns
-    float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
-    if (m0 + r < nb) a = *reinterpret_cast<const float4*>(qa + static_cast<int64_t>(m0 + r) * D + 4 * c4);
-    if (n0 + r < nb) b = *reinterpret_cast<const float4*>(ka + static_cast<int64_t>(n0 + r) * D + 4 * c4);
-    As[(4 * c4 + 0) * LD + r] = a.x; As[(4 * c4 + 1) * LD + r] = a.y;
-    As[(4 * c4 + 2) * LD + r] = a.z; As[(4 * c4 + 3) * LD + r] = a.w;
-    Bs[(4 * c4 + 0) * LD + r] = b.x; Bs[(4 * c4 + 1) * LD + r] = b.y;
-    Bs[(4 * c4 + 2) * LD + r] = b.z; Bs[(4 * c4 + 3) * LD + r] = b.w;
+  const int m0 = blockIdx.y * kLgT, n0 = blockIdx.x * kLgT;
+  const double* qa = qbar + static_cast<int64_t>(bh) * nb * D;
+  const double* ka = kbar + static_cast<int64_t>(bh) * nb * D;
+  const int tid = threadIdx.x, ty = tid / 16, tx = tid % 16;
+  double acc[8][8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[i][j] = 0.0;
+  for (int kc = 0; kc < D; kc += kLgK) {
+    __syncthreads();
+    for (int i = tid; i < kLgT * kLgK; i += 256) {
+      const int r = i / kLgK, kk = i % kLgK;   // consecutive threads: consecutive k (coalesced)
+      As[kk][r] = (m0 + r < nb) ? qa[static_cast<int64_t>(m0 + r) * D + kc + kk] : 0.0;
+      Bs[kk][r] = (n0 + r < nb) ? ka[static_cast<int64_t>(n0 + r) * D + kc + kk] : 0.0;
+    }
+    __syncthreads();
+#pragma unroll 4
+    for (int kk = 0; kk < kLgK; ++kk) {
+      double a[8], b[8];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const double2 va = *reinterpret_cast<const double2*>(&As[kk][2 * ty + 32 * i]);
+        const double2 vb = *reinterpret_cast<const double2*>(&Bs[kk][2 * tx + 32 * i]);
+        a[2 * i] = va.x; a[2 * i + 1] = va.y;
+        b[2 * i] = vb.x; b[2 * i + 1] = vb.y;
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[i][j] = fma(a[i], b[j], acc[i][j]);
+    }
   }
-  __syncthreads();
-  const int ty = tid / 16, tx = tid % 16;
-  float acc[4][4];
+  double* out = L + static_cast<int64_t>(bh) * nb * nb;
 #pragma unroll
-  for (int i = 0; i < 4; ++i)
-#pragma unroll
-    for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
-#pragma unroll 8
-  for (int kk = 0; kk < D; ++kk) {
-    const float4 a = *reinterpret_cast<const float4*>(As + kk * LD + ty * 4);
-    const float4 b = *reinterpret_cast<const float4*>(Bs + kk * LD + tx * 4);
-    const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
-  }
-  float* out = L + static_cast<int64_t>(bh) * nb * nb;
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int m = m0 + ty * 4 + i;
+  for (int i = 0; i < 8; ++i) {
+    const int m = m0 + 2 * ty + 32 * (i >> 1) + (i & 1);
     if (m >= nb) continue;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int n = n0 + tx * 4 + j;
+    for (int j = 0; j < 8; ++j) {
+      const int n = n0 + 2 * tx + 32 * (j >> 1) + (j & 1);
       if (n < nb) out[static_cast<int64_t>(m) * nb + n] = acc[i][j] * inv_sqrt_d;
     }
   }
@@ -140,17 +144,17 @@ __global__ void __launch_bounds__(256) logits_kernel(const float* __restrict__ q
 
 // ------------------------------------------------------------------ selection
 
-// Butterfly sum; lanes may differ in the last ulp (different association), so
+// Butterfly sums; lanes may differ in the last ulp (different association), so
 // lane 0's value is broadcast: every lane takes the same branch on it.
-__device__ __forceinline__ float warp_sum(float v) {
+__device__ __forceinline__ double warp_sum(double v) {
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
   return __shfl_sync(0xffffffffu, v, 0);
 }
 
-__device__ __forceinline__ float warp_max(float v) {
+__device__ __forceinline__ double warp_max(double v) {
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
+  for (int off = 16; off > 0; off >>= 1) v = fmax(v, __shfl_xor_sync(0xffffffffu, v, off));
   return v;
 }
 
@@ -160,13 +164,11 @@ __device__ __forceinline__ uint32_t warp_max_u32(uint32_t v) {
   return v;
 }
 
-// Mass of the row at or above bit pattern v (p >= 0, so bit order = value order).
-__device__ __forceinline__ float mass_at_or_above(const float* p, int nb, int lane, uint32_t v) {
-  float s = 0.f;
-  for (int c = lane; c < nb; c += 32) {
-    const float x = p[c];
-    s += (__float_as_uint(x) >= v) ? x : 0.f;
-  }
+// fp64 mass of the entries whose ordering key is at least v.
+__device__ __forceinline__ double mass_at_or_above(const double* p, const uint32_t* key, int nb,
+                                                   int lane, uint32_t v) {
+  double s = 0.0;
+  for (int c = lane; c < nb; c += 32) s += (key[c] >= v) ? p[c] : 0.0;
   return warp_sum(s);
 }
 
@@ -176,95 +178,105 @@ struct SelectParams {
   int Tt, Th, Tw;
 };
 
-// One warp per row g = bh*nb + r.  Dynamic shared memory: 8 rows x nb floats.
-__global__ void __launch_bounds__(256) select_kernel(const float* __restrict__ L, int64_t nrows,
-                                                     int nb, SelectParams prm,
+// One warp per row g = bh*nb + r; `wpc` warps per CTA.  Shared memory per warp:
+// p (fp64, nb) and its ordering key (nb x u32).  Softmax and every mass sum
+// are fp64.  Rows are ordered by the key = bit pattern of fp32(p), ties by
+// block index: entries whose fp64 probabilities differ by less than one fp32
+// ulp (relative 6e-8) are ordered by index.
+__global__ void __launch_bounds__(256) select_kernel(const double* __restrict__ L, int64_t nrows,
+                                                     int nb, int wpc, SelectParams prm,
                                                      uint32_t* __restrict__ bits,
                                                      int32_t* __restrict__ counts,
                                                      uint8_t* __restrict__ mask_u8) {
-  extern __shared__ float sel_smem[];
+  extern __shared__ double sel_smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t g = static_cast<int64_t>(blockIdx.x) * 8 + warp;
+  const int64_t g = static_cast<int64_t>(blockIdx.x) * wpc + warp;
   if (g >= nrows) return;
   const int r = static_cast<int>(g % nb);
   const int nw = (nb + 31) >> 5;
-  float* p = sel_smem + warp * nb;
-  const float* Lrow = L + g * nb;
+  double* p = sel_smem + static_cast<int64_t>(warp) * nb;
+  uint32_t* key = reinterpret_cast<uint32_t*>(sel_smem + static_cast<int64_t>(wpc) * nb) +
+                  static_cast<int64_t>(warp) * nb;
+  const double* Lrow = L + g * nb;
 
-  // softmax over the row (max subtracted), p = e / Z
-  float mx = -INFINITY;
+  // softmax over the row (max subtracted), p = e / Z, all fp64
+  double mx = -INFINITY;
   for (int c = lane; c < nb; c += 32) {
-    const float x = Lrow[c];
+    const double x = Lrow[c];
     p[c] = x;
-    mx = fmaxf(mx, x);
+    mx = fmax(mx, x);
   }
   mx = warp_max(mx);
-  float z = 0.f;
+  double z = 0.0;
   for (int c = lane; c < nb; c += 32) {
-    const float e = expf(p[c] - mx);
+    const double e = exp(p[c] - mx);
     p[c] = e;
     z += e;
   }
   z = warp_sum(z);
-  uint32_t pmax_bits = 0;
+  uint32_t kmax = 0;
   for (int c = lane; c < nb; c += 32) {
-    const float v = p[c] / z;
+    const double v = p[c] / z;
     p[c] = v;
-    pmax_bits = max(pmax_bits, __float_as_uint(v));
+    const uint32_t kv = __float_as_uint(__double2float_rn(v));
+    key[c] = kv;
+    kmax = max(kmax, kv);
   }
-  pmax_bits = warp_max_u32(pmax_bits);
+  kmax = warp_max_u32(kmax);
   __syncwarp();
 
-  // threshold v*: largest bit pattern whose mass-at-or-above reaches 1 - thr
-  const float target = 1.f - prm.thr;
+  // v*: largest key whose mass-at-or-above reaches 1 - thr.  Entries with a
+  // larger key are kept; entries with key v* are taken in block order while
+  // the exclusive prefix mass stays below the target.  The first entry of the
+  // sorted row is always kept.
+  const double target = 1.0 - static_cast<double>(prm.thr);
   bool keep_all = prm.thr <= 0.f;
-  uint32_t vstar = pmax_bits;
-  int tied_keep = 1;
-  if (!keep_all) {
-    if (target > 0.f) {
-      const float total = mass_at_or_above(p, nb, lane, 0u);
-      if (total < target) {
-        keep_all = true;   // every exclusive prefix stays below the target
-      } else {
-        uint32_t lo = 0u, hi = pmax_bits + 1u;   // mass(lo) >= target > mass(hi)
-        while (hi - lo > 1u) {
-          const uint32_t mid = lo + ((hi - lo) >> 1);
-          if (mass_at_or_above(p, nb, lane, mid) >= target) lo = mid; else hi = mid;
-        }
-        vstar = lo;
-        const float above = mass_at_or_above(p, nb, lane, vstar + 1u);   // < target
-        const float pv = __uint_as_float(vstar);
-        int ntied = 0;
-        for (int c = lane; c < nb; c += 32) ntied += __float_as_uint(p[c]) == vstar;
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) ntied += __shfl_xor_sync(0xffffffffu, ntied, off);
-        // tied entries in block order: entry j (0-based) is kept iff above + j*pv < target
-        int j = 1;
-        while (j < ntied && above + static_cast<float>(j) * pv < target) ++j;
-        tied_keep = j;
+  uint32_t vstar = kmax;
+  double above = 0.0;
+  if (!keep_all && target > 0.0) {
+    const double total = mass_at_or_above(p, key, nb, lane, 0u);
+    if (total < target) {
+      keep_all = true;   // every exclusive prefix stays below the target
+    } else {
+      uint32_t lo = 0u, hi = kmax + 1u;   // mass(lo) >= target > mass(hi)
+      while (hi - lo > 1u) {
+        const uint32_t mid = lo + ((hi - lo) >> 1);
+        if (mass_at_or_above(p, key, nb, lane, mid) >= target) lo = mid; else hi = mid;
       }
+      vstar = lo;
+      above = mass_at_or_above(p, key, nb, lane, vstar + 1u);   // < target
     }
-    // target <= 0 (thr >= 1): only the first entry of the top value (vstar = pmax)
   }
 
   // flags -> bitmap words, optional uint8 row, STA union, counts
   const int rt = r / (prm.Th * prm.Tw), rh = (r / prm.Tw) % prm.Th, rw = r % prm.Tw;
-  int tied_seen = 0, count = 0;
+  double carry = above;        // exclusive prefix mass before the next tied entry
+  bool first_tied = true;      // no tied entry seen yet
+  int count = 0;
   uint32_t* brow = bits + g * nw;
   uint8_t* mrow = mask_u8 ? mask_u8 + g * nb : nullptr;
   for (int w = 0; w < nw; ++w) {
     const int c = w * 32 + lane;
     const bool inrow = c < nb;
-    const uint32_t b = inrow ? __float_as_uint(p[c]) : 0u;
     bool keep;
     if (keep_all) {   // warp-uniform branch
       keep = inrow;
     } else {
-      const bool tied = inrow && b == vstar;
+      const uint32_t kv = inrow ? key[c] : 0u;
+      const bool tied = inrow && kv == vstar;
+      const double pv = tied ? p[c] : 0.0;
+      double incl = pv;   // inclusive scan of tied masses across lanes (lane order)
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const double y = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += y;
+      }
       const uint32_t tb = __ballot_sync(0xffffffffu, tied);
-      const int rank = tied_seen + __popc(tb & ((1u << lane) - 1u));
-      tied_seen += __popc(tb);
-      keep = inrow && (b > vstar || (tied && rank < tied_keep));
+      const bool is_first = first_tied && tied && (tb & ((1u << lane) - 1u)) == 0u;
+      const double excl = carry + (incl - pv);
+      keep = inrow && (kv > vstar || (tied && (excl < target || (is_first && vstar == kmax))));
+      carry += __shfl_sync(0xffffffffu, incl, 31);
+      if (tb) first_tied = false;
     }
     if (inrow && prm.use_sta) {
       const int ct = c / (prm.Th * prm.Tw), ch = (c / prm.Tw) % prm.Th, cw = c % prm.Tw;
@@ -380,8 +392,8 @@ __global__ void __launch_bounds__(256) fill_kernel(const uint32_t* __restrict__ 
 
 // ------------------------------------------------------------------ launchers
 
-cudaError_t launch_pool(const void* q, const void* k, float* qbar, float* kbar, int64_t nblocks,
-                        int d, cudaStream_t st) {
+cudaError_t launch_pool(const void* q, const void* k, double* qbar, double* kbar,
+                        int64_t nblocks, int d, cudaStream_t st) {
   const int64_t warps = 2 * nblocks;
   const unsigned grid = static_cast<unsigned>((warps * 32 + 255) / 256);
   if (d == 128)
@@ -395,36 +407,30 @@ cudaError_t launch_pool(const void* q, const void* k, float* qbar, float* kbar, 
   return cudaGetLastError();
 }
 
-cudaError_t launch_logits(const float* qbar, const float* kbar, float* L, int BH, int nb, int d,
-                          cudaStream_t st) {
-  const dim3 grid((nb + 63) / 64, (nb + 63) / 64, BH);
-  const size_t smem = 2ull * d * 68 * sizeof(float);
-  const float inv = 1.0f / sqrtf(static_cast<float>(d));
-  cudaError_t e;
-  if (d == 128) {
-    e = cudaFuncSetAttribute(logits_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-    logits_kernel<128><<<grid, 256, smem, st>>>(qbar, kbar, L, nb, inv);
-  } else {
-    e = cudaFuncSetAttribute(logits_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-    logits_kernel<64><<<grid, 256, smem, st>>>(qbar, kbar, L, nb, inv);
-  }
+cudaError_t launch_logits(const double* qbar, const double* kbar, double* L, int BH, int nb,
+                          int d, cudaStream_t st) {
+  const dim3 grid((nb + kLgT - 1) / kLgT, (nb + kLgT - 1) / kLgT, BH);
+  const double inv = 1.0 / sqrt(static_cast<double>(d));
+  if (d == 128)
+    logits_kernel<128><<<grid, 256, 0, st>>>(qbar, kbar, L, nb, inv);
+  else
+    logits_kernel<64><<<grid, 256, 0, st>>>(qbar, kbar, L, nb, inv);
   return cudaGetLastError();
 }
 
-cudaError_t launch_select(const float* L, int64_t nrows, int nb, float thr, int use_sta, int wt,
+cudaError_t launch_select(const double* L, int64_t nrows, int nb, float thr, int use_sta, int wt,
                           int wh, int ww, int Tt, int Th, int Tw, uint32_t* bits, int32_t* counts,
                           uint8_t* mask_u8, cudaStream_t st) {
   SelectParams prm{thr, use_sta, wt, wh, ww, Tt, Th, Tw};
-  const size_t smem = 8ull * nb * sizeof(float);
+  const size_t per_warp = static_cast<size_t>(nb) * (sizeof(double) + sizeof(uint32_t));
+  int wpc = static_cast<int>((200u * 1024u) / per_warp);
+  wpc = wpc < 1 ? 1 : (wpc > 8 ? 8 : wpc);
+  const size_t smem = per_warp * wpc;
   cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  const unsigned grid = static_cast<unsigned>((nrows + 7) / 8);
-  select_kernel<<<grid, 256, smem, st>>>(L, nrows, nb, prm, bits, counts, mask_u8);
+  const unsigned grid = static_cast<unsigned>((nrows + wpc - 1) / wpc);
+  select_kernel<<<grid, 32 * wpc, smem, st>>>(L, nrows, nb, wpc, prm, bits, counts, mask_u8);
   return cudaGetLastError();
 }
 

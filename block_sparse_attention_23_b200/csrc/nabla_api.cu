@@ -16,11 +16,11 @@
 #include "sm100_primitives.cuh"
 
 namespace nabla {
-cudaError_t launch_pool(const void* q, const void* k, float* qbar, float* kbar, int64_t nblocks,
-                        int d, cudaStream_t st);
-cudaError_t launch_logits(const float* qbar, const float* kbar, float* L, int BH, int nb, int d,
-                          cudaStream_t st);
-cudaError_t launch_select(const float* L, int64_t nrows, int nb, float thr, int use_sta, int wt,
+cudaError_t launch_pool(const void* q, const void* k, double* qbar, double* kbar,
+                        int64_t nblocks, int d, cudaStream_t st);
+cudaError_t launch_logits(const double* qbar, const double* kbar, double* L, int BH, int nb,
+                          int d, cudaStream_t st);
+cudaError_t launch_select(const double* L, int64_t nrows, int nb, float thr, int use_sta, int wt,
                           int wh, int ww, int Tt, int Th, int Tw, uint32_t* bits, int32_t* counts,
                           uint8_t* mask_u8, cudaStream_t st);
 cudaError_t launch_mask_bits(const uint8_t* mask, int64_t nrows, int nb, uint32_t* bits,
@@ -87,9 +87,9 @@ BuildLayout build_layout(const nabla_shape* s) {
   const size_t nb = s->S / 64, BH = static_cast<size_t>(s->B) * s->H, nw = (nb + 31) / 32;
   BuildLayout l;
   size_t off = kHeaderBytes;
-  l.qbar = off; off = align256(off + BH * nb * s->d * 4);
-  l.kbar = off; off = align256(off + BH * nb * s->d * 4);
-  l.logits = off; off = align256(off + BH * nb * nb * 4);
+  l.qbar = off; off = align256(off + BH * nb * s->d * 8);
+  l.kbar = off; off = align256(off + BH * nb * s->d * 8);
+  l.logits = off; off = align256(off + BH * nb * nb * 8);
   l.bits = off; off = align256(off + BH * nb * nw * 4);
   l.counts = off; off = align256(off + BH * nb * 4);
   l.total = off;
@@ -244,9 +244,9 @@ nabla_status nabla_build_mask(const nabla_shape* shape, const nabla_mask_params*
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const BuildLayout lay = build_layout(shape);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  float* qbar = reinterpret_cast<float*>(ws + lay.qbar);
-  float* kbar = reinterpret_cast<float*>(ws + lay.kbar);
-  float* L = reinterpret_cast<float*>(ws + lay.logits);
+  double* qbar = reinterpret_cast<double*>(ws + lay.qbar);
+  double* kbar = reinterpret_cast<double*>(ws + lay.kbar);
+  double* L = reinterpret_cast<double*>(ws + lay.logits);
   uint32_t* bits = reinterpret_cast<uint32_t*>(ws + lay.bits);
   int32_t* counts = reinterpret_cast<int32_t*>(ws + lay.counts);
   const int nb = shape->S / 64, BH = shape->B * shape->H;
