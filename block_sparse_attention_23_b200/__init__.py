@@ -30,8 +30,7 @@ STATUS_NAMES = {0: "NABLA_OK", 1: "NABLA_ERR_INVALID_ARG", 2: "NABLA_ERR_UNSUPPO
 OP_BUILD_MASK, OP_FWD, OP_FWD_WITH_MASK = 0, 1, 2
 EXPORTED = ["nabla_workspace_size", "nabla_workspace_init", "nabla_query_status",
             "nabla_build_mask", "bsa_fwd", "bsa_fwd_with_mask", "nabla_last_error",
-            "nabla_version", "nabla_set_wait_limit_ns", "nabla_set_pv_variant",
-            "nabla_selftest_mma"]
+            "nabla_version", "nabla_set_wait_limit_ns", "nabla_selftest_mma"]
 
 
 class NablaError(RuntimeError):
@@ -91,8 +90,6 @@ def lib() -> ctypes.CDLL:
             L.nabla_version.argtypes = []
             L.nabla_set_wait_limit_ns.restype = None
             L.nabla_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
-            L.nabla_set_pv_variant.restype = None
-            L.nabla_set_pv_variant.argtypes = [i32]
             L.nabla_selftest_mma.restype = i32
             L.nabla_selftest_mma.argtypes = [i32, vp, vp, vp, vp, vp]
             _lib = L
@@ -242,10 +239,6 @@ def bsa_fwd_with_mask(q, k, v, mask_u8, scale: Optional[float] = None,
 
 def set_wait_limit_ns(ns: int) -> None:
     lib().nabla_set_wait_limit_ns(int(ns))
-
-
-def set_pv_variant(variant: int) -> None:
-    lib().nabla_set_pv_variant(int(variant))
 
 
 def selftest_mma(variant: int, a, b, workspace: Optional[Workspace] = None, stream=None):

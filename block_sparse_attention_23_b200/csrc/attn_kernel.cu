@@ -12,26 +12,36 @@
 //   One CTA per (b, h, pair of query blocks): 128 query rows = query blocks
 //   2p and 2p+1.  The key blocks visited are the union of the two CSR rows;
 //   each union entry carries a 2-bit membership flag, and a query row whose
-//   block did not list the key block treats it as masked (probability 0).
-//   Key tiles are 128 keys = two union entries (the second may be a repeat
-//   that both rows mask).  Every 64-key block is one contiguous slab of the
-//   [B,H,S,d] tensor, so each is a plain 2D TMA box at row (bh*S + 64*j).
+//   block did not list the key block treats it as masked (probability 0, no
+//   exponentials evaluated).  Key tiles are 128 keys = two union entries (the
+//   second may be a repeat that both rows mask).  Every 64-key block is one
+//   contiguous slab of the [B,H,S,d] tensor, so each is a plain 2D TMA box at
+//   row (bh*S + 64*j).
 //
-// Roles (256 threads)
-//   warps 0-3  softmax: thread i owns query row i (= tensor-memory lane i):
-//              tcgen05.ld S, online max/exp2/sum, P as bf16, O rescale in
-//              tensor memory, epilogue (O / l, LSE).
-//   warp 4     TMA producer: Q once, then K and V tiles into 2-stage rings.
-//   warp 5     tensor-memory allocation and the single MMA-issuing thread:
-//              S_t = Q K_t^T into one of two S buffers, then O += P_t V_t.
-//   warps 6-7  help build the union list, then wait.
+// Roles (320 threads)
+//   warps 0-7  softmax.  Warp w serves tensor-memory lanes 32*(w%4).. (query
+//              rows) and key half w/4 of each tile, i.e. one 64-key block:
+//              tcgen05.ld of its S half, row max exchanged with the partner
+//              thread through shared memory, exp2, P (bf16) into tensor
+//              memory, O rescale of its half of the d columns, epilogue.
+//   warp 8     TMA producer (and the union-list compaction at set-up).
+//   warp 9     tensor-memory allocation and the single MMA-issuing thread:
+//              S_t = Q K_t^T into one of two S buffers, then O += P_t V_t with
+//              P read from tensor memory.
+//
+// Online softmax with a lazy maximum: the running max m used for the
+// exponentials is raised (and O, l rescaled by 2^(m_old - m_new)) only when a
+// tile's max exceeds it by more than 2^8; otherwise p <= 256 and the final
+// O / l and LSE = ln2 * (m + log2 l) are unchanged in exact arithmetic.
 //
 // Tensor memory (512 columns): S0 [0,128), S1 [128,256), O [256,256+d),
-// P (tensor-memory variant) [384,448).
+// P0 [384,448), P1 [448,512) (P as packed bf16 pairs).
 //
 // Every mbarrier wait is time-bounded; a wait that runs out records
 // kStatusTimeout, raises a CTA-wide abort flag, and the CTA drains its own TMA
 // loads and MMAs (bounded again) before freeing tensor memory and returning.
+// The softmax warps agree on every abort through bar.red.and, so their named
+// barriers never see a partial arrival.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -44,27 +54,28 @@ namespace nabla {
 constexpr int kBM = 128;        // query rows per CTA (two 64-token blocks)
 constexpr int kBN = 128;        // keys per tile (two 64-token blocks)
 constexpr int kStages = 2;      // K and V ring depth
-constexpr int kThreads = 256;
+constexpr int kSoftmaxThreads = 256;
+constexpr int kThreads = kSoftmaxThreads + 64;
+constexpr int kProducerWarp = 8, kMmaWarp = 9;
 constexpr int kMaxNb = 4096;    // blocks per head supported
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256, kColP = 384;
+constexpr float kRescaleThreshold = 8.0f;            // log2 units
 constexpr uint64_t kDrainLimitNs = 1000000000ull;   // 1 s for draining in-flight work
-
-enum PvVariant : int { kPvSmemN64 = 1, kPvSmemNd = 2, kPvTmemNd = 3 };
+constexpr int kSoftmaxBarrier = 1;                   // named barrier id of warps 0-7
 
 template <int D>
 struct AttnSmem {
   static constexpr int kDH = D / 64;                       // 64-column halves of d
   static constexpr uint32_t kQBytes = kBM * D * 2;
   static constexpr uint32_t kKVBytes = kBN * D * 2;        // one K or V stage
-  static constexpr uint32_t kPBytes = kBM * kBN * 2;
   static constexpr uint32_t kOffQ = 0;
   static constexpr uint32_t kOffK = kOffQ + kQBytes;
   static constexpr uint32_t kOffV = kOffK + kStages * kKVBytes;
-  static constexpr uint32_t kOffP = kOffV + kStages * kKVBytes;
-  static constexpr uint32_t kOffBar = kOffP + kPBytes;     // 32 mbarriers
+  static constexpr uint32_t kOffBar = kOffV + kStages * kKVBytes;   // 32 mbarriers
   static constexpr uint32_t kOffMisc = kOffBar + 256;      // tmem base, abort, n_u
-  static constexpr uint32_t kOffBitmap = kOffMisc + 64;    // 2 x kMaxNb/32 words
+  static constexpr uint32_t kOffRed = kOffMisc + 64;       // [3 slot][2 half][128] floats
+  static constexpr uint32_t kOffBitmap = kOffRed + 3 * 2 * kBM * 4;   // 2 x kMaxNb/32 words
   static constexpr uint32_t kOffList = kOffBitmap + 2 * (kMaxNb / 32) * 4;
   static constexpr uint32_t kBytes = kOffList + kMaxNb * 4;
   static constexpr uint32_t kAlloc = kBytes + 1024;        // slack for 1024-byte alignment
@@ -80,8 +91,8 @@ enum : int {
   kBarSFull = kBarVEmpty + kStages,   // + buffer (2)
   kBarSEmpty = kBarSFull + 2,
   kBarPFull = kBarSEmpty + 2,
-  kBarOFull = kBarPFull + 1,
-  kBarDrain = kBarOFull + 1,
+  kBarOFull = kBarPFull + 1,          // + (t & 1): PV_t done
+  kBarDrain = kBarOFull + 2,
   kNumBars = kBarDrain + 1
 };
 
@@ -108,7 +119,21 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, uint64_
   return __all_sync(0xffffffffu, mbar_wait(bar, parity, limit_ns, abort));
 }
 
-template <int D, int PV>
+// Named barrier over `n` threads that also ANDs a predicate across them.
+__device__ __forceinline__ bool bar_red_and(int id, int n, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 q, %1, 0;\n\t"
+      "bar.red.and.pred p, %2, %3, q;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(pred)), "r"(id), "r"(n)
+      : "memory");
+  return r != 0;
+}
+
+template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     bsa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const AttnParams prm) {
@@ -121,12 +146,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t sQ = base + L::kOffQ;
   const uint32_t sK = base + L::kOffK;
   const uint32_t sV = base + L::kOffV;
-  const uint32_t sP = base + L::kOffP;
   const uint32_t bar0 = base + L::kOffBar;
   uint32_t* misc = reinterpret_cast<uint32_t*>(gbase + L::kOffMisc);
   volatile uint32_t* tmem_holder = misc;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
   volatile int* n_union_s = reinterpret_cast<volatile int*>(misc + 2);
+  float* red = reinterpret_cast<float*>(gbase + L::kOffRed);
   uint32_t* bm1 = reinterpret_cast<uint32_t*>(gbase + L::kOffBitmap);
   uint32_t* bm2 = bm1 + kMaxNb / 32;
   int32_t* ulist = reinterpret_cast<int32_t*>(gbase + L::kOffList);
@@ -151,19 +176,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(bar(kBarSFull + b), 1);
-      mbar_init(bar(kBarSEmpty + b), 128);
+      mbar_init(bar(kBarSEmpty + b), kSoftmaxThreads);
+      mbar_init(bar(kBarOFull + b), 1);
     }
-    mbar_init(bar(kBarPFull), 128);
-    mbar_init(bar(kBarOFull), 1);
+    mbar_init(bar(kBarPFull), kSoftmaxThreads);
     mbar_init(bar(kBarDrain), 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tmem_alloc(smem_addr(misc), kTmemCols);
     tmem_relinquish();
   }
-  if (warp == 4 && lane == 0) {
+  if (warp == kProducerWarp && lane == 0) {
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
@@ -189,7 +214,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
   __syncthreads();
-  if (warp == 6) {   // compact the union in ascending block order
+  if (warp == kProducerWarp) {   // compact the union in ascending block order
     int run = 0;
     for (int w0 = 0; w0 < nw; w0 += 32) {
       const int w = w0 + lane;
@@ -221,7 +246,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int n_t = (n_u + 1) >> 1;
   const uint64_t lim = prm.wait_limit_ns;
 
-  if (warp == 4) {
+  if (warp == kProducerWarp) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0 && n_t > 0) {
       const int64_t row0 = static_cast<int64_t>(bh) * prm.S;
@@ -265,11 +290,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (armed_v[s]) mbar_wait(bar(kBarVFull + s), (armed_v[s] - 1) & 1, kDrainLimitNs, nullptr);
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0 && n_t > 0) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(kBM, kBN, false);
-      constexpr uint32_t idesc_pv = idesc_bf16_f32(kBM, PV == kPvSmemN64 ? 64 : D, true);
+      constexpr uint32_t idesc_pv = idesc_bf16_f32(kBM, D, true);
       bool ok = mbar_wait(bar(kBarQFull), 0, lim, abort_flag);
       tc_fence_after();
       auto issue_s = [&](int u) -> bool {
@@ -297,152 +322,143 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!mbar_wait(bar(kBarVFull + s), (t / kStages) & 1, lim, abort_flag)) { ok = false; break; }
         tc_fence_after();
         const uint32_t vt = sV + s * L::kKVBytes;
+        const uint32_t pcol = kColP + (t & 1) * 64;
 #pragma unroll
         for (int kk = 0; kk < kBN / 16; ++kk) {
-          const uint32_t acc = (t > 0 || kk > 0) ? 1u : 0u;
-          const uint32_t vrow = vt + kk * 16 * 128;     // 16 keys further down the tile
-          if constexpr (PV == kPvTmemNd) {
-            tc_mma_ts(tmem + kColO, tmem + kColP + kk * 8, sdesc_sw128(vrow, kBN * 128, 1024),
-                      idesc_pv, acc);
-          } else {
-            const uint64_t adesc =
-                sdesc_sw128(sP + (kk >> 2) * (kBM * 128) + (kk & 3) * 32, 16, 1024);
-            if constexpr (PV == kPvSmemNd) {
-              tc_mma_ss(tmem + kColO, adesc, sdesc_sw128(vrow, kBN * 128, 1024), idesc_pv, acc);
-            } else {
-#pragma unroll
-              for (int h = 0; h < L::kDH; ++h)
-                tc_mma_ss(tmem + kColO + h * 64, adesc,
-                          sdesc_sw128(vrow + h * kBN * 128, 1024, 1024), idesc_pv, acc);
-            }
-          }
+          // 16 keys per step: P columns [pcol + 8kk, +8); V rows [16kk, +16) of the tile,
+          // the 64-column halves of d kBN*128 bytes apart (MN-major operand)
+          tc_mma_ts(tmem + kColO, tmem + pcol + kk * 8, sdesc_sw128(vt + kk * 16 * 128, kBN * 128, 1024),
+                    idesc_pv, (t > 0 || kk > 0) ? 1u : 0u);
         }
         tc_commit(bar(kBarVEmpty + s));
-        tc_commit(bar(kBarOFull));
+        tc_commit(bar(kBarOFull + (t & 1)));
       }
       if (!ok) record_abort(abort_flag, prm.status, kStatusTimeout);
       // drain: all MMAs this thread issued must finish before tensor memory is freed
       tc_commit(bar(kBarDrain));
       mbar_wait(bar(kBarDrain), 0, kDrainLimitNs, nullptr);
     }
-  } else if (warp < 4) {
-    // ------------------------------------------------------------ softmax
-    const int row = tid;                     // tensor-memory lane == query row
-    const int qh = row >> 6;                 // 0: block r1, 1: block r2
+  } else {
+    // ------------------------------------------------------------ softmax (warps 0-7)
+    const int quarter = warp & 3;
+    const int half = warp >> 2;                // key block of the tile this warp handles
+    const int row = quarter * 32 + lane;       // query row == tensor-memory lane
+    const int qh = row >> 6;                   // 0: block r1, 1: block r2
     const bool row_valid = qh == 0 || has2;
     const int bitsel = 1 << (16 + qh);
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const float sl2 = prm.scale_log2;
-    float m = -INFINITY, l = 0.f;
+    float m = -INFINITY;        // running (lazy) max, log2 units, same in both halves
+    float l = 0.f;              // this half's share of the row sum
     bool ok = true;
     for (int t = 0; t < n_t; ++t) {
       const int b = t & 1;
-      if (!warp_wait(bar(kBarSFull + b), (t >> 1) & 1, lim, abort_flag)) { ok = false; break; }
-      tc_fence_after();
-      const int e0 = ulist[2 * t];
-      const int e1 = (2 * t + 1 < n_u) ? ulist[2 * t + 1] : 0;
-      const bool v0 = (e0 & bitsel) != 0, v1 = (e1 & bitsel) != 0;   // uniform per warp
-      uint32_t sreg[4][32];
-      const uint32_t sbase = tmem + lane_off + (b ? kColS1 : kColS0);
-      if (v0) { tmem_ld32(sbase + 0, sreg[0]); tmem_ld32(sbase + 32, sreg[1]); }
-      if (v1) { tmem_ld32(sbase + 64, sreg[2]); tmem_ld32(sbase + 96, sreg[3]); }
-      tmem_ld_wait();
-      tc_fence_before();
-      mbar_arrive(bar(kBarSEmpty + b));
-      float mx = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        if ((c < 2 && v0) || (c >= 2 && v1)) {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) mx = fmaxf(mx, __uint_as_float(sreg[c][i]));
-        }
-      }
-      const float m_new = fmaxf(m, mx * sl2);
-      if (t > 0) {
-        if (!warp_wait(bar(kBarOFull), (t - 1) & 1, lim, abort_flag)) { ok = false; break; }
+      const int e = (2 * t + half < n_u) ? ulist[2 * t + half] : 0;
+      const bool valid = (e & bitsel) != 0;    // uniform per warp
+      uint32_t sreg[2][32];
+      float mloc = -INFINITY;
+      bool got = warp_wait(bar(kBarSFull + b), (t >> 1) & 1, lim, abort_flag);
+      if (got) {
         tc_fence_after();
-      }
-      const bool need = (m > -INFINITY) && (m_new > m);
-      if (__any_sync(0xffffffffu, need)) {
-        const float alpha = need ? fast_exp2(m - m_new) : 1.f;
-        l *= alpha;
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t o[32];
-          const uint32_t oa = tmem + lane_off + kColO + c * 32;
-          tmem_ld32(oa, o);
+        if (valid) {
+          const uint32_t sbase = tmem + lane_off + (b ? kColS1 : kColS0) + half * 64;
+          tmem_ld32(sbase, sreg[0]);
+          tmem_ld32(sbase + 32, sreg[1]);
           tmem_ld_wait();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-          tmem_st32(oa, o);
         }
-        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(bar(kBarSEmpty + b));
+        if (valid) {
+          float mx[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            mx[i] = fmaxf(__uint_as_float(sreg[0][i]), __uint_as_float(sreg[1][i]));
+#pragma unroll
+          for (int i = 8; i < 32; ++i)
+            mx[i & 7] = fmaxf(mx[i & 7], fmaxf(__uint_as_float(sreg[0][i]), __uint_as_float(sreg[1][i])));
+          mloc = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                       fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * sl2;
+        }
       }
-      m = m_new;
-      const float mneg = (m == -INFINITY) ? 0.f : -m;   // all-masked so far: p stays 0
-      float rowsum = 0.f;
-      uint32_t pk[4][16];
+      float* red_t = red + (t & 1) * (2 * kBM);
+      red_t[half * kBM + row] = mloc;
+      ok = bar_red_and(kSoftmaxBarrier, kSoftmaxThreads, ok && got);
+      if (!ok) break;
+      const float m_tile = fmaxf(mloc, red_t[(half ^ 1) * kBM + row]);
+      const float m_new = fmaxf(m, m_tile);
+      // lazy rescale: only when the max grows by more than 2^kRescaleThreshold
+      const bool need = (m > -INFINITY) && (m_new > m + kRescaleThreshold);
+      if (__any_sync(0xffffffffu, need)) {
+        if (t > 0 && !warp_wait(bar(kBarOFull + ((t - 1) & 1)), ((t - 1) >> 1) & 1, lim, abort_flag)) {
+          ok = false;
+        } else {
+          tc_fence_after();
+          const float alpha = need ? fast_exp2(m - m_new) : 1.f;
+          l *= alpha;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        const bool valid = (c < 2) ? v0 : v1;
+          for (int c = 0; c < D / 64; ++c) {
+            uint32_t o[32];
+            const uint32_t oa = tmem + lane_off + kColO + half * (D / 2) + c * 32;
+            tmem_ld32(oa, o);
+            tmem_ld_wait();
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          float p0 = 0.f, p1 = 0.f;
-          if (valid) {
-            p0 = fast_exp2(fmaf(__uint_as_float(sreg[c][2 * i]), sl2, mneg));
-            p1 = fast_exp2(fmaf(__uint_as_float(sreg[c][2 * i + 1]), sl2, mneg));
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            tmem_st32(oa, o);
           }
-          rowsum += p0 + p1;
-          pk[c][i] = pack_bf16x2(p0, p1);
+          tmem_st_wait();
         }
       }
-      if constexpr (PV == kPvTmemNd) {
-        uint32_t lo[32], hi[32];
+      if (m == -INFINITY || need) m = m_new;
+      // p = 2^(s*scale*log2e - m); masked halves and not-yet-valid rows give 0
+      uint32_t pk[32];
+      float rs[4] = {0.f, 0.f, 0.f, 0.f};
+      if (valid && m > -INFINITY) {
+        const float mneg = -m;
 #pragma unroll
-        for (int i = 0; i < 16; ++i) { lo[i] = pk[0][i]; lo[16 + i] = pk[1][i]; hi[i] = pk[2][i]; hi[16 + i] = pk[3][i]; }
-        tmem_st32(tmem + lane_off + kColP, lo);
-        tmem_st32(tmem + lane_off + kColP + 32, hi);
-        tmem_st_wait();
+        for (int c = 0; c < 2; ++c)
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float p0 = fast_exp2(fmaf(__uint_as_float(sreg[c][2 * i]), sl2, mneg));
+            const float p1 = fast_exp2(fmaf(__uint_as_float(sreg[c][2 * i + 1]), sl2, mneg));
+            rs[i & 3] += p0 + p1;
+            pk[c * 16 + i] = pack_bf16x2(p0, p1);
+          }
       } else {
-        // P row into the 128-byte-swizzled K-major layout: half kh holds keys
-        // [64kh, 64kh+64); 16-byte chunk j of the row sits at chunk j ^ (row & 7).
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const uint32_t rowbase = sP + (c >> 1) * (kBM * 128) + row * 128;
-#pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4) {
-            const int chunk = (c & 1) * 4 + q4;
-            const uint32_t addr = rowbase + ((chunk ^ (row & 7)) << 4);
-            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr),
-                         "r"(pk[c][4 * q4]), "r"(pk[c][4 * q4 + 1]), "r"(pk[c][4 * q4 + 2]),
-                         "r"(pk[c][4 * q4 + 3])
-                         : "memory");
-          }
-        }
-        fence_proxy_async_smem();
+        for (int i = 0; i < 32; ++i) pk[i] = 0u;
       }
-      tc_fence_before();
-      mbar_arrive(bar(kBarPFull));
-      l += rowsum;
+      l += (rs[0] + rs[1]) + (rs[2] + rs[3]);
+      // P_t goes to P[t&1]; PV_{t-2} (which read that buffer) must be complete
+      if (ok && t >= 2 && !warp_wait(bar(kBarOFull + (t & 1)), ((t - 2) >> 1) & 1, lim, abort_flag))
+        ok = false;
+      if (ok) {
+        tmem_st32(tmem + lane_off + kColP + (t & 1) * 64 + half * 32, pk);
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(bar(kBarPFull));
+      }
     }
-    if (!ok) record_abort(abort_flag, prm.status, kStatusTimeout);
     // ------------------------------------------------------------ epilogue
     bool have_o = false;
     if (ok && n_t > 0) {
-      have_o = warp_wait(bar(kBarOFull), (n_t - 1) & 1, lim, abort_flag);
-      if (!have_o) record_abort(abort_flag, prm.status, kStatusTimeout);
+      have_o = warp_wait(bar(kBarOFull + ((n_t - 1) & 1)), ((n_t - 1) >> 1) & 1, lim, abort_flag);
       tc_fence_after();
     }
-    const bool write = row_valid && (ok && (n_t == 0 || have_o));
+    float* red_l = red + 4 * kBM;              // slot 2: row-sum exchange (slots 0/1: maxima)
+    red_l[half * kBM + row] = l;
+    const bool all_ok = bar_red_and(kSoftmaxBarrier, kSoftmaxThreads, ok && (n_t == 0 || have_o));
+    if (!all_ok) record_abort(abort_flag, prm.status, kStatusTimeout);
+    const float lt = l + red_l[(half ^ 1) * kBM + row];
+    const bool write = row_valid && all_ok;
     const int qrow = (qh ? r2 : r1) * 64 + (row & 63);
     const int64_t grow = static_cast<int64_t>(bh) * prm.S + qrow;
-    const float inv_l = l > 0.f ? 1.f / l : 0.f;
-    __nv_bfloat16* orow = prm.o + grow * D;
+    const float inv_l = lt > 0.f ? 1.f / lt : 0.f;
+    __nv_bfloat16* orow = prm.o + grow * D + half * (D / 2);
 #pragma unroll
-    for (int c = 0; c < D / 32; ++c) {
+    for (int c = 0; c < D / 64; ++c) {
       uint32_t o[32];
-      if (have_o) {
-        tmem_ld32(tmem + lane_off + kColO + c * 32, o);
+      if (have_o && all_ok) {
+        tmem_ld32(tmem + lane_off + kColO + half * (D / 2) + c * 32, o);
         tmem_ld_wait();
       } else {
 #pragma unroll
@@ -458,13 +474,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
       }
     }
-    if (write && prm.lse != nullptr)
-      prm.lse[grow] = l > 0.f ? (m + __log2f(l)) * 0.69314718055994530942f : -INFINITY;
+    if (write && half == 0 && prm.lse != nullptr)
+      prm.lse[grow] = lt > 0.f ? (m + __log2f(lt)) * 0.69314718055994530942f : -INFINITY;
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
@@ -572,21 +588,21 @@ __global__ void __launch_bounds__(160, 1)
 
 // ---------------------------------------------------------------- launchers
 
-template <int D, int PV>
+template <int D>
 static cudaError_t launch_fwd_t(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
                                 const AttnParams& prm, int64_t nitems, cudaStream_t st) {
   constexpr uint32_t smem = AttnSmem<D>::kAlloc;
-  cudaError_t e = cudaFuncSetAttribute(bsa_fwd_kernel<D, PV>,
+  cudaError_t e = cudaFuncSetAttribute(bsa_fwd_kernel<D>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  bsa_fwd_kernel<D, PV><<<static_cast<unsigned>(nitems), kThreads, smem, st>>>(q, k, v, prm);
+  bsa_fwd_kernel<D><<<static_cast<unsigned>(nitems), kThreads, smem, st>>>(q, k, v, prm);
   return cudaGetLastError();
 }
 
 cudaError_t launch_bsa_fwd(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
                            const int32_t* row_ptr, const int32_t* col_idx, void* o, float* lse,
                            int* status, int BH, int H, int S, int d, float scale,
-                           uint64_t wait_limit_ns, int pv_variant, cudaStream_t st) {
+                           uint64_t wait_limit_ns, cudaStream_t st) {
   AttnParams prm;
   prm.row_ptr = row_ptr;
   prm.col_idx = col_idx;
@@ -601,18 +617,8 @@ cudaError_t launch_bsa_fwd(const CUtensorMap& q, const CUtensorMap& k, const CUt
   prm.wait_limit_ns = wait_limit_ns;
   const int64_t nitems = static_cast<int64_t>(BH) * prm.npairs;
   if (nitems == 0) return cudaSuccess;
-  if (d == 128) {
-    switch (pv_variant) {
-      case kPvSmemN64: return launch_fwd_t<128, kPvSmemN64>(q, k, v, prm, nitems, st);
-      case kPvSmemNd: return launch_fwd_t<128, kPvSmemNd>(q, k, v, prm, nitems, st);
-      default: return launch_fwd_t<128, kPvTmemNd>(q, k, v, prm, nitems, st);
-    }
-  }
-  switch (pv_variant) {
-    case kPvSmemN64: return launch_fwd_t<64, kPvSmemN64>(q, k, v, prm, nitems, st);
-    case kPvSmemNd: return launch_fwd_t<64, kPvSmemNd>(q, k, v, prm, nitems, st);
-    default: return launch_fwd_t<64, kPvTmemNd>(q, k, v, prm, nitems, st);
-  }
+  if (d == 128) return launch_fwd_t<128>(q, k, v, prm, nitems, st);
+  return launch_fwd_t<64>(q, k, v, prm, nitems, st);
 }
 
 cudaError_t launch_mma_selftest(const CUtensorMap& a, const CUtensorMap& b, const void* a_glob,

@@ -31,7 +31,7 @@ cudaError_t launch_scan_fill(const uint32_t* bits, const int32_t* counts, int64_
 cudaError_t launch_bsa_fwd(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
                            const int32_t* row_ptr, const int32_t* col_idx, void* o, float* lse,
                            int* status, int BH, int H, int S, int d, float scale,
-                           uint64_t wait_limit_ns, int pv_variant, cudaStream_t st);
+                           uint64_t wait_limit_ns, cudaStream_t st);
 cudaError_t launch_mma_selftest(const CUtensorMap& a, const CUtensorMap& b, const void* a_glob,
                                 float* c, int variant, int* status, uint64_t lim,
                                 cudaStream_t st);
@@ -45,8 +45,6 @@ constexpr int kMaxNbSupported = 4096;
 
 thread_local std::string g_last_error;
 std::atomic<uint64_t> g_wait_limit_ns{kDefaultWaitLimitNs};
-std::atomic<int> g_pv_variant{0};
-constexpr int kDefaultPvVariant = 1;
 
 nabla_status fail(nabla_status s, const std::string& msg) {
   g_last_error = msg;
@@ -150,11 +148,6 @@ nabla_status make_map(CUtensorMap* map, const void* ptr, uint64_t rows, uint64_t
 
 int* status_ptr(void* ws) { return static_cast<int*>(ws); }
 
-int pv_variant() {
-  const int v = g_pv_variant.load();
-  return v == 0 ? kDefaultPvVariant : v;
-}
-
 nabla_status run_fwd(const nabla_shape* shape, const void* q, const void* k, const void* v,
                      const int32_t* row_ptr, const int32_t* col_idx, float scale, void* o,
                      float* lse, void* workspace, cudaStream_t st) {
@@ -167,8 +160,7 @@ nabla_status run_fwd(const nabla_shape* shape, const void* q, const void* k, con
   if (!(scale > 0.f)) scale = 1.0f / std::sqrt(static_cast<float>(shape->d));
   cudaError_t e = nabla::launch_bsa_fwd(mq, mk, mv, row_ptr, col_idx, o, lse,
                                         status_ptr(workspace), shape->B * shape->H, shape->H,
-                                        shape->S, shape->d, scale, g_wait_limit_ns.load(),
-                                        pv_variant(), st);
+                                        shape->S, shape->d, scale, g_wait_limit_ns.load(), st);
   if (e != cudaSuccess) return cuda_fail(e, "bsa_fwd launch");
   return NABLA_OK;
 }
@@ -183,10 +175,6 @@ const char* nabla_last_error(void) { return g_last_error.c_str(); }
 
 void nabla_set_wait_limit_ns(uint64_t ns) {
   g_wait_limit_ns.store(ns == 0 ? kDefaultWaitLimitNs : ns);
-}
-
-void nabla_set_pv_variant(int variant) {
-  g_pv_variant.store((variant >= 1 && variant <= 3) ? variant : 0);
 }
 
 size_t nabla_workspace_size(const nabla_shape* shape, int op) {

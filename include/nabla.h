@@ -161,10 +161,6 @@ NABLA_API int nabla_version(void);
  * memory, record NABLA_ERR_TIMEOUT and return.  Tests set a tiny limit to
  * check that path without hanging anything.
  *
- * nabla_set_pv_variant: which tcgen05 form the P.V product uses
- * (0 = default; 1 = P in shared memory, two N=64 MMAs; 2 = P in shared
- * memory, one N=d MMA; 3 = P in tensor memory, one N=d MMA).
- *
  * nabla_selftest_mma: one 128 x N x 128 bf16 product through the same
  * tcgen05/TMA building blocks the attention kernel uses, for layout checks.
  *   variant 0: C[m][n] = sum_k A[m][k] B[n][k]   (both K-major, N = 128)
@@ -174,7 +170,6 @@ NABLA_API int nabla_version(void);
  *   a, b: device bf16 [128][128] row-major; c: device fp32 [128][128].
  */
 NABLA_API void nabla_set_wait_limit_ns(uint64_t ns);
-NABLA_API void nabla_set_pv_variant(int variant);
 NABLA_API nabla_status nabla_selftest_mma(int variant, const void* a, const void* b, float* c,
                                 void* workspace, nabla_stream_t stream);
 

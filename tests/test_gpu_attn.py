@@ -15,13 +15,6 @@ def nl():
     return nl
 
 
-@pytest.fixture(autouse=True)
-def _default_variant(nl):
-    nl.set_pv_variant(0)
-    yield
-    nl.set_pv_variant(0)
-
-
 def _gather(o, lse, rows, S):
     o = o.float().cpu().numpy().reshape(-1, o.shape[-1])
     lse = lse.cpu().numpy().reshape(-1)
@@ -50,18 +43,6 @@ def test_attention_parity_all_rows(nl, oracle_mod, synth_mod, name):
     go, gl = _gather(o, lse, rows, w.S)
     mx, mean = compare_attention(go, gl, ro, rl)
     print(f"{name}: max-abs {mx:.3g} mean-abs {mean:.3g}")
-
-
-@pytest.mark.parametrize("variant", [1, 2, 3])
-def test_attention_pv_variants(nl, oracle_mod, synth_mod, variant):
-    nl.set_pv_variant(variant)
-    w = synth_mod.WORKLOADS["small"]
-    q, k, v = synth_mod.make_qkv(w)
-    o, lse, mask = _nabla_layer(nl, w, q, k, v)
-    rows = sample_rows(w.B, w.H, w.S, 6, 16, seed=variant)
-    ro, rl = oracle_mod.masked_attention(q, k, v, mask, rows)
-    go, gl = _gather(o, lse, rows, w.S)
-    compare_attention(go, gl, ro, rl)
 
 
 @pytest.mark.parametrize("name", ["hunyuan720p", "wan720p"])
