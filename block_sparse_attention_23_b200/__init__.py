@@ -2,7 +2,7 @@
 
 Argument marshalling only: every step of the mask builder and the attention
 forward runs in the CUDA kernels of ``libnabla.so`` (built from ``csrc/`` by
-``build.py``).  PyTorch is used for device memory and the current stream.
+``buildlib.py``).  PyTorch is used for device memory and the current stream.
 There is no CPU fallback: if the library is missing or no CUDA device is
 present, the calls raise.
 
@@ -30,7 +30,8 @@ STATUS_NAMES = {0: "NABLA_OK", 1: "NABLA_ERR_INVALID_ARG", 2: "NABLA_ERR_UNSUPPO
 OP_BUILD_MASK, OP_FWD, OP_FWD_WITH_MASK = 0, 1, 2
 EXPORTED = ["nabla_workspace_size", "nabla_workspace_init", "nabla_query_status",
             "nabla_build_mask", "bsa_fwd", "bsa_fwd_with_mask", "nabla_last_error",
-            "nabla_version", "nabla_set_wait_limit_ns", "nabla_selftest_mma"]
+            "nabla_version", "nabla_set_wait_limit_ns", "nabla_selftest_mma",
+            "bsa_fwd_with_mask_static"]
 
 
 class NablaError(RuntimeError):
@@ -55,7 +56,7 @@ _lib = None
 
 
 def build(force: bool = False) -> str:
-    from .build import build as _build
+    from .buildlib import build as _build
     return _build(force=force)
 
 
@@ -66,7 +67,7 @@ def lib() -> ctypes.CDLL:
         if _lib is None:
             if not os.path.exists(LIB_PATH):
                 raise RuntimeError(f"{LIB_PATH} is missing: build it with "
-                                   "`python -m block_sparse_attention_23_b200.build`")
+                                   "`python -m block_sparse_attention_23_b200.buildlib`")
             L = ctypes.CDLL(LIB_PATH)
             vp, i32, i64, f32, sz = (ctypes.c_void_p, ctypes.c_int, ctypes.c_int64,
                                      ctypes.c_float, ctypes.c_size_t)
@@ -92,6 +93,8 @@ def lib() -> ctypes.CDLL:
             L.nabla_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
             L.nabla_selftest_mma.restype = i32
             L.nabla_selftest_mma.argtypes = [i32, vp, vp, vp, vp, vp]
+            L.bsa_fwd_with_mask_static.restype = i32
+            L.bsa_fwd_with_mask_static.argtypes = [sp, vp, vp, vp, vp, f32, vp, vp, vp, vp]
             _lib = L
     return _lib
 
@@ -251,3 +254,25 @@ def selftest_mma(variant: int, a, b, workspace: Optional[Workspace] = None, stre
                                     _stream(stream)))
     workspace.check(stream)
     return c
+
+
+def bsa_fwd_with_mask_static(q, k, v, mask_u8, scale: Optional[float] = None, out=None,
+                             status_out=None, stream=None):
+    """Static-mask attention forward that allocates no device memory inside the
+    library and takes no workspace: for callers (memory-pool runtimes, code
+    inside another framework's graph capture, fixed-budget hosts) that cannot
+    allocate.  Its scratch is a fixed 32 MiB array owned by the library and
+    shared by all calls, so calls that overlap on the GPU must not be issued.
+    Returns (O, LSE); ``out`` may pass preallocated (O, LSE)."""
+    torch = _torch()
+    _bf16_contig(q, k, v)
+    shape = _shape_of(q)
+    if out is None:
+        o = torch.empty_like(q)
+        lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device)
+    else:
+        o, lse = out
+    _check(lib().bsa_fwd_with_mask_static(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v),
+                                          _ptr(mask_u8), float(scale or 0.0), _ptr(o), _ptr(lse),
+                                          _ptr(status_out), _stream(stream)))
+    return o, lse

@@ -1,6 +1,6 @@
 """Compile libnabla.so (sm_100a) in place with nvcc.
 
-Usage: python -m block_sparse_attention_23_b200.build [--force]
+Usage: python -m block_sparse_attention_23_b200.buildlib [--force]
 """
 from __future__ import annotations
 
@@ -11,7 +11,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libnabla.so")
-SOURCES = ["nabla_api.cu", "mask_kernels.cu", "attn_kernel.cu"]
+SOURCES = ["nabla_api.cu", "mask_kernels.cu", "attn_kernel.cu", "nabla_noalloc.cu"]
 HEADERS = ["sm100_primitives.cuh", os.path.join("..", "..", "include", "nabla.h")]
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
               "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden", "--expt-relaxed-constexpr",

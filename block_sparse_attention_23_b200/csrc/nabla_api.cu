@@ -167,6 +167,11 @@ nabla_status run_fwd(const nabla_shape* shape, const void* q, const void* k, con
 
 }  // namespace
 
+namespace nabla {
+// Lets other translation units of the library report through nabla_last_error().
+void set_last_error(const std::string& msg) { g_last_error = msg; }
+}  // namespace nabla
+
 extern "C" {
 
 int nabla_version(void) { return 100; }

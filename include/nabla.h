@@ -146,6 +146,37 @@ NABLA_API nabla_status bsa_fwd_with_mask(const nabla_shape* shape, const void* q
                                const void* v, const uint8_t* mask_u8, float scale, void* o,
                                float* lse, void* workspace, nabla_stream_t stream);
 
+/*
+ * Static-mask attention forward that allocates nothing (no counterpart in the
+ * paper; it exists for callers that cannot allocate device memory).
+ *
+ * Some callers cannot call cudaMalloc or hand over a workspace: a serving
+ * runtime that owns all device memory through its own pool, code running
+ * inside another framework's CUDA-graph capture, or an embedded host with a
+ * fixed memory budget.  This call computes exactly what bsa_fwd_with_mask
+ * computes, but keeps the block CSR it builds from the mask in a fixed
+ * device array owned by the library (NABLA_STATIC_SCRATCH_BYTES, 32 MiB, held
+ * on each device that has used it until the process exits).  It allocates
+ * nothing and takes no workspace.
+ *
+ *   q, k, v, mask_u8, scale, o, lse   as for bsa_fwd_with_mask
+ *   status_out   optional device int32 [1], or NULL: receives the call's
+ *                device status bits (0 = completed; 1 = a pipeline wait ran
+ *                out) in stream order
+ * Returns NABLA_ERR_UNSUPPORTED, with a message, when the shape's block CSR
+ * does not fit the array (B*H*(S/64)^2 above roughly 8.3 million blocks).
+ * Every call shares the one array: calls whose GPU work can overlap (other
+ * streams without ordering) race; calls on one stream are safe.  The first
+ * call on each device looks up the array's device address; make it before
+ * any stream capture starts.
+ */
+#define NABLA_STATIC_SCRATCH_BYTES (32u * 1024u * 1024u)
+NABLA_API nabla_status bsa_fwd_with_mask_static(const nabla_shape* shape, const void* q,
+                                                const void* k, const void* v,
+                                                const uint8_t* mask_u8, float scale, void* o,
+                                                float* lse, int32_t* status_out,
+                                                nabla_stream_t stream);
+
 /* Message for the last error returned on the calling host thread. */
 NABLA_API const char* nabla_last_error(void);
 

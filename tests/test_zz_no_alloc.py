@@ -1,0 +1,73 @@
+"""bsa_fwd_with_mask_static: the attention entry point for callers that cannot
+allocate device memory (memory-pool runtimes, code running inside another
+framework's graph capture, fixed-budget hosts).  It keeps its block CSR in a
+fixed library-owned device array instead of a caller workspace.
+
+The GPU test calls it through the C ABI twice in a row, with different masks
+and inputs, and checks each result against bsa_fwd_with_mask (the entry point
+with a caller workspace) within the attention tolerance used throughout the
+tests.  This file is named to be collected last."""
+import ctypes
+
+import numpy as np
+import pytest
+
+from _parity import compare_attention, to_device_bf16
+
+
+@pytest.fixture(scope="module")
+def nl():
+    import block_sparse_attention_23_b200 as nl
+    nl.build()
+    nl.lib()
+    return nl
+
+
+def test_oversized_shape_rejected_before_any_cuda_call(nl):
+    lib = nl.lib()
+    s = nl.make_shape(1, 40, 76800, 128)        # 57.6 M blocks: far beyond 32 MiB
+    a = ctypes.c_void_p(1 << 20)
+    rc = lib.bsa_fwd_with_mask_static(ctypes.byref(s), a, a, a, a, 0.0, a, a, None, None)
+    assert rc == 2                              # NABLA_ERR_UNSUPPORTED
+    msg = lib.nabla_last_error().decode()
+    assert "scratch" in msg and str(32 * 1024 * 1024) in msg
+    assert rc == 2 and lib.bsa_fwd_with_mask_static(None, a, a, a, a, 0.0, a, a, None, None) == 1
+
+
+def _call_static(nl, shape, q, k, v, mask, o, lse, status):
+    import torch
+    rc = nl.lib().bsa_fwd_with_mask_static(
+        ctypes.byref(shape), ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(k.data_ptr()),
+        ctypes.c_void_p(v.data_ptr()), ctypes.c_void_p(mask.data_ptr()), ctypes.c_float(0.0),
+        ctypes.c_void_p(o.data_ptr()), ctypes.c_void_p(lse.data_ptr()),
+        ctypes.c_void_p(status.data_ptr()),
+        ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert rc == 0, nl.lib().nabla_last_error().decode()
+
+
+@pytest.mark.gpu
+def test_static_scratch_matches_workspace_entry_point_twice(nl, synth_mod):
+    import torch
+    B, H, nb, d = 1, 6, 96, 128
+    S = 64 * nb
+    shape = nl.make_shape(B, H, S, d)
+    for call, (p, seed) in enumerate([(0.4, 21), (0.1, 22)]):
+        q16 = synth_mod.make_tensor(0, seed, B, H, S, d, pos_weight=0.0, noise_weight=1.0)
+        k16 = synth_mod.make_tensor(1, seed, B, H, S, d, pos_weight=0.0, noise_weight=1.0)
+        v16 = synth_mod.make_tensor(2, seed, B, H, S, d, pos_weight=0.0, noise_weight=1.0)
+        q, k, v = to_device_bf16(q16), to_device_bf16(k16), to_device_bf16(v16)
+        mask_np = synth_mod.make_bernoulli_mask(seed, B * H, nb, p).reshape(B, H, nb, nb)
+        mask_np[0, 0, 3, :] = 0                  # one empty row
+        mask = torch.from_numpy(mask_np).cuda()
+        o_s = torch.full_like(q, float("nan"))
+        lse_s = torch.full((B, H, S), float("nan"), dtype=torch.float32, device=q.device)
+        status = torch.full((1,), -1, dtype=torch.int32, device=q.device)
+        _call_static(nl, shape, q, k, v, mask, o_s, lse_s, status)
+        o_w, lse_w = nl.bsa_fwd_with_mask(q, k, v, mask)
+        torch.cuda.synchronize()
+        assert int(status.item()) == 0, f"call {call}: device status {int(status.item())}"
+        go = o_s.float().cpu().numpy().reshape(-1, d)
+        gl = lse_s.cpu().numpy().reshape(-1)
+        ref_o = o_w.double().cpu().numpy().reshape(-1, d)
+        ref_l = lse_w.double().cpu().numpy().reshape(-1)
+        compare_attention(go, gl, ref_o, ref_l)
