@@ -18,30 +18,39 @@
 //   contiguous slab of the [B,H,S,d] tensor, so each is a plain 2D TMA box at
 //   row (bh*S + 64*j).
 //
-// Roles (320 threads)
+// Two independent softmax streams per row
+//   Key half h of every tile (the tile's h-th 64-key block) feeds its own
+//   accumulator O_h with its own running max m_h and sum l_h, so the two
+//   threads that serve a row never wait for each other inside the key loop.
+//   The epilogue merges them exactly:
+//     M = max(m_0, m_1),  f_h = 2^(m_h - M),
+//     O = (f_0 O_0 + f_1 O_1) / (f_0 l_0 + f_1 l_1),  LSE = ln2 (M + log2 L).
+//   Each stream keeps a lazy maximum: m_h is raised (and O_h, l_h rescaled by
+//   2^(m_old - m_new)) only when a tile exceeds it by more than 2^8, so p <= 256.
+//
+// Roles (352 threads)
 //   warps 0-7  softmax.  Warp w serves tensor-memory lanes 32*(w%4).. (query
-//              rows) and key half w/4 of each tile, i.e. one 64-key block:
-//              tcgen05.ld of its S half, row max exchanged with the partner
-//              thread through shared memory, exp2, P (bf16) into tensor
-//              memory, O rescale of its half of the d columns, epilogue.
-//   warp 8     TMA producer (and the union-list compaction at set-up).
+//              rows) and key half w/4: tcgen05.ld of its 64 S columns,
+//              max, exp2, P (bf16) written over the first 32 of those
+//              columns, lazy rescale of its O_h row, epilogue.
+//   warp 8     TMA producer of Q and K (and the union-list compaction).
+//   warp 10    TMA producer of V.
 //   warp 9     tensor-memory allocation and the single MMA-issuing thread:
-//              S_t = Q K_t^T into one of two S buffers, then O += P_t V_t with
-//              P read from tensor memory.
+//              S_t = Q K_t^T into buffer t&1, then O_h += P_t,h V_t,h for
+//              h = 0, 1 as soon as that half of P is in place (A operand read
+//              from tensor memory).
 //
-// Online softmax with a lazy maximum: the running max m used for the
-// exponentials is raised (and O, l rescaled by 2^(m_old - m_new)) only when a
-// tile's max exceeds it by more than 2^8; otherwise p <= 256 and the final
-// O / l and LSE = ln2 * (m + log2 l) are unchanged in exact arithmetic.
-//
-// Tensor memory (512 columns): S0 [0,128), S1 [128,256), O [256,256+d),
-// P0 [384,448), P1 [448,512) (P as packed bf16 pairs).
+// Tensor memory (512 columns): S/P buffers [0,128) and [128,256), O_0 at 256,
+// O_1 at 384 (d columns each).  Ordering of the in-place P: S_{t+2} reuses
+// buffer t&1 and is issued after PV_t by the same thread, and MMAs of one
+// thread execute in issue order; the completion of S_t (which the softmax
+// waits for) also implies the completion of PV_{t-2}, which read P_{t-2}.
 //
 // Every mbarrier wait is time-bounded; a wait that runs out records
 // kStatusTimeout, raises a CTA-wide abort flag, and the CTA drains its own TMA
 // loads and MMAs (bounded again) before freeing tensor memory and returning.
-// The softmax warps agree on every abort through bar.red.and, so their named
-// barriers never see a partial arrival.
+// The softmax warps share one named barrier, in the epilogue, and agree on
+// aborts there through bar.red.and.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -53,13 +62,14 @@ namespace nabla {
 
 constexpr int kBM = 128;        // query rows per CTA (two 64-token blocks)
 constexpr int kBN = 128;        // keys per tile (two 64-token blocks)
-constexpr int kStages = 2;      // K and V ring depth
+constexpr int kKStages = 3;     // K ring depth (K is needed one S-MMA after its slot frees)
+constexpr int kVStages = 2;     // V ring depth
 constexpr int kSoftmaxThreads = 256;
-constexpr int kThreads = kSoftmaxThreads + 64;
-constexpr int kProducerWarp = 8, kMmaWarp = 9;
+constexpr int kThreads = kSoftmaxThreads + 96;
+constexpr int kProducerWarp = 8, kMmaWarp = 9, kVProducerWarp = 10;
 constexpr int kMaxNb = 4096;    // blocks per head supported
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256, kColP = 384;
+constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO0 = 256, kColO1 = 384;
 constexpr float kRescaleThreshold = 8.0f;            // log2 units
 constexpr uint64_t kDrainLimitNs = 1000000000ull;   // 1 s for draining in-flight work
 constexpr int kSoftmaxBarrier = 1;                   // named barrier id of warps 0-7
@@ -71,11 +81,11 @@ struct AttnSmem {
   static constexpr uint32_t kKVBytes = kBN * D * 2;        // one K or V stage
   static constexpr uint32_t kOffQ = 0;
   static constexpr uint32_t kOffK = kOffQ + kQBytes;
-  static constexpr uint32_t kOffV = kOffK + kStages * kKVBytes;
-  static constexpr uint32_t kOffBar = kOffV + kStages * kKVBytes;   // 32 mbarriers
+  static constexpr uint32_t kOffV = kOffK + kKStages * kKVBytes;
+  static constexpr uint32_t kOffBar = kOffV + kVStages * kKVBytes;  // 32 mbarriers
   static constexpr uint32_t kOffMisc = kOffBar + 256;      // tmem base, abort, n_u
-  static constexpr uint32_t kOffRed = kOffMisc + 64;       // [3 slot][2 half][128] floats
-  static constexpr uint32_t kOffBitmap = kOffRed + 3 * 2 * kBM * 4;   // 2 x kMaxNb/32 words
+  static constexpr uint32_t kOffRed = kOffMisc + 64;       // [2 quantity][2 half][128] floats
+  static constexpr uint32_t kOffBitmap = kOffRed + 2 * 2 * kBM * 4;   // 2 x kMaxNb/32 words
   static constexpr uint32_t kOffList = kOffBitmap + 2 * (kMaxNb / 32) * 4;
   static constexpr uint32_t kBytes = kOffList + kMaxNb * 4;
   static constexpr uint32_t kAlloc = kBytes + 1024;        // slack for 1024-byte alignment
@@ -84,15 +94,14 @@ struct AttnSmem {
 // Barrier slots inside the barrier area.
 enum : int {
   kBarQFull = 0,
-  kBarKFull = 1,                   // + stage
-  kBarKEmpty = kBarKFull + kStages,
-  kBarVFull = kBarKEmpty + kStages,
-  kBarVEmpty = kBarVFull + kStages,
-  kBarSFull = kBarVEmpty + kStages,   // + buffer (2)
-  kBarSEmpty = kBarSFull + 2,
-  kBarPFull = kBarSEmpty + 2,
-  kBarOFull = kBarPFull + 1,          // + (t & 1): PV_t done
-  kBarDrain = kBarOFull + 2,
+  kBarKFull = 1,                      // + stage
+  kBarKEmpty = kBarKFull + kKStages,
+  kBarVFull = kBarKEmpty + kKStages,
+  kBarVEmpty = kBarVFull + kVStages,
+  kBarSFull = kBarVEmpty + kVStages,  // + (t & 1): S_t ready
+  kBarPFull = kBarSFull + 2,          // + 2*half + (t & 1): P_t,h written
+  kBarOFull = kBarPFull + 4,          // + 2*half + (t & 1): PV_t,h done
+  kBarDrain = kBarOFull + 4,
   kNumBars = kBarDrain + 1
 };
 
@@ -168,18 +177,22 @@ __global__ void __launch_bounds__(kThreads, 1)
   // ---------------------------------------------------------------- setup
   if (tid == 0) {
     mbar_init(bar(kBarQFull), 1);
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < kKStages; ++s) {
       mbar_init(bar(kBarKFull + s), 1);
       mbar_init(bar(kBarKEmpty + s), 1);
+    }
+    for (int s = 0; s < kVStages; ++s) {
       mbar_init(bar(kBarVFull + s), 1);
       mbar_init(bar(kBarVEmpty + s), 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(bar(kBarSFull + b), 1);
-      mbar_init(bar(kBarSEmpty + b), kSoftmaxThreads);
+    for (int b = 0; b < 2; ++b) mbar_init(bar(kBarSFull + b), 1);
+    // P and O barriers alternate with the tile parity: a half's softmax can run
+    // one tile ahead of the MMA thread, never two, so no barrier is ever two
+    // phases ahead of its waiter
+    for (int b = 0; b < 4; ++b) {
+      mbar_init(bar(kBarPFull + b), kSoftmaxThreads / 2);
       mbar_init(bar(kBarOFull + b), 1);
     }
-    mbar_init(bar(kBarPFull), kSoftmaxThreads);
     mbar_init(bar(kBarDrain), 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -246,49 +259,44 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int n_t = (n_u + 1) >> 1;
   const uint64_t lim = prm.wait_limit_ns;
 
-  if (warp == kProducerWarp) {
-    // ------------------------------------------------------------ TMA producer
+  if (warp == kProducerWarp || warp == kVProducerWarp) {
+    // ------------------------------------------------------------ TMA producers
+    // warp 8 streams Q and K, warp 10 streams V: a V slot frees only after the
+    // softmax of its tile, and must not hold back the K prefetch
     if (lane == 0 && n_t > 0) {
       const int64_t row0 = static_cast<int64_t>(bh) * prm.S;
-      int armed_k[kStages] = {}, armed_v[kStages] = {};
-      mbar_arrive_expect_tx(bar(kBarQFull), L::kQBytes);
-      for (int qb = 0; qb < 2; ++qb)
-        for (int h = 0; h < L::kDH; ++h)
-          tma_load_2d(sQ + h * kBM * 128 + qb * 64 * 128, &tmQ, bar(kBarQFull), h * 64,
-                      static_cast<int32_t>(row0 + (r1 + qb) * 64));
+      const bool is_k = warp == kProducerWarp;
+      const int nst = is_k ? kKStages : kVStages;
+      const uint32_t ring = is_k ? sK : sV;
+      const CUtensorMap* map = is_k ? &tmK : &tmV;
+      const int full0 = is_k ? kBarKFull : kBarVFull, empty0 = is_k ? kBarKEmpty : kBarVEmpty;
+      int armed[kKStages] = {0, 0, 0};
+      if (is_k) {
+        mbar_arrive_expect_tx(bar(kBarQFull), L::kQBytes);
+        for (int qb = 0; qb < 2; ++qb)
+          for (int h = 0; h < L::kDH; ++h)
+            tma_load_2d(sQ + h * kBM * 128 + qb * 64 * 128, &tmQ, bar(kBarQFull), h * 64,
+                        static_cast<int32_t>(row0 + (r1 + qb) * 64));
+      }
       for (int t = 0; t < n_t; ++t) {
-        const int s = t % kStages, n = t / kStages;
+        const int s = t % nst, n = t / nst;
         const int j0 = ulist[2 * t] & 0xFFFF;
         const int j1 = (2 * t + 1 < n_u) ? (ulist[2 * t + 1] & 0xFFFF) : j0;
-        if (t >= kStages && !mbar_wait(bar(kBarKEmpty + s), (n - 1) & 1, lim, abort_flag)) {
+        if (t >= nst && !mbar_wait(bar(empty0 + s), (n - 1) & 1, lim, abort_flag)) {
           record_abort(abort_flag, prm.status, kStatusTimeout);
           break;
         }
-        mbar_arrive_expect_tx(bar(kBarKFull + s), L::kKVBytes);
-        ++armed_k[s];
+        mbar_arrive_expect_tx(bar(full0 + s), L::kKVBytes);
+        ++armed[s];
         for (int kb = 0; kb < 2; ++kb)
           for (int h = 0; h < L::kDH; ++h)
-            tma_load_2d(sK + s * L::kKVBytes + h * kBN * 128 + kb * 64 * 128, &tmK,
-                        bar(kBarKFull + s), h * 64,
-                        static_cast<int32_t>(row0 + (kb ? j1 : j0) * 64));
-        if (t >= kStages && !mbar_wait(bar(kBarVEmpty + s), (n - 1) & 1, lim, abort_flag)) {
-          record_abort(abort_flag, prm.status, kStatusTimeout);
-          break;
-        }
-        mbar_arrive_expect_tx(bar(kBarVFull + s), L::kKVBytes);
-        ++armed_v[s];
-        for (int kb = 0; kb < 2; ++kb)
-          for (int h = 0; h < L::kDH; ++h)
-            tma_load_2d(sV + s * L::kKVBytes + h * kBN * 128 + kb * 64 * 128, &tmV,
-                        bar(kBarVFull + s), h * 64,
-                        static_cast<int32_t>(row0 + (kb ? j1 : j0) * 64));
+            tma_load_2d(ring + s * L::kKVBytes + h * kBN * 128 + kb * 64 * 128, map, bar(full0 + s),
+                        h * 64, static_cast<int32_t>(row0 + (kb ? j1 : j0) * 64));
       }
       // drain: every armed phase must complete before shared memory is released
-      mbar_wait(bar(kBarQFull), 0, kDrainLimitNs, nullptr);
-      for (int s = 0; s < kStages; ++s) {
-        if (armed_k[s]) mbar_wait(bar(kBarKFull + s), (armed_k[s] - 1) & 1, kDrainLimitNs, nullptr);
-        if (armed_v[s]) mbar_wait(bar(kBarVFull + s), (armed_v[s] - 1) & 1, kDrainLimitNs, nullptr);
-      }
+      if (is_k) mbar_wait(bar(kBarQFull), 0, kDrainLimitNs, nullptr);
+      for (int s = 0; s < nst; ++s)
+        if (armed[s]) mbar_wait(bar(full0 + s), (armed[s] - 1) & 1, kDrainLimitNs, nullptr);
     }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
@@ -298,40 +306,44 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = mbar_wait(bar(kBarQFull), 0, lim, abort_flag);
       tc_fence_after();
       auto issue_s = [&](int u) -> bool {
-        const int b = u & 1, s = u % kStages;
-        if (u >= 2 && !mbar_wait(bar(kBarSEmpty + b), ((u >> 1) - 1) & 1, lim, abort_flag)) return false;
-        if (!mbar_wait(bar(kBarKFull + s), (u / kStages) & 1, lim, abort_flag)) return false;
+        const int s = u % kKStages;
+        if (!mbar_wait(bar(kBarKFull + s), (u / kKStages) & 1, lim, abort_flag)) return false;
         tc_fence_after();
         const uint32_t kt = sK + s * L::kKVBytes;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * (kBM * 128) + (kk & 3) * 32;
           const uint32_t offk = (kk >> 2) * (kBN * 128) + (kk & 3) * 32;
-          tc_mma_ss(tmem + (b ? kColS1 : kColS0), sdesc_sw128(sQ + off, 16, 1024),
+          tc_mma_ss(tmem + ((u & 1) ? kColS1 : kColS0), sdesc_sw128(sQ + off, 16, 1024),
                     sdesc_sw128(kt + offk, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
         }
         tc_commit(bar(kBarKEmpty + s));
-        tc_commit(bar(kBarSFull + b));
+        tc_commit(bar(kBarSFull + (u & 1)));
         return true;
       };
       if (ok) ok = issue_s(0);
       for (int t = 0; ok && t < n_t; ++t) {
+        // S_{t+1} goes ahead of PV_t so the softmax of tile t+1 can start while PV_t runs
         if (t + 1 < n_t && !issue_s(t + 1)) { ok = false; break; }
-        const int s = t % kStages;
-        if (!mbar_wait(bar(kBarPFull), t & 1, lim, abort_flag)) { ok = false; break; }
-        if (!mbar_wait(bar(kBarVFull + s), (t / kStages) & 1, lim, abort_flag)) { ok = false; break; }
-        tc_fence_after();
+        const int s = t % kVStages;
+        if (!mbar_wait(bar(kBarVFull + s), (t / kVStages) & 1, lim, abort_flag)) { ok = false; break; }
         const uint32_t vt = sV + s * L::kKVBytes;
-        const uint32_t pcol = kColP + (t & 1) * 64;
+        const uint32_t pbuf = tmem + ((t & 1) ? kColS1 : kColS0);
 #pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk) {
-          // 16 keys per step: P columns [pcol + 8kk, +8); V rows [16kk, +16) of the tile,
-          // the 64-column halves of d kBN*128 bytes apart (MN-major operand)
-          tc_mma_ts(tmem + kColO, tmem + pcol + kk * 8, sdesc_sw128(vt + kk * 16 * 128, kBN * 128, 1024),
-                    idesc_pv, (t > 0 || kk > 0) ? 1u : 0u);
+        for (int h = 0; h < 2; ++h) {
+          if (!mbar_wait(bar(kBarPFull + 2 * h + (t & 1)), (t >> 1) & 1, lim, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          // keys [64h, 64h+64) of the tile: P columns pbuf + 64h + [0,32) (bf16 pairs),
+          // V rows [64h, 64h+64); the two 64-column halves of d are kBN*128 bytes apart
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            tc_mma_ts(tmem + (h ? kColO1 : kColO0), pbuf + h * 64 + kk * 8,
+                      sdesc_sw128(vt + (h * 4 + kk) * 16 * 128, kBN * 128, 1024), idesc_pv,
+                      (t > 0 || kk > 0) ? 1u : 0u);
+          tc_commit(bar(kBarOFull + 2 * h + (t & 1)));
         }
+        if (!ok) break;
         tc_commit(bar(kBarVEmpty + s));
-        tc_commit(bar(kBarOFull + (t & 1)));
       }
       if (!ok) record_abort(abort_flag, prm.status, kStatusTimeout);
       // drain: all MMAs this thread issued must finish before tensor memory is freed
@@ -341,141 +353,176 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ------------------------------------------------------------ softmax (warps 0-7)
     const int quarter = warp & 3;
-    const int half = warp >> 2;                // key block of the tile this warp handles
+    const int half = warp >> 2;                // key half of every tile this warp handles
     const int row = quarter * 32 + lane;       // query row == tensor-memory lane
     const int qh = row >> 6;                   // 0: block r1, 1: block r2
     const bool row_valid = qh == 0 || has2;
     const int bitsel = 1 << (16 + qh);
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const uint32_t o_col = half ? kColO1 : kColO0;
     const float sl2 = prm.scale_log2;
-    float m = -INFINITY;        // running (lazy) max, log2 units, same in both halves
-    float l = 0.f;              // this half's share of the row sum
+    float m = -INFINITY;        // lazy running max of this stream, log2 units
+    float l = 0.f;              // running sum of this stream
     bool ok = true;
     for (int t = 0; t < n_t; ++t) {
       const int b = t & 1;
       const int e = (2 * t + half < n_u) ? ulist[2 * t + half] : 0;
       const bool valid = (e & bitsel) != 0;    // uniform per warp
-      uint32_t sreg[2][32];
-      float mloc = -INFINITY;
-      bool got = warp_wait(bar(kBarSFull + b), (t >> 1) & 1, lim, abort_flag);
-      if (got) {
-        tc_fence_after();
-        if (valid) {
-          const uint32_t sbase = tmem + lane_off + (b ? kColS1 : kColS0) + half * 64;
-          tmem_ld32(sbase, sreg[0]);
-          tmem_ld32(sbase + 32, sreg[1]);
-          tmem_ld_wait();
-        }
-        tc_fence_before();
-        mbar_arrive(bar(kBarSEmpty + b));
-        if (valid) {
-          float mx[8];
+      if (!warp_wait(bar(kBarSFull + b), (t >> 1) & 1, lim, abort_flag)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t scol = tmem + lane_off + (b ? kColS1 : kColS0) + half * 64;
+      uint32_t pk[32];
+      if (valid) {
+        uint32_t s0[32], s1[32];
+        tmem_ld32(scol, s0);
+        tmem_ld_wait();
+        tmem_ld32(scol + 32, s1);   // in flight while the first 32 columns are processed
+        float mx[8];
+        float rs[4] = {0.f, 0.f, 0.f, 0.f};
+        // Speculative exponentials against the lazy max m: the tile max is formed
+        // alongside them and only a rise of more than 2^8 (or no max yet) sends
+        // the warp through the slow path below.
+        const bool spec = __all_sync(0xffffffffu, m > -INFINITY);
+        const float mneg = spec ? -m : 0.f;
 #pragma unroll
-          for (int i = 0; i < 8; ++i)
-            mx[i] = fmaxf(__uint_as_float(sreg[0][i]), __uint_as_float(sreg[1][i]));
+        for (int i = 0; i < 8; ++i) mx[i] = __uint_as_float(s0[i]);
 #pragma unroll
-          for (int i = 8; i < 32; ++i)
-            mx[i & 7] = fmaxf(mx[i & 7], fmaxf(__uint_as_float(sreg[0][i]), __uint_as_float(sreg[1][i])));
-          mloc = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                       fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * sl2;
+        for (int i = 8; i < 32; ++i) mx[i & 7] = fmaxf(mx[i & 7], __uint_as_float(s0[i]));
+        if (spec) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float p0 = fast_exp2(fmaf(__uint_as_float(s0[2 * i]), sl2, mneg));
+            const float p1 = fast_exp2(fmaf(__uint_as_float(s0[2 * i + 1]), sl2, mneg));
+            rs[i & 3] += p0 + p1;
+            pk[i] = pack_bf16x2(p0, p1);
+          }
         }
-      }
-      float* red_t = red + (t & 1) * (2 * kBM);
-      red_t[half * kBM + row] = mloc;
-      ok = bar_red_and(kSoftmaxBarrier, kSoftmaxThreads, ok && got);
-      if (!ok) break;
-      const float m_tile = fmaxf(mloc, red_t[(half ^ 1) * kBM + row]);
-      const float m_new = fmaxf(m, m_tile);
-      // lazy rescale: only when the max grows by more than 2^kRescaleThreshold
-      const bool need = (m > -INFINITY) && (m_new > m + kRescaleThreshold);
-      if (__any_sync(0xffffffffu, need)) {
-        if (t > 0 && !warp_wait(bar(kBarOFull + ((t - 1) & 1)), ((t - 1) >> 1) & 1, lim, abort_flag)) {
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) mx[i & 7] = fmaxf(mx[i & 7], __uint_as_float(s1[i]));
+        if (spec) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float p0 = fast_exp2(fmaf(__uint_as_float(s1[2 * i]), sl2, mneg));
+            const float p1 = fast_exp2(fmaf(__uint_as_float(s1[2 * i + 1]), sl2, mneg));
+            rs[i & 3] += p0 + p1;
+            pk[16 + i] = pack_bf16x2(p0, p1);
+          }
+        }
+        const float m_tile = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                                   fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * sl2;
+        const bool first = m == -INFINITY;
+        const bool need = !first && (m_tile > m + kRescaleThreshold);   // rescale O_h, l
+        const bool redo = first || need || !spec;                         // recompute p
+        const float m_old = m;
+        if (__any_sync(0xffffffffu, redo)) {
+          if (first || need) m = m_tile;
+          const float mn = -m;
+          if (redo) {
+            rs[0] = rs[1] = rs[2] = rs[3] = 0.f;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const float p0 = fast_exp2(fmaf(__uint_as_float(s0[2 * i]), sl2, mn));
+              const float p1 = fast_exp2(fmaf(__uint_as_float(s0[2 * i + 1]), sl2, mn));
+              const float p2 = fast_exp2(fmaf(__uint_as_float(s1[2 * i]), sl2, mn));
+              const float p3 = fast_exp2(fmaf(__uint_as_float(s1[2 * i + 1]), sl2, mn));
+              rs[i & 3] += (p0 + p1) + (p2 + p3);
+              pk[i] = pack_bf16x2(p0, p1);
+              pk[16 + i] = pack_bf16x2(p2, p3);
+            }
+          }
+        }
+        // P_t,h over the first 32 of this thread's S columns (S is already in registers)
+        tmem_st32(scol, pk);
+        // O_h must hold PV_{t-1},h before it is rescaled by 2^(m_old - m)
+        bool rescale = __any_sync(0xffffffffu, need);
+        if (rescale && t > 0 &&
+            !warp_wait(bar(kBarOFull + 2 * half + ((t - 1) & 1)), ((t - 1) >> 1) & 1, lim,
+                       abort_flag)) {
           ok = false;
-        } else {
+          rescale = false;
+        }
+        if (rescale) {
           tc_fence_after();
-          const float alpha = need ? fast_exp2(m - m_new) : 1.f;
+          const float alpha = need ? fast_exp2(m_old - m) : 1.f;
           l *= alpha;
 #pragma unroll
-          for (int c = 0; c < D / 64; ++c) {
+          for (int c = 0; c < D / 32; ++c) {
             uint32_t o[32];
-            const uint32_t oa = tmem + lane_off + kColO + half * (D / 2) + c * 32;
-            tmem_ld32(oa, o);
+            tmem_ld32(tmem + lane_off + o_col + c * 32, o);
             tmem_ld_wait();
 #pragma unroll
             for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-            tmem_st32(oa, o);
+            tmem_st32(tmem + lane_off + o_col + c * 32, o);
           }
-          tmem_st_wait();
         }
-      }
-      if (m == -INFINITY || need) m = m_new;
-      // p = 2^(s*scale*log2e - m); masked halves and not-yet-valid rows give 0
-      uint32_t pk[32];
-      float rs[4] = {0.f, 0.f, 0.f, 0.f};
-      if (valid && m > -INFINITY) {
-        const float mneg = -m;
-#pragma unroll
-        for (int c = 0; c < 2; ++c)
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const float p0 = fast_exp2(fmaf(__uint_as_float(sreg[c][2 * i]), sl2, mneg));
-            const float p1 = fast_exp2(fmaf(__uint_as_float(sreg[c][2 * i + 1]), sl2, mneg));
-            rs[i & 3] += p0 + p1;
-            pk[c * 16 + i] = pack_bf16x2(p0, p1);
-          }
+        l += (rs[0] + rs[1]) + (rs[2] + rs[3]);
       } else {
 #pragma unroll
         for (int i = 0; i < 32; ++i) pk[i] = 0u;
+        tmem_st32(scol, pk);
       }
-      l += (rs[0] + rs[1]) + (rs[2] + rs[3]);
-      // P_t goes to P[t&1]; PV_{t-2} (which read that buffer) must be complete
-      if (ok && t >= 2 && !warp_wait(bar(kBarOFull + (t & 1)), ((t - 2) >> 1) & 1, lim, abort_flag))
-        ok = false;
-      if (ok) {
-        tmem_st32(tmem + lane_off + kColP + (t & 1) * 64 + half * 32, pk);
-        tmem_st_wait();
-        tc_fence_before();
-        mbar_arrive(bar(kBarPFull));
-      }
+      tmem_st_wait();
+      if (!ok) break;
+      tc_fence_before();
+      mbar_arrive(bar(kBarPFull + 2 * half + (t & 1)));
     }
+    if (!ok) record_abort(abort_flag, prm.status, kStatusTimeout);
     // ------------------------------------------------------------ epilogue
     bool have_o = false;
     if (ok && n_t > 0) {
-      have_o = warp_wait(bar(kBarOFull + ((n_t - 1) & 1)), ((n_t - 1) >> 1) & 1, lim, abort_flag);
+      have_o = warp_wait(bar(kBarOFull + 2 * half + ((n_t - 1) & 1)), ((n_t - 1) >> 1) & 1, lim,
+                         abort_flag);
       tc_fence_after();
     }
-    float* red_l = red + 4 * kBM;              // slot 2: row-sum exchange (slots 0/1: maxima)
-    red_l[half * kBM + row] = l;
+    red[half * kBM + row] = m;
+    red[2 * kBM + half * kBM + row] = l;
+    // each half waited for its own last PV; after this barrier both O_0 and O_1 are final
+    tc_fence_before();
     const bool all_ok = bar_red_and(kSoftmaxBarrier, kSoftmaxThreads, ok && (n_t == 0 || have_o));
+    tc_fence_after();
     if (!all_ok) record_abort(abort_flag, prm.status, kStatusTimeout);
-    const float lt = l + red_l[(half ^ 1) * kBM + row];
+    const float m0 = red[row], m1 = red[kBM + row];
+    const float l0 = red[2 * kBM + row], l1 = red[3 * kBM + row];
+    const float M = fmaxf(m0, m1);
+    const float f0 = l0 > 0.f ? fast_exp2(m0 - M) : 0.f;
+    const float f1 = l1 > 0.f ? fast_exp2(m1 - M) : 0.f;
+    const float lt = f0 * l0 + f1 * l1;
+    const float inv_l = lt > 0.f ? 1.f / lt : 0.f;
+    const float g0 = f0 * inv_l, g1 = f1 * inv_l;
     const bool write = row_valid && all_ok;
     const int qrow = (qh ? r2 : r1) * 64 + (row & 63);
     const int64_t grow = static_cast<int64_t>(bh) * prm.S + qrow;
-    const float inv_l = lt > 0.f ? 1.f / lt : 0.f;
+    // this thread writes d columns [half*D/2, half*D/2 + D/2) of its row
     __nv_bfloat16* orow = prm.o + grow * D + half * (D / 2);
+    const bool read = all_ok && n_t > 0;
 #pragma unroll
     for (int c = 0; c < D / 64; ++c) {
-      uint32_t o[32];
-      if (have_o && all_ok) {
-        tmem_ld32(tmem + lane_off + kColO + half * (D / 2) + c * 32, o);
+      const uint32_t col = half * (D / 2) + c * 32;
+      uint32_t a[32], b2[32];
+      if (read) {
+        tmem_ld32(tmem + lane_off + kColO0 + col, a);
+        tmem_ld32(tmem + lane_off + kColO1 + col, b2);
         tmem_ld_wait();
-      } else {
-#pragma unroll
-        for (int i = 0; i < 32; ++i) o[i] = 0u;
       }
       if (write) {
         uint32_t w[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
-          w[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l);
+        for (int i = 0; i < 16; ++i) {
+          // a stream with l == 0 contributed nothing (its O may never have been written)
+          const float x0 = (g0 > 0.f ? __uint_as_float(a[2 * i]) * g0 : 0.f) +
+                           (g1 > 0.f ? __uint_as_float(b2[2 * i]) * g1 : 0.f);
+          const float x1 = (g0 > 0.f ? __uint_as_float(a[2 * i + 1]) * g0 : 0.f) +
+                           (g1 > 0.f ? __uint_as_float(b2[2 * i + 1]) * g1 : 0.f);
+          w[i] = pack_bf16x2(x0, x1);
+        }
         uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
 #pragma unroll
         for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
       }
     }
     if (write && half == 0 && prm.lse != nullptr)
-      prm.lse[grow] = lt > 0.f ? (m + __log2f(lt)) * 0.69314718055994530942f : -INFINITY;
+      prm.lse[grow] = lt > 0.f ? (M + __log2f(lt)) * 0.69314718055994530942f : -INFINITY;
   }
 
   tc_fence_before();
