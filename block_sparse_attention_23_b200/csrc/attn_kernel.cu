@@ -9,48 +9,47 @@
 // are computed).
 //
 // Work decomposition
-//   One CTA per (b, h, pair of query blocks): 128 query rows = query blocks
-//   2p and 2p+1.  The key blocks visited are the union of the two CSR rows;
-//   each union entry carries a 2-bit membership flag, and a query row whose
-//   block did not list the key block treats it as masked (probability 0, no
-//   exponentials evaluated).  Key tiles are 128 keys = two union entries (the
-//   second may be a repeat that both rows mask).  Every 64-key block is one
-//   contiguous slab of the [B,H,S,d] tensor, so each is a plain 2D TMA box at
-//   row (bh*S + 64*j).
+//   One CTA per (b, h, group of four query blocks 4g..4g+3) = two query
+//   tiles of 128 rows: tile 0 = blocks 4g, 4g+1; tile 1 = blocks 4g+2, 4g+3.
+//   The key blocks visited are the union of the four CSR rows, each entry with
+//   a 4-bit membership mask.  Key tiles are 128 keys = two union entries (the
+//   second may be a repeat that every row masks); each entry is one contiguous
+//   64 x d slab of the [B,H,S,d] tensor, loaded as a plain 2D TMA box, so both
+//   query tiles share every K/V tile that is loaded.  A query tile computes a
+//   key tile only if one of its two blocks lists one of the tile's entries; a
+//   row whose block did not list an entry gives it probability 0 (no
+//   exponentials evaluated).
 //
-// Two independent softmax streams per row
-//   Key half h of every tile (the tile's h-th 64-key block) feeds its own
-//   accumulator O_h with its own running max m_h and sum l_h, so the two
-//   threads that serve a row never wait for each other inside the key loop.
-//   The epilogue merges them exactly:
-//     M = max(m_0, m_1),  f_h = 2^(m_h - M),
-//     O = (f_0 O_0 + f_1 O_1) / (f_0 l_0 + f_1 l_1),  LSE = ln2 (M + log2 L).
-//   Each stream keeps a lazy maximum: m_h is raised (and O_h, l_h rescaled by
-//   2^(m_old - m_new)) only when a tile exceeds it by more than 2^8, so p <= 256.
+// Roles (384 threads)
+//   warps 0-3   softmax of query tile 0, warps 4-7 of query tile 1: thread i of
+//               the group owns row i (= tensor-memory lane i) for all 128 keys
+//               of a tile: tcgen05.ld of S, lazy running max, exp2, P (bf16)
+//               written over the first 64 S columns, O rescale, epilogue.
+//   warp 8      TMA producer of Q and K (and the union-list compaction).
+//   warp 9      tensor-memory allocation and the single MMA-issuing thread.
+//   warp 10     TMA producer of V; warp 11 idles (completes warpgroup 2).
 //
-// Roles (352 threads)
-//   warps 0-7  softmax.  Warp w serves tensor-memory lanes 32*(w%4).. (query
-//              rows) and key half w/4: tcgen05.ld of its 64 S columns,
-//              max, exp2, P (bf16) written over the first 32 of those
-//              columns, lazy rescale of its O_h row, epilogue.
-//   warp 8     TMA producer of Q and K (and the union-list compaction).
-//   warp 10    TMA producer of V.
-//   warp 9     tensor-memory allocation and the single MMA-issuing thread:
-//              S_t = Q K_t^T into buffer t&1, then O_h += P_t,h V_t,h for
-//              h = 0, 1 as soon as that half of P is in place (A operand read
-//              from tensor memory).
+// MMA order (ping-pong between the two query tiles)
+//   S_0(0), S_1(0), then for every key tile t: PV_0(t), S_0(t+1), PV_1(t),
+//   S_1(t+1).  While softmax 0 works on S_0(t) the tensor cores run PV_1(t-1)
+//   and S_1(t), and the other way round, so each softmax group has about two
+//   MMA tile-products of time.  S_x(t+1) overwrites the S/P buffer of tile x
+//   only after PV_x(t), which read P_x(t), was issued by the same thread (MMAs
+//   of one thread execute in issue order).
 //
-// Tensor memory (512 columns): S/P buffers [0,128) and [128,256), O_0 at 256,
-// O_1 at 384 (d columns each).  Ordering of the in-place P: S_{t+2} reuses
-// buffer t&1 and is issued after PV_t by the same thread, and MMAs of one
-// thread execute in issue order; the completion of S_t (which the softmax
-// waits for) also implies the completion of PV_{t-2}, which read P_{t-2}.
+// Online softmax with a lazy maximum: the running max m of a row is raised
+// (and O, l rescaled by 2^(m_old - m_new)) only when a tile's max exceeds it by
+// more than 2^8; otherwise p <= 256 and O / l, LSE = ln2 (m + log2 l) are
+// unchanged in exact arithmetic.  Exponentials are computed against m while
+// the tile max is formed; a rise past the threshold (or a row's first tile)
+// recomputes them from the S values still in tensor memory.
+//
+// Tensor memory (512 columns): tile 0 S/P [0,128), O [128,256);
+// tile 1 S/P [256,384), O [384,512).
 //
 // Every mbarrier wait is time-bounded; a wait that runs out records
 // kStatusTimeout, raises a CTA-wide abort flag, and the CTA drains its own TMA
 // loads and MMAs (bounded again) before freeing tensor memory and returning.
-// The softmax warps share one named barrier, in the epilogue, and agree on
-// aborts there through bar.red.and.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -60,33 +59,38 @@
 
 namespace nabla {
 
-constexpr int kBM = 128;        // query rows per CTA (two 64-token blocks)
+constexpr int kBM = 128;        // rows per query tile (two 64-token blocks)
+constexpr int kQTiles = 2;      // query tiles per CTA
 constexpr int kBN = 128;        // keys per tile (two 64-token blocks)
-constexpr int kKStages = 3;     // K ring depth (K is needed one S-MMA after its slot frees)
+constexpr int kKStages = 2;     // K ring depth
 constexpr int kVStages = 2;     // V ring depth
 constexpr int kSoftmaxThreads = 256;
-constexpr int kThreads = kSoftmaxThreads + 96;
-constexpr int kProducerWarp = 8, kMmaWarp = 9, kVProducerWarp = 10;
+constexpr int kThreads = kSoftmaxThreads + 128;   // warpgroups 0, 1 softmax; 2 load/MMA
+constexpr int kProducerWarp = 8, kMmaWarp = 9, kVProducerWarp = 10;   // warp 11 idles
+// Register budgets after set-up: a softmax thread holds a whole S row (128
+// values); the load/MMA warpgroup needs few.  8*216 + 4*72 = 12*168, the
+// launch allocation (checked on the host before launch).
+constexpr int kRegsSoftmax = 216, kRegsOther = 72, kRegsLaunch = 168;
 constexpr int kMaxNb = 4096;    // blocks per head supported
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO0 = 256, kColO1 = 384;
 constexpr float kRescaleThreshold = 8.0f;            // log2 units
 constexpr uint64_t kDrainLimitNs = 1000000000ull;   // 1 s for draining in-flight work
-constexpr int kSoftmaxBarrier = 1;                   // named barrier id of warps 0-7
+
+__host__ __device__ constexpr uint32_t col_s(int x) { return x ? 256u : 0u; }
+__host__ __device__ constexpr uint32_t col_o(int x) { return x ? 384u : 128u; }
 
 template <int D>
 struct AttnSmem {
   static constexpr int kDH = D / 64;                       // 64-column halves of d
-  static constexpr uint32_t kQBytes = kBM * D * 2;
+  static constexpr uint32_t kQBytes = kBM * D * 2;         // one query tile
   static constexpr uint32_t kKVBytes = kBN * D * 2;        // one K or V stage
   static constexpr uint32_t kOffQ = 0;
-  static constexpr uint32_t kOffK = kOffQ + kQBytes;
+  static constexpr uint32_t kOffK = kOffQ + kQTiles * kQBytes;
   static constexpr uint32_t kOffV = kOffK + kKStages * kKVBytes;
   static constexpr uint32_t kOffBar = kOffV + kVStages * kKVBytes;  // 32 mbarriers
   static constexpr uint32_t kOffMisc = kOffBar + 256;      // tmem base, abort, n_u
-  static constexpr uint32_t kOffRed = kOffMisc + 64;       // [2 quantity][2 half][128] floats
-  static constexpr uint32_t kOffBitmap = kOffRed + 2 * 2 * kBM * 4;   // 2 x kMaxNb/32 words
-  static constexpr uint32_t kOffList = kOffBitmap + 2 * (kMaxNb / 32) * 4;
+  static constexpr uint32_t kOffBitmap = kOffMisc + 64;    // 4 x kMaxNb/32 words
+  static constexpr uint32_t kOffList = kOffBitmap + 4 * (kMaxNb / 32) * 4;
   static constexpr uint32_t kBytes = kOffList + kMaxNb * 4;
   static constexpr uint32_t kAlloc = kBytes + 1024;        // slack for 1024-byte alignment
 };
@@ -98,10 +102,10 @@ enum : int {
   kBarKEmpty = kBarKFull + kKStages,
   kBarVFull = kBarKEmpty + kKStages,
   kBarVEmpty = kBarVFull + kVStages,
-  kBarSFull = kBarVEmpty + kVStages,  // + (t & 1): S_t ready
-  kBarPFull = kBarSFull + 2,          // + 2*half + (t & 1): P_t,h written
-  kBarOFull = kBarPFull + 4,          // + 2*half + (t & 1): PV_t,h done
-  kBarDrain = kBarOFull + 4,
+  kBarSFull = kBarVEmpty + kVStages,  // + query tile: S ready
+  kBarPFull = kBarSFull + kQTiles,    // + query tile: P written
+  kBarOFull = kBarPFull + kQTiles,    // + query tile: PV done
+  kBarDrain = kBarOFull + kQTiles,
   kNumBars = kBarDrain + 1
 };
 
@@ -111,7 +115,7 @@ struct AttnParams {
   __nv_bfloat16* o;
   float* lse;
   int* status;
-  int H, S, nb, npairs;
+  int H, S, nb, ngroups;
   float scale_log2;        // softmax scale * log2(e)
   uint64_t wait_limit_ns;
 };
@@ -128,19 +132,8 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, uint64_
   return __all_sync(0xffffffffu, mbar_wait(bar, parity, limit_ns, abort));
 }
 
-// Named barrier over `n` threads that also ANDs a predicate across them.
-__device__ __forceinline__ bool bar_red_and(int id, int n, bool pred) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\t"
-      "setp.ne.u32 q, %1, 0;\n\t"
-      "bar.red.and.pred p, %2, %3, q;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(r)
-      : "r"(static_cast<uint32_t>(pred)), "r"(id), "r"(n)
-      : "memory");
-  return r != 0;
-}
+// Membership mask of query tile x (bits of its two blocks) in union entry e.
+__device__ __forceinline__ int tile_bits(int e, int x) { return (e >> (16 + 2 * x)) & 3; }
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -160,18 +153,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile uint32_t* tmem_holder = misc;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
   volatile int* n_union_s = reinterpret_cast<volatile int*>(misc + 2);
-  float* red = reinterpret_cast<float*>(gbase + L::kOffRed);
-  uint32_t* bm1 = reinterpret_cast<uint32_t*>(gbase + L::kOffBitmap);
-  uint32_t* bm2 = bm1 + kMaxNb / 32;
+  uint32_t* bm = reinterpret_cast<uint32_t*>(gbase + L::kOffBitmap);   // [4][kMaxNb/32]
   int32_t* ulist = reinterpret_cast<int32_t*>(gbase + L::kOffList);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int item = blockIdx.x;
-  const int bh = item / prm.npairs;
-  const int pair = item % prm.npairs;
+  const int bh = item / prm.ngroups;
+  const int grp = item % prm.ngroups;
   const int nb = prm.nb;
-  const int r1 = 2 * pair, r2 = 2 * pair + 1;
-  const bool has2 = r2 < nb;
+  const int r0 = 4 * grp;                       // first query block of the group
+  const int nq = min(4, nb - r0);               // query blocks present (1..4)
   auto bar = [&](int i) { return bar0 + 8u * static_cast<uint32_t>(i); };
 
   // ---------------------------------------------------------------- setup
@@ -185,13 +176,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar(kBarVFull + s), 1);
       mbar_init(bar(kBarVEmpty + s), 1);
     }
-    for (int b = 0; b < 2; ++b) mbar_init(bar(kBarSFull + b), 1);
-    // P and O barriers alternate with the tile parity: a half's softmax can run
-    // one tile ahead of the MMA thread, never two, so no barrier is ever two
-    // phases ahead of its waiter
-    for (int b = 0; b < 4; ++b) {
-      mbar_init(bar(kBarPFull + b), kSoftmaxThreads / 2);
-      mbar_init(bar(kBarOFull + b), 1);
+    for (int x = 0; x < kQTiles; ++x) {
+      mbar_init(bar(kBarSFull + x), 1);
+      mbar_init(bar(kBarPFull + x), kSoftmaxThreads / kQTiles);
+      mbar_init(bar(kBarOFull + x), 1);
     }
     mbar_init(bar(kBarDrain), 1);
     *abort_flag = 0;
@@ -207,23 +195,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_prefetch_desc(&tmV);
   }
   const int nw = (nb + 31) >> 5;
-  for (int i = tid; i < 2 * nw; i += kThreads) (i < nw ? bm1[i] : bm2[i - nw]) = 0u;
+  for (int i = tid; i < 4 * (kMaxNb / 32); i += kThreads) bm[i] = 0u;
   __syncthreads();
-  {
-    const int64_t g1 = static_cast<int64_t>(bh) * nb + r1;
-    const int b1 = prm.row_ptr[g1], e1 = prm.row_ptr[g1 + 1];
-    for (int i = b1 + tid; i < e1; i += kThreads) {
+  for (int qb = 0; qb < nq; ++qb) {
+    const int64_t g = static_cast<int64_t>(bh) * nb + r0 + qb;
+    const int b = prm.row_ptr[g], e = prm.row_ptr[g + 1];
+    uint32_t* bmq = bm + qb * (kMaxNb / 32);
+    for (int i = b + tid; i < e; i += kThreads) {
       const int c = prm.col_idx[i];
-      if (static_cast<unsigned>(c) < static_cast<unsigned>(nb)) atomicOr(&bm1[c >> 5], 1u << (c & 31));
+      if (static_cast<unsigned>(c) < static_cast<unsigned>(nb)) atomicOr(&bmq[c >> 5], 1u << (c & 31));
       else atomicOr(prm.status, kStatusBadIndex);
-    }
-    if (has2) {
-      const int b2 = prm.row_ptr[g1 + 1], e2 = prm.row_ptr[g1 + 2];
-      for (int i = b2 + tid; i < e2; i += kThreads) {
-        const int c = prm.col_idx[i];
-        if (static_cast<unsigned>(c) < static_cast<unsigned>(nb)) atomicOr(&bm2[c >> 5], 1u << (c & 31));
-        else atomicOr(prm.status, kStatusBadIndex);
-      }
     }
   }
   __syncthreads();
@@ -231,9 +212,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     int run = 0;
     for (int w0 = 0; w0 < nw; w0 += 32) {
       const int w = w0 + lane;
-      const uint32_t u1 = w < nw ? bm1[w] : 0u, u2 = w < nw ? bm2[w] : 0u;
-      uint32_t u = u1 | u2;
-      const int cnt = __popc(u);
+      uint32_t u[4];
+#pragma unroll
+      for (int qb = 0; qb < 4; ++qb) u[qb] = w < nw ? bm[qb * (kMaxNb / 32) + w] : 0u;
+      uint32_t any = u[0] | u[1] | u[2] | u[3];
+      const int cnt = __popc(any);
       int incl = cnt;
 #pragma unroll
       for (int off = 1; off < 32; off <<= 1) {
@@ -241,11 +224,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane >= off) incl += y;
       }
       int pos = run + incl - cnt;
-      while (u) {
-        const int b = __ffs(u) - 1;
-        u &= u - 1;
-        ulist[pos++] = (w * 32 + b) | (static_cast<int>((u1 >> b) & 1u) << 16) |
-                       (static_cast<int>((u2 >> b) & 1u) << 17);
+      while (any) {
+        const int b = __ffs(any) - 1;
+        any &= any - 1;
+        int mem = 0;
+#pragma unroll
+        for (int qb = 0; qb < 4; ++qb) mem |= static_cast<int>((u[qb] >> b) & 1u) << qb;
+        ulist[pos++] = (w * 32 + b) | (mem << 16);
       }
       run += __shfl_sync(0xffffffffu, incl, 31);
     }
@@ -258,7 +243,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int n_u = *n_union_s;
   const int n_t = (n_u + 1) >> 1;
   const uint64_t lim = prm.wait_limit_ns;
+  // membership of key tile t: OR of its two entries
+  auto tile_entry = [&](int t, int i) { return (2 * t + i < n_u) ? ulist[2 * t + i] : 0; };
+  auto tile_active = [&](int t, int x) {
+    return tile_bits(tile_entry(t, 0) | tile_entry(t, 1), x) != 0;
+  };
 
+  if (warp >= 8) {
+  setmaxnreg_dec<kRegsOther>();
   if (warp == kProducerWarp || warp == kVProducerWarp) {
     // ------------------------------------------------------------ TMA producers
     // warp 8 streams Q and K, warp 10 streams V: a V slot frees only after the
@@ -270,13 +262,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t ring = is_k ? sK : sV;
       const CUtensorMap* map = is_k ? &tmK : &tmV;
       const int full0 = is_k ? kBarKFull : kBarVFull, empty0 = is_k ? kBarKEmpty : kBarVEmpty;
-      int armed[kKStages] = {0, 0, 0};
+      int armed0 = 0, armed1 = 0;
       if (is_k) {
-        mbar_arrive_expect_tx(bar(kBarQFull), L::kQBytes);
-        for (int qb = 0; qb < 2; ++qb)
+        mbar_arrive_expect_tx(bar(kBarQFull), kQTiles * L::kQBytes);
+        for (int qb = 0; qb < 4; ++qb)
           for (int h = 0; h < L::kDH; ++h)
-            tma_load_2d(sQ + h * kBM * 128 + qb * 64 * 128, &tmQ, bar(kBarQFull), h * 64,
-                        static_cast<int32_t>(row0 + (r1 + qb) * 64));
+            tma_load_2d(sQ + (qb >> 1) * L::kQBytes + h * kBM * 128 + (qb & 1) * 64 * 128, &tmQ,
+                        bar(kBarQFull), h * 64, static_cast<int32_t>(row0 + (r0 + qb) * 64));
       }
       for (int t = 0; t < n_t; ++t) {
         const int s = t % nst, n = t / nst;
@@ -287,7 +279,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         mbar_arrive_expect_tx(bar(full0 + s), L::kKVBytes);
-        ++armed[s];
+        (s ? armed1 : armed0) += 1;
         for (int kb = 0; kb < 2; ++kb)
           for (int h = 0; h < L::kDH; ++h)
             tma_load_2d(ring + s * L::kKVBytes + h * kBN * 128 + kb * 64 * 128, map, bar(full0 + s),
@@ -295,234 +287,201 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // drain: every armed phase must complete before shared memory is released
       if (is_k) mbar_wait(bar(kBarQFull), 0, kDrainLimitNs, nullptr);
-      for (int s = 0; s < nst; ++s)
-        if (armed[s]) mbar_wait(bar(full0 + s), (armed[s] - 1) & 1, kDrainLimitNs, nullptr);
+      if (armed0) mbar_wait(bar(full0 + 0), (armed0 - 1) & 1, kDrainLimitNs, nullptr);
+      if (armed1) mbar_wait(bar(full0 + 1), (armed1 - 1) & 1, kDrainLimitNs, nullptr);
     }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0 && n_t > 0) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(kBM, kBN, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(kBM, D, true);
+      int n_pv[kQTiles] = {0, 0};   // PV products issued per query tile
       bool ok = mbar_wait(bar(kBarQFull), 0, lim, abort_flag);
       tc_fence_after();
-      auto issue_s = [&](int u) -> bool {
-        const int s = u % kKStages;
-        if (!mbar_wait(bar(kBarKFull + s), (u / kKStages) & 1, lim, abort_flag)) return false;
-        tc_fence_after();
-        const uint32_t kt = sK + s * L::kKVBytes;
+      auto issue_s = [&](int x, int t) {
+        const uint32_t kt = sK + (t % kKStages) * L::kKVBytes;
+        const uint32_t qt = sQ + x * L::kQBytes;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * (kBM * 128) + (kk & 3) * 32;
           const uint32_t offk = (kk >> 2) * (kBN * 128) + (kk & 3) * 32;
-          tc_mma_ss(tmem + ((u & 1) ? kColS1 : kColS0), sdesc_sw128(sQ + off, 16, 1024),
+          tc_mma_ss(tmem + col_s(x), sdesc_sw128(qt + off, 16, 1024),
                     sdesc_sw128(kt + offk, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
         }
-        tc_commit(bar(kBarKEmpty + s));
-        tc_commit(bar(kBarSFull + (u & 1)));
+        tc_commit(bar(kBarSFull + x));
+      };
+      auto issue_pv = [&](int x, int t) -> bool {
+        if (!mbar_wait(bar(kBarPFull + x), n_pv[x] & 1, lim, abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t vt = sV + (t % kVStages) * L::kKVBytes;
+#pragma unroll
+        for (int kk = 0; kk < kBN / 16; ++kk)
+          // 16 keys per step: P columns [8kk, 8kk+8) of the S/P buffer, V rows
+          // [16kk, 16kk+16); the 64-column halves of d are kBN*128 bytes apart
+          tc_mma_ts(tmem + col_o(x), tmem + col_s(x) + kk * 8,
+                    sdesc_sw128(vt + kk * 16 * 128, kBN * 128, 1024), idesc_pv,
+                    (n_pv[x] > 0 || kk > 0) ? 1u : 0u);
+        tc_commit(bar(kBarOFull + x));
+        ++n_pv[x];
         return true;
       };
-      if (ok) ok = issue_s(0);
+      if (ok) ok = mbar_wait(bar(kBarKFull + 0), 0, lim, abort_flag);
+      if (ok) {
+        tc_fence_after();
+        for (int x = 0; x < kQTiles; ++x)
+          if (tile_active(0, x)) issue_s(x, 0);
+        tc_commit(bar(kBarKEmpty + 0));
+      }
       for (int t = 0; ok && t < n_t; ++t) {
-        // S_{t+1} goes ahead of PV_t so the softmax of tile t+1 can start while PV_t runs
-        if (t + 1 < n_t && !issue_s(t + 1)) { ok = false; break; }
-        const int s = t % kVStages;
-        if (!mbar_wait(bar(kBarVFull + s), (t / kVStages) & 1, lim, abort_flag)) { ok = false; break; }
-        const uint32_t vt = sV + s * L::kKVBytes;
-        const uint32_t pbuf = tmem + ((t & 1) ? kColS1 : kColS0);
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          if (!mbar_wait(bar(kBarPFull + 2 * h + (t & 1)), (t >> 1) & 1, lim, abort_flag)) { ok = false; break; }
-          tc_fence_after();
-          // keys [64h, 64h+64) of the tile: P columns pbuf + 64h + [0,32) (bf16 pairs),
-          // V rows [64h, 64h+64); the two 64-column halves of d are kBN*128 bytes apart
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            tc_mma_ts(tmem + (h ? kColO1 : kColO0), pbuf + h * 64 + kk * 8,
-                      sdesc_sw128(vt + (h * 4 + kk) * 16 * 128, kBN * 128, 1024), idesc_pv,
-                      (t > 0 || kk > 0) ? 1u : 0u);
-          tc_commit(bar(kBarOFull + 2 * h + (t & 1)));
+        const bool more = t + 1 < n_t;
+        if (!mbar_wait(bar(kBarVFull + t % kVStages), (t / kVStages) & 1, lim, abort_flag)) { ok = false; break; }
+        if (more && !mbar_wait(bar(kBarKFull + (t + 1) % kKStages), ((t + 1) / kKStages) & 1, lim,
+                               abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        for (int x = 0; x < kQTiles; ++x) {
+          if (tile_active(t, x) && !issue_pv(x, t)) { ok = false; break; }
+          if (more && tile_active(t + 1, x)) issue_s(x, t + 1);
         }
         if (!ok) break;
-        tc_commit(bar(kBarVEmpty + s));
+        if (more) tc_commit(bar(kBarKEmpty + (t + 1) % kKStages));
+        tc_commit(bar(kBarVEmpty + t % kVStages));
       }
       if (!ok) record_abort(abort_flag, prm.status, kStatusTimeout);
       // drain: all MMAs this thread issued must finish before tensor memory is freed
       tc_commit(bar(kBarDrain));
       mbar_wait(bar(kBarDrain), 0, kDrainLimitNs, nullptr);
     }
+  }
   } else {
+    setmaxnreg_inc<kRegsSoftmax>();
     // ------------------------------------------------------------ softmax (warps 0-7)
+    const int x = warp >> 2;                   // query tile of this warp group
     const int quarter = warp & 3;
-    const int half = warp >> 2;                // key half of every tile this warp handles
-    const int row = quarter * 32 + lane;       // query row == tensor-memory lane
-    const int qh = row >> 6;                   // 0: block r1, 1: block r2
-    const bool row_valid = qh == 0 || has2;
-    const int bitsel = 1 << (16 + qh);
+    const int row = quarter * 32 + lane;       // row of the tile == tensor-memory lane
+    const int qh = row >> 6;                   // block 4g + 2x + qh
+    const int qblock = r0 + 2 * x + qh;
+    const bool row_valid = qblock < nb;
+    const int bit = 1 << (16 + 2 * x + qh);
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-    const uint32_t o_col = half ? kColO1 : kColO0;
+    const uint32_t s_base = tmem + lane_off + col_s(x);
+    const uint32_t o_base = tmem + lane_off + col_o(x);
     const float sl2 = prm.scale_log2;
-    float m = -INFINITY;        // lazy running max of this stream, log2 units
-    float l = 0.f;              // running sum of this stream
+    float m = -INFINITY;        // lazy running max of the row, log2 units
+    float l = 0.f;              // running sum of the row
+    int c = 0;                  // key tiles this query tile has processed
     bool ok = true;
     for (int t = 0; t < n_t; ++t) {
-      const int b = t & 1;
-      const int e = (2 * t + half < n_u) ? ulist[2 * t + half] : 0;
-      const bool valid = (e & bitsel) != 0;    // uniform per warp
-      if (!warp_wait(bar(kBarSFull + b), (t >> 1) & 1, lim, abort_flag)) { ok = false; break; }
+      if (!tile_active(t, x)) continue;        // same decision as the MMA issuer
+      const bool v0 = (tile_entry(t, 0) & bit) != 0;   // uniform per warp
+      const bool v1 = (tile_entry(t, 1) & bit) != 0;
+      if (!warp_wait(bar(kBarSFull + x), c & 1, lim, abort_flag)) { ok = false; break; }
       tc_fence_after();
-      const uint32_t scol = tmem + lane_off + (b ? kColS1 : kColS0) + half * 64;
-      uint32_t pk[32];
-      if (valid) {
-        uint32_t s0[32], s1[32];
-        tmem_ld32(scol, s0);
-        tmem_ld_wait();
-        tmem_ld32(scol + 32, s1);   // in flight while the first 32 columns are processed
-        float mx[8];
-        float rs[4] = {0.f, 0.f, 0.f, 0.f};
-        // Speculative exponentials against the lazy max m: the tile max is formed
-        // alongside them and only a rise of more than 2^8 (or no max yet) sends
-        // the warp through the slow path below.
-        const bool spec = __all_sync(0xffffffffu, m > -INFINITY);
-        const float mneg = spec ? -m : 0.f;
+      // the whole S row in one batch of loads (one load latency per tile)
+      uint32_t sv[4][32];
+      if (v0) { tmem_ld32(s_base, sv[0]); tmem_ld32(s_base + 32, sv[1]); }
+      if (v1) { tmem_ld32(s_base + 64, sv[2]); tmem_ld32(s_base + 96, sv[3]); }
+      tmem_ld_wait();
+      float mx[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) mx[i] = __uint_as_float(s0[i]);
+      for (int i = 0; i < 8; ++i) mx[i] = -INFINITY;
 #pragma unroll
-        for (int i = 8; i < 32; ++i) mx[i & 7] = fmaxf(mx[i & 7], __uint_as_float(s0[i]));
-        if (spec) {
+      for (int ch = 0; ch < 4; ++ch) {
+        if ((ch < 2) ? v0 : v1) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) mx[i & 7] = fmaxf(mx[i & 7], __uint_as_float(sv[ch][i]));
+        }
+      }
+      const float m_tile = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                                 fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * sl2;
+      const bool has = m_tile > -INFINITY;
+      const bool first = m == -INFINITY;
+      const bool need = has && !first && (m_tile > m + kRescaleThreshold);   // rescale O, l
+      const float m_old = m;
+      if (has && (first || need)) m = m_tile;
+      // O must hold the previous PV of this tile before it is rescaled by 2^(m_old - m)
+      bool rescale = __any_sync(0xffffffffu, need);
+      if (rescale && c > 0 && !warp_wait(bar(kBarOFull + x), (c - 1) & 1, lim, abort_flag)) {
+        ok = false;
+        rescale = false;
+      }
+      if (rescale) {
+        tc_fence_after();
+        const float alpha = need ? fast_exp2(m_old - m) : 1.f;
+        l *= alpha;
+#pragma unroll 1
+        for (int cc = 0; cc < D / 16; ++cc) {
+          uint32_t o[16];
+          tmem_ld16(o_base + cc * 16, o);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 16; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          tmem_st16(o_base + cc * 16, o);
+          tmem_st_wait();
+        }
+      }
+      // p = 2^(s*scale*log2e - m); P chunk ch (keys [32ch, 32ch+32)) goes to
+      // columns [16ch, 16ch+16), whose S values are already in registers
+      const bool live = m > -INFINITY;
+      const float mneg = live ? -m : 0.f;
+      float rs[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int ch = 0; ch < 4; ++ch) {
+        uint32_t pk[16];
+        if (((ch < 2) ? v0 : v1) && live) {
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            const float p0 = fast_exp2(fmaf(__uint_as_float(s0[2 * i]), sl2, mneg));
-            const float p1 = fast_exp2(fmaf(__uint_as_float(s0[2 * i + 1]), sl2, mneg));
+            const float p0 = fast_exp2(fmaf(__uint_as_float(sv[ch][2 * i]), sl2, mneg));
+            const float p1 = fast_exp2(fmaf(__uint_as_float(sv[ch][2 * i + 1]), sl2, mneg));
             rs[i & 3] += p0 + p1;
             pk[i] = pack_bf16x2(p0, p1);
           }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) pk[i] = 0u;
         }
-        tmem_ld_wait();
-#pragma unroll
-        for (int i = 0; i < 32; ++i) mx[i & 7] = fmaxf(mx[i & 7], __uint_as_float(s1[i]));
-        if (spec) {
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const float p0 = fast_exp2(fmaf(__uint_as_float(s1[2 * i]), sl2, mneg));
-            const float p1 = fast_exp2(fmaf(__uint_as_float(s1[2 * i + 1]), sl2, mneg));
-            rs[i & 3] += p0 + p1;
-            pk[16 + i] = pack_bf16x2(p0, p1);
-          }
-        }
-        const float m_tile = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                                   fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * sl2;
-        const bool first = m == -INFINITY;
-        const bool need = !first && (m_tile > m + kRescaleThreshold);   // rescale O_h, l
-        const bool redo = first || need || !spec;                         // recompute p
-        const float m_old = m;
-        if (__any_sync(0xffffffffu, redo)) {
-          if (first || need) m = m_tile;
-          const float mn = -m;
-          if (redo) {
-            rs[0] = rs[1] = rs[2] = rs[3] = 0.f;
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const float p0 = fast_exp2(fmaf(__uint_as_float(s0[2 * i]), sl2, mn));
-              const float p1 = fast_exp2(fmaf(__uint_as_float(s0[2 * i + 1]), sl2, mn));
-              const float p2 = fast_exp2(fmaf(__uint_as_float(s1[2 * i]), sl2, mn));
-              const float p3 = fast_exp2(fmaf(__uint_as_float(s1[2 * i + 1]), sl2, mn));
-              rs[i & 3] += (p0 + p1) + (p2 + p3);
-              pk[i] = pack_bf16x2(p0, p1);
-              pk[16 + i] = pack_bf16x2(p2, p3);
-            }
-          }
-        }
-        // P_t,h over the first 32 of this thread's S columns (S is already in registers)
-        tmem_st32(scol, pk);
-        // O_h must hold PV_{t-1},h before it is rescaled by 2^(m_old - m)
-        bool rescale = __any_sync(0xffffffffu, need);
-        if (rescale && t > 0 &&
-            !warp_wait(bar(kBarOFull + 2 * half + ((t - 1) & 1)), ((t - 1) >> 1) & 1, lim,
-                       abort_flag)) {
-          ok = false;
-          rescale = false;
-        }
-        if (rescale) {
-          tc_fence_after();
-          const float alpha = need ? fast_exp2(m_old - m) : 1.f;
-          l *= alpha;
-#pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t o[32];
-            tmem_ld32(tmem + lane_off + o_col + c * 32, o);
-            tmem_ld_wait();
-#pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-            tmem_st32(tmem + lane_off + o_col + c * 32, o);
-          }
-        }
-        l += (rs[0] + rs[1]) + (rs[2] + rs[3]);
-      } else {
-#pragma unroll
-        for (int i = 0; i < 32; ++i) pk[i] = 0u;
-        tmem_st32(scol, pk);
+        tmem_st16(s_base + ch * 16, pk);
       }
+      l += (rs[0] + rs[1]) + (rs[2] + rs[3]);
       tmem_st_wait();
       if (!ok) break;
       tc_fence_before();
-      mbar_arrive(bar(kBarPFull + 2 * half + (t & 1)));
+      mbar_arrive(bar(kBarPFull + x));
+      ++c;
     }
     if (!ok) record_abort(abort_flag, prm.status, kStatusTimeout);
     // ------------------------------------------------------------ epilogue
     bool have_o = false;
-    if (ok && n_t > 0) {
-      have_o = warp_wait(bar(kBarOFull + 2 * half + ((n_t - 1) & 1)), ((n_t - 1) >> 1) & 1, lim,
-                         abort_flag);
+    if (ok && c > 0) {
+      have_o = warp_wait(bar(kBarOFull + x), (c - 1) & 1, lim, abort_flag);
+      if (!have_o) record_abort(abort_flag, prm.status, kStatusTimeout);
       tc_fence_after();
     }
-    red[half * kBM + row] = m;
-    red[2 * kBM + half * kBM + row] = l;
-    // each half waited for its own last PV; after this barrier both O_0 and O_1 are final
-    tc_fence_before();
-    const bool all_ok = bar_red_and(kSoftmaxBarrier, kSoftmaxThreads, ok && (n_t == 0 || have_o));
-    tc_fence_after();
-    if (!all_ok) record_abort(abort_flag, prm.status, kStatusTimeout);
-    const float m0 = red[row], m1 = red[kBM + row];
-    const float l0 = red[2 * kBM + row], l1 = red[3 * kBM + row];
-    const float M = fmaxf(m0, m1);
-    const float f0 = l0 > 0.f ? fast_exp2(m0 - M) : 0.f;
-    const float f1 = l1 > 0.f ? fast_exp2(m1 - M) : 0.f;
-    const float lt = f0 * l0 + f1 * l1;
-    const float inv_l = lt > 0.f ? 1.f / lt : 0.f;
-    const float g0 = f0 * inv_l, g1 = f1 * inv_l;
-    const bool write = row_valid && all_ok;
-    const int qrow = (qh ? r2 : r1) * 64 + (row & 63);
-    const int64_t grow = static_cast<int64_t>(bh) * prm.S + qrow;
-    // this thread writes d columns [half*D/2, half*D/2 + D/2) of its row
-    __nv_bfloat16* orow = prm.o + grow * D + half * (D / 2);
-    const bool read = all_ok && n_t > 0;
+    const bool write = row_valid && ok && (c == 0 || have_o);
+    const int64_t grow = static_cast<int64_t>(bh) * prm.S + static_cast<int64_t>(qblock) * 64 + (row & 63);
+    const float inv_l = l > 0.f ? 1.f / l : 0.f;
+    __nv_bfloat16* orow = prm.o + grow * D;
 #pragma unroll
-    for (int c = 0; c < D / 64; ++c) {
-      const uint32_t col = half * (D / 2) + c * 32;
-      uint32_t a[32], b2[32];
-      if (read) {
-        tmem_ld32(tmem + lane_off + kColO0 + col, a);
-        tmem_ld32(tmem + lane_off + kColO1 + col, b2);
+    for (int cc = 0; cc < D / 32; ++cc) {
+      uint32_t o[32];
+      if (have_o) {
+        tmem_ld32(o_base + cc * 32, o);
         tmem_ld_wait();
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) o[i] = 0u;
       }
       if (write) {
         uint32_t w[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          // a stream with l == 0 contributed nothing (its O may never have been written)
-          const float x0 = (g0 > 0.f ? __uint_as_float(a[2 * i]) * g0 : 0.f) +
-                           (g1 > 0.f ? __uint_as_float(b2[2 * i]) * g1 : 0.f);
-          const float x1 = (g0 > 0.f ? __uint_as_float(a[2 * i + 1]) * g0 : 0.f) +
-                           (g1 > 0.f ? __uint_as_float(b2[2 * i + 1]) * g1 : 0.f);
-          w[i] = pack_bf16x2(x0, x1);
-        }
-        uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+        for (int i = 0; i < 16; ++i)
+          w[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l);
+        uint4* dst = reinterpret_cast<uint4*>(orow + cc * 32);
 #pragma unroll
         for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
       }
     }
-    if (write && half == 0 && prm.lse != nullptr)
-      prm.lse[grow] = lt > 0.f ? (M + __log2f(lt)) * 0.69314718055994530942f : -INFINITY;
+    if (write && prm.lse != nullptr)
+      prm.lse[grow] = l > 0.f ? (m + __log2f(l)) * 0.69314718055994530942f : -INFINITY;
   }
 
   tc_fence_before();
@@ -639,8 +598,14 @@ template <int D>
 static cudaError_t launch_fwd_t(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
                                 const AttnParams& prm, int64_t nitems, cudaStream_t st) {
   constexpr uint32_t smem = AttnSmem<D>::kAlloc;
-  cudaError_t e = cudaFuncSetAttribute(bsa_fwd_kernel<D>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  static_assert(8 * kRegsSoftmax + 4 * kRegsOther <= 12 * kRegsLaunch, "register split");
+  cudaFuncAttributes attr;
+  cudaError_t e = cudaFuncGetAttributes(&attr, bsa_fwd_kernel<D>);
+  if (e != cudaSuccess) return e;
+  // the in-kernel register split assumes the launch allocation of kRegsLaunch
+  // registers per thread; anything less would make setmaxnreg.inc wait forever
+  if (attr.numRegs < kRegsLaunch) return cudaErrorInvalidConfiguration;
+  e = cudaFuncSetAttribute(bsa_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   bsa_fwd_kernel<D><<<static_cast<unsigned>(nitems), kThreads, smem, st>>>(q, k, v, prm);
   return cudaGetLastError();
@@ -659,10 +624,10 @@ cudaError_t launch_bsa_fwd(const CUtensorMap& q, const CUtensorMap& k, const CUt
   prm.H = H;
   prm.S = S;
   prm.nb = S / 64;
-  prm.npairs = (prm.nb + 1) / 2;
+  prm.ngroups = (prm.nb + 3) / 4;
   prm.scale_log2 = scale * 1.4426950408889634f;
   prm.wait_limit_ns = wait_limit_ns;
-  const int64_t nitems = static_cast<int64_t>(BH) * prm.npairs;
+  const int64_t nitems = static_cast<int64_t>(BH) * prm.ngroups;
   if (nitems == 0) return cudaSuccess;
   if (d == 128) return launch_fwd_t<128>(q, k, v, prm, nitems, st);
   return launch_fwd_t<64>(q, k, v, prm, nitems, st);
