@@ -20,9 +20,11 @@
 // {p > v*} plus the first tied entries (by block index) of value v*, where v*
 // is the largest probability whose "mass at or above" reaches 1 - thr; v* is
 // found by bisection on the fp32 bit pattern (order-preserving for p >= 0).
-// That is the same set a descending sort + cumulative sum selects, with the
-// partial sums taken in block order instead of sorted order (fp32 rounding of
-// those sums is the only difference).
+// That is the set a descending sort + cumulative sum selects, with the partial
+// sums taken in block order instead of sorted order.  Pooling and the reduced
+// map are fp64 (fp32 logits reorder blocks whose probabilities agree to a few
+// 1e-6, which moved cuts); the row softmax and the masses are fp32 values
+// from the fp64 map, summed in fp64 across each warp.
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 #include <cstdint>
@@ -85,41 +87,67 @@ __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restri
 // of 256 threads; each thread owns rows {2ty, 2ty+1} + 32i and columns
 // {2tx, 2tx+1} + 32j (i, j < 4), so its shared-memory reads are 16-byte
 // vectors that are broadcast (A) or contiguous across the half-warp (B).
-// k is staged in chunks of 16.  Every element is one fixed-order FMA chain.
+// k is staged in chunks of 16 through two shared-memory stages, the next
+// chunk's global loads in flight while the current one is multiplied.  Every
+// element is one fixed-order FMA chain.
 constexpr int kLgT = 128, kLgK = 16, kLgLD = kLgT + 2;
+constexpr int kLgBuf = kLgK * kLgLD;                       // doubles per operand buffer
+constexpr size_t kLgSmem = 2ull * 2 * kLgBuf * sizeof(double);   // 2 stages x (A, B)
 
 template <int D>
 __global__ void __launch_bounds__(256) logits_kernel(const double* __restrict__ qbar,
                                                      const double* __restrict__ kbar,
                                                      double* __restrict__ L, int nb,
                                                      double inv_sqrt_d) {
-  __shared__ __align__(16) double As[kLgK][kLgLD];   // As[k][m]
-  __shared__ __align__(16) double Bs[kLgK][kLgLD];   // Bs[k][n]
+  extern __shared__ double lg_smem[];   // [stage][A | B][kLgK][kLgLD]; As[k][m], Bs[k][n]
   const int bh = blockIdx.z;
   const int m0 = blockIdx.y * kLgT, n0 = blockIdx.x * kLgT;
   const double* qa = qbar + static_cast<int64_t>(bh) * nb * D;
   const double* ka = kbar + static_cast<int64_t>(bh) * nb * D;
   const int tid = threadIdx.x, ty = tid / 16, tx = tid % 16;
+  // each thread moves 8 elements of A and 8 of B per k-chunk; consecutive
+  // threads take consecutive k of one row (coalesced 128-byte rows)
+  double ra[8], rb[8];
+  auto fetch = [&](int kc) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int i = tid + j * 256, r = i / kLgK, kk = i % kLgK;
+      ra[j] = (m0 + r < nb) ? qa[static_cast<int64_t>(m0 + r) * D + kc + kk] : 0.0;
+      rb[j] = (n0 + r < nb) ? ka[static_cast<int64_t>(n0 + r) * D + kc + kk] : 0.0;
+    }
+  };
+  auto stash = [&](int st) {
+    double* As = lg_smem + st * 2 * kLgBuf;
+    double* Bs = As + kLgBuf;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int i = tid + j * 256, r = i / kLgK, kk = i % kLgK;
+      As[kk * kLgLD + r] = ra[j];
+      Bs[kk * kLgLD + r] = rb[j];
+    }
+  };
   double acc[8][8];
 #pragma unroll
   for (int i = 0; i < 8; ++i)
 #pragma unroll
     for (int j = 0; j < 8; ++j) acc[i][j] = 0.0;
-  for (int kc = 0; kc < D; kc += kLgK) {
-    __syncthreads();
-    for (int i = tid; i < kLgT * kLgK; i += 256) {
-      const int r = i / kLgK, kk = i % kLgK;   // consecutive threads: consecutive k (coalesced)
-      As[kk][r] = (m0 + r < nb) ? qa[static_cast<int64_t>(m0 + r) * D + kc + kk] : 0.0;
-      Bs[kk][r] = (n0 + r < nb) ? ka[static_cast<int64_t>(n0 + r) * D + kc + kk] : 0.0;
-    }
-    __syncthreads();
-#pragma unroll 4
+  fetch(0);
+  stash(0);
+  __syncthreads();
+  constexpr int kChunks = D / kLgK;
+#pragma unroll 1
+  for (int ch = 0; ch < kChunks; ++ch) {
+    const int st = ch & 1;
+    if (ch + 1 < kChunks) fetch((ch + 1) * kLgK);   // in flight during the FMAs below
+    const double* As = lg_smem + st * 2 * kLgBuf;
+    const double* Bs = As + kLgBuf;
+#pragma unroll
     for (int kk = 0; kk < kLgK; ++kk) {
       double a[8], b[8];
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const double2 va = *reinterpret_cast<const double2*>(&As[kk][2 * ty + 32 * i]);
-        const double2 vb = *reinterpret_cast<const double2*>(&Bs[kk][2 * tx + 32 * i]);
+        const double2 va = *reinterpret_cast<const double2*>(&As[kk * kLgLD + 2 * ty + 32 * i]);
+        const double2 vb = *reinterpret_cast<const double2*>(&Bs[kk * kLgLD + 2 * tx + 32 * i]);
         a[2 * i] = va.x; a[2 * i + 1] = va.y;
         b[2 * i] = vb.x; b[2 * i + 1] = vb.y;
       }
@@ -128,6 +156,8 @@ __global__ void __launch_bounds__(256) logits_kernel(const double* __restrict__ 
 #pragma unroll
         for (int j = 0; j < 8; ++j) acc[i][j] = fma(a[i], b[j], acc[i][j]);
     }
+    if (ch + 1 < kChunks) stash(st ^ 1);
+    __syncthreads();
   }
   double* out = L + static_cast<int64_t>(bh) * nb * nb;
 #pragma unroll
@@ -164,12 +194,16 @@ __device__ __forceinline__ uint32_t warp_max_u32(uint32_t v) {
   return v;
 }
 
-// fp64 mass of the entries whose ordering key is at least v.
-__device__ __forceinline__ double mass_at_or_above(const double* p, const uint32_t* key, int nb,
-                                                   int lane, uint32_t v) {
-  double s = 0.0;
-  for (int c = lane; c < nb; c += 32) s += (key[c] >= v) ? p[c] : 0.0;
-  return warp_sum(s);
+// Mass of the entries whose ordering key (fp32 bit pattern of p) is at least
+// v: fp32 sums per lane (at most 128 terms), fp64 across the warp.
+__device__ __forceinline__ double mass_at_or_above(const uint32_t* key, int nb, int lane,
+                                                   uint32_t v) {
+  float s = 0.f;
+  for (int c = lane; c < nb; c += 32) {
+    const uint32_t k = key[c];
+    s += (k >= v) ? __uint_as_float(k) : 0.f;
+  }
+  return warp_sum(static_cast<double>(s));
 }
 
 struct SelectParams {
@@ -178,47 +212,42 @@ struct SelectParams {
   int Tt, Th, Tw;
 };
 
-// One warp per row g = bh*nb + r; `wpc` warps per CTA.  Shared memory per warp:
-// p (fp64, nb) and its ordering key (nb x u32).  Softmax and every mass sum
-// are fp64.  Rows are ordered by the key = bit pattern of fp32(p), ties by
-// block index: entries whose fp64 probabilities differ by less than one fp32
-// ulp (relative 6e-8) are ordered by index.
+// One warp per row g = bh*nb + r; `wpc` warps per CTA; shared memory: one
+// 32-bit key per entry.  The reduced map arrives in fp64.  p = exp(L - max) / Z
+// is formed in fp32 from the fp64 difference (a few ulp), and its fp32 bit
+// pattern is the ordering key (order-preserving for p >= 0); equal keys go by
+// block index.  Masses are summed from those fp32 values, fp64 across the warp.
+// Relative to the fp64 rule this can move the cut only for rows whose cut
+// mass is within a few 1e-6 of 1 - thr, or swap blocks whose probabilities
+// agree to ~1e-7.
 __global__ void __launch_bounds__(256) select_kernel(const double* __restrict__ L, int64_t nrows,
                                                      int nb, int wpc, SelectParams prm,
                                                      uint32_t* __restrict__ bits,
                                                      int32_t* __restrict__ counts,
                                                      uint8_t* __restrict__ mask_u8) {
-  extern __shared__ double sel_smem[];
+  extern __shared__ uint32_t sel_keys[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t g = static_cast<int64_t>(blockIdx.x) * wpc + warp;
   if (g >= nrows) return;
   const int r = static_cast<int>(g % nb);
   const int nw = (nb + 31) >> 5;
-  double* p = sel_smem + static_cast<int64_t>(warp) * nb;
-  uint32_t* key = reinterpret_cast<uint32_t*>(sel_smem + static_cast<int64_t>(wpc) * nb) +
-                  static_cast<int64_t>(warp) * nb;
+  uint32_t* key = sel_keys + static_cast<int64_t>(warp) * nb;
   const double* Lrow = L + g * nb;
 
-  // softmax over the row (max subtracted), p = e / Z, all fp64
+  // softmax over the row (max subtracted in fp64)
   double mx = -INFINITY;
-  for (int c = lane; c < nb; c += 32) {
-    const double x = Lrow[c];
-    p[c] = x;
-    mx = fmax(mx, x);
-  }
+  for (int c = lane; c < nb; c += 32) mx = fmax(mx, Lrow[c]);
   mx = warp_max(mx);
-  double z = 0.0;
+  float zl = 0.f;
   for (int c = lane; c < nb; c += 32) {
-    const double e = exp(p[c] - mx);
-    p[c] = e;
-    z += e;
+    const float e = expf(static_cast<float>(Lrow[c] - mx));
+    key[c] = __float_as_uint(e);
+    zl += e;
   }
-  z = warp_sum(z);
+  const float z = static_cast<float>(warp_sum(static_cast<double>(zl)));
   uint32_t kmax = 0;
   for (int c = lane; c < nb; c += 32) {
-    const double v = p[c] / z;
-    p[c] = v;
-    const uint32_t kv = __float_as_uint(__double2float_rn(v));
+    const uint32_t kv = __float_as_uint(__uint_as_float(key[c]) / z);
     key[c] = kv;
     kmax = max(kmax, kv);
   }
@@ -234,22 +263,23 @@ __global__ void __launch_bounds__(256) select_kernel(const double* __restrict__ 
   uint32_t vstar = kmax;
   double above = 0.0;
   if (!keep_all && target > 0.0) {
-    const double total = mass_at_or_above(p, key, nb, lane, 0u);
+    const double total = mass_at_or_above(key, nb, lane, 0u);
     if (total < target) {
       keep_all = true;   // every exclusive prefix stays below the target
     } else {
       uint32_t lo = 0u, hi = kmax + 1u;   // mass(lo) >= target > mass(hi)
       while (hi - lo > 1u) {
         const uint32_t mid = lo + ((hi - lo) >> 1);
-        if (mass_at_or_above(p, key, nb, lane, mid) >= target) lo = mid; else hi = mid;
+        if (mass_at_or_above(key, nb, lane, mid) >= target) lo = mid; else hi = mid;
       }
       vstar = lo;
-      above = mass_at_or_above(p, key, nb, lane, vstar + 1u);   // < target
+      above = mass_at_or_above(key, nb, lane, vstar + 1u);   // < target
     }
   }
 
   // flags -> bitmap words, optional uint8 row, STA union, counts
   const int rt = r / (prm.Th * prm.Tw), rh = (r / prm.Tw) % prm.Th, rw = r % prm.Tw;
+  const double pstar = static_cast<double>(__uint_as_float(vstar));
   double carry = above;        // exclusive prefix mass before the next tied entry
   bool first_tied = true;      // no tied entry seen yet
   int count = 0;
@@ -264,18 +294,12 @@ __global__ void __launch_bounds__(256) select_kernel(const double* __restrict__ 
     } else {
       const uint32_t kv = inrow ? key[c] : 0u;
       const bool tied = inrow && kv == vstar;
-      const double pv = tied ? p[c] : 0.0;
-      double incl = pv;   // inclusive scan of tied masses across lanes (lane order)
-#pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const double y = __shfl_up_sync(0xffffffffu, incl, off);
-        if (lane >= off) incl += y;
-      }
       const uint32_t tb = __ballot_sync(0xffffffffu, tied);
-      const bool is_first = first_tied && tied && (tb & ((1u << lane) - 1u)) == 0u;
-      const double excl = carry + (incl - pv);
+      const int rank = __popc(tb & ((1u << lane) - 1u));   // tied entries before this one
+      const bool is_first = first_tied && tied && rank == 0;
+      const double excl = carry + rank * pstar;
       keep = inrow && (kv > vstar || (tied && (excl < target || (is_first && vstar == kmax))));
-      carry += __shfl_sync(0xffffffffu, incl, 31);
+      carry += __popc(tb) * pstar;
       if (tb) first_tied = false;
     }
     if (inrow && prm.use_sta) {
@@ -411,10 +435,18 @@ cudaError_t launch_logits(const double* qbar, const double* kbar, double* L, int
                           int d, cudaStream_t st) {
   const dim3 grid((nb + kLgT - 1) / kLgT, (nb + kLgT - 1) / kLgT, BH);
   const double inv = 1.0 / sqrt(static_cast<double>(d));
-  if (d == 128)
-    logits_kernel<128><<<grid, 256, 0, st>>>(qbar, kbar, L, nb, inv);
-  else
-    logits_kernel<64><<<grid, 256, 0, st>>>(qbar, kbar, L, nb, inv);
+  cudaError_t e;
+  if (d == 128) {
+    e = cudaFuncSetAttribute(logits_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(kLgSmem));
+    if (e != cudaSuccess) return e;
+    logits_kernel<128><<<grid, 256, kLgSmem, st>>>(qbar, kbar, L, nb, inv);
+  } else {
+    e = cudaFuncSetAttribute(logits_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(kLgSmem));
+    if (e != cudaSuccess) return e;
+    logits_kernel<64><<<grid, 256, kLgSmem, st>>>(qbar, kbar, L, nb, inv);
+  }
   return cudaGetLastError();
 }
 
@@ -422,7 +454,7 @@ cudaError_t launch_select(const double* L, int64_t nrows, int nb, float thr, int
                           int wh, int ww, int Tt, int Th, int Tw, uint32_t* bits, int32_t* counts,
                           uint8_t* mask_u8, cudaStream_t st) {
   SelectParams prm{thr, use_sta, wt, wh, ww, Tt, Th, Tw};
-  const size_t per_warp = static_cast<size_t>(nb) * (sizeof(double) + sizeof(uint32_t));
+  const size_t per_warp = static_cast<size_t>(nb) * sizeof(uint32_t);
   int wpc = static_cast<int>((200u * 1024u) / per_warp);
   wpc = wpc < 1 ? 1 : (wpc > 8 ? 8 : wpc);
   const size_t smem = per_warp * wpc;
