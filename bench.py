@@ -323,6 +323,24 @@ def run_ours(args):
     h2d = sum(t.numel() * t.element_size() for t in pinned)
     d2h = o_host.numel() * 2 + lse_host.numel() * 4
 
+    # token reordering (raster -> tile-major of one [B,H,S,d] tensor), timed on
+    # its own after the layer: algorithmic bytes = read + write of the tensor
+    qr = torch.empty_like(q)
+    for _ in range(3):
+        nl.nabla_reorder_tokens(q, w.tile_grid, nl.TO_TILE_MAJOR, out=qr)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n_re = 20
+    torch.cuda.synchronize()
+    a.record(stream)
+    for _ in range(n_re):
+        nl.nabla_reorder_tokens(q, w.tile_grid, nl.TO_TILE_MAJOR, out=qr)
+    b.record(stream)
+    torch.cuda.synchronize()
+    re_ms = a.elapsed_time(b) / n_re
+    re_bytes = 2.0 * q.numel() * q.element_size()
+    re_gbs = re_bytes / (re_ms * 1e-3) / 1e9
+    del qr
+
     attn_tflops = kept_flops / (attn_ms * 1e-3) / 1e12
     peak = peaks["bf16_tflops_sustained"]
     traffic = _traffic_per_launch()
@@ -352,6 +370,9 @@ def run_ours(args):
                           "bytes": mask_bytes},
         "e2e": {"value": e2e_val, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "reorder": {"bound": "hbm", "ms": re_ms, "achieved": re_gbs, "peak": peaks["hbm_gbs"],
+                    "unit": "GB/s", "frac": re_gbs / peaks["hbm_gbs"], "bytes": re_bytes,
+                    "what": "raster -> tile-major of one [B,H,S,d] bf16 tensor, outside the step"},
         "gpu_launches": 6 * args.steps,
         "clocks": clk,
     }

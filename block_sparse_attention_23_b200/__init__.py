@@ -31,7 +31,8 @@ OP_BUILD_MASK, OP_FWD, OP_FWD_WITH_MASK = 0, 1, 2
 EXPORTED = ["nabla_workspace_size", "nabla_workspace_init", "nabla_query_status",
             "nabla_build_mask", "bsa_fwd", "bsa_fwd_with_mask", "nabla_last_error",
             "nabla_version", "nabla_set_wait_limit_ns", "nabla_selftest_mma",
-            "bsa_fwd_with_mask_static"]
+            "bsa_fwd_with_mask_static", "nabla_reorder_tokens"]
+TO_TILE_MAJOR, TO_RASTER = 0, 1
 
 
 class NablaError(RuntimeError):
@@ -48,7 +49,7 @@ class _Shape(ctypes.Structure):
 
 class _MaskParams(ctypes.Structure):
     _fields_ = [("thr", ctypes.c_float), ("use_sta", ctypes.c_int32), ("wt", ctypes.c_int32),
-                ("wh", ctypes.c_int32), ("ww", ctypes.c_int32)]
+                ("wh", ctypes.c_int32), ("ww", ctypes.c_int32), ("topk", ctypes.c_int32)]
 
 
 _lock = threading.Lock()
@@ -93,6 +94,8 @@ def lib() -> ctypes.CDLL:
             L.nabla_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
             L.nabla_selftest_mma.restype = i32
             L.nabla_selftest_mma.argtypes = [i32, vp, vp, vp, vp, vp]
+            L.nabla_reorder_tokens.restype = i32
+            L.nabla_reorder_tokens.argtypes = [sp, i32, vp, vp, vp]
             L.bsa_fwd_with_mask_static.restype = i32
             L.bsa_fwd_with_mask_static.argtypes = [sp, vp, vp, vp, vp, f32, vp, vp, vp, vp]
             _lib = L
@@ -171,8 +174,9 @@ def _bf16_contig(*ts):
 
 def nabla_build_mask(q, k, tile_grid, thr: float, sta: Optional[Tuple[int, int, int]] = None,
                      want_mask: bool = False, col_capacity: Optional[int] = None,
-                     workspace: Optional[Workspace] = None, out=None, stream=None):
-    """NABLA block mask of (q, k) as block CSR.
+                     workspace: Optional[Workspace] = None, out=None, stream=None,
+                     topk: int = 0):
+    """NABLA block mask of (q, k) as block CSR (``topk`` > 0: fixed top-k rule).
 
     Returns (row_ptr int32 [B*H*nb+1], col_idx int32 [capacity], nnz int32 [1],
     mask uint8 [B,H,nb,nb] or None).  Only the first nnz entries of col_idx
@@ -193,7 +197,8 @@ def nabla_build_mask(q, k, tile_grid, thr: float, sta: Optional[Tuple[int, int, 
     else:
         row_ptr, col_idx, nnz, mask = out
         cap = col_idx.numel() if col_capacity is None else col_capacity
-    prm = _MaskParams(float(thr), 1 if sta is not None else 0, *(sta if sta is not None else (0, 0, 0)))
+    prm = _MaskParams(float(thr), 1 if sta is not None else 0,
+                      *(sta if sta is not None else (0, 0, 0)), int(topk))
     _check(lib().nabla_build_mask(ctypes.byref(shape), ctypes.byref(prm), _ptr(q), _ptr(k),
                                   _ptr(mask), _ptr(row_ptr), _ptr(col_idx), int(cap), _ptr(nnz),
                                   _ptr(workspace.buf), _stream(stream)))
@@ -276,3 +281,15 @@ def bsa_fwd_with_mask_static(q, k, v, mask_u8, scale: Optional[float] = None, ou
                                           _ptr(mask_u8), float(scale or 0.0), _ptr(o), _ptr(lse),
                                           _ptr(status_out), _stream(stream)))
     return o, lse
+
+
+def nabla_reorder_tokens(x, tile_grid, direction: int = TO_TILE_MAJOR, out=None, stream=None):
+    """Permute the token axis of a [B,H,S,d] bf16 tensor between raster (t,h,w)
+    order and tile-major order (4x4x4 tiles, one per 64-token block)."""
+    torch = _torch()
+    _bf16_contig(x)
+    shape = _shape_of(x, tile_grid)
+    y = torch.empty_like(x) if out is None else out
+    _check(lib().nabla_reorder_tokens(ctypes.byref(shape), int(direction), _ptr(x), _ptr(y),
+                                      _stream(stream)))
+    return y

@@ -10,7 +10,7 @@
 // Kernels (all stream-ordered, no host synchronisation):
 //   pool_kernel        Q, K bf16 [BH,S,d] -> Qbar, Kbar fp32 [BH,nb,d]     HBM-bound
 //   logits_kernel      per head Qbar Kbar^T / sqrt(d) -> L fp32 [BH,nb,nb] fp32 FFMA
-//   select_kernel      one warp per row: softmax, prefix selection, STA OR ->
+//   select_kernel      one warp per row: softmax, prefix (or top-k) selection, STA OR ->
 //                      keep bitmap [BH*nb, nw] + counts (+ optional uint8 mask)
 //   mask_bits_kernel   external uint8 mask -> keep bitmap + counts
 //   scan_kernel        counts -> row_ptr (exclusive scan), nnz, capacity check
@@ -206,10 +206,20 @@ __device__ __forceinline__ double mass_at_or_above(const uint32_t* key, int nb, 
   return warp_sum(static_cast<double>(s));
 }
 
+// Entries whose ordering key is at least v.
+__device__ __forceinline__ int count_at_or_above(const uint32_t* key, int nb, int lane, uint32_t v) {
+  int n = 0;
+  for (int c = lane; c < nb; c += 32) n += key[c] >= v;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) n += __shfl_xor_sync(0xffffffffu, n, off);
+  return n;
+}
+
 struct SelectParams {
   float thr;
   int use_sta, wt, wh, ww;
   int Tt, Th, Tw;
+  int topk;        // > 0: keep the topk most probable blocks instead of the mass rule
 };
 
 // One warp per row g = bh*nb + r; `wpc` warps per CTA; shared memory: one
@@ -259,10 +269,21 @@ __global__ void __launch_bounds__(256) select_kernel(const double* __restrict__ 
   // the exclusive prefix mass stays below the target.  The first entry of the
   // sorted row is always kept.
   const double target = 1.0 - static_cast<double>(prm.thr);
-  bool keep_all = prm.thr <= 0.f;
+  const bool topk_mode = prm.topk > 0;
+  bool keep_all = topk_mode ? prm.topk >= nb : prm.thr <= 0.f;
   uint32_t vstar = kmax;
   double above = 0.0;
-  if (!keep_all && target > 0.0) {
+  int tied_quota = 0;          // top-k: tied entries kept, in block order
+  if (topk_mode && !keep_all) {
+    // v*: largest key with at least topk entries at or above it
+    uint32_t lo = 0u, hi = kmax + 1u;   // count(lo) = nb >= topk > count(hi) = 0
+    while (hi - lo > 1u) {
+      const uint32_t mid = lo + ((hi - lo) >> 1);
+      if (count_at_or_above(key, nb, lane, mid) >= prm.topk) lo = mid; else hi = mid;
+    }
+    vstar = lo;
+    tied_quota = prm.topk - count_at_or_above(key, nb, lane, vstar + 1u);
+  } else if (!keep_all && target > 0.0) {
     const double total = mass_at_or_above(key, nb, lane, 0u);
     if (total < target) {
       keep_all = true;   // every exclusive prefix stays below the target
@@ -282,6 +303,7 @@ __global__ void __launch_bounds__(256) select_kernel(const double* __restrict__ 
   const double pstar = static_cast<double>(__uint_as_float(vstar));
   double carry = above;        // exclusive prefix mass before the next tied entry
   bool first_tied = true;      // no tied entry seen yet
+  int tied_seen = 0;
   int count = 0;
   uint32_t* brow = bits + g * nw;
   uint8_t* mrow = mask_u8 ? mask_u8 + g * nb : nullptr;
@@ -298,8 +320,12 @@ __global__ void __launch_bounds__(256) select_kernel(const double* __restrict__ 
       const int rank = __popc(tb & ((1u << lane) - 1u));   // tied entries before this one
       const bool is_first = first_tied && tied && rank == 0;
       const double excl = carry + rank * pstar;
-      keep = inrow && (kv > vstar || (tied && (excl < target || (is_first && vstar == kmax))));
+      if (topk_mode)
+        keep = inrow && (kv > vstar || (tied && tied_seen + rank < tied_quota));
+      else
+        keep = inrow && (kv > vstar || (tied && (excl < target || (is_first && vstar == kmax))));
       carry += __popc(tb) * pstar;
+      tied_seen += __popc(tb);
       if (tb) first_tied = false;
     }
     if (inrow && prm.use_sta) {
@@ -450,10 +476,10 @@ cudaError_t launch_logits(const double* qbar, const double* kbar, double* L, int
   return cudaGetLastError();
 }
 
-cudaError_t launch_select(const double* L, int64_t nrows, int nb, float thr, int use_sta, int wt,
-                          int wh, int ww, int Tt, int Th, int Tw, uint32_t* bits, int32_t* counts,
-                          uint8_t* mask_u8, cudaStream_t st) {
-  SelectParams prm{thr, use_sta, wt, wh, ww, Tt, Th, Tw};
+cudaError_t launch_select(const double* L, int64_t nrows, int nb, float thr, int topk,
+                          int use_sta, int wt, int wh, int ww, int Tt, int Th, int Tw,
+                          uint32_t* bits, int32_t* counts, uint8_t* mask_u8, cudaStream_t st) {
+  SelectParams prm{thr, use_sta, wt, wh, ww, Tt, Th, Tw, topk};
   const size_t per_warp = static_cast<size_t>(nb) * sizeof(uint32_t);
   int wpc = static_cast<int>((200u * 1024u) / per_warp);
   wpc = wpc < 1 ? 1 : (wpc > 8 ? 8 : wpc);

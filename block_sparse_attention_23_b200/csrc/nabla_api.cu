@@ -20,9 +20,9 @@ cudaError_t launch_pool(const void* q, const void* k, double* qbar, double* kbar
                         int64_t nblocks, int d, cudaStream_t st);
 cudaError_t launch_logits(const double* qbar, const double* kbar, double* L, int BH, int nb,
                           int d, cudaStream_t st);
-cudaError_t launch_select(const double* L, int64_t nrows, int nb, float thr, int use_sta, int wt,
-                          int wh, int ww, int Tt, int Th, int Tw, uint32_t* bits, int32_t* counts,
-                          uint8_t* mask_u8, cudaStream_t st);
+cudaError_t launch_select(const double* L, int64_t nrows, int nb, float thr, int topk,
+                          int use_sta, int wt, int wh, int ww, int Tt, int Th, int Tw,
+                          uint32_t* bits, int32_t* counts, uint8_t* mask_u8, cudaStream_t st);
 cudaError_t launch_mask_bits(const uint8_t* mask, int64_t nrows, int nb, uint32_t* bits,
                              int32_t* counts, cudaStream_t st);
 cudaError_t launch_scan_fill(const uint32_t* bits, const int32_t* counts, int64_t nrows, int nb,
@@ -32,6 +32,8 @@ cudaError_t launch_bsa_fwd(const CUtensorMap& q, const CUtensorMap& k, const CUt
                            const int32_t* row_ptr, const int32_t* col_idx, void* o, float* lse,
                            int* status, int BH, int H, int S, int d, float scale,
                            uint64_t wait_limit_ns, cudaStream_t st);
+cudaError_t launch_reorder(const void* src, void* dst, int64_t BH, int Tt, int Th, int Tw,
+                           int row_bytes, int to_tile_major, cudaStream_t st);
 cudaError_t launch_mma_selftest(const CUtensorMap& a, const CUtensorMap& b, const void* a_glob,
                                 float* c, int variant, int* status, uint64_t lim,
                                 cudaStream_t st);
@@ -174,7 +176,7 @@ void set_last_error(const std::string& msg) { g_last_error = msg; }
 
 extern "C" {
 
-int nabla_version(void) { return 100; }
+int nabla_version(void) { return 200; }
 
 const char* nabla_last_error(void) { return g_last_error.c_str(); }
 
@@ -224,6 +226,7 @@ nabla_status nabla_build_mask(const nabla_shape* shape, const nabla_mask_params*
   if (params == nullptr) return fail(NABLA_ERR_INVALID_ARG, "params is NULL");
   if (!(params->thr >= 0.f && params->thr <= 1.f))
     return fail(NABLA_ERR_UNSUPPORTED, "thr must lie in [0, 1]");
+  if (params->topk < 0) return fail(NABLA_ERR_INVALID_ARG, "topk must be >= 0");
   if (params->use_sta && (params->wt < 0 || params->wh < 0 || params->ww < 0))
     return fail(NABLA_ERR_INVALID_ARG, "STA half-windows must be non-negative");
   if (shape->Tt <= 0 || shape->Th <= 0 || shape->Tw <= 0 ||
@@ -248,9 +251,9 @@ nabla_status nabla_build_mask(const nabla_shape* shape, const nabla_mask_params*
   if (e != cudaSuccess) return cuda_fail(e, "pool launch");
   e = nabla::launch_logits(qbar, kbar, L, BH, nb, shape->d, st);
   if (e != cudaSuccess) return cuda_fail(e, "logits launch");
-  e = nabla::launch_select(L, nrows, nb, params->thr, params->use_sta ? 1 : 0, params->wt,
-                           params->wh, params->ww, shape->Tt, shape->Th, shape->Tw, bits, counts,
-                           mask_u8, st);
+  e = nabla::launch_select(L, nrows, nb, params->thr, params->topk, params->use_sta ? 1 : 0,
+                           params->wt, params->wh, params->ww, shape->Tt, shape->Th, shape->Tw,
+                           bits, counts, mask_u8, st);
   if (e != cudaSuccess) return cuda_fail(e, "select launch");
   e = nabla::launch_scan_fill(bits, counts, nrows, nb, row_ptr, col_idx, col_capacity, nnz_out,
                               status_ptr(workspace), st);
@@ -299,6 +302,30 @@ nabla_status bsa_fwd_with_mask(const nabla_shape* shape, const void* q, const vo
                               status_ptr(workspace), st);
   if (e != cudaSuccess) return cuda_fail(e, "scan/fill launch");
   return run_fwd(shape, q, k, v, row_ptr, col_idx, scale, o, lse, workspace, st);
+}
+
+nabla_status nabla_reorder_tokens(const nabla_shape* shape, int direction, const void* src,
+                                  void* dst, nabla_stream_t stream) {
+  if (shape == nullptr) return fail(NABLA_ERR_INVALID_ARG, "shape is NULL");
+  if (shape->B <= 0 || shape->H <= 0 || shape->d <= 0 || shape->Tt <= 0 || shape->Th <= 0 ||
+      shape->Tw <= 0)
+    return fail(NABLA_ERR_INVALID_ARG, "B, H, d and the tile grid must be positive");
+  if (static_cast<int64_t>(shape->Tt) * shape->Th * shape->Tw * 64 != shape->S)
+    return fail(NABLA_ERR_INVALID_ARG, "S must equal 64*Tt*Th*Tw");
+  if ((shape->d * 2) % 16 != 0) return fail(NABLA_ERR_UNSUPPORTED, "d must be a multiple of 8");
+  if (direction != NABLA_TO_TILE_MAJOR && direction != NABLA_TO_RASTER)
+    return fail(NABLA_ERR_INVALID_ARG, "unknown direction");
+  if (!src || !dst) return fail(NABLA_ERR_INVALID_ARG, "null pointer");
+  if (src == dst) return fail(NABLA_ERR_INVALID_ARG, "src and dst must not alias");
+  if (!aligned16(src) || !aligned16(dst)) return fail(NABLA_ERR_INVALID_ARG, "src, dst need 16-byte alignment");
+  const int64_t BH = static_cast<int64_t>(shape->B) * shape->H;
+  if (BH * shape->Tt * shape->Th * shape->Tw >= (static_cast<int64_t>(1) << 31))
+    return fail(NABLA_ERR_UNSUPPORTED, "B*H*S/64 must stay below 2^31");
+  cudaError_t e = nabla::launch_reorder(src, dst, BH, shape->Tt, shape->Th, shape->Tw,
+                                        shape->d * 2, direction == NABLA_TO_TILE_MAJOR ? 1 : 0,
+                                        reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "reorder launch");
+  return NABLA_OK;
 }
 
 nabla_status nabla_selftest_mma(int variant, const void* a, const void* b, float* c,

@@ -64,6 +64,8 @@ typedef struct {
     float thr;            /* keep the smallest sorted prefix with mass >= 1 - thr; thr in [0, 1] */
     int32_t use_sta;      /* nonzero: OR in the sliding-tile window below */
     int32_t wt, wh, ww;   /* STA half-window in tiles along t, h, w (>= 0) */
+    int32_t topk;         /* > 0: keep the topk most probable blocks per row instead of the
+                             mass rule (thr is then ignored); 0: mass rule */
 } nabla_mask_params;
 
 enum {
@@ -95,6 +97,9 @@ NABLA_API nabla_status nabla_query_status(void* workspace, nabla_stream_t stream
  * top block is always kept).  With use_sta, OR in the sliding-tile window of
  * "Sliding Tile Attention" (clipped at the grid edge).  The result is written
  * as block CSR with ascending column indices per row.
+ * With params->topk > 0 the row keeps instead its topk most probable blocks
+ * (same order and ties), the fixed-budget baseline the NABLA paper's
+ * Appendix C compares the mass rule with.
  *
  *   q, k          device bf16 [B,H,S,d]
  *   mask_u8       optional device uint8 [B,H,nb,nb] (1 = kept), or NULL
@@ -176,6 +181,23 @@ NABLA_API nabla_status bsa_fwd_with_mask_static(const nabla_shape* shape, const 
                                                 const uint8_t* mask_u8, float scale, void* o,
                                                 float* lse, int32_t* status_out,
                                                 nabla_stream_t stream);
+
+/*
+ * Token reordering between raster and tile-major order (the neighbourhood
+ * reorder of "NABLA: Neighborhood Adaptive Block-Level Attention", review
+ * Figure 4, with 4x4x4 tiles: each 64-token attention block becomes one tile
+ * of the T x H x W = 4Tt x 4Th x 4Tw token grid).
+ *   raster      s_r = (t*H + h)*W + w
+ *   tile-major  s_m = ((tt*Th + th)*Tw + tw)*64 + (ut*4 + uh)*4 + uw,
+ *               t = 4tt + ut, h = 4th + uh, w = 4tw + uw
+ * NABLA_TO_TILE_MAJOR moves token s_r of src to s_m of dst; NABLA_TO_RASTER is
+ * the inverse (for O after attention).  src, dst: device [B,H,S,d] rows of d
+ * 16-bit elements (bf16), 16-byte aligned, not aliasing; S = 64*Tt*Th*Tw;
+ * d a multiple of 8.  Stream-ordered; no workspace.
+ */
+enum { NABLA_TO_TILE_MAJOR = 0, NABLA_TO_RASTER = 1 };
+NABLA_API nabla_status nabla_reorder_tokens(const nabla_shape* shape, int direction,
+                                            const void* src, void* dst, nabla_stream_t stream);
 
 /* Message for the last error returned on the calling host thread. */
 NABLA_API const char* nabla_last_error(void);

@@ -63,12 +63,16 @@ def _load():
             lib.oracle_sta_or.argtypes = [vp, i32, i32, i32, i32, i32, i32, i32]
             lib.oracle_build_mask.restype = None
             lib.oracle_build_mask.argtypes = [vp, vp, i64, i64, i32, i32, i32, i32, f64, i32,
-                                              i32, i32, i32, vp, vp, vp]
+                                              i32, i32, i32, i32, vp, vp, vp]
+            lib.oracle_row_select_topk.restype = i32
+            lib.oracle_row_select_topk.argtypes = [vp, i32, i32, vp, vp]
             lib.oracle_masked_attention.restype = None
             lib.oracle_masked_attention.argtypes = [vp, vp, vp, i64, i64, i32, vp, f64, i64, vp,
                                                     vp, vp]
             lib.oracle_dense_attention.restype = None
             lib.oracle_dense_attention.argtypes = [vp, vp, vp, i64, i64, i32, f64, i64, vp, vp, vp]
+            lib.oracle_reorder.restype = None
+            lib.oracle_reorder.argtypes = [vp, vp, i64, i32, i32, i32, i32, i32]
             lib.oracle_max_threads.restype = i32
             lib.oracle_max_threads.argtypes = []
             _lib = lib
@@ -125,6 +129,14 @@ def row_select(p: np.ndarray, thr: float):
     return keep, int(cnt), diag
 
 
+def row_select_topk(p: np.ndarray, k: int):
+    """Fixed top-k selection of one probability row -> (keep uint8[n], count)."""
+    p = np.ascontiguousarray(p, dtype=np.float64)
+    keep = np.empty(p.shape[0], dtype=np.uint8)
+    cnt = _load().oracle_row_select_topk(p.ctypes.data, p.shape[0], int(k), keep.ctypes.data, None)
+    return keep, int(cnt)
+
+
 def sta_row(r: int, tile_grid, window) -> np.ndarray:
     """The clipped sliding-tile window of query tile r, as a uint8 row."""
     Tt, Th, Tw = tile_grid
@@ -134,8 +146,9 @@ def sta_row(r: int, tile_grid, window) -> np.ndarray:
 
 
 def build_mask(q: np.ndarray, k: np.ndarray, tile_grid, thr: float, sta=None,
-               with_diag: bool = False):
-    """q, k: [B,H,S,d] bf16 bits -> mask [B,H,nb,nb] uint8 (and diagnostics)."""
+               with_diag: bool = False, topk: int = 0):
+    """q, k: [B,H,S,d] bf16 bits -> mask [B,H,nb,nb] uint8 (and diagnostics).
+    topk > 0 uses the fixed top-k rule instead of the mass rule."""
     q, k = _u16(q), _u16(k)
     B, H, S, d = q.shape
     nb = S // BLOCK
@@ -146,8 +159,8 @@ def build_mask(q: np.ndarray, k: np.ndarray, tile_grid, thr: float, sta=None,
     wt, wh, ww = sta if use_sta else (0, 0, 0)
     Tt, Th, Tw = tile_grid
     _load().oracle_build_mask(q.ctypes.data, k.ctypes.data, B * H, S, d, Tt, Th, Tw, float(thr),
-                              1 if use_sta else 0, wt, wh, ww, mask.ctypes.data, diag.ctypes.data,
-                              counts.ctypes.data)
+                              int(topk), 1 if use_sta else 0, wt, wh, ww, mask.ctypes.data,
+                              diag.ctypes.data, counts.ctypes.data)
     if with_diag:
         return mask, diag, counts
     return mask
@@ -187,6 +200,21 @@ def dense_attention(q, k, v, rows=None, scale=None):
                                    float(scale), rows.shape[0], rows.ctypes.data, O.ctypes.data,
                                    lse.ctypes.data)
     return O, lse
+
+
+def reorder(x: np.ndarray, tile_grid, to_tile_major: bool = True) -> np.ndarray:
+    """[..., S, d] 16-bit rows -> the same rows moved between raster (t,h,w)
+    order and tile-major order (4x4x4 tiles)."""
+    x = _u16(x)
+    S, d = x.shape[-2], x.shape[-1]
+    Tt, Th, Tw = tile_grid
+    if S != 64 * Tt * Th * Tw:
+        raise ValueError("S must equal 64*Tt*Th*Tw")
+    BH = int(np.prod(x.shape[:-2])) if x.ndim > 2 else 1
+    out = np.empty_like(x)
+    _load().oracle_reorder(x.ctypes.data, out.ctypes.data, BH, Tt, Th, Tw, d,
+                           1 if to_tile_major else 0)
+    return out
 
 
 def near_cut_rows(diag: np.ndarray, thr: float, band: float = 1e-4) -> np.ndarray:

@@ -123,6 +123,25 @@ int oracle_row_select(const double* p, int n, double thr, uint8_t* keep, double*
     return count;
 }
 
+/* Fixed-budget baseline (NABLA review, "What carries the argument": Appendix C
+ * compares the mass rule with keeping a fixed Top-k of blocks per row): keep
+ * the k entries that come first in the descending order (ties: lower block
+ * index).  Returns the kept count, min(k, n). */
+int oracle_row_select_topk(const double* p, int n, int k, uint8_t* keep, double* diag) {
+    pv_t* v = (pv_t*)malloc(sizeof(pv_t) * (size_t)n);
+    for (int c = 0; c < n; ++c) { v[c].p = p[c]; v[c].idx = c; keep[c] = 0; }
+    qsort(v, (size_t)n, sizeof(pv_t), cmp_desc);
+    int count = 0;
+    for (int j = 0; j < n && j < k; ++j) { keep[v[j].idx] = 1; ++count; }
+    if (diag) {   /* no mass cut; probabilities at the last kept and first dropped position */
+        diag[0] = diag[1] = -1.0;
+        diag[2] = v[count - 1].p;
+        diag[3] = (count < n) ? v[count].p : -1.0;
+    }
+    free(v);
+    return count;
+}
+
 /* OR the sliding-tile window of query tile r into one mask row (tile
  * coordinates; the window is clipped to the grid). */
 void oracle_sta_or(uint8_t* row, int r, int Tt, int Th, int Tw, int wt, int wh, int ww) {
@@ -134,11 +153,12 @@ void oracle_sta_or(uint8_t* row, int r, int Tt, int Th, int Tw, int wt, int wh, 
 }
 
 /* Full mask builder: q, k [BH, S, d] bf16 bits -> mask [BH, nb, nb] uint8.
+ * topk > 0 selects the fixed top-k rule in place of the mass rule.
  * diag (may be NULL): [BH, nb, 4] as in oracle_row_select (before the STA OR).
  * adaptive_counts (may be NULL): [BH, nb] kept count before the STA OR. */
 void oracle_build_mask(const uint16_t* q, const uint16_t* k, int64_t BH, int64_t S, int d,
-                       int Tt, int Th, int Tw, double thr, int use_sta, int wt, int wh, int ww,
-                       uint8_t* mask, double* diag, int32_t* adaptive_counts) {
+                       int Tt, int Th, int Tw, double thr, int topk, int use_sta, int wt, int wh,
+                       int ww, uint8_t* mask, double* diag, int32_t* adaptive_counts) {
     int nb = (int)(S / ORACLE_BLOCK);
 #pragma omp parallel for schedule(dynamic, 1)
     for (int64_t bh = 0; bh < BH; ++bh) {
@@ -152,7 +172,12 @@ void oracle_build_mask(const uint16_t* q, const uint16_t* k, int64_t BH, int64_t
         for (int r = 0; r < nb; ++r) {
             uint8_t* row = mask + (bh * nb + r) * (int64_t)nb;
             oracle_softmax_row(L + (int64_t)r * nb, nb, P);
-            int cnt = oracle_row_select(P, nb, thr, row, diag ? diag + (bh * nb + r) * 4 : NULL);
+            int cnt;
+            if (topk > 0) {
+                cnt = oracle_row_select_topk(P, nb, topk, row, diag ? diag + (bh * nb + r) * 4 : NULL);
+            } else {
+                cnt = oracle_row_select(P, nb, thr, row, diag ? diag + (bh * nb + r) * 4 : NULL);
+            }
             if (adaptive_counts) adaptive_counts[bh * nb + r] = cnt;
             if (use_sta) oracle_sta_or(row, r, Tt, Th, Tw, wt, wh, ww);
         }
@@ -237,6 +262,31 @@ void oracle_dense_attention(const uint16_t* q, const uint16_t* k, const uint16_t
         LSE[n] = m + log(l);
         free(s);
     }
+}
+
+/* Token reordering (NABLA review, Figure 4: neighbouring tokens are gathered
+ * so that each attention block is one spatial-temporal patch; here the patch
+ * is the 4x4x4 tile).  For every token (t, h, w) of the 4Tt x 4Th x 4Tw grid:
+ * raster position (t*H + h)*W + w, tile-major position
+ * ((t/4*Th + h/4)*Tw + w/4)*64 + ((t%4)*4 + h%4)*4 + w%4.
+ * to_tile_major = 1 moves raster rows to tile-major rows, 0 the reverse.
+ * src, dst: [BH, S, d] 16-bit rows (copied bit for bit). */
+void oracle_reorder(const uint16_t* src, uint16_t* dst, int64_t BH, int Tt, int Th, int Tw, int d,
+                    int to_tile_major) {
+    const int64_t T = 4 * (int64_t)Tt, H = 4 * (int64_t)Th, W = 4 * (int64_t)Tw;
+    const int64_t S = T * H * W;
+    for (int64_t bh = 0; bh < BH; ++bh)
+        for (int64_t t = 0; t < T; ++t)
+            for (int64_t h = 0; h < H; ++h)
+                for (int64_t w = 0; w < W; ++w) {
+                    int64_t raster = (t * H + h) * W + w;
+                    int64_t tile = ((t / 4) * Th + h / 4) * Tw + w / 4;
+                    int64_t major = tile * 64 + ((t % 4) * 4 + h % 4) * 4 + w % 4;
+                    int64_t from = to_tile_major ? raster : major;
+                    int64_t to = to_tile_major ? major : raster;
+                    memcpy(dst + (bh * S + to) * d, src + (bh * S + from) * d,
+                           (size_t)d * sizeof(uint16_t));
+                }
 }
 
 /* Threads OpenMP will use (for reporting the CPU baseline's core count). */

@@ -118,3 +118,31 @@ def test_package_does_not_import_oracle():
                 text = open(os.path.join(dirpath, f)).read()
                 assert "import oracle" not in text and "from oracle" not in text, f
                 assert "nabla_oracle" not in text, f
+
+
+def test_topk_argument_checked(nl):
+    lib = nl.lib()
+    null = ctypes.c_void_p(0)
+    a = ctypes.c_void_p(1 << 20)
+    s = nl.make_shape(1, 1, 128, 64, (1, 1, 2))
+    prm = nl._MaskParams(0.2, 0, 0, 0, 0, -3)
+    assert lib.nabla_build_mask(ctypes.byref(s), ctypes.byref(prm), a, a, null, a, a, 4, null, a,
+                                null) == 1
+    assert lib.nabla_version() >= 200
+
+
+def test_reorder_arguments_checked(nl):
+    lib = nl.lib()
+    null = ctypes.c_void_p(0)
+    a, b = ctypes.c_void_p(1 << 20), ctypes.c_void_p(1 << 21)
+    good = nl.make_shape(1, 2, 128, 64, (1, 1, 2))
+    bad_s = nl.make_shape(1, 2, 192, 64, (1, 1, 2))
+    bad_d = nl.make_shape(1, 2, 128, 60, (1, 1, 2))
+    f = lib.nabla_reorder_tokens
+    assert f(None, 0, a, b, null) == 1
+    assert f(ctypes.byref(bad_s), 0, a, b, null) == 1
+    assert f(ctypes.byref(bad_d), 0, a, b, null) == 2
+    assert f(ctypes.byref(good), 7, a, b, null) == 1
+    assert f(ctypes.byref(good), 0, null, b, null) == 1
+    assert f(ctypes.byref(good), 0, a, a, null) == 1
+    assert f(ctypes.byref(good), 1, ctypes.c_void_p((1 << 20) + 8), b, null) == 1

@@ -103,3 +103,21 @@ def test_mask_capacity_overflow_reported(nl, synth_mod):
     row_ptr, col_idx, nnz, gmask, st = _gpu_mask(nl, q, k, w.tile_grid, 0.2, None, cap=5)
     assert st == 3   # NABLA_ERR_CAPACITY; row_ptr stays exact
     assert nnz == int(gmask.sum()) == row_ptr[-1]
+
+
+@pytest.mark.parametrize("name,topk", [("tiny", 3), ("small", 1), ("small", 17), ("small", 200),
+                                       ("hunyuan720p", 300)])
+def test_topk_mask_parity(nl, oracle_mod, synth_mod, name, topk):
+    """Fixed top-k rule: the same kept sets as the oracle's (rows whose k-th and
+    (k+1)-th probabilities tie to 1e-6 may swap one block)."""
+    w = synth_mod.WORKLOADS[name]
+    q, k, _ = synth_mod.make_qkv(w)
+    qd, kd = to_device_bf16(q), to_device_bf16(k)
+    row_ptr, col_idx, nnz, mask = nl.nabla_build_mask(qd, kd, w.tile_grid, w.thr, w.sta,
+                                                      want_mask=True, topk=topk)
+    gmask = mask.cpu().numpy()
+    omask, diag, _ = oracle_mod.build_mask(q, k, w.tile_grid, w.thr, w.sta, with_diag=True,
+                                           topk=topk)
+    compare_masks(gmask, omask, diag, w.thr)
+    if w.sta is None:
+        assert (gmask.sum(-1) == min(topk, w.nb)).all()

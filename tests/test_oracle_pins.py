@@ -346,3 +346,115 @@ def test_thr0_mask_reproduces_full_attention(oracle_mod, synth_mod):
     O2, l2 = oracle_mod.dense_attention(q, k, v, rows)
     np.testing.assert_allclose(O1, O2, atol=1e-13, rtol=0)
     np.testing.assert_allclose(l1, l2, atol=1e-13, rtol=0)
+
+
+# ---------------------------------------------------------------- fixed top-k rule
+
+def test_topk_keeps_k_largest_with_lower_index_ties(oracle_mod):
+    rng = np.random.default_rng(11)
+    for trial in range(200):
+        n = int(rng.integers(1, 200))
+        k = int(rng.integers(1, n + 5))
+        p = rng.dirichlet(np.full(n, 0.5))
+        if trial % 5 == 0:                      # force ties
+            p = np.round(p * 8) / 8
+        keep, cnt = oracle_mod.row_select_topk(p, k)
+        assert cnt == min(k, n) == keep.sum()
+        order = sorted(range(n), key=lambda c: (-p[c], c))   # independent ordering
+        assert set(np.nonzero(keep)[0]) == set(order[:min(k, n)])
+
+
+def test_topk_matches_mass_rule_at_its_own_count(oracle_mod):
+    """At k = the mass rule's kept count both rules keep the same blocks."""
+    rng = np.random.default_rng(12)
+    for _ in range(100):
+        p = rng.dirichlet(np.full(int(rng.integers(2, 120)), 0.3))
+        keep_m, cnt, _ = oracle_mod.row_select(p, 0.3)
+        keep_t, cnt_t = oracle_mod.row_select_topk(p, cnt)
+        assert cnt_t == cnt and np.array_equal(keep_m, keep_t)
+
+
+def test_topk_geometric_pipeline(oracle_mod):
+    nb, d, delta = 32, 64, 0.125
+    x = np.zeros((nb * 64, d), dtype=np.float32)
+    x[:, 0] = 8.0
+    y = np.zeros((nb * 64, d), dtype=np.float32)
+    y[:, 0] = np.repeat(-delta * np.arange(nb), 64)
+    q, k = _bf16_bits(x)[None, None], _bf16_bits(y)[None, None]
+    for topk in (1, 5, 32, 40):
+        mask = oracle_mod.build_mask(q, k, (2, 4, 4), 0.2, None, topk=topk)
+        kk = min(topk, nb)
+        assert (mask[0, 0][:, :kk] == 1).all() and (mask[0, 0][:, kk:] == 0).all()
+
+
+# ---------------------------------------------------------------------------
+# Token reordering (NABLA review, Figure 4: each attention block becomes one
+# 4x4x4 spatial-temporal patch of the token grid).
+
+
+def _coord_rows(T, H, W, d):
+    """Raster-ordered rows whose first three channels hold (t, h, w) exactly."""
+    t, h, w = np.meshgrid(np.arange(T), np.arange(H), np.arange(W), indexing="ij")
+    rows = np.zeros((T * H * W, d), dtype=np.float32)
+    rows[:, 0], rows[:, 1], rows[:, 2] = t.ravel(), h.ravel(), w.ravel()
+    rows[:, 3:] = np.arange(d - 3, dtype=np.float32)  # integers < 256: exact in bf16
+    return (rows.view(np.uint32) >> 16).astype(np.uint16)
+
+
+@pytest.mark.parametrize("grid", [(1, 1, 1), (2, 3, 1), (3, 2, 5)])
+def test_reorder_matches_numpy_axis_permutation(oracle_mod, grid):
+    # Tile-major order is the raster grid reshaped to (Tt,4,Th,4,Tw,4) with the
+    # tile axes moved in front of the in-tile axes: a numpy transpose.
+    Tt, Th, Tw = grid
+    d = 8
+    x = _coord_rows(4 * Tt, 4 * Th, 4 * Tw, d)
+    y = oracle_mod.reorder(x, grid, to_tile_major=True)
+    ref = x.reshape(Tt, 4, Th, 4, Tw, 4, d).transpose(0, 2, 4, 1, 3, 5, 6).reshape(-1, d)
+    assert np.array_equal(y, ref)
+    back = oracle_mod.reorder(y, grid, to_tile_major=False)
+    assert np.array_equal(back, x)
+
+
+def test_reorder_tiles_are_local_patches(oracle_mod):
+    # Every 64-row block after the reorder spans exactly a 4x4x4 patch whose
+    # corner is a multiple of 4 along each axis.
+    grid = (2, 3, 2)
+    x = _coord_rows(8, 12, 8, 8)
+    y = oracle_mod.reorder(x, grid, to_tile_major=True)
+    c = (y[:, :3].astype(np.uint32) << 16).view(np.float32).astype(np.int64)
+    for b in range(y.shape[0] // 64):
+        blk = c[b * 64:(b + 1) * 64]
+        lo = blk.min(axis=0)
+        assert np.all(lo % 4 == 0)
+        assert np.all(blk.max(axis=0) - lo == 3)
+        assert len({tuple(r) for r in blk}) == 64
+
+
+def test_reorder_agrees_with_synth_tile_major_positions(oracle_mod, synth_mod):
+    # The seeded generator lays tokens out tile-major; its noise-free tensor
+    # must equal the raster-ordered embedding moved by the oracle's reorder.
+    grid = (2, 2, 3)
+    Tt, Th, Tw = grid
+    d = 24
+    S = 64 * Tt * Th * Tw
+    tm = synth_mod.make_tensor(0, 5, 1, 1, S, d, grid=grid, pos_weight=1.0, noise_weight=0.0)
+    T, H, W = 4 * Tt, 4 * Th, 4 * Tw
+    raster = np.empty((S, d), dtype=np.float64)
+    for t in range(T):
+        for h in range(H):
+            for w in range(W):
+                raster[(t * H + h) * W + w] = synth_mod.embedding(d, t, h, w)
+    to_bf16 = np.vectorize(lambda v: int(synth_mod.lib().synth_f64_to_bf16(float(v))))
+    raster_bits = to_bf16(raster).astype(np.uint16)
+    moved = oracle_mod.reorder(raster_bits.reshape(1, 1, S, d), grid, to_tile_major=True)
+    assert np.array_equal(moved.reshape(S, d), tm.reshape(S, d))
+
+
+def test_reorder_batched_heads_independent(oracle_mod):
+    rng = np.random.default_rng(3)
+    grid = (1, 2, 2)
+    x = rng.integers(0, 1 << 16, size=(2, 3, 64 * 4, 16), dtype=np.uint16)
+    y = oracle_mod.reorder(x, grid)
+    for b in range(2):
+        for h in range(3):
+            assert np.array_equal(y[b, h], oracle_mod.reorder(x[b, h], grid))
