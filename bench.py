@@ -341,6 +341,49 @@ def run_ours(args):
     re_gbs = re_bytes / (re_ms * 1e-3) / 1e9
     del qr
 
+    # block energy over the step's own block list (the retained-mass check of
+    # the NABLA mask) and one calibration vote pass over the energy map
+    energy = torch.empty((B, H, nb, nb), dtype=torch.float32, device=dev)
+    bmass = torch.empty((B, H, nb), dtype=torch.float32, device=dev)
+    votes = torch.zeros((B, H, nb, nb), dtype=torch.int32, device=dev)
+    row_ptr, col_idx = mask_out[0], mask_out[1]
+    # dense LSE (every block listed) so that E is the true block attention map
+    # and the retained mass of the NABLA list is its fidelity
+    full_rp = torch.arange(0, B * H * nb + 1, dtype=torch.int64, device=dev).mul_(nb).to(torch.int32)
+    full_ci = torch.arange(nb, dtype=torch.int32, device=dev).repeat(B * H * nb)
+    o_dense = torch.empty_like(q)
+    lse_dense = torch.empty_like(lse)
+    nl.bsa_fwd(q, k, v, full_rp, full_ci, workspace=ws_fwd, out=(o_dense, lse_dense))
+    del full_rp, full_ci, o_dense
+
+    def energy_call():
+        nl.nabla_block_energy(q, k, lse_dense, row_ptr, col_idx, workspace=ws_fwd,
+                              out=(energy, bmass))
+
+    for _ in range(2):
+        energy_call()
+    n_en = 3
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    a.record(stream)
+    for _ in range(n_en):
+        energy_call()
+    b.record(stream)
+    torch.cuda.synchronize()
+    en_ms = a.elapsed_time(b) / n_en
+    ws_fwd.check()
+    en_flops = 2.0 * d * 64 * 64 * kept
+    en_tflops = en_flops / (en_ms * 1e-3) / 1e12
+    retained = float(bmass.mean().item())
+    retained_min = float(bmass.min().item())
+    nl.nabla_calib_accumulate(energy, 0.2, votes)
+    a.record(stream)
+    nl.nabla_calib_accumulate(energy, 0.2, votes)
+    b.record(stream)
+    torch.cuda.synchronize()
+    cal_ms = a.elapsed_time(b)
+    del energy, votes
+
     attn_tflops = kept_flops / (attn_ms * 1e-3) / 1e12
     peak = peaks["bf16_tflops_sustained"]
     traffic = _traffic_per_launch()
@@ -373,6 +416,14 @@ def run_ours(args):
         "reorder": {"bound": "hbm", "ms": re_ms, "achieved": re_gbs, "peak": peaks["hbm_gbs"],
                     "unit": "GB/s", "frac": re_gbs / peaks["hbm_gbs"], "bytes": re_bytes,
                     "what": "raster -> tile-major of one [B,H,S,d] bf16 tensor, outside the step"},
+        "block_energy": {"bound": "tensor", "ms": en_ms, "achieved": en_tflops, "peak": peak,
+                         "unit": "TFLOP/s", "frac": en_tflops / peak,
+                         "flops": en_flops, "blocks": kept,
+                         "mean_true_mass_retained_by_mask": retained,
+                         "min_true_mass_retained_by_mask": retained_min,
+                         "what": "E over the step's kept blocks (QK^T + exp + block sums), "
+                                 "outside the step; FLOPs = 2*d*64*64 per block"},
+        "calib_accumulate_ms": cal_ms,
         "gpu_launches": 6 * args.steps,
         "clocks": clk,
     }

@@ -31,7 +31,8 @@ OP_BUILD_MASK, OP_FWD, OP_FWD_WITH_MASK = 0, 1, 2
 EXPORTED = ["nabla_workspace_size", "nabla_workspace_init", "nabla_query_status",
             "nabla_build_mask", "bsa_fwd", "bsa_fwd_with_mask", "nabla_last_error",
             "nabla_version", "nabla_set_wait_limit_ns", "nabla_selftest_mma",
-            "bsa_fwd_with_mask_static", "nabla_reorder_tokens"]
+            "bsa_fwd_with_mask_static", "nabla_reorder_tokens", "nabla_block_energy",
+            "nabla_calib_accumulate", "nabla_calib_finalize"]
 TO_TILE_MAJOR, TO_RASTER = 0, 1
 
 
@@ -96,6 +97,12 @@ def lib() -> ctypes.CDLL:
             L.nabla_selftest_mma.argtypes = [i32, vp, vp, vp, vp, vp]
             L.nabla_reorder_tokens.restype = i32
             L.nabla_reorder_tokens.argtypes = [sp, i32, vp, vp, vp]
+            L.nabla_block_energy.restype = i32
+            L.nabla_block_energy.argtypes = [sp, vp, vp, vp, vp, vp, f32, vp, vp, vp, vp]
+            L.nabla_calib_accumulate.restype = i32
+            L.nabla_calib_accumulate.argtypes = [sp, vp, f32, vp, vp]
+            L.nabla_calib_finalize.restype = i32
+            L.nabla_calib_finalize.argtypes = [sp, vp, i32, vp, vp]
             L.bsa_fwd_with_mask_static.restype = i32
             L.bsa_fwd_with_mask_static.argtypes = [sp, vp, vp, vp, vp, f32, vp, vp, vp, vp]
             _lib = L
@@ -293,3 +300,56 @@ def nabla_reorder_tokens(x, tile_grid, direction: int = TO_TILE_MAJOR, out=None,
     _check(lib().nabla_reorder_tokens(ctypes.byref(shape), int(direction), _ptr(x), _ptr(y),
                                       _stream(stream)))
     return y
+
+
+def nabla_block_energy(q, k, lse, row_ptr, col_idx, scale: Optional[float] = None,
+                       workspace: Optional[Workspace] = None, out=None, want_block_mass=True,
+                       stream=None):
+    """Per-block attention energy E [B,H,nb,nb] fp32 over the blocks of a CSR
+    (zeros elsewhere), and the row sums of the listed E [B,H,nb] (or None)."""
+    torch = _torch()
+    _bf16_contig(q, k)
+    shape = _shape_of(q)
+    B, H, S, _ = q.shape
+    nb = S // 64
+    if lse.dtype != torch.float32 or not lse.is_contiguous() or tuple(lse.shape) != (B, H, S):
+        raise ValueError("lse must be a contiguous fp32 tensor [B, H, S]")
+    if workspace is None:
+        workspace = Workspace.create(shape, OP_FWD, q.device, stream)
+    if out is None:
+        energy = torch.empty((B, H, nb, nb), dtype=torch.float32, device=q.device)
+        mass = (torch.empty((B, H, nb), dtype=torch.float32, device=q.device)
+                if want_block_mass else None)
+    else:
+        energy, mass = out
+    _check(lib().nabla_block_energy(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(lse),
+                                    _ptr(row_ptr), _ptr(col_idx), float(scale or 0.0),
+                                    _ptr(energy), _ptr(mass) if mass is not None else None,
+                                    _ptr(workspace.buf), _stream(stream)))
+    return energy, mass
+
+
+def nabla_calib_accumulate(energy, eps: float, votes, stream=None):
+    """votes[b,h,r,c] += 1 for each block the minimal-prefix rule keeps at eps."""
+    torch = _torch()
+    for t, dt in ((energy, torch.float32), (votes, torch.int32)):
+        if t.dtype != dt or not t.is_cuda or not t.is_contiguous() or t.dim() != 4:
+            raise ValueError("energy fp32 and votes int32 must be contiguous CUDA [B,H,nb,nb]")
+    B, H, nb, _ = energy.shape
+    shape = make_shape(B, H, nb * 64, 64)
+    _check(lib().nabla_calib_accumulate(ctypes.byref(shape), _ptr(energy), float(eps), _ptr(votes),
+                                        _stream(stream)))
+    return votes
+
+
+def nabla_calib_finalize(votes, min_votes: int = 1, out=None, stream=None):
+    """uint8 static mask [B,H,nb,nb] = votes >= min_votes."""
+    torch = _torch()
+    if votes.dtype != torch.int32 or not votes.is_cuda or not votes.is_contiguous() or votes.dim() != 4:
+        raise ValueError("votes must be a contiguous int32 CUDA tensor [B,H,nb,nb]")
+    B, H, nb, _ = votes.shape
+    mask = torch.empty(votes.shape, dtype=torch.uint8, device=votes.device) if out is None else out
+    shape = make_shape(B, H, nb * 64, 64)
+    _check(lib().nabla_calib_finalize(ctypes.byref(shape), _ptr(votes), int(min_votes), _ptr(mask),
+                                      _stream(stream)))
+    return mask

@@ -230,11 +230,18 @@ struct SelectParams {
 // Relative to the fp64 rule this can move the cut only for rows whose cut
 // mass is within a few 1e-6 of 1 - thr, or swap blocks whose probabilities
 // agree to ~1e-7.
-__global__ void __launch_bounds__(256) select_kernel(const double* __restrict__ L, int64_t nrows,
+//
+// kEnergy: the row holds non-negative fp32 weights (block energies) instead of
+// logits; p = w / sum(w) replaces the softmax, and a row of zero total keeps
+// nothing.  votes (optional, [nrows, nb] int32) gets +1 for every kept entry;
+// bits and counts are optional too.
+template <bool kEnergy>
+__global__ void __launch_bounds__(256) select_kernel(const void* __restrict__ in, int64_t nrows,
                                                      int nb, int wpc, SelectParams prm,
                                                      uint32_t* __restrict__ bits,
                                                      int32_t* __restrict__ counts,
-                                                     uint8_t* __restrict__ mask_u8) {
+                                                     uint8_t* __restrict__ mask_u8,
+                                                     int32_t* __restrict__ votes) {
   extern __shared__ uint32_t sel_keys[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t g = static_cast<int64_t>(blockIdx.x) * wpc + warp;
@@ -242,22 +249,34 @@ __global__ void __launch_bounds__(256) select_kernel(const double* __restrict__ 
   const int r = static_cast<int>(g % nb);
   const int nw = (nb + 31) >> 5;
   uint32_t* key = sel_keys + static_cast<int64_t>(warp) * nb;
-  const double* Lrow = L + g * nb;
 
-  // softmax over the row (max subtracted in fp64)
-  double mx = -INFINITY;
-  for (int c = lane; c < nb; c += 32) mx = fmax(mx, Lrow[c]);
-  mx = warp_max(mx);
   float zl = 0.f;
-  for (int c = lane; c < nb; c += 32) {
-    const float e = expf(static_cast<float>(Lrow[c] - mx));
-    key[c] = __float_as_uint(e);
-    zl += e;
+  bool empty_row = false;
+  if (kEnergy) {
+    const float* Erow = static_cast<const float*>(in) + g * nb;
+    for (int c = lane; c < nb; c += 32) {
+      const float e = Erow[c];
+      const float w = e > 0.f ? e : 0.f;   // negative or NaN weights count as zero
+      key[c] = __float_as_uint(w);
+      zl += w;
+    }
+  } else {
+    // softmax over the row (max subtracted in fp64)
+    const double* Lrow = static_cast<const double*>(in) + g * nb;
+    double mx = -INFINITY;
+    for (int c = lane; c < nb; c += 32) mx = fmax(mx, Lrow[c]);
+    mx = warp_max(mx);
+    for (int c = lane; c < nb; c += 32) {
+      const float e = expf(static_cast<float>(Lrow[c] - mx));
+      key[c] = __float_as_uint(e);
+      zl += e;
+    }
   }
   const float z = static_cast<float>(warp_sum(static_cast<double>(zl)));
+  if (kEnergy) empty_row = !(z > 0.f);   // uniform: z is lane 0's value
   uint32_t kmax = 0;
   for (int c = lane; c < nb; c += 32) {
-    const uint32_t kv = __float_as_uint(__uint_as_float(key[c]) / z);
+    const uint32_t kv = empty_row ? 0u : __float_as_uint(__uint_as_float(key[c]) / z);
     key[c] = kv;
     kmax = max(kmax, kv);
   }
@@ -305,13 +324,15 @@ __global__ void __launch_bounds__(256) select_kernel(const double* __restrict__ 
   bool first_tied = true;      // no tied entry seen yet
   int tied_seen = 0;
   int count = 0;
-  uint32_t* brow = bits + g * nw;
+  uint32_t* brow = bits ? bits + g * nw : nullptr;
   uint8_t* mrow = mask_u8 ? mask_u8 + g * nb : nullptr;
   for (int w = 0; w < nw; ++w) {
     const int c = w * 32 + lane;
     const bool inrow = c < nb;
     bool keep;
-    if (keep_all) {   // warp-uniform branch
+    if (empty_row) {   // warp-uniform branch
+      keep = false;
+    } else if (keep_all) {   // warp-uniform branch
       keep = inrow;
     } else {
       const uint32_t kv = inrow ? key[c] : 0u;
@@ -333,11 +354,21 @@ __global__ void __launch_bounds__(256) select_kernel(const double* __restrict__ 
       keep |= abs(ct - rt) <= prm.wt && abs(ch - rh) <= prm.wh && abs(cw - rw) <= prm.ww;
     }
     if (mrow && inrow) mrow[c] = keep ? 1 : 0;
+    if (votes && keep) votes[g * nb + c] += 1;
     const uint32_t word = __ballot_sync(0xffffffffu, keep);
-    if (lane == 0) brow[w] = word;
+    if (brow && lane == 0) brow[w] = word;
     count += __popc(word);
   }
-  if (lane == 0) counts[g] = count;
+  if (counts && lane == 0) counts[g] = count;
+}
+
+// Calibrated mask from accumulated votes: keep (r, c) iff votes >= min_votes.
+__global__ void __launch_bounds__(256) vote_mask_kernel(const int32_t* __restrict__ votes,
+                                                        int64_t n, int32_t min_votes,
+                                                        uint8_t* __restrict__ mask) {
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+    mask[i] = votes[i] >= min_votes ? 1 : 0;
 }
 
 // External uint8 mask row -> bitmap + count.  One warp per row.
@@ -484,11 +515,39 @@ cudaError_t launch_select(const double* L, int64_t nrows, int nb, float thr, int
   int wpc = static_cast<int>((200u * 1024u) / per_warp);
   wpc = wpc < 1 ? 1 : (wpc > 8 ? 8 : wpc);
   const size_t smem = per_warp * wpc;
-  cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t e = cudaFuncSetAttribute(select_kernel<false>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   const unsigned grid = static_cast<unsigned>((nrows + wpc - 1) / wpc);
-  select_kernel<<<grid, 32 * wpc, smem, st>>>(L, nrows, nb, wpc, prm, bits, counts, mask_u8);
+  select_kernel<false><<<grid, 32 * wpc, smem, st>>>(L, nrows, nb, wpc, prm, bits, counts,
+                                                     mask_u8, nullptr);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_calib_select(const float* energy, int64_t nrows, int nb, float eps,
+                                int32_t* votes, cudaStream_t st) {
+  SelectParams prm{eps, 0, 0, 0, 0, 1, 1, 1, 0};
+  const size_t per_warp = static_cast<size_t>(nb) * sizeof(uint32_t);
+  int wpc = static_cast<int>((200u * 1024u) / per_warp);
+  wpc = wpc < 1 ? 1 : (wpc > 8 ? 8 : wpc);
+  const size_t smem = per_warp * wpc;
+  cudaError_t e = cudaFuncSetAttribute(select_kernel<true>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  const unsigned grid = static_cast<unsigned>((nrows + wpc - 1) / wpc);
+  select_kernel<true><<<grid, 32 * wpc, smem, st>>>(energy, nrows, nb, wpc, prm, nullptr, nullptr,
+                                                    nullptr, votes);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_vote_mask(const int32_t* votes, int64_t n, int32_t min_votes, uint8_t* mask,
+                             cudaStream_t st) {
+  if (n == 0) return cudaSuccess;
+  int64_t blocks = (n + 255) / 256;
+  if (blocks > 148 * 16) blocks = 148 * 16;
+  vote_mask_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(votes, n, min_votes, mask);
   return cudaGetLastError();
 }
 

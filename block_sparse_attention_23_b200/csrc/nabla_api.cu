@@ -34,6 +34,14 @@ cudaError_t launch_bsa_fwd(const CUtensorMap& q, const CUtensorMap& k, const CUt
                            uint64_t wait_limit_ns, cudaStream_t st);
 cudaError_t launch_reorder(const void* src, void* dst, int64_t BH, int Tt, int Th, int Tw,
                            int row_bytes, int to_tile_major, cudaStream_t st);
+cudaError_t launch_block_energy(const CUtensorMap& q, const CUtensorMap& k, const int32_t* row_ptr,
+                                const int32_t* col_idx, const float* lse, float* energy,
+                                float* block_mass, int* status, int BH, int S, int d, float scale,
+                                uint64_t wait_limit_ns, cudaStream_t st);
+cudaError_t launch_calib_select(const float* energy, int64_t nrows, int nb, float eps,
+                                int32_t* votes, cudaStream_t st);
+cudaError_t launch_vote_mask(const int32_t* votes, int64_t n, int32_t min_votes, uint8_t* mask,
+                             cudaStream_t st);
 cudaError_t launch_mma_selftest(const CUtensorMap& a, const CUtensorMap& b, const void* a_glob,
                                 float* c, int variant, int* status, uint64_t lim,
                                 cudaStream_t st);
@@ -325,6 +333,57 @@ nabla_status nabla_reorder_tokens(const nabla_shape* shape, int direction, const
                                         shape->d * 2, direction == NABLA_TO_TILE_MAJOR ? 1 : 0,
                                         reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "reorder launch");
+  return NABLA_OK;
+}
+
+nabla_status nabla_block_energy(const nabla_shape* shape, const void* q, const void* k,
+                                const float* lse, const int32_t* row_ptr, const int32_t* col_idx,
+                                float scale, float* energy, float* block_mass, void* workspace,
+                                nabla_stream_t stream) {
+  nabla_status s = check_shape(shape);
+  if (s != NABLA_OK) return s;
+  if (!q || !k || !lse || !row_ptr || !col_idx || !energy || !workspace)
+    return fail(NABLA_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(q) || !aligned16(k)) return fail(NABLA_ERR_INVALID_ARG, "q, k must be 16-byte aligned");
+  if (!std::isfinite(scale)) return fail(NABLA_ERR_INVALID_ARG, "scale must be finite");
+  const uint64_t rows = static_cast<uint64_t>(shape->B) * shape->H * shape->S;
+  CUtensorMap mq, mk;
+  if ((s = make_map(&mq, q, rows, shape->d)) != NABLA_OK) return s;
+  if ((s = make_map(&mk, k, rows, shape->d)) != NABLA_OK) return s;
+  if (!(scale > 0.f)) scale = 1.0f / std::sqrt(static_cast<float>(shape->d));
+  cudaError_t e = nabla::launch_block_energy(mq, mk, row_ptr, col_idx, lse, energy, block_mass,
+                                             status_ptr(workspace), shape->B * shape->H, shape->S,
+                                             shape->d, scale, g_wait_limit_ns.load(),
+                                             reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "block_energy launch");
+  return NABLA_OK;
+}
+
+nabla_status nabla_calib_accumulate(const nabla_shape* shape, const float* energy, float eps,
+                                    int32_t* votes, nabla_stream_t stream) {
+  nabla_status s = check_shape(shape);
+  if (s != NABLA_OK) return s;
+  if (!(eps >= 0.f && eps <= 1.f)) return fail(NABLA_ERR_UNSUPPORTED, "eps must lie in [0, 1]");
+  if (!energy || !votes) return fail(NABLA_ERR_INVALID_ARG, "null pointer");
+  const int nb = shape->S / 64;
+  const int64_t nrows = static_cast<int64_t>(shape->B) * shape->H * nb;
+  cudaError_t e = nabla::launch_calib_select(energy, nrows, nb, eps, votes,
+                                             reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "calib select launch");
+  return NABLA_OK;
+}
+
+nabla_status nabla_calib_finalize(const nabla_shape* shape, const int32_t* votes,
+                                  int32_t min_votes, uint8_t* mask_u8, nabla_stream_t stream) {
+  nabla_status s = check_shape(shape);
+  if (s != NABLA_OK) return s;
+  if (!votes || !mask_u8) return fail(NABLA_ERR_INVALID_ARG, "null pointer");
+  if (min_votes < 1) return fail(NABLA_ERR_INVALID_ARG, "min_votes must be at least 1");
+  const int64_t nb = shape->S / 64;
+  const int64_t n = static_cast<int64_t>(shape->B) * shape->H * nb * nb;
+  cudaError_t e = nabla::launch_vote_mask(votes, n, min_votes, mask_u8,
+                                          reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "vote mask launch");
   return NABLA_OK;
 }
 

@@ -199,6 +199,55 @@ enum { NABLA_TO_TILE_MAJOR = 0, NABLA_TO_RASTER = 1 };
 NABLA_API nabla_status nabla_reorder_tokens(const nabla_shape* shape, int direction,
                                             const void* src, void* dst, nabla_stream_t stream);
 
+/*
+ * Block attention energy: for every (query block r, key block c) pair listed
+ * in the block CSR, the softmax mass the 64 queries of r place on the 64 keys
+ * of c, averaged over the queries:
+ *     E[r][c] = (1/64) sum_{i in r} sum_{j in c} exp(scale * q_i.k_j - lse_i)
+ * This is the per-block "energy" that CalibAtt's offline calibration
+ * thresholds ("Accelerating Video Diffusion with Calibrated Sparse Attention",
+ * Methodology A) and the true block mass of the fidelity check the NABLA
+ * review asks for (major comment 1).  With lse from a dense bsa_fwd (every
+ * block listed) each row of E sums to 1.
+ *   q, k        device bf16 [B,H,S,d], 16-byte aligned (tile-major tokens)
+ *   lse         device fp32 [B,H,S] natural-log LSE per query row; a row with
+ *               lse = -inf (or any non-finite value) contributes nothing
+ *   row_ptr, col_idx  block CSR as for bsa_fwd (the blocks to evaluate)
+ *   scale       softmax scale; <= 0 selects 1/sqrt(d)
+ *   energy      device fp32 [B,H,nb,nb], written in full: unlisted blocks 0
+ *   block_mass  device fp32 [B,H,nb] or NULL: sum of the row's listed E
+ *   workspace   device, nabla_workspace_size(shape, NABLA_OP_FWD) bytes
+ * Device-side failures (timeouts, bad column indices) are recorded in the
+ * workspace status word; a CTA that timed out leaves its two rows unwritten.
+ */
+NABLA_API nabla_status nabla_block_energy(const nabla_shape* shape, const void* q, const void* k,
+                                          const float* lse, const int32_t* row_ptr,
+                                          const int32_t* col_idx, float scale, float* energy,
+                                          float* block_mass, void* workspace,
+                                          nabla_stream_t stream);
+
+/*
+ * Calibrated static masks (CalibAtt, Methodology A: per (timestep, layer,
+ * head) the minimal block set holding 1 - eps of each row's energy, averaged
+ * over the calibration runs; blocks that are consistently missed are skipped).
+ * nabla_calib_accumulate applies the minimal-prefix rule of nabla_build_mask
+ * (thr = eps, ties to the lower block index, the largest block always kept,
+ * eps = 0 keeps every block) to each row of energy normalised by its sum, and
+ * adds 1 to votes[b,h,r,c] for each kept block; a row whose energy sums to 0
+ * keeps nothing.  Call it once per calibration run (eps is the caller's eps(t)
+ * for the timestep being calibrated), starting from votes = 0.
+ * nabla_calib_finalize writes mask_u8 = (votes >= min_votes), the uint8
+ * [B,H,nb,nb] mask that bsa_fwd_with_mask takes; min_votes = 1 skips exactly
+ * the blocks no run selected.
+ *   energy   device fp32 [B,H,nb,nb];  votes  device int32 [B,H,nb,nb]
+ * Both calls are stream-ordered and need no workspace.
+ */
+NABLA_API nabla_status nabla_calib_accumulate(const nabla_shape* shape, const float* energy,
+                                              float eps, int32_t* votes, nabla_stream_t stream);
+NABLA_API nabla_status nabla_calib_finalize(const nabla_shape* shape, const int32_t* votes,
+                                            int32_t min_votes, uint8_t* mask_u8,
+                                            nabla_stream_t stream);
+
 /* Message for the last error returned on the calling host thread. */
 NABLA_API const char* nabla_last_error(void);
 

@@ -73,6 +73,13 @@ def _load():
             lib.oracle_dense_attention.argtypes = [vp, vp, vp, i64, i64, i32, f64, i64, vp, vp, vp]
             lib.oracle_reorder.restype = None
             lib.oracle_reorder.argtypes = [vp, vp, i64, i32, i32, i32, i32, i32]
+            lib.oracle_block_energy.restype = None
+            lib.oracle_block_energy.argtypes = [vp, vp, vp, i64, i64, i32, vp, f64, i64, vp, vp,
+                                                vp]
+            lib.oracle_calib_accumulate.restype = None
+            lib.oracle_calib_accumulate.argtypes = [vp, i64, i32, f64, vp]
+            lib.oracle_calib_finalize.restype = None
+            lib.oracle_calib_finalize.argtypes = [vp, i64, i32, vp]
             lib.oracle_max_threads.restype = i32
             lib.oracle_max_threads.argtypes = []
             _lib = lib
@@ -215,6 +222,51 @@ def reorder(x: np.ndarray, tile_grid, to_tile_major: bool = True) -> np.ndarray:
     _load().oracle_reorder(x.ctypes.data, out.ctypes.data, BH, Tt, Th, Tw, d,
                            1 if to_tile_major else 0)
     return out
+
+
+def block_energy(q, k, lse, mask, scale=None, rows=None):
+    """Per-block attention energy over the listed blocks (0 elsewhere) and its
+    row sums.  lse: [B,H,S], any float dtype.  rows=None: returns
+    ([B,H,nb,nb], [B,H,nb]); else rows = global block-row ids bh*nb + r and
+    the result is ([len(rows), nb], [len(rows)])."""
+    q, k = _u16(q), _u16(k)
+    B, H, S, d = q.shape
+    nb = S // BLOCK
+    mask = np.ascontiguousarray(mask, dtype=np.uint8).reshape(B, H, nb, nb)
+    lse = np.ascontiguousarray(lse, dtype=np.float64).reshape(B, H, S)
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    if rows is None:
+        n, rp = B * H * nb, None
+        energy = np.empty((B, H, nb, nb), dtype=np.float64)
+        mass = np.empty((B, H, nb), dtype=np.float64)
+    else:
+        rows = np.ascontiguousarray(rows, dtype=np.int64)
+        n, rp = rows.shape[0], rows.ctypes.data
+        energy = np.empty((n, nb), dtype=np.float64)
+        mass = np.empty(n, dtype=np.float64)
+    _load().oracle_block_energy(q.ctypes.data, k.ctypes.data, lse.ctypes.data, B * H, S, d,
+                                mask.ctypes.data, float(scale), n, rp, energy.ctypes.data,
+                                mass.ctypes.data)
+    return energy, mass
+
+
+def calib_accumulate(energy: np.ndarray, eps: float, votes: np.ndarray) -> np.ndarray:
+    """votes += the minimal-prefix selection (thr = eps) of each normalised energy row."""
+    energy = np.ascontiguousarray(energy, dtype=np.float64)
+    if votes.dtype != np.int32 or not votes.flags.c_contiguous or votes.shape != energy.shape:
+        raise ValueError("votes must be a C-contiguous int32 array shaped like energy")
+    nb = energy.shape[-1]
+    _load().oracle_calib_accumulate(energy.ctypes.data, energy.size // nb, nb, float(eps),
+                                    votes.ctypes.data)
+    return votes
+
+
+def calib_finalize(votes: np.ndarray, min_votes: int = 1) -> np.ndarray:
+    votes = np.ascontiguousarray(votes, dtype=np.int32)
+    mask = np.empty(votes.shape, dtype=np.uint8)
+    _load().oracle_calib_finalize(votes.ctypes.data, votes.size, int(min_votes), mask.ctypes.data)
+    return mask
 
 
 def near_cut_rows(diag: np.ndarray, thr: float, band: float = 1e-4) -> np.ndarray:

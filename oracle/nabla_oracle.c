@@ -289,6 +289,82 @@ void oracle_reorder(const uint16_t* src, uint16_t* dst, int64_t BH, int Tt, int 
                 }
 }
 
+/* Block attention energy ("Accelerating Video Diffusion with Calibrated
+ * Sparse Attention", Methodology A: the energy, i.e. summed attention scores,
+ * of each block; NABLA review, major comment 1: the true attention mass of an
+ * N x N block).  For each listed (r, c):
+ *   E[r][c] = (1/64) sum_{i in block r} sum_{j in block c} exp(scale q_i.k_j - lse_i)
+ * mask [BH, nb, nb] uint8 marks the listed blocks; lse [BH*S] is given (a row
+ * with a non-finite lse contributes nothing).  The block rows evaluated are
+ * rows[0..nrows) (global ids bh*nb + r), or every row when rows is NULL;
+ * energy [nrows, nb] is written in full, 0 where unlisted; block_mass (may be
+ * NULL) [nrows] = sum_c E[r][c]. */
+void oracle_block_energy(const uint16_t* q, const uint16_t* k, const double* lse, int64_t BH,
+                         int64_t S, int d, const uint8_t* mask, double scale, int64_t nrows,
+                         const int64_t* rows, double* energy, double* block_mass) {
+    const int64_t nb = S / ORACLE_BLOCK;
+    if (rows == NULL) nrows = BH * nb;
+#pragma omp parallel for schedule(dynamic)
+    for (int64_t n = 0; n < nrows; ++n) {
+        int64_t br = rows ? rows[n] : n;
+        int64_t bh = br / nb, r = br % nb;
+        double total = 0.0;
+        for (int64_t c = 0; c < nb; ++c) {
+            double e = 0.0;
+            if (mask[br * nb + c]) {
+                for (int64_t i = r * ORACLE_BLOCK; i < (r + 1) * ORACLE_BLOCK; ++i) {
+                    double li = lse[bh * S + i];
+                    if (!isfinite(li)) continue;
+                    for (int64_t j = c * ORACLE_BLOCK; j < (c + 1) * ORACLE_BLOCK; ++j) {
+                        double dot = 0.0;
+                        for (int t = 0; t < d; ++t)
+                            dot += bf16_to_f64(q[(bh * S + i) * d + t]) *
+                                   bf16_to_f64(k[(bh * S + j) * d + t]);
+                        e += exp(scale * dot - li);
+                    }
+                }
+                e /= ORACLE_BLOCK;
+            }
+            energy[n * nb + c] = e;
+            total += e;
+        }
+        if (block_mass) block_mass[n] = total;
+    }
+}
+
+/* One calibration run (CalibAtt, Methodology A, "threshold" step): each energy
+ * row, normalised by its sum, goes through the same minimal-prefix rule as the
+ * NABLA mask with thr = eps; votes[r][c] += 1 for every kept block.  A row
+ * whose energy sums to zero keeps nothing; negative or NaN energies count as
+ * zero. */
+void oracle_calib_accumulate(const double* energy, int64_t nrows, int nb, double eps,
+                             int32_t* votes) {
+#pragma omp parallel for schedule(static)
+    for (int64_t g = 0; g < nrows; ++g) {
+        double* p = (double*)malloc(sizeof(double) * (size_t)nb);
+        uint8_t* keep = (uint8_t*)malloc((size_t)nb);
+        double z = 0.0;
+        for (int c = 0; c < nb; ++c) {
+            double e = energy[g * nb + c];
+            p[c] = e > 0.0 ? e : 0.0;
+            z += p[c];
+        }
+        if (z > 0.0) {
+            for (int c = 0; c < nb; ++c) p[c] /= z;
+            oracle_row_select(p, nb, eps, keep, NULL);
+            for (int c = 0; c < nb; ++c) votes[g * nb + c] += keep[c];
+        }
+        free(p);
+        free(keep);
+    }
+}
+
+/* Aggregation over the calibration runs (CalibAtt, Methodology A: blocks that
+ * the runs consistently miss are skipped): mask = votes >= min_votes. */
+void oracle_calib_finalize(const int32_t* votes, int64_t n, int32_t min_votes, uint8_t* mask) {
+    for (int64_t i = 0; i < n; ++i) mask[i] = votes[i] >= min_votes ? 1 : 0;
+}
+
 /* Threads OpenMP will use (for reporting the CPU baseline's core count). */
 int oracle_max_threads(void) {
 #ifdef _OPENMP

@@ -458,3 +458,146 @@ def test_reorder_batched_heads_independent(oracle_mod):
     for b in range(2):
         for h in range(3):
             assert np.array_equal(y[b, h], oracle_mod.reorder(x[b, h], grid))
+
+
+# ---------------------------------------------------------------------------
+# Block energy (CalibAtt's per-block energy; the NABLA review's true block mass)
+
+
+def _torch_block_energy(q, k, scale=None):
+    """fp64 torch: dense softmax of the score matrix, summed over 64 x 64 blocks
+    and divided by 64 (mean over the block's queries)."""
+    import torch
+    B, H, S, d = q.shape
+    nb = S // 64
+    qf = torch.from_numpy(_f(q))
+    kf = torch.from_numpy(_f(k))
+    s = torch.einsum("bhid,bhjd->bhij", qf, kf) * (scale if scale else 1.0 / math.sqrt(d))
+    p = torch.softmax(s, dim=-1)
+    e = p.reshape(B, H, nb, 64, nb, 64).sum(dim=(3, 5)) / 64.0
+    lse = torch.logsumexp(s, dim=-1)
+    return e.numpy(), lse.numpy()
+
+
+def test_block_energy_matches_torch_dense_softmax(oracle_mod):
+    rng = np.random.default_rng(21)
+    B, H, S, d = 1, 2, 256, 64
+    q = _rand_bits(rng, (B, H, S, d), 0.6)
+    k = _rand_bits(rng, (B, H, S, d), 0.6)
+    want, lse = _torch_block_energy(q, k)
+    full = np.ones((B, H, S // 64, S // 64), dtype=np.uint8)
+    got, mass = oracle_mod.block_energy(q, k, lse, full)
+    np.testing.assert_allclose(got, want, rtol=1e-10, atol=1e-14)
+    np.testing.assert_allclose(mass, 1.0, rtol=0, atol=1e-12)
+    # the block map is not symmetric in (r, c): a transposed index would show
+    assert np.abs(want - np.swapaxes(want, -1, -2)).max() > 1e-3
+    # a row subset returns the same rows
+    rows = np.array([3, 0, 6], dtype=np.int64)
+    sub, smass = oracle_mod.block_energy(q, k, lse, full, rows=rows)
+    np.testing.assert_array_equal(sub, got.reshape(-1, S // 64)[rows])
+    np.testing.assert_array_equal(smass, mass.reshape(-1)[rows])
+
+
+def test_block_energy_rows_sum_to_one_with_dense_lse(oracle_mod, synth_mod):
+    w = synth_mod.WORKLOADS["tiny"]
+    q, k, v = synth_mod.make_qkv(w)
+    _, lse = oracle_mod.dense_attention(q, k, v)
+    full = np.ones((w.B, w.H, w.nb, w.nb), dtype=np.uint8)
+    E, mass = oracle_mod.block_energy(q, k, lse.reshape(w.B, w.H, w.S), full)
+    np.testing.assert_allclose(E.sum(axis=-1), 1.0, atol=1e-12)
+    np.testing.assert_allclose(mass, 1.0, atol=1e-12)
+    assert (E > 0).all()
+
+
+def test_block_energy_uniform_attention_closed_form(oracle_mod):
+    # q = 0: every score is 0, LSE = ln S, and each block holds 64*64/S of the
+    # mass of its 64 queries: E = 64/S = 1/nb at listed blocks, 0 elsewhere.
+    rng = np.random.default_rng(4)
+    B, H, S, d = 1, 1, 512, 64
+    nb = S // 64
+    q = np.zeros((B, H, S, d), dtype=np.uint16)
+    k = _rand_bits(rng, (B, H, S, d))
+    lse = np.full((B, H, S), math.log(S))
+    mask = (rng.random((B, H, nb, nb)) < 0.4).astype(np.uint8)
+    E, mass = oracle_mod.block_energy(q, k, lse, mask)
+    np.testing.assert_allclose(E, mask / nb, rtol=1e-14, atol=0)
+    np.testing.assert_allclose(mass, mask.sum(-1) / nb, rtol=1e-14)
+
+
+def test_block_energy_nonfinite_lse_rows_contribute_nothing(oracle_mod):
+    rng = np.random.default_rng(5)
+    B, H, S, d = 1, 1, 256, 64
+    q = _rand_bits(rng, (B, H, S, d))
+    k = _rand_bits(rng, (B, H, S, d))
+    want, lse = _torch_block_energy(q, k)
+    lse = lse.copy()
+    lse[0, 0, 64:128] = -np.inf          # query block 1 has no kept key
+    lse[0, 0, 130] = np.nan              # and one row of block 2 is undefined
+    full = np.ones((B, H, 4, 4), dtype=np.uint8)
+    E, _ = oracle_mod.block_energy(q, k, lse, full)
+    assert (E[0, 0, 1] == 0).all()
+    np.testing.assert_allclose(E[0, 0, [0, 3]], want[0, 0, [0, 3]], rtol=1e-10)
+    assert (E[0, 0, 2] < want[0, 0, 2]).all()
+
+
+# ---------------------------------------------------------------------------
+# Calibration (CalibAtt, Methodology A: threshold per row, aggregate over runs)
+
+
+@pytest.mark.parametrize("rho,eps", [(0.8, 0.2), (0.9, 0.4), (0.97, 0.1)])
+def test_calib_geometric_energy_closed_form(oracle_mod, rho, eps):
+    # an energy row proportional to rho^c (any positive scale) keeps the
+    # closed-form count of the geometric model, at the largest blocks
+    n = 96
+    x = math.log(1.0 - (1.0 - eps) * (1.0 - rho ** n)) / math.log(rho)
+    assert abs(x - round(x)) > 1e-6
+    want = _geometric_count(rho, n, eps)
+    rng = np.random.default_rng(9)
+    perm = rng.permutation(n)
+    row = np.empty(n)
+    row[perm] = 3.7e-3 * rho ** np.arange(n)     # unnormalised energies
+    votes = np.zeros((1, 1, 1, n), dtype=np.int32)
+    oracle_mod.calib_accumulate(row.reshape(1, 1, 1, n), eps, votes)
+    assert votes.sum() == want
+    assert set(np.nonzero(votes[0, 0, 0])[0]) == set(perm[:want])
+
+
+def test_calib_votes_union_and_intersection(oracle_mod):
+    rng = np.random.default_rng(12)
+    nb = 24
+    runs = [rng.gamma(0.5, size=(1, 2, nb, nb)) for _ in range(3)]
+    votes = np.zeros((1, 2, nb, nb), dtype=np.int32)
+    sel = []
+    for e in runs:
+        one = np.zeros_like(votes)
+        oracle_mod.calib_accumulate(e, 0.3, one)
+        sel.append(one.astype(bool))
+        oracle_mod.calib_accumulate(e, 0.3, votes)
+    assert votes.max() <= 3
+    np.testing.assert_array_equal(votes, sum(s.astype(np.int32) for s in sel))
+    union = oracle_mod.calib_finalize(votes, 1).astype(bool)
+    inter = oracle_mod.calib_finalize(votes, 3).astype(bool)
+    np.testing.assert_array_equal(union, sel[0] | sel[1] | sel[2])
+    np.testing.assert_array_equal(inter, sel[0] & sel[1] & sel[2])
+    # each run keeps at least the row's largest block
+    for e, s in zip(runs, sel):
+        am = e.argmax(-1)
+        assert np.take_along_axis(s, am[..., None], -1).all()
+
+
+def test_calib_scale_invariance_and_zero_rows(oracle_mod):
+    rng = np.random.default_rng(13)
+    nb = 40
+    e = rng.gamma(0.7, size=(1, 1, nb, nb))
+    e[0, 0, 5] = 0.0                  # an all-zero row keeps nothing
+    e[0, 0, 6, :3] = -1.0             # negative energies count as zero
+    a = np.zeros(e.shape, dtype=np.int32)
+    b = np.zeros(e.shape, dtype=np.int32)
+    oracle_mod.calib_accumulate(e, 0.25, a)
+    oracle_mod.calib_accumulate(e * 1024.0, 0.25, b)
+    np.testing.assert_array_equal(a, b)
+    assert a[0, 0, 5].sum() == 0
+    assert (a[0, 0, 6, :3] == 0).all()
+    full = np.zeros(e.shape, dtype=np.int32)
+    oracle_mod.calib_accumulate(e, 0.0, full)      # eps = 0 keeps every block of a live row
+    assert full[0, 0, 5].sum() == 0 and (np.delete(full[0, 0], 5, axis=0) == 1).all()
