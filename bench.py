@@ -384,6 +384,31 @@ def run_ours(args):
     cal_ms = a.elapsed_time(b)
     del energy, votes
 
+    # backward over the step's block list (dO ~ N(0,1)), outside the step;
+    # algorithmic FLOPs = the five 64x64xd products per kept block pair
+    g = torch.Generator(device=dev).manual_seed(args.seed + 17)
+    dout = torch.randn(q.shape, device=dev, generator=g).to(torch.bfloat16)
+    ws_bwd = nl.Workspace.create(shape, nl.OP_BWD, dev)
+    grads = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v))
+
+    def bwd_call():
+        nl.bsa_bwd(q, k, v, o, dout, lse, row_ptr, col_idx, workspace=ws_bwd, out=grads)
+
+    bwd_call()
+    torch.cuda.synchronize()
+    ws_bwd.check()
+    n_bw = 3
+    a.record(stream)
+    for _ in range(n_bw):
+        bwd_call()
+    b.record(stream)
+    torch.cuda.synchronize()
+    ws_bwd.check()
+    bwd_ms = a.elapsed_time(b) / n_bw
+    bwd_flops = 2.5 * kept_flops
+    bwd_tflops = bwd_flops / (bwd_ms * 1e-3) / 1e12
+    del dout, grads
+
     attn_tflops = kept_flops / (attn_ms * 1e-3) / 1e12
     peak = peaks["bf16_tflops_sustained"]
     traffic = _traffic_per_launch()
@@ -424,6 +449,10 @@ def run_ours(args):
                          "what": "E over the step's kept blocks (QK^T + exp + block sums), "
                                  "outside the step; FLOPs = 2*d*64*64 per block"},
         "calib_accumulate_ms": cal_ms,
+        "bwd": {"bound": "tensor", "ms": bwd_ms, "achieved": bwd_tflops, "peak": peak,
+                "unit": "TFLOP/s", "frac": bwd_tflops / peak, "flops": bwd_flops,
+                "what": "bsa_bwd (D, column bitmaps, dK/dV and dQ kernels) over the step's "
+                        "block list, outside the step; FLOPs = 10*d*64*64 per kept block"},
         "gpu_launches": 6 * args.steps,
         "clocks": clk,
     }

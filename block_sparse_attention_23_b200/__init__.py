@@ -27,12 +27,12 @@ NABLA_OK = 0
 STATUS_NAMES = {0: "NABLA_OK", 1: "NABLA_ERR_INVALID_ARG", 2: "NABLA_ERR_UNSUPPORTED",
                 3: "NABLA_ERR_CAPACITY", 4: "NABLA_ERR_CUDA", 5: "NABLA_ERR_TIMEOUT",
                 6: "NABLA_ERR_BAD_INDEX"}
-OP_BUILD_MASK, OP_FWD, OP_FWD_WITH_MASK = 0, 1, 2
+OP_BUILD_MASK, OP_FWD, OP_FWD_WITH_MASK, OP_BWD = 0, 1, 2, 3
 EXPORTED = ["nabla_workspace_size", "nabla_workspace_init", "nabla_query_status",
             "nabla_build_mask", "bsa_fwd", "bsa_fwd_with_mask", "nabla_last_error",
             "nabla_version", "nabla_set_wait_limit_ns", "nabla_selftest_mma",
             "bsa_fwd_with_mask_static", "nabla_reorder_tokens", "nabla_block_energy",
-            "nabla_calib_accumulate", "nabla_calib_finalize"]
+            "nabla_calib_accumulate", "nabla_calib_finalize", "bsa_bwd"]
 TO_TILE_MAJOR, TO_RASTER = 0, 1
 
 
@@ -103,6 +103,8 @@ def lib() -> ctypes.CDLL:
             L.nabla_calib_accumulate.argtypes = [sp, vp, f32, vp, vp]
             L.nabla_calib_finalize.restype = i32
             L.nabla_calib_finalize.argtypes = [sp, vp, i32, vp, vp]
+            L.bsa_bwd.restype = i32
+            L.bsa_bwd.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, vp, f32, vp, vp, vp, vp, vp]
             L.bsa_fwd_with_mask_static.restype = i32
             L.bsa_fwd_with_mask_static.argtypes = [sp, vp, vp, vp, vp, f32, vp, vp, vp, vp]
             _lib = L
@@ -353,3 +355,25 @@ def nabla_calib_finalize(votes, min_votes: int = 1, out=None, stream=None):
     _check(lib().nabla_calib_finalize(ctypes.byref(shape), _ptr(votes), int(min_votes), _ptr(mask),
                                       _stream(stream)))
     return mask
+
+
+def bsa_bwd(q, k, v, o, dout, lse, row_ptr, col_idx, scale: Optional[float] = None,
+            workspace: Optional[Workspace] = None, out=None, stream=None):
+    """Gradients (dQ, dK, dV), bf16 [B,H,S,d], of the block-sparse forward over
+    the same CSR, from its O and LSE and the output gradient dO."""
+    torch = _torch()
+    _bf16_contig(q, k, v, o, dout)
+    shape = _shape_of(q)
+    B, H, S, _ = q.shape
+    if lse.dtype != torch.float32 or not lse.is_contiguous() or tuple(lse.shape) != (B, H, S):
+        raise ValueError("lse must be a contiguous fp32 tensor [B, H, S]")
+    if workspace is None:
+        workspace = Workspace.create(shape, OP_BWD, q.device, stream)
+    if out is None:
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    else:
+        dq, dk, dv = out
+    _check(lib().bsa_bwd(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout),
+                         _ptr(lse), _ptr(row_ptr), _ptr(col_idx), float(scale or 0.0), _ptr(dq),
+                         _ptr(dk), _ptr(dv), _ptr(workspace.buf), _stream(stream)))
+    return dq, dk, dv

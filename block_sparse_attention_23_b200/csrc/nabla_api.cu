@@ -42,6 +42,12 @@ cudaError_t launch_calib_select(const float* energy, int64_t nrows, int nb, floa
                                 int32_t* votes, cudaStream_t st);
 cudaError_t launch_vote_mask(const int32_t* votes, int64_t n, int32_t min_votes, uint8_t* mask,
                              cudaStream_t st);
+cudaError_t launch_bsa_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                           const CUtensorMap& mdo, const void* o, const void* dout,
+                           const float* lse, const int32_t* row_ptr, const int32_t* col_idx,
+                           float* dvec, uint32_t* colbits, void* dq, void* dk, void* dv,
+                           int* status, int BH, int S, int d, float scale, uint64_t wait_limit_ns,
+                           cudaStream_t st);
 cudaError_t launch_mma_selftest(const CUtensorMap& a, const CUtensorMap& b, const void* a_glob,
                                 float* c, int variant, int* status, uint64_t lim,
                                 cudaStream_t st);
@@ -100,6 +106,20 @@ BuildLayout build_layout(const nabla_shape* s) {
   l.logits = off; off = align256(off + BH * nb * nb * 8);
   l.bits = off; off = align256(off + BH * nb * nw * 4);
   l.counts = off; off = align256(off + BH * nb * 4);
+  l.total = off;
+  return l;
+}
+
+struct BwdLayout {
+  size_t dvec, colbits, total;
+};
+
+BwdLayout bwd_layout(const nabla_shape* s) {
+  const size_t nb = s->S / 64, BH = static_cast<size_t>(s->B) * s->H, nw = (nb + 31) / 32;
+  BwdLayout l;
+  size_t off = kHeaderBytes;
+  l.dvec = off; off = align256(off + BH * s->S * 4);
+  l.colbits = off; off = align256(off + BH * nb * nw * 4);
   l.total = off;
   return l;
 }
@@ -198,6 +218,7 @@ size_t nabla_workspace_size(const nabla_shape* shape, int op) {
     case NABLA_OP_BUILD_MASK: return build_layout(shape).total;
     case NABLA_OP_FWD: return kHeaderBytes;
     case NABLA_OP_FWD_WITH_MASK: return mask_layout(shape).total;
+    case NABLA_OP_BWD: return bwd_layout(shape).total;
     default: g_last_error = "unknown op"; return 0;
   }
 }
@@ -384,6 +405,39 @@ nabla_status nabla_calib_finalize(const nabla_shape* shape, const int32_t* votes
   cudaError_t e = nabla::launch_vote_mask(votes, n, min_votes, mask_u8,
                                           reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "vote mask launch");
+  return NABLA_OK;
+}
+
+nabla_status bsa_bwd(const nabla_shape* shape, const void* q, const void* k, const void* v,
+                     const void* o, const void* dout, const float* lse, const int32_t* row_ptr,
+                     const int32_t* col_idx, float scale, void* dq, void* dk, void* dv,
+                     void* workspace, nabla_stream_t stream) {
+  nabla_status s = check_shape(shape);
+  if (s != NABLA_OK) return s;
+  if (!q || !k || !v || !o || !dout || !lse || !row_ptr || !col_idx || !dq || !dk || !dv ||
+      !workspace)
+    return fail(NABLA_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) ||
+      !aligned16(lse) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv) ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return fail(NABLA_ERR_INVALID_ARG,
+                "tensors and lse need 16-byte and workspace 256-byte alignment");
+  if (!std::isfinite(scale)) return fail(NABLA_ERR_INVALID_ARG, "scale must be finite");
+  const uint64_t rows = static_cast<uint64_t>(shape->B) * shape->H * shape->S;
+  CUtensorMap mq, mk, mv, mdo;
+  if ((s = make_map(&mq, q, rows, shape->d)) != NABLA_OK) return s;
+  if ((s = make_map(&mk, k, rows, shape->d)) != NABLA_OK) return s;
+  if ((s = make_map(&mv, v, rows, shape->d)) != NABLA_OK) return s;
+  if ((s = make_map(&mdo, dout, rows, shape->d)) != NABLA_OK) return s;
+  if (!(scale > 0.f)) scale = 1.0f / std::sqrt(static_cast<float>(shape->d));
+  const BwdLayout lay = bwd_layout(shape);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  cudaError_t e = nabla::launch_bsa_bwd(
+      mq, mk, mv, mdo, o, dout, lse, row_ptr, col_idx, reinterpret_cast<float*>(ws + lay.dvec),
+      reinterpret_cast<uint32_t*>(ws + lay.colbits), dq, dk, dv, status_ptr(workspace),
+      shape->B * shape->H, shape->S, shape->d, scale, g_wait_limit_ns.load(),
+      reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "bsa_bwd launch");
   return NABLA_OK;
 }
 

@@ -71,7 +71,8 @@ typedef struct {
 enum {
     NABLA_OP_BUILD_MASK = 0,     /* workspace for nabla_build_mask */
     NABLA_OP_FWD = 1,            /* workspace for bsa_fwd */
-    NABLA_OP_FWD_WITH_MASK = 2   /* workspace for bsa_fwd_with_mask */
+    NABLA_OP_FWD_WITH_MASK = 2,  /* workspace for bsa_fwd_with_mask */
+    NABLA_OP_BWD = 3             /* workspace for bsa_bwd */
 };
 
 /* Bytes of workspace the operation needs for this shape (0 on a bad shape).
@@ -181,6 +182,32 @@ NABLA_API nabla_status bsa_fwd_with_mask_static(const nabla_shape* shape, const 
                                                 const uint8_t* mask_u8, float scale, void* o,
                                                 float* lse, int32_t* status_out,
                                                 nabla_stream_t stream);
+
+/*
+ * Block-sparse attention backward: the gradients of bsa_fwd's O with respect
+ * to Q, K and V over the same block CSR (FlashAttention's backward, which
+ * recomputes P from the saved LSE; NABLA trains through the same block mask,
+ * "NABLA: Neighborhood Adaptive Block-Level Attention", review summary).  With
+ * P = exp(scale Q K^T - LSE) on kept blocks (0 elsewhere) and
+ * D_i = sum_k dO_ik O_ik:
+ *     dV = P^T dO,  dS = P o (dO V^T - D),  dQ = scale dS K,  dK = scale dS^T Q
+ *   q, k, v, o, dout   device bf16 [B,H,S,d], 16-byte aligned; o and lse are
+ *                      bsa_fwd's outputs for the same q, k, v, CSR and scale
+ *   lse                device fp32 [B,H,S], 16-byte aligned
+ *   row_ptr, col_idx   the forward's block CSR (any column order; duplicates
+ *                      count once; out-of-range indices are skipped and
+ *                      reported as NABLA_ERR_BAD_INDEX)
+ *   scale              <= 0 selects 1/sqrt(d)
+ *   dq, dk, dv         device bf16 [B,H,S,d] outputs, written in full (rows
+ *                      that no kept block reaches get 0)
+ *   workspace          device, nabla_workspace_size(shape, NABLA_OP_BWD) bytes
+ * Stream-ordered; deterministic (no atomics in the gradient sums).
+ */
+NABLA_API nabla_status bsa_bwd(const nabla_shape* shape, const void* q, const void* k,
+                               const void* v, const void* o, const void* dout, const float* lse,
+                               const int32_t* row_ptr, const int32_t* col_idx, float scale,
+                               void* dq, void* dk, void* dv, void* workspace,
+                               nabla_stream_t stream);
 
 /*
  * Token reordering between raster and tile-major order (the neighbourhood

@@ -80,6 +80,9 @@ def _load():
             lib.oracle_calib_accumulate.argtypes = [vp, i64, i32, f64, vp]
             lib.oracle_calib_finalize.restype = None
             lib.oracle_calib_finalize.argtypes = [vp, i64, i32, vp]
+            lib.oracle_attention_bwd.restype = None
+            lib.oracle_attention_bwd.argtypes = [vp, vp, vp, vp, i64, i64, i32, vp, f64, i64, vp,
+                                                 vp, i64, vp, vp, vp]
             lib.oracle_max_threads.restype = i32
             lib.oracle_max_threads.argtypes = []
             _lib = lib
@@ -267,6 +270,34 @@ def calib_finalize(votes: np.ndarray, min_votes: int = 1) -> np.ndarray:
     mask = np.empty(votes.shape, dtype=np.uint8)
     _load().oracle_calib_finalize(votes.ctypes.data, votes.size, int(min_votes), mask.ctypes.data)
     return mask
+
+
+def attention_bwd(q, k, v, dO, mask, scale=None, qrows=None, krows=None):
+    """Gradients of block-masked softmax attention in fp64.
+
+    q, k, v, dO: [B,H,S,d] bf16 bits; mask [B,H,nb,nb].  qrows / krows: global
+    row ids (bh*S + i) for dQ and for dK, dV; None = every row, an empty array
+    = none.  Returns (dQ [nq,d], dK [nk,d], dV [nk,d]) fp64."""
+    q, k, v, dO = _u16(q), _u16(k), _u16(v), _u16(dO)
+    B, H, S, d = q.shape
+    nb = S // BLOCK
+    mask = np.ascontiguousarray(mask, dtype=np.uint8).reshape(B, H, nb, nb)
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    def sel(rows):
+        if rows is None:
+            return B * H * S, None, None
+        rows = np.ascontiguousarray(rows, dtype=np.int64)
+        return rows.shape[0], rows, rows.ctypes.data
+    nq, qa, qp = sel(qrows)
+    nk, ka, kp = sel(krows)
+    dQ = np.empty((nq, d), dtype=np.float64)
+    dK = np.empty((nk, d), dtype=np.float64)
+    dV = np.empty((nk, d), dtype=np.float64)
+    _load().oracle_attention_bwd(q.ctypes.data, k.ctypes.data, v.ctypes.data, dO.ctypes.data,
+                                 B * H, S, d, mask.ctypes.data, float(scale), nq, qp,
+                                 dQ.ctypes.data, nk, kp, dK.ctypes.data, dV.ctypes.data)
+    return dQ, dK, dV
 
 
 def near_cut_rows(diag: np.ndarray, thr: float, band: float = 1e-4) -> np.ndarray:

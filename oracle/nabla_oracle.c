@@ -365,6 +365,105 @@ void oracle_calib_finalize(const int32_t* votes, int64_t n, int32_t min_votes, u
     for (int64_t i = 0; i < n; ++i) mask[i] = votes[i] >= min_votes ? 1 : 0;
 }
 
+/* Row statistics of block-masked attention for query row i of head bh:
+ * lse = ln sum_j exp(scale q_i.k_j) over kept keys (-inf when none) and
+ * D = dO_i . O_i with O_i the exact fp64 attention output (0 when none). */
+static void attn_row_stats(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                           const uint16_t* dO, int64_t bh, int64_t S, int d, const uint8_t* mask,
+                           double scale, int64_t i, double* lse_out, double* D_out) {
+    const int64_t nb = S / ORACLE_BLOCK;
+    const uint8_t* mrow = mask + (bh * nb + i / ORACLE_BLOCK) * nb;
+    double m = -INFINITY;
+    for (int64_t j = 0; j < S; ++j) {
+        if (!mrow[j / ORACLE_BLOCK]) continue;
+        double dot = 0.0;
+        for (int c = 0; c < d; ++c)
+            dot += bf16_to_f64(q[(bh * S + i) * d + c]) * bf16_to_f64(k[(bh * S + j) * d + c]);
+        if (scale * dot > m) m = scale * dot;
+    }
+    if (m == -INFINITY) { *lse_out = -INFINITY; *D_out = 0.0; return; }
+    double l = 0.0, D = 0.0;
+    for (int64_t j = 0; j < S; ++j) {
+        if (!mrow[j / ORACLE_BLOCK]) continue;
+        double dot = 0.0, dv = 0.0;
+        for (int c = 0; c < d; ++c) {
+            dot += bf16_to_f64(q[(bh * S + i) * d + c]) * bf16_to_f64(k[(bh * S + j) * d + c]);
+            dv += bf16_to_f64(dO[(bh * S + i) * d + c]) * bf16_to_f64(v[(bh * S + j) * d + c]);
+        }
+        double w = exp(scale * dot - m);
+        l += w;
+        D += w * dv;   /* sum_j p_ij (dO_i . v_j) = dO_i . O_i, up to the 1/l below */
+    }
+    *lse_out = m + log(l);
+    *D_out = D / l;
+}
+
+/* Backward of block-masked softmax attention (FlashAttention's backward: the
+ * probabilities are recomputed from the forward's log-sum-exp; the mask is
+ * the one the forward used).  For kept (i, j), p_ij = exp(scale q_i.k_j -
+ * lse_i), dP_ij = dO_i.v_j, dS_ij = p_ij (dP_ij - D_i) with D_i = dO_i.O_i:
+ *   dQ_i = scale sum_j dS_ij k_j,  dK_j = scale sum_i dS_ij q_i,  dV_j = sum_i p_ij dO_i.
+ * qrows (nq global row ids bh*S + i; NULL = every row) select the dQ rows,
+ * krows (nk ids bh*S + j; NULL = every key) the dK, dV rows; outputs fp64
+ * [nq, d] and [nk, d].  Inputs q, k, v, dO are bf16 bits [BH, S, d]. */
+void oracle_attention_bwd(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                          const uint16_t* dO, int64_t BH, int64_t S, int d, const uint8_t* mask,
+                          double scale, int64_t nq, const int64_t* qrows, double* dQ, int64_t nk,
+                          const int64_t* krows, double* dK, double* dV) {
+    const int64_t nb = S / ORACLE_BLOCK;
+    if (qrows == NULL) nq = BH * S;
+    if (krows == NULL) nk = BH * S;
+#pragma omp parallel for schedule(dynamic)
+    for (int64_t n = 0; n < nq; ++n) {
+        const int64_t g = qrows ? qrows[n] : n, bh = g / S, i = g % S;
+        double lse, D;
+        attn_row_stats(q, k, v, dO, bh, S, d, mask, scale, i, &lse, &D);
+        for (int c = 0; c < d; ++c) dQ[n * d + c] = 0.0;
+        if (lse == -INFINITY) continue;
+        const uint8_t* mrow = mask + (bh * nb + i / ORACLE_BLOCK) * nb;
+        for (int64_t j = 0; j < S; ++j) {
+            if (!mrow[j / ORACLE_BLOCK]) continue;
+            double dot = 0.0, dp = 0.0;
+            for (int c = 0; c < d; ++c) {
+                dot += bf16_to_f64(q[(bh * S + i) * d + c]) * bf16_to_f64(k[(bh * S + j) * d + c]);
+                dp += bf16_to_f64(dO[(bh * S + i) * d + c]) * bf16_to_f64(v[(bh * S + j) * d + c]);
+            }
+            double p = exp(scale * dot - lse);
+            double ds = p * (dp - D);
+            for (int c = 0; c < d; ++c) dQ[n * d + c] += scale * ds * bf16_to_f64(k[(bh * S + j) * d + c]);
+        }
+    }
+    if (nk == 0) return;
+    /* row statistics of every query row of every head */
+    double* lse_all = (double*)malloc(sizeof(double) * (size_t)(BH * S));
+    double* D_all = (double*)malloc(sizeof(double) * (size_t)(BH * S));
+#pragma omp parallel for schedule(dynamic)
+    for (int64_t g = 0; g < BH * S; ++g)
+        attn_row_stats(q, k, v, dO, g / S, S, d, mask, scale, g % S, &lse_all[g], &D_all[g]);
+#pragma omp parallel for schedule(dynamic)
+    for (int64_t n = 0; n < nk; ++n) {
+        const int64_t g = krows ? krows[n] : n, bh = g / S, j = g % S;
+        for (int c = 0; c < d; ++c) { dK[n * d + c] = 0.0; dV[n * d + c] = 0.0; }
+        for (int64_t i = 0; i < S; ++i) {
+            if (!mask[(bh * nb + i / ORACLE_BLOCK) * nb + j / ORACLE_BLOCK]) continue;
+            const double lse = lse_all[bh * S + i];
+            double dot = 0.0, dp = 0.0;
+            for (int c = 0; c < d; ++c) {
+                dot += bf16_to_f64(q[(bh * S + i) * d + c]) * bf16_to_f64(k[(bh * S + j) * d + c]);
+                dp += bf16_to_f64(dO[(bh * S + i) * d + c]) * bf16_to_f64(v[(bh * S + j) * d + c]);
+            }
+            double p = exp(scale * dot - lse);
+            double ds = p * (dp - D_all[bh * S + i]);
+            for (int c = 0; c < d; ++c) {
+                dK[n * d + c] += scale * ds * bf16_to_f64(q[(bh * S + i) * d + c]);
+                dV[n * d + c] += p * bf16_to_f64(dO[(bh * S + i) * d + c]);
+            }
+        }
+    }
+    free(lse_all);
+    free(D_all);
+}
+
 /* Threads OpenMP will use (for reporting the CPU baseline's core count). */
 int oracle_max_threads(void) {
 #ifdef _OPENMP

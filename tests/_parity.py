@@ -76,3 +76,18 @@ def sample_rows(B, H, S, nblocks_per_head, rows_per_block, seed=0):
             rows = rng.choice(64, size=min(rows_per_block, 64), replace=False)
             out.extend((bh * S + r * 64 + rows).tolist())
     return np.array(sorted(out), dtype=np.int64)
+
+
+def rows_with_same_mask(rows, gpu_mask, ora_mask, S, min_frac=0.95):
+    """The oracle computes attention with its own mask only; the GPU layer ran
+    with the GPU's mask.  Keep the sampled rows whose query block has the same
+    mask row on both sides (the rest differ only at near-cut rows, which the
+    mask tests check) and require that most of them do."""
+    nb = S // 64
+    g = gpu_mask.reshape(-1, nb)
+    o = ora_mask.reshape(-1, nb)
+    same = (g == o).all(axis=1)
+    blk = (rows // S) * nb + (rows % S) // 64
+    keep = same[blk]
+    assert keep.mean() >= min_frac, f"only {keep.mean():.3f} of sampled rows share a mask row"
+    return rows[keep]

@@ -1,9 +1,11 @@
-"""Block-sparse attention forward on the GPU vs the fp64 oracle fed the GPU's
-own mask: bf16 O within max-abs 2e-2 / mean-abs 2e-3, fp32 LSE within 1e-3."""
+"""Block-sparse attention forward on the GPU vs the fp64 oracle: bf16 O within
+max-abs 2e-2 / mean-abs 2e-3, fp32 LSE within 1e-3.  The oracle always uses
+its own mask (or a host-made static mask); for the composed NABLA layer the
+rows compared are those whose mask row the GPU and the oracle agree on."""
 import numpy as np
 import pytest
 
-from _parity import compare_attention, sample_rows, to_device_bf16
+from _parity import compare_attention, rows_with_same_mask, sample_rows, to_device_bf16
 
 pytestmark = pytest.mark.gpu
 
@@ -37,8 +39,9 @@ def _nabla_layer(nl, w, q, k, v, thr=None, sta="cfg"):
 def test_attention_parity_all_rows(nl, oracle_mod, synth_mod, name):
     w = synth_mod.WORKLOADS[name]
     q, k, v = synth_mod.make_qkv(w)
-    o, lse, mask = _nabla_layer(nl, w, q, k, v)
-    rows = np.arange(w.B * w.H * w.S, dtype=np.int64)
+    o, lse, gmask = _nabla_layer(nl, w, q, k, v)
+    mask = oracle_mod.build_mask(q, k, w.tile_grid, w.thr, w.sta)
+    rows = rows_with_same_mask(np.arange(w.B * w.H * w.S, dtype=np.int64), gmask, mask, w.S)
     ro, rl = oracle_mod.masked_attention(q, k, v, mask, rows)
     go, gl = _gather(o, lse, rows, w.S)
     mx, mean = compare_attention(go, gl, ro, rl)
@@ -49,8 +52,9 @@ def test_attention_parity_all_rows(nl, oracle_mod, synth_mod, name):
 def test_attention_parity_full_size(nl, oracle_mod, synth_mod, name):
     w = synth_mod.WORKLOADS[name]
     q, k, v = synth_mod.make_qkv(w)
-    o, lse, mask = _nabla_layer(nl, w, q, k, v)
-    rows = sample_rows(w.B, w.H, w.S, 2, 8, seed=1)
+    o, lse, gmask = _nabla_layer(nl, w, q, k, v)
+    mask = oracle_mod.build_mask(q, k, w.tile_grid, w.thr, w.sta)
+    rows = rows_with_same_mask(sample_rows(w.B, w.H, w.S, 2, 8, seed=1), gmask, mask, w.S)
     ro, rl = oracle_mod.masked_attention(q, k, v, mask, rows)
     go, gl = _gather(o, lse, rows, w.S)
     mx, mean = compare_attention(go, gl, ro, rl)

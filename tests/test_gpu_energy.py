@@ -1,7 +1,7 @@
 """Block energy and calibrated static masks on the GPU vs the fp64 oracle.
 
-Energy: both sides get the same fp32 LSE (from the GPU's dense forward); the
-GPU's S = QK^T is a bf16 MMA with fp32 accumulation, exp2 is approximate and
+Energy: both sides get the same fp32 LSE, computed by the oracle (its fp64
+attention LSE rounded to fp32); the GPU's S = QK^T is a bf16 MMA with fp32 accumulation, exp2 is approximate and
 the sums are fp32, so E agrees to a relative 2e-4 (every term is positive, so
 the relative error of a block sum is at most the largest relative error of its
 terms).  Calibration votes are integers: bit-exact except rows whose cut sits
@@ -49,6 +49,16 @@ def _dense_lse(nl, qd, kd, vd):
     return lse
 
 
+def _oracle_lse(oracle_mod, q, k, v, mask=None):
+    """fp64 oracle LSE [B,H,S] rounded to fp32 (dense when mask is None)."""
+    B, H, S, _ = q.shape
+    if mask is None:
+        _, lse = oracle_mod.dense_attention(q, k, v)
+    else:
+        _, lse = oracle_mod.masked_attention(q, k, v, mask)
+    return lse.astype(np.float32).reshape(B, H, S)
+
+
 def _gpu_energy(nl, qd, kd, lse, mask):
     B, H, S, d = qd.shape
     rp, ci = _csr(mask)
@@ -71,9 +81,10 @@ def test_energy_parity_dense_and_nabla_lists(nl, oracle_mod, synth_mod, name):
         q, k, v = q[:, :2].copy(), k[:, :2].copy(), v[:, :2].copy()
     B, H, S, d = q.shape
     nb = S // 64
-    qd, kd, vd = to_device_bf16(q), to_device_bf16(k), to_device_bf16(v)
-    lse = _dense_lse(nl, qd, kd, vd)
-    lse_h = lse.cpu().numpy()
+    import torch
+    qd, kd = to_device_bf16(q), to_device_bf16(k)
+    lse_h = _oracle_lse(oracle_mod, q, k, v)
+    lse = torch.from_numpy(lse_h).cuda()
     full = np.ones((B, H, nb, nb), dtype=np.uint8)
     E, mass = _gpu_energy(nl, qd, kd, lse, full)
     ref, ref_mass = oracle_mod.block_energy(q, k, lse_h, full)
@@ -98,7 +109,7 @@ def test_energy_edge_cases(nl, oracle_mod, synth_mod, B, H, nb, d):
     import torch
     S = 64 * nb
     q, k, v = _random_qkv(synth_mod, B, H, S, d, seed=40 + nb)
-    qd, kd, vd = to_device_bf16(q), to_device_bf16(k), to_device_bf16(v)
+    qd, kd = to_device_bf16(q), to_device_bf16(k)
     rng = np.random.default_rng(nb)
     mask = (rng.random((B, H, nb, nb)) < 0.4).astype(np.uint8)
     mask[..., 0, :] = 0
@@ -107,11 +118,9 @@ def test_energy_edge_cases(nl, oracle_mod, synth_mod, B, H, nb, d):
         mask[..., 1, nb - 1] = 1
     if nb > 2:
         mask[..., 2, :] = 1
-    # LSE of the masked forward: row block 0 is empty (LSE = -inf)
-    ws = nl.Workspace.create(nl.make_shape(B, H, S, d), nl.OP_FWD_WITH_MASK)
-    _, lse = nl.bsa_fwd_with_mask(qd, kd, vd, torch.from_numpy(mask).cuda(), workspace=ws)
-    assert ws.query_status() == 0
-    lse_h = lse.cpu().numpy()
+    # the mask's own LSE: row block 0 is empty (LSE = -inf)
+    lse_h = _oracle_lse(oracle_mod, q, k, v, mask)
+    lse = torch.from_numpy(lse_h).cuda()
     E, mass = _gpu_energy(nl, qd, kd, lse, mask)
     ref, ref_mass = oracle_mod.block_energy(q, k, lse_h, mask)
     np.testing.assert_allclose(E, ref, rtol=E_RTOL, atol=0)
@@ -122,8 +131,9 @@ def test_energy_edge_cases(nl, oracle_mod, synth_mod, B, H, nb, d):
 
 
 def test_energy_full_size_wan_sampled_rows(nl, oracle_mod, synth_mod):
-    """Wan 720p layer, dense block list: every row of E sums to 1 (any size),
-    and sampled rows agree with the oracle."""
+    """Wan 720p layer, dense block list: with the GPU's own dense LSE every row
+    of E sums to 1 (a property at any size); sampled block rows, whose LSE
+    entries are replaced by the oracle's, agree with the oracle."""
     import torch
     w = synth_mod.WORKLOADS["wan720p"]
     q, k, v = synth_mod.make_qkv(w)
@@ -131,6 +141,15 @@ def test_energy_full_size_wan_sampled_rows(nl, oracle_mod, synth_mod):
     lse = _dense_lse(nl, qd, kd, vd)
     nb = w.nb
     BH = w.B * w.H
+    rng = np.random.default_rng(7)
+    rows = np.sort(rng.choice(BH * nb, 6, replace=False)).astype(np.int64)
+    tok = ((rows // nb) * w.S + (rows % nb) * 64)[:, None] + np.arange(64)[None, :]
+    _, ora_lse = oracle_mod.dense_attention(q, k, v, tok.reshape(-1))
+    lse_flat = lse.reshape(-1)
+    lse_flat[torch.from_numpy(tok.reshape(-1)).cuda()] = torch.from_numpy(
+        ora_lse.astype(np.float32)).cuda()
+    lse_sampled = np.full(BH * w.S, np.nan)          # the oracle reads only the sampled rows
+    lse_sampled[tok.reshape(-1)] = ora_lse.astype(np.float32)
     row_ptr = torch.arange(0, BH * nb + 1, dtype=torch.int64, device="cuda").mul_(nb).to(torch.int32)
     col_idx = torch.arange(nb, dtype=torch.int32, device="cuda").repeat(BH * nb)
     ws = nl.Workspace.create(nl.make_shape(w.B, w.H, w.S, w.d), nl.OP_FWD)
@@ -138,10 +157,8 @@ def test_energy_full_size_wan_sampled_rows(nl, oracle_mod, synth_mod):
     assert ws.query_status() == 0
     m = mass.cpu().numpy()
     assert np.abs(m - 1.0).max() < 2e-3
-    rng = np.random.default_rng(7)
-    rows = np.sort(rng.choice(BH * nb, 6, replace=False)).astype(np.int64)
     full = np.ones((w.B, w.H, nb, nb), dtype=np.uint8)
-    ref, _ = oracle_mod.block_energy(q, k, lse.cpu().numpy(), full, rows=rows)
+    ref, _ = oracle_mod.block_energy(q, k, lse_sampled.reshape(w.B, w.H, w.S), full, rows=rows)
     got = E.reshape(-1, nb)[torch.from_numpy(rows).cuda()].cpu().numpy()
     np.testing.assert_allclose(got, ref, rtol=E_RTOL, atol=0)
 
@@ -188,8 +205,9 @@ def test_calibration_votes_and_mask_parity(nl, oracle_mod):
 
 def test_calibration_pipeline_to_static_mask_attention(nl, oracle_mod, synth_mod):
     """Two calibration runs (different seeds) of the tiny layer: dense LSE ->
-    block energy -> votes -> static mask -> masked attention, every stage
-    against the oracle on the GPU's own intermediate inputs."""
+    block energy -> votes -> static mask -> masked attention.  Each GPU stage
+    runs on the oracle's result of the stage before (the oracle never reads a
+    GPU result), and is compared with the oracle's result of that stage."""
     import torch
     from _parity import compare_attention
     w = synth_mod.WORKLOADS["tiny"]
@@ -200,15 +218,19 @@ def test_calibration_pipeline_to_static_mask_attention(nl, oracle_mod, synth_mod
     full = np.ones((w.B, w.H, nb, nb), dtype=np.uint8)
     for seed in (0, 1):
         q, k, v = synth_mod.make_qkv(w, seed=seed)
-        qd, kd, vd = to_device_bf16(q), to_device_bf16(k), to_device_bf16(v)
-        lse = _dense_lse(nl, qd, kd, vd)
-        E, _ = _gpu_energy(nl, qd, kd, lse, full)
-        assert not _exempt_rows(oracle_mod, E, eps).any()
-        nl.nabla_calib_accumulate(torch.from_numpy(E).cuda(), eps, votes)
-        oracle_mod.calib_accumulate(E.astype(np.float64), eps, votes_o)
+        qd, kd = to_device_bf16(q), to_device_bf16(k)
+        lse_h = _oracle_lse(oracle_mod, q, k, v)
+        E, _ = _gpu_energy(nl, qd, kd, torch.from_numpy(lse_h).cuda(), full)
+        E_o, _ = oracle_mod.block_energy(q, k, lse_h, full)
+        np.testing.assert_allclose(E, E_o, rtol=E_RTOL, atol=0)
+        E_o32 = E_o.astype(np.float32)
+        assert not _exempt_rows(oracle_mod, E_o32, eps).any()
+        nl.nabla_calib_accumulate(torch.from_numpy(E_o32).cuda(), eps, votes)
+        oracle_mod.calib_accumulate(E_o32.astype(np.float64), eps, votes_o)
     np.testing.assert_array_equal(votes.cpu().numpy(), votes_o)
     mask = nl.nabla_calib_finalize(votes, 1)
-    mask_h = mask.cpu().numpy()
+    mask_h = oracle_mod.calib_finalize(votes_o, 1)
+    np.testing.assert_array_equal(mask.cpu().numpy(), mask_h)
     assert 0 < mask_h.sum() < mask_h.size
     q, k, v = synth_mod.make_qkv(w, seed=2)         # inference on a new input
     qd, kd, vd = to_device_bf16(q), to_device_bf16(k), to_device_bf16(v)

@@ -5,7 +5,7 @@ the same context computes correct results."""
 import numpy as np
 import pytest
 
-from _parity import compare_attention, sample_rows, to_device_bf16
+from _parity import compare_attention, rows_with_same_mask, sample_rows, to_device_bf16
 
 pytestmark = pytest.mark.gpu
 
@@ -27,8 +27,10 @@ def test_wait_limit_reports_timeout_and_context_survives(oracle_mod, synth_mod):
         nl.set_wait_limit_ns(0)
     o, lse = nl.bsa_fwd(qd, kd, vd, row_ptr, col_idx, workspace=ws)
     assert ws.query_status() == 0
-    rows = sample_rows(w.B, w.H, w.S, 4, 16, seed=9)
-    ro, rl = oracle_mod.masked_attention(q, k, v, mask.cpu().numpy(), rows)
+    ora_mask = oracle_mod.build_mask(q, k, w.tile_grid, w.thr, w.sta)
+    rows = rows_with_same_mask(sample_rows(w.B, w.H, w.S, 4, 16, seed=9), mask.cpu().numpy(),
+                               ora_mask, w.S)
+    ro, rl = oracle_mod.masked_attention(q, k, v, ora_mask, rows)
     go = o.float().cpu().numpy().reshape(-1, w.d)[rows]
     gl = lse.cpu().numpy().reshape(-1)[rows]
     compare_attention(go, gl, ro, rl)

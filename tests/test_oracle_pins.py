@@ -601,3 +601,85 @@ def test_calib_scale_invariance_and_zero_rows(oracle_mod):
     full = np.zeros(e.shape, dtype=np.int32)
     oracle_mod.calib_accumulate(e, 0.0, full)      # eps = 0 keeps every block of a live row
     assert full[0, 0, 5].sum() == 0 and (np.delete(full[0, 0], 5, axis=0) == 1).all()
+
+
+# ---------------------------------------------------------------------------
+# Backward of block-masked attention
+
+
+def _torch_masked_attention_grads(q, k, v, dO, mask, scale=None):
+    """fp64 torch autograd of O = softmax(scale QK^T, kept blocks) V; rows with
+    no kept block give O = 0 and carry no gradient."""
+    import torch
+    B, H, S, d = q.shape
+    nb = S // 64
+    tq, tk, tv = (torch.from_numpy(_f(a)).requires_grad_(True) for a in (q, k, v))
+    tdo = torch.from_numpy(_f(dO))
+    keep = torch.from_numpy(np.repeat(np.repeat(mask.astype(bool), 64, axis=2), 64, axis=3))
+    live = keep.any(dim=-1, keepdim=True)
+    s = torch.einsum("bhid,bhjd->bhij", tq, tk) * (scale if scale else 1.0 / math.sqrt(d))
+    s = torch.where(keep, s, torch.full_like(s, -math.inf))
+    s = torch.where(live, s, torch.zeros_like(s))          # empty rows: finite, then zeroed
+    p = torch.softmax(s, dim=-1) * live
+    o = torch.einsum("bhij,bhjd->bhid", p, tv)
+    (o * tdo).sum().backward()
+    return tq.grad.numpy(), tk.grad.numpy(), tv.grad.numpy()
+
+
+def test_attention_bwd_matches_torch_autograd(oracle_mod):
+    rng = np.random.default_rng(31)
+    B, H, S, d = 1, 2, 320, 64
+    nb = S // 64
+    q, k, v, dO = (_rand_bits(rng, (B, H, S, d), sc) for sc in (0.7, 0.7, 1.0, 1.0))
+    mask = (rng.random((B, H, nb, nb)) < 0.5).astype(np.uint8)
+    mask[..., np.arange(nb), np.arange(nb)] = 1
+    mask[0, 1, 3, :] = 0                                   # one empty query block
+    gq, gk, gv = _torch_masked_attention_grads(q, k, v, dO, mask)
+    dQ, dK, dV = oracle_mod.attention_bwd(q, k, v, dO, mask)
+    for got, want in ((dQ, gq), (dK, gk), (dV, gv)):
+        np.testing.assert_allclose(got, want.reshape(-1, d), rtol=1e-9, atol=1e-12)
+    assert np.all(dQ.reshape(B, H, S, d)[0, 1, 192:256] == 0)
+
+
+def test_attention_bwd_invariants(oracle_mod):
+    # sum_j dS_ij = 0 for every row, so dK summed over a head's keys vanishes;
+    # sum_j p_ij = 1, so dV summed over keys equals dO summed over live rows
+    rng = np.random.default_rng(32)
+    B, H, S, d = 1, 1, 256, 64
+    nb = S // 64
+    q, k, v, dO = (_rand_bits(rng, (B, H, S, d)) for _ in range(4))
+    mask = (rng.random((B, H, nb, nb)) < 0.6).astype(np.uint8)
+    mask[0, 0, 2, :] = 0
+    mask[0, 0, 0, 0] = 1
+    dQ, dK, dV = oracle_mod.attention_bwd(q, k, v, dO, mask)
+    live_rows = np.repeat(mask[0, 0].any(axis=1), 64)
+    np.testing.assert_allclose(dK.sum(axis=0), 0.0, atol=1e-10)
+    np.testing.assert_allclose(dV.sum(axis=0), _f(dO)[0, 0][live_rows].sum(axis=0), atol=1e-10)
+    # uniform attention (q = 0): p = 1/n over the n kept keys of a row
+    q0 = np.zeros_like(q)
+    _, _, dV0 = oracle_mod.attention_bwd(q0, k, v, dO, mask)
+    n_kept = 64 * mask[0, 0].sum(axis=1)                    # keys per query block
+    want = np.zeros((S, d))
+    for r in range(nb):
+        if n_kept[r] == 0:
+            continue
+        g = _f(dO)[0, 0, 64 * r:64 * (r + 1)].sum(axis=0) / n_kept[r]
+        for c in np.nonzero(mask[0, 0, r])[0]:
+            want[64 * c:64 * (c + 1)] += g
+    np.testing.assert_allclose(dV0, want, atol=1e-12)
+
+
+def test_attention_bwd_row_subsets(oracle_mod):
+    rng = np.random.default_rng(33)
+    B, H, S, d = 2, 1, 192, 64
+    q, k, v, dO = (_rand_bits(rng, (B, H, S, d)) for _ in range(4))
+    mask = (rng.random((B, H, 3, 3)) < 0.7).astype(np.uint8)
+    dQ, dK, dV = oracle_mod.attention_bwd(q, k, v, dO, mask)
+    qr = np.array([5, 300, 191], dtype=np.int64)
+    kr = np.array([0, 250], dtype=np.int64)
+    sq, sk, sv = oracle_mod.attention_bwd(q, k, v, dO, mask, qrows=qr, krows=kr)
+    np.testing.assert_array_equal(sq, dQ[qr])
+    np.testing.assert_array_equal(sk, dK[kr])
+    np.testing.assert_array_equal(sv, dV[kr])
+    eq, ek, ev = oracle_mod.attention_bwd(q, k, v, dO, mask, qrows=qr, krows=np.empty(0, np.int64))
+    assert ek.shape == (0, d) and np.array_equal(eq, dQ[qr])
