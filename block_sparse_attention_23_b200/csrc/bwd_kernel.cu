@@ -63,8 +63,8 @@ struct BwdSmem {
   static constexpr uint32_t kOffY = 2 * kTile;                     // [stage][Y1, Y2]
   static constexpr uint32_t kOffVec = kOffY + kBStages * 2 * kTile;   // [stage][lse | D][128] fp32
   static constexpr uint32_t kVecBytes = 2 * kBT * 4;
-  static constexpr uint32_t kOffBar = kOffVec + kBStages * kVecBytes;  // 16 mbarriers
-  static constexpr uint32_t kOffMisc = kOffBar + 128;
+  static constexpr uint32_t kOffBar = kOffVec + kBStages * kVecBytes;  // 32 mbarriers
+  static constexpr uint32_t kOffMisc = kOffBar + 256;
   static constexpr uint32_t kOffBitmap = kOffMisc + 64;            // [2][kBMaxNb/32]
   static constexpr uint32_t kOffList = kOffBitmap + 2 * (kBMaxNb / 32) * 4;
   static constexpr uint32_t kBytes = kOffList + kBMaxNb * 4;
@@ -75,14 +75,17 @@ enum : int {
   kBBarXFull = 0,
   kBBarYFull = 1,                          // + stage
   kBBarYEmpty = kBBarYFull + kBStages,     // + stage
-  kBBarSFull = kBBarYEmpty + kBStages,     // MMA1 + MMA2 of the tile done
-  kBBarPFull = kBBarSFull + 1,             // elementwise results written
-  kBBarAccFull = kBBarPFull + 1,           // every accumulating MMA done
+  kBBarSFull = kBBarYEmpty + kBStages,     // MMA1 (S or S^T) done
+  kBBarDPFull = kBBarSFull + 1,            // MMA2 (dP or dP^T) done
+  kBBarSDone = kBBarDPFull + 1,            // key-stationary: P^T written; query-stationary: S read
+  kBBarDSReady = kBBarSDone + 1,           // dS (dS^T) written
+  kBBarAccFull = kBBarDSReady + 1,         // every accumulating MMA done
   kBBarDrain = kBBarAccFull + 1,
-  kBBarLoaded = kBBarDrain + 1,            // + lane quarter: both column halves loaded
-  kBNumBars = kBBarLoaded + 4
+  kBBarPairS = kBBarDrain + 1,             // + lane quarter: both S halves loaded
+  kBBarPairDP = kBBarPairS + 4,            // + lane quarter: both dP halves loaded
+  kBNumBars = kBBarPairDP + 4
 };
-static_assert(kBNumBars * 8 <= 128, "barrier area");
+static_assert(kBNumBars * 8 <= 256, "barrier area");
 
 struct BwdParams {
   const int32_t* row_ptr;      // CSR (query-stationary) or unused
@@ -176,7 +179,6 @@ __global__ void __launch_bounds__(kBThreads, 1)
   const uint32_t sX = base + L::kOffX;
   const uint32_t sY = base + L::kOffY;
   const uint32_t sVec = base + L::kOffVec;
-  const float* vec = reinterpret_cast<const float*>(gbase + L::kOffVec);
   const uint32_t bar0 = base + L::kOffBar;
   uint32_t* misc = reinterpret_cast<uint32_t*>(gbase + L::kOffMisc);
   volatile uint32_t* tmem_holder = misc;
@@ -201,10 +203,15 @@ __global__ void __launch_bounds__(kBThreads, 1)
       mbar_init(bar(kBBarYEmpty + s), 1);
     }
     mbar_init(bar(kBBarSFull), 1);
-    mbar_init(bar(kBBarPFull), kBEwWarps * 32);
+    mbar_init(bar(kBBarDPFull), 1);
+    mbar_init(bar(kBBarSDone), kBEwWarps * 32);
+    mbar_init(bar(kBBarDSReady), kBEwWarps * 32);
     mbar_init(bar(kBBarAccFull), 1);
     mbar_init(bar(kBBarDrain), 1);
-    for (int qd = 0; qd < 4; ++qd) mbar_init(bar(kBBarLoaded + qd), 64);
+    for (int qd = 0; qd < 4; ++qd) {
+      mbar_init(bar(kBBarPairS + qd), 64);
+      mbar_init(bar(kBBarPairDP + qd), 64);
+    }
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -321,48 +328,93 @@ __global__ void __launch_bounds__(kBThreads, 1)
     }
   } else if (warp == kBMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
+    // key-stationary, per tile: wait P^T -> dV += P^T dO, S^T(t+1) | wait dS^T
+    //   -> dK += dS^T Q, dP^T(t+1).  dP^T runs under the exponentials, dV and
+    //   the next S^T under the dS^T pass; each product that overwrites a
+    //   tensor-memory operand is issued after the product that reads it.
+    // query-stationary: S(t+1) is issued once the elementwise warps have read
+    //   S(t), so it runs under the dS(t) pass; dS goes over dP, which dP(t+1)
+    //   overwrites only after dQ(t) (issued first) has read it.
     if (lane == 0 && n_t > 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(kBT, kBT, false);
       constexpr uint32_t idesc_acc = idesc_bf16_f32(kBT, D, true);
-      bool ok = mbar_wait(bar(kBBarXFull), 0, lim, abort_flag);
-      int t = 0;
-      for (; ok && t < n_t; ++t) {
-        const int s = t % kBStages;
-        if (!mbar_wait(bar(kBBarYFull + s), (t / kBStages) & 1, lim, abort_flag)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t y1 = sY + s * 2 * L::kTile, y2 = y1 + L::kTile;
+      auto stage_y1 = [&](int t) { return sY + (t % kBStages) * 2 * L::kTile; };
+      auto issue_ss = [&](uint32_t dcol, uint32_t xa, uint32_t yb) {
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * (kBT * 128) + (kk & 3) * 32;
-          tc_mma_ss(tmem + kColS, sdesc_sw128(sX + off, 16, 1024), sdesc_sw128(y1 + off, 16, 1024),
+          tc_mma_ss(tmem + dcol, sdesc_sw128(xa + off, 16, 1024), sdesc_sw128(yb + off, 16, 1024),
                     idesc_s, kk > 0 ? 1u : 0u);
         }
+      };
+      // acc += (tensor-memory operand at acol) x (streaming tile yb, MN-major):
+      // 16 streaming rows per step, packed bf16 columns [8kk, 8kk+8)
+      auto issue_ts = [&](uint32_t dcol, uint32_t acol, uint32_t yb, bool first) {
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * (kBT * 128) + (kk & 3) * 32;
-          tc_mma_ss(tmem + kColDP, sdesc_sw128(sX + L::kTile + off, 16, 1024),
-                    sdesc_sw128(y2 + off, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
+        for (int kk = 0; kk < kBT / 16; ++kk)
+          tc_mma_ts(tmem + dcol, tmem + acol + kk * 8, sdesc_sw128(yb + kk * 16 * 128, kBT * 128, 1024),
+                    idesc_acc, (!first || kk > 0) ? 1u : 0u);
+      };
+      auto wait_y = [&](int t) {
+        return mbar_wait(bar(kBBarYFull + t % kBStages), (t / kBStages) & 1, lim, abort_flag);
+      };
+      bool ok = mbar_wait(bar(kBBarXFull), 0, lim, abort_flag);
+      if (kKV) {
+        if (ok && !wait_y(0)) ok = false;
+        if (ok) {
+          tc_fence_after();
+          issue_ss(kColS, sX, stage_y1(0));                         // S^T(0) = K Q^T
+          tc_commit(bar(kBBarSFull));
+          issue_ss(kColDP, sX + L::kTile, stage_y1(0) + L::kTile);  // dP^T(0) = V dO^T
+          tc_commit(bar(kBBarDPFull));
         }
-        tc_commit(bar(kBBarSFull));
-        if (!mbar_wait(bar(kBBarPFull), t & 1, lim, abort_flag)) { ok = false; break; }
-        tc_fence_after();
-        // 16 streaming rows per step: packed bf16 columns [8kk, 8kk+8) of the
-        // elementwise result, rows [16kk, 16kk+16) of the streaming tile read
-        // MN-major (the 64-column halves of d are kBT*128 bytes apart)
-#pragma unroll
-        for (int kk = 0; kk < kBT / 16; ++kk) {
-          const uint32_t acc = (t > 0 || kk > 0) ? 1u : 0u;
-          if (kKV) {
-            tc_mma_ts(tmem + kColAcc, tmem + kColS + kk * 8,
-                      sdesc_sw128(y2 + kk * 16 * 128, kBT * 128, 1024), idesc_acc, acc);   // dV += P^T dO
-            tc_mma_ts(tmem + kColAcc + D, tmem + kColDP + kk * 8,
-                      sdesc_sw128(y1 + kk * 16 * 128, kBT * 128, 1024), idesc_acc, acc);   // dK += dS^T Q
-          } else {
-            tc_mma_ts(tmem + kColAcc, tmem + kColS + kk * 8,
-                      sdesc_sw128(y1 + kk * 16 * 128, kBT * 128, 1024), idesc_acc, acc);   // dQ += dS K
+        for (int t = 0; ok && t < n_t; ++t) {
+          const bool more = t + 1 < n_t;
+          const uint32_t y1 = stage_y1(t), y2 = y1 + L::kTile;
+          if (!mbar_wait(bar(kBBarSDone), t & 1, lim, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          issue_ts(kColAcc, kColS, y2, t == 0);                     // dV += P^T dO
+          if (more) {   // S^T(t+1) overwrites P^T(t) after dV(t) has read it (issue order)
+            if (!wait_y(t + 1)) { ok = false; break; }
+            tc_fence_after();
+            issue_ss(kColS, sX, stage_y1(t + 1));
+            tc_commit(bar(kBBarSFull));
+          }
+          if (!mbar_wait(bar(kBBarDSReady), t & 1, lim, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          issue_ts(kColAcc + D, kColDP, y1, t == 0);                // dK += dS^T Q
+          tc_commit(bar(kBBarYEmpty + t % kBStages));
+          if (more) {   // dP^T(t+1) overwrites dS^T(t) after dK(t) has read it
+            issue_ss(kColDP, sX + L::kTile, stage_y1(t + 1) + L::kTile);
+            tc_commit(bar(kBBarDPFull));
           }
         }
-        tc_commit(bar(kBBarYEmpty + s));
+      } else {
+        if (ok && !wait_y(0)) ok = false;
+        if (ok) {
+          tc_fence_after();
+          issue_ss(kColS, sX, stage_y1(0));                       // S(0) = Q K^T
+          tc_commit(bar(kBBarSFull));
+          issue_ss(kColDP, sX + L::kTile, stage_y1(0) + L::kTile);  // dP(0) = dO V^T
+          tc_commit(bar(kBBarDPFull));
+        }
+        for (int t = 0; ok && t < n_t; ++t) {
+          const bool more = t + 1 < n_t;
+          if (more) {
+            if (!wait_y(t + 1) || !mbar_wait(bar(kBBarSDone), t & 1, lim, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            issue_ss(kColS, sX, stage_y1(t + 1));                 // S(t+1)
+            tc_commit(bar(kBBarSFull));
+          }
+          if (!mbar_wait(bar(kBBarDSReady), t & 1, lim, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          issue_ts(kColAcc, kColDP, stage_y1(t), t == 0);         // dQ += dS K
+          tc_commit(bar(kBBarYEmpty + t % kBStages));
+          if (more) {
+            issue_ss(kColDP, sX + L::kTile, stage_y1(t + 1) + L::kTile);   // dP(t+1)
+            tc_commit(bar(kBBarDPFull));
+          }
+        }
       }
       if (ok) tc_commit(bar(kBBarAccFull));
       else b_abort(abort_flag, prm.status);
@@ -391,62 +443,110 @@ __global__ void __launch_bounds__(kBThreads, 1)
       const int s = t % kBStages;
       const int e = tile_entry(t, half);
       const bool member = ((e >> (16 + x)) & 1) != 0;   // uniform per warp
+      // LSE and D of this entry's 64 queries (key-stationary), read as 16-byte vectors
+      const uint32_t vl_addr = sVec + s * L::kVecBytes + 64 * half * 4;
+      const uint32_t vd_addr = vl_addr + kBT * 4;
+      auto load32 = [&](uint32_t addr, float (&r)[32]) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const float4 f = lds_f4(addr + 16 * j);
+          r[4 * j] = f.x; r[4 * j + 1] = f.y; r[4 * j + 2] = f.z; r[4 * j + 3] = f.w;
+        }
+      };
+      // ---- S (S^T): probabilities, kept in registers
       if (!b_warp_wait(bar(kBBarSFull), t & 1, lim, abort_flag)) { ok = false; break; }
       tc_fence_after();
-      uint32_t sv[2][32], dv[2][32];
+      // query-stationary: P in fp32; key-stationary: P^T packed to bf16 (the
+      // values the dV product uses), which also feeds dS^T and keeps the
+      // thread's live registers below the split (a spill would go to L2:
+      // shared memory leaves almost no L1)
+      float p[kKV ? 1 : 64];
+      uint32_t pk[2][16];
+      {
+        uint32_t sv[2][32];
+        if (member) {
+          tmem_ld32(tb + kColS + 64 * half, sv[0]);
+          tmem_ld32(tb + kColS + 64 * half + 32, sv[1]);
+          tmem_ld_wait();
+        }
+        if (kKV) {
+          // P^T goes over S^T in place: both column halves of these rows
+          // must be in registers first (a bounded wait: the partner may have aborted)
+          mbar_arrive(bar(kBBarPairS + quarter));
+          if (!b_warp_wait(bar(kBBarPairS + quarter), t & 1, lim, abort_flag)) { ok = false; break; }
+        } else {
+          tc_fence_before();
+          mbar_arrive(bar(kBBarSDone));            // S(t) read: S(t+1) may be computed
+        }
+        if (kKV) {
+#pragma unroll
+          for (int ch = 0; ch < 2; ++ch) {
+            float lv[32];
+            load32(vl_addr + 128 * ch, lv);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              float e[2];
+#pragma unroll
+              for (int u = 0; u < 2; ++u)
+                e[u] = member ? fast_exp2(fmaf(__uint_as_float(sv[ch][2 * i + u]), sl2,
+                                               -lv[2 * i + u] * kL2e))
+                              : 0.f;
+              pk[ch][i] = pack_bf16x2(e[0], e[1]);
+            }
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < 64; ++c)
+            p[c & (kKV ? 0 : 63)] =
+                member ? fast_exp2(fmaf(__uint_as_float(sv[c >> 5][c & 31]), sl2, row_nlse2)) : 0.f;
+        }
+      }
+      if (kKV) {
+        tmem_st16(tb + kColS + 32 * half, pk[0]);
+        tmem_st16(tb + kColS + 32 * half + 16, pk[1]);
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(bar(kBBarSDone));              // P^T written: dV += P^T dO may run
+      }
+      // ---- dP (dP^T): dS = P o (dP - D), written over dP in place
+      if (!b_warp_wait(bar(kBBarDPFull), t & 1, lim, abort_flag)) { ok = false; break; }
+      tc_fence_after();
+      uint32_t dv[2][32];
       if (member) {
-        tmem_ld32(tb + kColS + 64 * half, sv[0]);
-        tmem_ld32(tb + kColS + 64 * half + 32, sv[1]);
         tmem_ld32(tb + kColDP + 64 * half, dv[0]);
         tmem_ld32(tb + kColDP + 64 * half + 32, dv[1]);
         tmem_ld_wait();
       }
-      // both column halves of these rows must be in registers before either
-      // warp overwrites them (a bounded wait: the partner may have aborted)
-      mbar_arrive(bar(kBBarLoaded + quarter));
-      if (!b_warp_wait(bar(kBBarLoaded + quarter), t & 1, lim, abort_flag)) { ok = false; break; }
-      const float* vl = vec + s * (L::kVecBytes / 4) + 64 * half;   // LSE of this entry's queries
-      const float* vd = vl + kBT;                                   // D of this entry's queries
+      mbar_arrive(bar(kBBarPairDP + quarter));
+      if (!b_warp_wait(bar(kBBarPairDP + quarter), t & 1, lim, abort_flag)) { ok = false; break; }
 #pragma unroll
       for (int ch = 0; ch < 2; ++ch) {
-        uint32_t pk[16], dk[16];
-        if (member) {
+        uint32_t dk[16];
+        float dvv[32];
+        if (kKV) load32(vd_addr + 128 * ch, dvv);
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            float p[2], ds[2];
+        for (int i = 0; i < 16; ++i) {
+          float ds[2];
 #pragma unroll
-            for (int u = 0; u < 2; ++u) {
-              const int c = ch * 32 + 2 * i + u;
-              float nl2, dd;
-              if (kKV) {
-                nl2 = -vl[c] * kL2e;
-                dd = vd[c];
-              } else {
-                nl2 = row_nlse2;
-                dd = row_d;
-              }
-              p[u] = fast_exp2(fmaf(__uint_as_float(sv[ch][2 * i + u]), sl2, nl2));
-              ds[u] = p[u] * (__uint_as_float(dv[ch][2 * i + u]) - dd);
+          for (int u = 0; u < 2; ++u) {
+            const int c = 32 * ch + 2 * i + u;
+            float pc, dd;
+            if (kKV) {
+              pc = __uint_as_float(u ? (pk[ch][i] & 0xFFFF0000u) : (pk[ch][i] << 16));
+              dd = dvv[2 * i + u];
+            } else {
+              pc = p[c & (kKV ? 0 : 63)];
+              dd = row_d;
             }
-            pk[i] = pack_bf16x2(p[0], p[1]);
-            dk[i] = pack_bf16x2(ds[0], ds[1]);
+            ds[u] = member ? pc * (__uint_as_float(dv[ch][2 * i + u]) - dd) : 0.f;
           }
-        } else {
-#pragma unroll
-          for (int i = 0; i < 16; ++i) pk[i] = dk[i] = 0u;
+          dk[i] = pack_bf16x2(ds[0], ds[1]);
         }
-        // packed columns [32 half + 16 ch, +16): P^T over S^T and dS^T over
-        // dP^T (key-stationary); dS over S (query-stationary)
-        if (kKV) {
-          tmem_st16(tb + kColS + 32 * half + 16 * ch, pk);
-          tmem_st16(tb + kColDP + 32 * half + 16 * ch, dk);
-        } else {
-          tmem_st16(tb + kColS + 32 * half + 16 * ch, dk);
-        }
+        tmem_st16(tb + kColDP + 32 * half + 16 * ch, dk);
       }
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(bar(kBBarPFull));
+      mbar_arrive(bar(kBBarDSReady));
     }
     if (!ok) b_abort(abort_flag, prm.status);
     // ------------------------------------------------------------ epilogue

@@ -276,6 +276,15 @@ __device__ __forceinline__ void setmaxnreg_dec() {
 
 // ----------------------------------------------------------------- misc
 
+// 16-byte shared-memory load (volatile: stays after the waits that precede it).
+__device__ __forceinline__ float4 lds_f4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(addr));
+  return v;
+}
+
 __device__ __forceinline__ float fast_exp2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
