@@ -472,8 +472,10 @@ __global__ void __launch_bounds__(kBThreads, 1)
         if (kKV) {
           // P^T goes over S^T in place: both column halves of these rows
           // must be in registers first (a bounded wait: the partner may have aborted)
+          tc_fence_before();
           mbar_arrive(bar(kBBarPairS + quarter));
           if (!b_warp_wait(bar(kBBarPairS + quarter), t & 1, lim, abort_flag)) { ok = false; break; }
+          tc_fence_after();
         } else {
           tc_fence_before();
           mbar_arrive(bar(kBBarSDone));            // S(t) read: S(t+1) may be computed
@@ -517,8 +519,10 @@ __global__ void __launch_bounds__(kBThreads, 1)
         tmem_ld32(tb + kColDP + 64 * half + 32, dv[1]);
         tmem_ld_wait();
       }
+      tc_fence_before();
       mbar_arrive(bar(kBBarPairDP + quarter));
       if (!b_warp_wait(bar(kBBarPairDP + quarter), t & 1, lim, abort_flag)) { ok = false; break; }
+      tc_fence_after();
 #pragma unroll
       for (int ch = 0; ch < 2; ++ch) {
         uint32_t dk[16];

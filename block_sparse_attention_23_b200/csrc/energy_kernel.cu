@@ -24,9 +24,11 @@
 // query block add their warp sums into a shared-memory row of E (exactly two
 // addends onto zero: the result does not depend on their order).
 //
-// Roles (192 threads): warps 0-3 exponentiate and sum, warp 4 compacts the
-// union list and issues the TMA loads, warp 5 owns tensor memory and issues
-// the MMAs.  Every mbarrier wait is time-bounded; a wait that runs out records
+// Roles (384 threads): warps 0-7 exponentiate and sum in two groups of four
+// (group g takes the tiles t = g mod 2 and the S buffer g, so two warps per
+// SM sub-partition keep the exponential unit busy), warp 8 compacts the union
+// list and issues the TMA loads, warp 9 owns tensor memory and issues the MMAs,
+// warps 10-11 idle.  Every mbarrier wait is time-bounded; a wait that runs out records
 // kStatusTimeout, raises the CTA's abort flag and the CTA drains its own work
 // before freeing tensor memory; an aborted CTA writes no output.
 #include <cuda.h>
@@ -40,9 +42,9 @@ namespace nabla {
 constexpr int kEM = 128;            // query rows per CTA (two blocks)
 constexpr int kEN = 128;            // keys per tile (two list entries)
 constexpr int kEStages = 3;         // K ring depth
-constexpr int kEThreads = 192;
-constexpr int kESumWarps = 4;
-constexpr int kEProducerWarp = 4, kEMmaWarp = 5;
+constexpr int kEThreads = 384;
+constexpr int kESumWarps = 8;                     // two groups of four, one per S buffer
+constexpr int kEProducerWarp = 8, kEMmaWarp = 9;
 constexpr int kEMaxNb = 4096;
 constexpr uint32_t kETmemCols = 256;
 constexpr uint64_t kEDrainNs = 1000000000ull;
@@ -138,7 +140,7 @@ __global__ void __launch_bounds__(kEThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(bar(kEBarSFull + b), 1);
-      mbar_init(bar(kEBarSFree + b), kESumWarps * 32);
+      mbar_init(bar(kEBarSFree + b), (kESumWarps / 2) * 32);
     }
     mbar_init(bar(kEBarDrain), 1);
     *abort_flag = 0;
@@ -245,7 +247,7 @@ __global__ void __launch_bounds__(kEThreads, 1)
       for (int t = 0; ok && t < n_t; ++t) {
         const int b = t & 1, s = t % kEStages;
         if (!mbar_wait(bar(kEBarKFull + s), (t / kEStages) & 1, lim, abort_flag)) { ok = false; break; }
-        // the S buffer is free once all four summing warps have loaded tile t-2
+        // the S buffer is free once its group of four warps has loaded tile t-2
         if (t >= 2 && !mbar_wait(bar(kEBarSFree + b), ((t >> 1) - 1) & 1, lim, abort_flag)) {
           ok = false;
           break;
@@ -266,12 +268,14 @@ __global__ void __launch_bounds__(kEThreads, 1)
       tc_commit(bar(kEBarDrain));
       mbar_wait(bar(kEBarDrain), 0, kEDrainNs, nullptr);
     }
-  } else {
+  } else if (warp < kESumWarps) {
     // ------------------------------------------------------------ exponentiate and sum
-    const int row = warp * 32 + lane;          // tile row == tensor-memory lane
+    const int grp = warp >> 2;                 // tiles t = grp mod 2, S buffer grp
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;       // tile row == tensor-memory lane
     const int qh = row >> 6;                   // query block r0 + qh (uniform per warp)
     const int bit = 1 << (16 + qh);
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const float sl2 = prm.scale_log2;
     float neg_lse2 = 0.f;
     bool live = false;
@@ -283,8 +287,8 @@ __global__ void __launch_bounds__(kEThreads, 1)
     }
     float* myE = rowE + qh * kEMaxNb;
     bool ok = true;
-    for (int t = 0; t < n_t; ++t) {
-      const int b = t & 1;
+    for (int t = grp; t < n_t; t += 2) {
+      const int b = grp;
       const int e0 = tile_entry(t, 0), e1 = tile_entry(t, 1);
       const bool v0 = (e0 & bit) != 0, v1 = (e1 & bit) != 0;   // uniform per warp
       if (!e_warp_wait(bar(kEBarSFull + b), (t >> 1) & 1, lim, abort_flag)) { ok = false; break; }
