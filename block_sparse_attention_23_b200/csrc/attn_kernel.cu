@@ -12,9 +12,8 @@
 //   One CTA per (b, h, group of four query blocks 4g..4g+3) = two query
 //   tiles of 128 rows: tile 0 = blocks 4g, 4g+1; tile 1 = blocks 4g+2, 4g+3.
 //   The key blocks visited are the union of the four CSR rows, each entry with
-//   a 4-bit membership mask, grouped by that mask.  Key tiles are 128 keys =
-//   two union entries (the second may be a repeat that every row masks); each
-//   entry is one contiguous
+//   a 4-bit membership mask.  Key tiles are 128 keys = two union entries (the
+//   second may be a repeat that every row masks); each entry is one contiguous
 //   64 x d slab of the [B,H,S,d] tensor, loaded as a plain 2D TMA box, so both
 //   query tiles share every K/V tile that is loaded.  A query tile computes a
 //   key tile only if one of its two blocks lists one of the tile's entries; a
@@ -209,38 +208,31 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
   __syncthreads();
-  if (warp == kProducerWarp) {
-    // Compact the union grouped by membership pattern (the 4-bit set of query
-    // blocks that list the entry), ascending within a pattern.  Key tiles pair
-    // consecutive entries, so equal patterns share tiles: fewer tiles carry
-    // blocks that only one query tile needs (1.12 -> 1.08 executed/kept tile
-    // products at the Wan 720p mask).  The order of key tiles does not change
-    // the result beyond rounding.
+  if (warp == kProducerWarp) {   // compact the union in ascending block order
     int run = 0;
-    for (int pat = 1; pat < 16; ++pat) {
-      for (int w0 = 0; w0 < nw; w0 += 32) {
-        const int w = w0 + lane;
-        uint32_t sel = w < nw ? 0xffffffffu : 0u;
+    for (int w0 = 0; w0 < nw; w0 += 32) {
+      const int w = w0 + lane;
+      uint32_t u[4];
 #pragma unroll
-        for (int qb = 0; qb < 4; ++qb) {
-          const uint32_t u = w < nw ? bm[qb * (kMaxNb / 32) + w] : 0u;
-          sel &= ((pat >> qb) & 1) ? u : ~u;
-        }
-        const int cnt = __popc(sel);
-        int incl = cnt;
+      for (int qb = 0; qb < 4; ++qb) u[qb] = w < nw ? bm[qb * (kMaxNb / 32) + w] : 0u;
+      uint32_t any = u[0] | u[1] | u[2] | u[3];
+      const int cnt = __popc(any);
+      int incl = cnt;
 #pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-          const int y = __shfl_up_sync(0xffffffffu, incl, off);
-          if (lane >= off) incl += y;
-        }
-        int pos = run + incl - cnt;
-        while (sel) {
-          const int b = __ffs(sel) - 1;
-          sel &= sel - 1;
-          ulist[pos++] = (w * 32 + b) | (pat << 16);
-        }
-        run += __shfl_sync(0xffffffffu, incl, 31);
+      for (int off = 1; off < 32; off <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += y;
       }
+      int pos = run + incl - cnt;
+      while (any) {
+        const int b = __ffs(any) - 1;
+        any &= any - 1;
+        int mem = 0;
+#pragma unroll
+        for (int qb = 0; qb < 4; ++qb) mem |= static_cast<int>((u[qb] >> b) & 1u) << qb;
+        ulist[pos++] = (w * 32 + b) | (mem << 16);
+      }
+      run += __shfl_sync(0xffffffffu, incl, 31);
     }
     if (lane == 0) *n_union_s = run;
   }
