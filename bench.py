@@ -341,6 +341,34 @@ def run_ours(args):
     re_gbs = re_bytes / (re_ms * 1e-3) / 1e9
     del qr
 
+    # the same layer on raster-ordered tokens, read in place (reorder fused into
+    # the pooling loads and the attention's TMA boxes and O / LSE stores)
+    qr, kr, vr = (nl.nabla_reorder_tokens(t, w.tile_grid, nl.TO_RASTER) for t in (q, k, v))
+    shape_r = nl.make_shape(B, H, S, d, w.tile_grid, nl.LAYOUT_RASTER)
+    ws_mask_r = nl.Workspace.create(shape_r, nl.OP_BUILD_MASK, dev)
+    ws_fwd_r = nl.Workspace.create(shape_r, nl.OP_FWD, dev)
+    o_r, lse_r = torch.empty_like(q), torch.empty_like(lse)
+
+    def raster_step():
+        rp, ci, _, _ = nl.nabla_build_mask(qr, kr, w.tile_grid, w.thr, w.sta, workspace=ws_mask_r,
+                                           out=mask_out, layout=nl.LAYOUT_RASTER)
+        nl.bsa_fwd(qr, kr, vr, rp, ci, workspace=ws_fwd_r, out=(o_r, lse_r), tile_grid=w.tile_grid,
+                   layout=nl.LAYOUT_RASTER)
+
+    for _ in range(2):
+        raster_step()
+    torch.cuda.synchronize()
+    n_ra = 3
+    a.record(stream)
+    for _ in range(n_ra):
+        raster_step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    ws_mask_r.check()
+    ws_fwd_r.check()
+    raster_ms = a.elapsed_time(b) / n_ra
+    del qr, kr, vr, o_r, lse_r
+
     # block energy over the step's own block list (the retained-mass check of
     # the NABLA mask) and one calibration vote pass over the energy map
     energy = torch.empty((B, H, nb, nb), dtype=torch.float32, device=dev)
@@ -453,6 +481,9 @@ def run_ours(args):
                 "unit": "TFLOP/s", "frac": bwd_tflops / peak, "flops": bwd_flops,
                 "what": "bsa_bwd (D, column bitmaps, dK/dV and dQ kernels) over the step's "
                         "block list, outside the step; FLOPs = 10*d*64*64 per kept block"},
+        "raster_layer": {"ms_per_layer": raster_ms, "vs_tile_major": raster_ms / ms_per_step,
+                         "what": "mask + attention on raster-ordered Q, K, V (O, LSE raster), "
+                                 "token reorder fused into the loads; outside the step"},
         "gpu_launches": 6 * args.steps,
         "clocks": clk,
     }

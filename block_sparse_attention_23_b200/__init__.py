@@ -28,6 +28,7 @@ STATUS_NAMES = {0: "NABLA_OK", 1: "NABLA_ERR_INVALID_ARG", 2: "NABLA_ERR_UNSUPPO
                 3: "NABLA_ERR_CAPACITY", 4: "NABLA_ERR_CUDA", 5: "NABLA_ERR_TIMEOUT",
                 6: "NABLA_ERR_BAD_INDEX"}
 OP_BUILD_MASK, OP_FWD, OP_FWD_WITH_MASK, OP_BWD = 0, 1, 2, 3
+LAYOUT_TILE_MAJOR, LAYOUT_RASTER = 0, 1
 EXPORTED = ["nabla_workspace_size", "nabla_workspace_init", "nabla_query_status",
             "nabla_build_mask", "bsa_fwd", "bsa_fwd_with_mask", "nabla_last_error",
             "nabla_version", "nabla_set_wait_limit_ns", "nabla_selftest_mma",
@@ -45,7 +46,7 @@ class NablaError(RuntimeError):
 class _Shape(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int32), ("H", ctypes.c_int32), ("S", ctypes.c_int32),
                 ("d", ctypes.c_int32), ("Tt", ctypes.c_int32), ("Th", ctypes.c_int32),
-                ("Tw", ctypes.c_int32)]
+                ("Tw", ctypes.c_int32), ("layout", ctypes.c_int32)]
 
 
 class _MaskParams(ctypes.Structure):
@@ -133,9 +134,10 @@ def _ptr(t) -> ctypes.c_void_p:
     return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
 
 
-def make_shape(B: int, H: int, S: int, d: int, tile_grid=(0, 0, 0)) -> _Shape:
-    Tt, Th, Tw = tile_grid
-    return _Shape(B, H, S, d, Tt, Th, Tw)
+def make_shape(B: int, H: int, S: int, d: int, tile_grid=(0, 0, 0),
+               layout: int = LAYOUT_TILE_MAJOR) -> _Shape:
+    Tt, Th, Tw = tile_grid if tile_grid is not None else (0, 0, 0)
+    return _Shape(B, H, S, d, Tt, Th, Tw, int(layout))
 
 
 def workspace_size(shape: _Shape, op: int) -> int:
@@ -167,11 +169,11 @@ class Workspace:
         _check(self.query_status(stream))
 
 
-def _shape_of(q, tile_grid=(0, 0, 0)) -> _Shape:
+def _shape_of(q, tile_grid=(0, 0, 0), layout: int = LAYOUT_TILE_MAJOR) -> _Shape:
     if q.dim() != 4:
         raise ValueError("q must be [B, H, S, d]")
     B, H, S, d = q.shape
-    return make_shape(B, H, S, d, tile_grid)
+    return make_shape(B, H, S, d, tile_grid, layout)
 
 
 def _bf16_contig(*ts):
@@ -184,15 +186,16 @@ def _bf16_contig(*ts):
 def nabla_build_mask(q, k, tile_grid, thr: float, sta: Optional[Tuple[int, int, int]] = None,
                      want_mask: bool = False, col_capacity: Optional[int] = None,
                      workspace: Optional[Workspace] = None, out=None, stream=None,
-                     topk: int = 0):
-    """NABLA block mask of (q, k) as block CSR (``topk`` > 0: fixed top-k rule).
+                     topk: int = 0, layout: int = LAYOUT_TILE_MAJOR):
+    """NABLA block mask of (q, k) as block CSR (``topk`` > 0: fixed top-k rule;
+    ``layout`` = LAYOUT_RASTER reads raster-ordered tokens in place).
 
     Returns (row_ptr int32 [B*H*nb+1], col_idx int32 [capacity], nnz int32 [1],
     mask uint8 [B,H,nb,nb] or None).  Only the first nnz entries of col_idx
     are meaningful.  ``out`` may pass preallocated (row_ptr, col_idx, nnz, mask)."""
     torch = _torch()
     _bf16_contig(q, k)
-    shape = _shape_of(q, tile_grid)
+    shape = _shape_of(q, tile_grid, layout)
     B, H, S, d = q.shape
     nb = S // 64
     if workspace is None:
@@ -215,11 +218,13 @@ def nabla_build_mask(q, k, tile_grid, thr: float, sta: Optional[Tuple[int, int, 
 
 
 def bsa_fwd(q, k, v, row_ptr, col_idx, scale: Optional[float] = None,
-            workspace: Optional[Workspace] = None, out=None, stream=None):
-    """Block-sparse attention forward over a block CSR.  Returns (O bf16, LSE fp32)."""
+            workspace: Optional[Workspace] = None, out=None, stream=None, tile_grid=None,
+            layout: int = LAYOUT_TILE_MAJOR):
+    """Block-sparse attention forward over a block CSR.  Returns (O bf16, LSE fp32).
+    ``layout`` = LAYOUT_RASTER (with ``tile_grid``) takes and returns raster-ordered tokens."""
     torch = _torch()
     _bf16_contig(q, k, v)
-    shape = _shape_of(q)
+    shape = _shape_of(q, tile_grid, layout)
     if workspace is None:
         workspace = Workspace.create(shape, OP_FWD, q.device, stream)
     if out is None:
@@ -234,11 +239,12 @@ def bsa_fwd(q, k, v, row_ptr, col_idx, scale: Optional[float] = None,
 
 
 def bsa_fwd_with_mask(q, k, v, mask_u8, scale: Optional[float] = None,
-                      workspace: Optional[Workspace] = None, out=None, stream=None):
+                      workspace: Optional[Workspace] = None, out=None, stream=None,
+                      tile_grid=None, layout: int = LAYOUT_TILE_MAJOR):
     """Block-sparse attention forward with a static uint8 block mask [B,H,nb,nb]."""
     torch = _torch()
     _bf16_contig(q, k, v)
-    shape = _shape_of(q)
+    shape = _shape_of(q, tile_grid, layout)
     if mask_u8.dtype != torch.uint8 or not mask_u8.is_cuda or not mask_u8.is_contiguous():
         raise ValueError("mask must be a contiguous uint8 CUDA tensor [B, H, nb, nb]")
     if workspace is None:
@@ -271,7 +277,8 @@ def selftest_mma(variant: int, a, b, workspace: Optional[Workspace] = None, stre
 
 
 def bsa_fwd_with_mask_static(q, k, v, mask_u8, scale: Optional[float] = None, out=None,
-                             status_out=None, stream=None):
+                             status_out=None, stream=None, tile_grid=None,
+                             layout: int = LAYOUT_TILE_MAJOR):
     """Static-mask attention forward that allocates no device memory inside the
     library and takes no workspace: for callers (memory-pool runtimes, code
     inside another framework's graph capture, fixed-budget hosts) that cannot
@@ -280,7 +287,7 @@ def bsa_fwd_with_mask_static(q, k, v, mask_u8, scale: Optional[float] = None, ou
     Returns (O, LSE); ``out`` may pass preallocated (O, LSE)."""
     torch = _torch()
     _bf16_contig(q, k, v)
-    shape = _shape_of(q)
+    shape = _shape_of(q, tile_grid, layout)
     if out is None:
         o = torch.empty_like(q)
         lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device)

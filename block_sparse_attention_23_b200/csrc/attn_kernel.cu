@@ -37,6 +37,11 @@
 //   only after PV_x(t), which read P_x(t), was issued by the same thread (MMAs
 //   of one thread execute in issue order).
 //
+// Token order: tile-major tensors are read as 2D boxes; raster-ordered ones
+// (token (t,h,w) at (t*H + h)*W + w) as 5D boxes that gather one 4x4x4 tile,
+// so the reorder to tile-major happens inside the TMA loads, and O / LSE rows
+// are stored back at their raster positions.
+//
 // Online softmax with a lazy maximum: the running max m of a row is raised
 // (and O, l rescaled by 2^(m_old - m_new)) only when a tile's max exceeds it by
 // more than 2^8; otherwise p <= 256 and O / l, LSE = ln2 (m + log2 l) are
@@ -116,9 +121,35 @@ struct AttnParams {
   float* lse;
   int* status;
   int H, S, nb, ngroups;
+  int Th, Tw;              // tile grid (raster token order only)
   float scale_log2;        // softmax scale * log2(e)
   uint64_t wait_limit_ns;
 };
+
+// One 64-token block of a [B,H,S,d] tensor as a 64 x 64 shared-memory box
+// (columns [64h, 64h+64) of d).  Tile-major order: rows 64*blk.. of head bh,
+// a 2D box.  Raster order: the block is tile blk of the 4Tt x 4Th x 4Tw token
+// grid, read by one 5D box (d, w, h, t, bh) of 64 x 4 x 4 x 4 x 1, which lands
+// its tokens in the same (t, h, w)-major row order.
+template <bool kRaster>
+__device__ __forceinline__ void load_block(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                           int h, int bh, int blk, int64_t S, int Th, int Tw) {
+  if (kRaster) {
+    const int tw = blk % Tw, th = (blk / Tw) % Th, tt = blk / (Tw * Th);
+    tma_load_5d(dst, map, bar, h * 64, 4 * tw, 4 * th, 4 * tt, bh);
+  } else {
+    tma_load_2d(dst, map, bar, h * 64, static_cast<int32_t>(static_cast<int64_t>(bh) * S + static_cast<int64_t>(blk) * 64));
+  }
+}
+
+// Position along S of row u of block blk.
+template <bool kRaster>
+__device__ __forceinline__ int64_t token_of(int blk, int u, int Th, int Tw) {
+  if (!kRaster) return static_cast<int64_t>(blk) * 64 + u;
+  const int tw = blk % Tw, th = (blk / Tw) % Th, tt = blk / (Tw * Th);
+  const int64_t H = 4ll * Th, W = 4ll * Tw;
+  return ((4ll * tt + (u >> 4)) * H + 4ll * th + ((u >> 2) & 3)) * W + 4ll * tw + (u & 3);
+}
 
 __device__ __forceinline__ void record_abort(volatile int* abort, int* status, int bit) {
   *abort = 1;
@@ -135,7 +166,7 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, uint64_
 // Membership mask of query tile x (bits of its two blocks) in union entry e.
 __device__ __forceinline__ int tile_bits(int e, int x) { return (e >> (16 + 2 * x)) & 3; }
 
-template <int D>
+template <int D, bool kRaster>
 __global__ void __launch_bounds__(kThreads, 1)
     bsa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const AttnParams prm) {
@@ -256,7 +287,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     // warp 8 streams Q and K, warp 10 streams V: a V slot frees only after the
     // softmax of its tile, and must not hold back the K prefetch
     if (lane == 0 && n_t > 0) {
-      const int64_t row0 = static_cast<int64_t>(bh) * prm.S;
       const bool is_k = warp == kProducerWarp;
       const int nst = is_k ? kKStages : kVStages;
       const uint32_t ring = is_k ? sK : sV;
@@ -265,10 +295,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       int armed0 = 0, armed1 = 0;
       if (is_k) {
         mbar_arrive_expect_tx(bar(kBarQFull), kQTiles * L::kQBytes);
-        for (int qb = 0; qb < 4; ++qb)
+        for (int qb = 0; qb < 4; ++qb)   // blocks past the end repeat the last (rows unused)
           for (int h = 0; h < L::kDH; ++h)
-            tma_load_2d(sQ + (qb >> 1) * L::kQBytes + h * kBM * 128 + (qb & 1) * 64 * 128, &tmQ,
-                        bar(kBarQFull), h * 64, static_cast<int32_t>(row0 + (r0 + qb) * 64));
+            load_block<kRaster>(sQ + (qb >> 1) * L::kQBytes + h * kBM * 128 + (qb & 1) * 64 * 128,
+                                &tmQ, bar(kBarQFull), h, bh, min(r0 + qb, nb - 1), prm.S, prm.Th,
+                                prm.Tw);
       }
       for (int t = 0; t < n_t; ++t) {
         const int s = t % nst, n = t / nst;
@@ -282,8 +313,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         (s ? armed1 : armed0) += 1;
         for (int kb = 0; kb < 2; ++kb)
           for (int h = 0; h < L::kDH; ++h)
-            tma_load_2d(ring + s * L::kKVBytes + h * kBN * 128 + kb * 64 * 128, map, bar(full0 + s),
-                        h * 64, static_cast<int32_t>(row0 + (kb ? j1 : j0) * 64));
+            load_block<kRaster>(ring + s * L::kKVBytes + h * kBN * 128 + kb * 64 * 128, map,
+                                bar(full0 + s), h, bh, kb ? j1 : j0, prm.S, prm.Th, prm.Tw);
       }
       // drain: every armed phase must complete before shared memory is released
       if (is_k) mbar_wait(bar(kBarQFull), 0, kDrainLimitNs, nullptr);
@@ -457,7 +488,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
     }
     const bool write = row_valid && ok && (c == 0 || have_o);
-    const int64_t grow = static_cast<int64_t>(bh) * prm.S + static_cast<int64_t>(qblock) * 64 + (row & 63);
+    const int64_t grow = static_cast<int64_t>(bh) * prm.S +
+                         (row_valid ? token_of<kRaster>(qblock, row & 63, prm.Th, prm.Tw) : 0);
     const float inv_l = l > 0.f ? 1.f / l : 0.f;
     __nv_bfloat16* orow = prm.o + grow * D;
 #pragma unroll
@@ -594,27 +626,28 @@ __global__ void __launch_bounds__(160, 1)
 
 // ---------------------------------------------------------------- launchers
 
-template <int D>
+template <int D, bool kRaster>
 static cudaError_t launch_fwd_t(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
                                 const AttnParams& prm, int64_t nitems, cudaStream_t st) {
   constexpr uint32_t smem = AttnSmem<D>::kAlloc;
   static_assert(8 * kRegsSoftmax + 4 * kRegsOther <= 12 * kRegsLaunch, "register split");
   cudaFuncAttributes attr;
-  cudaError_t e = cudaFuncGetAttributes(&attr, bsa_fwd_kernel<D>);
+  cudaError_t e = cudaFuncGetAttributes(&attr, bsa_fwd_kernel<D, kRaster>);
   if (e != cudaSuccess) return e;
   // the in-kernel register split assumes the launch allocation of kRegsLaunch
   // registers per thread; anything less would make setmaxnreg.inc wait forever
   if (attr.numRegs < kRegsLaunch) return cudaErrorInvalidConfiguration;
-  e = cudaFuncSetAttribute(bsa_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  e = cudaFuncSetAttribute(bsa_fwd_kernel<D, kRaster>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           smem);
   if (e != cudaSuccess) return e;
-  bsa_fwd_kernel<D><<<static_cast<unsigned>(nitems), kThreads, smem, st>>>(q, k, v, prm);
+  bsa_fwd_kernel<D, kRaster><<<static_cast<unsigned>(nitems), kThreads, smem, st>>>(q, k, v, prm);
   return cudaGetLastError();
 }
 
 cudaError_t launch_bsa_fwd(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
                            const int32_t* row_ptr, const int32_t* col_idx, void* o, float* lse,
-                           int* status, int BH, int H, int S, int d, float scale,
-                           uint64_t wait_limit_ns, cudaStream_t st) {
+                           int* status, int BH, int H, int S, int d, float scale, int raster,
+                           int Th, int Tw, uint64_t wait_limit_ns, cudaStream_t st) {
   AttnParams prm;
   prm.row_ptr = row_ptr;
   prm.col_idx = col_idx;
@@ -625,12 +658,18 @@ cudaError_t launch_bsa_fwd(const CUtensorMap& q, const CUtensorMap& k, const CUt
   prm.S = S;
   prm.nb = S / 64;
   prm.ngroups = (prm.nb + 3) / 4;
+  prm.Th = Th;
+  prm.Tw = Tw;
   prm.scale_log2 = scale * 1.4426950408889634f;
   prm.wait_limit_ns = wait_limit_ns;
   const int64_t nitems = static_cast<int64_t>(BH) * prm.ngroups;
   if (nitems == 0) return cudaSuccess;
-  if (d == 128) return launch_fwd_t<128>(q, k, v, prm, nitems, st);
-  return launch_fwd_t<64>(q, k, v, prm, nitems, st);
+  if (raster) {
+    if (d == 128) return launch_fwd_t<128, true>(q, k, v, prm, nitems, st);
+    return launch_fwd_t<64, true>(q, k, v, prm, nitems, st);
+  }
+  if (d == 128) return launch_fwd_t<128, false>(q, k, v, prm, nitems, st);
+  return launch_fwd_t<64, false>(q, k, v, prm, nitems, st);
 }
 
 cudaError_t launch_mma_selftest(const CUtensorMap& a, const CUtensorMap& b, const void* a_glob,

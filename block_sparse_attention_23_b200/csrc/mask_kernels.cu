@@ -8,8 +8,9 @@
 // "Sliding Tile Attention", and compact to block CSR.
 //
 // Kernels (all stream-ordered, no host synchronisation):
-//   pool_kernel        Q, K bf16 [BH,S,d] -> Qbar, Kbar fp32 [BH,nb,d]     HBM-bound
-//   logits_kernel      per head Qbar Kbar^T / sqrt(d) -> L fp32 [BH,nb,nb] fp32 FFMA
+//   pool_kernel        Q, K bf16 [BH,S,d] -> Qbar, Kbar fp64 [BH,nb,d]     HBM-bound
+//                      (tile-major or raster token order)
+//   logits_kernel      per head Qbar Kbar^T / sqrt(d) -> L fp64 [BH,nb,nb] fp64 FMA
 //   select_kernel      one warp per row: softmax, prefix (or top-k) selection, STA OR ->
 //                      keep bitmap [BH*nb, nw] + counts (+ optional uint8 mask)
 //   mask_bits_kernel   external uint8 mask -> keep bitmap + counts
@@ -37,11 +38,14 @@ namespace nabla {
 // One warp per (tensor, bh, block): 64 rows of d bf16.  A row is d/8 16-byte
 // chunks; the warp covers 32/(d/8) rows per step with 128-bit loads.  Sums are
 // fp64, so the mean of 64 bf16 values is exact.
-template <int D>
+// Raster token order (kRaster): block r of a head is tile r of the 4Tt x 4Th x
+// 4Tw grid, its row u the token ((4tt + u/16)*H + 4th + (u/4)%4)*W + 4tw + u%4.
+template <int D, bool kRaster>
 __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restrict__ q,
                                                    const __nv_bfloat16* __restrict__ k,
                                                    double* __restrict__ qbar,
-                                                   double* __restrict__ kbar, int64_t nblocks) {
+                                                   double* __restrict__ kbar, int64_t nblocks,
+                                                   int nb, int Th, int Tw) {
   constexpr int kLanesPerRow = D / 8;              // 16 (d=128) or 8 (d=64)
   constexpr int kRowsPerStep = 32 / kLanesPerRow;  // 2 or 4
   constexpr int kSteps = 64 / kRowsPerStep;        // 32 or 16
@@ -50,7 +54,16 @@ __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restri
   if (wid >= 2 * nblocks) return;
   const bool is_k = wid >= nblocks;
   const int64_t blk = is_k ? wid - nblocks : wid;
-  const __nv_bfloat16* src = (is_k ? k : q) + blk * 64 * D;
+  const __nv_bfloat16* src = (is_k ? k : q) + blk * 64 * D;   // tile-major: block rows
+  int64_t head = 0;
+  int tt = 0, th = 0, tw = 0;
+  if (kRaster) {   // row u of the block is at head + token offset (see above)
+    const int64_t bh = blk / nb;
+    const int r = static_cast<int>(blk % nb);
+    tw = r % Tw; th = (r / Tw) % Th; tt = r / (Tw * Th);
+    head = bh * static_cast<int64_t>(nb) * 64;
+    src = (is_k ? k : q) + head * D;
+  }
   double* dst = (is_k ? kbar : qbar) + blk * D;
   const int chunk = lane % kLanesPerRow;
   const int sub = lane / kLanesPerRow;
@@ -60,7 +73,11 @@ __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restri
 #pragma unroll 8
   for (int s = 0; s < kSteps; ++s) {
     const int row = s * kRowsPerStep + sub;
-    const uint4 v = __ldg(reinterpret_cast<const uint4*>(src + row * D) + chunk);
+    int64_t tok = row;
+    if (kRaster)
+      tok = ((4ll * tt + (row >> 4)) * (4ll * Th) + 4ll * th + ((row >> 2) & 3)) * (4ll * Tw) +
+            4ll * tw + (row & 3);
+    const uint4 v = __ldg(reinterpret_cast<const uint4*>(src + tok * D) + chunk);
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -474,17 +491,19 @@ __global__ void __launch_bounds__(256) fill_kernel(const uint32_t* __restrict__ 
 // ------------------------------------------------------------------ launchers
 
 cudaError_t launch_pool(const void* q, const void* k, double* qbar, double* kbar,
-                        int64_t nblocks, int d, cudaStream_t st) {
+                        int64_t nblocks, int d, int nb, int raster, int Th, int Tw,
+                        cudaStream_t st) {
   const int64_t warps = 2 * nblocks;
   const unsigned grid = static_cast<unsigned>((warps * 32 + 255) / 256);
-  if (d == 128)
-    pool_kernel<128><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(q),
-                                            static_cast<const __nv_bfloat16*>(k), qbar, kbar,
-                                            nblocks);
-  else
-    pool_kernel<64><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(q),
-                                           static_cast<const __nv_bfloat16*>(k), qbar, kbar,
-                                           nblocks);
+  const __nv_bfloat16* qq = static_cast<const __nv_bfloat16*>(q);
+  const __nv_bfloat16* kk = static_cast<const __nv_bfloat16*>(k);
+  if (raster) {
+    if (d == 128) pool_kernel<128, true><<<grid, 256, 0, st>>>(qq, kk, qbar, kbar, nblocks, nb, Th, Tw);
+    else pool_kernel<64, true><<<grid, 256, 0, st>>>(qq, kk, qbar, kbar, nblocks, nb, Th, Tw);
+  } else {
+    if (d == 128) pool_kernel<128, false><<<grid, 256, 0, st>>>(qq, kk, qbar, kbar, nblocks, nb, Th, Tw);
+    else pool_kernel<64, false><<<grid, 256, 0, st>>>(qq, kk, qbar, kbar, nblocks, nb, Th, Tw);
+  }
   return cudaGetLastError();
 }
 

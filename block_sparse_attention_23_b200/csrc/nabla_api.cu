@@ -17,7 +17,8 @@
 
 namespace nabla {
 cudaError_t launch_pool(const void* q, const void* k, double* qbar, double* kbar,
-                        int64_t nblocks, int d, cudaStream_t st);
+                        int64_t nblocks, int d, int nb, int raster, int Th, int Tw,
+                        cudaStream_t st);
 cudaError_t launch_logits(const double* qbar, const double* kbar, double* L, int BH, int nb,
                           int d, cudaStream_t st);
 cudaError_t launch_select(const double* L, int64_t nrows, int nb, float thr, int topk,
@@ -30,8 +31,8 @@ cudaError_t launch_scan_fill(const uint32_t* bits, const int32_t* counts, int64_
                              int32_t* nnz_out, int* status, cudaStream_t st);
 cudaError_t launch_bsa_fwd(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
                            const int32_t* row_ptr, const int32_t* col_idx, void* o, float* lse,
-                           int* status, int BH, int H, int S, int d, float scale,
-                           uint64_t wait_limit_ns, cudaStream_t st);
+                           int* status, int BH, int H, int S, int d, float scale, int raster,
+                           int Th, int Tw, uint64_t wait_limit_ns, cudaStream_t st);
 cudaError_t launch_reorder(const void* src, void* dst, int64_t BH, int Tt, int Th, int Tw,
                            int row_bytes, int to_tile_major, cudaStream_t st);
 cudaError_t launch_block_energy(const CUtensorMap& q, const CUtensorMap& k, const int32_t* row_ptr,
@@ -90,6 +91,19 @@ nabla_status check_shape(const nabla_shape* s) {
     return fail(NABLA_ERR_UNSUPPORTED, "B*H*nb*nb must stay below 2^31");
   if (static_cast<int64_t>(s->B) * s->H * s->S >= (static_cast<int64_t>(1) << 31))
     return fail(NABLA_ERR_UNSUPPORTED, "B*H*S must stay below 2^31");
+  if (s->layout != NABLA_LAYOUT_TILE_MAJOR && s->layout != NABLA_LAYOUT_RASTER)
+    return fail(NABLA_ERR_INVALID_ARG, "unknown token layout");
+  if (s->layout == NABLA_LAYOUT_RASTER &&
+      (s->Tt <= 0 || s->Th <= 0 || s->Tw <= 0 ||
+       static_cast<int64_t>(s->Tt) * s->Th * s->Tw != nb))
+    return fail(NABLA_ERR_INVALID_ARG, "raster layout needs a tile grid with Tt*Th*Tw = S/64");
+  return NABLA_OK;
+}
+
+// For calls that take tile-major tokens only.
+nabla_status require_tile_major(const nabla_shape* s) {
+  if (s->layout != NABLA_LAYOUT_TILE_MAJOR)
+    return fail(NABLA_ERR_UNSUPPORTED, "this call takes tile-major tokens; use nabla_reorder_tokens");
   return NABLA_OK;
 }
 
@@ -176,21 +190,47 @@ nabla_status make_map(CUtensorMap* map, const void* ptr, uint64_t rows, uint64_t
   return NABLA_OK;
 }
 
+// [BH][4Tt][4Th][4Tw][d] bf16 (raster token order); 5D boxes of 64 x 4 x 4 x 4 x 1 =
+// one 4x4x4 tile, 128-byte swizzle, rows landing in (t, h, w)-major order.
+nabla_status make_map_raster(CUtensorMap* map, const void* ptr, const nabla_shape* s) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return fail(NABLA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+  const cuuint64_t d = s->d, W = 4ull * s->Tw, H = 4ull * s->Th, T = 4ull * s->Tt;
+  const cuuint64_t BH = static_cast<cuuint64_t>(s->B) * s->H;
+  cuuint64_t dims[5] = {d, W, H, T, BH};
+  cuuint64_t strides[4] = {d * 2, W * d * 2, H * W * d * 2, T * H * W * d * 2};
+  cuuint32_t box[5] = {64, 4, 4, 4, 1};
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(ptr), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(NABLA_ERR_CUDA, "cuTensorMapEncodeTiled (5D) failed");
+  return NABLA_OK;
+}
+
 int* status_ptr(void* ws) { return static_cast<int*>(ws); }
 
 nabla_status run_fwd(const nabla_shape* shape, const void* q, const void* k, const void* v,
                      const int32_t* row_ptr, const int32_t* col_idx, float scale, void* o,
                      float* lse, void* workspace, cudaStream_t st) {
   const uint64_t rows = static_cast<uint64_t>(shape->B) * shape->H * shape->S;
+  const bool raster = shape->layout == NABLA_LAYOUT_RASTER;
   CUtensorMap mq, mk, mv;
   nabla_status s;
-  if ((s = make_map(&mq, q, rows, shape->d)) != NABLA_OK) return s;
-  if ((s = make_map(&mk, k, rows, shape->d)) != NABLA_OK) return s;
-  if ((s = make_map(&mv, v, rows, shape->d)) != NABLA_OK) return s;
+  if (raster) {
+    if ((s = make_map_raster(&mq, q, shape)) != NABLA_OK) return s;
+    if ((s = make_map_raster(&mk, k, shape)) != NABLA_OK) return s;
+    if ((s = make_map_raster(&mv, v, shape)) != NABLA_OK) return s;
+  } else {
+    if ((s = make_map(&mq, q, rows, shape->d)) != NABLA_OK) return s;
+    if ((s = make_map(&mk, k, rows, shape->d)) != NABLA_OK) return s;
+    if ((s = make_map(&mv, v, rows, shape->d)) != NABLA_OK) return s;
+  }
   if (!(scale > 0.f)) scale = 1.0f / std::sqrt(static_cast<float>(shape->d));
   cudaError_t e = nabla::launch_bsa_fwd(mq, mk, mv, row_ptr, col_idx, o, lse,
                                         status_ptr(workspace), shape->B * shape->H, shape->H,
-                                        shape->S, shape->d, scale, g_wait_limit_ns.load(), st);
+                                        shape->S, shape->d, scale, raster ? 1 : 0, shape->Th,
+                                        shape->Tw, g_wait_limit_ns.load(), st);
   if (e != cudaSuccess) return cuda_fail(e, "bsa_fwd launch");
   return NABLA_OK;
 }
@@ -204,7 +244,7 @@ void set_last_error(const std::string& msg) { g_last_error = msg; }
 
 extern "C" {
 
-int nabla_version(void) { return 200; }
+int nabla_version(void) { return 210; }
 
 const char* nabla_last_error(void) { return g_last_error.c_str(); }
 
@@ -276,7 +316,9 @@ nabla_status nabla_build_mask(const nabla_shape* shape, const nabla_mask_params*
   int32_t* counts = reinterpret_cast<int32_t*>(ws + lay.counts);
   const int nb = shape->S / 64, BH = shape->B * shape->H;
   const int64_t nrows = static_cast<int64_t>(BH) * nb;
-  cudaError_t e = nabla::launch_pool(q, k, qbar, kbar, nrows, shape->d, st);
+  cudaError_t e = nabla::launch_pool(q, k, qbar, kbar, nrows, shape->d, nb,
+                                     shape->layout == NABLA_LAYOUT_RASTER ? 1 : 0, shape->Th,
+                                     shape->Tw, st);
   if (e != cudaSuccess) return cuda_fail(e, "pool launch");
   e = nabla::launch_logits(qbar, kbar, L, BH, nb, shape->d, st);
   if (e != cudaSuccess) return cuda_fail(e, "logits launch");
@@ -363,6 +405,7 @@ nabla_status nabla_block_energy(const nabla_shape* shape, const void* q, const v
                                 nabla_stream_t stream) {
   nabla_status s = check_shape(shape);
   if (s != NABLA_OK) return s;
+  if ((s = require_tile_major(shape)) != NABLA_OK) return s;
   if (!q || !k || !lse || !row_ptr || !col_idx || !energy || !workspace)
     return fail(NABLA_ERR_INVALID_ARG, "null pointer");
   if (!aligned16(q) || !aligned16(k)) return fail(NABLA_ERR_INVALID_ARG, "q, k must be 16-byte aligned");
@@ -414,6 +457,7 @@ nabla_status bsa_bwd(const nabla_shape* shape, const void* q, const void* k, con
                      void* workspace, nabla_stream_t stream) {
   nabla_status s = check_shape(shape);
   if (s != NABLA_OK) return s;
+  if ((s = require_tile_major(shape)) != NABLA_OK) return s;
   if (!q || !k || !v || !o || !dout || !lse || !row_ptr || !col_idx || !dq || !dk || !dv ||
       !workspace)
     return fail(NABLA_ERR_INVALID_ARG, "null pointer");

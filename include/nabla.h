@@ -58,7 +58,17 @@ typedef enum {
 typedef struct {
     int32_t B, H, S, d;   /* batch, heads, tokens, head dim */
     int32_t Tt, Th, Tw;   /* tile grid (4x4x4-token tiles); Tt*Th*Tw must equal S/64 */
+    int32_t layout;       /* token order of Q, K, V, O, LSE along S: NABLA_LAYOUT_TILE_MAJOR
+                             (0; block r = tokens 64r..64r+63) or NABLA_LAYOUT_RASTER (1;
+                             token (t,h,w) at (t*H + h)*W + w of the 4Tt x 4Th x 4Tw grid,
+                             block r = tile r of the grid, read in place: the reorder of the
+                             NABLA review's Figure 4 fused into the loads and the O/LSE
+                             stores).  RASTER needs the tile grid and is accepted by
+                             nabla_build_mask, bsa_fwd and bsa_fwd_with_mask(_static); the
+                             other calls return NABLA_ERR_UNSUPPORTED for it. */
 } nabla_shape;
+
+enum { NABLA_LAYOUT_TILE_MAJOR = 0, NABLA_LAYOUT_RASTER = 1 };
 
 typedef struct {
     float thr;            /* keep the smallest sorted prefix with mass >= 1 - thr; thr in [0, 1] */

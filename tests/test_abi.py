@@ -146,3 +146,21 @@ def test_reorder_arguments_checked(nl):
     assert f(ctypes.byref(good), 0, null, b, null) == 1
     assert f(ctypes.byref(good), 0, a, a, null) == 1
     assert f(ctypes.byref(good), 1, ctypes.c_void_p((1 << 20) + 8), b, null) == 1
+
+
+def test_layout_arguments_checked(nl):
+    lib = nl.lib()
+    null = ctypes.c_void_p(0)
+    a = ctypes.c_void_p(1 << 20)
+    no_grid = nl.make_shape(1, 1, 128, 64, (0, 0, 0), nl.LAYOUT_RASTER)
+    bad = nl.make_shape(1, 1, 128, 64, (1, 1, 2), 7)
+    raster = nl.make_shape(1, 1, 128, 64, (1, 1, 2), nl.LAYOUT_RASTER)
+    f = lib.bsa_fwd
+    assert f(ctypes.byref(no_grid), a, a, a, a, a, ctypes.c_float(0), a, a, a, null) == 1
+    assert f(ctypes.byref(bad), a, a, a, a, a, ctypes.c_float(0), a, a, a, null) == 1
+    # the backward and the energy kernel take tile-major tokens only
+    assert lib.bsa_bwd(ctypes.byref(raster), a, a, a, a, a, a, a, a, ctypes.c_float(0), a, a, a,
+                       a, null) == 2
+    assert lib.nabla_block_energy(ctypes.byref(raster), a, a, a, a, a, ctypes.c_float(0), a,
+                                  null, a, null) == 2
+    assert lib.nabla_version() >= 210
