@@ -83,6 +83,8 @@ def _load():
             lib.oracle_attention_bwd.restype = None
             lib.oracle_attention_bwd.argtypes = [vp, vp, vp, vp, i64, i64, i32, vp, f64, i64, vp,
                                                  vp, i64, vp, vp, vp]
+            lib.oracle_xattn_scores.restype = None
+            lib.oracle_xattn_scores.argtypes = [vp, vp, i64, i64, i32, i32, i64, vp, vp]
             lib.oracle_max_threads.restype = i32
             lib.oracle_max_threads.argtypes = []
             _lib = lib
@@ -298,6 +300,54 @@ def attention_bwd(q, k, v, dO, mask, scale=None, qrows=None, krows=None):
                                  B * H, S, d, mask.ctypes.data, float(scale), nq, qp,
                                  dQ.ctypes.data, nk, kp, dK.ctypes.data, dV.ctypes.data)
     return dQ, dK, dV
+
+
+def xattn_scores(q, k, stride: int = 8, rows=None):
+    """XAttention antidiagonal block scores in fp64: [B,H,nb,nb] (rows=None)
+    or [len(rows), nb] for global block-row ids bh*nb + r."""
+    q, k = _u16(q), _u16(k)
+    B, H, S, d = q.shape
+    nb = S // BLOCK
+    if BLOCK % stride:
+        raise ValueError("stride must divide 64")
+    if rows is None:
+        n, rp = B * H * nb, None
+        out = np.empty((B, H, nb, nb), dtype=np.float64)
+    else:
+        rows = np.ascontiguousarray(rows, dtype=np.int64)
+        n, rp = rows.shape[0], rows.ctypes.data
+        out = np.empty((n, nb), dtype=np.float64)
+    _load().oracle_xattn_scores(q.ctypes.data, k.ctypes.data, B * H, S, d, int(stride), n, rp,
+                                out.ctypes.data)
+    return out
+
+
+def select_rows(weights, tile_grid, thr: float, sta=None, topk: int = 0, with_diag=False):
+    """The builder's selection (a4-a6) on given block weights [B,H,nb,nb]: each
+    row normalised by its sum, then the mass rule at thr (or top-k), STA OR."""
+    weights = np.asarray(weights, dtype=np.float64)
+    B, H, nb, _ = weights.shape
+    Tt, Th, Tw = tile_grid
+    mask = np.zeros((B, H, nb, nb), dtype=np.uint8)
+    diag = np.zeros((B, H, nb, 4), dtype=np.float64)
+    for b in range(B):
+        for h in range(H):
+            for r in range(nb):
+                w = np.clip(weights[b, h, r], 0.0, None)
+                z = w.sum()
+                if z <= 0:
+                    keep = np.zeros(nb, dtype=np.uint8)
+                    dg = np.array([-1.0, -1.0, -1.0, -1.0])
+                elif topk > 0:
+                    keep, _ = row_select_topk(w / z, topk)
+                    dg = np.array([-1.0, -1.0, -1.0, -1.0])
+                else:
+                    keep, _, dg = row_select(w / z, thr)
+                if sta is not None:
+                    keep = keep | sta_row(r, tile_grid, sta)
+                mask[b, h, r] = keep
+                diag[b, h, r] = dg
+    return (mask, diag) if with_diag else mask
 
 
 def near_cut_rows(diag: np.ndarray, thr: float, band: float = 1e-4) -> np.ndarray:

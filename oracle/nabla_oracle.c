@@ -464,6 +464,49 @@ void oracle_attention_bwd(const uint16_t* q, const uint16_t* k, const uint16_t* 
     free(D_all);
 }
 
+/* XAttention antidiagonal block scores ("XAttention: Block Sparse Attention
+ * with Antidiagonal Scoring" notes: blocks are scored along antidiagonals and
+ * selected by a threshold).  Reading (the notes give no formula): stride St
+ * divides 64; strided query row i and key row j of a head stand for the St x St
+ * sub-block of Q K^T at rows i*St.., columns j*St..; their score is the mean of
+ * that sub-block's antidiagonal,
+ *   a_ij = (1/St) sum_{s<St} q_{i*St + St-1-s} . k_{j*St + s} / sqrt(d),
+ * p_i = softmax over all strided keys j of a_i, and the block score of query
+ * block r and key block c is the mean over r's 64/St strided rows of the mass
+ * p puts on c's 64/St strided keys (so each row of scores sums to 1).
+ * rows (nrows global block-row ids bh*nb + r; NULL = every row) select the
+ * rows computed; scores [nrows, nb]. */
+void oracle_xattn_scores(const uint16_t* q, const uint16_t* k, int64_t BH, int64_t S, int d,
+                         int St, int64_t nrows, const int64_t* rows, double* scores) {
+    const int64_t nb = S / ORACLE_BLOCK, L = S / St, per = ORACLE_BLOCK / St;
+    const double scale = 1.0 / (St * sqrt((double)d));
+    if (rows == NULL) nrows = BH * nb;
+#pragma omp parallel for schedule(dynamic)
+    for (int64_t n = 0; n < nrows; ++n) {
+        const int64_t g = rows ? rows[n] : n, bh = g / nb, r = g % nb;
+        double* a = (double*)malloc(sizeof(double) * (size_t)L);
+        for (int64_t c = 0; c < nb; ++c) scores[n * nb + c] = 0.0;
+        for (int64_t ii = 0; ii < per; ++ii) {
+            const int64_t i = r * per + ii;
+            double m = -INFINITY;
+            for (int64_t j = 0; j < L; ++j) {
+                double acc = 0.0;
+                for (int s = 0; s < St; ++s) {
+                    const uint16_t* qr = q + (bh * S + i * St + St - 1 - s) * d;
+                    const uint16_t* kr = k + (bh * S + j * St + s) * d;
+                    for (int t = 0; t < d; ++t) acc += bf16_to_f64(qr[t]) * bf16_to_f64(kr[t]);
+                }
+                a[j] = scale * acc;
+                if (a[j] > m) m = a[j];
+            }
+            double z = 0.0;
+            for (int64_t j = 0; j < L; ++j) z += exp(a[j] - m);
+            for (int64_t j = 0; j < L; ++j) scores[n * nb + j / per] += exp(a[j] - m) / z / per;
+        }
+        free(a);
+    }
+}
+
 /* Threads OpenMP will use (for reporting the CPU baseline's core count). */
 int oracle_max_threads(void) {
 #ifdef _OPENMP

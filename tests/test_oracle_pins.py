@@ -683,3 +683,78 @@ def test_attention_bwd_row_subsets(oracle_mod):
     np.testing.assert_array_equal(sv, dV[kr])
     eq, ek, ev = oracle_mod.attention_bwd(q, k, v, dO, mask, qrows=qr, krows=np.empty(0, np.int64))
     assert ek.shape == (0, d) and np.array_equal(eq, dQ[qr])
+
+
+# ---------------------------------------------------------------------------
+# XAttention antidiagonal scoring
+
+
+def _brute_xattn(q, k, St):
+    """Explicit antidiagonal sums of the full fp64 score matrix, scipy softmax,
+    block means; independent of the oracle's strided loops."""
+    from scipy.special import softmax
+    B, H, S, d = q.shape
+    nb, L, per = S // 64, S // St, 64 // St
+    out = np.zeros((B, H, nb, nb))
+    for b in range(B):
+        for h in range(H):
+            M = _f(q[b, h]) @ _f(k[b, h]).T / math.sqrt(d)
+            A = np.zeros((L, L))
+            for s in range(St):
+                A += M[np.arange(L)[:, None] * St + St - 1 - s, np.arange(L)[None, :] * St + s]
+            P = softmax(A / St, axis=1)
+            out[b, h] = P.reshape(nb, per, nb, per).sum(axis=(1, 3)) / per
+    return out
+
+
+@pytest.mark.parametrize("St", [1, 4, 8, 16])
+def test_xattn_matches_brute_force_antidiagonals(oracle_mod, St):
+    rng = np.random.default_rng(40 + St)
+    q = _rand_bits(rng, (1, 2, 256, 64), 0.7)
+    k = _rand_bits(rng, (1, 2, 256, 64), 0.7)
+    got = oracle_mod.xattn_scores(q, k, St)
+    np.testing.assert_allclose(got, _brute_xattn(q, k, St), rtol=1e-10, atol=1e-14)
+    np.testing.assert_allclose(got.sum(axis=-1), 1.0, atol=1e-12)
+    # an antidiagonal is not a diagonal: reversing the query order inside each
+    # stride group changes the scores (St > 1)
+    if St > 1:
+        qf = q.reshape(1, 2, 256 // St, St, 64)[:, :, :, ::-1].reshape(q.shape)
+        assert np.abs(oracle_mod.xattn_scores(np.ascontiguousarray(qf), k, St) - got).max() > 1e-4
+
+
+def test_xattn_stride1_is_block_energy(oracle_mod):
+    # stride 1: every strided row is a token and a_ij the attention logit, so
+    # the scores are the true block energies with the dense LSE
+    rng = np.random.default_rng(50)
+    q = _rand_bits(rng, (1, 1, 192, 64))
+    k = _rand_bits(rng, (1, 1, 192, 64))
+    v = _rand_bits(rng, (1, 1, 192, 64))
+    _, lse = oracle_mod.dense_attention(q, k, v)
+    E, _ = oracle_mod.block_energy(q, k, lse.reshape(1, 1, 192), np.ones((1, 1, 3, 3), np.uint8))
+    np.testing.assert_allclose(oracle_mod.xattn_scores(q, k, 1), E, rtol=1e-10)
+
+
+def test_xattn_uniform_and_rows(oracle_mod):
+    rng = np.random.default_rng(51)
+    q = np.zeros((1, 1, 320, 64), dtype=np.uint16)
+    k = _rand_bits(rng, (1, 1, 320, 64))
+    np.testing.assert_allclose(oracle_mod.xattn_scores(q, k, 8), 1.0 / 5, rtol=1e-13)
+    q = _rand_bits(rng, (2, 1, 320, 64))
+    k = _rand_bits(rng, (2, 1, 320, 64))
+    full = oracle_mod.xattn_scores(q, k, 8).reshape(-1, 5)
+    rows = np.array([7, 0, 4], dtype=np.int64)
+    np.testing.assert_array_equal(oracle_mod.xattn_scores(q, k, 8, rows=rows), full[rows])
+
+
+def test_select_rows_matches_builder_on_its_own_map(oracle_mod):
+    # the builder's selection applied to the softmax of its own reduced map
+    # gives the builder's mask
+    rng = np.random.default_rng(52)
+    grid = (1, 2, 2)
+    q = _rand_bits(rng, (1, 2, 256, 64))
+    k = _rand_bits(rng, (1, 2, 256, 64))
+    want = oracle_mod.build_mask(q, k, grid, 0.3, (0, 1, 0))
+    qb, kb = oracle_mod.pool(q), oracle_mod.pool(k)
+    P = np.stack([[np.stack([oracle_mod.softmax_row(r) for r in oracle_mod.logits(qb[0, h], kb[0, h])])
+                   for h in range(2)]])
+    np.testing.assert_array_equal(oracle_mod.select_rows(P * 3.0, grid, 0.3, (0, 1, 0)), want)
