@@ -437,6 +437,29 @@ def run_ours(args):
     bwd_tflops = bwd_flops / (bwd_ms * 1e-3) / 1e12
     del dout, grads
 
+    # XAttention scorer (stride 8) + the same selection, outside the step;
+    # algorithmic FLOPs = two passes over the strided score matrix
+    ws_x = nl.Workspace.create(shape, nl.OP_BUILD_XATTN, dev)
+
+    def xattn_call():
+        nl.nabla_build_mask_xattn(q, k, w.thr, 8, tile_grid=w.tile_grid, sta=w.sta,
+                                  workspace=ws_x, out=mask_out)
+
+    xattn_call()
+    torch.cuda.synchronize()
+    ws_x.check()
+    x_kept = int(mask_out[2].item())
+    n_x = 3
+    a.record(stream)
+    for _ in range(n_x):
+        xattn_call()
+    b.record(stream)
+    torch.cuda.synchronize()
+    ws_x.check()
+    x_ms = a.elapsed_time(b) / n_x
+    x_flops = 4.0 * S * S * d * B * H / 8
+    x_tflops = x_flops / (x_ms * 1e-3) / 1e12
+
     attn_tflops = kept_flops / (attn_ms * 1e-3) / 1e12
     peak = peaks["bf16_tflops_sustained"]
     traffic = _traffic_per_launch()
@@ -477,6 +500,11 @@ def run_ours(args):
                          "what": "E over the step's kept blocks (QK^T + exp + block sums), "
                                  "outside the step; FLOPs = 2*d*64*64 per block"},
         "calib_accumulate_ms": cal_ms,
+        "xattn_mask": {"bound": "tensor", "ms": x_ms, "achieved": x_tflops, "peak": peak,
+                       "unit": "TFLOP/s", "frac": x_tflops / peak, "flops": x_flops,
+                       "kept_blocks": x_kept, "density": x_kept / (B * H * nb * nb),
+                       "what": "XAttention antidiagonal scores (stride 8, two passes) + selection "
+                               "at the layer's thr and STA, outside the step"},
         "bwd": {"bound": "tensor", "ms": bwd_ms, "achieved": bwd_tflops, "peak": peak,
                 "unit": "TFLOP/s", "frac": bwd_tflops / peak, "flops": bwd_flops,
                 "what": "bsa_bwd (D, column bitmaps, dK/dV and dQ kernels) over the step's "

@@ -27,13 +27,14 @@ NABLA_OK = 0
 STATUS_NAMES = {0: "NABLA_OK", 1: "NABLA_ERR_INVALID_ARG", 2: "NABLA_ERR_UNSUPPORTED",
                 3: "NABLA_ERR_CAPACITY", 4: "NABLA_ERR_CUDA", 5: "NABLA_ERR_TIMEOUT",
                 6: "NABLA_ERR_BAD_INDEX"}
-OP_BUILD_MASK, OP_FWD, OP_FWD_WITH_MASK, OP_BWD = 0, 1, 2, 3
+OP_BUILD_MASK, OP_FWD, OP_FWD_WITH_MASK, OP_BWD, OP_BUILD_XATTN = 0, 1, 2, 3, 4
 LAYOUT_TILE_MAJOR, LAYOUT_RASTER = 0, 1
 EXPORTED = ["nabla_workspace_size", "nabla_workspace_init", "nabla_query_status",
             "nabla_build_mask", "bsa_fwd", "bsa_fwd_with_mask", "nabla_last_error",
             "nabla_version", "nabla_set_wait_limit_ns", "nabla_selftest_mma",
             "bsa_fwd_with_mask_static", "nabla_reorder_tokens", "nabla_block_energy",
-            "nabla_calib_accumulate", "nabla_calib_finalize", "bsa_bwd"]
+            "nabla_calib_accumulate", "nabla_calib_finalize", "bsa_bwd",
+            "nabla_build_mask_xattn"]
 TO_TILE_MAJOR, TO_RASTER = 0, 1
 
 
@@ -104,6 +105,9 @@ def lib() -> ctypes.CDLL:
             L.nabla_calib_accumulate.argtypes = [sp, vp, f32, vp, vp]
             L.nabla_calib_finalize.restype = i32
             L.nabla_calib_finalize.argtypes = [sp, vp, i32, vp, vp]
+            L.nabla_build_mask_xattn.restype = i32
+            L.nabla_build_mask_xattn.argtypes = [sp, ctypes.POINTER(_MaskParams), i32, vp, vp, vp,
+                                                 vp, vp, vp, i64, vp, vp, vp]
             L.bsa_bwd.restype = i32
             L.bsa_bwd.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, vp, f32, vp, vp, vp, vp, vp]
             L.bsa_fwd_with_mask_static.restype = i32
@@ -384,3 +388,38 @@ def bsa_bwd(q, k, v, o, dout, lse, row_ptr, col_idx, scale: Optional[float] = No
                          _ptr(lse), _ptr(row_ptr), _ptr(col_idx), float(scale or 0.0), _ptr(dq),
                          _ptr(dk), _ptr(dv), _ptr(workspace.buf), _stream(stream)))
     return dq, dk, dv
+
+
+def nabla_build_mask_xattn(q, k, thr: float, stride: int = 8, tile_grid=None,
+                           sta: Optional[Tuple[int, int, int]] = None, topk: int = 0,
+                           want_mask: bool = False, want_scores: bool = False,
+                           col_capacity: Optional[int] = None,
+                           workspace: Optional[Workspace] = None, out=None, stream=None):
+    """Block CSR selected from XAttention antidiagonal scores (stride 4, 8, 16).
+
+    Returns (row_ptr, col_idx, nnz, mask or None, scores fp32 [B,H,nb,nb] or None)."""
+    torch = _torch()
+    _bf16_contig(q, k)
+    shape = _shape_of(q, tile_grid)
+    B, H, S, d = q.shape
+    nb = S // 64
+    if workspace is None:
+        workspace = Workspace.create(shape, OP_BUILD_XATTN, q.device, stream)
+    if out is None:
+        cap = col_capacity if col_capacity is not None else B * H * nb * nb
+        row_ptr = torch.empty(B * H * nb + 1, dtype=torch.int32, device=q.device)
+        col_idx = torch.empty(max(cap, 1), dtype=torch.int32, device=q.device)
+        nnz = torch.empty(1, dtype=torch.int32, device=q.device)
+        mask = torch.empty((B, H, nb, nb), dtype=torch.uint8, device=q.device) if want_mask else None
+    else:
+        row_ptr, col_idx, nnz, mask = out
+        cap = col_idx.numel() if col_capacity is None else col_capacity
+    scores = (torch.empty((B, H, nb, nb), dtype=torch.float32, device=q.device)
+              if want_scores else None)
+    prm = _MaskParams(float(thr), 1 if sta is not None else 0,
+                      *(sta if sta is not None else (0, 0, 0)), int(topk))
+    _check(lib().nabla_build_mask_xattn(ctypes.byref(shape), ctypes.byref(prm), int(stride),
+                                        _ptr(q), _ptr(k), _ptr(scores), _ptr(mask), _ptr(row_ptr),
+                                        _ptr(col_idx), int(cap), _ptr(nnz), _ptr(workspace.buf),
+                                        _stream(stream)))
+    return row_ptr, col_idx, nnz, mask, scores

@@ -544,6 +544,28 @@ cudaError_t launch_select(const double* L, int64_t nrows, int nb, float thr, int
   return cudaGetLastError();
 }
 
+// The selection (a4-a6) on given non-negative block weights instead of the
+// softmax of the pooled map: each row normalised by its sum, then the mass
+// rule at thr or the top-k rule, then the STA window.
+cudaError_t launch_select_weights(const float* weights, int64_t nrows, int nb, float thr, int topk,
+                                  int use_sta, int wt, int wh, int ww, int Tt, int Th, int Tw,
+                                  uint32_t* bits, int32_t* counts, uint8_t* mask_u8,
+                                  cudaStream_t st) {
+  SelectParams prm{thr, use_sta, wt, wh, ww, Tt, Th, Tw, topk};
+  const size_t per_warp = static_cast<size_t>(nb) * sizeof(uint32_t);
+  int wpc = static_cast<int>((200u * 1024u) / per_warp);
+  wpc = wpc < 1 ? 1 : (wpc > 8 ? 8 : wpc);
+  const size_t smem = per_warp * wpc;
+  cudaError_t e = cudaFuncSetAttribute(select_kernel<true>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  const unsigned grid = static_cast<unsigned>((nrows + wpc - 1) / wpc);
+  select_kernel<true><<<grid, 32 * wpc, smem, st>>>(weights, nrows, nb, wpc, prm, bits, counts,
+                                                    mask_u8, nullptr);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_calib_select(const float* energy, int64_t nrows, int nb, float eps,
                                 int32_t* votes, cudaStream_t st) {
   SelectParams prm{eps, 0, 0, 0, 0, 1, 1, 1, 0};

@@ -49,6 +49,13 @@ cudaError_t launch_bsa_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const C
                            float* dvec, uint32_t* colbits, void* dq, void* dk, void* dv,
                            int* status, int BH, int S, int d, float scale, uint64_t wait_limit_ns,
                            cudaStream_t st);
+cudaError_t launch_select_weights(const float* weights, int64_t nrows, int nb, float thr, int topk,
+                                  int use_sta, int wt, int wh, int ww, int Tt, int Th, int Tw,
+                                  uint32_t* bits, int32_t* counts, uint8_t* mask_u8,
+                                  cudaStream_t st);
+cudaError_t launch_xattn_scores(const CUtensorMap& q, const CUtensorMap& k, float* lse2,
+                                float* scores, int* status, int BH, int S, int d, int St,
+                                uint64_t wait_limit_ns, cudaStream_t st);
 cudaError_t launch_mma_selftest(const CUtensorMap& a, const CUtensorMap& b, const void* a_glob,
                                 float* c, int variant, int* status, uint64_t lim,
                                 cudaStream_t st);
@@ -138,6 +145,23 @@ BwdLayout bwd_layout(const nabla_shape* s) {
   return l;
 }
 
+struct XattnLayout {
+  size_t lse2, scores, bits, counts, total;
+};
+
+// Sized for the smallest supported stride (4): S/4 strided rows per head.
+XattnLayout xattn_layout(const nabla_shape* s) {
+  const size_t nb = s->S / 64, BH = static_cast<size_t>(s->B) * s->H, nw = (nb + 31) / 32;
+  XattnLayout l;
+  size_t off = kHeaderBytes;
+  l.lse2 = off; off = align256(off + BH * (s->S / 4) * 4);
+  l.scores = off; off = align256(off + BH * nb * nb * 4);
+  l.bits = off; off = align256(off + BH * nb * nw * 4);
+  l.counts = off; off = align256(off + BH * nb * 4);
+  l.total = off;
+  return l;
+}
+
 struct MaskLayout {
   size_t bits, counts, row_ptr, col_idx, total;
 };
@@ -208,6 +232,22 @@ nabla_status make_map_raster(CUtensorMap* map, const void* ptr, const nabla_shap
   return NABLA_OK;
 }
 
+// [rows][St][d] bf16 viewed as stride-St groups of token rows: 3D boxes of
+// 64 x 1 x 128 pick one token of each of 128 consecutive groups (128-byte swizzle).
+nabla_status make_map_strided(CUtensorMap* map, const void* ptr, uint64_t groups, int St, int d) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return fail(NABLA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(St), groups};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(St) * d * 2};
+  cuuint32_t box[3] = {64, 1, 128};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(NABLA_ERR_CUDA, "cuTensorMapEncodeTiled (3D) failed");
+  return NABLA_OK;
+}
+
 int* status_ptr(void* ws) { return static_cast<int*>(ws); }
 
 nabla_status run_fwd(const nabla_shape* shape, const void* q, const void* k, const void* v,
@@ -259,6 +299,7 @@ size_t nabla_workspace_size(const nabla_shape* shape, int op) {
     case NABLA_OP_FWD: return kHeaderBytes;
     case NABLA_OP_FWD_WITH_MASK: return mask_layout(shape).total;
     case NABLA_OP_BWD: return bwd_layout(shape).total;
+    case NABLA_OP_BUILD_XATTN: return xattn_layout(shape).total;
     default: g_last_error = "unknown op"; return 0;
   }
 }
@@ -482,6 +523,59 @@ nabla_status bsa_bwd(const nabla_shape* shape, const void* q, const void* k, con
       shape->B * shape->H, shape->S, shape->d, scale, g_wait_limit_ns.load(),
       reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "bsa_bwd launch");
+  return NABLA_OK;
+}
+
+nabla_status nabla_build_mask_xattn(const nabla_shape* shape, const nabla_mask_params* params,
+                                    int32_t stride, const void* q, const void* k, float* scores,
+                                    uint8_t* mask_u8, int32_t* row_ptr, int32_t* col_idx,
+                                    int64_t col_capacity, int32_t* nnz_out, void* workspace,
+                                    nabla_stream_t stream) {
+  nabla_status s = check_shape(shape);
+  if (s != NABLA_OK) return s;
+  if ((s = require_tile_major(shape)) != NABLA_OK) return s;
+  if (params == nullptr) return fail(NABLA_ERR_INVALID_ARG, "params is NULL");
+  if (stride != 4 && stride != 8 && stride != 16)
+    return fail(NABLA_ERR_UNSUPPORTED, "stride must be 4, 8 or 16");
+  if (!(params->thr >= 0.f && params->thr <= 1.f))
+    return fail(NABLA_ERR_UNSUPPORTED, "thr must lie in [0, 1]");
+  if (params->topk < 0) return fail(NABLA_ERR_INVALID_ARG, "topk must be >= 0");
+  if (params->use_sta && (params->wt < 0 || params->wh < 0 || params->ww < 0))
+    return fail(NABLA_ERR_INVALID_ARG, "STA half-windows must be non-negative");
+  if (params->use_sta && (shape->Tt <= 0 || shape->Th <= 0 || shape->Tw <= 0 ||
+                          static_cast<int64_t>(shape->Tt) * shape->Th * shape->Tw != shape->S / 64))
+    return fail(NABLA_ERR_INVALID_ARG, "the STA window needs a tile grid with Tt*Th*Tw = S/64");
+  if (!q || !k || !row_ptr || !workspace) return fail(NABLA_ERR_INVALID_ARG, "null pointer");
+  if (col_capacity > 0 && col_idx == nullptr) return fail(NABLA_ERR_INVALID_ARG, "col_idx is NULL");
+  if (col_capacity < 0) return fail(NABLA_ERR_INVALID_ARG, "col_capacity is negative");
+  if (!aligned16(q) || !aligned16(k) || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return fail(NABLA_ERR_INVALID_ARG, "q, k need 16-byte and workspace 256-byte alignment");
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const XattnLayout lay = xattn_layout(shape);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  float* lse2 = reinterpret_cast<float*>(ws + lay.lse2);
+  float* X = scores ? scores : reinterpret_cast<float*>(ws + lay.scores);
+  uint32_t* bits = reinterpret_cast<uint32_t*>(ws + lay.bits);
+  int32_t* counts = reinterpret_cast<int32_t*>(ws + lay.counts);
+  const int nb = shape->S / 64, BH = shape->B * shape->H;
+  const int64_t nrows = static_cast<int64_t>(BH) * nb;
+  const uint64_t groups = static_cast<uint64_t>(BH) * (shape->S / stride);
+  CUtensorMap mq, mk;
+  if ((s = make_map_strided(&mq, q, groups, stride, shape->d)) != NABLA_OK) return s;
+  if ((s = make_map_strided(&mk, k, groups, stride, shape->d)) != NABLA_OK) return s;
+  cudaError_t e = nabla::launch_xattn_scores(mq, mk, lse2, X, status_ptr(workspace), BH, shape->S,
+                                             shape->d, stride, g_wait_limit_ns.load(), st);
+  if (e != cudaSuccess) return cuda_fail(e, "xattn scores launch");
+  // without the STA window the tile grid is not used (a 1 x 1 x nb grid stands in)
+  const bool sta = params->use_sta != 0;
+  e = nabla::launch_select_weights(X, nrows, nb, params->thr, params->topk, sta ? 1 : 0,
+                                   params->wt, params->wh, params->ww, sta ? shape->Tt : nb,
+                                   sta ? shape->Th : 1, sta ? shape->Tw : 1, bits, counts,
+                                   mask_u8, st);
+  if (e != cudaSuccess) return cuda_fail(e, "select launch");
+  e = nabla::launch_scan_fill(bits, counts, nrows, nb, row_ptr, col_idx, col_capacity, nnz_out,
+                              status_ptr(workspace), st);
+  if (e != cudaSuccess) return cuda_fail(e, "scan/fill launch");
   return NABLA_OK;
 }
 

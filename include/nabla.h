@@ -82,7 +82,8 @@ enum {
     NABLA_OP_BUILD_MASK = 0,     /* workspace for nabla_build_mask */
     NABLA_OP_FWD = 1,            /* workspace for bsa_fwd */
     NABLA_OP_FWD_WITH_MASK = 2,  /* workspace for bsa_fwd_with_mask */
-    NABLA_OP_BWD = 3             /* workspace for bsa_bwd */
+    NABLA_OP_BWD = 3,            /* workspace for bsa_bwd */
+    NABLA_OP_BUILD_XATTN = 4     /* workspace for nabla_build_mask_xattn */
 };
 
 /* Bytes of workspace the operation needs for this shape (0 on a bad shape).
@@ -192,6 +193,30 @@ NABLA_API nabla_status bsa_fwd_with_mask_static(const nabla_shape* shape, const 
                                                 const uint8_t* mask_u8, float scale, void* o,
                                                 float* lse, int32_t* status_out,
                                                 nabla_stream_t stream);
+
+/*
+ * Block mask from XAttention antidiagonal scores instead of the pooled map
+ * ("XAttention: Block Sparse Attention with Antidiagonal Scoring" notes:
+ * blocks scored along antidiagonals, selected by a threshold).  With stride St
+ * (4, 8 or 16), strided rows i, j of a head score
+ *     a_ij = (1/St) sum_{s<St} q_{i*St + St-1-s} . k_{j*St + s} / sqrt(d)
+ * (the mean of the antidiagonal of the St x St sub-block of Q K^T), p_i =
+ * softmax over all strided keys, and block (r, c) scores the mean over r's
+ * 64/St strided rows of the mass p puts on c's strided keys; each row of
+ * scores sums to 1.  The scores then go through nabla_build_mask's selection
+ * (params: thr mass rule or topk, optional STA window; the tile grid is
+ * needed only for the STA window), giving the same CSR outputs.
+ *   scores   device fp32 [B,H,nb,nb] or NULL (then kept in the workspace)
+ *   workspace  device, nabla_workspace_size(shape, NABLA_OP_BUILD_XATTN) bytes
+ * Other arguments as for nabla_build_mask; tile-major tokens only.
+ */
+NABLA_API nabla_status nabla_build_mask_xattn(const nabla_shape* shape,
+                                              const nabla_mask_params* params, int32_t stride,
+                                              const void* q, const void* k, float* scores,
+                                              uint8_t* mask_u8, int32_t* row_ptr,
+                                              int32_t* col_idx, int64_t col_capacity,
+                                              int32_t* nnz_out, void* workspace,
+                                              nabla_stream_t stream);
 
 /*
  * Block-sparse attention backward: the gradients of bsa_fwd's O with respect
