@@ -1,0 +1,137 @@
+"""Numerical edge cases on the GPU vs the fp64 oracle: logits that rise
+steeply from key tile to key tile (every later tile's maximum exceeds the
+running maximum by more than 2^8, so the forward's lazy rescale of O and l
+runs on most tiles), all-equal scores, and thr = 1 (one block per row)."""
+import numpy as np
+import pytest
+
+from _parity import compare_attention, to_device_bf16
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def nl():
+    import block_sparse_attention_23_b200 as nl
+    nl.lib()
+    return nl
+
+
+def _bf16_bits(x):
+    x = np.asarray(x, dtype=np.float32)
+    u = x.view(np.uint32)
+    u = (u + 0x7FFF + ((u >> 16) & 1)) >> 16
+    return u.astype(np.uint16)
+
+
+def _rising(B, H, nb, d, step, seed):
+    """q = e0 + noise; key block c = (c * step) e0 + noise: the logits of key
+    block c are about c * step / sqrt(d) larger than those of block c - 1."""
+    rng = np.random.default_rng(seed)
+    S = 64 * nb
+    q = rng.standard_normal((B, H, S, d)).astype(np.float32) * 0.2
+    q[..., 0] += 1.0
+    k = rng.standard_normal((B, H, S, d)).astype(np.float32) * 0.2
+    k[..., 0] += np.repeat(np.arange(nb) * step, 64)[None, None, :]
+    v = rng.standard_normal((B, H, S, d)).astype(np.float32)
+    return _bf16_bits(q), _bf16_bits(k), _bf16_bits(v)
+
+
+@pytest.mark.parametrize("d,nb,order", [(128, 12, "ascending"), (64, 9, "ascending"),
+                                        (128, 12, "descending")])
+def test_forward_lazy_rescale_path(nl, oracle_mod, d, nb, order):
+    import torch
+    B, H = 1, 2
+    step = 1.0 * np.sqrt(d) * 10.0 / 1.4427     # ~10 log2 units per key block > 2^8 threshold
+    q, k, v = _rising(B, H, nb, d, step, seed=nb)
+    if order == "descending":                   # the first tile holds the maximum
+        k = np.ascontiguousarray(k.reshape(B, H, nb, 64, d)[:, :, ::-1].reshape(k.shape))
+    mask = np.ones((B, H, nb, nb), dtype=np.uint8)
+    mask[:, :, 1, ::2] = 0                      # a row with gaps
+    qd, kd, vd = to_device_bf16(q), to_device_bf16(k), to_device_bf16(v)
+    ws = nl.Workspace.create(nl.make_shape(B, H, 64 * nb, d), nl.OP_FWD_WITH_MASK)
+    o, lse = nl.bsa_fwd_with_mask(qd, kd, vd, torch.from_numpy(mask).cuda(), workspace=ws)
+    assert ws.query_status() == 0
+    rows = np.arange(B * H * 64 * nb, dtype=np.int64)
+    ro, rl = oracle_mod.masked_attention(q, k, v, mask, rows)
+    compare_attention(o.float().cpu().numpy().reshape(-1, d), lse.cpu().numpy().reshape(-1), ro, rl)
+
+
+def test_backward_and_energy_with_rising_logits(nl, oracle_mod):
+    import torch
+    from test_gpu_bwd import _compare, _csr, _host
+    B, H, nb, d = 1, 2, 8, 128
+    step = np.sqrt(d) * 6.0 / 1.4427
+    q, k, v = _rising(B, H, nb, d, step, seed=3)
+    dO = _bf16_bits(np.random.default_rng(4).standard_normal(q.shape).astype(np.float32))
+    mask = (np.random.default_rng(5).random((B, H, nb, nb)) < 0.6).astype(np.uint8)
+    mask[..., np.arange(nb), np.arange(nb)] = 1
+    qd, kd, vd, dod = (to_device_bf16(a) for a in (q, k, v, dO))
+    rp, ci = _csr(mask)
+    shape = nl.make_shape(B, H, 64 * nb, d)
+    o, lse = nl.bsa_fwd(qd, kd, vd, rp, ci, workspace=nl.Workspace.create(shape, nl.OP_FWD))
+    dq, dk, dv = nl.bsa_bwd(qd, kd, vd, o, dod, lse, rp, ci)
+    rq, rk, rv = oracle_mod.attention_bwd(q, k, v, dO, mask)
+    _compare("dK", _host(dk), rk)
+    _compare("dV", _host(dv), rv)
+    # dQ = scale sum_j dS_ij k_j sums terms far larger than the result here
+    # (the keys share a component of ~300 that the terms cancel), so its error
+    # is bounded by the rounding unit times the magnitude of the terms: dS and
+    # the D term enter the products as bf16 (u = 2^-9), D from the bf16 O
+    err = np.abs(_host(dq) - rq)
+    bound = _dq_term_bound(q, k, v, dO, mask)
+    assert (err <= 4 * 2.0 ** -9 * bound + 2e-2 * np.abs(rq).max()).all(), \
+        f"max err / bound {np.max(err / (bound + 1e-30)):.3g}"
+    _, ora_lse = oracle_mod.masked_attention(q, k, v, mask)
+    lse32 = torch.from_numpy(ora_lse.astype(np.float32).reshape(B, H, 64 * nb)).cuda()
+    E, _ = nl.nabla_block_energy(qd, kd, lse32, rp, ci)
+    ref, _ = oracle_mod.block_energy(q, k, ora_lse.reshape(B, H, 64 * nb), mask)
+    # blocks far below the row maximum carry ~0 mass in both; compare where it matters
+    big = ref > 1e-30
+    np.testing.assert_allclose(E.cpu().numpy()[big], ref[big], rtol=2e-4, atol=0)
+    assert np.abs(E.cpu().numpy()[~big]).max(initial=0.0) < 1e-30
+
+
+def _f32(bits):
+    return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def _dq_term_bound(q, k, v, dO, mask):
+    """Per element of dQ: scale * (sum_j |dS_ij| |k_jc| + |D_i| sum_j p_ij |k_jc|),
+    the magnitude of the terms dQ sums, in fp64 on the host."""
+    B, H, S, d = q.shape
+    scale = 1.0 / np.sqrt(d)
+    out = np.zeros((B, H, S, d))
+    keep = np.repeat(np.repeat(mask.astype(bool), 64, axis=2), 64, axis=3)
+    for b in range(B):
+        for h in range(H):
+            Q, K, V, G = (_f32(a[b, h]) for a in (q, k, v, dO))
+            s = Q @ K.T * scale
+            s = np.where(keep[b, h], s, -np.inf)
+            p = np.exp(s - s.max(axis=1, keepdims=True))
+            p /= p.sum(axis=1, keepdims=True)
+            dP = G @ V.T
+            D = (p * dP).sum(axis=1, keepdims=True)
+            dS = p * (dP - D)
+            out[b, h] = scale * (np.abs(dS) @ np.abs(K) + np.abs(D) * (p @ np.abs(K)))
+    return out.reshape(-1, d)
+
+
+def test_equal_scores_and_thr_one(nl, oracle_mod, synth_mod):
+    import torch
+    # q = 0: every score ties; thr = 1 keeps exactly the first sorted block,
+    # which ties go to the lower index (block 0) in every row
+    B, H, nb, d = 1, 2, 6, 64
+    S = 64 * nb
+    q = np.zeros((B, H, S, d), dtype=np.uint16)
+    k = synth_mod.make_tensor(1, 8, B, H, S, d, pos_weight=0.0, noise_weight=1.0)
+    v = synth_mod.make_tensor(2, 8, B, H, S, d, pos_weight=0.0, noise_weight=1.0)
+    qd, kd, vd = to_device_bf16(q), to_device_bf16(k), to_device_bf16(v)
+    rp, ci, nnz, mask = nl.nabla_build_mask(qd, kd, (1, 2, 3), 1.0, None, want_mask=True)
+    m = mask.cpu().numpy()
+    assert (m.sum(axis=-1) == 1).all() and (m[..., 0] == 1).all()
+    om = oracle_mod.build_mask(q, k, (1, 2, 3), 1.0, None)
+    assert np.array_equal(m, om)
+    o, lse = nl.bsa_fwd(qd, kd, vd, rp, ci)
+    ro, rl = oracle_mod.masked_attention(q, k, v, om)
+    compare_attention(o.float().cpu().numpy().reshape(-1, d), lse.cpu().numpy().reshape(-1), ro, rl)
