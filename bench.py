@@ -159,14 +159,36 @@ def oracle_sample(w, q, k, v, nrows: int, head: int = 0, seed: int = 0):
     rng = np.random.default_rng(seed)
     rows = np.sort(rng.choice(S, size=nrows, replace=False)).astype(np.int64)
     t1 = time.perf_counter()
-    oracle.masked_attention(qh, kh, vh, mask, rows)
+    ro, rl = oracle.masked_attention(qh, kh, vh, mask, rows)
     t_attn = time.perf_counter() - t1
     kept_blocks = mask[0, 0].sum(axis=1)[rows // 64]
     flops = float((4.0 * w.d * 64 * kept_blocks).sum())
     t = t_attn + t_mask * nrows / S      # the mask cost of the sampled rows' share
     desc = (f"head {head}: full oracle mask ({t_mask:.2f} s, charged pro rata) + oracle "
             f"attention on {nrows} seeded query rows ({t_attn:.2f} s)")
-    return flops / t / 1e12, t, desc
+    return flops / t / 1e12, t, desc, (mask[0, 0], rows, ro, rl)
+
+
+def parity_sample(gpu_row_ptr, gpu_col_idx, gpu_o, gpu_lse, nb, d, sample):
+    """The bench layer's head 0 against the oracle's run above: mask rows that
+    differ, and O / LSE errors on the sampled rows whose mask row agrees."""
+    omask, rows, ro, rl = sample
+    rp = gpu_row_ptr[:nb + 1].cpu().numpy()
+    ci = gpu_col_idx[:int(rp[-1])].cpu().numpy()
+    gmask = np.zeros((nb, nb), dtype=np.uint8)
+    gmask[np.repeat(np.arange(nb), np.diff(rp)), ci] = 1
+    same = (gmask == omask).all(axis=1)
+    keep = same[rows // 64]
+    go = gpu_o[0, 0].float().cpu().numpy()[rows[keep]]
+    gl = gpu_lse[0, 0].cpu().numpy()[rows[keep]]
+    err = np.abs(go - ro[keep])
+    some = bool(keep.any())
+    return {"head": 0, "mask_rows_differing": int((~same).sum()), "mask_rows": nb,
+            "rows_compared": int(keep.sum()),
+            "o_max_abs": float(err.max()) if some else None,
+            "o_mean_abs": float(err.mean()) if some else None,
+            "lse_max_abs": float(np.abs(gl - rl[keep]).max()) if some else None,
+            "bars": {"o_max_abs": 2e-2, "o_mean_abs": 2e-3, "lse_max_abs": 1e-3}}
 
 
 def run_reference(args):
@@ -184,7 +206,7 @@ def run_reference(args):
         oracle_sample(w, q, k, v, nrows, head=i % w.H, seed=i)
     vals, times, desc = [], [], ""
     for i in range(args.steps):
-        val, t, desc = oracle_sample(w, q, k, v, nrows, head=(args.warmup + i) % w.H,
+        val, t, desc, _ = oracle_sample(w, q, k, v, nrows, head=(args.warmup + i) % w.H,
                                      seed=1000 + i)
         vals.append(val)
         times.append(t)
@@ -349,9 +371,12 @@ def run_ours(args):
     ws_fwd_r = nl.Workspace.create(shape_r, nl.OP_FWD, dev)
     o_r, lse_r = torch.empty_like(q), torch.empty_like(lse)
 
+    # separate CSR buffers: the step's own CSR stays intact for the parity sample
+    mask_out_x = tuple(t.clone() if t is not None else None for t in mask_out)
+
     def raster_step():
         rp, ci, _, _ = nl.nabla_build_mask(qr, kr, w.tile_grid, w.thr, w.sta, workspace=ws_mask_r,
-                                           out=mask_out, layout=nl.LAYOUT_RASTER)
+                                           out=mask_out_x, layout=nl.LAYOUT_RASTER)
         nl.bsa_fwd(qr, kr, vr, rp, ci, workspace=ws_fwd_r, out=(o_r, lse_r), tile_grid=w.tile_grid,
                    layout=nl.LAYOUT_RASTER)
 
@@ -443,12 +468,12 @@ def run_ours(args):
 
     def xattn_call():
         nl.nabla_build_mask_xattn(q, k, w.thr, 8, tile_grid=w.tile_grid, sta=w.sta,
-                                  workspace=ws_x, out=mask_out)
+                                  workspace=ws_x, out=mask_out_x)
 
     xattn_call()
     torch.cuda.synchronize()
     ws_x.check()
-    x_kept = int(mask_out[2].item())
+    x_kept = int(mask_out_x[2].item())
     n_x = 3
     a.record(stream)
     for _ in range(n_x):
@@ -520,9 +545,10 @@ def run_ours(args):
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         import oracle
         oracle.build()
-        val, t, desc = oracle_sample(w, q16, k16, v16, args.ref_rows, head=0, seed=0)
+        val, t, desc, sample = oracle_sample(w, q16, k16, v16, args.ref_rows, head=0, seed=0)
         line["cpu_baseline"] = {"value": val, "unit": "TFLOP/s", "cores": oracle.max_threads(),
                                 "kind": "oracle", "sample": desc}
+        line["parity_sample"] = parity_sample(mask_out[0], mask_out[1], o, lse, nb, d, sample)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if ws > 1:
