@@ -91,7 +91,7 @@ struct BwdParams {
   const int32_t* row_ptr;      // CSR (query-stationary) or unused
   const int32_t* col_idx;
   const uint32_t* colbits;     // [BH*nb][nw] column bitmaps (key-stationary)
-  const float* lse;            // [BH*S]
+  const float* lse2;           // [BH*S] LSE * log2(e)
   const float* dvec;           // [BH*S] rowsum(dO o O)
   __nv_bfloat16* out1;         // dV or dQ
   __nv_bfloat16* out2;         // dK or null
@@ -116,10 +116,13 @@ __device__ __forceinline__ void b_abort(volatile int* abort, int* status) {
 
 // D_i = sum_k dO_ik O_ik in fp32 from the bf16 tensors.  d/8 lanes per row
 // (16-byte loads), rows packed into warps.  HBM-bound: reads O and dO once.
+// It also writes lse2 = LSE * log2(e), the form the exponentials take.
 template <int D>
 __global__ void __launch_bounds__(256) bwd_dvec_kernel(const __nv_bfloat16* __restrict__ o,
                                                        const __nv_bfloat16* __restrict__ dout,
-                                                       float* __restrict__ dvec, int64_t rows) {
+                                                       const float* __restrict__ lse,
+                                                       float* __restrict__ dvec,
+                                                       float* __restrict__ lse2, int64_t rows) {
   constexpr int kLanes = D / 8;
   const int64_t gt = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   const int64_t row = gt / kLanes;
@@ -137,7 +140,10 @@ __global__ void __launch_bounds__(256) bwd_dvec_kernel(const __nv_bfloat16* __re
   }
 #pragma unroll
   for (int off = kLanes / 2; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-  if (row < rows && chunk == 0) dvec[row] = s;
+  if (row < rows && chunk == 0) {
+    dvec[row] = s;
+    lse2[row] = lse[row] * 1.4426950408889634f;
+  }
 }
 
 // Column bitmaps of the block CSR: bit r of colbits[bh*nb + c] is set iff row
@@ -317,7 +323,7 @@ __global__ void __launch_bounds__(kBThreads, 1)
           }
           if (kKV) {   // LSE and D of the 64 query rows of entry e
             const uint32_t vs = sVec + s * L::kVecBytes;
-            bulk_load(vs + e * 256, prm.lse + row0 + static_cast<int64_t>(j) * 64, 256, fb);
+            bulk_load(vs + e * 256, prm.lse2 + row0 + static_cast<int64_t>(j) * 64, 256, fb);
             bulk_load(vs + kBT * 4 + e * 256, prm.dvec + row0 + static_cast<int64_t>(j) * 64, 256, fb);
           }
         }
@@ -431,11 +437,10 @@ __global__ void __launch_bounds__(kBThreads, 1)
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const uint32_t tb = tmem + lane_off;
     const float sl2 = prm.scale_log2;
-    constexpr float kL2e = 1.4426950408889634f;
     float row_nlse2 = 0.f, row_d = 0.f;
     if (!kKV && x < nx) {
       const int64_t gr = static_cast<int64_t>(bh) * prm.S + static_cast<int64_t>(r0 + x) * 64 + (row & 63);
-      row_nlse2 = -prm.lse[gr] * kL2e;
+      row_nlse2 = -prm.lse2[gr];
       row_d = prm.dvec[gr];
     }
     bool ok = true;
@@ -491,7 +496,7 @@ __global__ void __launch_bounds__(kBThreads, 1)
 #pragma unroll
               for (int u = 0; u < 2; ++u)
                 e[u] = member ? fast_exp2(fmaf(__uint_as_float(sv[ch][2 * i + u]), sl2,
-                                               -lv[2 * i + u] * kL2e))
+                                               -lv[2 * i + u]))
                               : 0.f;
               pk[ch][i] = pack_bf16x2(e[0], e[1]);
             }
@@ -530,21 +535,19 @@ __global__ void __launch_bounds__(kBThreads, 1)
         if (kKV) load32(vd_addr + 128 * ch, dvv);
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          float ds[2];
-#pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int c = 32 * ch + 2 * i + u;
-            float pc, dd;
-            if (kKV) {
-              pc = __uint_as_float(u ? (pk[ch][i] & 0xFFFF0000u) : (pk[ch][i] << 16));
-              dd = dvv[2 * i + u];
-            } else {
-              pc = p[c & (kKV ? 0 : 63)];
-              dd = row_d;
-            }
-            ds[u] = member ? pc * (__uint_as_float(dv[ch][2 * i + u]) - dd) : 0.f;
+          // dS = P o (dP - D), two lanes of work per packed instruction
+          const int c = 32 * ch + 2 * i;
+          float2 pc, dd;
+          if (kKV) {
+            pc = make_float2(__uint_as_float(pk[ch][i] << 16), __uint_as_float(pk[ch][i] & 0xFFFF0000u));
+            dd = make_float2(dvv[2 * i], dvv[2 * i + 1]);
+          } else {
+            pc = make_float2(p[c & (kKV ? 0 : 63)], p[(c + 1) & (kKV ? 0 : 63)]);
+            dd = make_float2(row_d, row_d);
           }
-          dk[i] = pack_bf16x2(ds[0], ds[1]);
+          const float2 ds = fsubmul2(make_float2(__uint_as_float(dv[ch][2 * i]),
+                                                 __uint_as_float(dv[ch][2 * i + 1])), dd, pc);
+          dk[i] = member ? pack_bf16x2(ds.x, ds.y) : 0u;
         }
         tmem_st16(tb + kColDP + 32 * half + 16 * ch, dk);
       }
@@ -623,7 +626,7 @@ static cudaError_t launch_bwd_t(const CUtensorMap* maps, const BwdParams& prm, i
 cudaError_t launch_bsa_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                            const CUtensorMap& mdo, const void* o, const void* dout,
                            const float* lse, const int32_t* row_ptr, const int32_t* col_idx,
-                           float* dvec, uint32_t* colbits, void* dq, void* dk, void* dv,
+                           float* dvec, float* lse2, uint32_t* colbits, void* dq, void* dk, void* dv,
                            int* status, int BH, int S, int d, float scale, uint64_t wait_limit_ns,
                            cudaStream_t st) {
   const int nb = S / 64;
@@ -635,10 +638,12 @@ cudaError_t launch_bsa_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const C
     const unsigned grid = static_cast<unsigned>((threads + 255) / 256);
     if (d == 128)
       bwd_dvec_kernel<128><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(o),
-                                                 static_cast<const __nv_bfloat16*>(dout), dvec, rows);
+                                                 static_cast<const __nv_bfloat16*>(dout), lse, dvec,
+                                                 lse2, rows);
     else
       bwd_dvec_kernel<64><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(o),
-                                                static_cast<const __nv_bfloat16*>(dout), dvec, rows);
+                                                static_cast<const __nv_bfloat16*>(dout), lse, dvec,
+                                                lse2, rows);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
@@ -656,7 +661,7 @@ cudaError_t launch_bsa_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const C
   prm.row_ptr = row_ptr;
   prm.col_idx = col_idx;
   prm.colbits = colbits;
-  prm.lse = lse;
+  prm.lse2 = lse2;
   prm.dvec = dvec;
   prm.status = status;
   prm.S = S;

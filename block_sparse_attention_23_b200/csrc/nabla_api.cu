@@ -48,9 +48,9 @@ cudaError_t launch_vote_mask(const int32_t* votes, int64_t n, int32_t min_votes,
 cudaError_t launch_bsa_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                            const CUtensorMap& mdo, const void* o, const void* dout,
                            const float* lse, const int32_t* row_ptr, const int32_t* col_idx,
-                           float* dvec, uint32_t* colbits, void* dq, void* dk, void* dv,
-                           int* status, int BH, int S, int d, float scale, uint64_t wait_limit_ns,
-                           cudaStream_t st);
+                           float* dvec, float* lse2, uint32_t* colbits, void* dq, void* dk,
+                           void* dv, int* status, int BH, int S, int d, float scale,
+                           uint64_t wait_limit_ns, cudaStream_t st);
 cudaError_t launch_select_weights(const float* weights, int64_t nrows, int nb, float thr, int topk,
                                   int use_sta, int wt, int wh, int ww, int Tt, int Th, int Tw,
                                   uint32_t* bits, int32_t* counts, uint8_t* mask_u8,
@@ -141,7 +141,7 @@ BuildLayout build_layout(const nabla_shape* s) {
 }
 
 struct BwdLayout {
-  size_t dvec, colbits, total;
+  size_t dvec, lse2, colbits, total;
 };
 
 BwdLayout bwd_layout(const nabla_shape* s) {
@@ -149,6 +149,7 @@ BwdLayout bwd_layout(const nabla_shape* s) {
   BwdLayout l;
   size_t off = kHeaderBytes;
   l.dvec = off; off = align256(off + BH * s->S * 4);
+  l.lse2 = off; off = align256(off + BH * s->S * 4);
   l.colbits = off; off = align256(off + BH * nb * nw * 4);
   l.total = off;
   return l;
@@ -534,7 +535,7 @@ nabla_status bsa_bwd(const nabla_shape* shape, const void* q, const void* k, con
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   cudaError_t e = nabla::launch_bsa_bwd(
       mq, mk, mv, mdo, o, dout, lse, row_ptr, col_idx, reinterpret_cast<float*>(ws + lay.dvec),
-      reinterpret_cast<uint32_t*>(ws + lay.colbits), dq, dk, dv, status_ptr(workspace),
+      reinterpret_cast<float*>(ws + lay.lse2), reinterpret_cast<uint32_t*>(ws + lay.colbits), dq, dk, dv, status_ptr(workspace),
       shape->B * shape->H, shape->S, shape->d, scale, g_wait_limit_ns.load(),
       reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "bsa_bwd launch");

@@ -299,6 +299,18 @@ __device__ __forceinline__ void setmaxnreg_dec() {
 
 // ----------------------------------------------------------------- misc
 
+// Packed fp32 pairs (sm_100 f32x2 instructions): (a - b) * c for two lanes of
+// work in two instructions, same rounding as the scalar forms.
+__device__ __forceinline__ float2 fsubmul2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+      "sub.rn.f32x2 rd, ra, rb;\n\tmul.rn.f32x2 rd, rd, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+
 // 16-byte shared-memory load (volatile: stays after the waits that precede it).
 __device__ __forceinline__ float4 lds_f4(uint32_t addr) {
   float4 v;
