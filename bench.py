@@ -222,7 +222,7 @@ def run_reference(args):
     import oracle
     import synth
     oracle.build()
-    w = synth.WORKLOADS[WORKLOAD]
+    w = synth.WORKLOADS[args.workload]
     q, k, v = synth.make_qkv(w)
     cores = oracle.max_threads()
     nrows = args.ref_rows
@@ -262,7 +262,7 @@ def run_ours(args):
     import synth
     import block_sparse_attention_23_b200 as nl
     nl.lib()
-    w = synth.WORKLOADS[WORKLOAD]
+    w = synth.WORKLOADS[args.workload]
     if args.profile_heads:
         import dataclasses
         w = dataclasses.replace(w, H=args.profile_heads)   # profiling subset, not a bench line
@@ -509,11 +509,39 @@ def run_ours(args):
     x_flops = 4.0 * S * S * d * B * H / 8
     x_tflops = x_flops / (x_ms * 1e-3) / 1e12
 
+    # static-mask attention over a density sweep (i.i.d. N(0,1) Q, K, V on the
+    # 32,768-token sweep shape, Bernoulli block masks, diagonal forced), outside the step
+    sweep = []
+    if not args.profile_heads:
+        ws_ = synth.WORKLOADS["sweep"]
+        qs16, ks16, vs16 = synth.make_qkv(ws_, seed=args.seed)
+        qs, ks, vs = (torch.from_numpy(t.view(np.int16)).view(torch.bfloat16).to(dev)
+                      for t in (qs16, ks16, vs16))
+        shape_s = nl.make_shape(ws_.B, ws_.H, ws_.S, ws_.d)
+        wsw = nl.Workspace.create(shape_s, nl.OP_FWD_WITH_MASK, dev)
+        os_, ls_ = torch.empty_like(qs), torch.empty((ws_.B, ws_.H, ws_.S), dtype=torch.float32,
+                                                     device=dev)
+        for pden in ws_.densities:
+            mk = torch.from_numpy(synth.make_bernoulli_mask(0, ws_.B * ws_.H, ws_.nb, pden)).to(dev)
+            for _ in range(2):
+                nl.bsa_fwd_with_mask(qs, ks, vs, mk, workspace=wsw, out=(os_, ls_))
+            a.record(stream)
+            for _ in range(3):
+                nl.bsa_fwd_with_mask(qs, ks, vs, mk, workspace=wsw, out=(os_, ls_))
+            b.record(stream)
+            torch.cuda.synchronize()
+            wsw.check()
+            ms_ = a.elapsed_time(b) / 3
+            kept_s = int(mk.sum().item())
+            sweep.append({"density": pden, "kept_fraction": kept_s / mk.numel(), "ms": ms_,
+                          "kept_tflops": 4.0 * ws_.d * 64 * 64 * kept_s / (ms_ * 1e-3) / 1e12})
+        del qs, ks, vs, os_, ls_
+
     attn_tflops = kept_flops / (attn_ms * 1e-3) / 1e12
     peak = peaks["bf16_tflops_sustained"]
     exec_tiles = executed_tile_products(mask_out[0], mask_out[1], B * H, nb)
     exec_flops = 4.0 * d * 128 * 128 * exec_tiles
-    traffic = _traffic_per_launch()
+    traffic = _traffic_per_launch() if (args.workload == WORKLOAD and not args.profile_heads) else None
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": ws,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
@@ -522,7 +550,7 @@ def run_ours(args):
         "config": {"workload": _workload_desc(w), "global_batch": B * ws, "seq_len": S,
                    "heads": H, "head_dim": d,
                    "parallelism": "replicas" if ws > 1 else "single GPU",
-                   "l2": "inputs (Q,K,V 2.36 GB per rank) larger than L2; no flush",
+                   "l2": f"inputs (Q,K,V {3 * q.numel() * 2 / 1e9:.2f} GB per rank) larger than L2; no flush",
                    "kept_blocks": kept, "density": kept / (B * H * nb * nb),
                    "mask_arith": "fp64", "attn_arith": "bf16 MMA, fp32 accumulate"},
         "ms_per_layer": ms_per_step, "mask_ms": mask_ms, "attn_ms": attn_ms,
@@ -556,6 +584,10 @@ def run_ours(args):
                          "what": "E over the step's kept blocks (QK^T + exp + block sums), "
                                  "outside the step; FLOPs = 2*d*64*64 per block"},
         "calib_accumulate_ms": cal_ms,
+        "static_mask_sweep": {"workload": "32,768 tokens, 24 heads, d 128, Q,K,V ~ N(0,1), "
+                                          "Bernoulli(p) block masks with the diagonal forced; "
+                                          "mask compaction + attention per call",
+                              "points": sweep},
         "xattn_mask": {"bound": "tensor", "ms": x_ms, "achieved": x_tflops, "peak": peak,
                        "unit": "TFLOP/s", "frac": x_tflops / peak, "flops": x_flops,
                        "kept_blocks": x_kept, "density": x_kept / (B * H * nb * nb),
@@ -600,6 +632,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile-heads", type=int, default=0,
                     help="profiling only: run the layer with this many heads")
+    ap.add_argument("--workload", default=WORKLOAD, choices=["wan720p", "hunyuan720p", "small"],
+                    help="layer to time (default: the Wan 2.1 720p-shaped layer)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
