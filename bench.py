@@ -25,6 +25,7 @@ import json
 import os
 import statistics
 import subprocess
+import tempfile
 import sys
 import time
 
@@ -78,10 +79,11 @@ class ClockSampler:
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, index: int):
+    def __init__(self, index: int, log_dir=None):
         self.index = index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
+        base = log_dir or tempfile.gettempdir()
+        self.path = os.path.join(base, f"nabla_clocks_rank{index}.csv")
 
     def start(self):
         try:
@@ -307,7 +309,7 @@ def run_ours(args):
     torch.cuda.synchronize()
     if ws > 1:
         dist.barrier()
-    clocks = ClockSampler(local)
+    clocks = ClockSampler(local, args.clock_log_dir)
     clocks.start()
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
            torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
@@ -630,6 +632,8 @@ def main():
     ap.add_argument("--ref-rows", type=int, default=2048,
                     help="oracle attention rows per CPU sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--clock-log-dir", default=None,
+                    help="directory for the raw nvidia-smi clock samples (default: the temp dir)")
     ap.add_argument("--profile-heads", type=int, default=0,
                     help="profiling only: run the layer with this many heads")
     ap.add_argument("--workload", default=WORKLOAD, choices=["wan720p", "hunyuan720p", "small"],
