@@ -34,7 +34,8 @@ EXPORTED = ["nabla_workspace_size", "nabla_workspace_init", "nabla_query_status"
             "nabla_version", "nabla_set_wait_limit_ns", "nabla_selftest_mma",
             "bsa_fwd_with_mask_static", "nabla_reorder_tokens", "nabla_block_energy",
             "nabla_calib_accumulate", "nabla_calib_finalize", "bsa_bwd",
-            "nabla_build_mask_xattn"]
+            "nabla_build_mask_xattn", "nabla_layer_host_workspace_size", "nabla_layer_host",
+            "nabla_layer_host_chunks"]
 TO_TILE_MAJOR, TO_RASTER = 0, 1
 
 
@@ -112,6 +113,13 @@ def lib() -> ctypes.CDLL:
             L.bsa_bwd.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, vp, f32, vp, vp, vp, vp, vp]
             L.bsa_fwd_with_mask_static.restype = i32
             L.bsa_fwd_with_mask_static.argtypes = [sp, vp, vp, vp, vp, f32, vp, vp, vp, vp]
+            L.nabla_layer_host_workspace_size.restype = sz
+            L.nabla_layer_host_workspace_size.argtypes = [sp, i32]
+            L.nabla_layer_host_chunks.restype = ctypes.c_int64
+            L.nabla_layer_host_chunks.argtypes = [ctypes.c_int64, i32, vp, ctypes.c_int64]
+            L.nabla_layer_host.restype = i32
+            L.nabla_layer_host.argtypes = [sp, ctypes.POINTER(_MaskParams), vp, vp, vp, vp, vp,
+                                           i32, vp, vp]
             _lib = L
     return _lib
 
@@ -158,9 +166,11 @@ class Workspace:
     op: int
 
     @classmethod
-    def create(cls, shape: _Shape, op: int, device=None, stream=None) -> "Workspace":
+    def create(cls, shape: _Shape, op: int, device=None, stream=None, nbytes=None) -> "Workspace":
         torch = _torch()
-        n = workspace_size(shape, op)
+        n = workspace_size(shape, op) if nbytes is None else int(nbytes)
+        if n == 0:
+            raise NablaError(1, lib().nabla_last_error().decode())
         buf = torch.empty(n, dtype=torch.uint8, device=device or "cuda")
         _check(lib().nabla_workspace_init(_ptr(buf), _stream(stream)))
         return cls(buf, op)
@@ -300,6 +310,54 @@ def bsa_fwd_with_mask_static(q, k, v, mask_u8, scale: Optional[float] = None, ou
     _check(lib().bsa_fwd_with_mask_static(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v),
                                           _ptr(mask_u8), float(scale or 0.0), _ptr(o), _ptr(lse),
                                           _ptr(status_out), _stream(stream)))
+    return o, lse
+
+
+def layer_host_workspace(shape: _Shape, heads_per_chunk: int, device=None,
+                         stream=None) -> Workspace:
+    """Device workspace for nabla_layer_host with this shape and chunking."""
+    n = lib().nabla_layer_host_workspace_size(ctypes.byref(shape), int(heads_per_chunk))
+    return Workspace.create(shape, OP_BUILD_MASK, device, stream, nbytes=n)
+
+
+def layer_host_chunks(heads: int, heads_per_chunk: int):
+    """Chunk sizes (heads) nabla_layer_host streams B*H = ``heads`` heads in."""
+    n = int(lib().nabla_layer_host_chunks(int(heads), int(heads_per_chunk), None, 0))
+    buf = (ctypes.c_int32 * max(n, 1))()
+    lib().nabla_layer_host_chunks(int(heads), int(heads_per_chunk), buf, n)
+    return [int(buf[i]) for i in range(n)]
+
+
+def nabla_layer_host(q, k, v, tile_grid, thr: float, sta: Optional[Tuple[int, int, int]] = None,
+                     topk: int = 0, heads_per_chunk: int = 4,
+                     workspace: Optional[Workspace] = None, out=None, stream=None):
+    """One NABLA layer (mask + block-sparse forward, scale 1/sqrt(d)) on host
+    tensors: q, k, v contiguous bf16 CPU tensors [B,H,S,d] (pinned for
+    copy/compute overlap).  Heads stream through the device in chunks of at
+    most ``heads_per_chunk`` (``layer_host_chunks`` gives the schedule).  Returns host (O bf16, LSE fp32); ``out`` may pass
+    preallocated host (O, LSE).  The call only queues the work: synchronise
+    ``stream`` (the current stream by default) before reading the outputs."""
+    torch = _torch()
+    for t in (q, k, v):
+        if t.dtype != torch.bfloat16 or t.is_cuda or not t.is_contiguous() or t.dim() != 4:
+            raise ValueError("q, k, v must be contiguous bf16 host tensors [B, H, S, d]")
+    B, H, S, d = q.shape
+    shape = make_shape(B, H, S, d, tile_grid)
+    if workspace is None:
+        workspace = layer_host_workspace(shape, heads_per_chunk, stream=stream)
+    if out is None:
+        pin = q.is_pinned()
+        o = torch.empty(q.shape, dtype=torch.bfloat16, pin_memory=pin)
+        lse = torch.empty((B, H, S), dtype=torch.float32, pin_memory=pin)
+    else:
+        o, lse = out
+        if o.is_cuda or lse.is_cuda or not (o.is_contiguous() and lse.is_contiguous()):
+            raise ValueError("out must be contiguous host tensors")
+    prm = _MaskParams(float(thr), 1 if sta is not None else 0,
+                      *(sta if sta is not None else (0, 0, 0)), int(topk))
+    _check(lib().nabla_layer_host(ctypes.byref(shape), ctypes.byref(prm), _ptr(q), _ptr(k),
+                                  _ptr(v), _ptr(o), _ptr(lse), int(heads_per_chunk),
+                                  _ptr(workspace.buf), _stream(stream)))
     return o, lse
 
 

@@ -290,11 +290,19 @@ nabla_status run_fwd(const nabla_shape* shape, const void* q, const void* k, con
 namespace nabla {
 // Lets other translation units of the library report through nabla_last_error().
 void set_last_error(const std::string& msg) { g_last_error = msg; }
+// nabla_build_mask with its device status bits OR-ed into `status` instead of
+// the workspace header (the host-buffer layer shares one header between the
+// chunks it runs on two streams).
+nabla_status build_mask_with_status(const nabla_shape* shape, const nabla_mask_params* params,
+                                    const void* q, const void* k, uint8_t* mask_u8,
+                                    int32_t* row_ptr, int32_t* col_idx, int64_t col_capacity,
+                                    int32_t* nnz_out, void* workspace, int* status,
+                                    nabla_stream_t stream);
 }  // namespace nabla
 
 extern "C" {
 
-int nabla_version(void) { return 210; }
+int nabla_version(void) { return 220; }
 
 const char* nabla_last_error(void) { return g_last_error.c_str(); }
 
@@ -342,6 +350,19 @@ nabla_status nabla_build_mask(const nabla_shape* shape, const nabla_mask_params*
                               int32_t* col_idx, int64_t col_capacity, int32_t* nnz_out,
                               void* workspace, nabla_stream_t stream) {
   CallRange range("nabla_build_mask");
+  return nabla::build_mask_with_status(shape, params, q, k, mask_u8, row_ptr, col_idx, col_capacity,
+                                       nnz_out, workspace, static_cast<int*>(workspace), stream);
+}
+
+}  // extern "C"
+
+namespace nabla {
+
+nabla_status build_mask_with_status(const nabla_shape* shape, const nabla_mask_params* params,
+                                    const void* q, const void* k, uint8_t* mask_u8,
+                                    int32_t* row_ptr, int32_t* col_idx, int64_t col_capacity,
+                                    int32_t* nnz_out, void* workspace, int* status,
+                                    nabla_stream_t stream) {
   nabla_status s = check_shape(shape);
   if (s != NABLA_OK) return s;
   if (params == nullptr) return fail(NABLA_ERR_INVALID_ARG, "params is NULL");
@@ -353,7 +374,7 @@ nabla_status nabla_build_mask(const nabla_shape* shape, const nabla_mask_params*
   if (shape->Tt <= 0 || shape->Th <= 0 || shape->Tw <= 0 ||
       static_cast<int64_t>(shape->Tt) * shape->Th * shape->Tw != shape->S / 64)
     return fail(NABLA_ERR_INVALID_ARG, "tile grid Tt*Th*Tw must equal S/64");
-  if (!q || !k || !row_ptr || !workspace) return fail(NABLA_ERR_INVALID_ARG, "null pointer");
+  if (!q || !k || !row_ptr || !workspace || !status) return fail(NABLA_ERR_INVALID_ARG, "null pointer");
   if (col_capacity > 0 && col_idx == nullptr) return fail(NABLA_ERR_INVALID_ARG, "col_idx is NULL");
   if (col_capacity < 0) return fail(NABLA_ERR_INVALID_ARG, "col_capacity is negative");
   if (!aligned16(q) || !aligned16(k) || (reinterpret_cast<uintptr_t>(workspace) & 255u))
@@ -379,10 +400,15 @@ nabla_status nabla_build_mask(const nabla_shape* shape, const nabla_mask_params*
                            bits, counts, mask_u8, st);
   if (e != cudaSuccess) return cuda_fail(e, "select launch");
   e = nabla::launch_scan_fill(bits, counts, nrows, nb, row_ptr, col_idx, col_capacity, nnz_out,
-                              status_ptr(workspace), st);
+                              status, st);
   if (e != cudaSuccess) return cuda_fail(e, "scan/fill launch");
   return NABLA_OK;
 }
+
+}  // namespace nabla
+
+extern "C" {
+
 
 nabla_status bsa_fwd(const nabla_shape* shape, const void* q, const void* k, const void* v,
                      const int32_t* row_ptr, const int32_t* col_idx, float scale, void* o,

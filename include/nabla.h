@@ -195,6 +195,48 @@ NABLA_API nabla_status bsa_fwd_with_mask_static(const nabla_shape* shape, const 
                                                 nabla_stream_t stream);
 
 /*
+ * One NABLA attention layer on host-resident tensors: per head, the mask of
+ * nabla_build_mask (Algorithm 1 of the NABLA paper, optional STA union) and
+ * then bsa_fwd over it, with Q, K, V read from and O, LSE written to host
+ * memory.  The result equals nabla_build_mask + bsa_fwd (scale 1/sqrt(d)) on
+ * device copies of the same tensors.
+ *
+ * Heads are independent, so the call moves them in chunks of at most
+ * heads_per_chunk heads through two device slots: while chunk c computes on
+ * `stream`, chunk c+1's inputs go host-to-device and chunk c-1's outputs go
+ * device-to-host on two streams the library owns, ordered with events.  With
+ * page-locked (pinned) host buffers the copies overlap the kernels; pageable
+ * buffers give the same result without the overlap.  The chunks ramp up
+ * (1, 2, 4, ... heads) and end on a chunk of heads_per_chunk/4 heads, so that
+ * the first input copy and the last output copy, which overlap nothing, stay
+ * short; nabla_layer_host_chunks gives the schedule.
+ *
+ *   q_host, k_host, v_host   host bf16 [B,H,S,d], tile-major tokens
+ *   o_host                   host bf16 [B,H,S,d]
+ *   lse_host                 host fp32 [B,H,S]
+ *   heads_per_chunk          heads per pipeline chunk (> 0; 4 suits S = 76800)
+ *   workspace    device, nabla_layer_host_workspace_size(shape, heads_per_chunk)
+ *                bytes, 256-byte aligned; its first 256 bytes are the status
+ *                header (nabla_workspace_init once, nabla_query_status after)
+ * Returns once the work is queued.  All of it, the last output copy
+ * included, is ordered before anything later queued on `stream`: synchronise
+ * `stream` before reading o_host or lse_host.  The library's copy streams are
+ * per device, so two calls in flight at once on one device (other host
+ * threads, or other streams without ordering) are not supported.
+ */
+NABLA_API size_t nabla_layer_host_workspace_size(const nabla_shape* shape, int heads_per_chunk);
+/* Chunk schedule of nabla_layer_host for `heads` = B*H heads: returns the
+ * number of chunks (0 on a non-positive argument) and writes the first
+ * min(count, capacity) chunk sizes, in order, to host `sizes` (may be NULL). */
+NABLA_API int64_t nabla_layer_host_chunks(int64_t heads, int heads_per_chunk, int32_t* sizes,
+                                          int64_t capacity);
+NABLA_API nabla_status nabla_layer_host(const nabla_shape* shape, const nabla_mask_params* params,
+                                        const void* q_host, const void* k_host,
+                                        const void* v_host, void* o_host, float* lse_host,
+                                        int heads_per_chunk, void* workspace,
+                                        nabla_stream_t stream);
+
+/*
  * Block mask from XAttention antidiagonal scores instead of the pooled map
  * ("XAttention: Block Sparse Attention with Antidiagonal Scoring" notes:
  * blocks scored along antidiagonals, selected by a threshold).  With stride St

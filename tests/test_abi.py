@@ -164,3 +164,46 @@ def test_layout_arguments_checked(nl):
     assert lib.nabla_block_energy(ctypes.byref(raster), a, a, a, a, a, ctypes.c_float(0), a,
                                   null, a, null) == 2
     assert lib.nabla_version() >= 210
+
+
+def test_layer_host_arguments_checked(nl):
+    lib = nl.lib()
+    null = ctypes.c_void_p(0)
+    a = ctypes.c_void_p(1 << 20)
+    s = nl.make_shape(1, 40, 76800, 128, (5, 12, 20))
+    prm = nl._MaskParams(0.2, 1, 1, 2, 2, 0)
+    one = lib.nabla_layer_host_workspace_size(ctypes.byref(s), 4)
+    # two slots of 4 heads (Q, K, V, O and LSE) beyond one chunk's mask workspace
+    assert one >= 2 * (4 * 4 * 76800 * 128 * 2 + 4 * 76800 * 4)
+    assert one > lib.nabla_layer_host_workspace_size(ctypes.byref(s), 2)
+    assert lib.nabla_layer_host_workspace_size(ctypes.byref(s), 0) == 0
+    bad = nl.make_shape(1, 40, 76800, 96, (5, 12, 20))
+    assert lib.nabla_layer_host_workspace_size(ctypes.byref(bad), 4) == 0
+    f = lib.nabla_layer_host
+    assert f(ctypes.byref(s), ctypes.byref(prm), a, a, a, a, a, 0, a, null) == 1
+    assert f(ctypes.byref(s), ctypes.byref(prm), a, null, a, a, a, 4, a, null) == 1
+    assert f(ctypes.byref(bad), ctypes.byref(prm), a, a, a, a, a, 4, a, null) == 1
+    raster = nl.make_shape(1, 40, 76800, 128, (5, 12, 20), nl.LAYOUT_RASTER)
+    assert f(ctypes.byref(raster), ctypes.byref(prm), a, a, a, a, a, 4, a, null) == 2
+    # the workspace must be 256-byte aligned
+    assert f(ctypes.byref(s), ctypes.byref(prm), a, a, a, a, a, 4,
+             ctypes.c_void_p((1 << 20) + 16), null) == 1
+    assert lib.nabla_version() >= 220
+
+
+@pytest.mark.parametrize("heads,hpc", [(40, 8), (40, 4), (40, 1), (40, 64), (1, 4), (2, 8),
+                                       (3, 2), (24, 6), (96, 16), (7, 7)])
+def test_layer_host_chunk_schedule(nl, heads, hpc):
+    sizes = nl.layer_host_chunks(heads, hpc)
+    assert sum(sizes) == heads
+    assert all(1 <= s <= hpc for s in sizes)
+    assert sizes[0] == 1
+    # ramp: each chunk at most twice the one before it until the full size
+    for a, b in zip(sizes, sizes[1:]):
+        if a < hpc // 2:
+            assert b <= 2 * a
+    assert nl.layer_host_chunks(0, hpc) == [] and nl.layer_host_chunks(heads, 0) == []
+
+
+def test_layer_host_schedule_wan(nl):
+    assert nl.layer_host_chunks(40, 8) == [1, 2, 4, 8, 8, 8, 7, 2]
