@@ -45,9 +45,10 @@
 // Online softmax with a lazy maximum: the running max m of a row is raised
 // (and O, l rescaled by 2^(m_old - m_new)) only when a tile's max exceeds it by
 // more than 2^8; otherwise p <= 256 and O / l, LSE = ln2 (m + log2 l) are
-// unchanged in exact arithmetic.  Exponentials are computed against m while
-// the tile max is formed; a rise past the threshold (or a row's first tile)
-// recomputes them from the S values still in tensor memory.
+// unchanged in exact arithmetic.  The tile max is formed from the S row in
+// registers, then the exponentials; a tile whose two key blocks the row both
+// lists (the common case) runs that as one straight-line block without
+// per-chunk branches, which lets the compiler interleave the whole row.
 //
 // Tensor memory (512 columns): tile 0 S/P [0,128), O [128,256);
 // tile 1 S/P [256,384), O [384,512).
@@ -409,17 +410,27 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       // the whole S row in one batch of loads (one load latency per tile)
       uint32_t sv[4][32];
-      if (v0) { tmem_ld32(s_base, sv[0]); tmem_ld32(s_base + 32, sv[1]); }
-      if (v1) { tmem_ld32(s_base + 64, sv[2]); tmem_ld32(s_base + 96, sv[3]); }
-      tmem_ld_wait();
       float mx[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) mx[i] = -INFINITY;
+      if (v0 && v1) {   // both entries listed: loads and max without per-chunk branches
 #pragma unroll
-      for (int ch = 0; ch < 4; ++ch) {
-        if ((ch < 2) ? v0 : v1) {
+        for (int ch = 0; ch < 4; ++ch) tmem_ld32(s_base + 32 * ch, sv[ch]);
+        tmem_ld_wait();
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch)
 #pragma unroll
           for (int i = 0; i < 32; ++i) mx[i & 7] = fmaxf(mx[i & 7], __uint_as_float(sv[ch][i]));
+      } else {
+        if (v0) { tmem_ld32(s_base, sv[0]); tmem_ld32(s_base + 32, sv[1]); }
+        if (v1) { tmem_ld32(s_base + 64, sv[2]); tmem_ld32(s_base + 96, sv[3]); }
+        tmem_ld_wait();
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch) {
+          if ((ch < 2) ? v0 : v1) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) mx[i & 7] = fmaxf(mx[i & 7], __uint_as_float(sv[ch][i]));
+          }
         }
       }
       const float m_tile = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
@@ -455,6 +466,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool live = m > -INFINITY;
       const float mneg = live ? -m : 0.f;
       float rs[4] = {0.f, 0.f, 0.f, 0.f};
+      if (v0 && v1 && __all_sync(0xffffffffu, live)) {
+        // common case, one straight-line block: every column of the row is listed
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float p0 = fast_exp2(fmaf(__uint_as_float(sv[ch][2 * i]), sl2, mneg));
+            const float p1 = fast_exp2(fmaf(__uint_as_float(sv[ch][2 * i + 1]), sl2, mneg));
+            rs[i & 3] += p0 + p1;
+            pk[i] = pack_bf16x2(p0, p1);
+          }
+          tmem_st16(s_base + ch * 16, pk);
+        }
+      } else
 #pragma unroll
       for (int ch = 0; ch < 4; ++ch) {
         uint32_t pk[16];
