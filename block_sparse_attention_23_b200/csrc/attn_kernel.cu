@@ -9,33 +9,35 @@
 // are computed).
 //
 // Work decomposition
-//   One CTA per (b, h, group of four query blocks 4g..4g+3) = two query
-//   tiles of 128 rows: tile 0 = blocks 4g, 4g+1; tile 1 = blocks 4g+2, 4g+3.
-//   The key blocks visited are the union of the four CSR rows, each entry with
-//   a 4-bit membership mask.  Key tiles are 128 keys = two union entries (the
-//   second may be a repeat that every row masks); each entry is one contiguous
-//   64 x d slab of the [B,H,S,d] tensor, loaded as a plain 2D TMA box, so both
-//   query tiles share every K/V tile that is loaded.  A query tile computes a
-//   key tile only if one of its two blocks lists one of the tile's entries; a
-//   row whose block did not list an entry gives it probability 0 (no
-//   exponentials evaluated).
+//   One CTA per (b, h, pair of query blocks 2g, 2g+1) = one query tile of 128
+//   rows.  The key blocks visited are the union of the two CSR rows, each entry
+//   with a 2-bit membership mask, taken four at a time: a key tile is 256 keys
+//   (the last one repeats its final entry, masked for every row).  Each entry
+//   is one contiguous 64 x d slab of the [B,H,S,d] tensor, loaded as a plain 2D
+//   TMA box.  A row whose block did not list an entry gives it probability 0
+//   (no exponentials evaluated).
 //
 // Roles (384 threads)
-//   warps 0-3   softmax of query tile 0, warps 4-7 of query tile 1: thread i of
-//               the group owns row i (= tensor-memory lane i) for all 128 keys
-//               of a tile: tcgen05.ld of S, lazy running max, exp2, P (bf16)
-//               written over the first 64 S columns, O rescale, epilogue.
+//   warps 0-7   softmax: warp w owns tensor-memory lane quarter q = w % 4 (rows
+//               32q..32q+31 of the tile) and column half c = w / 4 (keys
+//               [128c, 128c+128) of each key tile, its entries 2c and 2c+1).
+//               The two warps of a lane quarter trade partial row maxima (and,
+//               at the end, partial row sums) through shared memory, meeting on
+//               an mbarrier with a bounded wait.
 //   warp 8      TMA producer of Q and K (and the union-list compaction).
 //   warp 9      tensor-memory allocation and the single MMA-issuing thread.
 //   warp 10     TMA producer of V; warp 11 idles (completes warpgroup 2).
 //
-// MMA order (ping-pong between the two query tiles)
-//   S_0(0), S_1(0), then for every key tile t: PV_0(t), S_0(t+1), PV_1(t),
-//   S_1(t+1).  While softmax 0 works on S_0(t) the tensor cores run PV_1(t-1)
-//   and S_1(t), and the other way round, so each softmax group has about two
-//   MMA tile-products of time.  S_x(t+1) overwrites the S/P buffer of tile x
-//   only after PV_x(t), which read P_x(t), was issued by the same thread (MMAs
-//   of one thread execute in issue order).
+// Tensor memory (512 columns): S [0,256) fp32, P [256,384) (bf16 pairs), O
+// [384, 384+d).  P has its own columns, so the tensor cores do not wait for a
+// softmax to finish before computing the next S:
+//   S(0); then for every key tile t: S(t+1) as soon as the softmax has copied
+//   S(t) to registers (and K(t+1) is in), PV(t) once P(t) is written.
+// While the softmax works on tile t the tensor cores run S(t+1) and PV(t-1);
+// the softmax stores P(t) only after PV(t-1), which read P(t-1), completed,
+// and keeps P(t) in registers until then.  S at N = 256 runs at the full
+// tensor rate (an N = 128 product with both operands in shared memory does
+// not), and the per-tile softmax overhead is spread over 256 keys.
 //
 // Token order: tile-major tensors are read as 2D boxes; raster-ordered ones
 // (token (t,h,w) at (t*H + h)*W + w) as 5D boxes that gather one 4x4x4 tile,
@@ -46,12 +48,9 @@
 // (and O, l rescaled by 2^(m_old - m_new)) only when a tile's max exceeds it by
 // more than 2^8; otherwise p <= 256 and O / l, LSE = ln2 (m + log2 l) are
 // unchanged in exact arithmetic.  The tile max is formed from the S row in
-// registers, then the exponentials; a tile whose two key blocks the row both
+// registers, then the exponentials; a warp whose two entries the row both
 // lists (the common case) runs that as one straight-line block without
 // per-chunk branches, which lets the compiler interleave the whole row.
-//
-// Tensor memory (512 columns): tile 0 S/P [0,128), O [128,256);
-// tile 1 S/P [256,384), O [384,512).
 //
 // Every mbarrier wait is time-bounded; a wait that runs out records
 // kStatusTimeout, raises a CTA-wide abort flag, and the CTA drains its own TMA
@@ -66,37 +65,34 @@
 namespace nabla {
 
 constexpr int kBM = 128;        // rows per query tile (two 64-token blocks)
-constexpr int kQTiles = 2;      // query tiles per CTA
-constexpr int kBN = 128;        // keys per tile (two 64-token blocks)
-constexpr int kKStages = 2;     // K ring depth
-constexpr int kVStages = 2;     // V ring depth
+constexpr int kBN = 256;        // keys per tile (four 64-token blocks)
+constexpr int kEntries = 4;     // union entries per key tile
 constexpr int kSoftmaxThreads = 256;
 constexpr int kThreads = kSoftmaxThreads + 128;   // warpgroups 0, 1 softmax; 2 load/MMA
 constexpr int kProducerWarp = 8, kMmaWarp = 9, kVProducerWarp = 10;   // warp 11 idles
-// Register budgets after set-up: a softmax thread holds a whole S row (128
-// values); the load/MMA warpgroup needs few.  8*216 + 4*72 = 12*168, the
-// launch allocation (checked on the host before launch).
+// Register budgets after set-up: a softmax thread holds 128 S values of its
+// row and the packed P; the load/MMA warpgroup needs few.  8*216 + 4*72 =
+// 12*168, the launch allocation (checked on the host before launch).
 constexpr int kRegsSoftmax = 216, kRegsOther = 72, kRegsLaunch = 168;
 constexpr int kMaxNb = 4096;    // blocks per head supported
 constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColS = 0, kColP = 256, kColO = 384;
 constexpr float kRescaleThreshold = 8.0f;            // log2 units
 constexpr uint64_t kDrainLimitNs = 1000000000ull;   // 1 s for draining in-flight work
-
-__host__ __device__ constexpr uint32_t col_s(int x) { return x ? 256u : 0u; }
-__host__ __device__ constexpr uint32_t col_o(int x) { return x ? 384u : 128u; }
 
 template <int D>
 struct AttnSmem {
   static constexpr int kDH = D / 64;                       // 64-column halves of d
-  static constexpr uint32_t kQBytes = kBM * D * 2;         // one query tile
-  static constexpr uint32_t kKVBytes = kBN * D * 2;        // one K or V stage
+  static constexpr uint32_t kQBytes = kBM * D * 2;         // the query tile
+  static constexpr uint32_t kKVBytes = kBN * D * 2;        // one K or V tile
   static constexpr uint32_t kOffQ = 0;
-  static constexpr uint32_t kOffK = kOffQ + kQTiles * kQBytes;
-  static constexpr uint32_t kOffV = kOffK + kKStages * kKVBytes;
-  static constexpr uint32_t kOffBar = kOffV + kVStages * kKVBytes;  // 32 mbarriers
-  static constexpr uint32_t kOffMisc = kOffBar + 256;      // tmem base, abort, n_u
-  static constexpr uint32_t kOffBitmap = kOffMisc + 64;    // 4 x kMaxNb/32 words
-  static constexpr uint32_t kOffList = kOffBitmap + 4 * (kMaxNb / 32) * 4;
+  static constexpr uint32_t kOffK = kOffQ + kQBytes;
+  static constexpr uint32_t kOffV = kOffK + kKVBytes;
+  static constexpr uint32_t kOffBar = kOffV + kKVBytes;    // 16 mbarriers
+  static constexpr uint32_t kOffMisc = kOffBar + 128;      // tmem base, abort, n_u
+  static constexpr uint32_t kOffXch = kOffMisc + 64;       // [2 parities][2 halves][128 rows] fp32
+  static constexpr uint32_t kOffBitmap = kOffXch + 2 * 2 * kBM * 4;   // 2 x kMaxNb/32 words
+  static constexpr uint32_t kOffList = kOffBitmap + 2 * (kMaxNb / 32) * 4;
   static constexpr uint32_t kBytes = kOffList + kMaxNb * 4;
   static constexpr uint32_t kAlloc = kBytes + 1024;        // slack for 1024-byte alignment
 };
@@ -104,15 +100,17 @@ struct AttnSmem {
 // Barrier slots inside the barrier area.
 enum : int {
   kBarQFull = 0,
-  kBarKFull = 1,                      // + stage
-  kBarKEmpty = kBarKFull + kKStages,
-  kBarVFull = kBarKEmpty + kKStages,
-  kBarVEmpty = kBarVFull + kVStages,
-  kBarSFull = kBarVEmpty + kVStages,  // + query tile: S ready
-  kBarPFull = kBarSFull + kQTiles,    // + query tile: P written
-  kBarOFull = kBarPFull + kQTiles,    // + query tile: PV done
-  kBarDrain = kBarOFull + kQTiles,
-  kNumBars = kBarDrain + 1
+  kBarKFull,     // K(t) landed
+  kBarKEmpty,    // S(t) done: the K buffer is free
+  kBarVFull,     // V(t) landed
+  kBarVEmpty,    // PV(t) done: the V buffer is free
+  kBarSFull,     // S(t) in tensor memory
+  kBarSFree,     // every softmax thread copied S(t) to registers
+  kBarPFull,     // every softmax thread wrote P(t) (and rescaled its O half)
+  kBarOFull,     // PV(t) done
+  kBarDrain,
+  kBarPair,      // + lane quarter: the two warps of a quarter met (4 slots)
+  kNumBars = kBarPair + 4
 };
 
 struct AttnParams {
@@ -164,9 +162,6 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, uint64_
   return __all_sync(0xffffffffu, mbar_wait(bar, parity, limit_ns, abort));
 }
 
-// Membership mask of query tile x (bits of its two blocks) in union entry e.
-__device__ __forceinline__ int tile_bits(int e, int x) { return (e >> (16 + 2 * x)) & 3; }
-
 template <int D, bool kRaster>
 __global__ void __launch_bounds__(kThreads, 1)
     bsa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -185,7 +180,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile uint32_t* tmem_holder = misc;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
   volatile int* n_union_s = reinterpret_cast<volatile int*>(misc + 2);
-  uint32_t* bm = reinterpret_cast<uint32_t*>(gbase + L::kOffBitmap);   // [4][kMaxNb/32]
+  float* xch = reinterpret_cast<float*>(gbase + L::kOffXch);           // [2][2][kBM]
+  uint32_t* bm = reinterpret_cast<uint32_t*>(gbase + L::kOffBitmap);   // [2][kMaxNb/32]
   int32_t* ulist = reinterpret_cast<int32_t*>(gbase + L::kOffList);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -193,27 +189,23 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int bh = item / prm.ngroups;
   const int grp = item % prm.ngroups;
   const int nb = prm.nb;
-  const int r0 = 4 * grp;                       // first query block of the group
-  const int nq = min(4, nb - r0);               // query blocks present (1..4)
+  const int r0 = 2 * grp;                       // first query block of the tile
+  const int nq = min(2, nb - r0);               // query blocks present (1 or 2)
   auto bar = [&](int i) { return bar0 + 8u * static_cast<uint32_t>(i); };
 
   // ---------------------------------------------------------------- setup
   if (tid == 0) {
     mbar_init(bar(kBarQFull), 1);
-    for (int s = 0; s < kKStages; ++s) {
-      mbar_init(bar(kBarKFull + s), 1);
-      mbar_init(bar(kBarKEmpty + s), 1);
-    }
-    for (int s = 0; s < kVStages; ++s) {
-      mbar_init(bar(kBarVFull + s), 1);
-      mbar_init(bar(kBarVEmpty + s), 1);
-    }
-    for (int x = 0; x < kQTiles; ++x) {
-      mbar_init(bar(kBarSFull + x), 1);
-      mbar_init(bar(kBarPFull + x), kSoftmaxThreads / kQTiles);
-      mbar_init(bar(kBarOFull + x), 1);
-    }
+    mbar_init(bar(kBarKFull), 1);
+    mbar_init(bar(kBarKEmpty), 1);
+    mbar_init(bar(kBarVFull), 1);
+    mbar_init(bar(kBarVEmpty), 1);
+    mbar_init(bar(kBarSFull), 1);
+    mbar_init(bar(kBarSFree), kSoftmaxThreads);
+    mbar_init(bar(kBarPFull), kSoftmaxThreads);
+    mbar_init(bar(kBarOFull), 1);
     mbar_init(bar(kBarDrain), 1);
+    for (int q = 0; q < 4; ++q) mbar_init(bar(kBarPair + q), 64);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -227,7 +219,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_prefetch_desc(&tmV);
   }
   const int nw = (nb + 31) >> 5;
-  for (int i = tid; i < 4 * (kMaxNb / 32); i += kThreads) bm[i] = 0u;
+  for (int i = tid; i < 2 * (kMaxNb / 32); i += kThreads) bm[i] = 0u;
   __syncthreads();
   for (int qb = 0; qb < nq; ++qb) {
     const int64_t g = static_cast<int64_t>(bh) * nb + r0 + qb;
@@ -244,10 +236,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     int run = 0;
     for (int w0 = 0; w0 < nw; w0 += 32) {
       const int w = w0 + lane;
-      uint32_t u[4];
-#pragma unroll
-      for (int qb = 0; qb < 4; ++qb) u[qb] = w < nw ? bm[qb * (kMaxNb / 32) + w] : 0u;
-      uint32_t any = u[0] | u[1] | u[2] | u[3];
+      const uint32_t u0 = w < nw ? bm[w] : 0u;
+      const uint32_t u1 = w < nw ? bm[(kMaxNb / 32) + w] : 0u;
+      uint32_t any = u0 | u1;
       const int cnt = __popc(any);
       int incl = cnt;
 #pragma unroll
@@ -259,9 +250,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       while (any) {
         const int b = __ffs(any) - 1;
         any &= any - 1;
-        int mem = 0;
-#pragma unroll
-        for (int qb = 0; qb < 4; ++qb) mem |= static_cast<int>((u[qb] >> b) & 1u) << qb;
+        const int mem = static_cast<int>((u0 >> b) & 1u) | (static_cast<int>((u1 >> b) & 1u) << 1);
         ulist[pos++] = (w * 32 + b) | (mem << 16);
       }
       run += __shfl_sync(0xffffffffu, incl, 31);
@@ -273,110 +262,103 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
   const int n_u = *n_union_s;
-  const int n_t = (n_u + 1) >> 1;
+  const int n_t = (n_u + kEntries - 1) / kEntries;
   const uint64_t lim = prm.wait_limit_ns;
-  // membership of key tile t: OR of its two entries
-  auto tile_entry = [&](int t, int i) { return (2 * t + i < n_u) ? ulist[2 * t + i] : 0; };
-  auto tile_active = [&](int t, int x) {
-    return tile_bits(tile_entry(t, 0) | tile_entry(t, 1), x) != 0;
+  // entry e of key tile t (0 past the end of the union: no row lists it)
+  auto tile_entry = [&](int t, int e) {
+    return (kEntries * t + e < n_u) ? ulist[kEntries * t + e] : 0;
   };
 
   if (warp >= 8) {
   setmaxnreg_dec<kRegsOther>();
   if (warp == kProducerWarp || warp == kVProducerWarp) {
     // ------------------------------------------------------------ TMA producers
-    // warp 8 streams Q and K, warp 10 streams V: a V slot frees only after the
-    // softmax of its tile, and must not hold back the K prefetch
+    // warp 8 streams Q and K, warp 10 streams V (one buffer each: K(t+1) may
+    // land once S(t) is done, V(t+1) once PV(t) is done)
     if (lane == 0 && n_t > 0) {
       const bool is_k = warp == kProducerWarp;
-      const int nst = is_k ? kKStages : kVStages;
-      const uint32_t ring = is_k ? sK : sV;
+      const uint32_t buf = is_k ? sK : sV;
       const CUtensorMap* map = is_k ? &tmK : &tmV;
-      const int full0 = is_k ? kBarKFull : kBarVFull, empty0 = is_k ? kBarKEmpty : kBarVEmpty;
-      int armed0 = 0, armed1 = 0;
+      const int full = is_k ? kBarKFull : kBarVFull, empty = is_k ? kBarKEmpty : kBarVEmpty;
+      int armed = 0;
       if (is_k) {
-        mbar_arrive_expect_tx(bar(kBarQFull), kQTiles * L::kQBytes);
-        for (int qb = 0; qb < 4; ++qb)   // blocks past the end repeat the last (rows unused)
+        mbar_arrive_expect_tx(bar(kBarQFull), L::kQBytes);
+        for (int qb = 0; qb < 2; ++qb)   // a block past the end repeats the last (rows unused)
           for (int h = 0; h < L::kDH; ++h)
-            load_block<kRaster>(sQ + (qb >> 1) * L::kQBytes + h * kBM * 128 + (qb & 1) * 64 * 128,
-                                &tmQ, bar(kBarQFull), h, bh, min(r0 + qb, nb - 1), prm.S, prm.Th,
-                                prm.Tw);
+            load_block<kRaster>(sQ + h * kBM * 128 + qb * 64 * 128, &tmQ, bar(kBarQFull), h, bh,
+                                min(r0 + qb, nb - 1), prm.S, prm.Th, prm.Tw);
       }
+      const int last = ulist[n_u - 1] & 0xFFFF;
       for (int t = 0; t < n_t; ++t) {
-        const int s = t % nst, n = t / nst;
-        const int j0 = ulist[2 * t] & 0xFFFF;
-        const int j1 = (2 * t + 1 < n_u) ? (ulist[2 * t + 1] & 0xFFFF) : j0;
-        if (t >= nst && !mbar_wait(bar(empty0 + s), (n - 1) & 1, lim, abort_flag)) {
+        if (t > 0 && !mbar_wait(bar(empty), (t - 1) & 1, lim, abort_flag)) {
           record_abort(abort_flag, prm.status, kStatusTimeout);
           break;
         }
-        mbar_arrive_expect_tx(bar(full0 + s), L::kKVBytes);
-        (s ? armed1 : armed0) += 1;
-        for (int kb = 0; kb < 2; ++kb)
+        mbar_arrive_expect_tx(bar(full), L::kKVBytes);
+        ++armed;
+        for (int e = 0; e < kEntries; ++e) {
+          const int j = (kEntries * t + e < n_u) ? (ulist[kEntries * t + e] & 0xFFFF) : last;
           for (int h = 0; h < L::kDH; ++h)
-            load_block<kRaster>(ring + s * L::kKVBytes + h * kBN * 128 + kb * 64 * 128, map,
-                                bar(full0 + s), h, bh, kb ? j1 : j0, prm.S, prm.Th, prm.Tw);
+            load_block<kRaster>(buf + h * kBN * 128 + e * 64 * 128, map, bar(full), h, bh, j,
+                                prm.S, prm.Th, prm.Tw);
+        }
       }
       // drain: every armed phase must complete before shared memory is released
       if (is_k) mbar_wait(bar(kBarQFull), 0, kDrainLimitNs, nullptr);
-      if (armed0) mbar_wait(bar(full0 + 0), (armed0 - 1) & 1, kDrainLimitNs, nullptr);
-      if (armed1) mbar_wait(bar(full0 + 1), (armed1 - 1) & 1, kDrainLimitNs, nullptr);
+      if (armed) mbar_wait(bar(full), (armed - 1) & 1, kDrainLimitNs, nullptr);
     }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0 && n_t > 0) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(kBM, kBN, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(kBM, D, true);
-      int n_pv[kQTiles] = {0, 0};   // PV products issued per query tile
-      bool ok = mbar_wait(bar(kBarQFull), 0, lim, abort_flag);
-      tc_fence_after();
-      auto issue_s = [&](int x, int t) {
-        const uint32_t kt = sK + (t % kKStages) * L::kKVBytes;
-        const uint32_t qt = sQ + x * L::kQBytes;
+      // S = Q K^T over the 256 keys of the tile in K buffer, 16-deep steps of d
+      auto issue_s = [&]() {
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * (kBM * 128) + (kk & 3) * 32;
+          const uint32_t offq = (kk >> 2) * (kBM * 128) + (kk & 3) * 32;
           const uint32_t offk = (kk >> 2) * (kBN * 128) + (kk & 3) * 32;
-          tc_mma_ss(tmem + col_s(x), sdesc_sw128(qt + off, 16, 1024),
-                    sdesc_sw128(kt + offk, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
+          tc_mma_ss(tmem + kColS, sdesc_sw128(sQ + offq, 16, 1024), sdesc_sw128(sK + offk, 16, 1024),
+                    idesc_qk, kk > 0 ? 1u : 0u);
         }
-        tc_commit(bar(kBarSFull + x));
+        tc_commit(bar(kBarSFull));
+        tc_commit(bar(kBarKEmpty));
       };
-      auto issue_pv = [&](int x, int t) -> bool {
-        if (!mbar_wait(bar(kBarPFull + x), n_pv[x] & 1, lim, abort_flag)) return false;
-        tc_fence_after();
-        const uint32_t vt = sV + (t % kVStages) * L::kKVBytes;
+      // O += P V: 16 keys per step, P columns [8kk, 8kk+8) of the P buffer, V
+      // rows [16kk, 16kk+16); the 64-column halves of d are kBN*128 bytes apart
+      auto issue_pv = [&](int t) {
 #pragma unroll
         for (int kk = 0; kk < kBN / 16; ++kk)
-          // 16 keys per step: P columns [8kk, 8kk+8) of the S/P buffer, V rows
-          // [16kk, 16kk+16); the 64-column halves of d are kBN*128 bytes apart
-          tc_mma_ts(tmem + col_o(x), tmem + col_s(x) + kk * 8,
-                    sdesc_sw128(vt + kk * 16 * 128, kBN * 128, 1024), idesc_pv,
-                    (n_pv[x] > 0 || kk > 0) ? 1u : 0u);
-        tc_commit(bar(kBarOFull + x));
-        ++n_pv[x];
-        return true;
+          tc_mma_ts(tmem + kColO, tmem + kColP + kk * 8,
+                    sdesc_sw128(sV + kk * 16 * 128, kBN * 128, 1024), idesc_pv,
+                    (t > 0 || kk > 0) ? 1u : 0u);
+        tc_commit(bar(kBarOFull));
+        tc_commit(bar(kBarVEmpty));
       };
-      if (ok) ok = mbar_wait(bar(kBarKFull + 0), 0, lim, abort_flag);
+      bool ok = mbar_wait(bar(kBarQFull), 0, lim, abort_flag) &&
+                mbar_wait(bar(kBarKFull), 0, lim, abort_flag);
       if (ok) {
         tc_fence_after();
-        for (int x = 0; x < kQTiles; ++x)
-          if (tile_active(0, x)) issue_s(x, 0);
-        tc_commit(bar(kBarKEmpty + 0));
+        issue_s();
       }
       for (int t = 0; ok && t < n_t; ++t) {
-        const bool more = t + 1 < n_t;
-        if (!mbar_wait(bar(kBarVFull + t % kVStages), (t / kVStages) & 1, lim, abort_flag)) { ok = false; break; }
-        if (more && !mbar_wait(bar(kBarKFull + (t + 1) % kKStages), ((t + 1) / kKStages) & 1, lim,
-                               abort_flag)) { ok = false; break; }
-        tc_fence_after();
-        for (int x = 0; x < kQTiles; ++x) {
-          if (tile_active(t, x) && !issue_pv(x, t)) { ok = false; break; }
-          if (more && tile_active(t + 1, x)) issue_s(x, t + 1);
+        if (t + 1 < n_t) {
+          // S(t+1) overwrites S(t): every softmax thread must hold S(t) in registers
+          if (!mbar_wait(bar(kBarSFree), t & 1, lim, abort_flag) ||
+              !mbar_wait(bar(kBarKFull), (t + 1) & 1, lim, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          issue_s();
         }
-        if (!ok) break;
-        if (more) tc_commit(bar(kBarKEmpty + (t + 1) % kKStages));
-        tc_commit(bar(kBarVEmpty + t % kVStages));
+        if (!mbar_wait(bar(kBarPFull), t & 1, lim, abort_flag) ||
+            !mbar_wait(bar(kBarVFull), t & 1, lim, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        issue_pv(t);
       }
       if (!ok) record_abort(abort_flag, prm.status, kStatusTimeout);
       // drain: all MMAs this thread issued must finish before tensor memory is freed
@@ -387,28 +369,28 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     setmaxnreg_inc<kRegsSoftmax>();
     // ------------------------------------------------------------ softmax (warps 0-7)
-    const int x = warp >> 2;                   // query tile of this warp group
     const int quarter = warp & 3;
-    const int row = quarter * 32 + lane;       // row of the tile == tensor-memory lane
-    const int qh = row >> 6;                   // block 4g + 2x + qh
-    const int qblock = r0 + 2 * x + qh;
+    const int half = warp >> 2;                  // column half of the key tile
+    const int row = quarter * 32 + lane;         // row of the tile == tensor-memory lane
+    const int qh = row >> 6;                     // block r0 + qh
+    const int qblock = r0 + qh;
     const bool row_valid = qblock < nb;
-    const int bit = 1 << (16 + 2 * x + qh);
+    const int bit = 1 << (16 + qh);
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-    const uint32_t s_base = tmem + lane_off + col_s(x);
-    const uint32_t o_base = tmem + lane_off + col_o(x);
+    const uint32_t s_base = tmem + lane_off + kColS + 128u * half;
+    const uint32_t p_base = tmem + lane_off + kColP + 64u * half;
+    const uint32_t o_base = tmem + lane_off + kColO + static_cast<uint32_t>(D / 2) * half;
+    const uint32_t pair_bar = bar(kBarPair + quarter);
     const float sl2 = prm.scale_log2;
-    float m = -INFINITY;        // lazy running max of the row, log2 units
-    float l = 0.f;              // running sum of the row
-    int c = 0;                  // key tiles this query tile has processed
+    float m = -INFINITY;        // lazy running max of the row, log2 units (same in both warps)
+    float l = 0.f;              // running sum over this warp's columns of the row
     bool ok = true;
     for (int t = 0; t < n_t; ++t) {
-      if (!tile_active(t, x)) continue;        // same decision as the MMA issuer
-      const bool v0 = (tile_entry(t, 0) & bit) != 0;   // uniform per warp
-      const bool v1 = (tile_entry(t, 1) & bit) != 0;
-      if (!warp_wait(bar(kBarSFull + x), c & 1, lim, abort_flag)) { ok = false; break; }
+      const bool v0 = (tile_entry(t, 2 * half) & bit) != 0;       // uniform per warp
+      const bool v1 = (tile_entry(t, 2 * half + 1) & bit) != 0;
+      if (!warp_wait(bar(kBarSFull), t & 1, lim, abort_flag)) { ok = false; break; }
       tc_fence_after();
-      // the whole S row in one batch of loads (one load latency per tile)
+      // this warp's 128 S columns of the row in one batch of loads
       uint32_t sv[4][32];
       float mx[8];
 #pragma unroll
@@ -433,25 +415,39 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      const float m_tile = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+      // S(t) is in registers: the tensor cores may overwrite it with S(t+1)
+      tc_fence_before();
+      mbar_arrive(bar(kBarSFree));
+      const float m_part = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
                                  fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * sl2;
+      // the row's max over all 256 keys: trade partial maxima with the other
+      // warp of this lane quarter (slots alternate with the tile's parity)
+      xch[((t & 1) * 2 + half) * kBM + row] = m_part;
+      mbar_arrive(pair_bar);
+      if (!warp_wait(pair_bar, t & 1, lim, abort_flag)) { ok = false; break; }
+      const float m_tile = fmaxf(m_part, xch[((t & 1) * 2 + (half ^ 1)) * kBM + row]);
       const bool has = m_tile > -INFINITY;
       const bool first = m == -INFINITY;
       const bool need = has && !first && (m_tile > m + kRescaleThreshold);   // rescale O, l
       const float m_old = m;
       if (has && (first || need)) m = m_tile;
-      // O must hold the previous PV of this tile before it is rescaled by 2^(m_old - m)
+      // O must hold PV(t-1) before it is rescaled by 2^(m_old - m); rare after
+      // the first tiles, so the wait is paid only then
       bool rescale = __any_sync(0xffffffffu, need);
-      if (rescale && c > 0 && !warp_wait(bar(kBarOFull + x), (c - 1) & 1, lim, abort_flag)) {
-        ok = false;
-        rescale = false;
+      bool pv_done = t == 0;                     // PV(t-1) completed (known so far)
+      if (rescale && !pv_done) {
+        if (!warp_wait(bar(kBarOFull), (t - 1) & 1, lim, abort_flag)) {
+          ok = false;
+          rescale = false;
+        }
+        pv_done = true;
       }
       if (rescale) {
         tc_fence_after();
         const float alpha = need ? fast_exp2(m_old - m) : 1.f;
         l *= alpha;
 #pragma unroll 1
-        for (int cc = 0; cc < D / 16; ++cc) {
+        for (int cc = 0; cc < D / 32; ++cc) {
           uint32_t o[16];
           tmem_ld16(o_base + cc * 16, o);
           tmem_ld_wait();
@@ -461,65 +457,79 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_st_wait();
         }
       }
-      // p = 2^(s*scale*log2e - m); P chunk ch (keys [32ch, 32ch+32)) goes to
-      // columns [16ch, 16ch+16), whose S values are already in registers
+      // p = 2^(s*scale*log2e - m), packed to bf16 pairs and kept in registers
+      // until PV(t-1) has read the P buffer
       const bool live = m > -INFINITY;
       const float mneg = live ? -m : 0.f;
       float rs[4] = {0.f, 0.f, 0.f, 0.f};
+      uint32_t pk[4][16];
       if (v0 && v1 && __all_sync(0xffffffffu, live)) {
         // common case, one straight-line block: every column of the row is listed
 #pragma unroll
         for (int ch = 0; ch < 4; ++ch) {
-          uint32_t pk[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
             const float p0 = fast_exp2(fmaf(__uint_as_float(sv[ch][2 * i]), sl2, mneg));
             const float p1 = fast_exp2(fmaf(__uint_as_float(sv[ch][2 * i + 1]), sl2, mneg));
             rs[i & 3] += p0 + p1;
-            pk[i] = pack_bf16x2(p0, p1);
+            pk[ch][i] = pack_bf16x2(p0, p1);
           }
-          tmem_st16(s_base + ch * 16, pk);
         }
-      } else
+      } else {
 #pragma unroll
-      for (int ch = 0; ch < 4; ++ch) {
-        uint32_t pk[16];
-        if (((ch < 2) ? v0 : v1) && live) {
+        for (int ch = 0; ch < 4; ++ch) {
+          if (((ch < 2) ? v0 : v1) && live) {
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const float p0 = fast_exp2(fmaf(__uint_as_float(sv[ch][2 * i]), sl2, mneg));
-            const float p1 = fast_exp2(fmaf(__uint_as_float(sv[ch][2 * i + 1]), sl2, mneg));
-            rs[i & 3] += p0 + p1;
-            pk[i] = pack_bf16x2(p0, p1);
+            for (int i = 0; i < 16; ++i) {
+              const float p0 = fast_exp2(fmaf(__uint_as_float(sv[ch][2 * i]), sl2, mneg));
+              const float p1 = fast_exp2(fmaf(__uint_as_float(sv[ch][2 * i + 1]), sl2, mneg));
+              rs[i & 3] += p0 + p1;
+              pk[ch][i] = pack_bf16x2(p0, p1);
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) pk[ch][i] = 0u;
           }
-        } else {
-#pragma unroll
-          for (int i = 0; i < 16; ++i) pk[i] = 0u;
         }
-        tmem_st16(s_base + ch * 16, pk);
       }
       l += (rs[0] + rs[1]) + (rs[2] + rs[3]);
-      tmem_st_wait();
       if (!ok) break;
+      if (!pv_done && !warp_wait(bar(kBarOFull), (t - 1) & 1, lim, abort_flag)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+#pragma unroll
+      for (int ch = 0; ch < 4; ++ch) tmem_st16(p_base + ch * 16, pk[ch]);
+      tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(bar(kBarPFull + x));
-      ++c;
+      mbar_arrive(bar(kBarPFull));
     }
     if (!ok) record_abort(abort_flag, prm.status, kStatusTimeout);
     // ------------------------------------------------------------ epilogue
     bool have_o = false;
-    if (ok && c > 0) {
-      have_o = warp_wait(bar(kBarOFull + x), (c - 1) & 1, lim, abort_flag);
+    if (ok && n_t > 0) {
+      have_o = warp_wait(bar(kBarOFull), (n_t - 1) & 1, lim, abort_flag);
       if (!have_o) record_abort(abort_flag, prm.status, kStatusTimeout);
       tc_fence_after();
     }
-    const bool write = row_valid && ok && (c == 0 || have_o);
+    // the row sum over all keys: trade partial sums with the other warp
+    bool have_l = ok;
+    float l_row = l;
+    if (ok) {
+      xch[((n_t & 1) * 2 + half) * kBM + row] = l;
+      mbar_arrive(pair_bar);
+      have_l = warp_wait(pair_bar, n_t & 1, lim, abort_flag);
+      if (!have_l) record_abort(abort_flag, prm.status, kStatusTimeout);
+      else l_row = l + xch[((n_t & 1) * 2 + (half ^ 1)) * kBM + row];
+    }
+    const bool write = row_valid && have_l && (n_t == 0 || have_o);
     const int64_t grow = static_cast<int64_t>(bh) * prm.S +
                          (row_valid ? token_of<kRaster>(qblock, row & 63, prm.Th, prm.Tw) : 0);
-    const float inv_l = l > 0.f ? 1.f / l : 0.f;
-    __nv_bfloat16* orow = prm.o + grow * D;
+    const float inv_l = l_row > 0.f ? 1.f / l_row : 0.f;
+    __nv_bfloat16* orow = prm.o + grow * D + (D / 2) * half;
 #pragma unroll
-    for (int cc = 0; cc < D / 32; ++cc) {
+    for (int cc = 0; cc < D / 64; ++cc) {
       uint32_t o[32];
       if (have_o) {
         tmem_ld32(o_base + cc * 32, o);
@@ -538,8 +548,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
       }
     }
-    if (write && prm.lse != nullptr)
-      prm.lse[grow] = l > 0.f ? (m + __log2f(l)) * 0.69314718055994530942f : -INFINITY;
+    if (write && half == 0 && prm.lse != nullptr)
+      prm.lse[grow] = l_row > 0.f ? (m + __log2f(l_row)) * 0.69314718055994530942f : -INFINITY;
   }
 
   tc_fence_before();
@@ -683,7 +693,7 @@ cudaError_t launch_bsa_fwd(const CUtensorMap& q, const CUtensorMap& k, const CUt
   prm.H = H;
   prm.S = S;
   prm.nb = S / 64;
-  prm.ngroups = (prm.nb + 3) / 4;
+  prm.ngroups = (prm.nb + 1) / 2;
   prm.Th = Th;
   prm.Tw = Tw;
   prm.scale_log2 = scale * 1.4426950408889634f;
