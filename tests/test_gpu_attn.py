@@ -157,3 +157,38 @@ def test_bad_csr_index_reported(nl, oracle_mod, synth_mod):
     ro, rl = oracle_mod.masked_attention(q, k, v, mask, rows)
     go, gl = _gather(o, lse, rows, S)
     compare_attention(go, gl, ro, rl)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_union_shapes_of_query_pairs(nl, oracle_mod, synth_mod, d):
+    """Pairs of query blocks whose union of key blocks has every size modulo
+    four (the last 256-key tile padded with 1, 2 or 3 masked entries), is
+    empty, or holds entries only one of the two blocks lists."""
+    import torch
+    B, H, nb = 1, 3, 12
+    S = 64 * nb
+    q, k, v = _random_qkv(synth_mod, B, H, S, d, seed=77 + d)
+    mask = np.zeros((B, H, nb, nb), dtype=np.uint8)
+    for h in range(H):
+        m = mask[0, h]
+        # pair 0 (rows 0, 1): both empty
+        m[2, (h + 5) % nb] = 1                           # pair 1: union of 1, row 3 empty
+        m[4, [1, 2]] = 1
+        m[5, 3 + h] = 1                                  # pair 2: union of 3, disjoint lists
+        m[6, 0:5] = 1
+        m[7, 5:9] = 1                                    # pair 3: union of 9
+        m[8, :] = 1
+        m[9, ::2] = 1                                    # pair 4: union of 12, row 9 half of it
+        m[10, [h, nb - 1 - h]] = 1
+        m[11, [h, (h + 6) % nb]] = 1                     # pair 5: union of 3 with one shared
+    qd, kd, vd = to_device_bf16(q), to_device_bf16(k), to_device_bf16(v)
+    ws = nl.Workspace.create(nl.make_shape(B, H, S, d), nl.OP_FWD_WITH_MASK)
+    o, lse = nl.bsa_fwd_with_mask(qd, kd, vd, torch.from_numpy(mask).cuda(), workspace=ws)
+    assert ws.query_status() == 0
+    rows = np.arange(B * H * S, dtype=np.int64)
+    ro, rl = oracle_mod.masked_attention(q, k, v, mask, rows)
+    go, gl = _gather(o, lse, rows, S)
+    compare_attention(go, gl, ro, rl)
+    empty = mask.reshape(B * H, nb, nb).sum(-1) == 0
+    assert np.all(go.reshape(B * H, nb, 64, d)[empty] == 0.0)
+    assert np.all(np.isneginf(gl.reshape(B * H, nb, 64)[empty]))
