@@ -103,9 +103,21 @@ std::vector<int> chunk_schedule(int64_t heads, int max_heads) {
 // Streams and events reused across calls (one set per device, created once).
 struct PipeRes {
   cudaStream_t h2d = nullptr, d2h = nullptr, comp = nullptr;
-  cudaEvent_t in_ready[kSlots], in_free[kSlots], out_ready[kSlots], out_free[kSlots];
+  cudaEvent_t in_ready[kSlots] = {}, in_free[kSlots] = {}, out_ready[kSlots] = {},
+              out_free[kSlots] = {};
+  cudaEvent_t join[3] = {};   // a failed call: the caller's stream waits for every stream
   bool ok = false;
 };
+
+void release(PipeRes& r) {
+  for (cudaStream_t* p : {&r.h2d, &r.d2h, &r.comp})
+    if (*p) { cudaStreamDestroy(*p); *p = nullptr; }
+  for (int i = 0; i < kSlots; ++i)
+    for (cudaEvent_t* p : {&r.in_ready[i], &r.in_free[i], &r.out_ready[i], &r.out_free[i]})
+      if (*p) { cudaEventDestroy(*p); *p = nullptr; }
+  for (cudaEvent_t& ev : r.join)
+    if (ev) { cudaEventDestroy(ev); ev = nullptr; }
+}
 constexpr int kMaxDevices = 64;
 std::mutex g_mutex;
 PipeRes g_res[kMaxDevices];
@@ -127,7 +139,12 @@ nabla_status resources(PipeRes** out) {
       if (e == cudaSuccess) e = cudaEventCreateWithFlags(&r.out_ready[i], cudaEventDisableTiming);
       if (e == cudaSuccess) e = cudaEventCreateWithFlags(&r.out_free[i], cudaEventDisableTiming);
     }
-    if (e != cudaSuccess) return cuda_fail(e, "pipeline streams/events");
+    for (int i = 0; i < 3 && e == cudaSuccess; ++i)
+      e = cudaEventCreateWithFlags(&r.join[i], cudaEventDisableTiming);
+    if (e != cudaSuccess) {
+      release(r);
+      return cuda_fail(e, "pipeline streams/events");
+    }
     r.ok = true;
   }
   *out = &r;
@@ -168,6 +185,16 @@ NABLA_API nabla_status nabla_layer_host(const nabla_shape* shape, const nabla_ma
     return fail(NABLA_ERR_UNSUPPORTED, "nabla_layer_host takes tile-major tokens");
   if (reinterpret_cast<uintptr_t>(workspace) & 255u)
     return fail(NABLA_ERR_INVALID_ARG, "workspace needs 256-byte alignment");
+  // every check the chunks' calls make, before any copy is queued: a call that
+  // fails later must not leave copies of the caller's buffers in flight
+  if (!(params->thr >= 0.f && params->thr <= 1.f))
+    return fail(NABLA_ERR_UNSUPPORTED, "thr must lie in [0, 1]");
+  if (params->topk < 0) return fail(NABLA_ERR_INVALID_ARG, "topk must be >= 0");
+  if (params->use_sta && (params->wt < 0 || params->wh < 0 || params->ww < 0))
+    return fail(NABLA_ERR_INVALID_ARG, "STA half-windows must be non-negative");
+  if (shape->Tt <= 0 || shape->Th <= 0 || shape->Tw <= 0 ||
+      static_cast<int64_t>(shape->Tt) * shape->Th * shape->Tw != shape->S / 64)
+    return fail(NABLA_ERR_INVALID_ARG, "tile grid Tt*Th*Tw must equal S/64");
   PipeRes* r = nullptr;
   nabla_status s = resources(&r);
   if (s != NABLA_OK) return s;
@@ -188,6 +215,7 @@ NABLA_API nabla_status nabla_layer_host(const nabla_shape* shape, const nabla_ma
       (e = cudaStreamWaitEvent(r->d2h, start, 0)) != cudaSuccess ||
       (e = cudaStreamWaitEvent(r->comp, start, 0)) != cudaSuccess)
     return cuda_fail(e, "pipeline start");
+  const nabla_status result = [&]() -> nabla_status {
   int64_t h0 = 0;
   for (int64_t c = 0; c < nchunks; h0 += sizes[c], ++c) {
     const int slot = static_cast<int>(c % kSlots);
@@ -250,6 +278,16 @@ NABLA_API nabla_status nabla_layer_host(const nabla_shape* shape, const nabla_ma
     if ((e = cudaStreamWaitEvent(st, r->out_free[i], 0)) != cudaSuccess)
       return cuda_fail(e, "final wait");
   return NABLA_OK;
+  }();
+  if (result != NABLA_OK) {
+    // whatever was queued before the failure is ordered before later work on
+    // the caller's stream, so the caller's buffers are not in use once it syncs
+    const cudaStream_t others[3] = {r->h2d, r->comp, r->d2h};
+    for (int i = 0; i < 3; ++i)
+      if (cudaEventRecord(r->join[i], others[i]) == cudaSuccess)
+        cudaStreamWaitEvent(st, r->join[i], 0);
+  }
+  return result;
 }
 
 }  // extern "C"

@@ -220,7 +220,10 @@ NABLA_API nabla_status bsa_fwd_with_mask_static(const nabla_shape* shape, const 
  *                header (nabla_workspace_init once, nabla_query_status after)
  * Returns once the work is queued.  All of it, the last output copy
  * included, is ordered before anything later queued on `stream`: synchronise
- * `stream` before reading o_host or lse_host.  The library's copy streams are
+ * `stream` before reading o_host or lse_host.  Argument errors (the mask
+ * parameters included) return before anything is queued; a CUDA error part
+ * way through still orders every copy already queued before later work on
+ * `stream`, so the host buffers are free once `stream` is synchronised.  The library's copy streams are
  * per device, so two calls in flight at once on one device (other host
  * threads, or other streams without ordering) are not supported.
  */

@@ -207,3 +207,21 @@ def test_layer_host_chunk_schedule(nl, heads, hpc):
 
 def test_layer_host_schedule_wan(nl):
     assert nl.layer_host_chunks(40, 8) == [1, 2, 4, 8, 8, 8, 7, 2]
+
+
+def test_layer_host_rejects_bad_mask_params_before_queuing(nl):
+    # the mask parameters are checked before any copy or CUDA call
+    lib = nl.lib()
+    null = ctypes.c_void_p(0)
+    a = ctypes.c_void_p(1 << 20)
+    s = nl.make_shape(1, 4, 1024, 64, (4, 2, 2))
+    f = lib.nabla_layer_host
+    bad_thr = nl._MaskParams(1.5, 0, 0, 0, 0, 0)
+    assert f(ctypes.byref(s), ctypes.byref(bad_thr), a, a, a, a, a, 2, a, null) == 2
+    bad_topk = nl._MaskParams(0.2, 0, 0, 0, 0, -1)
+    assert f(ctypes.byref(s), ctypes.byref(bad_topk), a, a, a, a, a, 2, a, null) == 1
+    bad_sta = nl._MaskParams(0.2, 1, -1, 0, 0, 0)
+    assert f(ctypes.byref(s), ctypes.byref(bad_sta), a, a, a, a, a, 2, a, null) == 1
+    no_grid = nl.make_shape(1, 4, 1024, 64, (4, 2, 3))
+    ok = nl._MaskParams(0.2, 0, 0, 0, 0, 0)
+    assert f(ctypes.byref(no_grid), ctypes.byref(ok), a, a, a, a, a, 2, a, null) == 1
