@@ -244,12 +244,13 @@ nabla_status make_map_raster(CUtensorMap* map, const void* ptr, const nabla_shap
 
 // [rows][St][d] bf16 viewed as stride-St groups of token rows: 3D boxes of
 // 64 x 1 x 128 pick one token of each of 128 consecutive groups (128-byte swizzle).
-nabla_status make_map_strided(CUtensorMap* map, const void* ptr, uint64_t groups, int St, int d) {
+nabla_status make_map_strided(CUtensorMap* map, const void* ptr, uint64_t groups, int St, int d,
+                              uint32_t box_rows) {
   EncodeTiledFn fn = encode_fn();
   if (fn == nullptr) return fail(NABLA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(St), groups};
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(St) * d * 2};
-  cuuint32_t box[3] = {64, 1, 128};
+  cuuint32_t box[3] = {64, 1, box_rows};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides,
                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -604,8 +605,9 @@ nabla_status nabla_build_mask_xattn(const nabla_shape* shape, const nabla_mask_p
   const int64_t nrows = static_cast<int64_t>(BH) * nb;
   const uint64_t groups = static_cast<uint64_t>(BH) * (shape->S / stride);
   CUtensorMap mq, mk;
-  if ((s = make_map_strided(&mq, q, groups, stride, shape->d)) != NABLA_OK) return s;
-  if ((s = make_map_strided(&mk, k, groups, stride, shape->d)) != NABLA_OK) return s;
+  // Q' boxes of 128 strided rows, K' boxes of 256 (the scorer's query and key tiles)
+  if ((s = make_map_strided(&mq, q, groups, stride, shape->d, 128)) != NABLA_OK) return s;
+  if ((s = make_map_strided(&mk, k, groups, stride, shape->d, 256)) != NABLA_OK) return s;
   cudaError_t e = nabla::launch_xattn_scores(mq, mk, lse2, X, status_ptr(workspace), BH, shape->S,
                                              shape->d, stride, g_wait_limit_ns.load(), st);
   if (e != cudaSuccess) return cuda_fail(e, "xattn scores launch");

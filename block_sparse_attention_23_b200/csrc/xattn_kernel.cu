@@ -16,13 +16,14 @@
 // Two passes of one kernel: pass 1 forms the log2-domain LSE of every strided
 // query row (online max and sum over the key tiles), pass 2 the block sums of
 // p = 2^(a log2e - lse2).  One CTA per (b, h, 128 strided query rows); key
-// tiles of 128 strided rows; S = Q' K'^T accumulates over St*d/64 chunks of 64
-// features, each chunk a pair of 3D TMA boxes (128 rows x 64 columns, rows
-// St apart in the token axis: the antidiagonal gather happens in the copy).
-// S is double-buffered in tensor memory; two groups of four warps take
-// alternate key tiles (so two warps share each SM sub-partition's exponential
-// unit), pass 1 combining the groups' running maxima and sums at the end, pass
-// 2 writing disjoint blocks.  The block sums over a query block's 64/St rows
+// tiles of 256 strided rows; S = Q' K'^T (N = 256: the full tensor rate)
+// accumulates over St*d/64 chunks of 64 features, each chunk a pair of 3D TMA
+// boxes (128 Q' rows and 256 K' rows x 64 columns, rows St apart in the token
+// axis: the antidiagonal gather happens in the copy).  S is double-buffered in
+// tensor memory (2 x 256 columns); two groups of four warps take alternate key
+// tiles (so two warps share each SM sub-partition's exponential unit), each
+// row's 256 columns in two halves of 128, pass 1 combining the groups' running
+// maxima and sums at the end, pass 2 writing disjoint blocks.  The block sums over a query block's 64/St rows
 // (consecutive lanes of a warp) are butterfly shuffles; each block score is
 // written once, by the lane that leads its rows.
 //
@@ -39,14 +40,15 @@
 namespace nabla {
 
 constexpr int kXM = 128;                        // strided query rows per CTA
-constexpr int kXN = 128;                        // strided key rows per tile
+constexpr int kXN = 256;                        // strided key rows per tile
 constexpr int kXStages = 4;                     // ring of (Q' chunk, K' chunk) pairs
 constexpr int kXThreads = 384;
 constexpr int kXExpWarps = 8;
 constexpr int kXProducerWarp = 8, kXMmaWarp = 9;
-constexpr uint32_t kXChunkBytes = 128 * 64 * 2;   // one operand chunk: 128 rows x 64 bf16
-constexpr uint32_t kXStageBytes = 2 * kXChunkBytes;
-constexpr uint32_t kXTmemCols = 256;
+constexpr uint32_t kXChunkQBytes = kXM * 64 * 2;   // Q' chunk: 128 rows x 64 bf16
+constexpr uint32_t kXChunkKBytes = kXN * 64 * 2;   // K' chunk: 256 rows x 64 bf16
+constexpr uint32_t kXStageBytes = kXChunkQBytes + kXChunkKBytes;
+constexpr uint32_t kXTmemCols = 512;
 // Register split after set-up (per warpgroup): 8*216 + 4*72 = 12*168, the
 // launch allocation (checked on the host before launch).
 constexpr int kXRegsExp = 216, kXRegsOther = 72, kXRegsLaunch = 168;
@@ -173,7 +175,7 @@ __global__ void __launch_bounds__(kXThreads, 1)
           ++armed[st];
           // Q' chunk: query rows i*St + (St-1-s); K' chunk: key rows j*St + s
           tma_load_3d(dst, &tmQ, bar(kXBarFull + st), h * 64, prm.St - 1 - s, qrow);
-          tma_load_3d(dst + kXChunkBytes, &tmK, bar(kXBarFull + st), h * 64, s, krow);
+          tma_load_3d(dst + kXChunkQBytes, &tmK, bar(kXBarFull + st), h * 64, s, krow);
         }
         if (stop) break;
       }
@@ -197,10 +199,10 @@ __global__ void __launch_bounds__(kXThreads, 1)
           const int st = u % kXStages;
           if (!mbar_wait(bar(kXBarFull + st), (u / kXStages) & 1, lim, abort_flag)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t a = sRing + st * kXStageBytes, bk = a + kXChunkBytes;
+          const uint32_t a = sRing + st * kXStageBytes, bk = a + kXChunkQBytes;
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            tc_mma_ss(tmem + b * 128u, sdesc_sw128(a + kk * 32, 16, 1024),
+            tc_mma_ss(tmem + b * static_cast<uint32_t>(kXN), sdesc_sw128(a + kk * 32, 16, 1024),
                       sdesc_sw128(bk + kk * 32, 16, 1024), idesc, (c > 0 || kk > 0) ? 1u : 0u);
           tc_commit(bar(kXBarEmpty + st));
         }
@@ -227,59 +229,73 @@ __global__ void __launch_bounds__(kXThreads, 1)
     float m = -INFINITY, l = 0.f;
     bool ok = true;
     for (int t = grp; t < n_t; t += 2) {
-      const int nvalid = min(kXN, prm.L - t * kXN);   // a multiple of kPer
+      const int nvalid_t = min(kXN, prm.L - t * kXN);   // a multiple of kPer
       if (!x_warp_wait(bar(kXBarSFull + grp), (t >> 1) & 1, lim, abort_flag)) { ok = false; break; }
       tc_fence_after();
-      const uint32_t sb = tmem + lane_off + grp * 128u;
-      uint32_t sv[4][32];
-#pragma unroll
-      for (int ch = 0; ch < 4; ++ch) tmem_ld32(sb + ch * 32, sv[ch]);
-      tmem_ld_wait();
-      tc_fence_before();
-      mbar_arrive(bar(kXBarSFree + grp));
-      if (kPass == 1) {
-        float mx = -INFINITY;
-#pragma unroll
-        for (int ch = 0; ch < 4; ++ch)
-#pragma unroll
-          for (int i = 0; i < 32; ++i)
-            if (ch * 32 + i < nvalid) mx = fmaxf(mx, __uint_as_float(sv[ch][i]));
-        const float m_new = fmaxf(m, mx * sl2);
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int ch = 0; ch < 4; ++ch)
-#pragma unroll
-          for (int i = 0; i < 32; ++i)
-            if (ch * 32 + i < nvalid)
-              acc[i & 3] += fast_exp2(fmaf(__uint_as_float(sv[ch][i]), sl2, -m_new));
-        l = l * fast_exp2(m - m_new) + ((acc[0] + acc[1]) + (acc[2] + acc[3]));
-        m = m_new;
-      } else {
-        // block sums of p over this row's kN / kPer key blocks, then over the
-        // kPer rows of the query block (consecutive lanes)
-        constexpr int kNkb = kXN / kPer;
-        float bs[kNkb];
-#pragma unroll
-        for (int j = 0; j < kNkb; ++j) {
-          float a = 0.f;
-#pragma unroll
-          for (int e = 0; e < kPer; ++e) {
-            const int c = j * kPer + e;
-            if (c < nvalid) a += fast_exp2(fmaf(__uint_as_float(sv[c >> 5][c & 31]), sl2, -lse2));
+#pragma unroll 1
+      for (int hf = 0; hf < 2; ++hf) {     // 128 columns at a time
+        const int nvalid = nvalid_t - 128 * hf;
+        if (nvalid <= 0) {
+          if (hf == 1) {   // the buffer is read (nothing in this half)
+            tc_fence_before();
+            mbar_arrive(bar(kXBarSFree + grp));
           }
-          bs[j] = row_valid ? a : 0.f;
+          continue;
         }
+        const uint32_t sb = tmem + lane_off + grp * static_cast<uint32_t>(kXN) + 128u * hf;
+        uint32_t sv[4][32];
 #pragma unroll
-        for (int o = 1; o < kPer; o <<= 1)
+        for (int ch = 0; ch < 4; ++ch) tmem_ld32(sb + ch * 32, sv[ch]);
+        tmem_ld_wait();
+        if (hf == 1) {   // both halves read: the tensor cores may refill the buffer
+          tc_fence_before();
+          mbar_arrive(bar(kXBarSFree + grp));
+        }
+        if (kPass == 1) {
+          float mx = -INFINITY;
 #pragma unroll
-          for (int j = 0; j < kNkb; ++j) bs[j] += __shfl_xor_sync(0xffffffffu, bs[j], o);
-        if ((lane % kPer) == 0 && row_valid && *abort_flag == 0) {
-          const int rb = qrow / kPer;                      // query block in the head
-          float* dst = prm.scores + (static_cast<int64_t>(bh) * prm.nb + rb) * prm.nb + t * (kXN / kPer);
-          const float inv = 1.0f / kPer;
+          for (int ch = 0; ch < 4; ++ch)
 #pragma unroll
-          for (int j = 0; j < kNkb; ++j)
-            if (j * kPer < nvalid) dst[j] = bs[j] * inv;
+            for (int i = 0; i < 32; ++i)
+              if (ch * 32 + i < nvalid) mx = fmaxf(mx, __uint_as_float(sv[ch][i]));
+          const float m_new = fmaxf(m, mx * sl2);
+          float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+          for (int ch = 0; ch < 4; ++ch)
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              if (ch * 32 + i < nvalid)
+                acc[i & 3] += fast_exp2(fmaf(__uint_as_float(sv[ch][i]), sl2, -m_new));
+          l = l * fast_exp2(m - m_new) + ((acc[0] + acc[1]) + (acc[2] + acc[3]));
+          m = m_new;
+        } else {
+          // block sums of p over this half's 128 / kPer key blocks, then over
+          // the kPer rows of the query block (consecutive lanes)
+          constexpr int kNkb = 128 / kPer;
+          float bs[kNkb];
+#pragma unroll
+          for (int j = 0; j < kNkb; ++j) {
+            float a = 0.f;
+#pragma unroll
+            for (int e = 0; e < kPer; ++e) {
+              const int c = j * kPer + e;
+              if (c < nvalid) a += fast_exp2(fmaf(__uint_as_float(sv[c >> 5][c & 31]), sl2, -lse2));
+            }
+            bs[j] = row_valid ? a : 0.f;
+          }
+#pragma unroll
+          for (int o = 1; o < kPer; o <<= 1)
+#pragma unroll
+            for (int j = 0; j < kNkb; ++j) bs[j] += __shfl_xor_sync(0xffffffffu, bs[j], o);
+          if ((lane % kPer) == 0 && row_valid && *abort_flag == 0) {
+            const int rb = qrow / kPer;                      // query block in the head
+            float* dst = prm.scores + (static_cast<int64_t>(bh) * prm.nb + rb) * prm.nb +
+                         (t * kXN + 128 * hf) / kPer;
+            const float inv = 1.0f / kPer;
+#pragma unroll
+            for (int j = 0; j < kNkb; ++j)
+              if (j * kPer < nvalid) dst[j] = bs[j] * inv;
+          }
         }
       }
     }
