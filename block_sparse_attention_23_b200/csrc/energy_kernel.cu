@@ -16,13 +16,15 @@
 //
 // Work decomposition: one CTA per (b, h, pair of query blocks 2p, 2p+1) = one
 // 128-row query tile; the key blocks visited are the union of the two CSR
-// rows (2-bit membership), two union entries per 128-key tile, each entry a
+// rows (2-bit membership), four union entries per 256-key tile, each entry a
 // contiguous 64 x d slab loaded by one 2D TMA box per 64 columns.  S = Q K^T
-// goes to tensor memory (two 128-column buffers, so the next tile's MMA runs
-// while the current one is exponentiated); a thread owns one query row,
-// exponentiates against its LSE and sums each 64-key half; the two warps of a
-// query block add their warp sums into a shared-memory row of E (exactly two
-// addends onto zero: the result does not depend on their order).
+// (N = 256: the full tensor rate) goes to tensor memory (two 256-column
+// buffers, so the next tile's MMA runs while the current one is
+// exponentiated); a thread owns one query row, reads its 256 columns in two
+// halves of 128, exponentiates against its LSE and sums each 64-key entry;
+// the two warps of a query block add their warp sums into a shared-memory row
+// of E (exactly two addends onto zero: the result does not depend on their
+// order).
 //
 // Roles (384 threads): warps 0-7 exponentiate and sum in two groups of four
 // (group g takes the tiles t = g mod 2 and the S buffer g, so two warps per
@@ -40,13 +42,13 @@
 namespace nabla {
 
 constexpr int kEM = 128;            // query rows per CTA (two blocks)
-constexpr int kEN = 128;            // keys per tile (two list entries)
-constexpr int kEStages = 3;         // K ring depth
+constexpr int kEN = 256;            // keys per tile (four list entries)
+constexpr int kEStages = 2;         // K ring depth
 constexpr int kEThreads = 384;
 constexpr int kESumWarps = 8;                     // two groups of four, one per S buffer
 constexpr int kEProducerWarp = 8, kEMmaWarp = 9;
 constexpr int kEMaxNb = 4096;
-constexpr uint32_t kETmemCols = 256;
+constexpr uint32_t kETmemCols = 512;
 constexpr uint64_t kEDrainNs = 1000000000ull;
 
 template <int D>
@@ -202,15 +204,15 @@ __global__ void __launch_bounds__(kEThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
   const int n_u = *n_union_s;
-  const int n_t = (n_u + 1) >> 1;
+  const int n_t = (n_u + 3) >> 2;
   const uint64_t lim = prm.wait_limit_ns;
-  auto tile_entry = [&](int t, int i) { return (2 * t + i < n_u) ? ulist[2 * t + i] : 0; };
+  auto tile_entry = [&](int t, int i) { return (4 * t + i < n_u) ? ulist[4 * t + i] : 0; };
 
   if (warp == kEProducerWarp) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0 && n_t > 0) {
       const int64_t row0 = static_cast<int64_t>(bh) * prm.S;
-      int armed[kEStages] = {0, 0, 0};
+      int armed[kEStages] = {0, 0};
       mbar_arrive_expect_tx(bar(kEBarQFull), L::kQBytes);
       for (int qb = 0; qb < 2; ++qb) {
         const int rb = r0 + (qb < nq ? qb : 0);   // a missing second block repeats the first
@@ -218,21 +220,22 @@ __global__ void __launch_bounds__(kEThreads, 1)
           tma_load_2d(sQ + h * kEM * 128 + qb * 64 * 128, &tmQ, bar(kEBarQFull), h * 64,
                       static_cast<int32_t>(row0 + static_cast<int64_t>(rb) * 64));
       }
+      const int last = ulist[n_u - 1] & 0xFFFF;   // padding entries repeat it (no row lists them)
       for (int t = 0; t < n_t; ++t) {
         const int s = t % kEStages, n = t / kEStages;
-        const int j0 = ulist[2 * t] & 0xFFFF;
-        const int j1 = (2 * t + 1 < n_u) ? (ulist[2 * t + 1] & 0xFFFF) : j0;
         if (t >= kEStages && !mbar_wait(bar(kEBarKEmpty + s), (n - 1) & 1, lim, abort_flag)) {
           e_abort(abort_flag, prm.status);
           break;
         }
         mbar_arrive_expect_tx(bar(kEBarKFull + s), L::kKBytes);
         ++armed[s];
-        for (int kb = 0; kb < 2; ++kb)
+        for (int kb = 0; kb < 4; ++kb) {
+          const int j = (4 * t + kb < n_u) ? (ulist[4 * t + kb] & 0xFFFF) : last;
           for (int h = 0; h < L::kDH; ++h)
             tma_load_2d(sK + s * L::kKBytes + h * kEN * 128 + kb * 64 * 128, &tmK,
                         bar(kEBarKFull + s), h * 64,
-                        static_cast<int32_t>(row0 + static_cast<int64_t>(kb ? j1 : j0) * 64));
+                        static_cast<int32_t>(row0 + static_cast<int64_t>(j) * 64));
+        }
       }
       // drain: every armed phase completes before shared memory is released
       mbar_wait(bar(kEBarQFull), 0, kEDrainNs, nullptr);
@@ -258,7 +261,7 @@ __global__ void __launch_bounds__(kEThreads, 1)
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t offq = (kk >> 2) * (kEM * 128) + (kk & 3) * 32;
           const uint32_t offk = (kk >> 2) * (kEN * 128) + (kk & 3) * 32;
-          tc_mma_ss(tmem + b * 128, sdesc_sw128(sQ + offq, 16, 1024),
+          tc_mma_ss(tmem + b * static_cast<uint32_t>(kEN), sdesc_sw128(sQ + offq, 16, 1024),
                     sdesc_sw128(kt + offk, 16, 1024), idesc, kk > 0 ? 1u : 0u);
         }
         tc_commit(bar(kEBarSFull + b));
@@ -289,33 +292,47 @@ __global__ void __launch_bounds__(kEThreads, 1)
     bool ok = true;
     for (int t = grp; t < n_t; t += 2) {
       const int b = grp;
-      const int e0 = tile_entry(t, 0), e1 = tile_entry(t, 1);
-      const bool v0 = (e0 & bit) != 0, v1 = (e1 & bit) != 0;   // uniform per warp
       if (!e_warp_wait(bar(kEBarSFull + b), (t >> 1) & 1, lim, abort_flag)) { ok = false; break; }
       tc_fence_after();
-      const uint32_t sb = tmem + lane_off + b * 128;
-      uint32_t sv[4][32];
-      if (v0) { tmem_ld32(sb, sv[0]); tmem_ld32(sb + 32, sv[1]); }
-      if (v1) { tmem_ld32(sb + 64, sv[2]); tmem_ld32(sb + 96, sv[3]); }
-      tmem_ld_wait();
-      tc_fence_before();
-      mbar_arrive(bar(kEBarSFree + b));
-      float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-#pragma unroll
-      for (int ch = 0; ch < 4; ++ch) {
-        if (((ch < 2) ? v0 : v1) && live) {
-#pragma unroll
-          for (int i = 0; i < 32; ++i)
-            acc[ch >> 1][i & 3] += fast_exp2(fmaf(__uint_as_float(sv[ch][i]), sl2, neg_lse2));
+#pragma unroll 1
+      for (int hf = 0; hf < 2; ++hf) {           // entries 4t + 2hf, 4t + 2hf + 1
+        const int e0 = tile_entry(t, 2 * hf), e1 = tile_entry(t, 2 * hf + 1);
+        const bool v0 = (e0 & bit) != 0, v1 = (e1 & bit) != 0;   // uniform per warp
+        const uint32_t sb = tmem + lane_off + b * static_cast<uint32_t>(kEN) + 128u * hf;
+        uint32_t sv[4][32];
+        if (v0) { tmem_ld32(sb, sv[0]); tmem_ld32(sb + 32, sv[1]); }
+        if (v1) { tmem_ld32(sb + 64, sv[2]); tmem_ld32(sb + 96, sv[3]); }
+        tmem_ld_wait();
+        if (hf == 1) {   // both halves read: the tensor cores may refill the buffer
+          tc_fence_before();
+          mbar_arrive(bar(kEBarSFree + b));
         }
-      }
-      if (v0) {
-        const float w = e_warp_sum((acc[0][0] + acc[0][1]) + (acc[0][2] + acc[0][3]));
-        if (lane == 0) atomicAdd(&myE[e0 & 0xFFFF], w);
-      }
-      if (v1) {
-        const float w = e_warp_sum((acc[1][0] + acc[1][1]) + (acc[1][2] + acc[1][3]));
-        if (lane == 0) atomicAdd(&myE[e1 & 0xFFFF], w);
+        float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        if (v0 && v1 && __all_sync(0xffffffffu, live)) {
+          // both entries listed: one straight-line block without per-chunk branches
+#pragma unroll
+          for (int ch = 0; ch < 4; ++ch)
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              acc[ch >> 1][i & 3] += fast_exp2(fmaf(__uint_as_float(sv[ch][i]), sl2, neg_lse2));
+        } else {
+#pragma unroll
+          for (int ch = 0; ch < 4; ++ch) {
+            if (((ch < 2) ? v0 : v1) && live) {
+#pragma unroll
+              for (int i = 0; i < 32; ++i)
+                acc[ch >> 1][i & 3] += fast_exp2(fmaf(__uint_as_float(sv[ch][i]), sl2, neg_lse2));
+            }
+          }
+        }
+        if (v0) {
+          const float w = e_warp_sum((acc[0][0] + acc[0][1]) + (acc[0][2] + acc[0][3]));
+          if (lane == 0) atomicAdd(&myE[e0 & 0xFFFF], w);
+        }
+        if (v1) {
+          const float w = e_warp_sum((acc[1][0] + acc[1][1]) + (acc[1][2] + acc[1][3]));
+          if (lane == 0) atomicAdd(&myE[e1 & 0xFFFF], w);
+        }
       }
     }
     if (!ok) e_abort(abort_flag, prm.status);
