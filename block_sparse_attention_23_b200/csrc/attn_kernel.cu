@@ -15,7 +15,9 @@
 //   (the last one repeats its final entry, masked for every row).  Each entry
 //   is one contiguous 64 x d slab of the [B,H,S,d] tensor, loaded as a plain 2D
 //   TMA box.  A row whose block did not list an entry gives it probability 0
-//   (no exponentials evaluated).
+//   (no exponentials evaluated).  Query tile g of a head starts at key tile
+//   floor(g * n_t / groups) of its n_t and wraps around, so that neighbouring
+//   CTAs in flight spread their K/V requests over the head.
 //
 // Roles (384 threads)
 //   warps 0-7   softmax: warp w owns tensor-memory lane quarter q = w % 4 (rows
@@ -264,9 +266,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int n_u = *n_union_s;
   const int n_t = (n_u + kEntries - 1) / kEntries;
   const uint64_t lim = prm.wait_limit_ns;
+  // The key tiles are visited from a start that moves with the query tile's
+  // place in the head (tile t is union tile (t + t_off) mod n_t), so the CTAs
+  // in flight, neighbours in the head, do not all request the same K/V blocks
+  // at the same moment; the online softmax does not depend on the order.
+  const int t_off =
+      n_t > 0 ? static_cast<int>((static_cast<int64_t>(grp) * n_t) / prm.ngroups) : 0;
+  auto tile_of = [&](int t) {
+    const int u = t + t_off;
+    return u >= n_t ? u - n_t : u;
+  };
   // entry e of key tile t (0 past the end of the union: no row lists it)
   auto tile_entry = [&](int t, int e) {
-    return (kEntries * t + e < n_u) ? ulist[kEntries * t + e] : 0;
+    const int u = tile_of(t);
+    return (kEntries * u + e < n_u) ? ulist[kEntries * u + e] : 0;
   };
 
   if (warp >= 8) {
@@ -297,7 +310,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive_expect_tx(bar(full), L::kKVBytes);
         ++armed;
         for (int e = 0; e < kEntries; ++e) {
-          const int j = (kEntries * t + e < n_u) ? (ulist[kEntries * t + e] & 0xFFFF) : last;
+          const int u = tile_of(t);
+          const int j = (kEntries * u + e < n_u) ? (ulist[kEntries * u + e] & 0xFFFF) : last;
           for (int h = 0; h < L::kDH; ++h)
             load_block<kRaster>(buf + h * kBN * 128 + e * 64 * 128, map, bar(full), h, bh, j,
                                 prm.S, prm.Th, prm.Tw);
