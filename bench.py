@@ -334,6 +334,8 @@ def run_ours(args):
     value = kept_flops * ws / (ms_per_step * 1e-3) / 1e12
     ws_mask.check()
     ws_fwd.check()
+    # forwards (check, warm-up, timed) that needed the exact-reference kernel
+    fwd_exact_passes = ws_fwd.exact_passes()
 
     # end to end through the public API with host buffers: nabla_layer_host
     # reads Q, K, V from pinned memory and writes O and LSE back to it every
@@ -559,6 +561,9 @@ def run_ours(args):
                           "over_kept": exec_flops / kept_flops,
                           "what": "128x128 S and PV products the kernel runs (union of two "
                                   "query blocks in 256-key tiles), counted on the host"},
+        "attn_exact_passes": {"count": fwd_exact_passes, "forwards": 1 + args.warmup + args.steps,
+                              "what": "forwards whose fixed-reference kernel asked the exact-"
+                                      "reference kernel to recompute the call"},
         "pct_of_dense_bf16_peak": {"attn_vs_sustained": attn_tflops / peak,
                                    "attn_vs_burst": attn_tflops / peaks["bf16_tflops"],
                                    "layer_vs_sustained": value / ws / peak},
@@ -600,7 +605,7 @@ def run_ours(args):
         "raster_layer": {"ms_per_layer": raster_ms, "vs_tile_major": raster_ms / ms_per_step,
                          "what": "mask + attention on raster-ordered Q, K, V (O, LSE raster), "
                                  "token reorder fused into the loads; outside the step"},
-        "gpu_launches": 6 * args.steps,
+        "gpu_launches": 7 * args.steps,
         "clocks": clk,
     }
     if args.profile_heads:

@@ -35,7 +35,7 @@ EXPORTED = ["nabla_workspace_size", "nabla_workspace_init", "nabla_query_status"
             "bsa_fwd_with_mask_static", "nabla_reorder_tokens", "nabla_block_energy",
             "nabla_calib_accumulate", "nabla_calib_finalize", "bsa_bwd",
             "nabla_build_mask_xattn", "nabla_layer_host_workspace_size", "nabla_layer_host",
-            "nabla_layer_host_chunks"]
+            "nabla_layer_host_chunks", "nabla_set_exact_reference", "nabla_query_exact_passes"]
 TO_TILE_MAJOR, TO_RASTER = 0, 1
 
 
@@ -96,6 +96,10 @@ def lib() -> ctypes.CDLL:
             L.nabla_version.argtypes = []
             L.nabla_set_wait_limit_ns.restype = None
             L.nabla_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
+            L.nabla_set_exact_reference.restype = None
+            L.nabla_set_exact_reference.argtypes = [i32]
+            L.nabla_query_exact_passes.restype = i32
+            L.nabla_query_exact_passes.argtypes = [vp, vp]
             L.nabla_selftest_mma.restype = i32
             L.nabla_selftest_mma.argtypes = [i32, vp, vp, vp, vp, vp]
             L.nabla_reorder_tokens.restype = i32
@@ -181,6 +185,14 @@ class Workspace:
 
     def check(self, stream=None) -> None:
         _check(self.query_status(stream))
+
+    def exact_passes(self, stream=None) -> int:
+        """Synchronise and return how many forwards on this workspace needed the
+        exact-reference kernel."""
+        n = int(lib().nabla_query_exact_passes(_ptr(self.buf), _stream(stream)))
+        if n < 0:
+            raise NablaError(4, lib().nabla_last_error().decode())
+        return n
 
 
 def _shape_of(q, tile_grid=(0, 0, 0), layout: int = LAYOUT_TILE_MAJOR) -> _Shape:
@@ -276,6 +288,11 @@ def bsa_fwd_with_mask(q, k, v, mask_u8, scale: Optional[float] = None,
 
 def set_wait_limit_ns(ns: int) -> None:
     lib().nabla_set_wait_limit_ns(int(ns))
+
+
+def set_exact_reference(on: bool) -> None:
+    """Process-wide: run every forward's exact-reference kernel alone."""
+    lib().nabla_set_exact_reference(1 if on else 0)
 
 
 def selftest_mma(variant: int, a, b, workspace: Optional[Workspace] = None, stream=None):

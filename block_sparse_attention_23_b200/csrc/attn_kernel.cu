@@ -23,9 +23,10 @@
 //   warps 0-7   softmax: warp w owns tensor-memory lane quarter q = w % 4 (rows
 //               32q..32q+31 of the tile) and column half c = w / 4 (keys
 //               [128c, 128c+128) of each key tile, its entries 2c and 2c+1).
-//               The two warps of a lane quarter trade partial row maxima (and,
-//               at the end, partial row sums) through shared memory, meeting on
-//               an mbarrier with a bounded wait.
+//               The two warps of a lane quarter trade partial row maxima
+//               when they agree on a reference (and, at the end, partial row
+//               sums) through shared memory, meeting on an mbarrier with a
+//               bounded wait.
 //   warp 8      TMA producer of Q and K (and the union-list compaction).
 //   warp 9      tensor-memory allocation and the single MMA-issuing thread.
 //   warp 10     TMA producer of V; warp 11 idles (completes warpgroup 2).
@@ -46,13 +47,19 @@
 // so the reorder to tile-major happens inside the TMA loads, and O / LSE rows
 // are stored back at their raster positions.
 //
-// Online softmax with a lazy maximum: the running max m of a row is raised
-// (and O, l rescaled by 2^(m_old - m_new)) only when a tile's max exceeds it by
-// more than 2^8; otherwise p <= 256 and O / l, LSE = ln2 (m + log2 l) are
-// unchanged in exact arithmetic.  The tile max is formed from the S row in
-// registers, then the exponentials; a warp whose two entries the row both
-// lists (the common case) runs that as one straight-line block without
-// per-chunk branches, which lets the compiler interleave the whole row.
+// Online softmax with a reference maximum per row.  Each launch runs two
+// passes over the same grid.  The fixed-reference pass: the two warps of a
+// lane quarter agree on the row max of the first key tile the row's block
+// lists, and that reference m stays for the rest of the row (no further max
+// or exchange per tile; p = 2^(s*scale*log2e - m) may exceed 1).  A warp
+// whose partial row sum of a tile (128 columns) exceeds 2^16 sets a flag in
+// the caller's workspace, and the exact-reference pass then recomputes the
+// whole launch: there the warps agree on every tile's max and raise m (with O
+// and l rescaled by 2^(m_old - m_new)) whenever it grows by more than 2^8, so
+// p <= 256.  Its CTAs return at once when the flag is clear.  O / l and
+// LSE = ln2 (m + log2 l) do not depend on the reference in exact arithmetic.
+// A warp whose two entries the row both lists (the common case) runs its
+// loads and exponentials as straight-line code without per-chunk branches.
 //
 // Every mbarrier wait is time-bounded; a wait that runs out records
 // kStatusTimeout, raises a CTA-wide abort flag, and the CTA drains its own TMA
@@ -80,6 +87,10 @@ constexpr int kMaxNb = 4096;    // blocks per head supported
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0, kColP = 256, kColO = 384;
 constexpr float kRescaleThreshold = 8.0f;            // log2 units
+// Largest partial row sum (one warp's 128 columns of a key tile, relative to
+// the row's fixed reference) the fixed-reference pass accepts: every p stays
+// below 2^16, so O and l keep the fp32 range the exact pass has for them.
+constexpr float kFixedRefSumLimit = 65536.0f;
 constexpr uint64_t kDrainLimitNs = 1000000000ull;   // 1 s for draining in-flight work
 
 template <int D>
@@ -125,6 +136,9 @@ struct AttnParams {
   int Th, Tw;              // tile grid (raster token order only)
   float scale_log2;        // softmax scale * log2(e)
   uint64_t wait_limit_ns;
+  int* redo;               // set by a pass that needs the exact-reference pass (see below)
+  int* exact_passes;       // counts the exact-reference passes that ran
+  int exact;               // 0: reference fixed per row; 1: the exact-reference pass
 };
 
 // One 64-token block of a [B,H,S,d] tensor as a 64 x 64 shared-memory box
@@ -188,6 +202,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int item = blockIdx.x;
+  // the exact-reference pass runs only after a fixed-reference pass asked for it
+  if (prm.exact) {
+    if (*prm.redo == 0) return;
+    if (item == 0 && tid == 0) atomicAdd(prm.exact_passes, 1);
+  }
   const int bh = item / prm.ngroups;
   const int grp = item % prm.ngroups;
   const int nb = prm.nb;
@@ -396,8 +415,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t o_base = tmem + lane_off + kColO + static_cast<uint32_t>(D / 2) * half;
     const uint32_t pair_bar = bar(kBarPair + quarter);
     const float sl2 = prm.scale_log2;
-    float m = -INFINITY;        // lazy running max of the row, log2 units (same in both warps)
+    float m = -INFINITY;        // reference max of the row, log2 units (same in both warps)
     float l = 0.f;              // running sum over this warp's columns of the row
+    int pair_n = 0;             // phases of the pair barrier used so far
     bool ok = true;
     for (int t = 0; t < n_t; ++t) {
       const bool v0 = (tile_entry(t, 2 * half) & bit) != 0;       // uniform per warp
@@ -406,21 +426,28 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       // this warp's 128 S columns of the row in one batch of loads
       uint32_t sv[4][32];
-      float mx[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) mx[i] = -INFINITY;
-      if (v0 && v1) {   // both entries listed: loads and max without per-chunk branches
+      if (v0 && v1) {
 #pragma unroll
         for (int ch = 0; ch < 4; ++ch) tmem_ld32(s_base + 32 * ch, sv[ch]);
-        tmem_ld_wait();
-#pragma unroll
-        for (int ch = 0; ch < 4; ++ch)
-#pragma unroll
-          for (int i = 0; i < 32; ++i) mx[i & 7] = fmaxf(mx[i & 7], __uint_as_float(sv[ch][i]));
       } else {
         if (v0) { tmem_ld32(s_base, sv[0]); tmem_ld32(s_base + 32, sv[1]); }
         if (v1) { tmem_ld32(s_base + 64, sv[2]); tmem_ld32(s_base + 96, sv[3]); }
-        tmem_ld_wait();
+      }
+      tmem_ld_wait();
+      // S(t) is in registers: the tensor cores may overwrite it with S(t+1)
+      tc_fence_before();
+      mbar_arrive(bar(kBarSFree));
+      // Reference of the exponentials.  Fixed-reference pass: the row's
+      // reference is the max of the first key tile the row's block lists
+      // (agreed with the other warp of the lane quarter), then kept.  Exact
+      // pass: the two warps agree on every tile's max and raise the reference
+      // lazily.  Both warps take the same branch (m is the same in both).
+      const bool agree = prm.exact || __any_sync(0xffffffffu, m == -INFINITY);
+      bool pv_done = t == 0;                     // PV(t-1) completed (known so far)
+      if (agree) {
+        float mx[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) mx[i] = -INFINITY;
 #pragma unroll
         for (int ch = 0; ch < 4; ++ch) {
           if ((ch < 2) ? v0 : v1) {
@@ -428,47 +455,43 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int i = 0; i < 32; ++i) mx[i & 7] = fmaxf(mx[i & 7], __uint_as_float(sv[ch][i]));
           }
         }
-      }
-      // S(t) is in registers: the tensor cores may overwrite it with S(t+1)
-      tc_fence_before();
-      mbar_arrive(bar(kBarSFree));
-      const float m_part = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                                 fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * sl2;
-      // the row's max over all 256 keys: trade partial maxima with the other
-      // warp of this lane quarter (slots alternate with the tile's parity)
-      xch[((t & 1) * 2 + half) * kBM + row] = m_part;
-      mbar_arrive(pair_bar);
-      if (!warp_wait(pair_bar, t & 1, lim, abort_flag)) { ok = false; break; }
-      const float m_tile = fmaxf(m_part, xch[((t & 1) * 2 + (half ^ 1)) * kBM + row]);
-      const bool has = m_tile > -INFINITY;
-      const bool first = m == -INFINITY;
-      const bool need = has && !first && (m_tile > m + kRescaleThreshold);   // rescale O, l
-      const float m_old = m;
-      if (has && (first || need)) m = m_tile;
-      // O must hold PV(t-1) before it is rescaled by 2^(m_old - m); rare after
-      // the first tiles, so the wait is paid only then
-      bool rescale = __any_sync(0xffffffffu, need);
-      bool pv_done = t == 0;                     // PV(t-1) completed (known so far)
-      if (rescale && !pv_done) {
-        if (!warp_wait(bar(kBarOFull), (t - 1) & 1, lim, abort_flag)) {
-          ok = false;
-          rescale = false;
+        const float m_part = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                                   fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * sl2;
+        // the row's max over all 256 keys: trade partial maxima with the other
+        // warp of this lane quarter (slots alternate with the barrier's phase)
+        xch[((pair_n & 1) * 2 + half) * kBM + row] = m_part;
+        mbar_arrive(pair_bar);
+        if (!warp_wait(pair_bar, pair_n & 1, lim, abort_flag)) { ok = false; break; }
+        const float m_tile = fmaxf(m_part, xch[((pair_n & 1) * 2 + (half ^ 1)) * kBM + row]);
+        ++pair_n;
+        const bool has = m_tile > -INFINITY;
+        const bool first = m == -INFINITY;
+        const bool need = has && !first && (m_tile > m + kRescaleThreshold);   // rescale O, l
+        const float m_old = m;
+        if (has && (first || need)) m = m_tile;
+        // O must hold PV(t-1) before it is rescaled by 2^(m_old - m)
+        bool rescale = __any_sync(0xffffffffu, need);
+        if (rescale && !pv_done) {
+          if (!warp_wait(bar(kBarOFull), (t - 1) & 1, lim, abort_flag)) {
+            ok = false;
+            rescale = false;
+          }
+          pv_done = true;
         }
-        pv_done = true;
-      }
-      if (rescale) {
-        tc_fence_after();
-        const float alpha = need ? fast_exp2(m_old - m) : 1.f;
-        l *= alpha;
+        if (rescale) {
+          tc_fence_after();
+          const float alpha = need ? fast_exp2(m_old - m) : 1.f;
+          l *= alpha;
 #pragma unroll 1
-        for (int cc = 0; cc < D / 32; ++cc) {
-          uint32_t o[16];
-          tmem_ld16(o_base + cc * 16, o);
-          tmem_ld_wait();
+          for (int cc = 0; cc < D / 32; ++cc) {
+            uint32_t o[16];
+            tmem_ld16(o_base + cc * 16, o);
+            tmem_ld_wait();
 #pragma unroll
-          for (int i = 0; i < 16; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-          tmem_st16(o_base + cc * 16, o);
-          tmem_st_wait();
+            for (int i = 0; i < 16; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            tmem_st16(o_base + cc * 16, o);
+            tmem_st_wait();
+          }
         }
       }
       // p = 2^(s*scale*log2e - m), packed to bf16 pairs and kept in registers
@@ -506,7 +529,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      l += (rs[0] + rs[1]) + (rs[2] + rs[3]);
+      const float l_tile = (rs[0] + rs[1]) + (rs[2] + rs[3]);
+      l += l_tile;
+      // a row whose later keys outgrow the fixed reference asks for the exact pass
+      if (!agree && __any_sync(0xffffffffu, !(l_tile <= kFixedRefSumLimit)) && lane == 0)
+        atomicExch(prm.redo, 1);
       if (!ok) break;
       if (!pv_done && !warp_wait(bar(kBarOFull), (t - 1) & 1, lim, abort_flag)) {
         ok = false;
@@ -531,11 +558,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool have_l = ok;
     float l_row = l;
     if (ok) {
-      xch[((n_t & 1) * 2 + half) * kBM + row] = l;
+      xch[((pair_n & 1) * 2 + half) * kBM + row] = l;
       mbar_arrive(pair_bar);
-      have_l = warp_wait(pair_bar, n_t & 1, lim, abort_flag);
+      have_l = warp_wait(pair_bar, pair_n & 1, lim, abort_flag);
       if (!have_l) record_abort(abort_flag, prm.status, kStatusTimeout);
-      else l_row = l + xch[((n_t & 1) * 2 + (half ^ 1)) * kBM + row];
+      else l_row = l + xch[((pair_n & 1) * 2 + (half ^ 1)) * kBM + row];
     }
     const bool write = row_valid && have_l && (n_t == 0 || have_o);
     const int64_t grow = static_cast<int64_t>(bh) * prm.S +
@@ -696,8 +723,9 @@ static cudaError_t launch_fwd_t(const CUtensorMap& q, const CUtensorMap& k, cons
 
 cudaError_t launch_bsa_fwd(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
                            const int32_t* row_ptr, const int32_t* col_idx, void* o, float* lse,
-                           int* status, int BH, int H, int S, int d, float scale, int raster,
-                           int Th, int Tw, uint64_t wait_limit_ns, cudaStream_t st) {
+                           int* status, int* redo, int* exact_passes, int exact_only, int BH,
+                           int H, int S, int d, float scale, int raster, int Th, int Tw,
+                           uint64_t wait_limit_ns, cudaStream_t st) {
   AttnParams prm;
   prm.row_ptr = row_ptr;
   prm.col_idx = col_idx;
@@ -712,14 +740,26 @@ cudaError_t launch_bsa_fwd(const CUtensorMap& q, const CUtensorMap& k, const CUt
   prm.Tw = Tw;
   prm.scale_log2 = scale * 1.4426950408889634f;
   prm.wait_limit_ns = wait_limit_ns;
+  prm.redo = redo;
+  prm.exact_passes = exact_passes;
   const int64_t nitems = static_cast<int64_t>(BH) * prm.ngroups;
   if (nitems == 0) return cudaSuccess;
-  if (raster) {
-    if (d == 128) return launch_fwd_t<128, true>(q, k, v, prm, nitems, st);
-    return launch_fwd_t<64, true>(q, k, v, prm, nitems, st);
+  // the fixed-reference pass, then the exact-reference pass, whose CTAs return
+  // at once unless the first pass set *redo (exact_only: the second pass alone)
+  cudaError_t e = cudaMemsetAsync(redo, exact_only ? 1 : 0, sizeof(int), st);
+  if (e != cudaSuccess) return e;
+  for (int exact = exact_only ? 1 : 0; exact < 2; ++exact) {
+    prm.exact = exact;
+    if (raster) {
+      e = d == 128 ? launch_fwd_t<128, true>(q, k, v, prm, nitems, st)
+                   : launch_fwd_t<64, true>(q, k, v, prm, nitems, st);
+    } else {
+      e = d == 128 ? launch_fwd_t<128, false>(q, k, v, prm, nitems, st)
+                   : launch_fwd_t<64, false>(q, k, v, prm, nitems, st);
+    }
+    if (e != cudaSuccess) return e;
   }
-  if (d == 128) return launch_fwd_t<128, false>(q, k, v, prm, nitems, st);
-  return launch_fwd_t<64, false>(q, k, v, prm, nitems, st);
+  return cudaSuccess;
 }
 
 cudaError_t launch_mma_selftest(const CUtensorMap& a, const CUtensorMap& b, const void* a_glob,

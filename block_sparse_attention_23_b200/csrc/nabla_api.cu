@@ -33,8 +33,9 @@ cudaError_t launch_scan_fill(const uint32_t* bits, const int32_t* counts, int64_
                              int32_t* nnz_out, int* status, cudaStream_t st);
 cudaError_t launch_bsa_fwd(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
                            const int32_t* row_ptr, const int32_t* col_idx, void* o, float* lse,
-                           int* status, int BH, int H, int S, int d, float scale, int raster,
-                           int Th, int Tw, uint64_t wait_limit_ns, cudaStream_t st);
+                           int* status, int* redo, int* exact_passes, int exact_only, int BH,
+                           int H, int S, int d, float scale, int raster, int Th, int Tw,
+                           uint64_t wait_limit_ns, cudaStream_t st);
 cudaError_t launch_reorder(const void* src, void* dst, int64_t BH, int Tt, int Th, int Tw,
                            int row_bytes, int to_tile_major, cudaStream_t st);
 cudaError_t launch_block_energy(const CUtensorMap& q, const CUtensorMap& k, const int32_t* row_ptr,
@@ -72,12 +73,18 @@ struct CallRange {
   ~CallRange() { nvtxRangePop(); }
 };
 
+// Workspace header (256 bytes, zeroed by nabla_workspace_init): int32 words
+// [0] status bits, [1] the forward's exact-pass request, [2] exact passes run
+// (a counter), [4 + slot] the exact-pass requests of the host-buffer layer's
+// two slots.
 constexpr size_t kHeaderBytes = 256;
+constexpr int kHdrRedo = 1, kHdrExactPasses = 2;
 constexpr uint64_t kDefaultWaitLimitNs = 2000000000ull;   // 2 s
 constexpr int kMaxNbSupported = 4096;
 
 thread_local std::string g_last_error;
 std::atomic<uint64_t> g_wait_limit_ns{kDefaultWaitLimitNs};
+std::atomic<int> g_exact_reference{0};
 
 nabla_status fail(nabla_status s, const std::string& msg) {
   g_last_error = msg;
@@ -263,7 +270,7 @@ int* status_ptr(void* ws) { return static_cast<int*>(ws); }
 
 nabla_status run_fwd(const nabla_shape* shape, const void* q, const void* k, const void* v,
                      const int32_t* row_ptr, const int32_t* col_idx, float scale, void* o,
-                     float* lse, void* workspace, cudaStream_t st) {
+                     float* lse, int* header, int* redo, cudaStream_t st) {
   const uint64_t rows = static_cast<uint64_t>(shape->B) * shape->H * shape->S;
   const bool raster = shape->layout == NABLA_LAYOUT_RASTER;
   CUtensorMap mq, mk, mv;
@@ -278,8 +285,9 @@ nabla_status run_fwd(const nabla_shape* shape, const void* q, const void* k, con
     if ((s = make_map(&mv, v, rows, shape->d)) != NABLA_OK) return s;
   }
   if (!(scale > 0.f)) scale = 1.0f / std::sqrt(static_cast<float>(shape->d));
-  cudaError_t e = nabla::launch_bsa_fwd(mq, mk, mv, row_ptr, col_idx, o, lse,
-                                        status_ptr(workspace), shape->B * shape->H, shape->H,
+  cudaError_t e = nabla::launch_bsa_fwd(mq, mk, mv, row_ptr, col_idx, o, lse, header, redo,
+                                        header + kHdrExactPasses, g_exact_reference.load(),
+                                        shape->B * shape->H, shape->H,
                                         shape->S, shape->d, scale, raster ? 1 : 0, shape->Th,
                                         shape->Tw, g_wait_limit_ns.load(), st);
   if (e != cudaSuccess) return cuda_fail(e, "bsa_fwd launch");
@@ -291,6 +299,16 @@ nabla_status run_fwd(const nabla_shape* shape, const void* q, const void* k, con
 namespace nabla {
 // Lets other translation units of the library report through nabla_last_error().
 void set_last_error(const std::string& msg) { g_last_error = msg; }
+// bsa_fwd with an explicit header (status word, exact-pass counter) and
+// exact-pass request word, for callers that run several forwards at once on
+// one header (arguments already checked).
+nabla_status fwd_with_header(const nabla_shape* shape, const void* q, const void* k,
+                             const void* v, const int32_t* row_ptr, const int32_t* col_idx,
+                             float scale, void* o, float* lse, int* header, int* redo,
+                             nabla_stream_t stream) {
+  return run_fwd(shape, q, k, v, row_ptr, col_idx, scale, o, lse, header, redo,
+                 reinterpret_cast<cudaStream_t>(stream));
+}
 // nabla_build_mask with its device status bits OR-ed into `status` instead of
 // the workspace header (the host-buffer layer shares one header between the
 // chunks it runs on two streams).
@@ -303,12 +321,31 @@ nabla_status build_mask_with_status(const nabla_shape* shape, const nabla_mask_p
 
 extern "C" {
 
-int nabla_version(void) { return 220; }
+int nabla_version(void) { return 230; }
 
 const char* nabla_last_error(void) { return g_last_error.c_str(); }
 
 void nabla_set_wait_limit_ns(uint64_t ns) {
   g_wait_limit_ns.store(ns == 0 ? kDefaultWaitLimitNs : ns);
+}
+
+void nabla_set_exact_reference(int on) { g_exact_reference.store(on ? 1 : 0); }
+
+int nabla_query_exact_passes(const void* workspace, nabla_stream_t stream) {
+  if (workspace == nullptr) {
+    g_last_error = "workspace is NULL";
+    return -1;
+  }
+  int n = 0;
+  cudaError_t e = cudaMemcpyAsync(&n, static_cast<const int*>(workspace) + kHdrExactPasses,
+                                  sizeof(int), cudaMemcpyDeviceToHost,
+                                  reinterpret_cast<cudaStream_t>(stream));
+  if (e == cudaSuccess) e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) {
+    g_last_error = std::string("nabla_query_exact_passes: ") + cudaGetErrorString(e);
+    return -1;
+  }
+  return n;
 }
 
 size_t nabla_workspace_size(const nabla_shape* shape, int op) {
@@ -422,8 +459,8 @@ nabla_status bsa_fwd(const nabla_shape* shape, const void* q, const void* k, con
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
     return fail(NABLA_ERR_INVALID_ARG, "q, k, v, o must be 16-byte aligned");
   if (!std::isfinite(scale)) return fail(NABLA_ERR_INVALID_ARG, "scale must be finite");
-  return run_fwd(shape, q, k, v, row_ptr, col_idx, scale, o, lse, workspace,
-                 reinterpret_cast<cudaStream_t>(stream));
+  return run_fwd(shape, q, k, v, row_ptr, col_idx, scale, o, lse, status_ptr(workspace),
+                 status_ptr(workspace) + kHdrRedo, reinterpret_cast<cudaStream_t>(stream));
 }
 
 nabla_status bsa_fwd_with_mask(const nabla_shape* shape, const void* q, const void* k,
@@ -453,7 +490,8 @@ nabla_status bsa_fwd_with_mask(const nabla_shape* shape, const void* q, const vo
   e = nabla::launch_scan_fill(bits, counts, nrows, nb, row_ptr, col_idx, cap, nullptr,
                               status_ptr(workspace), st);
   if (e != cudaSuccess) return cuda_fail(e, "scan/fill launch");
-  return run_fwd(shape, q, k, v, row_ptr, col_idx, scale, o, lse, workspace, st);
+  return run_fwd(shape, q, k, v, row_ptr, col_idx, scale, o, lse, status_ptr(workspace),
+                 status_ptr(workspace) + kHdrRedo, st);
 }
 
 nabla_status nabla_reorder_tokens(const nabla_shape* shape, int direction, const void* src,

@@ -3,12 +3,13 @@
 // independent, so the layer runs in chunks of heads through a two-slot device
 // pipeline: the host-to-device copies of chunk c+1 and the device-to-host
 // copies of chunk c-1 run on their own streams while chunk c computes, and
-// PCIe transfers hide behind the attention instead of adding to it.  Chunks of
-// slot 0 compute on the caller's stream and chunks of slot 1 on a second
-// compute stream, so one chunk's kernels start on the SMs that the previous
-// chunk's last wave leaves idle.  Plain cudaMemcpyAsync copies only; stream
-// order is kept with events, and the caller's stream waits for the last output
-// copies before the call's work is complete on it.
+// PCIe transfers hide behind the attention instead of adding to it.  Every
+// chunk computes on the caller's stream, one after another: a second compute
+// stream let one chunk's forward kernels queue behind the other chunk's whole
+// grid (each attention CTA holds most of an SM's shared memory), which
+// delayed the output copies and the next inputs.  Plain cudaMemcpyAsync
+// copies only; stream order is kept with events, and the caller's stream
+// waits for the last output copies before the call's work is complete on it.
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -26,6 +27,10 @@ nabla_status build_mask_with_status(const nabla_shape* shape, const nabla_mask_p
                                     int32_t* row_ptr, int32_t* col_idx, int64_t col_capacity,
                                     int32_t* nnz_out, void* workspace, int* status,
                                     nabla_stream_t stream);
+nabla_status fwd_with_header(const nabla_shape* shape, const void* q, const void* k,
+                             const void* v, const int32_t* row_ptr, const int32_t* col_idx,
+                             float scale, void* o, float* lse, int* header, int* redo,
+                             nabla_stream_t stream);
 }  // namespace nabla
 
 namespace {
@@ -102,15 +107,15 @@ std::vector<int> chunk_schedule(int64_t heads, int max_heads) {
 
 // Streams and events reused across calls (one set per device, created once).
 struct PipeRes {
-  cudaStream_t h2d = nullptr, d2h = nullptr, comp = nullptr;
+  cudaStream_t h2d = nullptr, d2h = nullptr;
   cudaEvent_t in_ready[kSlots] = {}, in_free[kSlots] = {}, out_ready[kSlots] = {},
               out_free[kSlots] = {};
-  cudaEvent_t join[3] = {};   // a failed call: the caller's stream waits for every stream
+  cudaEvent_t join[2] = {};   // a failed call: the caller's stream waits for the copy streams
   bool ok = false;
 };
 
 void release(PipeRes& r) {
-  for (cudaStream_t* p : {&r.h2d, &r.d2h, &r.comp})
+  for (cudaStream_t* p : {&r.h2d, &r.d2h})
     if (*p) { cudaStreamDestroy(*p); *p = nullptr; }
   for (int i = 0; i < kSlots; ++i)
     for (cudaEvent_t* p : {&r.in_ready[i], &r.in_free[i], &r.out_ready[i], &r.out_free[i]})
@@ -132,14 +137,13 @@ nabla_status resources(PipeRes** out) {
   if (!r.ok) {
     e = cudaStreamCreateWithFlags(&r.h2d, cudaStreamNonBlocking);
     if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&r.d2h, cudaStreamNonBlocking);
-    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&r.comp, cudaStreamNonBlocking);
     for (int i = 0; i < kSlots && e == cudaSuccess; ++i) {
       e = cudaEventCreateWithFlags(&r.in_ready[i], cudaEventDisableTiming);
       if (e == cudaSuccess) e = cudaEventCreateWithFlags(&r.in_free[i], cudaEventDisableTiming);
       if (e == cudaSuccess) e = cudaEventCreateWithFlags(&r.out_ready[i], cudaEventDisableTiming);
       if (e == cudaSuccess) e = cudaEventCreateWithFlags(&r.out_free[i], cudaEventDisableTiming);
     }
-    for (int i = 0; i < 3 && e == cudaSuccess; ++i)
+    for (int i = 0; i < 2 && e == cudaSuccess; ++i)
       e = cudaEventCreateWithFlags(&r.join[i], cudaEventDisableTiming);
     if (e != cudaSuccess) {
       release(r);
@@ -206,21 +210,19 @@ NABLA_API nabla_status nabla_layer_host(const nabla_shape* shape, const nabla_ma
   int* status = reinterpret_cast<int*>(ws);
   const std::vector<int> sizes = chunk_schedule(BH, hc);
   const int64_t nchunks = static_cast<int64_t>(sizes.size());
-  cudaStream_t comp[kSlots] = {st, r->comp};
   // the other streams start after the work already queued on the caller's stream
   cudaEvent_t start = r->out_free[0];
   cudaError_t e;
   if ((e = cudaEventRecord(start, st)) != cudaSuccess ||
       (e = cudaStreamWaitEvent(r->h2d, start, 0)) != cudaSuccess ||
-      (e = cudaStreamWaitEvent(r->d2h, start, 0)) != cudaSuccess ||
-      (e = cudaStreamWaitEvent(r->comp, start, 0)) != cudaSuccess)
+      (e = cudaStreamWaitEvent(r->d2h, start, 0)) != cudaSuccess)
     return cuda_fail(e, "pipeline start");
   const nabla_status result = [&]() -> nabla_status {
   int64_t h0 = 0;
   for (int64_t c = 0; c < nchunks; h0 += sizes[c], ++c) {
     const int slot = static_cast<int>(c % kSlots);
     const int h = sizes[c];
-    cudaStream_t cs = comp[slot];
+    cudaStream_t cs = st;
     const size_t tbytes = static_cast<size_t>(h) * shape->S * shape->d * 2;
     const size_t lbytes = static_cast<size_t>(h) * shape->S * 4;
     const size_t toff = static_cast<size_t>(h0) * shape->S * shape->d * 2;
@@ -257,8 +259,10 @@ NABLA_API nabla_status nabla_layer_host(const nabla_shape* shape, const nabla_ma
     s = nabla::build_mask_with_status(&chunk, params, dq, dk, nullptr, row_ptr, col_idx, lay.cap,
                                       nullptr, sb + lay.build, status, ns);
     if (s != NABLA_OK) return s;
-    // the forward's workspace is the status header alone
-    s = bsa_fwd(&chunk, dq, dk, dv, row_ptr, col_idx, 0.f, dout, dlse, ws, ns);
+    // the forward reports into the shared header, with the slot's own
+    // exact-pass request word (header word 4 + slot)
+    s = nabla::fwd_with_header(&chunk, dq, dk, dv, row_ptr, col_idx, 0.f, dout, dlse, status,
+                               status + 4 + slot, ns);
     if (s != NABLA_OK) return s;
     if ((e = cudaEventRecord(r->in_free[slot], cs)) != cudaSuccess ||
         (e = cudaEventRecord(r->out_ready[slot], cs)) != cudaSuccess)
@@ -273,7 +277,7 @@ NABLA_API nabla_status nabla_layer_host(const nabla_shape* shape, const nabla_ma
       return cuda_fail(e, "d2h copy");
   }
   // the call is complete on the caller's stream once the last outputs landed
-  // (each output copy follows its chunk's compute, on either compute stream)
+  // (each output copy follows its chunk's compute)
   for (int i = 0; i < kSlots && i < nchunks; ++i)
     if ((e = cudaStreamWaitEvent(st, r->out_free[i], 0)) != cudaSuccess)
       return cuda_fail(e, "final wait");
@@ -282,8 +286,8 @@ NABLA_API nabla_status nabla_layer_host(const nabla_shape* shape, const nabla_ma
   if (result != NABLA_OK) {
     // whatever was queued before the failure is ordered before later work on
     // the caller's stream, so the caller's buffers are not in use once it syncs
-    const cudaStream_t others[3] = {r->h2d, r->comp, r->d2h};
-    for (int i = 0; i < 3; ++i)
+    const cudaStream_t others[2] = {r->h2d, r->d2h};
+    for (int i = 0; i < 2; ++i)
       if (cudaEventRecord(r->join[i], others[i]) == cudaSuccess)
         cudaStreamWaitEvent(st, r->join[i], 0);
   }

@@ -143,6 +143,15 @@ NABLA_API nabla_status nabla_build_mask(const nabla_shape* shape, const nabla_ma
  * A query block with an empty list gets O = 0 and LSE = -inf.  Duplicate
  * column indices count once; indices outside [0, nb) are skipped and recorded
  * as NABLA_ERR_BAD_INDEX.
+ * The call runs two kernels.  The first takes, per row, the max of the first
+ * key tile the row's block lists as the softmax reference and keeps it; if a
+ * later tile's scores exceed that reference by more than 16 in log2 units
+ * (a tile's partial row sum above 2^16), it sets word 1 of the workspace
+ * header, and the second kernel recomputes the whole call with the reference
+ * raised as the scores grow (otherwise its blocks return at once).  Word 2
+ * of the header counts the recomputations (nabla_query_exact_passes); the
+ * result does not depend on which kernel produced it beyond rounding.  One
+ * workspace must not serve two calls that may run at the same time.
  */
 NABLA_API nabla_status bsa_fwd(const nabla_shape* shape, const void* q, const void* k, const void* v,
                      const int32_t* row_ptr, const int32_t* col_idx, float scale, void* o,
@@ -370,6 +379,15 @@ NABLA_API int nabla_version(void);
  * memory, record NABLA_ERR_TIMEOUT and return.  Tests set a tiny limit to
  * check that path without hanging anything.
  *
+ * nabla_set_exact_reference: 1 makes every forward run only its second,
+ * exact-reference kernel (the reference raised as each row's scores grow);
+ * 0 (the default) restores the two-kernel scheme described at bsa_fwd.
+ * Process-wide; for tests and for reproducing the exact-reference numerics.
+ *
+ * nabla_query_exact_passes: synchronises the stream and returns word 2 of a
+ * forward workspace's header: how many forwards on it needed the
+ * exact-reference kernel since nabla_workspace_init (-1 on a CUDA error).
+ *
  * nabla_selftest_mma: one 128 x N x 128 bf16 product through the same
  * tcgen05/TMA building blocks the attention kernel uses, for layout checks.
  *   variant 0: C[m][n] = sum_k A[m][k] B[n][k]   (both K-major, N = 128)
@@ -379,6 +397,8 @@ NABLA_API int nabla_version(void);
  *   a, b: device bf16 [128][128] row-major; c: device fp32 [128][128].
  */
 NABLA_API void nabla_set_wait_limit_ns(uint64_t ns);
+NABLA_API void nabla_set_exact_reference(int on);
+NABLA_API int nabla_query_exact_passes(const void* workspace, nabla_stream_t stream);
 NABLA_API nabla_status nabla_selftest_mma(int variant, const void* a, const void* b, float* c,
                                 void* workspace, nabla_stream_t stream);
 

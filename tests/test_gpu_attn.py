@@ -23,23 +23,34 @@ def _gather(o, lse, rows, S):
     return o[rows], lse[rows]
 
 
-def _nabla_layer(nl, w, q, k, v, thr=None, sta="cfg"):
+def _nabla_layer(nl, w, q, k, v, thr=None, sta="cfg", exact=False, passes=None):
+    """Mask + forward.  exact: run only the exact-reference kernel; passes: the
+    number of exact-reference recomputations the call must report."""
     thr = w.thr if thr is None else thr
     sta = w.sta if sta == "cfg" else sta
     qd, kd, vd = to_device_bf16(q), to_device_bf16(k), to_device_bf16(v)
     row_ptr, col_idx, nnz, mask = nl.nabla_build_mask(qd, kd, w.tile_grid, thr, sta,
                                                       want_mask=True)
     ws = nl.Workspace.create(nl.make_shape(w.B, w.H, w.S, w.d), nl.OP_FWD)
-    o, lse = nl.bsa_fwd(qd, kd, vd, row_ptr, col_idx, workspace=ws)
-    assert ws.query_status() == 0
+    nl.set_exact_reference(exact)
+    try:
+        o, lse = nl.bsa_fwd(qd, kd, vd, row_ptr, col_idx, workspace=ws)
+        assert ws.query_status() == 0
+    finally:
+        nl.set_exact_reference(False)
+    if passes is not None:
+        assert ws.exact_passes() == passes
     return o, lse, mask.cpu().numpy()
 
 
+@pytest.mark.parametrize("exact", [False, True], ids=["fixed-ref", "exact-ref"])
 @pytest.mark.parametrize("name", ["tiny", "small"])
-def test_attention_parity_all_rows(nl, oracle_mod, synth_mod, name):
+def test_attention_parity_all_rows(nl, oracle_mod, synth_mod, name, exact):
+    """Both forward kernels on the same inputs: the fixed-reference one (no
+    recomputation needed here) and the exact-reference one alone."""
     w = synth_mod.WORKLOADS[name]
     q, k, v = synth_mod.make_qkv(w)
-    o, lse, gmask = _nabla_layer(nl, w, q, k, v)
+    o, lse, gmask = _nabla_layer(nl, w, q, k, v, exact=exact, passes=1 if exact else 0)
     mask = oracle_mod.build_mask(q, k, w.tile_grid, w.thr, w.sta)
     rows = rows_with_same_mask(np.arange(w.B * w.H * w.S, dtype=np.int64), gmask, mask, w.S)
     ro, rl = oracle_mod.masked_attention(q, k, v, mask, rows)
@@ -52,7 +63,8 @@ def test_attention_parity_all_rows(nl, oracle_mod, synth_mod, name):
 def test_attention_parity_full_size(nl, oracle_mod, synth_mod, name):
     w = synth_mod.WORKLOADS[name]
     q, k, v = synth_mod.make_qkv(w)
-    o, lse, gmask = _nabla_layer(nl, w, q, k, v)
+    # the Wan-shaped layer runs on the fixed-reference kernel alone
+    o, lse, gmask = _nabla_layer(nl, w, q, k, v, passes=0 if name == "wan720p" else None)
     mask = oracle_mod.build_mask(q, k, w.tile_grid, w.thr, w.sta)
     rows = rows_with_same_mask(sample_rows(w.B, w.H, w.S, 2, 8, seed=1), gmask, mask, w.S)
     ro, rl = oracle_mod.masked_attention(q, k, v, mask, rows)

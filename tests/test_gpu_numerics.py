@@ -1,7 +1,8 @@
 """Numerical edge cases on the GPU vs the fp64 oracle: logits that rise
-steeply from key tile to key tile (every later tile's maximum exceeds the
-running maximum by more than 2^8, so the forward's lazy rescale of O and l
-runs on most tiles), all-equal scores, and thr = 1 (one block per row)."""
+steeply from key tile to key tile (later tiles exceed the first tile's
+reference by far more than 2^16, so the forward's exact-reference kernel
+recomputes the call, raising the reference and rescaling O and l on most
+tiles), all-equal scores, and thr = 1 (one block per row)."""
 import numpy as np
 import pytest
 
@@ -52,6 +53,8 @@ def test_forward_lazy_rescale_path(nl, oracle_mod, d, nb, order):
     ws = nl.Workspace.create(nl.make_shape(B, H, 64 * nb, d), nl.OP_FWD_WITH_MASK)
     o, lse = nl.bsa_fwd_with_mask(qd, kd, vd, torch.from_numpy(mask).cuda(), workspace=ws)
     assert ws.query_status() == 0
+    if order == "ascending":   # later keys outgrow the first tile's reference
+        assert ws.exact_passes() == 1
     rows = np.arange(B * H * 64 * nb, dtype=np.int64)
     ro, rl = oracle_mod.masked_attention(q, k, v, mask, rows)
     compare_attention(o.float().cpu().numpy().reshape(-1, d), lse.cpu().numpy().reshape(-1), ro, rl)
