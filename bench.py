@@ -604,7 +604,8 @@ def run_ours(args):
                         "block list, outside the step; FLOPs = 10*d*64*64 per kept block"},
         "raster_layer": {"ms_per_layer": raster_ms, "vs_tile_major": raster_ms / ms_per_step,
                          "what": "mask + attention on raster-ordered Q, K, V (O, LSE raster), "
-                                 "token reorder fused into the loads; outside the step"},
+                                 "Q read by 5D boxes, K and V reordered to tile-major copies in the "
+                                 "workspace first; outside the step"},
         "gpu_launches": 7 * args.steps,
         "clocks": clk,
     }

@@ -42,10 +42,13 @@
 // tensor rate (an N = 128 product with both operands in shared memory does
 // not), and the per-tile softmax overhead is spread over 256 keys.
 //
-// Token order: tile-major tensors are read as 2D boxes; raster-ordered ones
+// Token order: tile-major tensors are read as 2D boxes; a raster-ordered Q
 // (token (t,h,w) at (t*H + h)*W + w) as 5D boxes that gather one 4x4x4 tile,
-// so the reorder to tile-major happens inside the TMA loads, and O / LSE rows
-// are stored back at their raster positions.
+// so its reorder to tile-major happens inside the TMA loads, and O / LSE rows
+// are stored back at their raster positions.  Raster K and V, streamed once
+// per query tile, are read from tile-major copies when the caller's
+// workspace holds them (made by the token reorder before the launch), else
+// by 5D boxes as well (kv_raster).
 //
 // Online softmax with a reference maximum per row.  Each launch runs two
 // passes over the same grid.  The fixed-reference pass: the two warps of a
@@ -139,6 +142,7 @@ struct AttnParams {
   int* redo;               // set by a pass that needs the exact-reference pass (see below)
   int* exact_passes;       // counts the exact-reference passes that ran
   int exact;               // 0: reference fixed per row; 1: the exact-reference pass
+  int kv_raster;           // raster token order: K and V read by 5D boxes too (else 2D)
 };
 
 // One 64-token block of a [B,H,S,d] tensor as a 64 x 64 shared-memory box
@@ -321,6 +325,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 min(r0 + qb, nb - 1), prm.S, prm.Th, prm.Tw);
       }
       const int last = ulist[n_u - 1] & 0xFFFF;
+      const bool kv_raster = kRaster && prm.kv_raster;
       for (int t = 0; t < n_t; ++t) {
         if (t > 0 && !mbar_wait(bar(empty), (t - 1) & 1, lim, abort_flag)) {
           record_abort(abort_flag, prm.status, kStatusTimeout);
@@ -332,7 +337,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int u = tile_of(t);
           const int j = (kEntries * u + e < n_u) ? (ulist[kEntries * u + e] & 0xFFFF) : last;
           for (int h = 0; h < L::kDH; ++h)
-            load_block<kRaster>(buf + h * kBN * 128 + e * 64 * 128, map, bar(full), h, bh, j,
+            if (kv_raster)
+              load_block<true>(buf + h * kBN * 128 + e * 64 * 128, map, bar(full), h, bh, j,
+                               prm.S, prm.Th, prm.Tw);
+            else
+              load_block<false>(buf + h * kBN * 128 + e * 64 * 128, map, bar(full), h, bh, j,
                                 prm.S, prm.Th, prm.Tw);
         }
       }
@@ -724,8 +733,8 @@ static cudaError_t launch_fwd_t(const CUtensorMap& q, const CUtensorMap& k, cons
 cudaError_t launch_bsa_fwd(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
                            const int32_t* row_ptr, const int32_t* col_idx, void* o, float* lse,
                            int* status, int* redo, int* exact_passes, int exact_only, int BH,
-                           int H, int S, int d, float scale, int raster, int Th, int Tw,
-                           uint64_t wait_limit_ns, cudaStream_t st) {
+                           int H, int S, int d, float scale, int raster, int kv_raster, int Th,
+                           int Tw, uint64_t wait_limit_ns, cudaStream_t st) {
   AttnParams prm;
   prm.row_ptr = row_ptr;
   prm.col_idx = col_idx;
@@ -742,6 +751,7 @@ cudaError_t launch_bsa_fwd(const CUtensorMap& q, const CUtensorMap& k, const CUt
   prm.wait_limit_ns = wait_limit_ns;
   prm.redo = redo;
   prm.exact_passes = exact_passes;
+  prm.kv_raster = kv_raster;
   const int64_t nitems = static_cast<int64_t>(BH) * prm.ngroups;
   if (nitems == 0) return cudaSuccess;
   // the fixed-reference pass, then the exact-reference pass, whose CTAs return

@@ -34,8 +34,8 @@ cudaError_t launch_scan_fill(const uint32_t* bits, const int32_t* counts, int64_
 cudaError_t launch_bsa_fwd(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
                            const int32_t* row_ptr, const int32_t* col_idx, void* o, float* lse,
                            int* status, int* redo, int* exact_passes, int exact_only, int BH,
-                           int H, int S, int d, float scale, int raster, int Th, int Tw,
-                           uint64_t wait_limit_ns, cudaStream_t st);
+                           int H, int S, int d, float scale, int raster, int kv_raster, int Th,
+                           int Tw, uint64_t wait_limit_ns, cudaStream_t st);
 cudaError_t launch_reorder(const void* src, void* dst, int64_t BH, int Tt, int Th, int Tw,
                            int row_bytes, int to_tile_major, cudaStream_t st);
 cudaError_t launch_block_energy(const CUtensorMap& q, const CUtensorMap& k, const int32_t* row_ptr,
@@ -179,6 +179,17 @@ XattnLayout xattn_layout(const nabla_shape* s) {
   return l;
 }
 
+// One tile-major copy of K or V for a raster-ordered forward (256-aligned).
+size_t kv_copy_bytes(const nabla_shape* s) {
+  return align256(static_cast<size_t>(s->B) * s->H * s->S * s->d * 2);
+}
+
+// Bytes a forward needs after its other workspace contents: the tile-major
+// K and V copies for raster token order, nothing otherwise.
+size_t kv_scratch_bytes(const nabla_shape* s) {
+  return s->layout == NABLA_LAYOUT_RASTER ? 2 * kv_copy_bytes(s) : 0;
+}
+
 struct MaskLayout {
   size_t bits, counts, row_ptr, col_idx, total;
 };
@@ -268,17 +279,33 @@ nabla_status make_map_strided(CUtensorMap* map, const void* ptr, uint64_t groups
 
 int* status_ptr(void* ws) { return static_cast<int*>(ws); }
 
+// Raster token order: K and V are reordered into kv_scratch (2 tile-major
+// tensors) when the caller provides it, else read by 5D boxes in the kernel.
 nabla_status run_fwd(const nabla_shape* shape, const void* q, const void* k, const void* v,
                      const int32_t* row_ptr, const int32_t* col_idx, float scale, void* o,
-                     float* lse, int* header, int* redo, cudaStream_t st) {
+                     float* lse, int* header, int* redo, void* kv_scratch, cudaStream_t st) {
   const uint64_t rows = static_cast<uint64_t>(shape->B) * shape->H * shape->S;
   const bool raster = shape->layout == NABLA_LAYOUT_RASTER;
+  const bool kv_raster = raster && kv_scratch == nullptr;
   CUtensorMap mq, mk, mv;
   nabla_status s;
   if (raster) {
     if ((s = make_map_raster(&mq, q, shape)) != NABLA_OK) return s;
-    if ((s = make_map_raster(&mk, k, shape)) != NABLA_OK) return s;
-    if ((s = make_map_raster(&mv, v, shape)) != NABLA_OK) return s;
+    if (kv_raster) {
+      if ((s = make_map_raster(&mk, k, shape)) != NABLA_OK) return s;
+      if ((s = make_map_raster(&mv, v, shape)) != NABLA_OK) return s;
+    } else {
+      uint8_t* kt = static_cast<uint8_t*>(kv_scratch);
+      uint8_t* vt = kt + kv_copy_bytes(shape);
+      const int64_t BH = static_cast<int64_t>(shape->B) * shape->H;
+      cudaError_t e = nabla::launch_reorder(k, kt, BH, shape->Tt, shape->Th, shape->Tw,
+                                            shape->d * 2, 1, st);
+      if (e == cudaSuccess)
+        e = nabla::launch_reorder(v, vt, BH, shape->Tt, shape->Th, shape->Tw, shape->d * 2, 1, st);
+      if (e != cudaSuccess) return cuda_fail(e, "K/V reorder launch");
+      if ((s = make_map(&mk, kt, rows, shape->d)) != NABLA_OK) return s;
+      if ((s = make_map(&mv, vt, rows, shape->d)) != NABLA_OK) return s;
+    }
   } else {
     if ((s = make_map(&mq, q, rows, shape->d)) != NABLA_OK) return s;
     if ((s = make_map(&mk, k, rows, shape->d)) != NABLA_OK) return s;
@@ -288,8 +315,9 @@ nabla_status run_fwd(const nabla_shape* shape, const void* q, const void* k, con
   cudaError_t e = nabla::launch_bsa_fwd(mq, mk, mv, row_ptr, col_idx, o, lse, header, redo,
                                         header + kHdrExactPasses, g_exact_reference.load(),
                                         shape->B * shape->H, shape->H,
-                                        shape->S, shape->d, scale, raster ? 1 : 0, shape->Th,
-                                        shape->Tw, g_wait_limit_ns.load(), st);
+                                        shape->S, shape->d, scale, raster ? 1 : 0,
+                                        kv_raster ? 1 : 0, shape->Th, shape->Tw,
+                                        g_wait_limit_ns.load(), st);
   if (e != cudaSuccess) return cuda_fail(e, "bsa_fwd launch");
   return NABLA_OK;
 }
@@ -305,8 +333,16 @@ void set_last_error(const std::string& msg) { g_last_error = msg; }
 nabla_status fwd_with_header(const nabla_shape* shape, const void* q, const void* k,
                              const void* v, const int32_t* row_ptr, const int32_t* col_idx,
                              float scale, void* o, float* lse, int* header, int* redo,
-                             nabla_stream_t stream) {
-  return run_fwd(shape, q, k, v, row_ptr, col_idx, scale, o, lse, header, redo,
+                             void* kv_scratch, nabla_stream_t stream) {
+  nabla_status s = check_shape(shape);
+  if (s != NABLA_OK) return s;
+  if (!q || !k || !v || !row_ptr || !col_idx || !o || !header || !redo)
+    return fail(NABLA_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
+      (kv_scratch != nullptr && (reinterpret_cast<uintptr_t>(kv_scratch) & 255u)))
+    return fail(NABLA_ERR_INVALID_ARG, "q, k, v, o need 16-byte and K/V scratch 256-byte alignment");
+  if (!std::isfinite(scale)) return fail(NABLA_ERR_INVALID_ARG, "scale must be finite");
+  return run_fwd(shape, q, k, v, row_ptr, col_idx, scale, o, lse, header, redo, kv_scratch,
                  reinterpret_cast<cudaStream_t>(stream));
 }
 // nabla_build_mask with its device status bits OR-ed into `status` instead of
@@ -352,8 +388,8 @@ size_t nabla_workspace_size(const nabla_shape* shape, int op) {
   if (check_shape(shape) != NABLA_OK) return 0;
   switch (op) {
     case NABLA_OP_BUILD_MASK: return build_layout(shape).total;
-    case NABLA_OP_FWD: return kHeaderBytes;
-    case NABLA_OP_FWD_WITH_MASK: return mask_layout(shape).total;
+    case NABLA_OP_FWD: return kHeaderBytes + kv_scratch_bytes(shape);
+    case NABLA_OP_FWD_WITH_MASK: return mask_layout(shape).total + kv_scratch_bytes(shape);
     case NABLA_OP_BWD: return bwd_layout(shape).total;
     case NABLA_OP_BUILD_XATTN: return xattn_layout(shape).total;
     default: g_last_error = "unknown op"; return 0;
@@ -458,9 +494,14 @@ nabla_status bsa_fwd(const nabla_shape* shape, const void* q, const void* k, con
     return fail(NABLA_ERR_INVALID_ARG, "null pointer");
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
     return fail(NABLA_ERR_INVALID_ARG, "q, k, v, o must be 16-byte aligned");
+  if (shape->layout == NABLA_LAYOUT_RASTER && (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return fail(NABLA_ERR_INVALID_ARG, "a raster-order workspace needs 256-byte alignment");
   if (!std::isfinite(scale)) return fail(NABLA_ERR_INVALID_ARG, "scale must be finite");
+  void* kv_scratch = shape->layout == NABLA_LAYOUT_RASTER
+                         ? static_cast<uint8_t*>(workspace) + kHeaderBytes : nullptr;
   return run_fwd(shape, q, k, v, row_ptr, col_idx, scale, o, lse, status_ptr(workspace),
-                 status_ptr(workspace) + kHdrRedo, reinterpret_cast<cudaStream_t>(stream));
+                 status_ptr(workspace) + kHdrRedo, kv_scratch,
+                 reinterpret_cast<cudaStream_t>(stream));
 }
 
 nabla_status bsa_fwd_with_mask(const nabla_shape* shape, const void* q, const void* k,
@@ -490,8 +531,9 @@ nabla_status bsa_fwd_with_mask(const nabla_shape* shape, const void* q, const vo
   e = nabla::launch_scan_fill(bits, counts, nrows, nb, row_ptr, col_idx, cap, nullptr,
                               status_ptr(workspace), st);
   if (e != cudaSuccess) return cuda_fail(e, "scan/fill launch");
+  void* kv_scratch = shape->layout == NABLA_LAYOUT_RASTER ? ws + lay.total : nullptr;
   return run_fwd(shape, q, k, v, row_ptr, col_idx, scale, o, lse, status_ptr(workspace),
-                 status_ptr(workspace) + kHdrRedo, st);
+                 status_ptr(workspace) + kHdrRedo, kv_scratch, st);
 }
 
 nabla_status nabla_reorder_tokens(const nabla_shape* shape, int direction, const void* src,

@@ -35,6 +35,10 @@ cudaError_t launch_mask_bits(const uint8_t* mask, int64_t nrows, int nb, uint32_
 cudaError_t launch_scan_fill(const uint32_t* bits, const int32_t* counts, int64_t nrows, int nb,
                              int32_t* row_ptr, int32_t* col_idx, int64_t capacity,
                              int32_t* nnz_out, int* status, cudaStream_t st);
+nabla_status fwd_with_header(const nabla_shape* shape, const void* q, const void* k,
+                             const void* v, const int32_t* row_ptr, const int32_t* col_idx,
+                             float scale, void* o, float* lse, int* header, int* redo,
+                             void* kv_scratch, nabla_stream_t stream);
 }  // namespace nabla
 
 namespace {
@@ -124,8 +128,11 @@ NABLA_API nabla_status bsa_fwd_with_mask_static(const nabla_shape* shape, const 
                                 row_ptr, col_idx, static_cast<int64_t>(rows * nb), nullptr,
                                 reinterpret_cast<int*>(ws), st);
   if (e != cudaSuccess) return fail(NABLA_ERR_CUDA, std::string("mask compaction: ") + cudaGetErrorString(e));
-  s = bsa_fwd(shape, q, k, v, row_ptr, col_idx, scale, o, lse, ws, stream);
-  if (s != NABLA_OK) return s;   // bsa_fwd has set the message
+  // no room for tile-major K/V copies here: raster K and V are read by 5D boxes
+  s = nabla::fwd_with_header(shape, q, k, v, row_ptr, col_idx, scale, o, lse,
+                             reinterpret_cast<int*>(ws), reinterpret_cast<int*>(ws) + 1, nullptr,
+                             stream);
+  if (s != NABLA_OK) return s;   // the forward has set the message
   if (status_out != nullptr) {
     e = cudaMemcpyAsync(status_out, ws, sizeof(int32_t), cudaMemcpyDeviceToDevice, st);
     if (e != cudaSuccess) return fail(NABLA_ERR_CUDA, std::string("status copy: ") + cudaGetErrorString(e));

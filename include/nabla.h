@@ -139,7 +139,12 @@ NABLA_API nabla_status nabla_build_mask(const nabla_shape* shape, const nabla_ma
  *   scale         softmax scale; <= 0 selects 1/sqrt(d)
  *   o             device bf16 [B,H,S,d]
  *   lse           device fp32 [B,H,S] (may be NULL)
- *   workspace     device, nabla_workspace_size(shape, NABLA_OP_FWD) bytes
+ *   workspace     device, nabla_workspace_size(shape, NABLA_OP_FWD) bytes: the
+ *                 256-byte header for tile-major tokens; for raster token
+ *                 order (256-byte aligned) also tile-major copies of K and V
+ *                 (2 * B*H*S*d bf16), which the call fills with the token
+ *                 reorder before the attention kernels, so that only Q, O and
+ *                 LSE are addressed in raster order inside them
  * A query block with an empty list gets O = 0 and LSE = -inf.  Duplicate
  * column indices count once; indices outside [0, nb) are skipped and recorded
  * as NABLA_ERR_BAD_INDEX.
@@ -164,7 +169,9 @@ NABLA_API nabla_status bsa_fwd(const nabla_shape* shape, const void* q, const vo
  * "Inference": precomputed binary masks, only the selected blocks computed).
  *
  *   mask_u8       device uint8 [B,H,nb,nb]; nonzero = attend to the block
- *   workspace     device, nabla_workspace_size(shape, NABLA_OP_FWD_WITH_MASK)
+ *   workspace     device, nabla_workspace_size(shape, NABLA_OP_FWD_WITH_MASK),
+ *                 256-byte aligned (raster token order: with the K/V copies
+ *                 at its end, as for bsa_fwd)
  * Other arguments as for bsa_fwd.  The mask is compacted to block CSR inside
  * the workspace, then bsa_fwd runs on it.
  */
@@ -183,7 +190,8 @@ NABLA_API nabla_status bsa_fwd_with_mask(const nabla_shape* shape, const void* q
  * computes, but keeps the block CSR it builds from the mask in a fixed
  * device array owned by the library (NABLA_STATIC_SCRATCH_BYTES, 32 MiB, held
  * on each device that has used it until the process exits).  It allocates
- * nothing and takes no workspace.
+ * nothing and takes no workspace; with raster token order, K and V are read
+ * in place by 5D boxes (no tile-major copies), which is slower.
  *
  *   q, k, v, mask_u8, scale, o, lse   as for bsa_fwd_with_mask
  *   status_out   optional device int32 [1], or NULL: receives the call's

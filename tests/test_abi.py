@@ -51,6 +51,10 @@ def test_version_and_workspace_sizes(nl):
     n_build = nl.workspace_size(s, nl.OP_BUILD_MASK)
     n_mask = nl.workspace_size(s, nl.OP_FWD_WITH_MASK)
     assert n_fwd == 256
+    # raster token order: the header plus tile-major copies of K and V
+    r = nl.make_shape(1, 40, 76800, 128, (5, 12, 20), nl.LAYOUT_RASTER)
+    assert nl.workspace_size(r, nl.OP_FWD) == 256 + 2 * 40 * 76800 * 128 * 2
+    assert nl.workspace_size(r, nl.OP_FWD_WITH_MASK) == n_mask + 2 * 40 * 76800 * 128 * 2
     nb = 1200
     # pooled Q and K + reduced map + bitmap + counts
     assert n_build >= 2 * 40 * nb * 128 * 4 + 40 * nb * nb * 4

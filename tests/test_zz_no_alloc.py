@@ -71,3 +71,31 @@ def test_static_scratch_matches_workspace_entry_point_twice(nl, synth_mod):
         ref_o = o_w.double().cpu().numpy().reshape(-1, d)
         ref_l = lse_w.double().cpu().numpy().reshape(-1)
         compare_attention(go, gl, ref_o, ref_l)
+
+
+@pytest.mark.gpu
+def test_static_entry_raster_reads_kv_in_place(nl, synth_mod):
+    """Raster token order on the allocation-free entry point: with no room for
+    tile-major K/V copies, the kernel reads K and V through 5D boxes; the
+    result is bitwise the tile-major one, reordered."""
+    import torch
+    from test_gpu_raster import to_raster, to_tile_major
+    grid, B, H, d = (3, 2, 5), 1, 2, 128
+    S = 64 * 30
+    q16, k16, v16 = (synth_mod.make_tensor(i, 31, B, H, S, d, grid=grid) for i in range(3))
+    mask_np = synth_mod.make_bernoulli_mask(31, B * H, S // 64, 0.4).reshape(B, H, S // 64, S // 64)
+    mask = torch.from_numpy(mask_np).cuda()
+    q, k, v = (to_device_bf16(a) for a in (q16, k16, v16))
+    o_t, lse_t = nl.bsa_fwd_with_mask(q, k, v, mask, tile_grid=grid)
+    qr, kr, vr = (to_device_bf16(to_raster(a, grid)) for a in (q16, k16, v16))
+    shape = nl.make_shape(B, H, S, d, grid, nl.LAYOUT_RASTER)
+    o_r = torch.empty_like(qr)
+    lse_r = torch.empty((B, H, S), dtype=torch.float32, device=qr.device)
+    status = torch.full((1,), -1, dtype=torch.int32, device=qr.device)
+    _call_static(nl, shape, qr, kr, vr, mask, o_r, lse_r, status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    o_back = to_tile_major(o_r.view(torch.int16).cpu().numpy(), grid)
+    assert np.array_equal(o_back, o_t.view(torch.int16).cpu().numpy())
+    l_back = to_tile_major(lse_r.cpu().numpy()[..., None], grid)[..., 0]
+    assert np.array_equal(l_back, lse_t.cpu().numpy())
