@@ -195,6 +195,14 @@ class Workspace:
         return n
 
 
+def _check_workspace(workspace: Workspace, shape: _Shape, op: int) -> None:
+    """The library writes up to workspace_size(shape, op) bytes (raster token
+    order needs room for K/V copies): refuse a smaller buffer."""
+    need = workspace_size(shape, op)
+    if workspace.buf.numel() < need:
+        raise ValueError(f"workspace holds {workspace.buf.numel()} bytes; this call needs {need}")
+
+
 def _shape_of(q, tile_grid=(0, 0, 0), layout: int = LAYOUT_TILE_MAJOR) -> _Shape:
     if q.dim() != 4:
         raise ValueError("q must be [B, H, S, d]")
@@ -253,6 +261,7 @@ def bsa_fwd(q, k, v, row_ptr, col_idx, scale: Optional[float] = None,
     shape = _shape_of(q, tile_grid, layout)
     if workspace is None:
         workspace = Workspace.create(shape, OP_FWD, q.device, stream)
+    _check_workspace(workspace, shape, OP_FWD)
     if out is None:
         o = torch.empty_like(q)
         lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device)
@@ -275,6 +284,7 @@ def bsa_fwd_with_mask(q, k, v, mask_u8, scale: Optional[float] = None,
         raise ValueError("mask must be a contiguous uint8 CUDA tensor [B, H, nb, nb]")
     if workspace is None:
         workspace = Workspace.create(shape, OP_FWD_WITH_MASK, q.device, stream)
+    _check_workspace(workspace, shape, OP_FWD_WITH_MASK)
     if out is None:
         o = torch.empty_like(q)
         lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device)

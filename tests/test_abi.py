@@ -229,3 +229,16 @@ def test_layer_host_rejects_bad_mask_params_before_queuing(nl):
     no_grid = nl.make_shape(1, 4, 1024, 64, (4, 2, 3))
     ok = nl._MaskParams(0.2, 0, 0, 0, 0, 0)
     assert f(ctypes.byref(no_grid), ctypes.byref(ok), a, a, a, a, a, 2, a, null) == 1
+
+
+def test_forward_refuses_a_workspace_too_small_for_raster_order(nl):
+    """A raster-order forward writes tile-major K/V copies into its workspace:
+    the binding refuses a buffer sized for tile-major tokens before any device
+    call (the check bsa_fwd and bsa_fwd_with_mask run first)."""
+    import torch
+    shape = nl.make_shape(1, 2, 64 * 6, 64, (1, 2, 3), nl.LAYOUT_RASTER)
+    small = nl.Workspace(torch.empty(256, dtype=torch.uint8), nl.OP_FWD)
+    with pytest.raises(ValueError, match="workspace holds 256 bytes"):
+        nl._check_workspace(small, shape, nl.OP_FWD)
+    big = nl.Workspace(torch.empty(nl.workspace_size(shape, nl.OP_FWD), dtype=torch.uint8), nl.OP_FWD)
+    nl._check_workspace(big, shape, nl.OP_FWD)
