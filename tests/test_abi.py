@@ -242,3 +242,10 @@ def test_forward_refuses_a_workspace_too_small_for_raster_order(nl):
         nl._check_workspace(small, shape, nl.OP_FWD)
     big = nl.Workspace(torch.empty(nl.workspace_size(shape, nl.OP_FWD), dtype=torch.uint8), nl.OP_FWD)
     nl._check_workspace(big, shape, nl.OP_FWD)
+
+
+def test_exact_pass_counter_query_rejects_null(nl):
+    lib = nl.lib()
+    assert lib.nabla_query_exact_passes(None, None) == -1
+    assert "NULL" in lib.nabla_last_error().decode()
+    lib.nabla_set_exact_reference(0)          # the default; a no-op without a GPU
