@@ -7,8 +7,8 @@
 // With LSE from a dense forward pass, E is the true block-level attention map
 // (each row of E sums to 1).  It is the quantity two of the pages rank blocks
 // by: the "energy" (summed attention scores) per block that CalibAtt's offline
-// calibration thresholds ("Accelerating Video Diffusion with Calibrated Sparse
-// Attention", Methodology A), and the per-block true attention mass of the
+// calibration thresholds ("Accelerating Text-to-Video Generation with Calibrated
+// Sparse Attention", section 2 "Methodologie: CalibAtt", A "Offline Kalibratie"), and the per-block true attention mass of the
 // referee's fidelity check on NABLA's pooled proxy ("NABLA: Neighborhood
 // Adaptive Block-Level Attention", review, major comment 1).  block_mass[r],
 // the sum of E[r][c] over the listed c, is the fraction of the true mass that

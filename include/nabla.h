@@ -329,8 +329,8 @@ NABLA_API nabla_status nabla_reorder_tokens(const nabla_shape* shape, int direct
  * of c, averaged over the queries:
  *     E[r][c] = (1/64) sum_{i in r} sum_{j in c} exp(scale * q_i.k_j - lse_i)
  * This is the per-block "energy" that CalibAtt's offline calibration
- * thresholds ("Accelerating Video Diffusion with Calibrated Sparse Attention",
- * Methodology A) and the true block mass of the fidelity check the NABLA
+ * thresholds ("Accelerating Text-to-Video Generation with Calibrated Sparse
+ * Attention", section 2 "Methodologie: CalibAtt", A "Offline Kalibratie") and the true block mass of the fidelity check the NABLA
  * review asks for (major comment 1).  With lse from a dense bsa_fwd (every
  * block listed) each row of E sums to 1.
  *   q, k        device bf16 [B,H,S,d], 16-byte aligned (tile-major tokens)

@@ -289,8 +289,9 @@ void oracle_reorder(const uint16_t* src, uint16_t* dst, int64_t BH, int Tt, int 
                 }
 }
 
-/* Block attention energy ("Accelerating Video Diffusion with Calibrated
- * Sparse Attention", Methodology A: the energy, i.e. summed attention scores,
+/* Block attention energy ("Accelerating Text-to-Video Generation with
+ * Calibrated Sparse Attention", section 2 "Methodologie: CalibAtt", A "Offline
+ * Kalibratie": the energy, i.e. summed attention scores,
  * of each block; NABLA review, major comment 1: the true attention mass of an
  * N x N block).  For each listed (r, c):
  *   E[r][c] = (1/64) sum_{i in block r} sum_{j in block c} exp(scale q_i.k_j - lse_i)

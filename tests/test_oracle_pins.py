@@ -184,6 +184,99 @@ def test_row_select_monotone_in_thr(oracle_mod):
         assert counts[0] == 64 and counts[-1] == 1
 
 
+
+# ---------------------------------------------------------------- diagnostics and exemptions
+# The GPU/oracle mask comparison forgives a differing row only when the
+# oracle's own diagnostics put its cut inside the rounding band: E_{k*} or
+# E_{k*+1} within 1e-4 of 1 - thr ("near-cut"), or the probabilities at sorted
+# positions k* and k*+1 equal to 1e-6 relative ("near-tie").  These pins fix
+# what diag holds and what both predicates accept, on hand-built values.
+
+def test_row_select_diag_four_blocks(oracle_mod):
+    # p = (1, 8, 4, 3)/16, all exact in binary; sorted: 8/16 (block 1),
+    # 4/16 (block 2), 3/16 (block 3), 1/16 (block 0)
+    p = np.array([1.0, 8.0, 4.0, 3.0]) / 16.0
+    # thr 0.4: E_0 = 0 and E_1 = 1/2 lie below 0.6, E_2 = 3/4 does not -> k* = 1
+    keep, cnt, diag = oracle_mod.row_select(p, 0.4)
+    assert keep.tolist() == [0, 1, 1, 0] and cnt == 2
+    assert diag.tolist() == [0.5, 0.75, 0.25, 0.1875]
+    # thr 1: only the first sorted block (k = 0 rule) -> k* = 0
+    keep, cnt, diag = oracle_mod.row_select(p, 1.0)
+    assert keep.tolist() == [0, 1, 0, 0] and diag.tolist() == [0.0, 0.5, 0.5, 0.25]
+    # thr 0.01: every exclusive prefix (at most 15/16) stays below 0.99 -> all
+    # kept, k* = 3 is the last position and diag[3] = -1 (no k*+1)
+    keep, cnt, diag = oracle_mod.row_select(p, 0.01)
+    assert cnt == 4 and diag.tolist() == [0.9375, 1.0, 0.0625, -1.0]
+    # thr 0 keeps all by rule
+    keep, cnt, diag = oracle_mod.row_select(p, 0.0)
+    assert cnt == 4 and diag[3] == -1.0
+
+
+def _diag(e0, e1, a=0.3, b=0.1):
+    return np.array([e0, e1, a, b], dtype=np.float64)
+
+
+def test_near_cut_band_edges(oracle_mod):
+    nc = oracle_mod.near_cut_rows
+    t = 0.8                                               # thr 0.2
+    # E_{k*} just inside / just outside the band below the target
+    assert nc(_diag(t - 0.99e-4, 0.95), 0.2)
+    assert not nc(_diag(t - 1.01e-4, 0.95), 0.2)
+    # E_{k*+1} just inside / just outside above it
+    assert nc(_diag(0.5, t + 0.99e-4), 0.2)
+    assert not nc(_diag(0.5, t + 1.01e-4), 0.2)
+    # both far: no exemption
+    assert not nc(_diag(0.5, 0.95), 0.2)
+    # the target is 1 - thr, not thr
+    assert not nc(_diag(0.3, 0.9), 0.3) and nc(_diag(0.7 - 5e-5, 0.9), 0.3)
+    # the band is absolute mass: 0.9e-4 from the target is inside at target
+    # 0.8 and at 0.5 (a relative band would put it outside at both)
+    assert nc(_diag(0.8 - 0.9e-4, 0.95), 0.2) and nc(_diag(0.5 - 0.9e-4, 0.95), 0.5)
+    # a wider band is honoured
+    assert nc(_diag(t - 1.01e-4, 0.95), 0.2, band=1e-3)
+    # thr = 0 keeps every block: nothing is near a cut
+    assert not nc(_diag(1.0, 1.0), 0.0) and not nc(_diag(1.0 - 1e-9, 1.0), 0.0)
+    # shape: one flag per row, batched over leading axes
+    d = np.stack([_diag(t - 1e-5, 0.95), _diag(0.1, 0.95)] * 3).reshape(2, 3, 4)
+    got = nc(d, 0.2)
+    assert got.shape == (2, 3) and got.tolist() == [[True, False, True], [False, True, False]]
+
+
+def test_near_tie_band_edges(oracle_mod):
+    nt = oracle_mod.near_tie_rows
+    a = 0.25
+    assert nt(_diag(0, 0, a, a * (1 - 0.99e-6)))
+    assert not nt(_diag(0, 0, a, a * (1 - 1.01e-6)))
+    # relative, not absolute: 1e-8 vs 0.5e-8 differ by 5e-9 (under 1e-6
+    # absolute) but by half of themselves
+    assert not nt(_diag(0, 0, 1e-8, 0.5e-8))
+    assert nt(_diag(0, 0, 1e-8, 1e-8 * (1 - 0.5e-6)))
+    # no position k*+1 (every block kept): b = -1 never ties
+    assert not nt(_diag(0, 0, 0.5, -1.0)) and not nt(_diag(0, 0, 1e-300, -1.0))
+    # exact ties, including two zero probabilities
+    assert nt(_diag(0, 0, 0.125, 0.125)) and nt(_diag(0, 0, 0.0, 0.0))
+    got = nt(np.stack([_diag(0, 0, a, a), _diag(0, 0, a, 0.5 * a)]).reshape(1, 2, 4))
+    assert got.shape == (1, 2) and got.tolist() == [[True, False]]
+
+
+def test_exemptions_from_row_select_diagnostics(oracle_mod):
+    """The predicates applied to the oracle's own diagnostics of crafted rows."""
+    nc, nt = oracle_mod.near_cut_rows, oracle_mod.near_tie_rows
+    # thr 0.2 (target 0.8): sorted masses 0.5, 0.29995, 0.20005 -> E_2 = 0.79995
+    # stays below the target, k* = 2, E_{k*} 5e-5 from the target
+    keep, cnt, diag = oracle_mod.row_select(np.array([0.20005, 0.5, 0.29995]), 0.2)
+    assert cnt == 3 and nc(diag, 0.2) and not nt(diag)
+    # 0.29985: E_2 = 0.79985 is 1.5e-4 away and E_3 = 1 far: not near the cut
+    keep, cnt, diag = oracle_mod.row_select(np.array([0.20015, 0.5, 0.29985]), 0.2)
+    assert cnt == 3 and not nc(diag, 0.2)
+    # thr 0.4 (target 0.6): 0.4, 0.3 + e, 0.3 - e -> k* = 1; the cut separates
+    # 0.3 + e from 0.3 - e, a relative gap of 2e/0.3
+    for e, tie in [(1e-7, True), (2e-7, False)]:
+        keep, cnt, diag = oracle_mod.row_select(np.array([0.3 - e, 0.4, 0.3 + e]), 0.4)
+        assert keep.tolist() == [0, 1, 1] and not nc(diag, 0.4)
+        assert bool(nt(diag)) == tie
+
+
 # ---------------------------------------------------------------- STA window
 
 def _clipped(c, w, T):
