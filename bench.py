@@ -148,6 +148,36 @@ def _max_over_ranks(x: float, ws: int, device) -> float:
     return float(t.item())
 
 
+def _mask_kernel_rooflines(stage_ms, BH, nb, d, S, kept, peaks, fp64_peak):
+    """Per-kernel rooflines of the mask build from its stage times (ms):
+    pooling against HBM (Q, K read; fp64 block means written), the reduced map
+    against the measured fp64 FMA rate (2*nb^2*d per head), the selection
+    against HBM (the fp64 map read; bitmap and counts written), the compaction
+    against HBM (bitmap and counts read; row_ptr and col_idx written)."""
+    nw = (nb + 31) // 32
+    hbm = peaks["hbm_gbs"]
+    parts = {
+        "pool": ("hbm", 2.0 * BH * S * d * 2 + 2.0 * BH * nb * d * 8),
+        "reduced_map": ("fp64", 2.0 * BH * nb * nb * d),
+        "select": ("hbm", 8.0 * BH * nb * nb + 4.0 * BH * nb * nw + 4.0 * BH * nb),
+        "compact": ("hbm", 4.0 * BH * nb * nw + 8.0 * BH * nb + 4.0 * kept),
+    }
+    out = {}
+    for (name, (bound, work)), ms in zip(parts.items(), stage_ms):
+        if bound == "hbm":
+            ach = work / (ms * 1e-3) / 1e9
+            out[name] = {"bound": "hbm", "ms": float(ms), "bytes": work, "achieved": ach,
+                         "peak": hbm, "unit": "GB/s", "frac": ach / hbm}
+        else:
+            ach = work / (ms * 1e-3) / 1e12
+            out[name] = {"bound": "fp64", "ms": float(ms), "flops": work, "achieved": ach,
+                         "peak": fp64_peak, "unit": "TFLOP/s", "frac": ach / fp64_peak,
+                         "peak_source": "measured fp64 FMA chains (nabla_selftest_fp64_tflops)"}
+    out["what"] = ("the mask build's kernels timed one by one with events between them, "
+                   "outside the timed step")
+    return out
+
+
 # ------------------------------------------------------------------ CPU oracle
 def oracle_sample(w, q, k, v, nrows: int, head: int = 0, seed: int = 0):
     """Time the fp64 oracle on one head's full mask plus `nrows` sampled query
@@ -189,6 +219,46 @@ def executed_tile_products(row_ptr, col_idx, BH, nb):
             n_u = int(mem.sum())
             total += 2 * ((n_u + 3) // 4)
     return total
+
+
+def mask_parity_all_heads(w, q16, k16, gpu_row_ptr, gpu_col_idx):
+    """The timed layer's mask over every head against the oracle's: rows that
+    differ, and the oracle's near-cut rows (E_{k*} or E_{k*+1} within 1e-4 of
+    1 - thr) and near-tie rows (cut probabilities equal to 1e-6 relative), the
+    only rows allowed to differ."""
+    import oracle
+    t0 = time.perf_counter()
+    omask, diag, _ = oracle.build_mask(q16, k16, w.tile_grid, w.thr, w.sta, with_diag=True)
+    t_or = time.perf_counter() - t0
+    nb = w.nb
+    nrows = w.B * w.H * nb
+    rp = gpu_row_ptr[:nrows + 1].cpu().numpy()
+    ci = gpu_col_idx[:int(rp[-1])].cpu().numpy()
+    gmask = np.zeros((nrows, nb), dtype=np.uint8)
+    gmask[np.repeat(np.arange(nrows), np.diff(rp)), ci] = 1
+    o = omask.reshape(nrows, nb)
+    diff = (gmask != o).any(axis=1)
+    dg = diag.reshape(nrows, 4)
+    near_cut = oracle.near_cut_rows(dg, w.thr, 1e-4)
+    near_tie = oracle.near_tie_rows(dg)
+    exempt = near_cut | near_tie
+    return {"rows": nrows, "rows_differing": int(diff.sum()),
+            "rows_differing_not_exempt": int((diff & ~exempt).sum()),
+            "near_cut_rows": int(near_cut.sum()), "near_tie_rows": int(near_tie.sum()),
+            "oracle_mask_s": t_or,
+            "rule": "bit-exact except near-cut / near-tie rows of the oracle"}
+
+
+def sweep_executed_over_kept(mask):
+    """Executed / kept attention FLOPs of a static mask [B,H,nb,nb]: query
+    blocks in pairs, the union of their lists in 256-key tiles."""
+    BH, nb = int(np.prod(mask.shape[:-2])), mask.shape[-1]
+    m = mask.reshape(BH, nb, nb).astype(bool)
+    if nb % 2:
+        m = np.concatenate([m, np.zeros((BH, 1, nb), dtype=bool)], axis=1)
+    n_u = (m[:, 0::2] | m[:, 1::2]).sum(-1)
+    tiles = int(((n_u + 3) // 4).sum())
+    return 8.0 * tiles / max(int(mask.sum()), 1)
 
 
 def parity_sample(gpu_row_ptr, gpu_col_idx, gpu_o, gpu_lse, nb, d, sample):
@@ -336,6 +406,18 @@ def run_ours(args):
     ws_fwd.check()
     # forwards (check, warm-up, timed) that needed the exact-reference kernel
     fwd_exact_passes = ws_fwd.exact_passes()
+
+    # the mask build's four kernels timed one by one (events between them),
+    # outside the timed region, and the device's measured fp64 FMA rate
+    stage = np.zeros(4)
+    nl.nabla_build_mask_stage_ms(q, k, w.tile_grid, w.thr, w.sta, workspace=ws_mask, out=mask_out)
+    n_stage = 5
+    for _ in range(n_stage):
+        stage += np.array(nl.nabla_build_mask_stage_ms(q, k, w.tile_grid, w.thr, w.sta,
+                                                       workspace=ws_mask, out=mask_out))
+    stage /= n_stage
+    ws_mask.check()
+    fp64_peak = nl.selftest_fp64_tflops()
 
     # end to end through the public API with host buffers: nabla_layer_host
     # reads Q, K, V from pinned memory and writes O and LSE back to it every
@@ -534,8 +616,11 @@ def run_ours(args):
             wsw.check()
             ms_ = a.elapsed_time(b) / 3
             kept_s = int(mk.sum().item())
+            eok = sweep_executed_over_kept(mk.cpu().numpy())
+            kt = 4.0 * ws_.d * 64 * 64 * kept_s / (ms_ * 1e-3) / 1e12
             sweep.append({"density": pden, "kept_fraction": kept_s / mk.numel(), "ms": ms_,
-                          "kept_tflops": 4.0 * ws_.d * 64 * 64 * kept_s / (ms_ * 1e-3) / 1e12})
+                          "kept_tflops": kt, "kept_frac_of_sustained": kt / peaks["bf16_tflops_sustained"],
+                          "executed_over_kept": eok, "executed_tflops": kt * eok})
         del qs, ks, vs, os_, ls_
 
     attn_tflops = kept_flops / (attn_ms * 1e-3) / 1e12
@@ -553,7 +638,9 @@ def run_ours(args):
                    "parallelism": "replicas" if ws > 1 else "single GPU",
                    "l2": f"inputs (Q,K,V {3 * q.numel() * 2 / 1e9:.2f} GB per rank) larger than L2; no flush",
                    "kept_blocks": kept, "density": kept / (B * H * nb * nb),
-                   "mask_arith": "fp64", "attn_arith": "bf16 MMA, fp32 accumulate"},
+                   "mask_arith": "fp64 pooling, reduced map and row probabilities; exact "
+                                 "fixed-point prefix masses",
+                   "attn_arith": "bf16 MMA, fp32 accumulate"},
         "ms_per_layer": ms_per_step, "mask_ms": mask_ms, "attn_ms": attn_ms,
         "attn_kept_tflops": attn_tflops,
         "attn_executed": {"tile_products": exec_tiles, "flops": exec_flops,
@@ -575,6 +662,7 @@ def run_ours(args):
                           "peak": peaks["hbm_gbs"], "unit": "GB/s",
                           "frac": mask_bytes / (mask_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
                           "bytes": mask_bytes},
+        "mask_kernels": _mask_kernel_rooflines(stage, B * H, nb, d, S, kept, peaks, fp64_peak),
         "e2e": {"value": e2e_val, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
                 "call": "nabla_layer_host", "heads_per_chunk": hpc, "chunks": e2e_chunks},
@@ -618,6 +706,8 @@ def run_ours(args):
         line["cpu_baseline"] = {"value": val, "unit": "TFLOP/s", "cores": oracle.max_threads(),
                                 "kind": "oracle", "sample": desc}
         line["parity_sample"] = parity_sample(mask_out[0], mask_out[1], o, lse, nb, d, sample)
+        line["parity_sample"]["mask_all_heads"] = mask_parity_all_heads(w, q16, k16, mask_out[0],
+                                                                        mask_out[1])
     if rank == 0:
         print(json.dumps(line), flush=True)
     if ws > 1:

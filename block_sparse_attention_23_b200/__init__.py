@@ -35,7 +35,8 @@ EXPORTED = ["nabla_workspace_size", "nabla_workspace_init", "nabla_query_status"
             "bsa_fwd_with_mask_static", "nabla_reorder_tokens", "nabla_block_energy",
             "nabla_calib_accumulate", "nabla_calib_finalize", "bsa_bwd",
             "nabla_build_mask_xattn", "nabla_layer_host_workspace_size", "nabla_layer_host",
-            "nabla_layer_host_chunks", "nabla_set_exact_reference", "nabla_query_exact_passes"]
+            "nabla_layer_host_chunks", "nabla_set_exact_reference", "nabla_query_exact_passes",
+            "nabla_build_mask_stage_ms", "nabla_selftest_fp64_tflops"]
 TO_TILE_MAJOR, TO_RASTER = 0, 1
 
 
@@ -121,6 +122,11 @@ def lib() -> ctypes.CDLL:
             L.nabla_layer_host_workspace_size.argtypes = [sp, i32]
             L.nabla_layer_host_chunks.restype = ctypes.c_int64
             L.nabla_layer_host_chunks.argtypes = [ctypes.c_int64, i32, vp, ctypes.c_int64]
+            L.nabla_build_mask_stage_ms.restype = i32
+            L.nabla_build_mask_stage_ms.argtypes = [sp, ctypes.POINTER(_MaskParams), vp, vp, vp,
+                                                    vp, ctypes.c_int64, vp, vp, vp, vp]
+            L.nabla_selftest_fp64_tflops.restype = i32
+            L.nabla_selftest_fp64_tflops.argtypes = [vp, vp]
             L.nabla_layer_host.restype = i32
             L.nabla_layer_host.argtypes = [sp, ctypes.POINTER(_MaskParams), vp, vp, vp, vp, vp,
                                            i32, vp, vp]
@@ -249,6 +255,39 @@ def nabla_build_mask(q, k, tile_grid, thr: float, sta: Optional[Tuple[int, int, 
                                   _ptr(mask), _ptr(row_ptr), _ptr(col_idx), int(cap), _ptr(nnz),
                                   _ptr(workspace.buf), _stream(stream)))
     return row_ptr, col_idx, nnz, mask
+
+
+def nabla_build_mask_stage_ms(q, k, tile_grid, thr: float, sta=None, workspace=None, out=None,
+                              stream=None, topk: int = 0):
+    """Diagnostic: one mask build with events between its kernels.  Returns the
+    milliseconds of (pooling, reduced map, selection, compaction); synchronises."""
+    torch = _torch()
+    _bf16_contig(q, k)
+    shape = _shape_of(q, tile_grid, LAYOUT_TILE_MAJOR)
+    B, H, S, d = q.shape
+    nb = S // 64
+    if workspace is None:
+        workspace = Workspace.create(shape, OP_BUILD_MASK, q.device, stream)
+    if out is None:
+        out = (torch.empty(B * H * nb + 1, dtype=torch.int32, device=q.device),
+               torch.empty(B * H * nb * nb, dtype=torch.int32, device=q.device),
+               torch.empty(1, dtype=torch.int32, device=q.device), None)
+    row_ptr, col_idx, nnz = out[0], out[1], out[2]
+    prm = _MaskParams(float(thr), 1 if sta is not None else 0,
+                      *(sta if sta is not None else (0, 0, 0)), int(topk))
+    ms = (ctypes.c_float * 4)()
+    _check(lib().nabla_build_mask_stage_ms(ctypes.byref(shape), ctypes.byref(prm), _ptr(q),
+                                           _ptr(k), _ptr(row_ptr), _ptr(col_idx),
+                                           int(col_idx.numel()), _ptr(nnz), _ptr(workspace.buf),
+                                           _stream(stream), ms))
+    return tuple(float(x) for x in ms)
+
+
+def selftest_fp64_tflops(stream=None) -> float:
+    """Diagnostic: the device's measured fp64 FMA rate in TFLOP/s (synchronises)."""
+    out = ctypes.c_double(0.0)
+    _check(lib().nabla_selftest_fp64_tflops(_stream(stream), ctypes.byref(out)))
+    return float(out.value)
 
 
 def bsa_fwd(q, k, v, row_ptr, col_idx, scale: Optional[float] = None,

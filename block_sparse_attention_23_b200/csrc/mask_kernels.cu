@@ -11,21 +11,18 @@
 //   pool_kernel        Q, K bf16 [BH,S,d] -> Qbar, Kbar fp64 [BH,nb,d]     HBM-bound
 //                      (tile-major or raster token order)
 //   logits_kernel      per head Qbar Kbar^T / sqrt(d) -> L fp64 [BH,nb,nb] fp64 FMA
-//   select_kernel      one warp per row: softmax, prefix (or top-k) selection, STA OR ->
+//   select_kernel      one warp per row: fp64 softmax, prefix (or top-k) selection, STA OR ->
 //                      keep bitmap [BH*nb, nw] + counts (+ optional uint8 mask)
 //   mask_bits_kernel   external uint8 mask -> keep bitmap + counts
 //   scan_kernel        counts -> row_ptr (exclusive scan), nnz, capacity check
 //   fill_kernel        keep bitmap -> ascending col_idx per row
 //
-// The selection step does not sort.  The kept set of the sorted-prefix rule is
-// {p > v*} plus the first tied entries (by block index) of value v*, where v*
-// is the largest probability whose "mass at or above" reaches 1 - thr; v* is
-// found by bisection on the fp32 bit pattern (order-preserving for p >= 0).
-// That is the set a descending sort + cumulative sum selects, with the partial
-// sums taken in block order instead of sorted order.  Pooling and the reduced
-// map are fp64 (fp32 logits reorder blocks whose probabilities agree to a few
-// 1e-6, which moved cuts); the row softmax and the masses are fp32 values
-// from the fp64 map, summed in fp64 across each warp.
+// The selection step does not sort the row.  Pooling, the reduced map and the
+// row probabilities are fp64 (fp32 logits reorder blocks whose probabilities
+// agree to a few 1e-6, which moved cuts); the masses are exact fixed-point
+// integers of those probabilities, and the cut is located by value binning
+// down to at most 32 candidates, which are then ordered exactly (see the
+// selection section below).
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 #include <cstdint>
@@ -190,9 +187,52 @@ __global__ void __launch_bounds__(256) logits_kernel(const double* __restrict__ 
 }
 
 // ------------------------------------------------------------------ selection
+//
+// One CTA of 128 threads per row g = bh*nb + r.  The row's probabilities are formed in fp64
+// as the rule states them (p = exp(L - max) / sum over the row, or w / sum for
+// given non-negative weights) and kept in shared memory.  The kept set is the
+// smallest prefix of the row sorted by p descending (equal p: lower block index
+// first) whose exclusive prefix mass stays below 1 - thr, the first entry
+// always kept.  It is found without sorting the row:
+//   - masses are fixed-point integers F = round(p * 2^62), so every partial sum
+//     is exact and the same in any summation order;
+//   - the value range [lo, hi] of the candidates (at first the whole row) is
+//     split into 256 equal bins, a monotone map, so the bins are ordered
+//     intervals of p; the candidates' masses and counts are histogrammed with
+//     shared-memory integer atomics; a scan from the top bin finds the bin in
+//     which the cumulative mass reaches the target; entries of higher bins are
+//     kept, of lower bins dropped, and the crossing bin's entries are the next
+//     candidates (their range is the next level's [lo, hi]);
+//   - once at most 32 candidates remain one warp sorts them exactly on
+//     (p desc, block index asc) by a bitonic network, and each one's
+//     exclusive prefix mass decides it; candidates that all share one p are
+//     taken in block order.
+// Top-k mode does the same with a count of 1 per entry as the mass and k as
+// the target.  Everything is integer or exact comparison after p is formed,
+// so the kept set is the one a sort by p and an exact cumulative sum give.
 
-// Butterfly sums; lanes may differ in the last ulp (different association), so
-// lane 0's value is broadcast: every lane takes the same branch on it.
+constexpr int kSelBins = 256;
+constexpr double kSelFix = 4611686018427387904.0;   // 2^62, scale of the fixed-point masses
+constexpr int kSelMaxLevels = 16;                    // binning levels (8 always suffice for fp64)
+
+struct SelectParams {
+  float thr;
+  int use_sta, wt, wh, ww;
+  int Tt, Th, Tw;
+  int topk;        // > 0: keep the topk most probable blocks instead of the mass rule
+};
+
+// Shared memory of one row: p [nb] fp64, candidate list [nb] u16, keep bitmap
+// [nw] u32, bin masses [256] u64, bin counts [256] u32, and a small exchange
+// area for the CTA's reductions (8-byte aligned parts).
+constexpr int kSelThreads = 128, kSelWarps = kSelThreads / 32;
+constexpr size_t kSelXchBytes = 8 * 4 * kSelWarps + 64;
+__host__ __device__ inline size_t select_row_bytes(int nb) {
+  const size_t n = static_cast<size_t>(nb), nw = (n + 31) / 32;
+  return 8 * n + ((2 * n + 7) & ~static_cast<size_t>(7)) + 4 * ((nw + 1) & ~static_cast<size_t>(1)) +
+         12 * static_cast<size_t>(kSelBins) + kSelXchBytes;
+}
+
 __device__ __forceinline__ double warp_sum(double v) {
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
@@ -205,178 +245,337 @@ __device__ __forceinline__ double warp_max(double v) {
   return v;
 }
 
-__device__ __forceinline__ uint32_t warp_max_u32(uint32_t v) {
+__device__ __forceinline__ double warp_min(double v) {
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) v = max(v, __shfl_xor_sync(0xffffffffu, v, off));
+  for (int off = 16; off > 0; off >>= 1) v = fmin(v, __shfl_xor_sync(0xffffffffu, v, off));
   return v;
 }
 
-// Mass of the entries whose ordering key (fp32 bit pattern of p) is at least
-// v: fp32 sums per lane (at most 128 terms), fp64 across the warp.
-__device__ __forceinline__ double mass_at_or_above(const uint32_t* key, int nb, int lane,
-                                                   uint32_t v) {
-  float s = 0.f;
-  for (int c = lane; c < nb; c += 32) {
-    const uint32_t k = key[c];
-    s += (k >= v) ? __uint_as_float(k) : 0.f;
-  }
-  return warp_sum(static_cast<double>(s));
-}
-
-// Entries whose ordering key is at least v.
-__device__ __forceinline__ int count_at_or_above(const uint32_t* key, int nb, int lane, uint32_t v) {
-  int n = 0;
-  for (int c = lane; c < nb; c += 32) n += key[c] >= v;
+__device__ __forceinline__ unsigned long long warp_sum_u64(unsigned long long v) {
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) n += __shfl_xor_sync(0xffffffffu, n, off);
-  return n;
+  for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+  return v;
 }
 
-struct SelectParams {
-  float thr;
-  int use_sta, wt, wh, ww;
-  int Tt, Th, Tw;
-  int topk;        // > 0: keep the topk most probable blocks instead of the mass rule
-};
+// CTA-wide reductions in a fixed order (every thread gets the same value): the
+// warps reduce, warp w posts to slot w of xch, and every thread combines the
+// slots in warp order.  op 0: sum, 1: max, 2: min.
+template <int kOp>
+__device__ __forceinline__ double cta_reduce(double v, double* xch, int warp, int lane) {
+  v = kOp == 0 ? warp_sum(v) : (kOp == 1 ? warp_max(v) : warp_min(v));
+  if (lane == 0) xch[warp] = v;
+  __syncthreads();
+  double r = xch[0];
+#pragma unroll
+  for (int w = 1; w < kSelWarps; ++w) r = kOp == 0 ? r + xch[w] : (kOp == 1 ? fmax(r, xch[w]) : fmin(r, xch[w]));
+  __syncthreads();
+  return r;
+}
 
-// One warp per row g = bh*nb + r; `wpc` warps per CTA; shared memory: one
-// 32-bit key per entry.  The reduced map arrives in fp64.  p = exp(L - max) / Z
-// is formed in fp32 from the fp64 difference (a few ulp), and its fp32 bit
-// pattern is the ordering key (order-preserving for p >= 0); equal keys go by
-// block index.  Masses are summed from those fp32 values, fp64 across the warp.
-// Relative to the fp64 rule this can move the cut only for rows whose cut
-// mass is within a few 1e-6 of 1 - thr, or swap blocks whose probabilities
-// agree to ~1e-7.
-//
-// kEnergy: the row holds non-negative fp32 weights (block energies) instead of
-// logits; p = w / sum(w) replaces the softmax, and a row of zero total keeps
-// nothing.  votes (optional, [nrows, nb] int32) gets +1 for every kept entry;
-// bits and counts are optional too.
-template <bool kEnergy>
-__global__ void __launch_bounds__(256) select_kernel(const void* __restrict__ in, int64_t nrows,
-                                                     int nb, int wpc, SelectParams prm,
-                                                     uint32_t* __restrict__ bits,
-                                                     int32_t* __restrict__ counts,
-                                                     uint8_t* __restrict__ mask_u8,
-                                                     int32_t* __restrict__ votes) {
-  extern __shared__ uint32_t sel_keys[];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t g = static_cast<int64_t>(blockIdx.x) * wpc + warp;
+__device__ __forceinline__ unsigned long long cta_sum_u64(unsigned long long v,
+                                                          unsigned long long* xch, int warp,
+                                                          int lane) {
+  v = warp_sum_u64(v);
+  if (lane == 0) xch[warp] = v;
+  __syncthreads();
+  unsigned long long r = 0;
+#pragma unroll
+  for (int w = 0; w < kSelWarps; ++w) r += xch[w];
+  __syncthreads();
+  return r;
+}
+
+__device__ __forceinline__ unsigned long long sel_fix(double p) {
+  return __double2ull_rn(p * kSelFix);   // p in [0, 1]: at most 2^62
+}
+
+// Bin of p in [lo, hi] split into kSelBins equal parts (s = kSelBins / (hi - lo)).
+__device__ __forceinline__ int sel_bin(double p, double lo, double s) {
+  return static_cast<int>(fmin((p - lo) * s, static_cast<double>(kSelBins - 1)));
+}
+
+// q = a / b for 0 <= a < 4096, 1 <= b <= 4096: (a + 0.5) / b lies at least
+// 0.5 / b from an integer, far more than the fp32 error of the product.
+__device__ __forceinline__ int sel_div(int a, float inv_b) {
+  return __float2int_rz((static_cast<float>(a) + 0.5f) * inv_b);
+}
+
+template <bool kWeights>
+__global__ void __launch_bounds__(kSelThreads) select_kernel(const void* __restrict__ in,
+                                                             int64_t nrows, int nb,
+                                                             SelectParams prm,
+                                                             uint32_t* __restrict__ bits,
+                                                             int32_t* __restrict__ counts,
+                                                             uint8_t* __restrict__ mask_u8,
+                                                             int32_t* __restrict__ votes) {
+  extern __shared__ __align__(16) unsigned char sel_smem[];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int64_t g = blockIdx.x;
   if (g >= nrows) return;
+  const unsigned full = 0xffffffffu;
+  const unsigned lt_mask = (1u << lane) - 1u;
   const int r = static_cast<int>(g % nb);
   const int nw = (nb + 31) >> 5;
-  uint32_t* key = sel_keys + static_cast<int64_t>(warp) * nb;
+  double* pv = reinterpret_cast<double*>(sel_smem);
+  uint16_t* list = reinterpret_cast<uint16_t*>(sel_smem + 8ull * nb);
+  uint32_t* kbits = reinterpret_cast<uint32_t*>(sel_smem + 8ull * nb + ((2ull * nb + 7) & ~7ull));
+  unsigned long long* hm =
+      reinterpret_cast<unsigned long long*>(reinterpret_cast<unsigned char*>(kbits) +
+                                            4ull * ((nw + 1) & ~1));
+  uint32_t* hc = reinterpret_cast<uint32_t*>(hm + kSelBins);
+  double* xd = reinterpret_cast<double*>(hc + kSelBins);                  // [kSelWarps]
+  unsigned long long* xu = reinterpret_cast<unsigned long long*>(xd + kSelWarps);   // [kSelWarps]
+  int* xi = reinterpret_cast<int*>(xu + kSelWarps);                       // [2 * kSelWarps]
+  unsigned long long* xs = reinterpret_cast<unsigned long long*>(xi + 2 * kSelWarps);  // [4]
 
-  float zl = 0.f;
+  // ---- probabilities in fp64
   bool empty_row = false;
-  if (kEnergy) {
-    const float* Erow = static_cast<const float*>(in) + g * nb;
-    for (int c = lane; c < nb; c += 32) {
-      const float e = Erow[c];
-      const float w = e > 0.f ? e : 0.f;   // negative or NaN weights count as zero
-      key[c] = __float_as_uint(w);
-      zl += w;
+  double z;
+  if (kWeights) {
+    const float* W = static_cast<const float*>(in) + g * nb;
+    double zl = 0.0;
+    for (int c = tid; c < nb; c += kSelThreads) {
+      const float w = W[c];
+      const double x = w > 0.f ? static_cast<double>(w) : 0.0;   // negative or NaN count as zero
+      pv[c] = x;
+      zl += x;
     }
+    z = cta_reduce<0>(zl, xd, warp, lane);
+    empty_row = !(z > 0.0);
   } else {
-    // softmax over the row (max subtracted in fp64)
     const double* Lrow = static_cast<const double*>(in) + g * nb;
     double mx = -INFINITY;
-    for (int c = lane; c < nb; c += 32) mx = fmax(mx, Lrow[c]);
-    mx = warp_max(mx);
-    for (int c = lane; c < nb; c += 32) {
-      const float e = expf(static_cast<float>(Lrow[c] - mx));
-      key[c] = __float_as_uint(e);
+    for (int c = tid; c < nb; c += kSelThreads) mx = fmax(mx, Lrow[c]);
+    mx = cta_reduce<1>(mx, xd, warp, lane);
+    double zl = 0.0;
+#pragma unroll 4
+    for (int c = tid; c < nb; c += kSelThreads) {
+      const double e = exp(Lrow[c] - mx);
+      pv[c] = e;
       zl += e;
     }
+    z = cta_reduce<0>(zl, xd, warp, lane);
   }
-  const float z = static_cast<float>(warp_sum(static_cast<double>(zl)));
-  if (kEnergy) empty_row = !(z > 0.f);   // uniform: z is lane 0's value
-  uint32_t kmax = 0;
-  for (int c = lane; c < nb; c += 32) {
-    const uint32_t kv = empty_row ? 0u : __float_as_uint(__uint_as_float(key[c]) / z);
-    key[c] = kv;
-    kmax = max(kmax, kv);
-  }
-  kmax = warp_max_u32(kmax);
-  __syncwarp();
-
-  // v*: largest key whose mass-at-or-above reaches 1 - thr.  Entries with a
-  // larger key are kept; entries with key v* are taken in block order while
-  // the exclusive prefix mass stays below the target.  The first entry of the
-  // sorted row is always kept.
-  const double target = 1.0 - static_cast<double>(prm.thr);
+  double lo = INFINITY, hi = -INFINITY;
   const bool topk_mode = prm.topk > 0;
-  bool keep_all = topk_mode ? prm.topk >= nb : prm.thr <= 0.f;
-  uint32_t vstar = kmax;
-  double above = 0.0;
-  int tied_quota = 0;          // top-k: tied entries kept, in block order
-  if (topk_mode && !keep_all) {
-    // v*: largest key with at least topk entries at or above it
-    uint32_t lo = 0u, hi = kmax + 1u;   // count(lo) = nb >= topk > count(hi) = 0
-    while (hi - lo > 1u) {
-      const uint32_t mid = lo + ((hi - lo) >> 1);
-      if (count_at_or_above(key, nb, lane, mid) >= prm.topk) lo = mid; else hi = mid;
+  unsigned long long tot = 0;
+  if (!empty_row) {
+    for (int c = tid; c < nb; c += kSelThreads) {
+      const double p = pv[c] / z;
+      pv[c] = p;
+      lo = fmin(lo, p);
+      hi = fmax(hi, p);
+      tot += sel_fix(p);
     }
-    vstar = lo;
-    tied_quota = prm.topk - count_at_or_above(key, nb, lane, vstar + 1u);
-  } else if (!keep_all && target > 0.0) {
-    const double total = mass_at_or_above(key, nb, lane, 0u);
-    if (total < target) {
-      keep_all = true;   // every exclusive prefix stays below the target
-    } else {
-      uint32_t lo = 0u, hi = kmax + 1u;   // mass(lo) >= target > mass(hi)
-      while (hi - lo > 1u) {
-        const uint32_t mid = lo + ((hi - lo) >> 1);
-        if (mass_at_or_above(key, nb, lane, mid) >= target) lo = mid; else hi = mid;
+    lo = cta_reduce<2>(lo, xd, warp, lane);
+    hi = cta_reduce<1>(hi, xd, warp, lane);
+    if (!topk_mode) tot = cta_sum_u64(tot, xu, warp, lane);
+  }
+  for (int w = tid; w < nw; w += kSelThreads) kbits[w] = 0u;
+
+  // ---- the kept set (every branch below is uniform across the CTA)
+  bool keep_all = false;
+  unsigned long long T = 0;   // target: fixed-point mass, or the count k
+  if (topk_mode) {
+    keep_all = prm.topk >= nb;
+    T = static_cast<unsigned long long>(prm.topk);
+  } else {
+    keep_all = prm.thr <= 0.f;
+    const double t = 1.0 - static_cast<double>(prm.thr);
+    T = t > 0.0 ? sel_fix(t) : 0ull;
+    // every exclusive prefix stays below the target when the whole row does
+    if (!keep_all && !empty_row) keep_all = tot < T;
+  }
+  __syncthreads();
+  if (!keep_all && !empty_row) {
+    unsigned long long above = 0;   // mass (or count) of the entries ranked above the candidates
+    uint32_t above_n = 0;           // number of those entries
+    int n_c = nb;                   // candidates: every entry (implicit list) at level 0
+    bool implicit = true;
+    for (int level = 0; level < kSelMaxLevels && n_c > 32 && hi > lo; ++level) {
+      const double s = fmin(kSelBins / (hi - lo), 1.7976931348623157e308);
+      for (int i = tid; i < kSelBins; i += kSelThreads) {
+        hm[i] = 0ull;
+        hc[i] = 0u;
       }
-      vstar = lo;
-      above = mass_at_or_above(key, nb, lane, vstar + 1u);   // < target
+      __syncthreads();
+      for (int i = tid; i < n_c; i += kSelThreads) {
+        const int c = implicit ? i : list[i];
+        const double p = pv[c];
+        const int b = sel_bin(p, lo, s);
+        atomicAdd(&hm[b], topk_mode ? 1ull : sel_fix(p));
+        atomicAdd(&hc[b], 1u);
+      }
+      __syncthreads();
+      if (warp == 0) {
+        // lane l holds bins [8l, 8l+8); suffix sums over lanes >= l (inclusive)
+        unsigned long long loc = 0;
+        uint32_t locn = 0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          loc += hm[8 * lane + j];
+          locn += hc[8 * lane + j];
+        }
+        unsigned long long suf = loc;
+        uint32_t sufn = locn;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+          const unsigned long long y = __shfl_down_sync(full, suf, off);
+          const uint32_t yn = __shfl_down_sync(full, sufn, off);
+          if (lane + off < 32) {
+            suf += y;
+            sufn += yn;
+          }
+        }
+        // the crossing bin lies in the highest lane whose suffix reaches the
+        // target (lane 0's suffix is every candidate, which always does)
+        const uint32_t bal = __ballot_sync(full, above + suf >= T);
+        const int cl = 31 - __clz(bal | 1u);
+        if (lane == cl) {
+          unsigned long long run = above + (suf - loc);
+          uint32_t runn = above_n + (sufn - locn);
+          int b = 8 * lane + 7;
+          for (; b > 8 * lane; --b) {
+            if (run + hm[b] >= T) break;
+            run += hm[b];
+            runn += hc[b];
+          }
+          xi[0] = b;
+          xi[1] = static_cast<int>(hc[b]);
+          xs[0] = run;
+          xs[1] = runn;
+        }
+      }
+      __syncthreads();
+      const int bstar = xi[0], nb_star = xi[1];
+      above = xs[0];
+      above_n = static_cast<uint32_t>(xs[1]);
+      // keep the higher bins, carry the crossing bin's entries (stable order)
+      int kept_n = 0;
+      double nlo = INFINITY, nhi = -INFINITY;
+      for (int i0 = 0; i0 < n_c; i0 += kSelThreads) {
+        const int i = i0 + tid;
+        int c = -1, b = -1;
+        double p = 0.0;
+        if (i < n_c) {
+          c = implicit ? i : list[i];
+          p = pv[c];
+          b = sel_bin(p, lo, s);
+        }
+        if (implicit) {   // entry c = i: warp w of the chunk fills one bitmap word
+          const uint32_t kb = __ballot_sync(full, b > bstar);
+          if (lane == 0 && kb) kbits[i >> 5] |= kb;
+        } else if (b > bstar) {
+          atomicOr(&kbits[c >> 5], 1u << (c & 31));
+        }
+        const bool nxt = b == bstar;
+        const uint32_t bn = __ballot_sync(full, nxt);
+        if (lane == 0) xi[2 + warp] = __popc(bn);
+        __syncthreads();   // every element of this chunk has been read
+        int before = kept_n;
+        for (int w = 0; w < warp; ++w) before += xi[2 + w];
+        if (nxt) {
+          list[before + __popc(bn & lt_mask)] = static_cast<uint16_t>(c);
+          nlo = fmin(nlo, p);
+          nhi = fmax(nhi, p);
+        }
+        for (int w = 0; w < kSelWarps; ++w) kept_n += xi[2 + w];
+        __syncthreads();   // counts consumed before the next chunk posts its own
+      }
+      n_c = nb_star;
+      implicit = false;
+      lo = cta_reduce<2>(nlo, xd, warp, lane);
+      hi = cta_reduce<1>(nhi, xd, warp, lane);
+    }
+    if (n_c <= 32) {
+      if (warp == 0) {
+        // exact order of the last candidates: bitonic network on (p desc, index asc)
+        const int c = lane < n_c ? (implicit ? lane : static_cast<int>(list[lane])) : -1;
+        unsigned long long key =
+            c >= 0 ? static_cast<unsigned long long>(__double_as_longlong(pv[c])) : 0ull;
+        int idx = c >= 0 ? c : 0x7fffffff;
+#pragma unroll
+        for (int k = 2; k <= 32; k <<= 1) {
+#pragma unroll
+          for (int j = k >> 1; j > 0; j >>= 1) {
+            const unsigned long long ok = __shfl_xor_sync(full, key, j);
+            const int oi = __shfl_xor_sync(full, idx, j);
+            const bool other_first = ok > key || (ok == key && oi < idx);
+            const bool lower = (lane & j) == 0, up = (lane & k) == 0;
+            if ((lower == up) ? other_first : !other_first) {
+              key = ok;
+              idx = oi;
+            }
+          }
+        }
+        const bool valid = idx != 0x7fffffff;
+        const unsigned long long f =
+            valid ? (topk_mode ? 1ull : sel_fix(__longlong_as_double(static_cast<long long>(key))))
+                  : 0ull;
+        unsigned long long incl = f;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+          const unsigned long long y = __shfl_up_sync(full, incl, off);
+          if (lane >= off) incl += y;
+        }
+        const bool keep = valid && ((above_n == 0 && lane == 0) || above + (incl - f) < T);
+        if (keep) atomicOr(&kbits[idx >> 5], 1u << (idx & 31));
+      }
+    } else {
+      // the candidates share one p (or the level cap was reached): block order
+      const int c0 = implicit ? 0 : static_cast<int>(list[0]);
+      const unsigned long long f = topk_mode ? 1ull : sel_fix(pv[c0]);
+      int nkeep = 0;
+      if (above < T) {
+        const unsigned long long need = (T - above + f - 1) / (f > 0 ? f : 1ull);
+        nkeep = (f == 0 || need >= static_cast<unsigned long long>(n_c)) ? n_c : static_cast<int>(need);
+      }
+      if (above_n == 0 && nkeep == 0) nkeep = 1;
+      for (int i = tid; i < nkeep; i += kSelThreads) {
+        const int c = implicit ? i : static_cast<int>(list[i]);
+        atomicOr(&kbits[c >> 5], 1u << (c & 31));
+      }
     }
   }
+  __syncthreads();
 
-  // flags -> bitmap words, optional uint8 row, STA union, counts
-  const int rt = r / (prm.Th * prm.Tw), rh = (r / prm.Tw) % prm.Th, rw = r % prm.Tw;
-  const double pstar = static_cast<double>(__uint_as_float(vstar));
-  double carry = above;        // exclusive prefix mass before the next tied entry
-  bool first_tied = true;      // no tied entry seen yet
-  int tied_seen = 0;
+  // ---- flags -> bitmap words, optional uint8 row, STA union, votes, count
+  const float inv_tw = 1.0f / static_cast<float>(prm.Tw);
+  const float inv_thw = 1.0f / static_cast<float>(prm.Th * prm.Tw);
+  int rt = 0, rh = 0, rw = 0;
+  if (prm.use_sta) {
+    rt = sel_div(r, inv_thw);
+    const int rr = r - rt * prm.Th * prm.Tw;
+    rh = sel_div(rr, inv_tw);
+    rw = rr - rh * prm.Tw;
+  }
   int count = 0;
   uint32_t* brow = bits ? bits + g * nw : nullptr;
   uint8_t* mrow = mask_u8 ? mask_u8 + g * nb : nullptr;
-  for (int w = 0; w < nw; ++w) {
+  for (int w = warp; w < nw; w += kSelWarps) {
     const int c = w * 32 + lane;
     const bool inrow = c < nb;
-    bool keep;
-    if (empty_row) {   // warp-uniform branch
-      keep = false;
-    } else if (keep_all) {   // warp-uniform branch
-      keep = inrow;
-    } else {
-      const uint32_t kv = inrow ? key[c] : 0u;
-      const bool tied = inrow && kv == vstar;
-      const uint32_t tb = __ballot_sync(0xffffffffu, tied);
-      const int rank = __popc(tb & ((1u << lane) - 1u));   // tied entries before this one
-      const bool is_first = first_tied && tied && rank == 0;
-      const double excl = carry + rank * pstar;
-      if (topk_mode)
-        keep = inrow && (kv > vstar || (tied && tied_seen + rank < tied_quota));
-      else
-        keep = inrow && (kv > vstar || (tied && (excl < target || (is_first && vstar == kmax))));
-      carry += __popc(tb) * pstar;
-      tied_seen += __popc(tb);
-      if (tb) first_tied = false;
-    }
+    bool keep = inrow && !empty_row && (keep_all || ((kbits[w] >> lane) & 1u) != 0u);
     if (inrow && prm.use_sta) {
-      const int ct = c / (prm.Th * prm.Tw), ch = (c / prm.Tw) % prm.Th, cw = c % prm.Tw;
+      const int ct = sel_div(c, inv_thw);
+      const int cc = c - ct * prm.Th * prm.Tw;
+      const int ch = sel_div(cc, inv_tw);
+      const int cw = cc - ch * prm.Tw;
       keep |= abs(ct - rt) <= prm.wt && abs(ch - rh) <= prm.wh && abs(cw - rw) <= prm.ww;
     }
     if (mrow && inrow) mrow[c] = keep ? 1 : 0;
     if (votes && keep) votes[g * nb + c] += 1;
-    const uint32_t word = __ballot_sync(0xffffffffu, keep);
+    const uint32_t word = __ballot_sync(full, keep);
     if (brow && lane == 0) brow[w] = word;
     count += __popc(word);
   }
-  if (counts && lane == 0) counts[g] = count;
+  if (lane == 0) xi[2 + warp] = count;
+  __syncthreads();
+  if (counts && tid == 0) {
+    int total = 0;
+    for (int w = 0; w < kSelWarps; ++w) total += xi[2 + w];
+    counts[g] = total;
+  }
 }
 
 // Calibrated mask from accumulated votes: keep (r, c) iff votes >= min_votes.
@@ -490,6 +689,7 @@ __global__ void __launch_bounds__(256) fill_kernel(const uint32_t* __restrict__ 
 
 // ------------------------------------------------------------------ launchers
 
+
 cudaError_t launch_pool(const void* q, const void* k, double* qbar, double* kbar,
                         int64_t nblocks, int d, int nb, int raster, int Th, int Tw,
                         cudaStream_t st) {
@@ -530,17 +730,13 @@ cudaError_t launch_select(const double* L, int64_t nrows, int nb, float thr, int
                           int use_sta, int wt, int wh, int ww, int Tt, int Th, int Tw,
                           uint32_t* bits, int32_t* counts, uint8_t* mask_u8, cudaStream_t st) {
   SelectParams prm{thr, use_sta, wt, wh, ww, Tt, Th, Tw, topk};
-  const size_t per_warp = static_cast<size_t>(nb) * sizeof(uint32_t);
-  int wpc = static_cast<int>((200u * 1024u) / per_warp);
-  wpc = wpc < 1 ? 1 : (wpc > 8 ? 8 : wpc);
-  const size_t smem = per_warp * wpc;
+  const size_t smem = select_row_bytes(nb);
   cudaError_t e = cudaFuncSetAttribute(select_kernel<false>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  const unsigned grid = static_cast<unsigned>((nrows + wpc - 1) / wpc);
-  select_kernel<false><<<grid, 32 * wpc, smem, st>>>(L, nrows, nb, wpc, prm, bits, counts,
-                                                     mask_u8, nullptr);
+  select_kernel<false><<<static_cast<unsigned>(nrows), kSelThreads, smem, st>>>(
+      L, nrows, nb, prm, bits, counts, mask_u8, nullptr);
   return cudaGetLastError();
 }
 
@@ -552,34 +748,26 @@ cudaError_t launch_select_weights(const float* weights, int64_t nrows, int nb, f
                                   uint32_t* bits, int32_t* counts, uint8_t* mask_u8,
                                   cudaStream_t st) {
   SelectParams prm{thr, use_sta, wt, wh, ww, Tt, Th, Tw, topk};
-  const size_t per_warp = static_cast<size_t>(nb) * sizeof(uint32_t);
-  int wpc = static_cast<int>((200u * 1024u) / per_warp);
-  wpc = wpc < 1 ? 1 : (wpc > 8 ? 8 : wpc);
-  const size_t smem = per_warp * wpc;
+  const size_t smem = select_row_bytes(nb);
   cudaError_t e = cudaFuncSetAttribute(select_kernel<true>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  const unsigned grid = static_cast<unsigned>((nrows + wpc - 1) / wpc);
-  select_kernel<true><<<grid, 32 * wpc, smem, st>>>(weights, nrows, nb, wpc, prm, bits, counts,
-                                                    mask_u8, nullptr);
+  select_kernel<true><<<static_cast<unsigned>(nrows), kSelThreads, smem, st>>>(
+      weights, nrows, nb, prm, bits, counts, mask_u8, nullptr);
   return cudaGetLastError();
 }
 
 cudaError_t launch_calib_select(const float* energy, int64_t nrows, int nb, float eps,
                                 int32_t* votes, cudaStream_t st) {
   SelectParams prm{eps, 0, 0, 0, 0, 1, 1, 1, 0};
-  const size_t per_warp = static_cast<size_t>(nb) * sizeof(uint32_t);
-  int wpc = static_cast<int>((200u * 1024u) / per_warp);
-  wpc = wpc < 1 ? 1 : (wpc > 8 ? 8 : wpc);
-  const size_t smem = per_warp * wpc;
+  const size_t smem = select_row_bytes(nb);
   cudaError_t e = cudaFuncSetAttribute(select_kernel<true>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  const unsigned grid = static_cast<unsigned>((nrows + wpc - 1) / wpc);
-  select_kernel<true><<<grid, 32 * wpc, smem, st>>>(energy, nrows, nb, wpc, prm, nullptr, nullptr,
-                                                    nullptr, votes);
+  select_kernel<true><<<static_cast<unsigned>(nrows), kSelThreads, smem, st>>>(
+      energy, nrows, nb, prm, nullptr, nullptr, nullptr, votes);
   return cudaGetLastError();
 }
 

@@ -345,6 +345,19 @@ nabla_status fwd_with_header(const nabla_shape* shape, const void* q, const void
   return run_fwd(shape, q, k, v, row_ptr, col_idx, scale, o, lse, header, redo, kv_scratch,
                  reinterpret_cast<cudaStream_t>(stream));
 }
+// The argument checks of a forward call (shape, token layout and tile grid,
+// null pointers, 16-byte alignment of q, k, v, o, a finite scale), for entry
+// points that must reject a call before they enqueue any work.
+nabla_status check_fwd_args(const nabla_shape* shape, const void* q, const void* k,
+                            const void* v, const void* o, float scale) {
+  nabla_status s = check_shape(shape);
+  if (s != NABLA_OK) return s;
+  if (!q || !k || !v || !o) return fail(NABLA_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
+    return fail(NABLA_ERR_INVALID_ARG, "q, k, v, o need 16-byte alignment");
+  if (!std::isfinite(scale)) return fail(NABLA_ERR_INVALID_ARG, "scale must be finite");
+  return NABLA_OK;
+}
 // nabla_build_mask with its device status bits OR-ed into `status` instead of
 // the workspace header (the host-buffer layer shares one header between the
 // chunks it runs on two streams).
@@ -353,6 +366,11 @@ nabla_status build_mask_with_status(const nabla_shape* shape, const nabla_mask_p
                                     int32_t* row_ptr, int32_t* col_idx, int64_t col_capacity,
                                     int32_t* nnz_out, void* workspace, int* status,
                                     nabla_stream_t stream);
+nabla_status build_mask_staged(const nabla_shape* shape, const nabla_mask_params* params,
+                               const void* q, const void* k, uint8_t* mask_u8, int32_t* row_ptr,
+                               int32_t* col_idx, int64_t col_capacity, int32_t* nnz_out,
+                               void* workspace, int* status, nabla_stream_t stream,
+                               cudaEvent_t* stage_events);
 }  // namespace nabla
 
 extern "C" {
@@ -428,15 +446,44 @@ nabla_status nabla_build_mask(const nabla_shape* shape, const nabla_mask_params*
                                        nnz_out, workspace, static_cast<int*>(workspace), stream);
 }
 
+nabla_status nabla_build_mask_stage_ms(const nabla_shape* shape, const nabla_mask_params* params,
+                                       const void* q, const void* k, int32_t* row_ptr,
+                                       int32_t* col_idx, int64_t col_capacity, int32_t* nnz_out,
+                                       void* workspace, nabla_stream_t stream, float* ms_out) {
+  if (ms_out == nullptr) return fail(NABLA_ERR_INVALID_ARG, "ms_out is NULL");
+  cudaEvent_t ev[5] = {};
+  cudaError_t e = cudaSuccess;
+  int made = 0;
+  for (; made < 5 && e == cudaSuccess; ++made) e = cudaEventCreate(&ev[made]);
+  nabla_status s = NABLA_OK;
+  if (e != cudaSuccess) {
+    s = cuda_fail(e, "cudaEventCreate");
+    --made;
+  } else {
+    s = nabla::build_mask_staged(shape, params, q, k, nullptr, row_ptr, col_idx, col_capacity,
+                                 nnz_out, workspace, static_cast<int*>(workspace), stream, ev);
+    if (s == NABLA_OK) {
+      e = cudaEventSynchronize(ev[4]);
+      for (int i = 0; i < 4 && e == cudaSuccess; ++i) e = cudaEventElapsedTime(&ms_out[i], ev[i], ev[i + 1]);
+      if (e != cudaSuccess) s = cuda_fail(e, "stage timing");
+    }
+  }
+  for (int i = 0; i < made; ++i) cudaEventDestroy(ev[i]);
+  return s;
+}
+
 }  // extern "C"
 
 namespace nabla {
 
-nabla_status build_mask_with_status(const nabla_shape* shape, const nabla_mask_params* params,
-                                    const void* q, const void* k, uint8_t* mask_u8,
-                                    int32_t* row_ptr, int32_t* col_idx, int64_t col_capacity,
-                                    int32_t* nnz_out, void* workspace, int* status,
-                                    nabla_stream_t stream) {
+// The mask build; stage_events (may be NULL): five events recorded on the
+// stream before pooling, the reduced map, the selection, the compaction, and
+// after it.
+nabla_status build_mask_staged(const nabla_shape* shape, const nabla_mask_params* params,
+                               const void* q, const void* k, uint8_t* mask_u8, int32_t* row_ptr,
+                               int32_t* col_idx, int64_t col_capacity, int32_t* nnz_out,
+                               void* workspace, int* status, nabla_stream_t stream,
+                               cudaEvent_t* stage_events) {
   nabla_status s = check_shape(shape);
   if (s != NABLA_OK) return s;
   if (params == nullptr) return fail(NABLA_ERR_INVALID_ARG, "params is NULL");
@@ -463,20 +510,39 @@ nabla_status build_mask_with_status(const nabla_shape* shape, const nabla_mask_p
   int32_t* counts = reinterpret_cast<int32_t*>(ws + lay.counts);
   const int nb = shape->S / 64, BH = shape->B * shape->H;
   const int64_t nrows = static_cast<int64_t>(BH) * nb;
-  cudaError_t e = nabla::launch_pool(q, k, qbar, kbar, nrows, shape->d, nb,
-                                     shape->layout == NABLA_LAYOUT_RASTER ? 1 : 0, shape->Th,
-                                     shape->Tw, st);
+  auto mark = [&](int i) {
+    return stage_events ? cudaEventRecord(stage_events[i], st) : cudaSuccess;
+  };
+  cudaError_t e = mark(0);
+  if (e == cudaSuccess)
+    e = nabla::launch_pool(q, k, qbar, kbar, nrows, shape->d, nb,
+                           shape->layout == NABLA_LAYOUT_RASTER ? 1 : 0, shape->Th, shape->Tw, st);
   if (e != cudaSuccess) return cuda_fail(e, "pool launch");
-  e = nabla::launch_logits(qbar, kbar, L, BH, nb, shape->d, st);
+  e = mark(1);
+  if (e == cudaSuccess) e = nabla::launch_logits(qbar, kbar, L, BH, nb, shape->d, st);
   if (e != cudaSuccess) return cuda_fail(e, "logits launch");
-  e = nabla::launch_select(L, nrows, nb, params->thr, params->topk, params->use_sta ? 1 : 0,
-                           params->wt, params->wh, params->ww, shape->Tt, shape->Th, shape->Tw,
-                           bits, counts, mask_u8, st);
+  e = mark(2);
+  if (e == cudaSuccess)
+    e = nabla::launch_select(L, nrows, nb, params->thr, params->topk, params->use_sta ? 1 : 0,
+                             params->wt, params->wh, params->ww, shape->Tt, shape->Th, shape->Tw,
+                             bits, counts, mask_u8, st);
   if (e != cudaSuccess) return cuda_fail(e, "select launch");
-  e = nabla::launch_scan_fill(bits, counts, nrows, nb, row_ptr, col_idx, col_capacity, nnz_out,
-                              status, st);
+  e = mark(3);
+  if (e == cudaSuccess)
+    e = nabla::launch_scan_fill(bits, counts, nrows, nb, row_ptr, col_idx, col_capacity, nnz_out,
+                                status, st);
+  if (e == cudaSuccess) e = mark(4);
   if (e != cudaSuccess) return cuda_fail(e, "scan/fill launch");
   return NABLA_OK;
+}
+
+nabla_status build_mask_with_status(const nabla_shape* shape, const nabla_mask_params* params,
+                                    const void* q, const void* k, uint8_t* mask_u8,
+                                    int32_t* row_ptr, int32_t* col_idx, int64_t col_capacity,
+                                    int32_t* nnz_out, void* workspace, int* status,
+                                    nabla_stream_t stream) {
+  return build_mask_staged(shape, params, q, k, mask_u8, row_ptr, col_idx, col_capacity, nnz_out,
+                           workspace, status, stream, nullptr);
 }
 
 }  // namespace nabla

@@ -39,6 +39,8 @@ nabla_status fwd_with_header(const nabla_shape* shape, const void* q, const void
                              const void* v, const int32_t* row_ptr, const int32_t* col_idx,
                              float scale, void* o, float* lse, int* header, int* redo,
                              void* kv_scratch, nabla_stream_t stream);
+nabla_status check_fwd_args(const nabla_shape* shape, const void* q, const void* k,
+                            const void* v, const void* o, float scale);
 }  // namespace nabla
 
 namespace {
@@ -89,13 +91,11 @@ NABLA_API nabla_status bsa_fwd_with_mask_static(const nabla_shape* shape, const 
                                                 const uint8_t* mask_u8, float scale, void* o,
                                                 float* lse, int32_t* status_out,
                                                 nabla_stream_t stream) {
-  if (shape == nullptr) return fail(NABLA_ERR_INVALID_ARG, "shape is NULL");
-  if (shape->B <= 0 || shape->H <= 0 || shape->S <= 0 || shape->d <= 0)
-    return fail(NABLA_ERR_INVALID_ARG, "B, H, S and d must be positive");
-  if (shape->d != 64 && shape->d != 128) return fail(NABLA_ERR_UNSUPPORTED, "d must be 64 or 128");
-  if (shape->S % 64 != 0) return fail(NABLA_ERR_UNSUPPORTED, "S must be a multiple of 64");
-  if (!q || !k || !v || !mask_u8 || !o) return fail(NABLA_ERR_INVALID_ARG, "null pointer");
-  if (!std::isfinite(scale)) return fail(NABLA_ERR_INVALID_ARG, "scale must be finite");
+  // every argument check of the forward runs before anything is enqueued, so
+  // a rejected call leaves the shared scratch untouched
+  nabla_status s = nabla::check_fwd_args(shape, q, k, v, o, scale);
+  if (s != NABLA_OK) return s;
+  if (mask_u8 == nullptr) return fail(NABLA_ERR_INVALID_ARG, "null pointer");
   // block CSR of the mask, laid out as in a bsa_fwd_with_mask workspace
   const size_t nb = static_cast<size_t>(shape->S) / 64;
   const size_t rows = static_cast<size_t>(shape->B) * shape->H * nb, nw = (nb + 31) / 32;
@@ -110,7 +110,7 @@ NABLA_API nabla_status bsa_fwd_with_mask_static(const nabla_shape* shape, const 
                 "holds " + std::to_string(kStaticScratchBytes) + " (B*H*(S/64)^2 must stay "
                 "below about 8.3 million blocks)");
   void* base = nullptr;
-  nabla_status s = scratch_address(&base);
+  s = scratch_address(&base);
   if (s != NABLA_OK) return s;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   unsigned char* ws = static_cast<unsigned char*>(base);

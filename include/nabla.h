@@ -396,6 +396,15 @@ NABLA_API int nabla_version(void);
  * forward workspace's header: how many forwards on it needed the
  * exact-reference kernel since nabla_workspace_init (-1 on a CUDA error).
  *
+ * nabla_build_mask_stage_ms: runs nabla_build_mask once (no uint8 mask) with
+ * CUDA events between its kernels, synchronises the stream, and writes the
+ * milliseconds of its four stages to ms_out[0..3]: pooling, the reduced map,
+ * the selection, the CSR compaction.  Arguments as for nabla_build_mask.
+ *
+ * nabla_selftest_fp64_tflops: times independent fp64 fma chains on every SM
+ * (about 0.1 s), synchronises the stream and writes the measured fp64 rate in
+ * TFLOP/s: the denominator of the reduced map's roofline.
+ *
  * nabla_selftest_mma: one 128 x N x 128 bf16 product through the same
  * tcgen05/TMA building blocks the attention kernel uses, for layout checks.
  *   variant 0: C[m][n] = sum_k A[m][k] B[n][k]   (both K-major, N = 128)
@@ -409,6 +418,13 @@ NABLA_API void nabla_set_exact_reference(int on);
 NABLA_API int nabla_query_exact_passes(const void* workspace, nabla_stream_t stream);
 NABLA_API nabla_status nabla_selftest_mma(int variant, const void* a, const void* b, float* c,
                                 void* workspace, nabla_stream_t stream);
+NABLA_API nabla_status nabla_build_mask_stage_ms(const nabla_shape* shape,
+                                                 const nabla_mask_params* params, const void* q,
+                                                 const void* k, int32_t* row_ptr, int32_t* col_idx,
+                                                 int64_t col_capacity, int32_t* nnz_out,
+                                                 void* workspace, nabla_stream_t stream,
+                                                 float* ms_out);
+NABLA_API nabla_status nabla_selftest_fp64_tflops(nabla_stream_t stream, double* tflops_out);
 
 #ifdef __cplusplus
 }

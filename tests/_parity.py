@@ -35,18 +35,24 @@ def check_csr(row_ptr, col_idx, nrows, nb):
 def compare_masks(gpu_mask, ora_mask, diag, thr):
     """Mask parity: bit-exact except rows whose cut sits within CUT_BAND of
     1 - thr (or whose cut probabilities tie to 1e-6); those rows must differ
-    by at most two blocks.  Returns (n_rows, n_mismatch, n_exempt_rows)."""
+    by at most two blocks.  Returns a dict of counts: rows, rows that differ,
+    near-cut rows, near-tie rows, exempt rows (either) and exempt rows that
+    differ."""
     import oracle
     g = gpu_mask.reshape(-1, gpu_mask.shape[-1])
     o = ora_mask.reshape(-1, ora_mask.shape[-1])
     dg = diag.reshape(-1, 4)
     diff = (g != o).sum(axis=1)
-    exempt = oracle.near_cut_rows(dg, thr, CUT_BAND) | oracle.near_tie_rows(dg)
+    near_cut = oracle.near_cut_rows(dg, thr, CUT_BAND)
+    near_tie = oracle.near_tie_rows(dg)
+    exempt = near_cut | near_tie
     bad = (diff > 0) & ~exempt
     assert not bad.any(), (f"{bad.sum()} non-exempt rows differ; first {np.nonzero(bad)[0][:5]}, "
                            f"diff counts {diff[bad][:5]}")
     assert diff[exempt].max(initial=0) <= 2
-    return g.shape[0], int((diff > 0).sum()), int(exempt.sum())
+    return {"rows": int(g.shape[0]), "rows_differing": int((diff > 0).sum()),
+            "near_cut": int(near_cut.sum()), "near_tie": int(near_tie.sum()),
+            "exempt": int(exempt.sum()), "exempt_differing": int(((diff > 0) & exempt).sum())}
 
 
 def compare_attention(o_gpu, lse_gpu, o_ref, lse_ref):

@@ -25,3 +25,26 @@ def synth_mod():
     import synth
     synth.build()
     return synth
+
+
+# Parity records: counts and errors the GPU parity tests measured (exempt mask
+# rows per configuration, rows compared, error maxima), printed in the terminal
+# summary so that a quiet run still reports them.
+_PARITY_RECORDS = []
+
+
+@pytest.fixture
+def parity_record():
+    def add(what, **fields):
+        _PARITY_RECORDS.append((what, fields))
+    return add
+
+
+def pytest_terminal_summary(terminalreporter):
+    if not _PARITY_RECORDS:
+        return
+    terminalreporter.section("parity records")
+    for what, fields in _PARITY_RECORDS:
+        body = ", ".join(f"{k}={v:.3g}" if isinstance(v, float) else f"{k}={v}"
+                         for k, v in fields.items())
+        terminalreporter.write_line(f"{what}: {body}")

@@ -1,7 +1,11 @@
 """Block-sparse attention forward on the GPU vs the fp64 oracle: bf16 O within
 max-abs 2e-2 / mean-abs 2e-3, fp32 LSE within 1e-3.  The oracle always uses
-its own mask (or a host-made static mask); for the composed NABLA layer the
-rows compared are those whose mask row the GPU and the oracle agree on."""
+its own mask (or a host-made static mask) and never takes a GPU result as
+input.  For the composed NABLA layer (GPU mask -> GPU attention), the sampled
+rows whose mask row the GPU and the oracle agree on are compared directly;
+the rows of query blocks whose mask rows differ (near-cut rows) are compared
+after a second GPU forward over the oracle's own mask, so the attention on
+exactly those rows is checked as well."""
 import numpy as np
 import pytest
 
@@ -60,21 +64,35 @@ def test_attention_parity_all_rows(nl, oracle_mod, synth_mod, name, exact):
 
 
 @pytest.mark.parametrize("name", ["hunyuan720p", "wan720p"])
-def test_attention_parity_full_size(nl, oracle_mod, synth_mod, name):
+def test_attention_parity_full_size(nl, oracle_mod, synth_mod, parity_record, name):
+    """Every head x 64 seeded query blocks (plus the first and last) x all 64
+    rows of each block."""
+    import torch
     w = synth_mod.WORKLOADS[name]
     q, k, v = synth_mod.make_qkv(w)
     # the Wan-shaped layer runs on the fixed-reference kernel alone
     o, lse, gmask = _nabla_layer(nl, w, q, k, v, passes=0 if name == "wan720p" else None)
     mask = oracle_mod.build_mask(q, k, w.tile_grid, w.thr, w.sta)
-    rows = rows_with_same_mask(sample_rows(w.B, w.H, w.S, 2, 8, seed=1), gmask, mask, w.S)
+    rows = sample_rows(w.B, w.H, w.S, 64, 64, seed=1)
+    same_rows = rows_with_same_mask(rows, gmask, mask, w.S)
+    diff_rows = np.setdiff1d(rows, same_rows)
     ro, rl = oracle_mod.masked_attention(q, k, v, mask, rows)
-    go, gl = _gather(o, lse, rows, w.S)
-    mx, mean = compare_attention(go, gl, ro, rl)
-    print(f"{name}: {rows.size} sampled rows, max-abs {mx:.3g} mean-abs {mean:.3g}")
+    sel = np.isin(rows, same_rows)
+    go, gl = _gather(o, lse, same_rows, w.S)
+    mx, mean = compare_attention(go, gl, ro[sel], rl[sel])
+    if diff_rows.size:
+        # the same forward over the oracle's mask, on the rows whose masks differ
+        qd, kd, vd = to_device_bf16(q), to_device_bf16(k), to_device_bf16(v)
+        o2, lse2 = nl.bsa_fwd_with_mask(qd, kd, vd, torch.from_numpy(mask).cuda())
+        go2, gl2 = _gather(o2, lse2, diff_rows, w.S)
+        compare_attention(go2, gl2, ro[~sel], rl[~sel])
+    parity_record(f"attention {name}", sampled_rows=int(rows.size),
+                  rows_compared_on_gpu_mask=int(same_rows.size),
+                  rows_compared_on_oracle_mask=int(diff_rows.size), o_max_abs=mx, o_mean_abs=mean)
 
 
-@pytest.mark.parametrize("p", [0.05, 0.4, 1.0])
-def test_static_mask_sweep_parity(nl, oracle_mod, synth_mod, p):
+@pytest.mark.parametrize("p", [0.05, 0.1, 0.2, 0.4, 0.7, 1.0])
+def test_static_mask_sweep_parity(nl, oracle_mod, synth_mod, parity_record, p):
     w = synth_mod.WORKLOADS["sweep"]
     q, k, v = synth_mod.make_qkv(w)
     mask = synth_mod.make_bernoulli_mask(0, w.B * w.H, w.nb, p).reshape(w.B, w.H, w.nb, w.nb)
@@ -83,10 +101,12 @@ def test_static_mask_sweep_parity(nl, oracle_mod, synth_mod, p):
     ws = nl.Workspace.create(nl.make_shape(w.B, w.H, w.S, w.d), nl.OP_FWD_WITH_MASK)
     o, lse = nl.bsa_fwd_with_mask(qd, kd, vd, torch.from_numpy(mask).cuda(), workspace=ws)
     assert ws.query_status() == 0
-    rows = sample_rows(w.B, w.H, w.S, 2, 8, seed=2)
+    rows = sample_rows(w.B, w.H, w.S, 64, 64, seed=2)
     ro, rl = oracle_mod.masked_attention(q, k, v, mask, rows)
     go, gl = _gather(o, lse, rows, w.S)
-    compare_attention(go, gl, ro, rl)
+    mx, mean = compare_attention(go, gl, ro, rl)
+    parity_record(f"attention sweep p={p}", sampled_rows=int(rows.size), o_max_abs=mx,
+                  o_mean_abs=mean)
 
 
 def _random_qkv(synth_mod, B, H, S, d, seed):

@@ -28,7 +28,7 @@ def _gpu_mask(nl, q, k, grid, thr, sta, cap=None):
             mask.cpu().numpy(), status)
 
 
-def _run_config(nl, oracle_mod, synth_mod, name, thr=None, sta="cfg"):
+def _run_config(nl, oracle_mod, synth_mod, name, thr=None, sta="cfg", record=None):
     w = synth_mod.WORKLOADS[name]
     q, k, _ = synth_mod.make_qkv(w)
     thr = w.thr if thr is None else thr
@@ -40,20 +40,20 @@ def _run_config(nl, oracle_mod, synth_mod, name, thr=None, sta="cfg"):
     assert nnz == row_ptr[-1] == int(gmask.sum())
     assert np.array_equal(csr_to_mask(row_ptr, col_idx, nrows, w.nb), gmask.reshape(nrows, w.nb))
     omask, diag, _ = oracle_mod.build_mask(q, k, w.tile_grid, thr, sta, with_diag=True)
-    n, mism, exempt = compare_masks(gmask, omask, diag, thr)
-    print(f"{name} thr={thr}: rows {n}, mismatched {mism}, near-cut/tie rows {exempt}, "
-          f"density {gmask.mean():.4f}")
+    counts = compare_masks(gmask, omask, diag, thr)
+    if record is not None:
+        record(f"mask {name} thr={thr}", density=float(gmask.mean()), **counts)
     return gmask
 
 
 @pytest.mark.parametrize("name", ["tiny", "small"])
-def test_mask_parity_small_configs(nl, oracle_mod, synth_mod, name):
-    _run_config(nl, oracle_mod, synth_mod, name)
+def test_mask_parity_small_configs(nl, oracle_mod, synth_mod, parity_record, name):
+    _run_config(nl, oracle_mod, synth_mod, name, record=parity_record)
 
 
 @pytest.mark.parametrize("thr", [0.0, 0.05, 0.7, 1.0])
-def test_mask_parity_thresholds(nl, oracle_mod, synth_mod, thr):
-    m = _run_config(nl, oracle_mod, synth_mod, "small", thr=thr, sta=None)
+def test_mask_parity_thresholds(nl, oracle_mod, synth_mod, parity_record, thr):
+    m = _run_config(nl, oracle_mod, synth_mod, "small", thr=thr, sta=None, record=parity_record)
     if thr == 0.0:
         assert m.min() == 1
     if thr == 1.0:
@@ -61,8 +61,8 @@ def test_mask_parity_thresholds(nl, oracle_mod, synth_mod, thr):
 
 
 @pytest.mark.parametrize("name", ["hunyuan720p", "wan720p"])
-def test_mask_parity_full_size(nl, oracle_mod, synth_mod, name):
-    _run_config(nl, oracle_mod, synth_mod, name)
+def test_mask_parity_full_size(nl, oracle_mod, synth_mod, parity_record, name):
+    _run_config(nl, oracle_mod, synth_mod, name, record=parity_record)
 
 
 def test_mask_geometric_rows_closed_form(nl):

@@ -6,7 +6,7 @@ fixed library-owned device array instead of a caller workspace.
 The GPU test calls it through the C ABI twice in a row, with different masks
 and inputs, and checks each result against bsa_fwd_with_mask (the entry point
 with a caller workspace) within the attention tolerance used throughout the
-tests.  This file is named to be collected last."""
+tests, and against the fp64 oracle.  This file is named to be collected last."""
 import ctypes
 
 import numpy as np
@@ -34,6 +34,25 @@ def test_oversized_shape_rejected_before_any_cuda_call(nl):
     assert rc == 2 and lib.bsa_fwd_with_mask_static(None, a, a, a, a, 0.0, a, a, None, None) == 1
 
 
+def test_invalid_arguments_rejected_before_any_work(nl):
+    """Every argument check runs before the entry point touches the shared
+    scratch or the GPU: a raster tile grid that does not cover S/64, a
+    misaligned pointer, a non-finite scale."""
+    lib = nl.lib()
+    a = ctypes.c_void_p(1 << 20)
+    bad_grid = nl.make_shape(1, 2, 64 * 30, 128, (3, 2, 4), nl.LAYOUT_RASTER)   # 24 != 30
+    rc = lib.bsa_fwd_with_mask_static(ctypes.byref(bad_grid), a, a, a, a, 0.0, a, a, None, None)
+    assert rc == 1 and "tile grid" in lib.nabla_last_error().decode()
+    s = nl.make_shape(1, 2, 64 * 30, 128)
+    odd = ctypes.c_void_p((1 << 20) + 8)
+    rc = lib.bsa_fwd_with_mask_static(ctypes.byref(s), odd, a, a, a, 0.0, a, a, None, None)
+    assert rc == 1 and "alignment" in lib.nabla_last_error().decode()
+    rc = lib.bsa_fwd_with_mask_static(ctypes.byref(s), a, a, a, a, float("inf"), a, a, None, None)
+    assert rc == 1 and "finite" in lib.nabla_last_error().decode()
+    rc = lib.bsa_fwd_with_mask_static(ctypes.byref(s), a, a, a, None, 0.0, a, a, None, None)
+    assert rc == 1
+
+
 def _call_static(nl, shape, q, k, v, mask, o, lse, status):
     import torch
     rc = nl.lib().bsa_fwd_with_mask_static(
@@ -46,7 +65,10 @@ def _call_static(nl, shape, q, k, v, mask, o, lse, status):
 
 
 @pytest.mark.gpu
-def test_static_scratch_matches_workspace_entry_point_twice(nl, synth_mod):
+def test_static_scratch_matches_workspace_entry_point_twice(nl, synth_mod, oracle_mod):
+    """Two calls in a row with different masks and inputs: each result against
+    bsa_fwd_with_mask (same tolerance as every attention test) and, as an
+    independent check, against the fp64 oracle on every row."""
     import torch
     B, H, nb, d = 1, 6, 96, 128
     S = 64 * nb
@@ -71,6 +93,8 @@ def test_static_scratch_matches_workspace_entry_point_twice(nl, synth_mod):
         ref_o = o_w.double().cpu().numpy().reshape(-1, d)
         ref_l = lse_w.double().cpu().numpy().reshape(-1)
         compare_attention(go, gl, ref_o, ref_l)
+        ro, rl = oracle_mod.masked_attention(q16, k16, v16, mask_np)
+        compare_attention(go, gl, ro, rl)
 
 
 @pytest.mark.gpu
