@@ -97,71 +97,78 @@ __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restri
 }
 
 // ------------------------------------------------------------------ reduced map
-// Per head: L = Qbar Kbar^T * inv_sqrt_d in fp64.  128x128 output tile per CTA
-// of 256 threads; each thread owns rows {2ty, 2ty+1} + 32i and columns
-// {2tx, 2tx+1} + 32j (i, j < 4), so its shared-memory reads are 16-byte
-// vectors that are broadcast (A) or contiguous across the half-warp (B).
-// k is staged in chunks of 16 through two shared-memory stages, the next
+// Per head: L = Qbar Kbar^T * inv_sqrt_d in fp64.  A 64 x 128 output tile per
+// CTA of 128 threads (two CTAs share an SM, so one CTA's barrier waits and
+// loads overlap the other's multiplies); each thread owns rows {2ty, 2ty+1} +
+// 16i and columns {2tx, 2tx+1} + 32j (i, j < 4), so its shared-memory reads are
+// 16-byte vectors that are broadcast (A) or contiguous across the half-warp
+// (B).  k is staged in chunks of 16 through two shared-memory stages, the next
 // chunk's global loads in flight while the current one is multiplied.  Every
 // element is one fixed-order FMA chain.
-constexpr int kLgT = 128, kLgK = 16, kLgLD = kLgT + 2;
-constexpr int kLgBuf = kLgK * kLgLD;                       // doubles per operand buffer
-constexpr size_t kLgSmem = 2ull * 2 * kLgBuf * sizeof(double);   // 2 stages x (A, B)
+constexpr int kLgTM = 64, kLgTN = 128, kLgK = 16, kLgThreads = 128;
+constexpr int kLgLdA = kLgTM + 2, kLgLdB = kLgTN + 2;
+constexpr int kLgBufA = kLgK * kLgLdA, kLgBufB = kLgK * kLgLdB;   // doubles per operand buffer
+constexpr size_t kLgSmem = 2ull * (kLgBufA + kLgBufB) * sizeof(double);   // 2 stages x (A, B)
+constexpr int kLgPerA = kLgTM * kLgK / kLgThreads, kLgPerB = kLgTN * kLgK / kLgThreads;
 
 template <int D>
-__global__ void __launch_bounds__(256) logits_kernel(const double* __restrict__ qbar,
-                                                     const double* __restrict__ kbar,
-                                                     double* __restrict__ L, int nb,
-                                                     double inv_sqrt_d) {
-  extern __shared__ double lg_smem[];   // [stage][A | B][kLgK][kLgLD]; As[k][m], Bs[k][n]
+__global__ void __launch_bounds__(kLgThreads, 2) logits_kernel(const double* __restrict__ qbar,
+                                                              const double* __restrict__ kbar,
+                                                              double* __restrict__ L, int nb,
+                                                              double inv_sqrt_d) {
+  extern __shared__ double lg_smem[];   // [stage][A [kLgK][kLgLdA] | B [kLgK][kLgLdB]]
   const int bh = blockIdx.z;
-  const int m0 = blockIdx.y * kLgT, n0 = blockIdx.x * kLgT;
+  const int m0 = blockIdx.y * kLgTM, n0 = blockIdx.x * kLgTN;
   const double* qa = qbar + static_cast<int64_t>(bh) * nb * D;
   const double* ka = kbar + static_cast<int64_t>(bh) * nb * D;
   const int tid = threadIdx.x, ty = tid / 16, tx = tid % 16;
-  // each thread moves 8 elements of A and 8 of B per k-chunk; consecutive
-  // threads take consecutive k of one row (coalesced 128-byte rows)
-  double ra[8], rb[8];
-  auto fetch = [&](int kc) {
+  // the next chunk is copied straight into its shared-memory stage by 8-byte
+  // asynchronous copies (consecutive threads take consecutive k of one row:
+  // coalesced 128-byte rows); rows past nb are zero-filled
+  auto fetch = [&](int kc, int st) {
+    double* As = lg_smem + st * (kLgBufA + kLgBufB);
+    double* Bs = As + kLgBufA;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int i = tid + j * 256, r = i / kLgK, kk = i % kLgK;
-      ra[j] = (m0 + r < nb) ? qa[static_cast<int64_t>(m0 + r) * D + kc + kk] : 0.0;
-      rb[j] = (n0 + r < nb) ? ka[static_cast<int64_t>(n0 + r) * D + kc + kk] : 0.0;
+    for (int j = 0; j < kLgPerA; ++j) {
+      const int i = tid + j * kLgThreads, r = i / kLgK, kk = i % kLgK;
+      const bool in = m0 + r < nb;
+      const double* src = qa + static_cast<int64_t>(in ? m0 + r : 0) * D + kc + kk;
+      asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;" ::"r"(smem_addr(&As[kk * kLgLdA + r])),
+                   "l"(src), "r"(in ? 8 : 0) : "memory");
     }
-  };
-  auto stash = [&](int st) {
-    double* As = lg_smem + st * 2 * kLgBuf;
-    double* Bs = As + kLgBuf;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int i = tid + j * 256, r = i / kLgK, kk = i % kLgK;
-      As[kk * kLgLD + r] = ra[j];
-      Bs[kk * kLgLD + r] = rb[j];
+    for (int j = 0; j < kLgPerB; ++j) {
+      const int i = tid + j * kLgThreads, r = i / kLgK, kk = i % kLgK;
+      const bool in = n0 + r < nb;
+      const double* src = ka + static_cast<int64_t>(in ? n0 + r : 0) * D + kc + kk;
+      asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;" ::"r"(smem_addr(&Bs[kk * kLgLdB + r])),
+                   "l"(src), "r"(in ? 8 : 0) : "memory");
     }
+    asm volatile("cp.async.commit_group;" ::: "memory");
   };
   double acc[8][8];
 #pragma unroll
   for (int i = 0; i < 8; ++i)
 #pragma unroll
     for (int j = 0; j < 8; ++j) acc[i][j] = 0.0;
-  fetch(0);
-  stash(0);
-  __syncthreads();
   constexpr int kChunks = D / kLgK;
+  fetch(0, 0);
 #pragma unroll 1
   for (int ch = 0; ch < kChunks; ++ch) {
     const int st = ch & 1;
-    if (ch + 1 < kChunks) fetch((ch + 1) * kLgK);   // in flight during the FMAs below
-    const double* As = lg_smem + st * 2 * kLgBuf;
-    const double* Bs = As + kLgBuf;
+    // chunk ch landed (this thread's copies), then every thread's
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
+    __syncthreads();
+    if (ch + 1 < kChunks) fetch((ch + 1) * kLgK, st ^ 1);   // in flight during the FMAs below
+    const double* As = lg_smem + st * (kLgBufA + kLgBufB);
+    const double* Bs = As + kLgBufA;
 #pragma unroll
     for (int kk = 0; kk < kLgK; ++kk) {
       double a[8], b[8];
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const double2 va = *reinterpret_cast<const double2*>(&As[kk * kLgLD + 2 * ty + 32 * i]);
-        const double2 vb = *reinterpret_cast<const double2*>(&Bs[kk * kLgLD + 2 * tx + 32 * i]);
+        const double2 va = *reinterpret_cast<const double2*>(&As[kk * kLgLdA + 2 * ty + 16 * i]);
+        const double2 vb = *reinterpret_cast<const double2*>(&Bs[kk * kLgLdB + 2 * tx + 32 * i]);
         a[2 * i] = va.x; a[2 * i + 1] = va.y;
         b[2 * i] = vb.x; b[2 * i + 1] = vb.y;
       }
@@ -170,50 +177,57 @@ __global__ void __launch_bounds__(256) logits_kernel(const double* __restrict__ 
 #pragma unroll
         for (int j = 0; j < 8; ++j) acc[i][j] = fma(a[i], b[j], acc[i][j]);
     }
-    if (ch + 1 < kChunks) stash(st ^ 1);
-    __syncthreads();
   }
   double* out = L + static_cast<int64_t>(bh) * nb * nb;
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    const int m = m0 + 2 * ty + 32 * (i >> 1) + (i & 1);
+    const int m = m0 + 2 * ty + 16 * (i >> 1) + (i & 1);
     if (m >= nb) continue;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int n = n0 + 2 * tx + 32 * (j >> 1) + (j & 1);
-      if (n < nb) out[static_cast<int64_t>(m) * nb + n] = acc[i][j] * inv_sqrt_d;
+    for (int j = 0; j < 8; j += 2) {
+      const int n = n0 + 2 * tx + 32 * (j >> 1);
+      double* dst = out + static_cast<int64_t>(m) * nb + n;
+      if (n + 1 < nb && (nb & 1) == 0) {
+        *reinterpret_cast<double2*>(dst) = make_double2(acc[i][j] * inv_sqrt_d, acc[i][j + 1] * inv_sqrt_d);
+      } else {
+        if (n < nb) dst[0] = acc[i][j] * inv_sqrt_d;
+        if (n + 1 < nb) dst[1] = acc[i][j + 1] * inv_sqrt_d;
+      }
     }
   }
 }
 
 // ------------------------------------------------------------------ selection
 //
-// One CTA of 128 threads per row g = bh*nb + r.  The row's probabilities are formed in fp64
-// as the rule states them (p = exp(L - max) / sum over the row, or w / sum for
-// given non-negative weights) and kept in shared memory.  The kept set is the
-// smallest prefix of the row sorted by p descending (equal p: lower block index
-// first) whose exclusive prefix mass stays below 1 - thr, the first entry
-// always kept.  It is found without sorting the row:
-//   - masses are fixed-point integers F = round(p * 2^62), so every partial sum
-//     is exact and the same in any summation order;
+// One CTA of 128 threads per row g = bh*nb + r.  The row's weights are formed
+// in fp64 as the rule states them: v = exp(L - max) (the softmax numerators;
+// p = v / z with z their sum), or given non-negative weights v (p = v / z).
+// The kept set is the smallest prefix of the row sorted by p descending (equal
+// p: lower block index first) whose exclusive prefix mass stays below 1 - thr,
+// the first entry always kept.  It is found without sorting the row:
+//   - masses are fixed-point integers F = round(v * 2^50 / vmax), so every
+//     partial sum is exact and the same in any summation order, and the target
+//     is F((1 - thr) * z); comparing sums of v with (1 - thr) * z is the rule
+//     E_k < 1 - thr multiplied through by z;
 //   - the value range [lo, hi] of the candidates (at first the whole row) is
 //     split into 256 equal bins, a monotone map, so the bins are ordered
-//     intervals of p; the candidates' masses and counts are histogrammed with
-//     shared-memory integer atomics; a scan from the top bin finds the bin in
-//     which the cumulative mass reaches the target; entries of higher bins are
-//     kept, of lower bins dropped, and the crossing bin's entries are the next
-//     candidates (their range is the next level's [lo, hi]);
-//   - once at most 32 candidates remain one warp sorts them exactly on
-//     (p desc, block index asc) by a bitonic network, and each one's
-//     exclusive prefix mass decides it; candidates that all share one p are
+//     intervals of v; the candidates' masses and counts are histogrammed with
+//     shared-memory integer atomics (in the same pass that forms v at the first
+//     level); a scan from the top bin finds the bin in which the cumulative mass
+//     reaches the target; entries of higher bins are kept, of lower bins
+//     dropped, and the crossing bin's entries are the next candidates (their
+//     range is the next level's [lo, hi]);
+//   - once at most 32 candidates remain one warp orders them exactly on
+//     (p = v / z desc, block index asc) by a bitonic network, and each one's
+//     exclusive prefix mass decides it; candidates that all share one value are
 //     taken in block order.
 // Top-k mode does the same with a count of 1 per entry as the mass and k as
-// the target.  Everything is integer or exact comparison after p is formed,
-// so the kept set is the one a sort by p and an exact cumulative sum give.
+// the target.  The sliding-tile window is OR-ed in as one run of columns per
+// (t, h) row of the window.
 
 constexpr int kSelBins = 256;
-constexpr double kSelFix = 4611686018427387904.0;   // 2^62, scale of the fixed-point masses
-constexpr int kSelMaxLevels = 16;                    // binning levels (8 always suffice for fp64)
+constexpr double kSelFix = 1125899906842624.0;   // 2^50: mass of the row's largest entry
+constexpr int kSelMaxLevels = 16;                // binning levels (8 always suffice for fp64)
 
 struct SelectParams {
   float thr;
@@ -222,15 +236,14 @@ struct SelectParams {
   int topk;        // > 0: keep the topk most probable blocks instead of the mass rule
 };
 
-// Shared memory of one row: p [nb] fp64, candidate list [nb] u16, keep bitmap
-// [nw] u32, bin masses [256] u64, bin counts [256] u32, and a small exchange
-// area for the CTA's reductions (8-byte aligned parts).
+// Shared memory of one row: v [nb] fp64, keep and candidate bitmaps [nw] u32
+// each, bin masses [256] u64, bin counts [256] u32, and a small exchange area
+// for the CTA's reductions and the last candidates (8-byte aligned parts).
 constexpr int kSelThreads = 128, kSelWarps = kSelThreads / 32;
-constexpr size_t kSelXchBytes = 8 * 4 * kSelWarps + 64;
+constexpr size_t kSelXchBytes = 8 * 8 * kSelWarps + 64 + 4 * 32 + 4 * 132;
 __host__ __device__ inline size_t select_row_bytes(int nb) {
-  const size_t n = static_cast<size_t>(nb), nw = (n + 31) / 32;
-  return 8 * n + ((2 * n + 7) & ~static_cast<size_t>(7)) + 4 * ((nw + 1) & ~static_cast<size_t>(1)) +
-         12 * static_cast<size_t>(kSelBins) + kSelXchBytes;
+  const size_t n = static_cast<size_t>(nb), nw2 = ((n + 31) / 32 + 1) & ~static_cast<size_t>(1);
+  return 8 * n + 8 * nw2 + 12 * static_cast<size_t>(kSelBins) + kSelXchBytes;
 }
 
 __device__ __forceinline__ double warp_sum(double v) {
@@ -257,47 +270,18 @@ __device__ __forceinline__ unsigned long long warp_sum_u64(unsigned long long v)
   return v;
 }
 
-// CTA-wide reductions in a fixed order (every thread gets the same value): the
-// warps reduce, warp w posts to slot w of xch, and every thread combines the
-// slots in warp order.  op 0: sum, 1: max, 2: min.
-template <int kOp>
-__device__ __forceinline__ double cta_reduce(double v, double* xch, int warp, int lane) {
-  v = kOp == 0 ? warp_sum(v) : (kOp == 1 ? warp_max(v) : warp_min(v));
-  if (lane == 0) xch[warp] = v;
-  __syncthreads();
-  double r = xch[0];
-#pragma unroll
-  for (int w = 1; w < kSelWarps; ++w) r = kOp == 0 ? r + xch[w] : (kOp == 1 ? fmax(r, xch[w]) : fmin(r, xch[w]));
-  __syncthreads();
-  return r;
+// Bin of v in [lo, hi] split into kSelBins equal parts (s = kSelBins / (hi - lo)).
+__device__ __forceinline__ int sel_bin(double v, double lo, double s) {
+  return static_cast<int>(fmin((v - lo) * s, static_cast<double>(kSelBins - 1)));
 }
 
-__device__ __forceinline__ unsigned long long cta_sum_u64(unsigned long long v,
-                                                          unsigned long long* xch, int warp,
-                                                          int lane) {
-  v = warp_sum_u64(v);
-  if (lane == 0) xch[warp] = v;
-  __syncthreads();
-  unsigned long long r = 0;
-#pragma unroll
-  for (int w = 0; w < kSelWarps; ++w) r += xch[w];
-  __syncthreads();
-  return r;
-}
-
-__device__ __forceinline__ unsigned long long sel_fix(double p) {
-  return __double2ull_rn(p * kSelFix);   // p in [0, 1]: at most 2^62
-}
-
-// Bin of p in [lo, hi] split into kSelBins equal parts (s = kSelBins / (hi - lo)).
-__device__ __forceinline__ int sel_bin(double p, double lo, double s) {
-  return static_cast<int>(fmin((p - lo) * s, static_cast<double>(kSelBins - 1)));
-}
-
-// q = a / b for 0 <= a < 4096, 1 <= b <= 4096: (a + 0.5) / b lies at least
-// 0.5 / b from an integer, far more than the fp32 error of the product.
-__device__ __forceinline__ int sel_div(int a, float inv_b) {
-  return __float2int_rz((static_cast<float>(a) + 0.5f) * inv_b);
+// Set bits [c0, c1] of a bitmap (shared memory, atomically).
+__device__ __forceinline__ void sel_set_run(uint32_t* bm, int c0, int c1) {
+  for (int w = c0 >> 5; w <= (c1 >> 5); ++w) {
+    const int lo = max(c0, w * 32) - w * 32, hi = min(c1, w * 32 + 31) - w * 32;
+    const uint32_t m = (hi == 31 ? 0xffffffffu : ((1u << (hi + 1)) - 1u)) & ~((1u << lo) - 1u);
+    atomicOr(&bm[w], m);
+  }
 }
 
 template <bool kWeights>
@@ -313,100 +297,140 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const void* __restr
   const int64_t g = blockIdx.x;
   if (g >= nrows) return;
   const unsigned full = 0xffffffffu;
-  const unsigned lt_mask = (1u << lane) - 1u;
   const int r = static_cast<int>(g % nb);
   const int nw = (nb + 31) >> 5;
+  const int nw2 = (nw + 1) & ~1;
   double* pv = reinterpret_cast<double*>(sel_smem);
-  uint16_t* list = reinterpret_cast<uint16_t*>(sel_smem + 8ull * nb);
-  uint32_t* kbits = reinterpret_cast<uint32_t*>(sel_smem + 8ull * nb + ((2ull * nb + 7) & ~7ull));
-  unsigned long long* hm =
-      reinterpret_cast<unsigned long long*>(reinterpret_cast<unsigned char*>(kbits) +
-                                            4ull * ((nw + 1) & ~1));
+  uint32_t* kbits = reinterpret_cast<uint32_t*>(sel_smem + 8ull * nb);   // kept entries
+  uint32_t* cbits = kbits + nw2;                                          // candidates
+  unsigned long long* hm = reinterpret_cast<unsigned long long*>(cbits + nw2);
   uint32_t* hc = reinterpret_cast<uint32_t*>(hm + kSelBins);
-  double* xd = reinterpret_cast<double*>(hc + kSelBins);                  // [kSelWarps]
-  unsigned long long* xu = reinterpret_cast<unsigned long long*>(xd + kSelWarps);   // [kSelWarps]
+  double* xd = reinterpret_cast<double*>(hc + kSelBins);                  // [2 * kSelWarps]
+  unsigned long long* xu = reinterpret_cast<unsigned long long*>(xd + 2 * kSelWarps);  // [kSelWarps]
   int* xi = reinterpret_cast<int*>(xu + kSelWarps);                       // [2 * kSelWarps]
   unsigned long long* xs = reinterpret_cast<unsigned long long*>(xi + 2 * kSelWarps);  // [4]
+  int* slot = reinterpret_cast<int*>(xs + 4);                             // [32] last candidates
+  int* wpre = slot + 32;                                                  // [nw + 1] word prefix
 
-  // ---- probabilities in fp64
-  bool empty_row = false;
-  double z;
-  if (kWeights) {
-    const float* W = static_cast<const float*>(in) + g * nb;
-    double zl = 0.0;
-    for (int c = tid; c < nb; c += kSelThreads) {
-      const float w = W[c];
-      const double x = w > 0.f ? static_cast<double>(w) : 0.0;   // negative or NaN count as zero
-      pv[c] = x;
-      zl += x;
-    }
-    z = cta_reduce<0>(zl, xd, warp, lane);
-    empty_row = !(z > 0.0);
-  } else {
-    const double* Lrow = static_cast<const double*>(in) + g * nb;
-    double mx = -INFINITY;
-    for (int c = tid; c < nb; c += kSelThreads) mx = fmax(mx, Lrow[c]);
-    mx = cta_reduce<1>(mx, xd, warp, lane);
-    double zl = 0.0;
-#pragma unroll 4
-    for (int c = tid; c < nb; c += kSelThreads) {
-      const double e = exp(Lrow[c] - mx);
-      pv[c] = e;
-      zl += e;
-    }
-    z = cta_reduce<0>(zl, xd, warp, lane);
-  }
-  double lo = INFINITY, hi = -INFINITY;
   const bool topk_mode = prm.topk > 0;
-  unsigned long long tot = 0;
-  if (!empty_row) {
-    for (int c = tid; c < nb; c += kSelThreads) {
-      const double p = pv[c] / z;
-      pv[c] = p;
-      lo = fmin(lo, p);
-      hi = fmax(hi, p);
-      tot += sel_fix(p);
-    }
-    lo = cta_reduce<2>(lo, xd, warp, lane);
-    hi = cta_reduce<1>(hi, xd, warp, lane);
-    if (!topk_mode) tot = cta_sum_u64(tot, xu, warp, lane);
+  const bool keep_all_rule = topk_mode ? prm.topk >= nb : prm.thr <= 0.f;
+  for (int w = tid; w < nw2; w += kSelThreads) {
+    kbits[w] = 0u;
+    cbits[w] = 0u;
   }
-  for (int w = tid; w < nw; w += kSelThreads) kbits[w] = 0u;
+  for (int i = tid; i < kSelBins; i += kSelThreads) {
+    hm[i] = 0ull;
+    hc[i] = 0u;
+  }
+
+  // ---- pass 1: range of the row (max and min of L, or of the weights)
+  const double* Lrow = static_cast<const double*>(in) + g * nb;
+  const float* Wrow = static_cast<const float*>(in) + g * nb;
+  double a = -INFINITY, b = INFINITY;
+  for (int c = tid; c < nb; c += kSelThreads) {
+    double x;
+    if (kWeights) {
+      const float w = Wrow[c];
+      x = w > 0.f ? static_cast<double>(w) : 0.0;   // negative or NaN weights count as zero
+      pv[c] = x;
+    } else {
+      x = Lrow[c];
+    }
+    a = fmax(a, x);
+    b = fmin(b, x);
+  }
+  a = warp_max(a);
+  b = warp_min(b);
+  if (lane == 0) {
+    xd[warp] = a;
+    xd[kSelWarps + warp] = b;
+  }
+  __syncthreads();
+  double vmax = xd[0], vmin = xd[kSelWarps];
+#pragma unroll
+  for (int w = 1; w < kSelWarps; ++w) {
+    vmax = fmax(vmax, xd[w]);
+    vmin = fmin(vmin, xd[kSelWarps + w]);
+  }
+  // logits: v = exp(L - max) lies in [exp(min - max), 1]
+  const double mx = vmax;
+  double lo = kWeights ? vmin : exp(vmin - mx);
+  double hi = kWeights ? vmax : 1.0;
+  const double sigma = kWeights ? (vmax > 0.0 ? kSelFix / vmax : 0.0) : kSelFix;
+
+  // ---- pass 2: v, its sum, the total mass, and the first level's histogram
+  const bool bin0 = !keep_all_rule && hi > lo;
+  const double s0 = bin0 ? fmin(kSelBins / (hi - lo), 1.7976931348623157e308) : 0.0;
+  double zl = 0.0;
+  unsigned long long tot = 0;
+  for (int c = tid; c < nb; c += kSelThreads) {
+    double v;
+    if (kWeights) {
+      v = pv[c];
+    } else {
+      v = exp(Lrow[c] - mx);
+      pv[c] = v;
+    }
+    zl += v;
+    const unsigned long long f = topk_mode ? 1ull : __double2ull_rn(v * sigma);
+    tot += f;
+    if (bin0) {
+      const int bb = sel_bin(v, lo, s0);
+      atomicAdd(&hm[bb], f);
+      atomicAdd(&hc[bb], 1u);
+    }
+  }
+  zl = warp_sum(zl);
+  tot = warp_sum_u64(tot);
+  __syncthreads();   // xd consumed
+  if (lane == 0) {
+    xd[warp] = zl;
+    xu[warp] = tot;
+  }
+  __syncthreads();
+  double z = xd[0];
+  tot = xu[0];
+#pragma unroll
+  for (int w = 1; w < kSelWarps; ++w) {
+    z += xd[w];
+    tot += xu[w];
+  }
+  const bool empty_row = kWeights && !(z > 0.0);
 
   // ---- the kept set (every branch below is uniform across the CTA)
-  bool keep_all = false;
+  bool keep_all = keep_all_rule;
   unsigned long long T = 0;   // target: fixed-point mass, or the count k
   if (topk_mode) {
-    keep_all = prm.topk >= nb;
     T = static_cast<unsigned long long>(prm.topk);
   } else {
-    keep_all = prm.thr <= 0.f;
     const double t = 1.0 - static_cast<double>(prm.thr);
-    T = t > 0.0 ? sel_fix(t) : 0ull;
+    T = t > 0.0 ? __double2ull_rn(t * z * sigma) : 0ull;
     // every exclusive prefix stays below the target when the whole row does
     if (!keep_all && !empty_row) keep_all = tot < T;
   }
-  __syncthreads();
   if (!keep_all && !empty_row) {
     unsigned long long above = 0;   // mass (or count) of the entries ranked above the candidates
     uint32_t above_n = 0;           // number of those entries
-    int n_c = nb;                   // candidates: every entry (implicit list) at level 0
-    bool implicit = true;
+    int n_c = nb;                   // candidates: every entry at level 0, then those of cbits
+    bool all = true;
+    // entry c = i0 + tid: warp w of a chunk owns bitmap word i0/32 + w
     for (int level = 0; level < kSelMaxLevels && n_c > 32 && hi > lo; ++level) {
-      const double s = fmin(kSelBins / (hi - lo), 1.7976931348623157e308);
-      for (int i = tid; i < kSelBins; i += kSelThreads) {
-        hm[i] = 0ull;
-        hc[i] = 0u;
+      const double sl = level == 0 ? s0 : fmin(kSelBins / (hi - lo), 1.7976931348623157e308);
+      if (level > 0) {
+        for (int i = tid; i < kSelBins; i += kSelThreads) {
+          hm[i] = 0ull;
+          hc[i] = 0u;
+        }
+        __syncthreads();
+        for (int c = tid; c < nb; c += kSelThreads) {
+          if (!((cbits[c >> 5] >> (c & 31)) & 1u)) continue;
+          const double v = pv[c];
+          const int bb = sel_bin(v, lo, sl);
+          atomicAdd(&hm[bb], topk_mode ? 1ull : __double2ull_rn(v * sigma));
+          atomicAdd(&hc[bb], 1u);
+        }
+        __syncthreads();
       }
-      __syncthreads();
-      for (int i = tid; i < n_c; i += kSelThreads) {
-        const int c = implicit ? i : list[i];
-        const double p = pv[c];
-        const int b = sel_bin(p, lo, s);
-        atomicAdd(&hm[b], topk_mode ? 1ull : sel_fix(p));
-        atomicAdd(&hc[b], 1u);
-      }
-      __syncthreads();
       if (warp == 0) {
         // lane l holds bins [8l, 8l+8); suffix sums over lanes >= l (inclusive)
         unsigned long long loc = 0;
@@ -434,84 +458,114 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const void* __restr
         if (lane == cl) {
           unsigned long long run = above + (suf - loc);
           uint32_t runn = above_n + (sufn - locn);
-          int b = 8 * lane + 7;
-          for (; b > 8 * lane; --b) {
-            if (run + hm[b] >= T) break;
-            run += hm[b];
-            runn += hc[b];
+          int bb = 8 * lane + 7;
+          for (; bb > 8 * lane; --bb) {
+            if (run + hm[bb] >= T) break;
+            run += hm[bb];
+            runn += hc[bb];
           }
-          xi[0] = b;
-          xi[1] = static_cast<int>(hc[b]);
+          xi[0] = bb;
+          xi[1] = static_cast<int>(hc[bb]);
           xs[0] = run;
           xs[1] = runn;
         }
       }
       __syncthreads();
-      const int bstar = xi[0], nb_star = xi[1];
+      const int bstar = xi[0];
       above = xs[0];
       above_n = static_cast<uint32_t>(xs[1]);
-      // keep the higher bins, carry the crossing bin's entries (stable order)
-      int kept_n = 0;
+      // keep the higher bins; the crossing bin's entries are the next candidates
       double nlo = INFINITY, nhi = -INFINITY;
-      for (int i0 = 0; i0 < n_c; i0 += kSelThreads) {
-        const int i = i0 + tid;
-        int c = -1, b = -1;
-        double p = 0.0;
-        if (i < n_c) {
-          c = implicit ? i : list[i];
-          p = pv[c];
-          b = sel_bin(p, lo, s);
+      for (int i0 = 0; i0 < nb; i0 += kSelThreads) {
+        const int c = i0 + tid;
+        const int w = c >> 5;
+        bool cand = false, keep = false;
+        if (c < nb && (all || ((cbits[w] >> lane) & 1u))) {
+          const double v = pv[c];
+          const int bb = sel_bin(v, lo, sl);
+          keep = bb > bstar;
+          cand = bb == bstar;
+          if (cand) {
+            nlo = fmin(nlo, v);
+            nhi = fmax(nhi, v);
+          }
         }
-        if (implicit) {   // entry c = i: warp w of the chunk fills one bitmap word
-          const uint32_t kb = __ballot_sync(full, b > bstar);
-          if (lane == 0 && kb) kbits[i >> 5] |= kb;
-        } else if (b > bstar) {
-          atomicOr(&kbits[c >> 5], 1u << (c & 31));
+        const uint32_t kb = __ballot_sync(full, keep), cb = __ballot_sync(full, cand);
+        if (lane == 0 && w < nw) {
+          kbits[w] |= kb;
+          cbits[w] = cb;
         }
-        const bool nxt = b == bstar;
-        const uint32_t bn = __ballot_sync(full, nxt);
-        if (lane == 0) xi[2 + warp] = __popc(bn);
-        __syncthreads();   // every element of this chunk has been read
-        int before = kept_n;
-        for (int w = 0; w < warp; ++w) before += xi[2 + w];
-        if (nxt) {
-          list[before + __popc(bn & lt_mask)] = static_cast<uint16_t>(c);
-          nlo = fmin(nlo, p);
-          nhi = fmax(nhi, p);
-        }
-        for (int w = 0; w < kSelWarps; ++w) kept_n += xi[2 + w];
-        __syncthreads();   // counts consumed before the next chunk posts its own
       }
-      n_c = nb_star;
-      implicit = false;
-      lo = cta_reduce<2>(nlo, xd, warp, lane);
-      hi = cta_reduce<1>(nhi, xd, warp, lane);
+      n_c = xi[1];
+      all = false;
+      nlo = warp_min(nlo);
+      nhi = warp_max(nhi);
+      __syncthreads();   // xi, xs consumed; cbits and kbits written
+      if (lane == 0) {
+        xd[warp] = nlo;
+        xd[kSelWarps + warp] = nhi;
+      }
+      __syncthreads();
+      lo = xd[0];
+      hi = xd[kSelWarps];
+#pragma unroll
+      for (int w = 1; w < kSelWarps; ++w) {
+        lo = fmin(lo, xd[w]);
+        hi = fmax(hi, xd[kSelWarps + w]);
+      }
     }
     if (n_c <= 32) {
       if (warp == 0) {
-        // exact order of the last candidates: bitonic network on (p desc, index asc)
-        const int c = lane < n_c ? (implicit ? lane : static_cast<int>(list[lane])) : -1;
+        // gather the candidates (ascending index) into slot[0 .. n_c)
+        int base = 0;
+        for (int w0 = 0; w0 < nw; w0 += 32) {
+          const int w = w0 + lane;
+          uint32_t bitsw = 0u;
+          if (w < nw)
+            bitsw = all ? ((w == nw - 1 && (nb & 31)) ? (1u << (nb & 31)) - 1u : full) : cbits[w];
+          const int cnt = __popc(bitsw);
+          int incl = cnt;
+#pragma unroll
+          for (int off = 1; off < 32; off <<= 1) {
+            const int y = __shfl_up_sync(full, incl, off);
+            if (lane >= off) incl += y;
+          }
+          int pos = base + incl - cnt;
+          while (bitsw) {
+            const int bit = __ffs(bitsw) - 1;
+            bitsw &= bitsw - 1;
+            if (pos < 32) slot[pos] = w * 32 + bit;
+            ++pos;
+          }
+          base += __shfl_sync(full, incl, 31);
+        }
+        __syncwarp();
+        // exact order of the last candidates: bitonic network on
+        // (p = v / z desc, index asc); masses from v
+        const int c = lane < n_c ? slot[lane] : -1;
+        const double v = c >= 0 ? pv[c] : 0.0;
         unsigned long long key =
-            c >= 0 ? static_cast<unsigned long long>(__double_as_longlong(pv[c])) : 0ull;
+            c >= 0 ? static_cast<unsigned long long>(__double_as_longlong(v / z)) : 0ull;
+        unsigned long long f =
+            c >= 0 ? (topk_mode ? 1ull : __double2ull_rn(v * sigma)) : 0ull;
         int idx = c >= 0 ? c : 0x7fffffff;
 #pragma unroll
         for (int k = 2; k <= 32; k <<= 1) {
 #pragma unroll
           for (int j = k >> 1; j > 0; j >>= 1) {
             const unsigned long long ok = __shfl_xor_sync(full, key, j);
+            const unsigned long long of = __shfl_xor_sync(full, f, j);
             const int oi = __shfl_xor_sync(full, idx, j);
             const bool other_first = ok > key || (ok == key && oi < idx);
             const bool lower = (lane & j) == 0, up = (lane & k) == 0;
             if ((lower == up) ? other_first : !other_first) {
               key = ok;
+              f = of;
               idx = oi;
             }
           }
         }
         const bool valid = idx != 0x7fffffff;
-        const unsigned long long f =
-            valid ? (topk_mode ? 1ull : sel_fix(__longlong_as_double(static_cast<long long>(key))))
-                  : 0ull;
         unsigned long long incl = f;
 #pragma unroll
         for (int off = 1; off < 32; off <<= 1) {
@@ -522,53 +576,87 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const void* __restr
         if (keep) atomicOr(&kbits[idx >> 5], 1u << (idx & 31));
       }
     } else {
-      // the candidates share one p (or the level cap was reached): block order
-      const int c0 = implicit ? 0 : static_cast<int>(list[0]);
-      const unsigned long long f = topk_mode ? 1ull : sel_fix(pv[c0]);
+      // the candidates share one value (or the level cap was reached): the
+      // first nkeep of them in block order
+      if (warp == 0) {
+        // exclusive prefix of candidate counts over the words, and the first candidate
+        int base = 0, first = 0x7fffffff;
+        for (int w0 = 0; w0 < nw; w0 += 32) {
+          const int w = w0 + lane;
+          const uint32_t bitsw = w < nw ? cbits[w] : 0u;
+          if (bitsw) first = min(first, w * 32 + __ffs(bitsw) - 1);
+          const int cnt = __popc(bitsw);
+          int incl = cnt;
+#pragma unroll
+          for (int off = 1; off < 32; off <<= 1) {
+            const int y = __shfl_up_sync(full, incl, off);
+            if (lane >= off) incl += y;
+          }
+          if (w < nw) wpre[w] = base + incl - cnt;
+          base += __shfl_sync(full, incl, 31);
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) first = min(first, __shfl_xor_sync(full, first, off));
+        if (lane == 0) xi[0] = all ? 0 : first;
+      }
+      __syncthreads();
+      const int c0 = xi[0];
+      const unsigned long long f = topk_mode ? 1ull : __double2ull_rn(pv[c0] * sigma);
       int nkeep = 0;
       if (above < T) {
         const unsigned long long need = (T - above + f - 1) / (f > 0 ? f : 1ull);
         nkeep = (f == 0 || need >= static_cast<unsigned long long>(n_c)) ? n_c : static_cast<int>(need);
       }
       if (above_n == 0 && nkeep == 0) nkeep = 1;
-      for (int i = tid; i < nkeep; i += kSelThreads) {
-        const int c = implicit ? i : static_cast<int>(list[i]);
-        atomicOr(&kbits[c >> 5], 1u << (c & 31));
+      for (int c = tid; c < nb; c += kSelThreads) {
+        const int w = c >> 5;
+        bool take;
+        if (all) {
+          take = c < nkeep;
+        } else {
+          const uint32_t bitsw = cbits[w];
+          take = ((bitsw >> (c & 31)) & 1u) && wpre[w] + __popc(bitsw & ((1u << (c & 31)) - 1u)) < nkeep;
+        }
+        if (take) atomicOr(&kbits[w], 1u << (c & 31));
       }
     }
+  } else if (keep_all && !empty_row) {
+    for (int w = tid; w < nw; w += kSelThreads)
+      kbits[w] = (w == nw - 1 && (nb & 31)) ? (1u << (nb & 31)) - 1u : full;
   }
   __syncthreads();
 
-  // ---- flags -> bitmap words, optional uint8 row, STA union, votes, count
-  const float inv_tw = 1.0f / static_cast<float>(prm.Tw);
-  const float inv_thw = 1.0f / static_cast<float>(prm.Th * prm.Tw);
-  int rt = 0, rh = 0, rw = 0;
+  // ---- the sliding-tile window: one run of columns per (t, h) of the window
   if (prm.use_sta) {
-    rt = sel_div(r, inv_thw);
-    const int rr = r - rt * prm.Th * prm.Tw;
-    rh = sel_div(rr, inv_tw);
-    rw = rr - rh * prm.Tw;
-  }
-  int count = 0;
-  uint32_t* brow = bits ? bits + g * nw : nullptr;
-  uint8_t* mrow = mask_u8 ? mask_u8 + g * nb : nullptr;
-  for (int w = warp; w < nw; w += kSelWarps) {
-    const int c = w * 32 + lane;
-    const bool inrow = c < nb;
-    bool keep = inrow && !empty_row && (keep_all || ((kbits[w] >> lane) & 1u) != 0u);
-    if (inrow && prm.use_sta) {
-      const int ct = sel_div(c, inv_thw);
-      const int cc = c - ct * prm.Th * prm.Tw;
-      const int ch = sel_div(cc, inv_tw);
-      const int cw = cc - ch * prm.Tw;
-      keep |= abs(ct - rt) <= prm.wt && abs(ch - rh) <= prm.wh && abs(cw - rw) <= prm.ww;
+    const int thw = prm.Th * prm.Tw;
+    const int rt = r / thw, rh = (r / prm.Tw) % prm.Th, rw = r % prm.Tw;
+    const int nh = 2 * prm.wh + 1, nrun = (2 * prm.wt + 1) * nh;
+    const int w0 = max(rw - prm.ww, 0), w1 = min(rw + prm.ww, prm.Tw - 1);
+    for (int j = tid; j < nrun; j += kSelThreads) {
+      const int t = rt - prm.wt + j / nh, h = rh - prm.wh + j % nh;
+      if (t < 0 || t >= prm.Tt || h < 0 || h >= prm.Th) continue;
+      const int base = (t * prm.Th + h) * prm.Tw;
+      sel_set_run(kbits, base + w0, base + w1);
     }
-    if (mrow && inrow) mrow[c] = keep ? 1 : 0;
-    if (votes && keep) votes[g * nb + c] += 1;
-    const uint32_t word = __ballot_sync(full, keep);
-    if (brow && lane == 0) brow[w] = word;
+    __syncthreads();
+  }
+
+  // ---- outputs: bitmap words, count, optional uint8 row and votes
+  int count = 0;
+  for (int w = tid; w < nw; w += kSelThreads) {
+    const uint32_t word = kbits[w];
+    if (bits) bits[g * nw + w] = word;
     count += __popc(word);
   }
+  if (mask_u8 || votes) {
+    for (int c = tid; c < nb; c += kSelThreads) {
+      const bool keep = (kbits[c >> 5] >> (c & 31)) & 1u;
+      if (mask_u8) mask_u8[g * nb + c] = keep ? 1 : 0;
+      if (votes && keep) votes[g * nb + c] += 1;
+    }
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) count += __shfl_xor_sync(full, count, off);
   if (lane == 0) xi[2 + warp] = count;
   __syncthreads();
   if (counts && tid == 0) {
@@ -709,19 +797,19 @@ cudaError_t launch_pool(const void* q, const void* k, double* qbar, double* kbar
 
 cudaError_t launch_logits(const double* qbar, const double* kbar, double* L, int BH, int nb,
                           int d, cudaStream_t st) {
-  const dim3 grid((nb + kLgT - 1) / kLgT, (nb + kLgT - 1) / kLgT, BH);
+  const dim3 grid((nb + kLgTN - 1) / kLgTN, (nb + kLgTM - 1) / kLgTM, BH);
   const double inv = 1.0 / sqrt(static_cast<double>(d));
   cudaError_t e;
   if (d == 128) {
     e = cudaFuncSetAttribute(logits_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(kLgSmem));
     if (e != cudaSuccess) return e;
-    logits_kernel<128><<<grid, 256, kLgSmem, st>>>(qbar, kbar, L, nb, inv);
+    logits_kernel<128><<<grid, kLgThreads, kLgSmem, st>>>(qbar, kbar, L, nb, inv);
   } else {
     e = cudaFuncSetAttribute(logits_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(kLgSmem));
     if (e != cudaSuccess) return e;
-    logits_kernel<64><<<grid, 256, kLgSmem, st>>>(qbar, kbar, L, nb, inv);
+    logits_kernel<64><<<grid, kLgThreads, kLgSmem, st>>>(qbar, kbar, L, nb, inv);
   }
   return cudaGetLastError();
 }
