@@ -36,7 +36,7 @@ EXPORTED = ["nabla_workspace_size", "nabla_workspace_init", "nabla_query_status"
             "nabla_calib_accumulate", "nabla_calib_finalize", "bsa_bwd",
             "nabla_build_mask_xattn", "nabla_layer_host_workspace_size", "nabla_layer_host",
             "nabla_layer_host_chunks", "nabla_set_exact_reference", "nabla_query_exact_passes",
-            "nabla_build_mask_stage_ms", "nabla_selftest_fp64_tflops"]
+            "nabla_build_mask_stage_ms", "nabla_selftest_fp64_tflops", "nabla_selftest_mma_pair"]
 TO_TILE_MAJOR, TO_RASTER = 0, 1
 
 
@@ -125,6 +125,8 @@ def lib() -> ctypes.CDLL:
             L.nabla_build_mask_stage_ms.restype = i32
             L.nabla_build_mask_stage_ms.argtypes = [sp, ctypes.POINTER(_MaskParams), vp, vp, vp,
                                                     vp, ctypes.c_int64, vp, vp, vp, vp]
+            L.nabla_selftest_mma_pair.restype = i32
+            L.nabla_selftest_mma_pair.argtypes = [i32, vp, vp, vp, vp, vp]
             L.nabla_selftest_fp64_tflops.restype = i32
             L.nabla_selftest_fp64_tflops.argtypes = [vp, vp]
             L.nabla_layer_host.restype = i32
@@ -352,6 +354,19 @@ def selftest_mma(variant: int, a, b, workspace: Optional[Workspace] = None, stre
     c = torch.empty((128, 128), dtype=torch.float32, device=a.device)
     _check(lib().nabla_selftest_mma(int(variant), _ptr(a), _ptr(b), _ptr(c), _ptr(workspace.buf),
                                     _stream(stream)))
+    workspace.check(stream)
+    return c
+
+
+def selftest_mma_pair(variant: int, a, b, workspace: Optional[Workspace] = None, stream=None):
+    """One product over a pair of CTAs (layout check); returns C fp32
+    [256,256] (variant 0: A B^T) or [256,128] (variant 1: P V)."""
+    torch = _torch()
+    if workspace is None:
+        workspace = Workspace.create(make_shape(1, 1, 64, 64), OP_FWD, a.device, stream)
+    c = torch.empty((256, 256 if variant == 0 else 128), dtype=torch.float32, device=a.device)
+    _check(lib().nabla_selftest_mma_pair(int(variant), _ptr(a), _ptr(b), _ptr(c),
+                                         _ptr(workspace.buf), _stream(stream)))
     workspace.check(stream)
     return c
 

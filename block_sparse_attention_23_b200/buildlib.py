@@ -13,7 +13,7 @@ CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libnabla.so")
 SOURCES = ["nabla_api.cu", "mask_kernels.cu", "attn_kernel.cu", "nabla_noalloc.cu",
            "reorder_kernels.cu", "energy_kernel.cu", "bwd_kernel.cu",
-           "xattn_kernel.cu", "nabla_host.cu", "nabla_diag.cu"]
+           "xattn_kernel.cu", "nabla_host.cu", "nabla_diag.cu", "attn2_kernel.cu"]
 HEADERS = ["sm100_primitives.cuh", os.path.join("..", "..", "include", "nabla.h")]
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
               "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden", "--expt-relaxed-constexpr",

@@ -59,6 +59,9 @@ cudaError_t launch_select_weights(const float* weights, int64_t nrows, int nb, f
 cudaError_t launch_xattn_scores(const CUtensorMap& q, const CUtensorMap& k, float* lse2,
                                 float* scores, int* status, int BH, int S, int d, int St,
                                 uint64_t wait_limit_ns, cudaStream_t st);
+cudaError_t launch_mma_pair_selftest(const CUtensorMap& a, const CUtensorMap& b,
+                                     const void* p_glob, float* c, int variant, int* status,
+                                     uint64_t lim, cudaStream_t st);
 cudaError_t launch_mma_selftest(const CUtensorMap& a, const CUtensorMap& b, const void* a_glob,
                                 float* c, int variant, int* status, uint64_t lim,
                                 cudaStream_t st);
@@ -783,6 +786,24 @@ nabla_status nabla_selftest_mma(int variant, const void* a, const void* b, float
                                              g_wait_limit_ns.load(),
                                              reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "selftest launch");
+  return NABLA_OK;
+}
+
+nabla_status nabla_selftest_mma_pair(int variant, const void* a, const void* b, float* c,
+                                     void* workspace, nabla_stream_t stream) {
+  if (variant < 0 || variant > 1) return fail(NABLA_ERR_INVALID_ARG, "variant must be 0 or 1");
+  if (!a || !b || !c || !workspace) return fail(NABLA_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(a) || !aligned16(b)) return fail(NABLA_ERR_INVALID_ARG, "a, b need 16-byte alignment");
+  CUtensorMap ma, mb;
+  nabla_status s;
+  // variant 0: A [256][128], B [256][128]; variant 1: P [256][256] (read by
+  // threads, not by a map), V [256][128]
+  if ((s = make_map(&ma, variant == 0 ? a : b, 256, 128)) != NABLA_OK) return s;
+  if ((s = make_map(&mb, b, 256, 128)) != NABLA_OK) return s;
+  cudaError_t e = nabla::launch_mma_pair_selftest(ma, mb, a, c, variant, status_ptr(workspace),
+                                                  g_wait_limit_ns.load(),
+                                                  reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "pair selftest launch");
   return NABLA_OK;
 }
 

@@ -396,6 +396,13 @@ NABLA_API int nabla_version(void);
  * forward workspace's header: how many forwards on it needed the
  * exact-reference kernel since nabla_workspace_init (-1 on a CUDA error).
  *
+ * nabla_selftest_mma_pair: one product over a pair of CTAs (tcgen05
+ * cta_group::2, M = 256), each CTA holding half of A and half of B:
+ *   variant 0: C [256][256] = A B^T, a = A [256][128], b = B [256][128] (bf16)
+ *   variant 1: C [256][128] = P V, a = P [256][256] (staged in tensor memory),
+ *              b = V [256][128] (bf16, N-major halves)
+ *   c: device fp32, row-major.
+ *
  * nabla_build_mask_stage_ms: runs nabla_build_mask once (no uint8 mask) with
  * CUDA events between its kernels, synchronises the stream, and writes the
  * milliseconds of its four stages to ms_out[0..3]: pooling, the reduced map,
@@ -425,6 +432,8 @@ NABLA_API nabla_status nabla_build_mask_stage_ms(const nabla_shape* shape,
                                                  void* workspace, nabla_stream_t stream,
                                                  float* ms_out);
 NABLA_API nabla_status nabla_selftest_fp64_tflops(nabla_stream_t stream, double* tflops_out);
+NABLA_API nabla_status nabla_selftest_mma_pair(int variant, const void* a, const void* b, float* c,
+                                               void* workspace, nabla_stream_t stream);
 
 #ifdef __cplusplus
 }

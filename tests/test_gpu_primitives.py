@@ -24,3 +24,21 @@ def test_mma_selftest(nl, variant):
     Bm = b.double().numpy()
     want = A @ Bm.T if variant == 0 else A @ Bm
     np.testing.assert_allclose(c, want, rtol=0, atol=2e-3)
+
+
+@pytest.mark.parametrize("variant", [0, 1])
+def test_mma_pair_selftest(nl, variant):
+    """A product over a pair of CTAs (M = 256): each CTA holds half of A and of
+    B, the even CTA issues the product, each CTA reads its 128 rows of D."""
+    import torch
+    g = torch.Generator().manual_seed(10 + variant)
+    if variant == 0:
+        a = torch.randn(256, 128, generator=g).to(torch.bfloat16)
+        b = torch.randn(256, 128, generator=g).to(torch.bfloat16)
+        want = a.double().numpy() @ b.double().numpy().T
+    else:
+        a = torch.randn(256, 256, generator=g).to(torch.bfloat16)
+        b = torch.randn(256, 128, generator=g).to(torch.bfloat16)
+        want = a.double().numpy() @ b.double().numpy()
+    c = nl.selftest_mma_pair(variant, a.cuda(), b.cuda()).cpu().numpy().astype(np.float64)
+    np.testing.assert_allclose(c, want, rtol=0, atol=4e-3)
