@@ -36,7 +36,8 @@ EXPORTED = ["nabla_workspace_size", "nabla_workspace_init", "nabla_query_status"
             "nabla_calib_accumulate", "nabla_calib_finalize", "bsa_bwd",
             "nabla_build_mask_xattn", "nabla_layer_host_workspace_size", "nabla_layer_host",
             "nabla_layer_host_chunks", "nabla_set_exact_reference", "nabla_query_exact_passes",
-            "nabla_build_mask_stage_ms", "nabla_selftest_fp64_tflops", "nabla_selftest_mma_pair"]
+            "nabla_build_mask_stage_ms", "nabla_selftest_fp64_tflops", "nabla_selftest_mma_pair",
+            "nabla_set_pair_mode"]
 TO_TILE_MAJOR, TO_RASTER = 0, 1
 
 
@@ -125,6 +126,8 @@ def lib() -> ctypes.CDLL:
             L.nabla_build_mask_stage_ms.restype = i32
             L.nabla_build_mask_stage_ms.argtypes = [sp, ctypes.POINTER(_MaskParams), vp, vp, vp,
                                                     vp, ctypes.c_int64, vp, vp, vp, vp]
+            L.nabla_set_pair_mode.restype = None
+            L.nabla_set_pair_mode.argtypes = [i32]
             L.nabla_selftest_mma_pair.restype = i32
             L.nabla_selftest_mma_pair.argtypes = [i32, vp, vp, vp, vp, vp]
             L.nabla_selftest_fp64_tflops.restype = i32
@@ -356,6 +359,16 @@ def selftest_mma(variant: int, a, b, workspace: Optional[Workspace] = None, stre
                                     _stream(stream)))
     workspace.check(stream)
     return c
+
+
+PAIR_NEVER, PAIR_BUILDER_LISTS, PAIR_ALWAYS = 0, 1, 2
+
+
+def set_pair_mode(mode: int) -> None:
+    """Kernel for the forward's fixed-reference pass (d = 128, tile-major):
+    PAIR_NEVER (the default: one CTA per two query blocks), PAIR_BUILDER_LISTS
+    (CTA pairs for mask-builder block lists) or PAIR_ALWAYS.  Process-wide."""
+    lib().nabla_set_pair_mode(int(mode))
 
 
 def selftest_mma_pair(variant: int, a, b, workspace: Optional[Workspace] = None, stream=None):

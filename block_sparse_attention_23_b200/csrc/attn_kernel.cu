@@ -755,8 +755,11 @@ cudaError_t launch_bsa_fwd(const CUtensorMap& q, const CUtensorMap& k, const CUt
   const int64_t nitems = static_cast<int64_t>(BH) * prm.ngroups;
   if (nitems == 0) return cudaSuccess;
   // the fixed-reference pass, then the exact-reference pass, whose CTAs return
-  // at once unless the first pass set *redo (exact_only: the second pass alone)
-  cudaError_t e = cudaMemsetAsync(redo, exact_only ? 1 : 0, sizeof(int), st);
+  // at once unless the first pass set *redo (exact_only 1: the second pass
+  // alone, always recomputing; 2: the second pass alone, after a fixed-reference
+  // pass that another kernel ran and that left *redo set or clear)
+  cudaError_t e = exact_only == 2 ? cudaSuccess
+                                  : cudaMemsetAsync(redo, exact_only ? 1 : 0, sizeof(int), st);
   if (e != cudaSuccess) return e;
   for (int exact = exact_only ? 1 : 0; exact < 2; ++exact) {
     prm.exact = exact;

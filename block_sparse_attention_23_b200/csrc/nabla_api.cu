@@ -59,6 +59,10 @@ cudaError_t launch_select_weights(const float* weights, int64_t nrows, int nb, f
 cudaError_t launch_xattn_scores(const CUtensorMap& q, const CUtensorMap& k, float* lse2,
                                 float* scores, int* status, int BH, int S, int d, int St,
                                 uint64_t wait_limit_ns, cudaStream_t st);
+cudaError_t launch_bsa_fwd_pair(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
+                                const int32_t* row_ptr, const int32_t* col_idx, void* o,
+                                float* lse, int* status, int* redo, int BH, int S, float scale,
+                                uint64_t wait_limit_ns, cudaStream_t st);
 cudaError_t launch_mma_pair_selftest(const CUtensorMap& a, const CUtensorMap& b,
                                      const void* p_glob, float* c, int variant, int* status,
                                      uint64_t lim, cudaStream_t st);
@@ -88,6 +92,17 @@ constexpr int kMaxNbSupported = 4096;
 thread_local std::string g_last_error;
 std::atomic<uint64_t> g_wait_limit_ns{kDefaultWaitLimitNs};
 std::atomic<int> g_exact_reference{0};
+// Which kernel runs the fixed-reference pass of a d = 128 tile-major forward:
+// 0 (default) one CTA per two query blocks; 1 CTA pairs for block lists from
+// the mask builder (bsa_fwd and the host-buffer layer) only; 2 CTA pairs
+// always.  The pair kernel halves each SM's K/V traffic but puts cross-SM
+// arrivals on the softmax -> PV -> softmax chain of every tile; on the Wan
+// 720p-shaped layer it ran 19.4 ms against 15.0 ms for 8 heads.
+std::atomic<int> g_pair_mode{0};
+bool pair_for(bool builder_list) {
+  const int m = g_pair_mode.load();
+  return m == 2 || (m == 1 && builder_list);
+}
 
 nabla_status fail(nabla_status s, const std::string& msg) {
   g_last_error = msg;
@@ -286,7 +301,8 @@ int* status_ptr(void* ws) { return static_cast<int*>(ws); }
 // tensors) when the caller provides it, else read by 5D boxes in the kernel.
 nabla_status run_fwd(const nabla_shape* shape, const void* q, const void* k, const void* v,
                      const int32_t* row_ptr, const int32_t* col_idx, float scale, void* o,
-                     float* lse, int* header, int* redo, void* kv_scratch, cudaStream_t st) {
+                     float* lse, int* header, int* redo, void* kv_scratch, cudaStream_t st,
+                     bool use_pair) {
   const uint64_t rows = static_cast<uint64_t>(shape->B) * shape->H * shape->S;
   const bool raster = shape->layout == NABLA_LAYOUT_RASTER;
   const bool kv_raster = raster && kv_scratch == nullptr;
@@ -315,8 +331,20 @@ nabla_status run_fwd(const nabla_shape* shape, const void* q, const void* k, con
     if ((s = make_map(&mv, v, rows, shape->d)) != NABLA_OK) return s;
   }
   if (!(scale > 0.f)) scale = 1.0f / std::sqrt(static_cast<float>(shape->d));
+  int exact_only = g_exact_reference.load();
+  if (use_pair && exact_only == 0 && shape->d == 128 && !raster) {
+    // the fixed-reference pass on CTA pairs; the exact-reference pass (one-CTA
+    // kernel) follows and returns at once unless a row asked for it
+    cudaError_t e = cudaMemsetAsync(redo, 0, sizeof(int), st);
+    if (e == cudaSuccess)
+      e = nabla::launch_bsa_fwd_pair(mq, mk, mv, row_ptr, col_idx, o, lse, header, redo,
+                                     shape->B * shape->H, shape->S, scale, g_wait_limit_ns.load(),
+                                     st);
+    if (e != cudaSuccess) return cuda_fail(e, "bsa_fwd pair launch");
+    exact_only = 2;
+  }
   cudaError_t e = nabla::launch_bsa_fwd(mq, mk, mv, row_ptr, col_idx, o, lse, header, redo,
-                                        header + kHdrExactPasses, g_exact_reference.load(),
+                                        header + kHdrExactPasses, exact_only,
                                         shape->B * shape->H, shape->H,
                                         shape->S, shape->d, scale, raster ? 1 : 0,
                                         kv_raster ? 1 : 0, shape->Th, shape->Tw,
@@ -336,7 +364,7 @@ void set_last_error(const std::string& msg) { g_last_error = msg; }
 nabla_status fwd_with_header(const nabla_shape* shape, const void* q, const void* k,
                              const void* v, const int32_t* row_ptr, const int32_t* col_idx,
                              float scale, void* o, float* lse, int* header, int* redo,
-                             void* kv_scratch, nabla_stream_t stream) {
+                             void* kv_scratch, nabla_stream_t stream, bool builder_list) {
   nabla_status s = check_shape(shape);
   if (s != NABLA_OK) return s;
   if (!q || !k || !v || !row_ptr || !col_idx || !o || !header || !redo)
@@ -346,7 +374,7 @@ nabla_status fwd_with_header(const nabla_shape* shape, const void* q, const void
     return fail(NABLA_ERR_INVALID_ARG, "q, k, v, o need 16-byte and K/V scratch 256-byte alignment");
   if (!std::isfinite(scale)) return fail(NABLA_ERR_INVALID_ARG, "scale must be finite");
   return run_fwd(shape, q, k, v, row_ptr, col_idx, scale, o, lse, header, redo, kv_scratch,
-                 reinterpret_cast<cudaStream_t>(stream));
+                 reinterpret_cast<cudaStream_t>(stream), pair_for(builder_list));
 }
 // The argument checks of a forward call (shape, token layout and tile grid,
 // null pointers, 16-byte alignment of q, k, v, o, a finite scale), for entry
@@ -387,6 +415,8 @@ void nabla_set_wait_limit_ns(uint64_t ns) {
 }
 
 void nabla_set_exact_reference(int on) { g_exact_reference.store(on ? 1 : 0); }
+
+void nabla_set_pair_mode(int mode) { g_pair_mode.store(mode >= 0 && mode <= 2 ? mode : 0); }
 
 int nabla_query_exact_passes(const void* workspace, nabla_stream_t stream) {
   if (workspace == nullptr) {
@@ -570,7 +600,7 @@ nabla_status bsa_fwd(const nabla_shape* shape, const void* q, const void* k, con
                          ? static_cast<uint8_t*>(workspace) + kHeaderBytes : nullptr;
   return run_fwd(shape, q, k, v, row_ptr, col_idx, scale, o, lse, status_ptr(workspace),
                  status_ptr(workspace) + kHdrRedo, kv_scratch,
-                 reinterpret_cast<cudaStream_t>(stream));
+                 reinterpret_cast<cudaStream_t>(stream), pair_for(true));
 }
 
 nabla_status bsa_fwd_with_mask(const nabla_shape* shape, const void* q, const void* k,
@@ -602,7 +632,7 @@ nabla_status bsa_fwd_with_mask(const nabla_shape* shape, const void* q, const vo
   if (e != cudaSuccess) return cuda_fail(e, "scan/fill launch");
   void* kv_scratch = shape->layout == NABLA_LAYOUT_RASTER ? ws + lay.total : nullptr;
   return run_fwd(shape, q, k, v, row_ptr, col_idx, scale, o, lse, status_ptr(workspace),
-                 status_ptr(workspace) + kHdrRedo, kv_scratch, st);
+                 status_ptr(workspace) + kHdrRedo, kv_scratch, st, pair_for(false));
 }
 
 nabla_status nabla_reorder_tokens(const nabla_shape* shape, int direction, const void* src,

@@ -30,7 +30,7 @@ nabla_status build_mask_with_status(const nabla_shape* shape, const nabla_mask_p
 nabla_status fwd_with_header(const nabla_shape* shape, const void* q, const void* k,
                              const void* v, const int32_t* row_ptr, const int32_t* col_idx,
                              float scale, void* o, float* lse, int* header, int* redo,
-                             void* kv_scratch, nabla_stream_t stream);
+                             void* kv_scratch, nabla_stream_t stream, bool builder_list);
 }  // namespace nabla
 
 namespace {
@@ -262,7 +262,7 @@ NABLA_API nabla_status nabla_layer_host(const nabla_shape* shape, const nabla_ma
     // the forward reports into the shared header, with the slot's own
     // exact-pass request word (header word 4 + slot)
     s = nabla::fwd_with_header(&chunk, dq, dk, dv, row_ptr, col_idx, 0.f, dout, dlse, status,
-                               status + 4 + slot, nullptr, ns);
+                               status + 4 + slot, nullptr, ns, true);
     if (s != NABLA_OK) return s;
     if ((e = cudaEventRecord(r->in_free[slot], cs)) != cudaSuccess ||
         (e = cudaEventRecord(r->out_ready[slot], cs)) != cudaSuccess)

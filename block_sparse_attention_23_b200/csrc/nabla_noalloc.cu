@@ -38,7 +38,7 @@ cudaError_t launch_scan_fill(const uint32_t* bits, const int32_t* counts, int64_
 nabla_status fwd_with_header(const nabla_shape* shape, const void* q, const void* k,
                              const void* v, const int32_t* row_ptr, const int32_t* col_idx,
                              float scale, void* o, float* lse, int* header, int* redo,
-                             void* kv_scratch, nabla_stream_t stream);
+                             void* kv_scratch, nabla_stream_t stream, bool builder_list);
 nabla_status check_fwd_args(const nabla_shape* shape, const void* q, const void* k,
                             const void* v, const void* o, float scale);
 }  // namespace nabla
@@ -131,7 +131,7 @@ NABLA_API nabla_status bsa_fwd_with_mask_static(const nabla_shape* shape, const 
   // no room for tile-major K/V copies here: raster K and V are read by 5D boxes
   s = nabla::fwd_with_header(shape, q, k, v, row_ptr, col_idx, scale, o, lse,
                              reinterpret_cast<int*>(ws), reinterpret_cast<int*>(ws) + 1, nullptr,
-                             stream);
+                             stream, false);
   if (s != NABLA_OK) return s;   // the forward has set the message
   if (status_out != nullptr) {
     e = cudaMemcpyAsync(status_out, ws, sizeof(int32_t), cudaMemcpyDeviceToDevice, st);

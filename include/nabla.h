@@ -392,6 +392,15 @@ NABLA_API int nabla_version(void);
  * 0 (the default) restores the two-kernel scheme described at bsa_fwd.
  * Process-wide; for tests and for reproducing the exact-reference numerics.
  *
+ * nabla_set_pair_mode: which kernel runs a d = 128 tile-major forward's
+ * fixed-reference pass.  0 (the default): one CTA per two query blocks.  1: CTA
+ * pairs (each pair of CTAs walks the union of four query blocks' lists with
+ * M = 256 products, each CTA loading half of every K and V tile) for block
+ * lists from nabla_build_mask (bsa_fwd, nabla_layer_host), one CTA for caller
+ * masks.  2: CTA pairs always.  Process-wide; the results agree within
+ * rounding either way.  The pair kernel is slower on the layers measured here
+ * (its cross-SM handshakes lie on every tile's critical path).
+ *
  * nabla_query_exact_passes: synchronises the stream and returns word 2 of a
  * forward workspace's header: how many forwards on it needed the
  * exact-reference kernel since nabla_workspace_init (-1 on a CUDA error).
@@ -422,6 +431,7 @@ NABLA_API int nabla_version(void);
  */
 NABLA_API void nabla_set_wait_limit_ns(uint64_t ns);
 NABLA_API void nabla_set_exact_reference(int on);
+NABLA_API void nabla_set_pair_mode(int mode);
 NABLA_API int nabla_query_exact_passes(const void* workspace, nabla_stream_t stream);
 NABLA_API nabla_status nabla_selftest_mma(int variant, const void* a, const void* b, float* c,
                                 void* workspace, nabla_stream_t stream);
