@@ -50,17 +50,19 @@
 // workspace holds them (made by the token reorder before the launch), else
 // by 5D boxes as well (kv_raster).
 //
-// Online softmax with a reference maximum per row.  Each launch runs two
-// passes over the same grid.  The fixed-reference pass: the two warps of a
-// lane quarter agree on the row max of the first key tile the row's block
-// lists, and that reference m stays for the rest of the row (no further max
-// or exchange per tile; p = 2^(s*scale*log2e - m) may exceed 1).  A warp
-// whose partial row sum of a tile (128 columns) exceeds 2^16 sets a flag in
-// the caller's workspace, and the exact-reference pass then recomputes the
-// whole launch: there the warps agree on every tile's max and raise m (with O
-// and l rescaled by 2^(m_old - m_new)) whenever it grows by more than 2^8, so
-// p <= 256.  Its CTAs return at once when the flag is clear.  O / l and
-// LSE = ln2 (m + log2 l) do not depend on the reference in exact arithmetic.
+// Online softmax with a reference maximum per row, in up to two passes over
+// the CTA's query tile.  The fixed-reference pass: the two warps of a lane
+// quarter agree on the row max of the first key tile the row's block lists,
+// and that reference m stays for the rest of the row (no further max or
+// exchange per tile; p = 2^(s*scale*log2e - m) may exceed 1).  A warp whose
+// partial row sum of a tile (128 columns) exceeds 2^16 sets a flag in shared
+// memory, and the CTA then runs the exact-reference pass over the same tile
+// (the union list and Q stay in place, the barriers start afresh): there the
+// warps agree on every tile's max and raise m (with O and l rescaled by
+// 2^(m_old - m_new)) whenever it grows by more than 2^8, so p <= 256.  The
+// first CTA of a call that needs the second pass sets a word in the caller's
+// workspace and counts the call.  O / l and LSE = ln2 (m + log2 l) do not
+// depend on the reference in exact arithmetic.
 // A warp whose two entries the row both lists (the common case) runs its
 // loads and exponentials as straight-line code without per-chunk branches.
 //
@@ -139,9 +141,10 @@ struct AttnParams {
   int Th, Tw;              // tile grid (raster token order only)
   float scale_log2;        // softmax scale * log2(e)
   uint64_t wait_limit_ns;
-  int* redo;               // set by a pass that needs the exact-reference pass (see below)
-  int* exact_passes;       // counts the exact-reference passes that ran
-  int exact;               // 0: reference fixed per row; 1: the exact-reference pass
+  int* redo;               // set when a tile of the call needed the exact-reference pass
+  int* exact_passes;       // counts the forwards that needed it
+  int exact;               // 0: fixed reference, exact pass per tile when needed;
+                           // 1: exact pass alone; 2: exact pass alone if *redo is set
   int kv_raster;           // raster token order: K and V read by 5D boxes too (else 2D)
 };
 
@@ -200,17 +203,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile uint32_t* tmem_holder = misc;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
   volatile int* n_union_s = reinterpret_cast<volatile int*>(misc + 2);
+  volatile int* cta_redo = reinterpret_cast<volatile int*>(misc + 3);   // a row outgrew the reference
+  volatile int* pass_s = reinterpret_cast<volatile int*>(misc + 4);     // 0 fixed, 1 exact reference
   float* xch = reinterpret_cast<float*>(gbase + L::kOffXch);           // [2][2][kBM]
   uint32_t* bm = reinterpret_cast<uint32_t*>(gbase + L::kOffBitmap);   // [2][kMaxNb/32]
   int32_t* ulist = reinterpret_cast<int32_t*>(gbase + L::kOffList);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int item = blockIdx.x;
-  // the exact-reference pass runs only after a fixed-reference pass asked for it
-  if (prm.exact) {
-    if (*prm.redo == 0) return;
-    if (item == 0 && tid == 0) atomicAdd(prm.exact_passes, 1);
-  }
+  // exact 2: an exact-reference launch after another kernel's fixed-reference
+  // pass, which runs only if that pass asked for it
+  if (prm.exact == 2 && *prm.redo == 0) return;
+  if (prm.exact != 0 && item == 0 && tid == 0) atomicAdd(prm.exact_passes, 1);
+
   const int bh = item / prm.ngroups;
   const int grp = item % prm.ngroups;
   const int nb = prm.nb;
@@ -218,8 +223,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int nq = min(2, nb - r0);               // query blocks present (1 or 2)
   auto bar = [&](int i) { return bar0 + 8u * static_cast<uint32_t>(i); };
 
-  // ---------------------------------------------------------------- setup
-  if (tid == 0) {
+  auto init_bars = [&]() {
     mbar_init(bar(kBarQFull), 1);
     mbar_init(bar(kBarKFull), 1);
     mbar_init(bar(kBarKEmpty), 1);
@@ -231,8 +235,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar(kBarOFull), 1);
     mbar_init(bar(kBarDrain), 1);
     for (int q = 0; q < 4; ++q) mbar_init(bar(kBarPair + q), 64);
-    *abort_flag = 0;
     fence_barrier_init();
+  };
+
+  // ---------------------------------------------------------------- setup
+  if (tid == 0) {
+    init_bars();
+    *abort_flag = 0;
+    *cta_redo = 0;
+    *pass_s = prm.exact != 0 ? 1 : 0;
   }
   if (warp == kMmaWarp) {
     tmem_alloc(smem_addr(misc), kTmemCols);
@@ -305,8 +316,29 @@ __global__ void __launch_bounds__(kThreads, 1)
     return (kEntries * u + e < n_u) ? ulist[kEntries * u + e] : 0;
   };
 
+  // After a pass every thread meets here.  A second, exact-reference pass over
+  // the same tile follows when a row of the tile outgrew its fixed reference
+  // (the union list and Q stay in place; barriers start afresh).
+  auto next_pass = [&]() {
+    tc_fence_before();
+    __syncthreads();
+    const bool again = *pass_s == 0 && *cta_redo != 0 && *abort_flag == 0;
+    if (again) {
+      if (tid == 0) {
+        init_bars();
+        *pass_s = 1;
+        // count the forward once, at its first recomputed tile
+        if (atomicExch(prm.redo, 1) == 0) atomicAdd(prm.exact_passes, 1);
+      }
+      __syncthreads();
+    }
+    tc_fence_after();
+    return again;
+  };
+
   if (warp >= 8) {
   setmaxnreg_dec<kRegsOther>();
+  while (true) {
   if (warp == kProducerWarp || warp == kVProducerWarp) {
     // ------------------------------------------------------------ TMA producers
     // warp 8 streams Q and K, warp 10 streams V (one buffer each: K(t+1) may
@@ -317,12 +349,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       const CUtensorMap* map = is_k ? &tmK : &tmV;
       const int full = is_k ? kBarKFull : kBarVFull, empty = is_k ? kBarKEmpty : kBarVEmpty;
       int armed = 0;
-      if (is_k) {
+      if (is_k && !(*cta_redo)) {   // the first pass of this tile loads Q
         mbar_arrive_expect_tx(bar(kBarQFull), L::kQBytes);
         for (int qb = 0; qb < 2; ++qb)   // a block past the end repeats the last (rows unused)
           for (int h = 0; h < L::kDH; ++h)
             load_block<kRaster>(sQ + h * kBM * 128 + qb * 64 * 128, &tmQ, bar(kBarQFull), h, bh,
                                 min(r0 + qb, nb - 1), prm.S, prm.Th, prm.Tw);
+      } else if (is_k) {
+        mbar_arrive(bar(kBarQFull));   // Q is still in place from the first pass
       }
       const int last = ulist[n_u - 1] & 0xFFFF;
       const bool kv_raster = kRaster && prm.kv_raster;
@@ -408,6 +442,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_wait(bar(kBarDrain), 0, kDrainLimitNs, nullptr);
     }
   }
+  if (!next_pass()) break;
+  }
   } else {
     setmaxnreg_inc<kRegsSoftmax>();
     // ------------------------------------------------------------ softmax (warps 0-7)
@@ -424,6 +460,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t o_base = tmem + lane_off + kColO + static_cast<uint32_t>(D / 2) * half;
     const uint32_t pair_bar = bar(kBarPair + quarter);
     const float sl2 = prm.scale_log2;
+    while (true) {
     float m = -INFINITY;        // reference max of the row, log2 units (same in both warps)
     float l = 0.f;              // running sum over this warp's columns of the row
     int pair_n = 0;             // phases of the pair barrier used so far
@@ -451,7 +488,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // (agreed with the other warp of the lane quarter), then kept.  Exact
       // pass: the two warps agree on every tile's max and raise the reference
       // lazily.  Both warps take the same branch (m is the same in both).
-      const bool agree = prm.exact || __any_sync(0xffffffffu, m == -INFINITY);
+      const bool agree = *pass_s != 0 || __any_sync(0xffffffffu, m == -INFINITY);
       bool pv_done = t == 0;                     // PV(t-1) completed (known so far)
       if (agree) {
         float mx[8];
@@ -542,7 +579,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       l += l_tile;
       // a row whose later keys outgrow the fixed reference asks for the exact pass
       if (!agree && __any_sync(0xffffffffu, !(l_tile <= kFixedRefSumLimit)) && lane == 0)
-        atomicExch(prm.redo, 1);
+        *cta_redo = 1;
       if (!ok) break;
       if (!pv_done && !warp_wait(bar(kBarOFull), (t - 1) & 1, lim, abort_flag)) {
         ok = false;
@@ -600,6 +637,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (write && half == 0 && prm.lse != nullptr)
       prm.lse[grow] = l_row > 0.f ? (m + __log2f(l_row)) * 0.69314718055994530942f : -INFINITY;
+    if (!next_pass()) break;
+    }
   }
 
   tc_fence_before();
@@ -754,25 +793,22 @@ cudaError_t launch_bsa_fwd(const CUtensorMap& q, const CUtensorMap& k, const CUt
   prm.kv_raster = kv_raster;
   const int64_t nitems = static_cast<int64_t>(BH) * prm.ngroups;
   if (nitems == 0) return cudaSuccess;
-  // the fixed-reference pass, then the exact-reference pass, whose CTAs return
-  // at once unless the first pass set *redo (exact_only 1: the second pass
-  // alone, always recomputing; 2: the second pass alone, after a fixed-reference
-  // pass that another kernel ran and that left *redo set or clear)
-  cudaError_t e = exact_only == 2 ? cudaSuccess
-                                  : cudaMemsetAsync(redo, exact_only ? 1 : 0, sizeof(int), st);
+  // One launch.  exact_only 0: each CTA runs the fixed-reference pass and, if
+  // a row of its tile outgrew the reference, the exact-reference pass over the
+  // same tile (the first such CTA sets *redo and counts the forward); 1: the
+  // exact-reference pass alone; 2: the exact-reference pass alone, only if a
+  // fixed-reference pass that another kernel ran left *redo set.
+  cudaError_t e = exact_only == 2 ? cudaSuccess : cudaMemsetAsync(redo, 0, sizeof(int), st);
   if (e != cudaSuccess) return e;
-  for (int exact = exact_only ? 1 : 0; exact < 2; ++exact) {
-    prm.exact = exact;
-    if (raster) {
-      e = d == 128 ? launch_fwd_t<128, true>(q, k, v, prm, nitems, st)
-                   : launch_fwd_t<64, true>(q, k, v, prm, nitems, st);
-    } else {
-      e = d == 128 ? launch_fwd_t<128, false>(q, k, v, prm, nitems, st)
-                   : launch_fwd_t<64, false>(q, k, v, prm, nitems, st);
-    }
-    if (e != cudaSuccess) return e;
+  prm.exact = exact_only;
+  if (raster) {
+    e = d == 128 ? launch_fwd_t<128, true>(q, k, v, prm, nitems, st)
+                 : launch_fwd_t<64, true>(q, k, v, prm, nitems, st);
+  } else {
+    e = d == 128 ? launch_fwd_t<128, false>(q, k, v, prm, nitems, st)
+                 : launch_fwd_t<64, false>(q, k, v, prm, nitems, st);
   }
-  return cudaSuccess;
+  return e;
 }
 
 cudaError_t launch_mma_selftest(const CUtensorMap& a, const CUtensorMap& b, const void* a_glob,

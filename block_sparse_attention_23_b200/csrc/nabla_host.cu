@@ -3,13 +3,15 @@
 // independent, so the layer runs in chunks of heads through a two-slot device
 // pipeline: the host-to-device copies of chunk c+1 and the device-to-host
 // copies of chunk c-1 run on their own streams while chunk c computes, and
-// PCIe transfers hide behind the attention instead of adding to it.  Every
-// chunk computes on the caller's stream, one after another: a second compute
-// stream let one chunk's forward kernels queue behind the other chunk's whole
-// grid (each attention CTA holds most of an SM's shared memory), which
-// delayed the output copies and the next inputs.  Plain cudaMemcpyAsync
-// copies only; stream order is kept with events, and the caller's stream
-// waits for the last output copies before the call's work is complete on it.
+// PCIe transfers hide behind the attention instead of adding to it.  The two
+// slots compute on two streams (slot 0 on the caller's, slot 1 on a
+// library-owned one), so that the next chunk's kernels take the SMs that the
+// last wave of the current chunk's attention grid leaves idle; the forward is a
+// single launch per chunk (a query tile that needs the exact-reference pass
+// runs it inside the same kernel), so nothing of one chunk waits behind the
+// other chunk's grid.  Plain cudaMemcpyAsync copies only; stream order is kept
+// with events, and the caller's stream waits for the last output copies before
+// the call's work is complete on it.
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -107,15 +109,15 @@ std::vector<int> chunk_schedule(int64_t heads, int max_heads) {
 
 // Streams and events reused across calls (one set per device, created once).
 struct PipeRes {
-  cudaStream_t h2d = nullptr, d2h = nullptr;
+  cudaStream_t h2d = nullptr, d2h = nullptr, comp1 = nullptr;   // comp1: slot 1's compute
   cudaEvent_t in_ready[kSlots] = {}, in_free[kSlots] = {}, out_ready[kSlots] = {},
               out_free[kSlots] = {};
-  cudaEvent_t join[2] = {};   // a failed call: the caller's stream waits for the copy streams
+  cudaEvent_t join[3] = {};   // a failed call: the caller's stream waits for the other streams
   bool ok = false;
 };
 
 void release(PipeRes& r) {
-  for (cudaStream_t* p : {&r.h2d, &r.d2h})
+  for (cudaStream_t* p : {&r.h2d, &r.d2h, &r.comp1})
     if (*p) { cudaStreamDestroy(*p); *p = nullptr; }
   for (int i = 0; i < kSlots; ++i)
     for (cudaEvent_t* p : {&r.in_ready[i], &r.in_free[i], &r.out_ready[i], &r.out_free[i]})
@@ -137,13 +139,14 @@ nabla_status resources(PipeRes** out) {
   if (!r.ok) {
     e = cudaStreamCreateWithFlags(&r.h2d, cudaStreamNonBlocking);
     if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&r.d2h, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&r.comp1, cudaStreamNonBlocking);
     for (int i = 0; i < kSlots && e == cudaSuccess; ++i) {
       e = cudaEventCreateWithFlags(&r.in_ready[i], cudaEventDisableTiming);
       if (e == cudaSuccess) e = cudaEventCreateWithFlags(&r.in_free[i], cudaEventDisableTiming);
       if (e == cudaSuccess) e = cudaEventCreateWithFlags(&r.out_ready[i], cudaEventDisableTiming);
       if (e == cudaSuccess) e = cudaEventCreateWithFlags(&r.out_free[i], cudaEventDisableTiming);
     }
-    for (int i = 0; i < 2 && e == cudaSuccess; ++i)
+    for (int i = 0; i < 3 && e == cudaSuccess; ++i)
       e = cudaEventCreateWithFlags(&r.join[i], cudaEventDisableTiming);
     if (e != cudaSuccess) {
       release(r);
@@ -215,14 +218,15 @@ NABLA_API nabla_status nabla_layer_host(const nabla_shape* shape, const nabla_ma
   cudaError_t e;
   if ((e = cudaEventRecord(start, st)) != cudaSuccess ||
       (e = cudaStreamWaitEvent(r->h2d, start, 0)) != cudaSuccess ||
-      (e = cudaStreamWaitEvent(r->d2h, start, 0)) != cudaSuccess)
+      (e = cudaStreamWaitEvent(r->d2h, start, 0)) != cudaSuccess ||
+      (e = cudaStreamWaitEvent(r->comp1, start, 0)) != cudaSuccess)
     return cuda_fail(e, "pipeline start");
   const nabla_status result = [&]() -> nabla_status {
   int64_t h0 = 0;
   for (int64_t c = 0; c < nchunks; h0 += sizes[c], ++c) {
     const int slot = static_cast<int>(c % kSlots);
     const int h = sizes[c];
-    cudaStream_t cs = st;
+    cudaStream_t cs = slot == 0 ? st : r->comp1;
     const size_t tbytes = static_cast<size_t>(h) * shape->S * shape->d * 2;
     const size_t lbytes = static_cast<size_t>(h) * shape->S * 4;
     const size_t toff = static_cast<size_t>(h0) * shape->S * shape->d * 2;
@@ -286,8 +290,8 @@ NABLA_API nabla_status nabla_layer_host(const nabla_shape* shape, const nabla_ma
   if (result != NABLA_OK) {
     // whatever was queued before the failure is ordered before later work on
     // the caller's stream, so the caller's buffers are not in use once it syncs
-    const cudaStream_t others[2] = {r->h2d, r->d2h};
-    for (int i = 0; i < 2; ++i)
+    const cudaStream_t others[3] = {r->h2d, r->d2h, r->comp1};
+    for (int i = 0; i < 3; ++i)
       if (cudaEventRecord(r->join[i], others[i]) == cudaSuccess)
         cudaStreamWaitEvent(st, r->join[i], 0);
   }

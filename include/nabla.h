@@ -148,14 +148,14 @@ NABLA_API nabla_status nabla_build_mask(const nabla_shape* shape, const nabla_ma
  * A query block with an empty list gets O = 0 and LSE = -inf.  Duplicate
  * column indices count once; indices outside [0, nb) are skipped and recorded
  * as NABLA_ERR_BAD_INDEX.
- * The call runs two kernels.  The first takes, per row, the max of the first
- * key tile the row's block lists as the softmax reference and keeps it; if a
- * later tile's scores exceed that reference by more than 16 in log2 units
- * (a tile's partial row sum above 2^16), it sets word 1 of the workspace
- * header, and the second kernel recomputes the whole call with the reference
- * raised as the scores grow (otherwise its blocks return at once).  Word 2
- * of the header counts the recomputations (nabla_query_exact_passes); the
- * result does not depend on which kernel produced it beyond rounding.  One
+ * The call is one kernel launch.  Each query tile (two query blocks) takes,
+ * per row, the max of the first key tile the row's block lists as the softmax
+ * reference and keeps it; if a later tile's scores exceed that reference by
+ * more than 16 in log2 units (a tile's partial row sum above 2^16), the query
+ * tile is computed again with the reference raised as the scores grow.  Word
+ * 1 of the workspace header is set when any tile of the call was recomputed,
+ * and word 2 counts the calls that needed it (nabla_query_exact_passes); the
+ * result does not depend on which pass produced it beyond rounding.  One
  * workspace must not serve two calls that may run at the same time.
  */
 NABLA_API nabla_status bsa_fwd(const nabla_shape* shape, const void* q, const void* k, const void* v,
@@ -219,9 +219,11 @@ NABLA_API nabla_status bsa_fwd_with_mask_static(const nabla_shape* shape, const 
  * device copies of the same tensors.
  *
  * Heads are independent, so the call moves them in chunks of at most
- * heads_per_chunk heads through two device slots: while chunk c computes on
- * `stream`, chunk c+1's inputs go host-to-device and chunk c-1's outputs go
- * device-to-host on two streams the library owns, ordered with events.  With
+ * heads_per_chunk heads through two device slots: while chunk c computes,
+ * chunk c+1's inputs go host-to-device and chunk c-1's outputs go
+ * device-to-host on two streams the library owns, ordered with events.  The
+ * slots compute on `stream` and on a third library stream, so consecutive
+ * chunks' kernels may overlap on the GPU.  With
  * page-locked (pinned) host buffers the copies overlap the kernels; pageable
  * buffers give the same result without the overlap.  The chunks ramp up
  * (1, 2, 4, ... heads) and end on a chunk of heads_per_chunk/4 heads, so that
@@ -240,7 +242,7 @@ NABLA_API nabla_status bsa_fwd_with_mask_static(const nabla_shape* shape, const 
  * `stream` before reading o_host or lse_host.  Argument errors (the mask
  * parameters included) return before anything is queued; a CUDA error part
  * way through still orders every copy already queued before later work on
- * `stream`, so the host buffers are free once `stream` is synchronised.  The library's copy streams are
+ * `stream`, so the host buffers are free once `stream` is synchronised.  The library's streams are
  * per device, so two calls in flight at once on one device (other host
  * threads, or other streams without ordering) are not supported.
  */
@@ -387,9 +389,9 @@ NABLA_API int nabla_version(void);
  * memory, record NABLA_ERR_TIMEOUT and return.  Tests set a tiny limit to
  * check that path without hanging anything.
  *
- * nabla_set_exact_reference: 1 makes every forward run only its second,
- * exact-reference kernel (the reference raised as each row's scores grow);
- * 0 (the default) restores the two-kernel scheme described at bsa_fwd.
+ * nabla_set_exact_reference: 1 makes every forward compute every query tile
+ * with the exact reference only (the reference raised as each row's scores
+ * grow); 0 (the default) restores the scheme described at bsa_fwd.
  * Process-wide; for tests and for reproducing the exact-reference numerics.
  *
  * nabla_set_pair_mode: which kernel runs a d = 128 tile-major forward's
@@ -403,7 +405,8 @@ NABLA_API int nabla_version(void);
  *
  * nabla_query_exact_passes: synchronises the stream and returns word 2 of a
  * forward workspace's header: how many forwards on it needed the
- * exact-reference kernel since nabla_workspace_init (-1 on a CUDA error).
+ * exact-reference recomputation of a query tile since nabla_workspace_init
+ * (-1 on a CUDA error).
  *
  * nabla_selftest_mma_pair: one product over a pair of CTAs (tcgen05
  * cta_group::2, M = 256), each CTA holding half of A and half of B:
