@@ -694,7 +694,7 @@ def run_ours(args):
                          "what": "mask + attention on raster-ordered Q, K, V (O, LSE raster), "
                                  "Q read by 5D boxes, K and V reordered to tile-major copies in the "
                                  "workspace first; outside the step"},
-        "gpu_launches": 7 * args.steps,
+        "gpu_launches": 6 * args.steps,
         "clocks": clk,
     }
     if args.profile_heads:

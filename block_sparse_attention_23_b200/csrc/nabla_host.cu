@@ -110,8 +110,8 @@ std::vector<int> chunk_schedule(int64_t heads, int max_heads) {
 // Streams and events reused across calls (one set per device, created once).
 struct PipeRes {
   cudaStream_t h2d = nullptr, d2h = nullptr, comp1 = nullptr;   // comp1: slot 1's compute
-  cudaEvent_t in_ready[kSlots] = {}, in_free[kSlots] = {}, out_ready[kSlots] = {},
-              out_free[kSlots] = {};
+  cudaEvent_t qk_ready[kSlots] = {}, in_ready[kSlots] = {}, in_free[kSlots] = {},
+              out_ready[kSlots] = {}, out_free[kSlots] = {};
   cudaEvent_t join[3] = {};   // a failed call: the caller's stream waits for the other streams
   bool ok = false;
 };
@@ -120,7 +120,8 @@ void release(PipeRes& r) {
   for (cudaStream_t* p : {&r.h2d, &r.d2h, &r.comp1})
     if (*p) { cudaStreamDestroy(*p); *p = nullptr; }
   for (int i = 0; i < kSlots; ++i)
-    for (cudaEvent_t* p : {&r.in_ready[i], &r.in_free[i], &r.out_ready[i], &r.out_free[i]})
+    for (cudaEvent_t* p : {&r.qk_ready[i], &r.in_ready[i], &r.in_free[i], &r.out_ready[i],
+                           &r.out_free[i]})
       if (*p) { cudaEventDestroy(*p); *p = nullptr; }
   for (cudaEvent_t& ev : r.join)
     if (ev) { cudaEventDestroy(ev); ev = nullptr; }
@@ -141,7 +142,8 @@ nabla_status resources(PipeRes** out) {
     if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&r.d2h, cudaStreamNonBlocking);
     if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&r.comp1, cudaStreamNonBlocking);
     for (int i = 0; i < kSlots && e == cudaSuccess; ++i) {
-      e = cudaEventCreateWithFlags(&r.in_ready[i], cudaEventDisableTiming);
+      e = cudaEventCreateWithFlags(&r.qk_ready[i], cudaEventDisableTiming);
+      if (e == cudaSuccess) e = cudaEventCreateWithFlags(&r.in_ready[i], cudaEventDisableTiming);
       if (e == cudaSuccess) e = cudaEventCreateWithFlags(&r.in_free[i], cudaEventDisableTiming);
       if (e == cudaSuccess) e = cudaEventCreateWithFlags(&r.out_ready[i], cudaEventDisableTiming);
       if (e == cudaSuccess) e = cudaEventCreateWithFlags(&r.out_free[i], cudaEventDisableTiming);
@@ -246,13 +248,14 @@ NABLA_API nabla_status nabla_layer_host(const nabla_shape* shape, const nabla_ma
                              cudaMemcpyHostToDevice, r->h2d)) != cudaSuccess ||
         (e = cudaMemcpyAsync(dk, static_cast<const uint8_t*>(k_host) + toff, tbytes,
                              cudaMemcpyHostToDevice, r->h2d)) != cudaSuccess ||
+        (e = cudaEventRecord(r->qk_ready[slot], r->h2d)) != cudaSuccess ||
         (e = cudaMemcpyAsync(dv, static_cast<const uint8_t*>(v_host) + toff, tbytes,
                              cudaMemcpyHostToDevice, r->h2d)) != cudaSuccess ||
         (e = cudaEventRecord(r->in_ready[slot], r->h2d)) != cudaSuccess)
       return cuda_fail(e, "h2d copy");
-    // compute chunk c once its inputs are in and chunk c-2's outputs have left
-    // the slot
-    if ((e = cudaStreamWaitEvent(cs, r->in_ready[slot], 0)) != cudaSuccess)
+    // the mask of chunk c once its Q and K are in and chunk c-2's outputs have
+    // left the slot; its attention once V is in as well
+    if ((e = cudaStreamWaitEvent(cs, r->qk_ready[slot], 0)) != cudaSuccess)
       return cuda_fail(e, "compute wait");
     if (c >= kSlots && (e = cudaStreamWaitEvent(cs, r->out_free[slot], 0)) != cudaSuccess)
       return cuda_fail(e, "compute wait");
@@ -263,6 +266,8 @@ NABLA_API nabla_status nabla_layer_host(const nabla_shape* shape, const nabla_ma
     s = nabla::build_mask_with_status(&chunk, params, dq, dk, nullptr, row_ptr, col_idx, lay.cap,
                                       nullptr, sb + lay.build, status, ns);
     if (s != NABLA_OK) return s;
+    if ((e = cudaStreamWaitEvent(cs, r->in_ready[slot], 0)) != cudaSuccess)
+      return cuda_fail(e, "compute wait");
     // the forward reports into the shared header, with the slot's own
     // exact-pass request word (header word 4 + slot)
     s = nabla::fwd_with_header(&chunk, dq, dk, dv, row_ptr, col_idx, 0.f, dout, dlse, status,
