@@ -649,8 +649,8 @@ def run_ours(args):
                           "what": "128x128 S and PV products the kernel runs (union of two "
                                   "query blocks in 256-key tiles), counted on the host"},
         "attn_exact_passes": {"count": fwd_exact_passes, "forwards": 1 + args.warmup + args.steps,
-                              "what": "forwards whose fixed-reference kernel asked the exact-"
-                                      "reference kernel to recompute the call"},
+                              "what": "forwards in which some query tile outgrew its fixed "
+                                      "softmax reference and ran the exact-reference pass"},
         "pct_of_dense_bf16_peak": {"attn_vs_sustained": attn_tflops / peak,
                                    "attn_vs_burst": attn_tflops / peaks["bf16_tflops"],
                                    "layer_vs_sustained": value / ws / peak},

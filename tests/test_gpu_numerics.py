@@ -138,3 +138,28 @@ def test_equal_scores_and_thr_one(nl, oracle_mod, synth_mod):
     o, lse = nl.bsa_fwd(qd, kd, vd, rp, ci)
     ro, rl = oracle_mod.masked_attention(q, k, v, om)
     compare_attention(o.float().cpu().numpy().reshape(-1, d), lse.cpu().numpy().reshape(-1), ro, rl)
+
+
+def test_forward_recomputes_only_the_tiles_that_need_it(nl, oracle_mod):
+    """Head 0 has keys whose scores rise ~10 log2 units per block (its query
+    tiles outgrow the fixed reference and run the exact-reference pass),
+    head 1 has flat random scores (its tiles finish in the first pass): one
+    call, counted once, both heads within the attention bars."""
+    import torch
+    B, H, nb, d = 1, 2, 10, 128
+    step = np.sqrt(d) * 10.0 / 1.4427
+    q, k, v = _rising(B, H, nb, d, step, seed=21)
+    rng = np.random.default_rng(22)
+    flat = rng.standard_normal((64 * nb, d)).astype(np.float32) * 0.5
+    k[0, 1] = _bf16_bits(flat)
+    mask = np.ones((B, H, nb, nb), dtype=np.uint8)
+    mask[0, 1, ::3, 1::2] = 0
+    qd, kd, vd = to_device_bf16(q), to_device_bf16(k), to_device_bf16(v)
+    ws = nl.Workspace.create(nl.make_shape(B, H, 64 * nb, d), nl.OP_FWD_WITH_MASK)
+    for call in range(2):
+        o, lse = nl.bsa_fwd_with_mask(qd, kd, vd, torch.from_numpy(mask).cuda(), workspace=ws)
+        assert ws.query_status() == 0
+        assert ws.exact_passes() == call + 1
+    rows = np.arange(B * H * 64 * nb, dtype=np.int64)
+    ro, rl = oracle_mod.masked_attention(q, k, v, mask, rows)
+    compare_attention(o.float().cpu().numpy().reshape(-1, d), lse.cpu().numpy().reshape(-1), ro, rl)
