@@ -249,3 +249,21 @@ def test_exact_pass_counter_query_rejects_null(nl):
     assert lib.nabla_query_exact_passes(None, None) == -1
     assert "NULL" in lib.nabla_last_error().decode()
     lib.nabla_set_exact_reference(0)          # the default; a no-op without a GPU
+
+
+def test_diagnostics_reject_bad_arguments_before_any_cuda_call(nl):
+    """The stage-timing and self-test calls check their arguments on the host
+    (no GPU needed to see the rejections)."""
+    lib = nl.lib()
+    s = nl.make_shape(1, 2, 64 * 12, 128, (1, 3, 4))
+    prm = nl._MaskParams(0.2, 0, 0, 0, 0, 0)
+    a = ctypes.c_void_p(1 << 20)
+    # a null ms_out is refused before the build runs
+    rc = lib.nabla_build_mask_stage_ms(ctypes.byref(s), ctypes.byref(prm), a, a, a, a, 10, a, a,
+                                       None, None)
+    assert rc == 1 and "ms_out" in lib.nabla_last_error().decode()
+    assert lib.nabla_selftest_fp64_tflops(None, None) == 1
+    assert lib.nabla_selftest_mma_pair(2, a, a, a, a, None) == 1
+    assert "variant" in lib.nabla_last_error().decode()
+    assert lib.nabla_selftest_mma_pair(0, None, a, a, a, None) == 1
+
