@@ -40,7 +40,10 @@
 // the softmax stores P(t) only after PV(t-1), which read P(t-1), completed,
 // and keeps P(t) in registers until then.  S at N = 256 runs at the full
 // tensor rate (an N = 128 product with both operands in shared memory does
-// not), and the per-tile softmax overhead is spread over 256 keys.
+// not), and the per-tile softmax overhead is spread over 256 keys.  On a tile
+// with a fixed reference and both of its entries listed, a softmax warp loads
+// its first 32 columns, then the other 96 while it exponentiates the first,
+// and releases S(t) once those are in.
 //
 // Token order: tile-major tensors are read as 2D boxes; a raster-ordered Q
 // (token (t,h,w) at (t*H + h)*W + w) as 5D boxes that gather one 4x4x4 tile,
@@ -465,31 +468,45 @@ __global__ void __launch_bounds__(kThreads, 1)
     float l = 0.f;              // running sum over this warp's columns of the row
     int pair_n = 0;             // phases of the pair barrier used so far
     bool ok = true;
+    const bool exact_pass = *pass_s != 0;
+    // list entries of the tile this warp's columns cover, read one tile ahead
+    int e_next0 = tile_entry(0, 2 * half), e_next1 = tile_entry(0, 2 * half + 1);
     for (int t = 0; t < n_t; ++t) {
-      const bool v0 = (tile_entry(t, 2 * half) & bit) != 0;       // uniform per warp
-      const bool v1 = (tile_entry(t, 2 * half + 1) & bit) != 0;
+      const bool v0 = (e_next0 & bit) != 0;       // uniform per warp
+      const bool v1 = (e_next1 & bit) != 0;
       if (!warp_wait(bar(kBarSFull), t & 1, lim, abort_flag)) { ok = false; break; }
       tc_fence_after();
-      // this warp's 128 S columns of the row in one batch of loads
+      const bool agree = exact_pass || __any_sync(0xffffffffu, m == -INFINITY);
+      // Split loads when the reference is fixed and both entries are listed:
+      // the first 32 columns, then the other 96 while the first are
+      // exponentiated.  Otherwise this warp's columns in one batch.
+      const bool split = !agree && v0 && v1;
       uint32_t sv[4][32];
-      if (v0 && v1) {
-#pragma unroll
-        for (int ch = 0; ch < 4; ++ch) tmem_ld32(s_base + 32 * ch, sv[ch]);
+      if (split) {
+        tmem_ld32(s_base, sv[0]);
+        tmem_ld_wait();
+        reg_fence32(sv[0]);
+        tmem_ld32(s_base + 32, sv[1]);
+        tmem_ld32(s_base + 64, sv[2]);
+        tmem_ld32(s_base + 96, sv[3]);
       } else {
         if (v0) { tmem_ld32(s_base, sv[0]); tmem_ld32(s_base + 32, sv[1]); }
         if (v1) { tmem_ld32(s_base + 64, sv[2]); tmem_ld32(s_base + 96, sv[3]); }
+        tmem_ld_wait();
+        // S(t) is in registers: the tensor cores may overwrite it with S(t+1)
+        tc_fence_before();
+        mbar_arrive(bar(kBarSFree));
       }
-      tmem_ld_wait();
-      // S(t) is in registers: the tensor cores may overwrite it with S(t+1)
-      tc_fence_before();
-      mbar_arrive(bar(kBarSFree));
       // Reference of the exponentials.  Fixed-reference pass: the row's
       // reference is the max of the first key tile the row's block lists
       // (agreed with the other warp of the lane quarter), then kept.  Exact
       // pass: the two warps agree on every tile's max and raise the reference
       // lazily.  Both warps take the same branch (m is the same in both).
-      const bool agree = *pass_s != 0 || __any_sync(0xffffffffu, m == -INFINITY);
       bool pv_done = t == 0;                     // PV(t-1) completed (known so far)
+      if (t + 1 < n_t) {
+        e_next0 = tile_entry(t + 1, 2 * half);
+        e_next1 = tile_entry(t + 1, 2 * half + 1);
+      }
       if (agree) {
         float mx[8];
 #pragma unroll
@@ -557,6 +574,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             rs[i & 3] += p0 + p1;
             pk[ch][i] = pack_bf16x2(p0, p1);
           }
+          if (ch == 0 && split) {
+            tmem_ld_wait();
+            reg_fence32(sv[1]);
+            reg_fence32(sv[2]);
+            reg_fence32(sv[3]);
+            tc_fence_before();
+            mbar_arrive(bar(kBarSFree));
+          }
         }
       } else {
 #pragma unroll
@@ -577,9 +602,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       const float l_tile = (rs[0] + rs[1]) + (rs[2] + rs[3]);
       l += l_tile;
-      // a row whose later keys outgrow the fixed reference asks for the exact pass
-      if (!agree && __any_sync(0xffffffffu, !(l_tile <= kFixedRefSumLimit)) && lane == 0)
-        *cta_redo = 1;
       if (!ok) break;
       if (!pv_done && !warp_wait(bar(kBarOFull), (t - 1) & 1, lim, abort_flag)) {
         ok = false;
@@ -591,6 +613,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(bar(kBarPFull));
+      // a row whose later keys outgrow the fixed reference asks for the exact pass
+      if (!agree && __any_sync(0xffffffffu, !(l_tile <= kFixedRefSumLimit)) && lane == 0)
+        *cta_redo = 1;
     }
     if (!ok) record_abort(abort_flag, prm.status, kStatusTimeout);
     // ------------------------------------------------------------ epilogue

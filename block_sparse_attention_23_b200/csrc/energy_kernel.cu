@@ -300,21 +300,44 @@ __global__ void __launch_bounds__(kEThreads, 1)
         const bool v0 = (e0 & bit) != 0, v1 = (e1 & bit) != 0;   // uniform per warp
         const uint32_t sb = tmem + lane_off + b * static_cast<uint32_t>(kEN) + 128u * hf;
         uint32_t sv[4][32];
-        if (v0) { tmem_ld32(sb, sv[0]); tmem_ld32(sb + 32, sv[1]); }
-        if (v1) { tmem_ld32(sb + 64, sv[2]); tmem_ld32(sb + 96, sv[3]); }
-        tmem_ld_wait();
-        if (hf == 1) {   // both halves read: the tensor cores may refill the buffer
-          tc_fence_before();
-          mbar_arrive(bar(kEBarSFree + b));
+        // both entries listed (and every row live): the first 32 columns, then
+        // the other 96 while the first are exponentiated
+        const bool split = v0 && v1 && __all_sync(0xffffffffu, live);
+        if (split) {
+          tmem_ld32(sb, sv[0]);
+          tmem_ld_wait();
+          reg_fence32(sv[0]);
+          tmem_ld32(sb + 32, sv[1]);
+          tmem_ld32(sb + 64, sv[2]);
+          tmem_ld32(sb + 96, sv[3]);
+        } else {
+          if (v0) { tmem_ld32(sb, sv[0]); tmem_ld32(sb + 32, sv[1]); }
+          if (v1) { tmem_ld32(sb + 64, sv[2]); tmem_ld32(sb + 96, sv[3]); }
+          tmem_ld_wait();
+          if (hf == 1) {   // both halves read: the tensor cores may refill the buffer
+            tc_fence_before();
+            mbar_arrive(bar(kEBarSFree + b));
+          }
         }
         float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-        if (v0 && v1 && __all_sync(0xffffffffu, live)) {
-          // both entries listed: one straight-line block without per-chunk branches
+        if (split) {
+          // one straight-line block without per-chunk branches
 #pragma unroll
-          for (int ch = 0; ch < 4; ++ch)
+          for (int ch = 0; ch < 4; ++ch) {
 #pragma unroll
             for (int i = 0; i < 32; ++i)
               acc[ch >> 1][i & 3] += fast_exp2(fmaf(__uint_as_float(sv[ch][i]), sl2, neg_lse2));
+            if (ch == 0) {
+              tmem_ld_wait();
+              reg_fence32(sv[1]);
+              reg_fence32(sv[2]);
+              reg_fence32(sv[3]);
+              if (hf == 1) {   // both halves read: the tensor cores may refill the buffer
+                tc_fence_before();
+                mbar_arrive(bar(kEBarSFree + b));
+              }
+            }
+          }
         } else {
 #pragma unroll
           for (int ch = 0; ch < 4; ++ch) {
