@@ -148,18 +148,20 @@ def _max_over_ranks(x: float, ws: int, device) -> float:
     return float(t.item())
 
 
-def _mask_kernel_rooflines(stage_ms, BH, nb, d, S, kept, peaks, fp64_peak):
+def _mask_kernel_rooflines(stage_ms, BH, nb, d, S, kept, peaks, fp64_peak, exp_peak):
     """Per-kernel rooflines of the mask build from its stage times (ms):
     pooling against HBM (Q, K read; fp64 block means written), the reduced map
     against the measured fp64 FMA rate (2*nb^2*d per head), the selection
-    against HBM (the fp64 map read; bitmap and counts written), the compaction
-    against HBM (bitmap and counts read; row_ptr and col_idx written)."""
+    against the measured fp64 exp rate (one exp(L - max) per map entry, its one
+    transcendental step per entry; its HBM traffic, the fp64 map read once, is
+    reported beside it), the compaction against HBM (bitmap and counts read;
+    row_ptr and col_idx written)."""
     nw = (nb + 31) // 32
     hbm = peaks["hbm_gbs"]
     parts = {
         "pool": ("hbm", 2.0 * BH * S * d * 2 + 2.0 * BH * nb * d * 8),
         "reduced_map": ("fp64", 2.0 * BH * nb * nb * d),
-        "select": ("hbm", 8.0 * BH * nb * nb + 4.0 * BH * nb * nw + 4.0 * BH * nb),
+        "select": ("alu", float(BH) * nb * nb),
         "compact": ("hbm", 4.0 * BH * nb * nw + 8.0 * BH * nb + 4.0 * kept),
     }
     out = {}
@@ -168,6 +170,14 @@ def _mask_kernel_rooflines(stage_ms, BH, nb, d, S, kept, peaks, fp64_peak):
             ach = work / (ms * 1e-3) / 1e9
             out[name] = {"bound": "hbm", "ms": float(ms), "bytes": work, "achieved": ach,
                          "peak": hbm, "unit": "GB/s", "frac": ach / hbm}
+        elif bound == "alu":
+            ach = work / (ms * 1e-3) / 1e9
+            hbm_bytes = 8.0 * BH * nb * nb + 4.0 * BH * nb * nw + 4.0 * BH * nb
+            out[name] = {"bound": "alu", "ms": float(ms), "entries": work, "achieved": ach,
+                         "peak": exp_peak, "unit": "Gentry/s", "frac": ach / exp_peak,
+                         "peak_source": "measured fp64 exp chains (nabla_selftest_fp64_exp_rate), "
+                                        "one exp per entry",
+                         "hbm_frac": hbm_bytes / (ms * 1e-3) / 1e9 / hbm}
         else:
             ach = work / (ms * 1e-3) / 1e12
             out[name] = {"bound": "fp64", "ms": float(ms), "flops": work, "achieved": ach,
@@ -408,7 +418,7 @@ def run_ours(args):
     fwd_exact_passes = ws_fwd.exact_passes()
 
     # the mask build's four kernels timed one by one (events between them),
-    # outside the timed region, and the device's measured fp64 FMA rate
+    # outside the timed region, and the device's measured fp64 FMA and exp rates
     stage = np.zeros(4)
     nl.nabla_build_mask_stage_ms(q, k, w.tile_grid, w.thr, w.sta, workspace=ws_mask, out=mask_out)
     n_stage = 5
@@ -418,6 +428,7 @@ def run_ours(args):
     stage /= n_stage
     ws_mask.check()
     fp64_peak = nl.selftest_fp64_tflops()
+    exp_peak = nl.selftest_fp64_exp_rate()
 
     # end to end through the public API with host buffers: nabla_layer_host
     # reads Q, K, V from pinned memory and writes O and LSE back to it every
@@ -662,7 +673,8 @@ def run_ours(args):
                           "peak": peaks["hbm_gbs"], "unit": "GB/s",
                           "frac": mask_bytes / (mask_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
                           "bytes": mask_bytes},
-        "mask_kernels": _mask_kernel_rooflines(stage, B * H, nb, d, S, kept, peaks, fp64_peak),
+        "mask_kernels": _mask_kernel_rooflines(stage, B * H, nb, d, S, kept, peaks, fp64_peak,
+                                               exp_peak),
         "e2e": {"value": e2e_val, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
                 "call": "nabla_layer_host", "heads_per_chunk": hpc, "chunks": e2e_chunks},

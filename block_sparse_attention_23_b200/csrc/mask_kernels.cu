@@ -11,7 +11,7 @@
 //   pool_kernel        Q, K bf16 [BH,S,d] -> Qbar, Kbar fp64 [BH,nb,d]     HBM-bound
 //                      (tile-major or raster token order)
 //   logits_kernel      per head Qbar Kbar^T / sqrt(d) -> L fp64 [BH,nb,nb] fp64 FMA
-//   select_kernel      one warp per row: fp64 softmax, prefix (or top-k) selection, STA OR ->
+//   select_kernel      one CTA per row: fp64 softmax, prefix (or top-k) selection, STA OR ->
 //                      keep bitmap [BH*nb, nw] + counts (+ optional uint8 mask)
 //   mask_bits_kernel   external uint8 mask -> keep bitmap + counts
 //   scan_kernel        counts -> row_ptr (exclusive scan), nnz, capacity check

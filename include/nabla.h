@@ -421,8 +421,14 @@ NABLA_API int nabla_version(void);
  * the selection, the CSR compaction.  Arguments as for nabla_build_mask.
  *
  * nabla_selftest_fp64_tflops: times independent fp64 fma chains on every SM
- * (about 0.1 s), synchronises the stream and writes the measured fp64 rate in
- * TFLOP/s: the denominator of the reduced map's roofline.
+ * (a few milliseconds), synchronises the stream and writes the measured fp64
+ * rate in TFLOP/s: the denominator of the reduced map's roofline.
+ *
+ * nabla_selftest_fp64_exp_rate: times independent chains of fp64 exp on every
+ * SM (a few milliseconds), synchronises the stream and writes the measured
+ * rate in 1e9 exponentials per second: the denominator of the selection's
+ * arithmetic roofline (one fp64 exp per entry of the reduced map).
+ * Both return NABLA_ERR_INVALID_ARG for a NULL output before any CUDA call.
  *
  * nabla_selftest_mma: one 128 x N x 128 bf16 product through the same
  * tcgen05/TMA building blocks the attention kernel uses, for layout checks.
@@ -445,6 +451,7 @@ NABLA_API nabla_status nabla_build_mask_stage_ms(const nabla_shape* shape,
                                                  void* workspace, nabla_stream_t stream,
                                                  float* ms_out);
 NABLA_API nabla_status nabla_selftest_fp64_tflops(nabla_stream_t stream, double* tflops_out);
+NABLA_API nabla_status nabla_selftest_fp64_exp_rate(nabla_stream_t stream, double* gexp_out);
 NABLA_API nabla_status nabla_selftest_mma_pair(int variant, const void* a, const void* b, float* c,
                                                void* workspace, nabla_stream_t stream);
 

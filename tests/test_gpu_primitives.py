@@ -42,3 +42,14 @@ def test_mma_pair_selftest(nl, variant):
         want = a.double().numpy() @ b.double().numpy()
     c = nl.selftest_mma_pair(variant, a.cuda(), b.cuda()).cpu().numpy().astype(np.float64)
     np.testing.assert_allclose(c, want, rtol=0, atol=4e-3)
+
+
+def test_arithmetic_rate_selftests(nl):
+    """The measured fp64 FMA and exp rates that serve as roofline denominators are
+    finite and within what one GPU can do (fp64 FMA: between 1 and 200 TFLOP/s;
+    an fp64 exponential costs many FMAs, so its rate in Gexp/s stays below the
+    FMA rate in G-FMA/s)."""
+    tf = nl.selftest_fp64_tflops()
+    gexp = nl.selftest_fp64_exp_rate()
+    assert 1.0 < tf < 200.0
+    assert 1.0 < gexp < tf * 1e3 / 2
