@@ -259,6 +259,28 @@ def mask_parity_all_heads(w, q16, k16, gpu_row_ptr, gpu_col_idx):
             "rule": "bit-exact except near-cut / near-tie rows of the oracle"}
 
 
+def bwd_executed_flops(row_ptr, col_idx, BH, nb, d):
+    """FLOPs the two backward kernels execute for a block CSR: the dK/dV kernel
+    pairs key blocks and visits the union of the query blocks that list either,
+    two per 128-query tile, with four products per tile (S^T, dP^T, dV, dK);
+    the dQ kernel pairs query blocks and visits the union of their key blocks,
+    two per 128-key tile, with three (S, dP, dQ).  Each product is 128 x 128 x d."""
+    rp = row_ptr[:BH * nb + 1].cpu().numpy()
+    ci = col_idx[:int(rp[-1])].cpu().numpy()
+    m = np.zeros((BH * nb, nb), dtype=bool)
+    m[np.repeat(np.arange(BH * nb), np.diff(rp)), ci] = True
+    m = m.reshape(BH, nb, nb)
+
+    def tiles(a):   # blocks paired along axis 1, the union along axis 2, two per tile
+        if a.shape[1] % 2:
+            a = np.concatenate([a, np.zeros((a.shape[0], 1, a.shape[2]), dtype=bool)], axis=1)
+        return int(((((a[:, 0::2] | a[:, 1::2]).sum(-1)) + 1) // 2).sum())
+
+    tiles_q = tiles(m)
+    tiles_k = tiles(np.ascontiguousarray(m.transpose(0, 2, 1)))
+    return (3.0 * tiles_q + 4.0 * tiles_k) * 2.0 * 128 * 128 * d
+
+
 def sweep_executed_over_kept(mask):
     """Executed / kept attention FLOPs of a static mask [B,H,nb,nb]: query
     blocks in pairs, the union of their lists in 256-key tiles."""
@@ -578,6 +600,7 @@ def run_ours(args):
     bwd_ms = a.elapsed_time(b) / n_bw
     bwd_flops = 2.5 * kept_flops
     bwd_tflops = bwd_flops / (bwd_ms * 1e-3) / 1e12
+    bwd_exec = bwd_executed_flops(mask_out[0], mask_out[1], B * H, nb, d)
     del dout, grads
 
     # XAttention scorer (stride 8) + the same selection, outside the step;
@@ -700,6 +723,12 @@ def run_ours(args):
                                "at the layer's thr and STA, outside the step"},
         "bwd": {"bound": "tensor", "ms": bwd_ms, "achieved": bwd_tflops, "peak": peak,
                 "unit": "TFLOP/s", "frac": bwd_tflops / peak, "flops": bwd_flops,
+                "executed": {"flops": bwd_exec, "over_algorithmic": bwd_exec / bwd_flops,
+                             "tflops": bwd_exec / (bwd_ms * 1e-3) / 1e12,
+                             "frac_of_sustained": bwd_exec / (bwd_ms * 1e-3) / 1e12 / peak,
+                             "what": "products the two kernels run: 4 per 128-query tile of the "
+                                     "dK/dV kernel, 3 per 128-key tile of the dQ kernel, tiles "
+                                     "over unions of paired blocks, counted on the host"},
                 "what": "bsa_bwd (D, column bitmaps, dK/dV and dQ kernels) over the step's "
                         "block list, outside the step; FLOPs = 10*d*64*64 per kept block"},
         "raster_layer": {"ms_per_layer": raster_ms, "vs_tile_major": raster_ms / ms_per_step,
