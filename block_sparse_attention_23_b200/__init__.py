@@ -37,7 +37,7 @@ EXPORTED = ["nabla_workspace_size", "nabla_workspace_init", "nabla_query_status"
             "nabla_build_mask_xattn", "nabla_layer_host_workspace_size", "nabla_layer_host",
             "nabla_layer_host_chunks", "nabla_set_exact_reference", "nabla_query_exact_passes",
             "nabla_build_mask_stage_ms", "nabla_selftest_fp64_tflops",
-            "nabla_selftest_fp64_exp_rate", "nabla_selftest_mma_pair",
+            "nabla_selftest_fp64_exp_rate", "nabla_selftest_ex2_rate", "nabla_selftest_mma_pair",
             "nabla_set_pair_mode"]
 TO_TILE_MAJOR, TO_RASTER = 0, 1
 
@@ -135,6 +135,8 @@ def lib() -> ctypes.CDLL:
             L.nabla_selftest_fp64_tflops.argtypes = [vp, vp]
             L.nabla_selftest_fp64_exp_rate.restype = i32
             L.nabla_selftest_fp64_exp_rate.argtypes = [vp, vp]
+            L.nabla_selftest_ex2_rate.restype = i32
+            L.nabla_selftest_ex2_rate.argtypes = [vp, vp]
             L.nabla_layer_host.restype = i32
             L.nabla_layer_host.argtypes = [sp, ctypes.POINTER(_MaskParams), vp, vp, vp, vp, vp,
                                            i32, vp, vp]
@@ -302,6 +304,13 @@ def selftest_fp64_exp_rate(stream=None) -> float:
     """Diagnostic: the device's measured fp64 exp throughput in Gexp/s (synchronises)."""
     out = ctypes.c_double(0.0)
     _check(lib().nabla_selftest_fp64_exp_rate(_stream(stream), ctypes.byref(out)))
+    return float(out.value)
+
+
+def selftest_ex2_rate(stream=None) -> float:
+    """Diagnostic: the device's measured fp32 ex2.approx throughput in Gexp/s (synchronises)."""
+    out = ctypes.c_double(0.0)
+    _check(lib().nabla_selftest_ex2_rate(_stream(stream), ctypes.byref(out)))
     return float(out.value)
 
 

@@ -3,7 +3,11 @@
 //   - fp64 FMA rate: the reduced map is an fp64 product Qbar Kbar^T;
 //   - fp64 exponential rate: the selection forms one fp64 exp(L - max) per
 //     entry of the map, its one transcendental step per entry, so entries per
-//     second over this rate bounds how close it runs to its arithmetic.
+//     second over this rate bounds how close it runs to its arithmetic;
+//   - fp32 ex2.approx rate (the exponential unit): the block-energy kernel
+//     takes one exponential per score of a kept block, 4,096 per block against
+//     2*d*64*64 tensor FLOPs, so the exponential unit, not the tensor cores,
+//     sets its floor.
 // A grid of eight CTAs per SM runs independent chains; the rate is timed with
 // CUDA events on the caller's stream after a shorter warm-up launch.  No
 // device memory is allocated: the result that keeps the chains alive goes to a
@@ -52,6 +56,21 @@ __global__ void __launch_bounds__(kDiagThreads) fp64_exp_kernel(int iters) {
 #pragma unroll
   for (int i = 0; i < kChains; ++i) s += x[i];
   if (s == -1.25e300) g_fp64_sink = s;
+}
+
+// x <- 2^(-x) stays in [1/2, 1] from any start in [0, 1]
+__global__ void __launch_bounds__(kDiagThreads) ex2_kernel(int iters) {
+  float x[kChains];
+#pragma unroll
+  for (int i = 0; i < kChains; ++i) x[i] = (threadIdx.x & 63) * (1.f / 64) + i * (1.f / 128);
+  for (int it = 0; it < iters; ++it) {
+#pragma unroll
+    for (int i = 0; i < kChains; ++i) asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(x[i]) : "f"(-x[i]));
+  }
+  float s = 0.f;
+#pragma unroll
+  for (int i = 0; i < kChains; ++i) s += x[i];
+  if (s == -1.25e30f) g_fp64_sink = s;
 }
 
 // launch(iters) on the caller's stream: a warm-up with iters / 8, then the
@@ -119,6 +138,27 @@ nabla_status nabla_selftest_fp64_exp_rate(nabla_stream_t stream, double* gexp_ou
   }, &blocks, &ms);
   if (e != cudaSuccess) {
     nabla::set_last_error(std::string("nabla_selftest_fp64_exp_rate: ") + cudaGetErrorString(e));
+    return NABLA_ERR_CUDA;
+  }
+  const double exps = static_cast<double>(kChains) * iters * blocks * kDiagThreads;
+  *gexp_out = exps / (static_cast<double>(ms) * 1e-3) / 1e9;
+  return NABLA_OK;
+}
+
+nabla_status nabla_selftest_ex2_rate(nabla_stream_t stream, double* gexp_out) {
+  if (gexp_out == nullptr) {
+    nabla::set_last_error("gexp_out is NULL");
+    return NABLA_ERR_INVALID_ARG;
+  }
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int iters = 1 << 14;
+  int blocks = 0;
+  float ms = 0.f;
+  const cudaError_t e = time_chains(st, iters, [&](int g, int n) {
+    ex2_kernel<<<g, kDiagThreads, 0, st>>>(n);
+  }, &blocks, &ms);
+  if (e != cudaSuccess) {
+    nabla::set_last_error(std::string("nabla_selftest_ex2_rate: ") + cudaGetErrorString(e));
     return NABLA_ERR_CUDA;
   }
   const double exps = static_cast<double>(kChains) * iters * blocks * kDiagThreads;

@@ -428,7 +428,12 @@ NABLA_API int nabla_version(void);
  * SM (a few milliseconds), synchronises the stream and writes the measured
  * rate in 1e9 exponentials per second: the denominator of the selection's
  * arithmetic roofline (one fp64 exp per entry of the reduced map).
- * Both return NABLA_ERR_INVALID_ARG for a NULL output before any CUDA call.
+ *
+ * nabla_selftest_ex2_rate: the same for the fp32 ex2.approx instruction (the
+ * exponential unit), in 1e9 per second: the floor of the block-energy kernel,
+ * which takes 4,096 exponentials per kept 64 x 64 block.
+ * All three return NABLA_ERR_INVALID_ARG for a NULL output before any CUDA
+ * call.
  *
  * nabla_selftest_mma: one 128 x N x 128 bf16 product through the same
  * tcgen05/TMA building blocks the attention kernel uses, for layout checks.
@@ -452,6 +457,7 @@ NABLA_API nabla_status nabla_build_mask_stage_ms(const nabla_shape* shape,
                                                  float* ms_out);
 NABLA_API nabla_status nabla_selftest_fp64_tflops(nabla_stream_t stream, double* tflops_out);
 NABLA_API nabla_status nabla_selftest_fp64_exp_rate(nabla_stream_t stream, double* gexp_out);
+NABLA_API nabla_status nabla_selftest_ex2_rate(nabla_stream_t stream, double* gexp_out);
 NABLA_API nabla_status nabla_selftest_mma_pair(int variant, const void* a, const void* b, float* c,
                                                void* workspace, nabla_stream_t stream);
 

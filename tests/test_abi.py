@@ -264,6 +264,7 @@ def test_diagnostics_reject_bad_arguments_before_any_cuda_call(nl):
     assert rc == 1 and "ms_out" in lib.nabla_last_error().decode()
     assert lib.nabla_selftest_fp64_tflops(None, None) == 1
     assert lib.nabla_selftest_fp64_exp_rate(None, None) == 1
+    assert lib.nabla_selftest_ex2_rate(None, None) == 1
     assert lib.nabla_selftest_mma_pair(2, a, a, a, a, None) == 1
     assert "variant" in lib.nabla_last_error().decode()
     assert lib.nabla_selftest_mma_pair(0, None, a, a, a, None) == 1

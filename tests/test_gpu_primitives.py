@@ -45,11 +45,14 @@ def test_mma_pair_selftest(nl, variant):
 
 
 def test_arithmetic_rate_selftests(nl):
-    """The measured fp64 FMA and exp rates that serve as roofline denominators are
-    finite and within what one GPU can do (fp64 FMA: between 1 and 200 TFLOP/s;
-    an fp64 exponential costs many FMAs, so its rate in Gexp/s stays below the
-    FMA rate in G-FMA/s)."""
+    """The measured fp64 FMA, fp64 exp and fp32 ex2 rates that serve as roofline
+    denominators are finite and within what one GPU can do (fp64 FMA: between 1
+    and 200 TFLOP/s; an fp64 exponential costs many FMAs, so its rate in Gexp/s
+    stays below the FMA rate in G-FMA/s)."""
     tf = nl.selftest_fp64_tflops()
     gexp = nl.selftest_fp64_exp_rate()
     assert 1.0 < tf < 200.0
     assert 1.0 < gexp < tf * 1e3 / 2
+    # the exponential unit: 16 per clock per SM at most, so below 16 * 148 SMs * 2.1 GHz
+    ex2 = nl.selftest_ex2_rate()
+    assert 100.0 < ex2 < 16 * 148 * 2.1
