@@ -93,3 +93,26 @@ def test_executed_counts_closed_forms():
     rp, ci = _csr(diag)
     assert bench.executed_tile_products(rp, ci, 1, nb) == 3 * 2
     assert bench.bwd_executed_flops(rp, ci, 1, nb, d) == (3 * 3 + 4 * 3) * TILE * d
+
+
+def test_mask_kernel_rooflines_units():
+    """Per-kernel mask rooflines from stage times: pooling and compaction against
+    HBM bytes, the reduced map against the fp64 FMA rate, the selection against
+    the fp64 exp rate (one exponential per map entry) with its HBM fraction."""
+    BH, nb, d, S, kept = 2, 8, 128, 512, 40
+    peaks = {"hbm_gbs": 1000.0}
+    out = bench._mask_kernel_rooflines([1.0, 2.0, 4.0, 0.5], BH, nb, d, S, kept, peaks,
+                                       fp64_peak=10.0, exp_peak=50.0)
+    pool, rmap, sel, comp = out["pool"], out["reduced_map"], out["select"], out["compact"]
+    nw = (nb + 31) // 32
+    assert pool["bound"] == "hbm" and comp["bound"] == "hbm"
+    assert pool["bytes"] == 2.0 * BH * S * d * 2 + 2.0 * BH * nb * d * 8
+    assert pool["frac"] == pytest.approx(pool["bytes"] / 1e-3 / 1e9 / 1000.0)
+    assert rmap["bound"] == "fp64" and rmap["flops"] == 2.0 * BH * nb * nb * d
+    assert rmap["frac"] == pytest.approx(rmap["flops"] / 2e-3 / 1e12 / 10.0)
+    assert sel["bound"] == "alu" and sel["entries"] == BH * nb * nb
+    assert sel["achieved"] == pytest.approx(BH * nb * nb / 4e-3 / 1e9)
+    assert sel["frac"] == pytest.approx(sel["achieved"] / 50.0)
+    hbm_bytes = 8.0 * BH * nb * nb + 4.0 * BH * nb * nw + 4.0 * BH * nb
+    assert sel["hbm_frac"] == pytest.approx(hbm_bytes / 4e-3 / 1e9 / 1000.0)
+    assert comp["bytes"] == 4.0 * BH * nb * nw + 8.0 * BH * nb + 4.0 * kept
