@@ -269,3 +269,46 @@ def test_diagnostics_reject_bad_arguments_before_any_cuda_call(nl):
     assert "variant" in lib.nabla_last_error().decode()
     assert lib.nabla_selftest_mma_pair(0, None, a, a, a, None) == 1
 
+
+
+def test_calibration_xattn_and_init_arguments_checked(nl):
+    """The calibration calls, the XAttention builder and the workspace initialiser
+    reject bad arguments on the host, before any CUDA call (no GPU needed)."""
+    lib = nl.lib()
+    null = ctypes.c_void_p(0)
+    a = ctypes.c_void_p(1 << 20)
+    s = nl.make_shape(1, 2, 64 * 12, 128, (1, 3, 4))
+    assert lib.nabla_workspace_init(None, None) == 1
+    # nabla_calib_accumulate: eps outside [0, 1] (or NaN) is unsupported, null buffers invalid
+    assert lib.nabla_calib_accumulate(None, a, 0.1, a, None) == 1
+    assert lib.nabla_calib_accumulate(ctypes.byref(s), a, 1.5, a, None) == 2
+    assert lib.nabla_calib_accumulate(ctypes.byref(s), a, float("nan"), a, None) == 2
+    assert lib.nabla_calib_accumulate(ctypes.byref(s), null, 0.1, a, None) == 1
+    assert lib.nabla_calib_accumulate(ctypes.byref(s), a, 0.1, null, None) == 1
+    # nabla_calib_finalize: at least one vote, both buffers given
+    assert lib.nabla_calib_finalize(ctypes.byref(s), a, 0, a, None) == 1
+    assert "min_votes" in lib.nabla_last_error().decode()
+    assert lib.nabla_calib_finalize(ctypes.byref(s), null, 1, a, None) == 1
+    assert lib.nabla_calib_finalize(ctypes.byref(s), a, 1, null, None) == 1
+    # nabla_build_mask_xattn
+    prm = nl._MaskParams(0.2, 0, 0, 0, 0, 0)
+
+    def xattn(shape, params, stride, q=a, row_ptr=a, cap=10, col=a, ws=a):
+        return lib.nabla_build_mask_xattn(shape, params, stride, q, a, null, null, row_ptr, col,
+                                          cap, null, ws, None)
+
+    assert xattn(ctypes.byref(s), None, 8) == 1
+    assert xattn(ctypes.byref(s), ctypes.byref(prm), 5) == 2
+    assert "stride" in lib.nabla_last_error().decode()
+    assert xattn(ctypes.byref(s), ctypes.byref(nl._MaskParams(1.5, 0, 0, 0, 0, 0)), 8) == 2
+    assert xattn(ctypes.byref(s), ctypes.byref(nl._MaskParams(0.2, 0, 0, 0, 0, -1)), 8) == 1
+    assert xattn(ctypes.byref(s), ctypes.byref(nl._MaskParams(0.2, 1, -1, 0, 0, 0)), 8) == 1
+    bad_grid = nl.make_shape(1, 2, 64 * 12, 128, (1, 3, 5))
+    assert xattn(ctypes.byref(bad_grid), ctypes.byref(nl._MaskParams(0.2, 1, 1, 1, 1, 0)), 8) == 1
+    assert xattn(ctypes.byref(s), ctypes.byref(prm), 8, q=null) == 1
+    assert xattn(ctypes.byref(s), ctypes.byref(prm), 8, cap=-1) == 1
+    assert xattn(ctypes.byref(s), ctypes.byref(prm), 8, col=null) == 1
+    assert xattn(ctypes.byref(s), ctypes.byref(prm), 8, q=ctypes.c_void_p((1 << 20) + 8)) == 1
+    assert xattn(ctypes.byref(s), ctypes.byref(prm), 8, ws=ctypes.c_void_p((1 << 20) + 16)) == 1
+    raster = nl.make_shape(1, 2, 64 * 12, 128, (1, 3, 4), nl.LAYOUT_RASTER)
+    assert xattn(ctypes.byref(raster), ctypes.byref(prm), 8) == 2
